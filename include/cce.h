@@ -1,0 +1,120 @@
+/*
+ * cce.h -- C ABI of libcce.so, Cut Cross-Entropy (CCE) for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (Cut Cross-Entropy abstract, sentences 4-6 and 9):
+ *   for token embeddings E (N x D), classifier C (V x D) and labels y,
+ *     lse[i]  = log sum_v exp(E_i . C_v)
+ *     loss[i] = lse[i] - E_i . C_{y_i}          (0 where y_i == ignore_index)
+ *   without ever writing the N x V logit matrix to global memory; and the
+ *   gradients of sum_i dloss[i] * loss[i]:
+ *     G[i,v] = dloss[i] * (softmax(E_i C^T)[v] - [v == y_i]),
+ *     dE = G C,  dC = G^T E,
+ *   where the gradient tiles whose every |softmax - onehot| entry is below
+ *   filter_eps are skipped (the abstract's sentence 9: gradient work below
+ *   numerical precision is dropped).
+ *
+ * Conventions for every entry point:
+ *   - All matrix arguments are DEVICE pointers to row-major, contiguous data.
+ *     E, C are bf16 (raw 16-bit storage, passed as void*); y is int64;
+ *     loss, lse, dloss, dE, dC are fp32.
+ *   - D must be a multiple of 8 and E, C must be 16-byte aligned (the kernels
+ *     stream them with TMA).  N, D, V must be positive and fit in int32.
+ *   - The caller owns every buffer, including the workspace.  The library
+ *     never allocates device memory: the extra global memory of a call is
+ *     exactly the workspace, whose size is O(N) (see the *_workspace_size
+ *     functions).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and run on the current CUDA device.
+ *   - Argument errors are detected on the host: the call returns a non-zero
+ *     status and launches nothing.  Conditions found on the device (an
+ *     invalid label, a bounded wait that gave up) set bits in the status
+ *     block at the head of the workspace, read with cce_read_status.
+ *   - Not thread-safe across concurrent calls sharing one workspace.
+ */
+#ifndef CCE_H_
+#define CCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CCE_API __attribute__((visibility("default")))
+#else
+#define CCE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CCE_OK = 0,
+  CCE_ERR_INVALID_ARG = 1,        /* null pointer, non-positive or too large size, D % 8 != 0 */
+  CCE_ERR_MISALIGNED = 2,         /* E, C, or an fp32 vector not suitably aligned */
+  CCE_ERR_WORKSPACE_TOO_SMALL = 3,
+  CCE_ERR_UNSUPPORTED_DEVICE = 4, /* the current device is not sm_100 */
+  CCE_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+  CCE_ERR_TIMEOUT = 6,            /* device: a bounded wait gave up (cce_read_status) */
+  CCE_ERR_BAD_LABEL = 7           /* device: a label outside [0, V) (cce_read_status) */
+} cce_status_t;
+
+/* Status block decoded by cce_read_status. */
+typedef struct {
+  uint64_t flags;       /* bit 0: a wait timed out; bit 1: an invalid label was seen */
+  uint64_t live_tiles;  /* backward: 128x256 gradient tiles whose contraction ran */
+  uint64_t dead_tiles;  /* backward: tiles skipped by the filter */
+  uint64_t logit_tiles; /* 128x256 logit tiles computed on chip */
+} cce_counters_t;
+
+/* Workspace bytes needed by cce_forward for these sizes on the current device
+ * (N * splits * 8 bytes of per-split (max, sum) pairs plus a 256-byte status
+ * block, splits <= 64).  Returns 0 if the sizes are invalid or no device is
+ * usable. */
+CCE_API size_t cce_forward_workspace_size(int64_t N, int64_t D, int64_t V);
+
+/* Workspace bytes needed by cce_backward (the status block only). */
+CCE_API size_t cce_backward_workspace_size(int64_t N, int64_t D, int64_t V);
+
+/* Forward pass (abstract, sentences 4-6): per-token loss and log-sum-exp.
+ *   E     [N x D] bf16        token embeddings
+ *   C     [V x D] bf16        classifier rows
+ *   y     [N]     int64       labels; ignore_index marks tokens without a loss
+ *   loss  [N]     fp32 out    lse - correct logit; 0 if ignored; NaN if the
+ *                             label is outside [0, V) (status flag bit 1)
+ *   lse   [N]     fp32 out    log-sum-exp over the vocabulary (also for ignored rows)
+ *   workspace, workspace_bytes: device scratch, >= cce_forward_workspace_size
+ * The logits exist only in tensor memory on chip. */
+CCE_API cce_status_t cce_forward(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
+                         int64_t ignore_index, float* loss, float* lse, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Backward pass (abstract, sentences 4 and 9): gradients of sum_i dloss[i] * loss[i].
+ *   lse   [N] fp32   from cce_forward on the same E, C
+ *   dloss [N] fp32   upstream gradient per token (e.g. 1/#kept for a mean)
+ *   filter_eps       a 128x256 tile of (softmax - onehot) whose entries are
+ *                    all below filter_eps in magnitude is skipped; <= 0 keeps
+ *                    every tile (exact gradient)
+ *   dE    [N x D] fp32 out (overwritten), dC [V x D] fp32 out (overwritten)
+ * The logit tiles are recomputed on chip; rows with y == ignore_index
+ * contribute nothing.  Accumulation order across tiles is not fixed (fp32
+ * atomics), so results may differ in the last bits between runs. */
+CCE_API cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
+                          int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, float* dE,
+                          float* dC, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then copies the status block of `workspace` (as left
+ * by the last call that used it) into *out.  Returns CCE_ERR_TIMEOUT or
+ * CCE_ERR_BAD_LABEL if the corresponding flag is set, else CCE_OK. */
+CCE_API cce_status_t cce_read_status(const void* workspace, void* stream, cce_counters_t* out);
+
+/* Human-readable name of a status code (static storage). */
+CCE_API const char* cce_status_string(cce_status_t status);
+
+/* Library ABI version (major * 100 + minor). */
+CCE_API int cce_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CCE_H_ */

@@ -1,0 +1,34 @@
+/*
+ * cce_debug.h -- diagnostic entry points of libcce.so (not part of the loss API).
+ *
+ * These exist so that tests can localise a fault in the fused kernels.  They
+ * DO write logits to global memory, which the loss entry points never do.
+ */
+#ifndef CCE_DEBUG_H_
+#define CCE_DEBUG_H_
+
+#include "cce.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Runs the forward kernel's tensor-core mainloop unchanged and additionally
+ * stores every raw logit tile it forms:
+ *   logits [N x ceil(V/256)*256] fp32 device out, row-major; column v holds
+ *   E_i . C_v for v < V and 0 for the padding columns.
+ * loss/lse/workspace are as for cce_forward (which this call also computes). */
+CCE_API cce_status_t cce_debug_forward_logits(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D,
+                                      int64_t V, int64_t ignore_index, float* loss, float* lse, float* logits,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Upper bound (ns) on any single wait inside the kernels; a wait that runs
+ * longer gives up, sets the timeout status flag and the kernel exits.
+ * Default 1e9 (one second).  Process-wide. */
+CCE_API void cce_debug_set_wait_limit_ns(uint64_t limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CCE_DEBUG_H_ */

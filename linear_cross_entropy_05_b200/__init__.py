@@ -1,7 +1,135 @@
 """Cut Cross-Entropy for B200 (sm_100a): Python binding of libcce.so.
 
 The binding only marshals arguments; every step of the loss and its gradient
-runs in the library's CUDA kernels.  The native library is loaded on first use
-and a missing or unloadable library raises immediately (there is no CPU
-fallback).
+runs in the library's CUDA kernels (see include/cce.h).  The native library is
+loaded on first use; a missing or unloadable library raises immediately, and
+there is no CPU fallback.
+
+Low-level entry points carry the C names and take raw device pointers
+(Python ints):  cce_forward, cce_backward, cce_forward_workspace_size,
+cce_backward_workspace_size, cce_read_status, cce_status_string, cce_version,
+cce_debug_forward_logits, cce_debug_set_wait_limit_ns.
+
+Tensor helpers (torch supplies device memory and the current stream):
+forward(E, C, y) -> (loss, lse), backward(E, C, y, lse, dloss, filter_eps)
+-> (dE, dC), and linear_cross_entropy(E, C, y) for a mean-reduced loss with
+autograd.
 """
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+from . import _native
+from ._native import (CCEError, cce_backward, cce_backward_workspace_size, cce_debug_forward_logits,
+                      cce_debug_set_wait_limit_ns, cce_forward, cce_forward_workspace_size, cce_read_status,
+                      cce_status_string, cce_version, load_library)
+
+IGNORE_INDEX = -100
+
+__all__ = [
+    "CCEError", "IGNORE_INDEX", "cce_forward", "cce_backward", "cce_forward_workspace_size",
+    "cce_backward_workspace_size", "cce_read_status", "cce_status_string", "cce_version",
+    "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "load_library",
+    "forward", "backward", "read_status", "linear_cross_entropy", "Workspace",
+]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _check_inputs(E, C, y):
+    torch = _torch()
+    if E.dtype != torch.bfloat16 or C.dtype != torch.bfloat16:
+        raise TypeError("E and C must be torch.bfloat16")
+    if y.dtype != torch.int64:
+        raise TypeError("y must be torch.int64")
+    if not (E.is_cuda and C.is_cuda and y.is_cuda):
+        raise ValueError("E, C, y must be CUDA tensors")
+    if not (E.is_contiguous() and C.is_contiguous() and y.is_contiguous()):
+        raise ValueError("E, C, y must be contiguous")
+    if E.dim() != 2 or C.dim() != 2 or E.shape[1] != C.shape[1] or y.shape != (E.shape[0],):
+        raise ValueError("shapes must be E [N, D], C [V, D], y [N]")
+
+
+class Workspace:
+    """A caller-owned device scratch buffer (torch uint8), grown on demand."""
+
+    def __init__(self, device=None):
+        self.buf = None
+        self.device = device
+
+    def get(self, nbytes: int):
+        torch = _torch()
+        nbytes = max(int(nbytes), 256)
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf
+
+
+def _stream_ptr(stream) -> int:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def forward(E, C, y, ignore_index: int = IGNORE_INDEX, workspace: Optional[Workspace] = None,
+            stream=None, out=None) -> Tuple["object", "object"]:
+    """Per-token loss and log-sum-exp (fp32 tensors of shape [N])."""
+    torch = _torch()
+    _check_inputs(E, C, y)
+    N, D = E.shape
+    V = C.shape[0]
+    if out is None:
+        loss = torch.empty(N, dtype=torch.float32, device=E.device)
+        lse = torch.empty(N, dtype=torch.float32, device=E.device)
+    else:
+        loss, lse = out
+    ws_bytes = cce_forward_workspace_size(N, D, V)
+    if ws_bytes == 0:
+        raise CCEError(1, "cce_forward_workspace_size: invalid sizes or no sm_100 device")
+    ws = (workspace or Workspace(E.device)).get(ws_bytes)
+    cce_forward(E.data_ptr(), C.data_ptr(), y.data_ptr(), N, D, V, ignore_index, loss.data_ptr(),
+                lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    return loss, lse
+
+
+def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = IGNORE_INDEX,
+             workspace: Optional[Workspace] = None, stream=None, out=None):
+    """dE [N, D] and dC [V, D] (fp32) of sum_i dloss[i] * loss[i]."""
+    torch = _torch()
+    _check_inputs(E, C, y)
+    N, D = E.shape
+    V = C.shape[0]
+    for t, n in ((lse, "lse"), (dloss, "dloss")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.shape != (N,):
+            raise ValueError(f"{n} must be a contiguous CUDA float32 tensor of shape [N]")
+    if out is None:
+        dE = torch.empty((N, D), dtype=torch.float32, device=E.device)
+        dC = torch.empty((V, D), dtype=torch.float32, device=E.device)
+    else:
+        dE, dC = out
+    ws_bytes = cce_backward_workspace_size(N, D, V)
+    ws = (workspace or Workspace(E.device)).get(ws_bytes)
+    cce_backward(E.data_ptr(), C.data_ptr(), y.data_ptr(), lse.data_ptr(), dloss.data_ptr(), N, D, V,
+                 ignore_index, float(filter_eps), dE.data_ptr(), dC.data_ptr(), ws.data_ptr(), ws.numel(),
+                 _stream_ptr(stream))
+    return dE, dC
+
+
+def read_status(workspace: Workspace, stream=None, raise_on_flag: bool = False) -> dict:
+    """Synchronise the stream and decode the workspace's status block."""
+    st, c = cce_read_status(workspace.buf.data_ptr(), _stream_ptr(stream))
+    if raise_on_flag and st != 0:
+        raise CCEError(st, cce_status_string(st))
+    return {"status": st, "flags": c[0], "live_tiles": c[1], "dead_tiles": c[2], "logit_tiles": c[3]}
+
+
+def linear_cross_entropy(E, C, y, ignore_index: int = IGNORE_INDEX, filter_eps: float = 2.0 ** -12):
+    """Mean cross-entropy over non-ignored tokens of the logits E C^T, with
+    autograd support; the N x V logits are never materialised."""
+    from ._autograd import LinearCrossEntropy
+    return LinearCrossEntropy.apply(E, C, y, ignore_index, filter_eps)

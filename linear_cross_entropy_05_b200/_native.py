@@ -1,0 +1,123 @@
+"""ctypes declarations of libcce.so (include/cce.h, include/cce_debug.h)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcce.so")
+
+_lib = None
+_lock = threading.Lock()
+
+c_i64 = ctypes.c_int64
+c_vp = ctypes.c_void_p
+c_size = ctypes.c_size_t
+c_f32 = ctypes.c_float
+
+
+class CCECounters(ctypes.Structure):
+    _fields_ = [("flags", ctypes.c_uint64), ("live_tiles", ctypes.c_uint64),
+                ("dead_tiles", ctypes.c_uint64), ("logit_tiles", ctypes.c_uint64)]
+
+
+class CCEError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{msg} (status {status})")
+        self.status = status
+
+
+def load_library():
+    """Load libcce.so from the package directory; raise if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m linear_cross_entropy_05_b200.build` "
+                "(there is no CPU fallback)")
+        lib = ctypes.CDLL(LIB_PATH)
+        lib.cce_forward_workspace_size.argtypes = [c_i64, c_i64, c_i64]
+        lib.cce_forward_workspace_size.restype = c_size
+        lib.cce_backward_workspace_size.argtypes = [c_i64, c_i64, c_i64]
+        lib.cce_backward_workspace_size.restype = c_size
+        lib.cce_forward.argtypes = [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_size, c_vp]
+        lib.cce_forward.restype = ctypes.c_int
+        lib.cce_backward.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_vp, c_vp,
+                                     c_vp, c_size, c_vp]
+        lib.cce_backward.restype = ctypes.c_int
+        lib.cce_read_status.argtypes = [c_vp, c_vp, ctypes.POINTER(CCECounters)]
+        lib.cce_read_status.restype = ctypes.c_int
+        lib.cce_status_string.argtypes = [ctypes.c_int]
+        lib.cce_status_string.restype = ctypes.c_char_p
+        lib.cce_version.argtypes = []
+        lib.cce_version.restype = ctypes.c_int
+        lib.cce_debug_forward_logits.argtypes = [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp,
+                                                 c_vp, c_size, c_vp]
+        lib.cce_debug_forward_logits.restype = ctypes.c_int
+        lib.cce_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.cce_debug_set_wait_limit_ns.restype = None
+        _lib = lib
+        return lib
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise CCEError(st, f"{what}: {cce_status_string(st)}")
+
+
+def cce_status_string(status: int) -> str:
+    return load_library().cce_status_string(int(status)).decode()
+
+
+def cce_version() -> int:
+    return load_library().cce_version()
+
+
+def cce_forward_workspace_size(N: int, D: int, V: int) -> int:
+    return int(load_library().cce_forward_workspace_size(N, D, V))
+
+
+def cce_backward_workspace_size(N: int, D: int, V: int) -> int:
+    return int(load_library().cce_backward_workspace_size(N, D, V))
+
+
+def cce_forward(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: int, loss: int, lse: int,
+                workspace: int, workspace_bytes: int, stream: int, check: bool = True) -> int:
+    st = load_library().cce_forward(E, C, y, N, D, V, ignore_index, loss, lse, workspace, workspace_bytes,
+                                    stream)
+    if check:
+        _check(st, "cce_forward")
+    return st
+
+
+def cce_backward(E: int, C: int, y: int, lse: int, dloss: int, N: int, D: int, V: int, ignore_index: int,
+                 filter_eps: float, dE: int, dC: int, workspace: int, workspace_bytes: int, stream: int,
+                 check: bool = True) -> int:
+    st = load_library().cce_backward(E, C, y, lse, dloss, N, D, V, ignore_index, filter_eps, dE, dC, workspace,
+                                     workspace_bytes, stream)
+    if check:
+        _check(st, "cce_backward")
+    return st
+
+
+def cce_read_status(workspace: int, stream: int):
+    c = CCECounters()
+    st = load_library().cce_read_status(workspace, stream, ctypes.byref(c))
+    return st, (c.flags, c.live_tiles, c.dead_tiles, c.logit_tiles)
+
+
+def cce_debug_forward_logits(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: int, loss: int,
+                             lse: int, logits: int, workspace: int, workspace_bytes: int, stream: int,
+                             check: bool = True) -> int:
+    st = load_library().cce_debug_forward_logits(E, C, y, N, D, V, ignore_index, loss, lse, logits, workspace,
+                                                 workspace_bytes, stream)
+    if check:
+        _check(st, "cce_debug_forward_logits")
+    return st
+
+
+def cce_debug_set_wait_limit_ns(limit_ns: int) -> None:
+    load_library().cce_debug_set_wait_limit_ns(int(limit_ns))

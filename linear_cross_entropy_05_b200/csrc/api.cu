@@ -1,0 +1,284 @@
+// C-ABI front end of libcce.so: argument validation, workspace carving,
+// TMA descriptor construction and kernel launches.  See include/cce.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/cce.h"
+#include "../../include/cce_debug.h"
+#include "common.cuh"
+
+namespace cce {
+cudaError_t launch_fwd_lse(const CUtensorMap& tmE, const CUtensorMap& tmC, const FwdArgs& a, int grid,
+                           cudaStream_t stream);
+cudaError_t launch_fwd_finalize(const void* E, const void* C, const int64_t* y, const FinArgs& a, float* loss,
+                                float* lse, cudaStream_t stream);
+cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const BwdArgs& a, int grid,
+                       cudaStream_t stream);
+}  // namespace cce
+
+using namespace cce;
+
+namespace {
+
+std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  bool ok = false;
+  int sms = 0;
+};
+
+// Per-device facts, cached (at most 64 devices).
+DeviceInfo device_info() {
+  static DeviceInfo cache[64];
+  static std::once_flag flags[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceInfo{};
+  std::call_once(flags[dev], [dev] {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return;
+    cache[dev].ok = (major == 10 && minor == 0);
+    cache[dev].sms = sms;
+  });
+  return cache[dev];
+}
+
+bool sizes_ok(int64_t N, int64_t D, int64_t V) {
+  return N > 0 && D > 0 && V > 0 && N <= INT_MAX && V <= INT_MAX && D <= INT_MAX && (D % 8) == 0 &&
+         N * D <= (int64_t)1 << 40 && V * D <= (int64_t)1 << 40;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Vocabulary splits per 128-row token block.  Work units (block, split) are
+// dealt to the persistent CTAs round-robin; pick the split count that
+// minimises (units per CTA) x (tiles per unit).
+int choose_splits(int n_mblk, int n_vtile, int grid_max) {
+  long long best = LLONG_MAX;
+  int best_s = 1;
+  const int smax = std::min(64, n_vtile);
+  for (int s = 1; s <= smax; ++s) {
+    const long long units = (long long)n_mblk * s;
+    const long long per_cta = (units + grid_max - 1) / grid_max;
+    const long long tiles = (n_vtile + s - 1) / s;
+    const long long cost = per_cta * tiles;
+    if (cost < best) {
+      best = cost;
+      best_s = s;
+    }
+  }
+  return best_s;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t D, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct FwdPlan {
+  int n_mblk, n_vtile, n_split, grid;
+  size_t ws_bytes;
+};
+
+bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
+  if (!sizes_ok(N, D, V)) return false;
+  DeviceInfo di = device_info();
+  if (!di.ok || di.sms <= 0) return false;
+  p->n_mblk = (int)((N + BM - 1) / BM);
+  p->n_vtile = (int)((V + BN - 1) / BN);
+  p->n_split = choose_splits(p->n_mblk, p->n_vtile, di.sms);
+  const long long units = (long long)p->n_mblk * p->n_split;
+  p->grid = (int)std::min<long long>(units, di.sms);
+  p->ws_bytes = STATUS_BYTES + align_up((size_t)p->n_split * (size_t)N * sizeof(float2), 256);
+  return true;
+}
+
+cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
+                          int64_t ignore_index, float* loss, float* lse, float* dbg_logits, void* ws,
+                          size_t ws_bytes, void* stream_) {
+  if (!E || !C || !y || !loss || !lse || !ws) return CCE_ERR_INVALID_ARG;
+  if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
+  if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(loss, 4) || !aligned(lse, 4) ||
+      !aligned(ws, 256))
+    return CCE_ERR_MISALIGNED;
+  if (!device_info().ok) return CCE_ERR_UNSUPPORTED_DEVICE;
+  FwdPlan p;
+  if (!plan_forward(N, D, V, &p)) return CCE_ERR_INVALID_ARG;
+  if (ws_bytes < p.ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+
+  CUtensorMap tmE, tmC;
+  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN)) return CCE_ERR_CUDA;
+
+  unsigned long long* status = reinterpret_cast<unsigned long long*>(ws);
+  float2* partial = reinterpret_cast<float2*>(reinterpret_cast<char*>(ws) + STATUS_BYTES);
+  if (cudaMemsetAsync(status, 0, STATUS_BYTES, stream) != cudaSuccess) return CCE_ERR_CUDA;
+
+  FwdArgs a;
+  a.N = (int)N;
+  a.D = (int)D;
+  a.V = (int)V;
+  a.n_mblk = p.n_mblk;
+  a.n_vtile = p.n_vtile;
+  a.n_split = p.n_split;
+  a.n_units = p.n_mblk * p.n_split;
+  a.partial = partial;
+  a.dbg_logits = dbg_logits;
+  a.status = status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  if (launch_fwd_lse(tmE, tmC, a, p.grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
+
+  FinArgs f;
+  f.N = (int)N;
+  f.D = (int)D;
+  f.V = (int)V;
+  f.n_split = p.n_split;
+  f.ignore_index = ignore_index;
+  f.partial = partial;
+  f.status = status;
+  if (launch_fwd_finalize(E, C, y, f, loss, lse, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  return CCE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t cce_forward_workspace_size(int64_t N, int64_t D, int64_t V) {
+  FwdPlan p;
+  if (!plan_forward(N, D, V, &p)) return 0;
+  return p.ws_bytes;
+}
+
+size_t cce_backward_workspace_size(int64_t N, int64_t D, int64_t V) {
+  if (!sizes_ok(N, D, V)) return 0;
+  return STATUS_BYTES;
+}
+
+cce_status_t cce_forward(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
+                         int64_t ignore_index, float* loss, float* lse, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  return forward_impl(E, C, y, N, D, V, ignore_index, loss, lse, nullptr, workspace, workspace_bytes, stream);
+}
+
+cce_status_t cce_debug_forward_logits(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D,
+                                      int64_t V, int64_t ignore_index, float* loss, float* lse, float* logits,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!logits) return CCE_ERR_INVALID_ARG;
+  return forward_impl(E, C, y, N, D, V, ignore_index, loss, lse, logits, workspace, workspace_bytes, stream);
+}
+
+void cce_debug_set_wait_limit_ns(uint64_t limit_ns) {
+  g_wait_limit_ns.store(limit_ns ? limit_ns : 1000000000ull);
+}
+
+cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
+                          int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, float* dE,
+                          float* dC, void* workspace, size_t workspace_bytes, void* stream_) {
+  if (!E || !C || !y || !lse || !dloss || !dE || !dC || !workspace) return CCE_ERR_INVALID_ARG;
+  if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
+  if (!(filter_eps == filter_eps)) return CCE_ERR_INVALID_ARG;  // NaN
+  if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(lse, 4) || !aligned(dloss, 4) ||
+      !aligned(dE, 16) || !aligned(dC, 16) || !aligned(workspace, 256))
+    return CCE_ERR_MISALIGNED;
+  DeviceInfo di = device_info();
+  if (!di.ok) return CCE_ERR_UNSUPPORTED_DEVICE;
+  if (workspace_bytes < (size_t)STATUS_BYTES) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+
+  CUtensorMap tmE, tmC;
+  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN)) return CCE_ERR_CUDA;
+  unsigned long long* status = reinterpret_cast<unsigned long long*>(workspace);
+  if (cudaMemsetAsync(status, 0, STATUS_BYTES, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
+
+  BwdArgs a;
+  a.N = (int)N;
+  a.D = (int)D;
+  a.V = (int)V;
+  a.n_mblk = (int)((N + BM - 1) / BM);
+  a.n_vtile = (int)((V + BN - 1) / BN);
+  a.n_tiles = a.n_mblk * a.n_vtile;
+  a.group_m = std::min(a.n_mblk, 64);
+  a.filter_eps = filter_eps;
+  a.ignore_index = ignore_index;
+  a.y = y;
+  a.lse = lse;
+  a.dloss = dloss;
+  a.dE = dE;
+  a.dC = dC;
+  a.status = status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  const int grid = std::min(a.n_tiles, di.sms);
+  if (launch_bwd(tmE, tmC, a, grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  return CCE_OK;
+}
+
+cce_status_t cce_read_status(const void* workspace, void* stream, cce_counters_t* out) {
+  if (!workspace || !out) return CCE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CCE_ERR_CUDA;
+  unsigned long long h[4];
+  if (cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return CCE_ERR_CUDA;
+  out->flags = h[ST_FLAGS];
+  out->live_tiles = h[ST_LIVE_TILES];
+  out->dead_tiles = h[ST_DEAD_TILES];
+  out->logit_tiles = h[ST_TILES];
+  if (h[ST_FLAGS] & SF_TIMEOUT) return CCE_ERR_TIMEOUT;
+  if (h[ST_FLAGS] & SF_BAD_LABEL) return CCE_ERR_BAD_LABEL;
+  return CCE_OK;
+}
+
+const char* cce_status_string(cce_status_t s) {
+  switch (s) {
+    case CCE_OK: return "CCE_OK";
+    case CCE_ERR_INVALID_ARG: return "CCE_ERR_INVALID_ARG";
+    case CCE_ERR_MISALIGNED: return "CCE_ERR_MISALIGNED";
+    case CCE_ERR_WORKSPACE_TOO_SMALL: return "CCE_ERR_WORKSPACE_TOO_SMALL";
+    case CCE_ERR_UNSUPPORTED_DEVICE: return "CCE_ERR_UNSUPPORTED_DEVICE";
+    case CCE_ERR_CUDA: return "CCE_ERR_CUDA";
+    case CCE_ERR_TIMEOUT: return "CCE_ERR_TIMEOUT";
+    case CCE_ERR_BAD_LABEL: return "CCE_ERR_BAD_LABEL";
+  }
+  return "CCE_ERR_UNKNOWN";
+}
+
+int cce_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,371 @@
+// CCE backward: recompute logit tiles on chip, form the softmax gradient,
+// skip negligible tiles, contract the rest into dE and dC.
+//
+// Cut Cross-Entropy abstract, sentences 4 and 9: the logits are never stored,
+// so the backward pass recomputes each 128 x 256 logit tile S = E_m C_v^T in
+// TMEM, forms P = exp(S - lse) and D = P - onehot(y) in registers, and skips
+// the tile when every |D| is below filter_eps (gradient work under numerical
+// precision).  Live tiles are written as G = dloss * D in bf16 to shared
+// memory and contracted on the tensor cores:
+//     dE[m-block, d-chunk] += G   . C[v-tile, d-chunk]     (M=128, N=64, K=256)
+//     dC[v-tile,  d-chunk] += G^T . E[m-block, d-chunk]    (2 x M=128, N=64, K=128)
+// The C and E slices are the same TMA tiles the recompute streams (128-byte
+// swizzled rows of 64 d values); read K-major for S and MN-major for the
+// contractions.  Partial products are added to fp32 dE/dC with vector
+// reductions in L2.
+//
+// Roles (192 threads): warp 0 TMA producer, warp 1 UMMA issuer, warps 2-5
+// epilogue (one TMEM lane = one token row / one vocabulary row per thread).
+// TMEM columns: [0,256) logit tile, [256,320) dE chunk, [320,448) dC chunk.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace cce {
+
+namespace {
+constexpr uint32_t TM_S = 0;
+constexpr uint32_t TM_DE = 256;
+constexpr uint32_t TM_DC = 320;
+
+__device__ __forceinline__ void tile_coords(int t, int n_mblk, int n_vtile, int group_m, int& m, int& vt) {
+  // Raster: groups of group_m token blocks; inside a group the token block
+  // varies fastest so concurrent CTAs share the same C tile in L2 while the
+  // group's E rows stay resident.
+  const int gsize = group_m * n_vtile;
+  const int g = t / gsize;
+  const int rem = t - g * gsize;
+  const int gm = min(group_m, n_mblk - g * group_m);
+  vt = rem / gm;
+  m = g * group_m + (rem - vt * gm);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+}  // namespace
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                                   // BWD_STAGES x [128][64] bf16 (E slices)
+  uint8_t* sB = smem + BWD_STAGES * A_STAGE_BYTES;      // BWD_STAGES x [256][64] bf16 (C slices)
+  uint8_t* sG = sB + BWD_STAGES * B_STAGE_BYTES;        // 4 x [128][64] bf16, swizzled (G tile)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + G_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + BWD_STAGES;
+  uint64_t* s_full = bars + 2 * BWD_STAGES;
+  uint64_t* s_empty = s_full + 1;
+  uint64_t* g_full = s_full + 2;
+  uint64_t* g_empty = s_full + 3;
+  uint64_t* c_full = s_full + 4;
+  uint64_t* c_empty = s_full + 5;
+  uint64_t* drain = s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  // Per-tile live votes, a ring of 8 slots indexed by the CTA's tile counter.
+  // Slot kt%8 is written by the epilogue before g_full(kt) completes and read by
+  // every role after it; the epilogue clears slot (kt+4)%8 at tile kt, long
+  // after its last reader (tile kt-4) and before its next writer (tile kt+4).
+  volatile int* live_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < BWD_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, BM);
+    mbar_init(g_full, BM);
+    mbar_init(g_empty, 1);
+    mbar_init(c_full, 1);
+    mbar_init(c_empty, BM);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    for (int i = 0; i < 8; ++i) live_ring[i] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_map(&tmE);
+    tma_prefetch_map(&tmC);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, a.wait_limit_ns};
+  const int nkb = (a.D + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0, gph = 0, armed = 0;
+      int kt = 0;
+      for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++kt) {
+        int m, vt;
+        tile_coords(t, a.n_mblk, a.n_vtile, a.group_m, m, vt);
+        // logit recompute slices, then (if the tile is live) the same slices
+        // again as operands of the two contractions
+        for (int pass = 0; pass < 2; ++pass) {
+          if (pass == 1) {
+            if (!mbar_wait(g_full, gph, wc)) goto producer_done;
+            gph ^= 1u;
+            if (!live_ring[kt & 7]) break;
+          }
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
+            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+            tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
+            tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
+            armed |= 1u << stage;
+            if (++stage == BWD_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    producer_done : {
+      int dummy = 0;
+      WaitCtl exit_wc{&dummy, a.wait_limit_ns};
+      for (int s = 0; s < BWD_STAGES; ++s)
+        if (armed & (1u << s)) mbar_wait(&full[s], (s < stage) ? phase : (phase ^ 1u), exit_wc);
+    }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- UMMA issuer ----------------
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_DE = idesc_bf16_f32(BM, 64, false, true);
+      constexpr uint32_t IDESC_DC = idesc_bf16_f32(BM, 64, true, true);
+      const uint32_t g_addr = smem_u32(sG);
+      int stage = 0;
+      uint32_t phase = 0, sph = 0, gph = 0, cph = 0;
+      int kt = 0;
+      for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++kt) {
+        if (!mbar_wait(s_empty, sph ^ 1u, wc)) goto mma_done;
+        sph ^= 1u;
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * B_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16(tmem_base + TM_S, sdesc_sw128(a_addr + k * 32, 16, 1024),
+                      sdesc_sw128(b_addr + k * 32, 16, 1024), IDESC_S, (kb | k) != 0);
+          umma_commit(&empty[stage]);
+          if (++stage == BWD_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        umma_commit(s_full);
+        if (!mbar_wait(g_full, gph, wc)) goto mma_done;
+        gph ^= 1u;
+        tc_fence_after();
+        if (live_ring[kt & 7]) {
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
+            if (!mbar_wait(c_empty, cph ^ 1u, wc)) goto mma_done;
+            cph ^= 1u;
+            tc_fence_after();
+            const uint32_t e_addr = smem_u32(sA + stage * A_STAGE_BYTES);  // E[m-block, d-chunk]: 128 tok x 64 d
+            const uint32_t c_addr = smem_u32(sB + stage * B_STAGE_BYTES);  // C[v-tile, d-chunk]: 256 voc x 64 d
+            // dE chunk = G (128 tok x 256 voc, K-major) . Cchunk (K = voc rows, MN = d)
+#pragma unroll
+            for (int k = 0; k < BN / 16; ++k)
+              umma_bf16(tmem_base + TM_DE,
+                        sdesc_sw128(g_addr + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024),
+                        sdesc_sw128(c_addr + k * 2048, 16384, 1024), IDESC_DE, k != 0);
+            // dC chunk, vocabulary half h = G^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int k = 0; k < BM / 16; ++k)
+                umma_bf16(tmem_base + TM_DC + h * 64,
+                          sdesc_sw128(g_addr + (2 * h) * (BM * 128) + k * 2048, BM * 128, 1024),
+                          sdesc_sw128(e_addr + k * 2048, 16384, 1024), IDESC_DC, k != 0);
+            umma_commit(&empty[stage]);
+            umma_commit(c_full);
+            if (++stage == BWD_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          umma_commit(g_empty);
+        } else {
+          mbar_arrive(g_empty);
+        }
+      }
+    mma_done:
+      umma_commit(drain);
+      {
+        int dummy = 0;
+        WaitCtl exit_wc{&dummy, a.wait_limit_ns};
+        mbar_wait(drain, 0, exit_wc);
+      }
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int lane_grp = warp & 3;
+    const int rib = lane_grp * 32 + lane;  // row inside the tile (token, or vocab for dC)
+    const uint32_t lane_addr = (uint32_t)(lane_grp * 32) << 16;
+    const float eps = a.filter_eps;
+    const bool filter_on = eps > 0.f;
+    uint32_t sph = 0, gph = 0, cph = 0;
+    unsigned long long n_live = 0, n_dead = 0;
+    uint8_t* g_row = sG + rib * 128;
+    const int sw = rib & 7;
+    int kt = 0;
+    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++kt) {
+      int m, vt;
+      tile_coords(t, a.n_mblk, a.n_vtile, a.group_m, m, vt);
+      const int row = m * BM + rib;
+      bool valid = row < a.N;
+      long long yl = valid ? a.y[row] : a.ignore_index;
+      if (yl == a.ignore_index) valid = false;
+      if (valid && (yl < 0 || yl >= a.V)) {
+        valid = false;
+        atomicOr(a.status + ST_FLAGS, SF_BAD_LABEL);
+      }
+      const float lse2 = valid ? a.lse[row] * LOG2E : 0.f;
+      const float dl = valid ? a.dloss[row] : 0.f;
+      const int ycol = valid ? (int)(yl - (long long)vt * BN) : -1;  // may fall outside [0, BN)
+      const int ncols = min(BN, a.V - vt * BN);
+
+      if (!mbar_wait(s_full, sph, wc)) break;
+      sph ^= 1u;
+      if (!mbar_wait(g_empty, gph ^ 1u, wc)) break;
+      tc_fence_after();
+      bool live = !filter_on;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float x[32];
+        tmem_ld32(tmem_base + lane_addr + TM_S + c * 32, x);
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float g2[2];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int col = c * 32 + j + q;
+            float p = ex2_approx(fmaf(x[j + q], LOG2E, -lse2));
+            float d = (col == ycol) ? p - 1.f : p;
+            d = (valid && col < ncols) ? d : 0.f;
+            live |= fabsf(d) >= eps;
+            g2[q] = dl * d;
+          }
+          pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
+        }
+        // 32 columns = 64 bytes = four 16-byte chunks of the 128-byte row of
+        // K block (c / 2); 128B swizzle: chunk index ^= row % 8.
+        uint8_t* blk = g_row + (c >> 1) * (BM * 128);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = ((c & 1) * 4 + q) ^ sw;
+          *reinterpret_cast<uint4*>(blk + chunk * 16) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(s_empty);
+      fence_proxy_async_smem();
+      if (__any_sync(0xffffffffu, live) && lane == 0) atomicOr(const_cast<int*>(&live_ring[kt & 7]), 1);
+      __syncwarp();
+      if (rib == 0) live_ring[(kt + 4) & 7] = 0;
+      mbar_arrive(g_full);
+      if (!mbar_wait(g_full, gph, wc)) break;
+      gph ^= 1u;
+      const bool live_any = live_ring[kt & 7] != 0;
+      if (!live_any) {
+        ++n_dead;
+        continue;
+      }
+      ++n_live;
+      const int vrow0 = vt * BN + rib;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(c_full, cph, wc)) {
+          ok = false;
+          break;
+        }
+        cph ^= 1u;
+        tc_fence_after();
+        const int d0 = kb * BK;
+        // dE rows: token `row`
+#pragma unroll 1
+        for (int q = 0; q < 2; ++q) {
+          float v[32];
+          tmem_ld32(tmem_base + lane_addr + TM_DE + q * 32, v);
+          if (valid) {
+            float* dst = a.dE + (size_t)row * a.D + d0 + q * 32;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              if (d0 + q * 32 + i < a.D) red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+          }
+        }
+        // dC rows: vocabulary rows vt*256 + h*128 + rib
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          const int vr = vrow0 + h * BM;
+#pragma unroll 1
+          for (int q = 0; q < 2; ++q) {
+            float v[32];
+            tmem_ld32(tmem_base + lane_addr + TM_DC + h * 64 + q * 32, v);
+            if (vr < a.V) {
+              float* dst = a.dC + (size_t)vr * a.D + d0 + q * 32;
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                if (d0 + q * 32 + i < a.D) red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(c_empty);
+      }
+      if (!ok) break;
+    }
+    if (rib == 0) {
+      atomicAdd(a.status + ST_LIVE_TILES, n_live);
+      atomicAdd(a.status + ST_DEAD_TILES, n_dead);
+      atomicAdd(a.status + ST_TILES, n_live + n_dead);
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status + ST_FLAGS, SF_TIMEOUT);
+}
+
+size_t bwd_smem_bytes() { return 1024 + (size_t)BWD_STAGES * STAGE_BYTES + G_BYTES + 256; }
+
+cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const BwdArgs& a, int grid,
+                       cudaStream_t stream) {
+  const size_t smem = bwd_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  bwd_kernel<<<grid, NUM_THREADS, smem, stream>>>(tmE, tmC, a);
+  return cudaGetLastError();
+}
+
+}  // namespace cce

@@ -1,0 +1,78 @@
+// Definitions shared by the CCE kernels and the C-ABI front end.
+#pragma once
+
+#include <cstdint>
+
+namespace cce {
+
+// Tile geometry of the fused logit kernels.
+//   BM token rows (one TMEM lane each) x BN vocabulary columns per tile,
+//   BK = 64 bf16 along D per pipeline stage (one 128-byte swizzle row).
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int A_STAGE_BYTES = BM * BK * 2;  // E slice  [128 rows][64 d]
+constexpr int B_STAGE_BYTES = BN * BK * 2;  // C slice  [256 rows][64 d]
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int NUM_THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int FWD_STAGES = 4;
+constexpr int BWD_STAGES = 3;
+constexpr int G_BYTES = BM * BN * 2;        // bf16 softmax-gradient tile (4 swizzled K blocks)
+
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+// Status block at the head of every workspace (8 x u64, zeroed per call).
+enum StatusWord : int {
+  ST_FLAGS = 0,        // bit mask of StatusFlag
+  ST_LIVE_TILES = 1,   // backward: tiles whose gradient contraction ran
+  ST_DEAD_TILES = 2,   // backward: tiles skipped by the filter
+  ST_TILES = 3,        // tiles whose logits were computed
+};
+enum StatusFlag : unsigned long long {
+  SF_TIMEOUT = 1ull,    // a bounded wait gave up; outputs are incomplete
+  SF_BAD_LABEL = 2ull,  // a label outside [0, V) that is not ignore_index
+};
+constexpr int STATUS_BYTES = 256;
+
+struct FwdArgs {
+  int N, D, V;
+  int n_mblk;      // ceil(N / BM)
+  int n_vtile;     // ceil(V / BN)
+  int n_split;     // vocabulary splits per token block
+  int n_units;     // n_mblk * n_split
+  float2* partial; // [n_split][N]: (running max, sum of exp(z - max)) per split
+  float* dbg_logits;           // optional [N][n_vtile * BN] raw logits (debug build entry only)
+  unsigned long long* status;
+  unsigned long long wait_limit_ns;
+};
+
+struct FinArgs {
+  int N, D, V, n_split;
+  long long ignore_index;
+  const float2* partial;
+  unsigned long long* status;
+};
+
+struct BwdArgs {
+  int N, D, V;
+  int n_mblk, n_vtile;
+  int n_tiles;          // tiles to visit
+  int group_m;          // token blocks per raster group
+  float filter_eps;     // <= 0: every tile is live
+  long long ignore_index;
+  const int64_t* y;
+  const float* lse;
+  const float* dloss;
+  float* dE;            // [N][D] fp32, accumulated
+  float* dC;            // [V][D] fp32, accumulated
+  unsigned long long* status;
+  unsigned long long wait_limit_ns;
+};
+
+__host__ __device__ inline void split_range(int r, int n_vtile, int n_split, int& v0, int& v1) {
+  v0 = (int)(((long long)r * n_vtile) / n_split);
+  v1 = (int)(((long long)(r + 1) * n_vtile) / n_split);
+}
+
+}  // namespace cce

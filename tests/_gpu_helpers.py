@@ -1,0 +1,51 @@
+"""Helpers for the GPU parity tests: move generator output to the device,
+call the library through its C-ABI binding, compare with the oracle."""
+import numpy as np
+
+IGN = -100
+
+# Tolerances (the spec bar for this path)
+LOSS_ABS = 1e-2          # per-token loss, absolute
+MEAN_REL = 1e-4          # mean loss, relative
+GRAD_REL_FILTER_OFF = 5e-3   # dE, dC relative Frobenius error, filter off
+GRAD_REL_FILTER_ON = 1e-2    # dE, dC relative Frobenius error, filter on (vs the exact gradient)
+
+
+def to_dev(inp, device="cuda"):
+    import torch
+    E = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(device)
+    C = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).to(device)
+    y = torch.from_numpy(inp["y"]).to(device)
+    return E, C, y
+
+
+def rel_fro(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a))
+
+
+def mean_of(loss, y):
+    keep = y != IGN
+    return float(np.asarray(loss, dtype=np.float64)[keep].sum() / keep.sum()) if keep.any() else float("nan")
+
+
+def gpu_forward(E, C, y, ws=None):
+    import linear_cross_entropy_05_b200 as L
+    ws = ws or L.Workspace(E.device)
+    loss, lse = L.forward(E, C, y, IGN, workspace=ws)
+    st = L.read_status(ws)
+    return loss.cpu().numpy(), lse.cpu().numpy(), st
+
+
+def gpu_backward(E, C, y, lse, dloss_np, eps, ws=None):
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    ws = ws or L.Workspace(E.device)
+    dl = torch.from_numpy(np.asarray(dloss_np, dtype=np.float32)).to(E.device)
+    if not torch.is_tensor(lse):
+        lse = torch.from_numpy(np.asarray(lse, dtype=np.float32)).to(E.device)
+    dE, dC = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws)
+    st = L.read_status(ws)
+    return dE, dC, st

@@ -1,0 +1,128 @@
+"""The C-ABI library loads and exports every symbol its headers declare;
+host-side argument validation returns the documented codes without a GPU."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names |= set(re.findall(r"CCE_API\s+[\w\s\*]+?\b(cce_\w+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_cross_entropy_05_b200 import build, _native
+    build.build()
+    return _native.load_library()
+
+
+def test_headers_declare_the_boundary():
+    names = _declared_symbols()
+    for n in ("cce_forward", "cce_backward", "cce_forward_workspace_size", "cce_backward_workspace_size",
+              "cce_read_status", "cce_status_string", "cce_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_library_exports_nothing_else(lib):
+    from linear_cross_entropy_05_b200 import _native
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _native.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert exported == set(_declared_symbols())
+
+
+def test_status_strings(lib):
+    from linear_cross_entropy_05_b200 import cce_status_string
+    assert cce_status_string(0) == "CCE_OK"
+    assert cce_status_string(3) == "CCE_ERR_WORKSPACE_TOO_SMALL"
+    assert cce_status_string(7) == "CCE_ERR_BAD_LABEL"
+    assert cce_status_string(99) == "CCE_ERR_UNKNOWN"
+
+
+def test_version(lib):
+    from linear_cross_entropy_05_b200 import cce_version
+    assert cce_version() >= 100
+
+
+def _cpu_only():
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("validation-with-fake-pointers cases only run where no GPU could be touched")
+    except ImportError:
+        pass
+
+
+def test_forward_argument_errors_are_reported_on_the_host(lib):
+    _cpu_only()
+    from linear_cross_entropy_05_b200 import cce_forward
+    P = 1 << 20  # a non-null, 256-aligned fake address: never dereferenced by these cases
+    ok = dict(E=P, C=P, y=P, N=256, D=256, V=4096, ignore_index=-100, loss=P, lse=P, workspace=P,
+              workspace_bytes=1 << 20, stream=0)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return cce_forward(a["E"], a["C"], a["y"], a["N"], a["D"], a["V"], a["ignore_index"], a["loss"], a["lse"],
+                           a["workspace"], a["workspace_bytes"], a["stream"], check=False)
+
+    assert call(E=0) == 1
+    assert call(workspace=0) == 1
+    assert call(N=0) == 1
+    assert call(V=-5) == 1
+    assert call(D=260) == 1          # D % 8 != 0
+    assert call(N=1 << 40) == 1      # does not fit int32
+    assert call(E=P + 8) == 2        # bf16 matrices need 16-byte alignment
+    assert call(workspace=P + 64) == 2
+    assert call() == 4               # valid arguments, but no sm_100 device here
+
+
+def test_backward_argument_errors_are_reported_on_the_host(lib):
+    _cpu_only()
+    from linear_cross_entropy_05_b200 import cce_backward
+    P = 1 << 20
+    base = [P, P, P, P, P, 256, 256, 4096, -100, 0.0, P, P, P, 1 << 20, 0]
+
+    def call(i=None, v=None):
+        a = list(base)
+        if i is not None:
+            a[i] = v
+        return cce_backward(*a, check=False)
+
+    assert call(3, 0) == 1                 # lse null
+    assert call(7, 0) == 1                 # V = 0
+    assert call(6, 12) == 1                # D % 8
+    assert call(9, float("nan")) == 1      # NaN filter threshold
+    assert call(10, P + 4) == 2            # dE not 16-byte aligned
+    assert call() == 4
+
+
+def test_workspace_size_without_device_is_zero(lib):
+    _cpu_only()
+    from linear_cross_entropy_05_b200 import cce_backward_workspace_size, cce_forward_workspace_size
+    assert cce_forward_workspace_size(8192, 2304, 256000) == 0
+    assert cce_forward_workspace_size(0, 8, 8) == 0
+    assert cce_backward_workspace_size(8192, 2304, 256000) == 256
+    assert cce_backward_workspace_size(8192, 2305, 256000) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    from linear_cross_entropy_05_b200 import _native
+    monkeypatch.setattr(_native, "_lib", None)
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "libcce.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        _native.load_library()

@@ -1,0 +1,165 @@
+"""GPU parity of the forward pass (loss, lse) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from linear_cross_entropy_05_b200 import synth
+
+from _gpu_helpers import IGN, LOSS_ABS, MEAN_REL, gpu_forward, mean_of, to_dev
+
+pytestmark = pytest.mark.gpu
+
+# Shapes the oracle finishes in seconds; together they span several tiles in
+# both directions, ragged N / V / D tails, the minimal D and a vocabulary of 1.
+CASES = [
+    synth.TINY,
+    synth.TINY.with_sizes(N=300, V=4096 + 77, D=264),
+    synth.TINY.with_sizes(N=129, V=257, D=8),
+    synth.TINY.with_sizes(N=1, V=1, D=64),
+    synth.TINY.with_sizes(N=5, V=300, D=16),
+    synth.GEMMA2_2B.with_sizes(N=1000, V=20000),
+    synth.LLAMA3_8B.with_sizes(N=700, V=9000),
+    synth.SMALL_LARGE_VOCAB.with_sizes(N=2000, V=30000),
+    synth.SWEEP.with_sizes(N=512, V=40000),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=[w.name for w in CASES])
+def test_forward_matches_oracle(w):
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    assert st["status"] == 0 and st["flags"] == 0
+    ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    assert np.abs(loss - ol).max() <= LOSS_ABS
+    assert np.abs(lse - olse).max() <= LOSS_ABS
+    m, om = mean_of(loss, inp["y"]), mean_of(ol, inp["y"])
+    assert abs(m - om) <= MEAN_REL * abs(om)
+    assert (loss[inp["y"] == IGN] == 0).all()
+
+
+def test_raw_logit_tiles_match_definition():
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.TINY.with_sizes(N=300, V=4096 + 77, D=264)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    N, D, V = w.N, w.D, w.V
+    nv = (V + 255) // 256 * 256
+    logits = torch.full((N, nv), float("nan"), device="cuda")
+    loss = torch.empty(N, device="cuda")
+    lse = torch.empty(N, device="cuda")
+    ws = L.Workspace()
+    buf = ws.get(L.cce_forward_workspace_size(N, D, V))
+    L.cce_debug_forward_logits(E.data_ptr(), C.data_ptr(), y.data_ptr(), N, D, V, IGN, loss.data_ptr(),
+                               lse.data_ptr(), logits.data_ptr(), buf.data_ptr(), buf.numel(),
+                               torch.cuda.current_stream().cuda_stream)
+    g = logits.cpu().numpy()
+    z = oracle.logits(oracle.bf16_bits_to_f64(inp["E"]), oracle.bf16_bits_to_f64(inp["C"]))
+    # bf16 x bf16 products are exact in fp32; only the fp32 accumulation rounds
+    assert np.abs(g[:, :V] - z).max() <= 1e-5 * max(1.0, np.abs(z).max())
+    assert (g[:, V:] == 0).all()
+
+
+def test_zero_classifier_gives_log_V():
+    w = synth.TINY.with_sizes(N=300, V=5000, D=128)
+    inp = synth.make_inputs(w)
+    inp["C"][:] = 0
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    assert st["status"] == 0
+    np.testing.assert_allclose(loss, math.log(5000), atol=1e-5)
+    np.testing.assert_allclose(lse, math.log(5000), atol=1e-5)
+
+
+def test_extreme_logits_stay_finite():
+    # |z| up to ~1e4: the online max shift must keep exp() in range
+    w = synth.TINY.with_sizes(N=256, V=3000, D=256)
+    w = w.__class__(**{**w.__dict__, "std": 16.0})
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    assert np.isfinite(loss).all() and np.isfinite(lse).all()
+    assert np.abs(olse).max() > 1e3
+    # fp32 keeps ~7 significant digits of values near 1e4
+    assert np.abs(lse - olse).max() <= 2e-6 * np.abs(olse).max() + LOSS_ABS
+
+
+def test_ignored_and_invalid_labels():
+    w = synth.TINY.with_sizes(N=200, V=1000, D=64)
+    inp = synth.make_inputs(w)
+    y = inp["y"]
+    y[:50] = IGN
+    y[77] = 1000      # == V: invalid
+    y[78] = -3        # negative, not ignore_index: invalid
+    E, C, yd = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, yd)
+    assert st["status"] == 7 and st["flags"] & 2   # CCE_ERR_BAD_LABEL
+    assert math.isnan(loss[77]) and math.isnan(loss[78])
+    assert (loss[:50] == 0).all()
+    ol, olse = oracle.forward(inp["E"], inp["C"], y, IGN)
+    ok = np.ones(200, bool)
+    ok[[77, 78]] = False
+    assert np.abs(loss[ok] - ol[ok]).max() <= LOSS_ABS
+    assert np.abs(lse - olse).max() <= LOSS_ABS
+
+
+def test_all_tokens_ignored():
+    w = synth.TINY.with_sizes(N=130, V=600, D=32)
+    inp = synth.make_inputs(w)
+    inp["y"][:] = IGN
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    assert st["status"] == 0
+    assert (loss == 0).all() and np.isfinite(lse).all()
+    assert math.isnan(mean_of(loss, inp["y"]))
+
+
+def test_forward_is_deterministic_and_reuses_workspace():
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=700, V=12000, D=512)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    ws = L.Workspace()
+    a = gpu_forward(E, C, y, ws)
+    b = gpu_forward(E, C, y, ws)
+    assert (a[0] == b[0]).all() and (a[1] == b[1]).all()
+
+
+def test_workspace_too_small_is_rejected():
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.TINY
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    need = L.cce_forward_workspace_size(w.N, w.D, w.V)
+    assert need >= 256 + 8 * w.N
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    out = torch.empty(2, w.N, device="cuda")
+    st = L.cce_forward(E.data_ptr(), C.data_ptr(), y.data_ptr(), w.N, w.D, w.V, IGN, out[0].data_ptr(),
+                       out[1].data_ptr(), ws.data_ptr(), ws.numel(), 0, check=False)
+    assert st == 3
+
+
+def test_library_allocates_no_device_memory():
+    import torch
+    w = synth.GEMMA2_2B.with_sizes(N=2048, V=30000, D=1024)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    import linear_cross_entropy_05_b200 as L
+    ws = L.Workspace()
+    loss, lse = L.forward(E, C, y, IGN, workspace=ws)   # warm-up: module load
+    dl = torch.full((w.N,), 1.0 / w.N, device="cuda")
+    dE, dC = L.backward(E, C, y, lse, dl, 2.0 ** -12, IGN, workspace=ws)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    L.forward(E, C, y, IGN, workspace=ws, out=(loss, lse))
+    L.backward(E, C, y, lse, dl, 2.0 ** -12, IGN, workspace=ws, out=(dE, dC))
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    # the only extra global memory is the caller's workspace: O(N)
+    assert ws.buf.numel() <= 256 + 64 * 8 * w.N + 256
