@@ -1,0 +1,505 @@
+#!/usr/bin/env python
+"""Benchmark of the Cut Cross-Entropy hot path on B200.
+
+One step = cce_forward + cce_backward (gradient filter 2^-12) over one batch
+of the Gemma-2-2B-shaped classifier head: N = 8192 tokens, D = 2304,
+V = 256000, bf16 E, C ~ N(0, 0.02), Zipf(1.1) labels (synthetic, seeded).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
+replica of the same problem on its own GPU (the operator runs on one GPU; there
+is no data-path collective); timing is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the plain definition of the loss
+and its gradient) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CCE fwd+bwd tokens/s"
+UNIT = "tokens/s"
+IGN = -100
+BM, BN = 128, 256
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend: str):
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if ws > 1 else None
+
+
+def reduce_max(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate_throughput(dist, tokens_local: float, seconds_local: float, device):
+    """Whole-job throughput: tokens processed by all ranks / max time over ranks."""
+    tmax = reduce_max(dist, seconds_local, device)
+    tok = reduce_sum(dist, tokens_local, device)
+    return tok / tmax, tmax
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception as e:  # nvidia-smi missing
+            log("clock sampler unavailable:", e)
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons, pw = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                pw.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm), "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash(which: str) -> str:
+    base = os.path.join(ROOT, "linear_cross_entropy_05_b200", "csrc")
+    h = hashlib.sha256()
+    for f in (f"{which}.cu", "common.cuh", "ptx.cuh"):
+        with open(os.path.join(base, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash("fwd" if kernel.startswith("fwd") else "bwd"):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_step(inp, rows, eps):
+    """The oracle's forward + backward for the token rows `rows` (a whole
+    number of 128-row blocks): loss/lse for those rows, then their full
+    contribution to dE and dC (tile filter applied)."""
+    import oracle
+    E64 = oracle.bf16_bits_to_f64(inp["E"][rows])
+    C64 = oracle.bf16_bits_to_f64(inp["C"])
+    y = inp["y"][rows]
+    loss, lse = oracle.forward_f64(E64, C64, y, IGN)
+    dl = np.full(len(rows), 1.0 / max(1, len(rows)))
+    dE, dC = oracle.backward_f64(E64, C64, y, lse, dl, IGN, filter_eps=eps, tile=(BM, BN))
+    return loss
+
+
+def cpu_baseline(inp, w, rows_n: int):
+    rows = np.arange(rows_n)
+    t0 = time.perf_counter()
+    oracle_step(inp, rows, w.filter_eps)
+    dt = time.perf_counter() - t0
+    return {"value": rows_n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle forward+backward (tile filter {w.filter_eps:g}) on the first {rows_n} tokens "
+                      f"of the {w.name} workload (full V={w.V}, D={w.D}); {dt:.2f} s"}
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, w):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from linear_cross_entropy_05_b200 import synth
+    log(f"[reference] generating {w.name} ...")
+    inp = synth.make_inputs(w)
+    rows_n = args.ref_rows
+    rows = np.arange(rows_n)
+    for _ in range(args.warmup):
+        oracle_step(inp, rows, w.filter_eps)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(inp, rows, w.filter_eps)
+    dt = time.perf_counter() - t0
+    value = rows_n * args.steps / dt
+    sample = (f"each step: fp64 oracle forward+backward (tile filter {w.filter_eps:g}) on {rows_n} tokens of the "
+              f"{w.name} workload (full V={w.V}, D={w.D})")
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, ws), "gpu_launches": 0,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def config_of(w, world):
+    return {"workload": w.name, "N": w.N, "D": w.D, "V": w.V, "labels": f"{w.labels}({w.zipf_s})",
+            "input_std": w.std, "filter_eps": w.filter_eps, "global_batch": w.N * world, "seq_len": None,
+            "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
+            "l2": "inputs larger than L2 (C alone is %.2f GB, L2 126 MB); no flush" % (w.V * w.D * 2 / 1e9)}
+
+
+def run_gpu(args, w):
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl")
+    import linear_cross_entropy_05_b200 as L
+    from linear_cross_entropy_05_b200 import synth
+
+    t0 = time.perf_counter()
+    inp = synth.make_inputs(w)
+    log(f"[rank {rank}] generated {w.name} in {time.perf_counter() - t0:.1f} s")
+    N, D, V = w.N, w.D, w.V
+    E = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(dev)
+    C = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.from_numpy(inp["y"]).to(dev)
+    dloss = torch.from_numpy(synth.mean_dloss(inp["y"])).to(dev)
+    loss = torch.empty(N, device=dev)
+    lse = torch.empty(N, device=dev)
+    dE = torch.empty((N, D), device=dev)
+    dC = torch.empty((V, D), device=dev)
+    ws_f = L.Workspace(dev)
+    ws_b = L.Workspace(dev)
+    eps = w.filter_eps
+    stream = torch.cuda.current_stream()
+
+    def step():
+        L.forward(E, C, y, IGN, workspace=ws_f, out=(loss, lse))
+        L.backward(E, C, y, lse, dloss, eps, IGN, workspace=ws_b, out=(dE, dC))
+
+    # warm-up (also loads the module) and status check
+    for _ in range(max(3, args.warmup)):
+        step()
+    stf = L.read_status(ws_f)
+    stb = L.read_status(ws_b)
+    if stf["status"] != 0 or stb["status"] != 0:
+        raise RuntimeError(f"device status not clean: fwd {stf} bwd {stb}")
+    live, dead, pruned = stb["live_tiles"], stb["dead_tiles"], stb["pruned_tiles"]
+
+    # extra global memory of one step: the library allocates nothing itself
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info(dev)
+    step()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info(dev)
+    lib_alloc = max(0, free0 - free1)
+    extra_hbm = ws_f.buf.numel() + ws_b.buf.numel() + lib_alloc
+
+    # ---- timed region: K steps, per-kernel events through the library hook ----
+    K = args.steps
+    ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+          for k in (0, 1)}
+    for k in (0, 1):               # torch creates the CUDA event on first record
+        for a, b in ev[k]:
+            a.record(stream)
+            b.record(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(K):
+        L.cce_debug_set_kernel_events(0, ev[0][i][0].cuda_event, ev[0][i][1].cuda_event)
+        L.cce_debug_set_kernel_events(1, ev[1][i][0].cuda_event, ev[1][i][1].cuda_event)
+        step()
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    L.cce_debug_set_kernel_events(0, 0, 0)
+    L.cce_debug_set_kernel_events(1, 0, 0)
+    clk = clocks.stop()
+    sec_local = t_start.elapsed_time(t_stop) / 1e3
+    value, sec = aggregate_throughput(dist, float(N * K), sec_local, dev)
+    fwd_ms = float(np.mean([a.elapsed_time(b) for a, b in ev[0]]))
+    bwd_ms = float(np.mean([a.elapsed_time(b) for a, b in ev[1]]))
+    step_ms = 1e3 * sec / K
+
+    # ---- end to end through the public API with host buffers ----
+    E_h = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    C_h = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_h = torch.from_numpy(inp["y"]).pin_memory()
+    dl_h = torch.from_numpy(synth.mean_dloss(inp["y"])).pin_memory()
+    loss_h = torch.empty(N, dtype=torch.float32).pin_memory()
+    Ke = max(3, K // 4)
+
+    def e2e_step():
+        E.copy_(E_h, non_blocking=True)
+        C.copy_(C_h, non_blocking=True)
+        y.copy_(y_h, non_blocking=True)
+        dloss.copy_(dl_h, non_blocking=True)
+        step()
+        loss_h.copy_(loss, non_blocking=True)
+
+    h2d = E_h.numel() * 2 + C_h.numel() * 2 + y_h.numel() * 8 + dl_h.numel() * 4
+    d2h = loss_h.numel() * 4
+    e2e_value = None
+    if not args.no_e2e:
+        e2e_step()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_value, _ = aggregate_throughput(dist, float(N * Ke), e0.elapsed_time(e1) / 1e3, dev)
+
+    # ---- roofline of the dominant kernel ----
+    peaks, peak_src = measured_peaks()
+    tile_flop = 2.0 * BM * BN * D
+    n_tiles = live + dead
+    flop_fwd = 2.0 * N * D * V
+    flop_bwd = n_tiles * tile_flop + live * 2.0 * tile_flop
+    dominant = "bwd_kernel" if bwd_ms >= fwd_ms else "fwd_lse_kernel"
+    dom_flop, dom_ms = (flop_bwd, bwd_ms) if dominant == "bwd_kernel" else (flop_fwd, fwd_ms)
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    achieved = dom_flop / (dom_ms * 1e-3) / 1e12
+    traffic = ncu_traffic(dominant, w.name)
+    executed_flop = flop_fwd + flop_bwd
+    nominal_flop = 6.0 * N * D * V
+
+    out = None
+    if rank == 0:
+        cpu = cpu_baseline(inp, w, args.cpu_rows) if world == 1 and not args.no_cpu_baseline else None
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded numpy PCG64; random-init classifier, Zipf labels)",
+            "config": config_of(w, world),
+            "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                         "flop_per_launch": dom_flop, "launch_ms": dom_ms},
+            "kernels": {"fwd_lse_kernel": {"ms": fwd_ms, "tflops": flop_fwd / fwd_ms / 1e9},
+                        "bwd_kernel": {"ms": bwd_ms, "tflops": flop_bwd / bwd_ms / 1e9,
+                                       "live_tiles": live, "dead_tiles": dead, "pruned_tiles": pruned}},
+            "pct_bf16_peak_executed": executed_flop / (step_ms * 1e-3) / 1e12 / peak,
+            "pct_bf16_peak_nominal_6NDV": nominal_flop / (step_ms * 1e-3) / 1e12 / peak,
+            "live_tile_frac": live / max(1, n_tiles + pruned),
+            "extra_hbm_bytes": int(extra_hbm),
+            "materialised_logits_fp32_bytes": N * V * 4,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": 3 * K,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+def run_suite(args):
+    """Per-workload table (not the contract line): fwd-only and fwd+bwd time,
+    executed tensor fraction, tiles visited, extra global memory against the
+    size of the materialised fp32 logits.  One JSON object per workload."""
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    from linear_cross_entropy_05_b200 import synth
+    dev = torch.device("cuda", 0)
+    peaks, _ = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    cases = [synth.TINY, synth.GEMMA2_2B, synth.LLAMA3_8B, synth.SMALL_LARGE_VOCAB,
+             synth.SMALL_LARGE_VOCAB.__class__(**{**synth.SMALL_LARGE_VOCAB.__dict__, "filter_eps": 0.0,
+                                                   "name": "small-model-large-vocab[filter off]"})] + \
+            [synth.SWEEP.with_sizes(N=n, name=f"long-batch-sweep[N={n}]") for n in synth.SWEEP_NS]
+    for w in cases:
+        inp = synth.make_inputs(w)
+        N, D, V = w.N, w.D, w.V
+        E = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(dev)
+        C = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.from_numpy(inp["y"]).to(dev)
+        dl = torch.from_numpy(synth.mean_dloss(inp["y"])).to(dev)
+        wsf, wsb = L.Workspace(dev), L.Workspace(dev)
+        loss, lse = L.forward(E, C, y, IGN, workspace=wsf)
+        dE, dC = L.backward(E, C, y, lse, dl, w.filter_eps, IGN, workspace=wsb)
+        st = L.read_status(wsb)
+        reps = 5
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        torch.cuda.synchronize()
+        tf = tb = 0.0
+        for _ in range(reps):
+            ev[0].record()
+            L.forward(E, C, y, IGN, workspace=wsf, out=(loss, lse))
+            ev[1].record()
+            L.backward(E, C, y, lse, dl, w.filter_eps, IGN, workspace=wsb, out=(dE, dC))
+            ev[2].record()
+            torch.cuda.synchronize()
+            tf += ev[0].elapsed_time(ev[1]) / reps
+            tb += ev[1].elapsed_time(ev[2]) / reps
+        tile = 2.0 * BM * BN * D
+        visited = st["live_tiles"] + st["dead_tiles"]
+        executed = 2.0 * N * D * V + visited * tile + st["live_tiles"] * 2.0 * tile
+        print(json.dumps({
+            "workload": w.name, "N": N, "D": D, "V": V, "filter_eps": w.filter_eps,
+            "fwd_ms": tf, "fwd_tokens_per_s": N / tf * 1e3, "fwd_frac_of_peak": 2.0 * N * D * V / tf / 1e9 / peak,
+            "fwd_bwd_ms": tf + tb, "fwd_bwd_tokens_per_s": N / (tf + tb) * 1e3,
+            "executed_frac_of_peak": executed / (tf + tb) / 1e9 / peak,
+            "nominal_6NDV_frac_of_peak": 6.0 * N * D * V / (tf + tb) / 1e9 / peak,
+            "tiles": {k: st[k] for k in ("live_tiles", "dead_tiles", "pruned_tiles")},
+            "extra_hbm_bytes": {"forward_workspace": wsf.buf.numel(), "backward_workspace": wsb.buf.numel()},
+            "materialised_logits_fp32_bytes": N * V * 4, "peak_tflops": peak}), flush=True)
+        del E, C, y, dl, dE, dC, loss, lse, wsf, wsb
+        torch.cuda.empty_cache()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["cce", "reference"], default="cce")
+    ap.add_argument("--cpu-rows", type=int, default=1024, help="tokens in the CPU-oracle baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=128, help="tokens per step of the reference (oracle) arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--workload", default="gemma2-2b-head",
+                    help="workload name (the default is the headline Gemma-2-2B-shaped head)")
+    ap.add_argument("--N", type=int, default=None, help="override tokens (profiling cases)")
+    ap.add_argument("--V", type=int, default=None, help="override vocabulary (profiling cases)")
+    ap.add_argument("--suite", action="store_true",
+                    help="per-workload table instead of the benchmark line (documentation)")
+    args = ap.parse_args(argv)
+    if args.suite:
+        return run_suite(args)
+    if args.warmup < 3:
+        args.warmup = 3
+    from linear_cross_entropy_05_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.N or args.V:
+        w = w.with_sizes(N=args.N, V=args.V)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -64,6 +64,7 @@ typedef struct {
   uint64_t live_tiles;  /* backward: 128x256 gradient tiles whose contraction ran */
   uint64_t dead_tiles;  /* backward: tiles skipped by the filter */
   uint64_t logit_tiles; /* 128x256 logit tiles computed on chip */
+  uint64_t pruned_tiles;/* backward: tiles proven negligible without recomputing them */
 } cce_counters_t;
 
 /* Workspace bytes needed by cce_forward for these sizes on the current device
@@ -72,7 +73,10 @@ typedef struct {
  * usable. */
 CCE_API size_t cce_forward_workspace_size(int64_t N, int64_t D, int64_t V);
 
-/* Workspace bytes needed by cce_backward (the status block only). */
+/* Workspace bytes needed by cce_backward: the status block plus the
+ * candidate-tile pre-pass (O(N + V/256): one (block, tile) pair per token at
+ * most, a few words per 128-token block and per 256-row vocabulary tile).
+ * Returns 0 if the sizes are invalid. */
 CCE_API size_t cce_backward_workspace_size(int64_t N, int64_t D, int64_t V);
 
 /* Forward pass (abstract, sentences 4-6): per-token loss and log-sum-exp.
@@ -96,8 +100,12 @@ CCE_API cce_status_t cce_forward(const void* E, const void* C, const int64_t* y,
  *                    every tile (exact gradient)
  *   dE    [N x D] fp32 out (overwritten), dC [V x D] fp32 out (overwritten)
  * The logit tiles are recomputed on chip; rows with y == ignore_index
- * contribute nothing.  Accumulation order across tiles is not fixed (fp32
- * atomics), so results may differ in the last bits between runs. */
+ * contribute nothing.  With filter_eps > 0 a pre-pass bounds every logit by
+ * |E_i| max_v |C_v| (Cauchy-Schwarz): tiles that bound proves negligible and
+ * that hold no label are not recomputed (counted as pruned); the result is
+ * the same as recomputing and testing them.  Accumulation order across tiles
+ * is not fixed (fp32 atomics), so results may differ in the last bits between
+ * runs. */
 CCE_API cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
                           int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, float* dE,
                           float* dC, void* workspace, size_t workspace_bytes, void* stream);

@@ -15,8 +15,9 @@ extern "C" {
 
 /* Runs the forward kernel's tensor-core mainloop unchanged and additionally
  * stores every raw logit tile it forms:
- *   logits [N x ceil(V/256)*256] fp32 device out, row-major; column v holds
- *   E_i . C_v for v < V and 0 for the padding columns.
+ *   logits [N x ceil(V/256)*256] fp32 device out, row-major; column v < V
+ *   holds E_i . C_v; the padding columns v >= V are unspecified (the kernel
+ *   skips 32-column groups that lie wholly past V).
  * loss/lse/workspace are as for cce_forward (which this call also computes). */
 CCE_API cce_status_t cce_debug_forward_logits(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D,
                                       int64_t V, int64_t ignore_index, float* loss, float* lse, float* logits,
@@ -26,6 +27,15 @@ CCE_API cce_status_t cce_debug_forward_logits(const void* E, const void* C, cons
  * longer gives up, sets the timeout status flag and the kernel exits.
  * Default 1e9 (one second).  Process-wide. */
 CCE_API void cce_debug_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Profiling hook.  While set, every launch of the selected kernel records
+ * `start_event` on the call's stream immediately before the launch and
+ * `stop_event` immediately after it, so the caller can time that kernel alone
+ * with cudaEventElapsedTime.  kernel: 0 = forward logit/LSE kernel,
+ * 1 = backward kernel.  Events are cudaEvent_t handles created by the caller
+ * (passed as void*); NULL clears the hook.  Process-wide, not thread-safe.
+ * Returns CCE_ERR_INVALID_ARG for an unknown kernel id. */
+CCE_API cce_status_t cce_debug_set_kernel_events(int kernel, void* start_event, void* stop_event);
 
 #ifdef __cplusplus
 }

@@ -8,7 +8,7 @@ there is no CPU fallback.
 Low-level entry points carry the C names and take raw device pointers
 (Python ints):  cce_forward, cce_backward, cce_forward_workspace_size,
 cce_backward_workspace_size, cce_read_status, cce_status_string, cce_version,
-cce_debug_forward_logits, cce_debug_set_wait_limit_ns.
+cce_debug_forward_logits, cce_debug_set_wait_limit_ns, cce_debug_set_kernel_events.
 
 Tensor helpers (torch supplies device memory and the current stream):
 forward(E, C, y) -> (loss, lse), backward(E, C, y, lse, dloss, filter_eps)
@@ -23,7 +23,7 @@ from typing import Optional, Tuple
 
 from . import _native
 from ._native import (CCEError, cce_backward, cce_backward_workspace_size, cce_debug_forward_logits,
-                      cce_debug_set_wait_limit_ns, cce_forward, cce_forward_workspace_size, cce_read_status,
+                      cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns, cce_forward, cce_forward_workspace_size, cce_read_status,
                       cce_status_string, cce_version, load_library)
 
 IGNORE_INDEX = -100
@@ -31,7 +31,7 @@ IGNORE_INDEX = -100
 __all__ = [
     "CCEError", "IGNORE_INDEX", "cce_forward", "cce_backward", "cce_forward_workspace_size",
     "cce_backward_workspace_size", "cce_read_status", "cce_status_string", "cce_version",
-    "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "load_library",
+    "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "cce_debug_set_kernel_events", "load_library",
     "forward", "backward", "read_status", "linear_cross_entropy", "Workspace",
 ]
 
@@ -125,7 +125,8 @@ def read_status(workspace: Workspace, stream=None, raise_on_flag: bool = False) 
     st, c = cce_read_status(workspace.buf.data_ptr(), _stream_ptr(stream))
     if raise_on_flag and st != 0:
         raise CCEError(st, cce_status_string(st))
-    return {"status": st, "flags": c[0], "live_tiles": c[1], "dead_tiles": c[2], "logit_tiles": c[3]}
+    return {"status": st, "flags": c[0], "live_tiles": c[1], "dead_tiles": c[2], "logit_tiles": c[3],
+            "pruned_tiles": c[4]}
 
 
 def linear_cross_entropy(E, C, y, ignore_index: int = IGNORE_INDEX, filter_eps: float = 2.0 ** -12):

@@ -19,7 +19,8 @@ c_f32 = ctypes.c_float
 
 class CCECounters(ctypes.Structure):
     _fields_ = [("flags", ctypes.c_uint64), ("live_tiles", ctypes.c_uint64),
-                ("dead_tiles", ctypes.c_uint64), ("logit_tiles", ctypes.c_uint64)]
+                ("dead_tiles", ctypes.c_uint64), ("logit_tiles", ctypes.c_uint64),
+                ("pruned_tiles", ctypes.c_uint64)]
 
 
 class CCEError(RuntimeError):
@@ -59,6 +60,8 @@ def load_library():
         lib.cce_debug_forward_logits.restype = ctypes.c_int
         lib.cce_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         lib.cce_debug_set_wait_limit_ns.restype = None
+        lib.cce_debug_set_kernel_events.argtypes = [ctypes.c_int, c_vp, c_vp]
+        lib.cce_debug_set_kernel_events.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -106,7 +109,7 @@ def cce_backward(E: int, C: int, y: int, lse: int, dloss: int, N: int, D: int, V
 def cce_read_status(workspace: int, stream: int):
     c = CCECounters()
     st = load_library().cce_read_status(workspace, stream, ctypes.byref(c))
-    return st, (c.flags, c.live_tiles, c.dead_tiles, c.logit_tiles)
+    return st, (c.flags, c.live_tiles, c.dead_tiles, c.logit_tiles, c.pruned_tiles)
 
 
 def cce_debug_forward_logits(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: int, loss: int,
@@ -121,3 +124,8 @@ def cce_debug_forward_logits(E: int, C: int, y: int, N: int, D: int, V: int, ign
 
 def cce_debug_set_wait_limit_ns(limit_ns: int) -> None:
     load_library().cce_debug_set_wait_limit_ns(int(limit_ns))
+
+
+def cce_debug_set_kernel_events(kernel: int, start_event: int, stop_event: int) -> None:
+    _check(load_library().cce_debug_set_kernel_events(int(kernel), start_event, stop_event),
+           "cce_debug_set_kernel_events")

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <atomic>
 #include <climits>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -21,6 +22,8 @@ cudaError_t launch_fwd_finalize(const void* E, const void* C, const int64_t* y, 
                                 float* lse, cudaStream_t stream);
 cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const BwdArgs& a, int grid,
                        cudaStream_t stream);
+cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
+                        int sms, cudaStream_t stream);
 }  // namespace cce
 
 using namespace cce;
@@ -28,6 +31,14 @@ using namespace cce;
 namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
+
+// Optional per-kernel timing events (debug hook): [kernel][0 = start, 1 = stop].
+std::atomic<void*> g_events[2][2] = {{{nullptr}, {nullptr}}, {{nullptr}, {nullptr}}};
+
+cudaError_t record_event(int kernel, int which, cudaStream_t s) {
+  void* ev = g_events[kernel][which].load();
+  return ev ? cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), s) : cudaSuccess;
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -128,6 +139,32 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
   return true;
 }
 
+// Backward workspace: status | pre-pass header | count, offset, cursor
+// [n_vtile] | blk_flat, nonflat [n_mblk] | list [N] int2.  O(N + V/256).
+struct BwdPlan {
+  int n_mblk, n_vtile;
+  size_t off_hdr, off_count, off_offset, off_cursor, off_flat, off_nonflat, off_list, zero_bytes, ws_bytes;
+};
+
+bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p) {
+  if (!sizes_ok(N, D, V)) return false;
+  p->n_mblk = (int)((N + BM - 1) / BM);
+  p->n_vtile = (int)((V + BN - 1) / BN);
+  if ((int64_t)p->n_mblk * p->n_vtile >= ((int64_t)1 << 31)) return false;
+  const size_t vt4 = align_up((size_t)p->n_vtile * 4, 256);
+  const size_t mb4 = align_up((size_t)p->n_mblk * 4, 256);
+  p->off_hdr = STATUS_BYTES;
+  p->off_count = p->off_hdr + HDR_BYTES;
+  p->off_offset = p->off_count + vt4;
+  p->off_cursor = p->off_offset + vt4;
+  p->zero_bytes = p->off_cursor + vt4;  // status, header, count, offset, cursor start at zero
+  p->off_flat = p->zero_bytes;
+  p->off_nonflat = p->off_flat + mb4;
+  p->off_list = p->off_nonflat + mb4;
+  p->ws_bytes = p->off_list + align_up((size_t)N * sizeof(int2), 256);
+  return true;
+}
+
 cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
                           int64_t ignore_index, float* loss, float* lse, float* dbg_logits, void* ws,
                           size_t ws_bytes, void* stream_) {
@@ -161,7 +198,9 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   a.dbg_logits = dbg_logits;
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
+  if (record_event(0, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (launch_fwd_lse(tmE, tmC, a, p.grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (record_event(0, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
 
   FinArgs f;
   f.N = (int)N;
@@ -186,8 +225,9 @@ size_t cce_forward_workspace_size(int64_t N, int64_t D, int64_t V) {
 }
 
 size_t cce_backward_workspace_size(int64_t N, int64_t D, int64_t V) {
-  if (!sizes_ok(N, D, V)) return 0;
-  return STATUS_BYTES;
+  BwdPlan p;
+  if (!plan_backward(N, D, V, &p)) return 0;
+  return p.ws_bytes;
 }
 
 cce_status_t cce_forward(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
@@ -207,6 +247,13 @@ void cce_debug_set_wait_limit_ns(uint64_t limit_ns) {
   g_wait_limit_ns.store(limit_ns ? limit_ns : 1000000000ull);
 }
 
+cce_status_t cce_debug_set_kernel_events(int kernel, void* start_event, void* stop_event) {
+  if (kernel < 0 || kernel > 1) return CCE_ERR_INVALID_ARG;
+  g_events[kernel][0].store(start_event);
+  g_events[kernel][1].store(stop_event);
+  return CCE_OK;
+}
+
 cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
                           int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, float* dE,
                           float* dC, void* workspace, size_t workspace_bytes, void* stream_) {
@@ -216,15 +263,19 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
   if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(lse, 4) || !aligned(dloss, 4) ||
       !aligned(dE, 16) || !aligned(dC, 16) || !aligned(workspace, 256))
     return CCE_ERR_MISALIGNED;
+  BwdPlan bp;
+  if (!plan_backward(N, D, V, &bp)) return CCE_ERR_INVALID_ARG;
   DeviceInfo di = device_info();
   if (!di.ok) return CCE_ERR_UNSUPPORTED_DEVICE;
-  if (workspace_bytes < (size_t)STATUS_BYTES) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < bp.ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
   CUtensorMap tmE, tmC;
   if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN)) return CCE_ERR_CUDA;
-  unsigned long long* status = reinterpret_cast<unsigned long long*>(workspace);
-  if (cudaMemsetAsync(status, 0, STATUS_BYTES, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  char* ws = reinterpret_cast<char*>(workspace);
+  unsigned long long* status = reinterpret_cast<unsigned long long*>(ws);
+  const bool filter_on = filter_eps > 0.f;
+  if (cudaMemsetAsync(ws, 0, filter_on ? bp.zero_bytes : STATUS_BYTES, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
 
@@ -232,10 +283,14 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
   a.N = (int)N;
   a.D = (int)D;
   a.V = (int)V;
-  a.n_mblk = (int)((N + BM - 1) / BM);
-  a.n_vtile = (int)((V + BN - 1) / BN);
-  a.n_tiles = a.n_mblk * a.n_vtile;
+  a.n_mblk = bp.n_mblk;
+  a.n_vtile = bp.n_vtile;
+  a.n_tiles = bp.n_mblk * bp.n_vtile;
   a.group_m = std::min(a.n_mblk, 64);
+  a.list_mode = filter_on ? 1 : 0;
+  a.hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);
+  a.list = reinterpret_cast<const int2*>(ws + bp.off_list);
+  a.nonflat = reinterpret_cast<const int*>(ws + bp.off_nonflat);
   a.filter_eps = filter_eps;
   a.ignore_index = ignore_index;
   a.y = y;
@@ -245,8 +300,30 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
   a.dC = dC;
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
-  const int grid = std::min(a.n_tiles, di.sms);
+
+  if (filter_on) {
+    PrepArgs pp;
+    pp.N = (int)N;
+    pp.D = (int)D;
+    pp.V = (int)V;
+    pp.n_mblk = bp.n_mblk;
+    pp.n_vtile = bp.n_vtile;
+    pp.ignore_index = ignore_index;
+    pp.log_eps = logf(filter_eps);
+    pp.hdr = reinterpret_cast<unsigned*>(ws + bp.off_hdr);
+    pp.count = reinterpret_cast<unsigned*>(ws + bp.off_count);
+    pp.offset = reinterpret_cast<unsigned*>(ws + bp.off_offset);
+    pp.cursor = reinterpret_cast<unsigned*>(ws + bp.off_cursor);
+    pp.blk_flat = reinterpret_cast<int*>(ws + bp.off_flat);
+    pp.nonflat = reinterpret_cast<int*>(ws + bp.off_nonflat);
+    pp.list = reinterpret_cast<int2*>(ws + bp.off_list);
+    pp.status = status;
+    if (launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  }
+  const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
+  if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (launch_bwd(tmE, tmC, a, grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
   return CCE_OK;
 }
 
@@ -254,12 +331,13 @@ cce_status_t cce_read_status(const void* workspace, void* stream, cce_counters_t
   if (!workspace || !out) return CCE_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return CCE_ERR_CUDA;
-  unsigned long long h[4];
+  unsigned long long h[5];
   if (cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return CCE_ERR_CUDA;
   out->flags = h[ST_FLAGS];
   out->live_tiles = h[ST_LIVE_TILES];
   out->dead_tiles = h[ST_DEAD_TILES];
   out->logit_tiles = h[ST_TILES];
+  out->pruned_tiles = h[ST_PRUNED];
   if (h[ST_FLAGS] & SF_TIMEOUT) return CCE_ERR_TIMEOUT;
   if (h[ST_FLAGS] & SF_BAD_LABEL) return CCE_ERR_BAD_LABEL;
   return CCE_OK;
@@ -279,6 +357,6 @@ const char* cce_status_string(cce_status_t s) {
   return "CCE_ERR_UNKNOWN";
 }
 
-int cce_version(void) { return 100; }
+int cce_version(void) { return 101; }
 
 }  // extern "C"

@@ -43,6 +43,61 @@ __device__ __forceinline__ void tile_coords(int t, int n_mblk, int n_vtile, int 
   m = g * group_m + (rem - vt * gm);
 }
 
+// Adds a 32 x 32 fp32 block held one row per lane (32 consecutive columns
+// each) to global memory.  The block is staged through a 4 KB per-warp buffer
+// with 16-byte chunks XOR-swizzled by row, then read back so that each warp
+// instruction covers four rows x 128 contiguous bytes: the vector reductions
+// reach L2 as whole cache lines instead of 32 scattered 16-byte pieces.
+//   base: element (row 0, column 0) of the block; ld: row stride (elements)
+//   row_ok: bit r set if row r exists; ncols: valid columns (multiple of 4)
+__device__ __forceinline__ void red_block32(uint8_t* xb, int lane, const float (&v)[32], float* base, size_t ld,
+                                            uint32_t row_ok, int ncols) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(xb + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+  const int q = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + (lane >> 3);
+    const float4 t = *reinterpret_cast<const float4*>(xb + r * 128 + ((q ^ (r & 7)) << 4));
+    if (((row_ok >> r) & 1u) && q * 4 < ncols) red_add_v4(base + (size_t)r * ld + q * 4, t.x, t.y, t.z, t.w);
+  }
+  __syncwarp();
+}
+
+// Work item t -> (token block m, vocabulary tile vt).  Dense mode rasters the
+// whole grid; list mode visits the pre-pass list (label tiles of flat blocks,
+// vocabulary-major), then every tile of each block that is not flat.
+struct TileMap {
+  int T, L, nnf;
+  __device__ __forceinline__ void init(const BwdArgs& a) {
+    if (a.list_mode) {
+      T = (int)a.hdr[HDR_T];
+      L = (int)a.hdr[HDR_L];
+      nnf = (int)a.hdr[HDR_NNF];
+    } else {
+      T = a.n_tiles;
+      L = 0;
+      nnf = 0;
+    }
+  }
+  __device__ __forceinline__ void get(const BwdArgs& a, int t, int& m, int& vt) const {
+    if (!a.list_mode) {
+      tile_coords(t, a.n_mblk, a.n_vtile, a.group_m, m, vt);
+    } else if (t < L) {
+      const int2 e = a.list[t];
+      m = e.x;
+      vt = e.y;
+    } else {
+      const int k = t - L;
+      vt = k / nnf;
+      m = a.nonflat[k - vt * nnf];
+    }
+  }
+};
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -56,7 +111,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sA = smem;                                   // BWD_STAGES x [128][64] bf16 (E slices)
   uint8_t* sB = smem + BWD_STAGES * A_STAGE_BYTES;      // BWD_STAGES x [256][64] bf16 (C slices)
   uint8_t* sG = sB + BWD_STAGES * B_STAGE_BYTES;        // 4 x [128][64] bf16, swizzled (G tile)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + G_BYTES);
+  uint8_t* sX = sG + G_BYTES;                           // 4 x 4 KB reduction staging (one per epilogue warp)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 4 * 4096);
   uint64_t* full = bars;
   uint64_t* empty = bars + BWD_STAGES;
   uint64_t* s_full = bars + 2 * BWD_STAGES;
@@ -114,9 +170,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, gph = 0, armed = 0;
       int kt = 0;
-      for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++kt) {
+      TileMap tm;
+      tm.init(a);
+      for (int t = blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
         int m, vt;
-        tile_coords(t, a.n_mblk, a.n_vtile, a.group_m, m, vt);
+        tm.get(a, t, m, vt);
         // logit recompute slices, then (if the tile is live) the same slices
         // again as operands of the two contractions
         for (int pass = 0; pass < 2; ++pass) {
@@ -155,7 +213,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, sph = 0, gph = 0, cph = 0;
       int kt = 0;
-      for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++kt) {
+      TileMap tm;
+      tm.init(a);
+      for (int t = blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
         if (!mbar_wait(s_empty, sph ^ 1u, wc)) goto mma_done;
         sph ^= 1u;
         tc_fence_after();
@@ -230,11 +290,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t sph = 0, gph = 0, cph = 0;
     unsigned long long n_live = 0, n_dead = 0;
     uint8_t* g_row = sG + rib * 128;
+    uint8_t* xb = sX + (warp - 2) * 4096;
     const int sw = rib & 7;
     int kt = 0;
-    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++kt) {
+    TileMap tm;
+    tm.init(a);
+    for (int t = blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
       int m, vt;
-      tile_coords(t, a.n_mblk, a.n_vtile, a.group_m, m, vt);
+      tm.get(a, t, m, vt);
       const int row = m * BM + rib;
       bool valid = row < a.N;
       long long yl = valid ? a.y[row] : a.ignore_index;
@@ -297,6 +360,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       ++n_live;
       const int vrow0 = vt * BN + rib;
+      const uint32_t rows_dE = __ballot_sync(0xffffffffu, valid);
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(c_full, cph, wc)) {
@@ -306,32 +370,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         cph ^= 1u;
         tc_fence_after();
         const int d0 = kb * BK;
-        // dE rows: token `row`
+        // dE rows of this warp: tokens m*128 + lane_grp*32 + r
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
           float v[32];
           tmem_ld32(tmem_base + lane_addr + TM_DE + q * 32, v);
-          if (valid) {
-            float* dst = a.dE + (size_t)row * a.D + d0 + q * 32;
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              if (d0 + q * 32 + i < a.D) red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
-          }
+          const int c0 = d0 + q * 32;
+          if (c0 < a.D)
+            red_block32(xb, lane, v, a.dE + (size_t)(m * BM + lane_grp * 32) * a.D + c0, (size_t)a.D, rows_dE,
+                        min(32, a.D - c0));
         }
-        // dC rows: vocabulary rows vt*256 + h*128 + rib
+        // dC rows of this warp: vocabulary rows vt*256 + h*128 + lane_grp*32 + r
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          const int vr = vrow0 + h * BM;
+          const uint32_t rows_dC = __ballot_sync(0xffffffffu, vrow0 + h * BM < a.V);
 #pragma unroll 1
           for (int q = 0; q < 2; ++q) {
             float v[32];
             tmem_ld32(tmem_base + lane_addr + TM_DC + h * 64 + q * 32, v);
-            if (vr < a.V) {
-              float* dst = a.dC + (size_t)vr * a.D + d0 + q * 32;
-#pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                if (d0 + q * 32 + i < a.D) red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
-            }
+            const int c0 = d0 + q * 32;
+            if (c0 < a.D)
+              red_block32(xb, lane, v, a.dC + (size_t)(vt * BN + h * BM + lane_grp * 32) * a.D + c0, (size_t)a.D,
+                          rows_dC, min(32, a.D - c0));
           }
         }
         tc_fence_before();
@@ -357,7 +417,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status + ST_FLAGS, SF_TIMEOUT);
 }
 
-size_t bwd_smem_bytes() { return 1024 + (size_t)BWD_STAGES * STAGE_BYTES + G_BYTES + 256; }
+size_t bwd_smem_bytes() { return 1024 + (size_t)BWD_STAGES * STAGE_BYTES + G_BYTES + 4 * 4096 + 256; }
 
 cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const BwdArgs& a, int grid,
                        cudaStream_t stream) {

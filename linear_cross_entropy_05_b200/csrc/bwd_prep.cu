@@ -1,0 +1,180 @@
+// Backward pre-pass: the list of logit tiles the backward must recompute.
+//
+// The gradient filter (Cut Cross-Entropy abstract, sentence 9) drops a
+// 128 x 256 tile when every |P - onehot| < eps.  For a token i and a column
+// v that is not its label, P_iv = exp(E_i.C_v - lse_i) and, by Cauchy-Schwarz,
+// E_i.C_v <= |E_i| |C_v|.  So if |E_i| * max_v |C_v| < lse_i + ln(eps) for every
+// kept token of a 128-token block, every tile of that block that holds none
+// of its labels is dead, and its logits need not be recomputed at all.  Such
+// a block is "flat"; only its label tiles are visited (and still tested
+// exactly).  Blocks that are not flat are visited densely.  The visited set
+// is therefore a superset of the live tiles, and the gradients equal those of
+// the dense recompute with the same filter.
+//
+// Kernels (stream order):
+//   prep_cnorm    max_v |C_v| (fp32, atomicMax on the float's bits)
+//   prep_blocks   per token block: row norms, flatness, label-tile counts
+//   prep_scan     exclusive scan of the per-vocabulary-tile counts; totals
+//   prep_scatter  label tiles of flat blocks, ordered by vocabulary tile so
+//                 concurrent CTAs share C tiles in L2
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace cce {
+
+namespace {
+
+__device__ __forceinline__ float sumsq_bf16x8(const uint4 v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(h[j]);
+    s = fmaf(f.x, f.x, s);
+    s = fmaf(f.y, f.y, s);
+  }
+  return s;
+}
+
+__device__ __forceinline__ float warp_row_norm(const __nv_bfloat16* row, int D, int lane) {
+  const uint4* r = reinterpret_cast<const uint4*>(row);
+  const int nvec = D >> 3;
+  float s = 0.f;
+  for (int i = lane; i < nvec; i += 32) s += sumsq_bf16x8(__ldg(r + i));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return sqrtf(s);
+}
+
+__device__ __forceinline__ bool label_ok(long long t, long long ignore_index, int V) {
+  return t != ignore_index && t >= 0 && t < V;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(256) prep_cnorm_kernel(const __nv_bfloat16* __restrict__ C, PrepArgs p) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  float mx = 0.f;
+  for (int v = gw; v < p.V; v += nw) mx = fmaxf(mx, warp_row_norm(C + (size_t)v * p.D, p.D, lane));
+  if (lane == 0) atomicMax(p.hdr + HDR_CMAX, __float_as_uint(mx));  // non-negative: bit order = value order
+}
+
+// One CTA (128 threads) per token block.
+__global__ void __launch_bounds__(128) prep_blocks_kernel(const __nv_bfloat16* __restrict__ E,
+                                                          const int64_t* __restrict__ y,
+                                                          const float* __restrict__ lse, PrepArgs p) {
+  __shared__ float nrm[BM];
+  __shared__ int tl[BM];
+  const int m = blockIdx.x;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  for (int rr = 0; rr < 32; ++rr) {
+    const int r = warp * 32 + rr;
+    const int row = m * BM + r;
+    float n = 0.f;
+    if (row < p.N) n = warp_row_norm(E + (size_t)row * p.D, p.D, lane);
+    if (lane == 0) nrm[r] = n;
+  }
+  __syncthreads();
+  const int row = m * BM + t;
+  long long yl = row < p.N ? y[row] : p.ignore_index;
+  const bool valid = row < p.N && label_ok(yl, p.ignore_index, p.V);
+  if (row < p.N && yl != p.ignore_index && !valid) atomicOr(p.status + ST_FLAGS, SF_BAD_LABEL);
+  const float cmax = __uint_as_float(p.hdr[HDR_CMAX]);
+  // Margins cover the fp32 rounding of the norms, of the recomputed logits and
+  // of the exp2 in the exact test.
+  const float margin = 1.0f / 1024.0f;
+  bool flat = true;
+  if (valid) flat = nrm[t] * cmax * (1.0f + margin) + margin < lse[row] + p.log_eps - margin;
+  const int all_flat = __syncthreads_and(flat);
+  if (t == 0) p.blk_flat[m] = all_flat;
+  if (!all_flat) {
+    if (t == 0) p.nonflat[atomicAdd(p.hdr + HDR_NNF, 1u)] = m;
+    return;
+  }
+  tl[t] = valid ? (int)(yl / BN) : -1;
+  __syncthreads();
+  bool owner = valid;
+  for (int j = 0; j < t && owner; ++j) owner = tl[j] != tl[t];
+  if (owner) atomicAdd(p.count + tl[t], 1u);
+}
+
+// Single CTA: exclusive scan of count[] -> offset[]; totals into the header.
+__global__ void __launch_bounds__(1024) prep_scan_kernel(PrepArgs p) {
+  __shared__ unsigned warp_sums[32];
+  __shared__ unsigned carry_s;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (t == 0) carry_s = 0;
+  __syncthreads();
+  for (int base = 0; base < p.n_vtile; base += 1024) {
+    const int i = base + t;
+    const unsigned x = i < p.n_vtile ? p.count[i] : 0u;
+    unsigned incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      unsigned ws = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned n = __shfl_up_sync(0xffffffffu, ws, o);
+        if (lane >= o) ws += n;
+      }
+      warp_sums[lane] = ws;  // inclusive over warps
+    }
+    __syncthreads();
+    const unsigned carry = carry_s;
+    const unsigned excl = carry + (warp ? warp_sums[warp - 1] : 0u) + incl - x;
+    if (i < p.n_vtile) p.offset[i] = excl;
+    __syncthreads();
+    if (t == 1023) carry_s = carry + warp_sums[31];
+    __syncthreads();
+  }
+  if (t == 0) {
+    const unsigned L = carry_s;
+    const unsigned nnf = p.hdr[HDR_NNF];
+    const unsigned long long T = (unsigned long long)L + (unsigned long long)nnf * (unsigned long long)p.n_vtile;
+    p.hdr[HDR_L] = L;
+    p.hdr[HDR_T] = (unsigned)T;
+    p.status[ST_PRUNED] = (unsigned long long)p.n_mblk * (unsigned long long)p.n_vtile - T;
+  }
+}
+
+// One CTA (128 threads) per token block: place the flat block's label tiles.
+__global__ void __launch_bounds__(128) prep_scatter_kernel(const int64_t* __restrict__ y, PrepArgs p) {
+  __shared__ int tl[BM];
+  const int m = blockIdx.x;
+  if (!p.blk_flat[m]) return;
+  const int t = threadIdx.x;
+  const int row = m * BM + t;
+  const long long yl = row < p.N ? y[row] : p.ignore_index;
+  const bool valid = row < p.N && label_ok(yl, p.ignore_index, p.V);
+  tl[t] = valid ? (int)(yl / BN) : -1;
+  __syncthreads();
+  bool owner = valid;
+  for (int j = 0; j < t && owner; ++j) owner = tl[j] != tl[t];
+  if (owner) {
+    const int v = tl[t];
+    const unsigned slot = atomicAdd(p.cursor + v, 1u);
+    p.list[p.offset[v] + slot] = make_int2(m, v);
+  }
+}
+
+cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
+                        int sms, cudaStream_t stream) {
+  const int cgrid = sms * 8;
+  prep_cnorm_kernel<<<cgrid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(C), p);
+  prep_blocks_kernel<<<p.n_mblk, 128, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E), y, lse, p);
+  prep_scan_kernel<<<1, 1024, 0, stream>>>(p);
+  prep_scatter_kernel<<<p.n_mblk, 128, 0, stream>>>(y, p);
+  return cudaGetLastError();
+}
+
+}  // namespace cce

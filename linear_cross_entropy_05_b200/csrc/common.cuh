@@ -28,7 +28,16 @@ enum StatusWord : int {
   ST_LIVE_TILES = 1,   // backward: tiles whose gradient contraction ran
   ST_DEAD_TILES = 2,   // backward: tiles skipped by the filter
   ST_TILES = 3,        // tiles whose logits were computed
+  ST_PRUNED = 4,       // backward: tiles proven dead without recomputing them
 };
+// Header words of the backward pre-pass (u32, after the status block).
+enum PrepHeader : int {
+  HDR_CMAX = 0,  // max_v |C_v| as float bits
+  HDR_NNF = 1,   // token blocks that are not flat (visited densely)
+  HDR_L = 2,     // label tiles of flat blocks (list length)
+  HDR_T = 3,     // tiles to visit: L + NNF * n_vtile
+};
+constexpr int HDR_BYTES = 256;
 enum StatusFlag : unsigned long long {
   SF_TIMEOUT = 1ull,    // a bounded wait gave up; outputs are incomplete
   SF_BAD_LABEL = 2ull,  // a label outside [0, V) that is not ignore_index
@@ -54,11 +63,29 @@ struct FinArgs {
   unsigned long long* status;
 };
 
+struct PrepArgs {
+  int N, D, V, n_mblk, n_vtile;
+  long long ignore_index;
+  float log_eps;          // ln(filter_eps)
+  unsigned* hdr;          // PrepHeader words
+  unsigned* count;        // [n_vtile] label tiles per vocabulary tile
+  unsigned* offset;       // [n_vtile] exclusive scan of count
+  unsigned* cursor;       // [n_vtile] fill cursors
+  int* blk_flat;          // [n_mblk]
+  int* nonflat;           // [n_mblk] ids of blocks that are not flat
+  int2* list;             // [<= N] (token block, vocabulary tile), vocabulary-major
+  unsigned long long* status;
+};
+
 struct BwdArgs {
   int N, D, V;
   int n_mblk, n_vtile;
-  int n_tiles;          // tiles to visit
-  int group_m;          // token blocks per raster group
+  int n_tiles;          // tiles to visit (dense mode)
+  int group_m;          // token blocks per raster group (dense mode)
+  int list_mode;        // 1: visit the pre-pass list (hdr, list, nonflat)
+  const unsigned* hdr;
+  const int2* list;
+  const int* nonflat;
   float filter_eps;     // <= 0: every tile is live
   long long ignore_index;
   const int64_t* y;

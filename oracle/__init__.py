@@ -221,21 +221,22 @@ def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
     # dE rows: full logit row per token; the tile filter needs the Bn rows of
     # the token's tile block, so evaluate the whole block when filtering.
     out_dE = np.zeros((rows_dE.shape[0], E64.shape[1]), dtype=np.float64)
-    for k, i in enumerate(rows_dE):
-        if filter_eps > 0.0:
-            b0 = (int(i) // Bn) * Bn
-            b1 = min(N, b0 + Bn)
+    if filter_eps > 0.0:
+        # one evaluation per token block holding requested rows
+        for b in sorted({int(i) // Bn for i in rows_dE}):
+            b0, b1 = b * Bn, min(N, (b + 1) * Bn)
             z = logits(E64[b0:b1], C64)
             _, Dm, G = softmax_grad_f64(z, lse_all[b0:b1], y[b0:b1], dloss[b0:b1], ignore_index)
             live = tile_live_map_f64(Dm, b0, Bn, Bv, filter_eps)
             mask = np.repeat(live[0], Bv)[:V]
-            g = np.where(mask, G[int(i) - b0], 0.0)
-        else:
+            for k in np.nonzero((rows_dE >= b0) & (rows_dE < b1))[0]:
+                out_dE[k] = np.where(mask, G[int(rows_dE[k]) - b0], 0.0) @ C64
+    else:
+        for k, i in enumerate(rows_dE):
             z = logits(E64[int(i):int(i) + 1], C64)
             _, _, G = softmax_grad_f64(z, lse_all[int(i):int(i) + 1], y[int(i):int(i) + 1],
                                        dloss[int(i):int(i) + 1], ignore_index)
-            g = G[0]
-        out_dE[k] = g @ C64
+            out_dE[k] = G[0] @ C64
 
     # dC rows: the column v of G over all tokens.  With filtering, the column
     # tile of v must be evaluated in full for each token block.

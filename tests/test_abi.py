@@ -116,7 +116,11 @@ def test_workspace_size_without_device_is_zero(lib):
     from linear_cross_entropy_05_b200 import cce_backward_workspace_size, cce_forward_workspace_size
     assert cce_forward_workspace_size(8192, 2304, 256000) == 0
     assert cce_forward_workspace_size(0, 8, 8) == 0
-    assert cce_backward_workspace_size(8192, 2304, 256000) == 256
+    # status 256 + header 256 + 3 x [V/256] u32 + 2 x [N/128] i32 + N int2, each rounded to 256 bytes
+    up = lambda x: (x + 255) // 256 * 256
+    for N, V in ((8192, 256000), (300, 4173), (65536, 262144)):
+        want = 512 + 3 * up(4 * (-(-V // 256))) + 2 * up(4 * (-(-N // 128))) + up(8 * N)
+        assert cce_backward_workspace_size(N, 2304, V) == want
     assert cce_backward_workspace_size(8192, 2305, 256000) == 0
 
 

@@ -1,0 +1,180 @@
+"""GPU parity of the backward pass (dE, dC) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from linear_cross_entropy_05_b200 import synth
+
+from _gpu_helpers import (GRAD_REL_FILTER_OFF, GRAD_REL_FILTER_ON, IGN, gpu_backward, gpu_forward, rel_fro,
+                          to_dev)
+
+pytestmark = pytest.mark.gpu
+
+EPS = synth.EPS_BF16_FILTER
+TILE = (128, 256)
+
+CASES_OFF = [
+    synth.TINY,
+    synth.TINY.with_sizes(N=300, V=4096 + 77, D=264),
+    synth.TINY.with_sizes(N=129, V=257, D=8),
+    synth.TINY.with_sizes(N=3, V=1, D=64),
+    synth.GEMMA2_2B.with_sizes(N=600, V=9000),
+    synth.LLAMA3_8B.with_sizes(N=400, V=6000),
+    synth.SMALL_LARGE_VOCAB.with_sizes(N=1500, V=20000),
+]
+CASES_ON = [
+    synth.GEMMA2_2B.with_sizes(N=1000, V=20000),
+    synth.LLAMA3_8B.with_sizes(N=700, V=9000),
+    synth.SMALL_LARGE_VOCAB.with_sizes(N=2000, V=30000),
+    synth.SWEEP.with_sizes(N=512, V=40000),
+    synth.TINY.with_sizes(N=300, V=4096 + 77, D=264),
+]
+
+
+def _run(w, eps, dloss_seed=99):
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    assert st["status"] == 0
+    dloss = synth.random_dloss(dloss_seed, w.N)
+    dE, dC, st = gpu_backward(E, C, y, lse, dloss, eps)
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    return inp, dloss, olse, dE.cpu().numpy(), dC.cpu().numpy(), st
+
+
+@pytest.mark.parametrize("w", CASES_OFF, ids=[w.name for w in CASES_OFF])
+def test_backward_filter_off_matches_exact_gradient(w):
+    inp, dloss, olse, gE, gC, st = _run(w, 0.0)
+    assert st["status"] == 0 and st["flags"] == 0
+    n_tiles = -(-w.N // 128) * -(-w.V // 256)
+    assert st["live_tiles"] == n_tiles and st["dead_tiles"] == 0 and st["pruned_tiles"] == 0
+    rE, rC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
+    if w.V == 1:  # one class: the gradient is exactly zero
+        assert np.abs(gE).max() < 1e-6 and np.abs(gC).max() < 1e-6
+        return
+    assert rel_fro(gE, rE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(gC, rC) <= GRAD_REL_FILTER_OFF
+    ign = inp["y"] == IGN
+    assert (gE[ign] == 0).all()
+
+
+@pytest.mark.parametrize("w", CASES_ON, ids=[w.name for w in CASES_ON])
+def test_backward_filter_on(w):
+    inp, dloss, olse, gE, gC, st = _run(w, EPS)
+    assert st["status"] == 0 and st["flags"] == 0
+    fE, fC, live = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=TILE,
+                                   return_live=True)
+    xE, xC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
+    # same tiles dropped as the oracle's tile filter (the decision sits at
+    # |P - onehot| = eps; fp32 vs fp64 may flip a tile exactly at the edge)
+    assert abs(st["live_tiles"] - int(live.sum())) <= max(1, live.size // 1000)
+    assert st["live_tiles"] + st["dead_tiles"] + st["pruned_tiles"] == live.size
+    # tight against the tile-filtered oracle, spec bar against the exact one
+    assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(gE, xE) <= GRAD_REL_FILTER_ON
+    assert rel_fro(gC, xC) <= GRAD_REL_FILTER_ON
+
+
+def test_filter_threshold_edges():
+    # a huge eps kills every tile except those holding a label (|P - 1| ~ 1);
+    # eps above 1 kills every tile
+    w = synth.GEMMA2_2B.with_sizes(N=512, V=8192, D=256)
+    inp, dloss, olse, gE, gC, st = _run(w, 0.5)
+    live_o = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, 0.5, TILE)
+    assert st["live_tiles"] == int(live_o.sum())
+    yt = {(i // 128, int(inp["y"][i]) // 256) for i in range(w.N)}
+    assert st["live_tiles"] == len(yt)
+    inp, dloss, olse, gE, gC, st = _run(w, 2.0)
+    assert st["live_tiles"] == 0 and (gE == 0).all() and (gC == 0).all()
+
+
+def test_non_flat_blocks_are_recomputed_densely():
+    # token rows with large norms make their blocks' softmax peaky: the
+    # Cauchy-Schwarz pre-pass cannot clear them, so those blocks are visited
+    # in full and non-label tiles there can be live
+    w = synth.GEMMA2_2B.with_sizes(N=640, V=12000, D=256)
+    inp = synth.make_inputs(w)
+    E = oracle.bf16_bits_to_f64(inp["E"])
+    E[128:256] *= 120.0          # block 1: logits with std ~ 1.5
+    E[300] *= 300.0              # one row of block 2
+    inp["E"] = synth.round_to_bf16_bits(E.astype(np.float32))
+    Ed, Cd, yd = to_dev(inp)
+    loss, lse, st = gpu_forward(Ed, Cd, yd)
+    dloss = synth.random_dloss(4, w.N)
+    dE, dC, st = gpu_backward(Ed, Cd, yd, lse, dloss, EPS)
+    assert st["status"] == 0
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    fE, fC, live = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=TILE,
+                                   return_live=True)
+    nv = -(-w.V // 256)
+    label_tiles = {(i // 128, int(inp["y"][i]) // 256) for i in range(w.N)}
+    assert int(live.sum()) > len(label_tiles)          # the peaky blocks have live non-label tiles
+    assert st["live_tiles"] + st["dead_tiles"] >= 2 * nv  # blocks 1 and 2 visited in full
+    assert abs(st["live_tiles"] - int(live.sum())) <= 2
+    assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
+
+
+def test_zero_classifier_closed_form():
+    # C = 0: P = 1/V, dE_i = dloss_i (mean_v C_v - C_y) = 0,
+    # dC_v = (1/V) sum_i dloss_i E_i - sum_{i: y_i = v} dloss_i E_i
+    w = synth.TINY.with_sizes(N=300, V=1000, D=64)
+    inp = synth.make_inputs(w)
+    inp["C"][:] = 0
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    dloss = synth.random_dloss(5, w.N)
+    dE, dC, st = gpu_backward(E, C, y, lse, dloss, 0.0)
+    E64 = oracle.bf16_bits_to_f64(inp["E"])
+    want = np.tile((dloss[:, None] * E64).sum(0) / w.V, (w.V, 1))
+    for i in range(w.N):
+        want[inp["y"][i]] -= dloss[i] * E64[i]
+    assert np.abs(dE.cpu().numpy()).max() == 0.0
+    assert rel_fro(dC.cpu().numpy(), want) <= GRAD_REL_FILTER_OFF
+
+
+def test_gradient_identity_at_scale():
+    # <E, dE> = <C, dC> = sum G * z holds for any (filtered) G
+    import torch
+    w = synth.GEMMA2_2B.with_sizes(N=4096, V=64000)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    dE, dC, st = gpu_backward(E, C, y, lse, synth.mean_dloss(inp["y"]), EPS)
+    a = float((E.double() * dE.double()).sum())
+    b = float((C.double() * dC.double()).sum())
+    assert abs(a - b) <= 1e-2 * max(abs(a), abs(b))
+
+
+def test_backward_repeatable_within_atomic_reordering():
+    w = synth.GEMMA2_2B.with_sizes(N=600, V=9000, D=512)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    dl = synth.random_dloss(3, w.N)
+    a = gpu_backward(E, C, y, lse, dl, 0.0)
+    b = gpu_backward(E, C, y, lse, dl, 0.0)
+    assert rel_fro(a[0].cpu().numpy(), b[0].cpu().numpy()) < 1e-6
+    assert rel_fro(a[1].cpu().numpy(), b[1].cpu().numpy()) < 1e-6
+
+
+def test_autograd_wrapper_matches_oracle():
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.LLAMA3_8B.with_sizes(N=500, V=7000, D=256)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    E.requires_grad_(True)
+    C.requires_grad_(True)
+    out = L.linear_cross_entropy(E, C, y, IGN, filter_eps=0.0)
+    out.backward()
+    ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    keep = inp["y"] != IGN
+    assert abs(float(out) - ol[keep].mean()) <= 1e-4 * abs(ol[keep].mean())
+    rE, rC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, synth.mean_dloss(inp["y"]), IGN)
+    # the wrapper returns bf16 gradients (the dtype of E and C)
+    assert rel_fro(E.grad.float().cpu().numpy(), rE) <= 1e-2
+    assert rel_fro(C.grad.float().cpu().numpy(), rC) <= 1e-2

@@ -60,7 +60,8 @@ def test_raw_logit_tiles_match_definition():
     z = oracle.logits(oracle.bf16_bits_to_f64(inp["E"]), oracle.bf16_bits_to_f64(inp["C"]))
     # bf16 x bf16 products are exact in fp32; only the fp32 accumulation rounds
     assert np.abs(g[:, :V] - z).max() <= 1e-5 * max(1.0, np.abs(z).max())
-    assert (g[:, V:] == 0).all()
+    # the rest of the 32-column group holding column V-1 is zero-filled by TMA
+    assert (g[:, V:(V + 31) // 32 * 32] == 0).all()
 
 
 def test_zero_classifier_gives_log_V():
@@ -161,5 +162,9 @@ def test_library_allocates_no_device_memory():
     torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info()
     assert free1 == free0
-    # the only extra global memory is the caller's workspace: O(N)
-    assert ws.buf.numel() <= 256 + 64 * 8 * w.N + 256
+    # the only extra global memory is the caller's workspace: O(N + V)
+    fwd = L.cce_forward_workspace_size(w.N, w.D, w.V)
+    bwd = L.cce_backward_workspace_size(w.N, w.D, w.V)
+    assert ws.buf.numel() == max(fwd, bwd)
+    assert fwd <= 512 + 64 * 8 * w.N
+    assert bwd <= 4096 + 8 * w.N + 3 * 4 * (w.V // 256 + 64) + 2 * 4 * (w.N // 128 + 64)
