@@ -110,6 +110,32 @@ CCE_API cce_status_t cce_backward(const void* E, const void* C, const int64_t* y
                           int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, float* dE,
                           float* dC, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Allocation-free forward.  The paper has no counterpart: this entry point
+ * exists for callers that cannot allocate device memory when they need the
+ * loss -- code handed only its input and output buffers (plugins, hooks), a
+ * step running under an allocator that is locked, exhausted or forbids
+ * cudaMalloc -- and so cannot supply the workspace cce_forward needs.
+ * Inputs, outputs and results are those of cce_forward.  The scratch (status
+ * block and per-split partials) lives in a static 8 MiB device array inside
+ * the library, which every GPU that loads the library holds until the process
+ * exits.
+ *   - Problems whose forward workspace (cce_forward_workspace_size) exceeds
+ *     8 MiB are rejected with CCE_ERR_WORKSPACE_TOO_SMALL before anything is
+ *     launched (e.g. N = 65536 tokens, V = 262144); invalid sizes or no sm_100
+ *     device give CCE_ERR_INVALID_ARG.
+ *   - No cudaMalloc, cudaFree or other allocating routine is called.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents:
+ *     each call clears the status block it needs and overwrites every partial
+ *     it reads, but calls whose work overlaps on the GPU (unordered streams)
+ *     race on the array and corrupt each other's results.
+ *   - The status block is not readable by the caller; an invalid label still
+ *     shows as a NaN loss. */
+CCE_API cce_status_t cce_forward_noalloc(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D,
+                                         int64_t V, int64_t ignore_index, float* loss, float* lse, void* stream);
+
 /* Synchronises `stream`, then copies the status block of `workspace` (as left
  * by the last call that used it) into *out.  Returns CCE_ERR_TIMEOUT or
  * CCE_ERR_BAD_LABEL if the corresponding flag is set, else CCE_OK. */

@@ -6,7 +6,7 @@ loaded on first use; a missing or unloadable library raises immediately, and
 there is no CPU fallback.
 
 Low-level entry points carry the C names and take raw device pointers
-(Python ints):  cce_forward, cce_backward, cce_forward_workspace_size,
+(Python ints):  cce_forward, cce_forward_noalloc, cce_backward, cce_forward_workspace_size,
 cce_backward_workspace_size, cce_read_status, cce_status_string, cce_version,
 cce_debug_forward_logits, cce_debug_set_wait_limit_ns, cce_debug_set_kernel_events.
 
@@ -23,13 +23,14 @@ from typing import Optional, Tuple
 
 from . import _native
 from ._native import (CCEError, cce_backward, cce_backward_workspace_size, cce_debug_forward_logits,
-                      cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns, cce_forward, cce_forward_workspace_size, cce_read_status,
+                      cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns, cce_forward, cce_forward_noalloc,
+                      cce_forward_workspace_size, cce_read_status,
                       cce_status_string, cce_version, load_library)
 
 IGNORE_INDEX = -100
 
 __all__ = [
-    "CCEError", "IGNORE_INDEX", "cce_forward", "cce_backward", "cce_forward_workspace_size",
+    "CCEError", "IGNORE_INDEX", "cce_forward", "cce_forward_noalloc", "cce_backward", "cce_forward_workspace_size",
     "cce_backward_workspace_size", "cce_read_status", "cce_status_string", "cce_version",
     "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "cce_debug_set_kernel_events", "load_library",
     "forward", "backward", "read_status", "linear_cross_entropy", "Workspace",

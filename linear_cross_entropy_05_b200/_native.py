@@ -60,6 +60,8 @@ def load_library():
         lib.cce_debug_forward_logits.restype = ctypes.c_int
         lib.cce_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         lib.cce_debug_set_wait_limit_ns.restype = None
+        lib.cce_forward_noalloc.argtypes = [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp]
+        lib.cce_forward_noalloc.restype = ctypes.c_int
         lib.cce_debug_set_kernel_events.argtypes = [ctypes.c_int, c_vp, c_vp]
         lib.cce_debug_set_kernel_events.restype = ctypes.c_int
         _lib = lib
@@ -93,6 +95,16 @@ def cce_forward(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: in
                                     stream)
     if check:
         _check(st, "cce_forward")
+    return st
+
+
+def cce_forward_noalloc(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: int, loss: int, lse: int,
+                        stream: int, check: bool = True) -> int:
+    """Forward pass without a workspace, for callers that cannot allocate
+    device memory; scratch is a static 8 MiB device array in the library."""
+    st = load_library().cce_forward_noalloc(E, C, y, N, D, V, ignore_index, loss, lse, stream)
+    if check:
+        _check(st, "cce_forward_noalloc")
     return st
 
 
