@@ -28,6 +28,15 @@ CCE_API cce_status_t cce_debug_forward_logits(const void* E, const void* C, cons
  * Default 1e9 (one second).  Process-wide. */
 CCE_API void cce_debug_set_wait_limit_ns(uint64_t limit_ns);
 
+/* Failure-detection test hook.  While on, the fused kernels' TMA producer
+ * warps issue no copies, so the tensor-core and epilogue warps wait on data
+ * that never comes.  Each wait gives up after the wait limit (see
+ * cce_debug_set_wait_limit_ns), the CTA unwinds, frees its tensor memory and
+ * exits, and the call's status block carries the timeout flag
+ * (cce_read_status returns CCE_ERR_TIMEOUT).  Outputs are meaningless while
+ * it is on.  Process-wide; 0 turns it off. */
+CCE_API void cce_debug_withhold_loads(int on);
+
 /* Profiling hook.  While set, every launch of the selected kernel records
  * `start_event` on the call's stream immediately before the launch and
  * `stop_event` immediately after it, so the caller can time that kernel alone

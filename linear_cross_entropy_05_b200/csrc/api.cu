@@ -20,8 +20,8 @@ cudaError_t launch_fwd_lse(const CUtensorMap& tmE, const CUtensorMap& tmC, const
                            cudaStream_t stream);
 cudaError_t launch_fwd_finalize(const void* E, const void* C, const int64_t* y, const FinArgs& a, float* loss,
                                 float* lse, cudaStream_t stream);
-cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const BwdArgs& a, int grid,
-                       cudaStream_t stream);
+cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
+                       const CUtensorMap& tmdC, const BwdArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
                         int sms, cudaStream_t stream);
 }  // namespace cce
@@ -31,6 +31,9 @@ using namespace cce;
 namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
+
+// Test hook: when set, the next launches' TMA producers issue no copies.
+std::atomic<int> g_withhold_loads{0};
 
 // Optional per-kernel timing events (debug hook): [kernel][0 = start, 1 = stop].
 std::atomic<void*> g_events[2][2] = {{{nullptr}, {nullptr}}, {{nullptr}, {nullptr}}};
@@ -121,6 +124,21 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t D, int b
   return r == CUDA_SUCCESS;
 }
 
+// fp32 gradient tensor [rows][D] as 32 x 32 boxes with 128-byte swizzle: the
+// target of the backward kernel's bulk reduce-adds.
+bool make_map_f32(CUtensorMap* map, const void* base, int64_t rows, int64_t D) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 struct FwdPlan {
   int n_mblk, n_vtile, n_split, grid;
   size_t ws_bytes;
@@ -194,10 +212,13 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   a.n_vtile = p.n_vtile;
   a.n_split = p.n_split;
   a.n_units = p.n_mblk * p.n_split;
+  // keep at most ~48 MB of E rows in flight so they stay resident in the 126 MB L2
+  a.group_m = (int)std::max<int64_t>(1, std::min<int64_t>(p.n_mblk, (48ll << 20) / ((int64_t)BM * D * 2)));
   a.partial = partial;
   a.dbg_logits = dbg_logits;
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
+  a.withhold_loads = g_withhold_loads.load();
   if (record_event(0, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (launch_fwd_lse(tmE, tmC, a, p.grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (record_event(0, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
@@ -247,6 +268,8 @@ void cce_debug_set_wait_limit_ns(uint64_t limit_ns) {
   g_wait_limit_ns.store(limit_ns ? limit_ns : 1000000000ull);
 }
 
+void cce_debug_withhold_loads(int on) { g_withhold_loads.store(on ? 1 : 0); }
+
 cce_status_t cce_debug_set_kernel_events(int kernel, void* start_event, void* stop_event) {
   if (kernel < 0 || kernel > 1) return CCE_ERR_INVALID_ARG;
   g_events[kernel][0].store(start_event);
@@ -270,8 +293,10 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
   if (workspace_bytes < bp.ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
-  CUtensorMap tmE, tmC;
-  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN)) return CCE_ERR_CUDA;
+  CUtensorMap tmE, tmC, tmdE, tmdC;
+  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN) || !make_map_f32(&tmdE, dE, N, D) ||
+      !make_map_f32(&tmdC, dC, V, D))
+    return CCE_ERR_CUDA;
   char* ws = reinterpret_cast<char*>(workspace);
   unsigned long long* status = reinterpret_cast<unsigned long long*>(ws);
   const bool filter_on = filter_eps > 0.f;
@@ -300,6 +325,7 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
   a.dC = dC;
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
+  a.withhold_loads = g_withhold_loads.load();
 
   if (filter_on) {
     PrepArgs pp;
@@ -322,7 +348,7 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
   }
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
-  if (launch_bwd(tmE, tmC, a, grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (launch_bwd(tmE, tmC, tmdE, tmdC, a, grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
   return CCE_OK;
 }

@@ -11,12 +11,15 @@
 //     dC[v-tile,  d-chunk] += G^T . E[m-block, d-chunk]    (2 x M=128, N=64, K=128)
 // The C and E slices are the same TMA tiles the recompute streams (128-byte
 // swizzled rows of 64 d values); read K-major for S and MN-major for the
-// contractions.  Partial products are added to fp32 dE/dC with vector
-// reductions in L2.
+// contractions.  Partial products are added to fp32 dE/dC by the TMA engine
+// (bulk tensor reduce-add from a swizzled shared staging tile).
 //
 // Roles (192 threads): warp 0 TMA producer, warp 1 UMMA issuer, warps 2-5
 // epilogue (one TMEM lane = one token row / one vocabulary row per thread).
-// TMEM columns: [0,256) logit tile, [256,320) dE chunk, [320,448) dC chunk.
+// TMEM columns: [0,256) logit tile; contraction accumulators double-buffered:
+// buffer 0 = dE chunk [256,320) + dC chunk [320,448), buffer 1 = dE [0,64) +
+// dC [64,192) (inside the logit tile's columns, free once the epilogue has
+// read the tile; the next tile's logits wait until buffer 1 is drained).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -28,8 +31,8 @@ namespace cce {
 
 namespace {
 constexpr uint32_t TM_S = 0;
-constexpr uint32_t TM_DE = 256;
-constexpr uint32_t TM_DC = 320;
+__device__ __forceinline__ uint32_t tm_de(int b) { return b ? 0u : 256u; }   // dE chunk of buffer b
+__device__ __forceinline__ uint32_t tm_dc(int b) { return b ? 64u : 320u; }   // dC chunk of buffer b
 
 __device__ __forceinline__ void tile_coords(int t, int n_mblk, int n_vtile, int group_m, int& m, int& vt) {
   // Raster: groups of group_m token blocks; inside a group the token block
@@ -44,27 +47,24 @@ __device__ __forceinline__ void tile_coords(int t, int n_mblk, int n_vtile, int 
 }
 
 // Adds a 32 x 32 fp32 block held one row per lane (32 consecutive columns
-// each) to global memory.  The block is staged through a 4 KB per-warp buffer
-// with 16-byte chunks XOR-swizzled by row, then read back so that each warp
-// instruction covers four rows x 128 contiguous bytes: the vector reductions
-// reach L2 as whole cache lines instead of 32 scattered 16-byte pieces.
-//   base: element (row 0, column 0) of the block; ld: row stride (elements)
-//   row_ok: bit r set if row r exists; ncols: valid columns (multiple of 4)
-__device__ __forceinline__ void red_block32(uint8_t* xb, int lane, const float (&v)[32], float* base, size_t ld,
-                                            uint32_t row_ok, int ncols) {
+// each) to global memory through the TMA engine: the block is written to the
+// warp's 4 KB staging buffer in the 128-byte-swizzled layout of a {32, 32}
+// fp32 box and reduced into the tensor at (x = column, y = row) by one bulk
+// tensor reduce-add.  Rows/columns past the tensor's extent are clipped.
+__device__ __forceinline__ void tma_red_block32(uint8_t* xb, int lane, const float (&v)[32], const CUtensorMap* map,
+                                                int x, int y) {
+  if (lane == 0) bulk_wait_group_read0();  // the previous block has left the buffer
+  __syncwarp();
 #pragma unroll
   for (int q = 0; q < 8; ++q)
     *reinterpret_cast<float4*>(xb + lane * 128 + ((q ^ (lane & 7)) << 4)) =
         make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  fence_proxy_async_smem();
   __syncwarp();
-  const int q = lane & 7;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = 4 * i + (lane >> 3);
-    const float4 t = *reinterpret_cast<const float4*>(xb + r * 128 + ((q ^ (r & 7)) << 4));
-    if (((row_ok >> r) & 1u) && q * 4 < ncols) red_add_v4(base + (size_t)r * ld + q * 4, t.x, t.y, t.z, t.w);
+  if (lane == 0) {
+    tma_reduce_add_2d(map, xb, x, y);
+    bulk_commit_group();
   }
-  __syncwarp();
 }
 
 // Work item t -> (token block m, vocabulary tile vt).  Dense mode rasters the
@@ -105,7 +105,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }  // namespace
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    bwd_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC, const BwdArgs a) {
+    bwd_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
+               const __grid_constant__ CUtensorMap tmdE, const __grid_constant__ CUtensorMap tmdC, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                                   // BWD_STAGES x [128][64] bf16 (E slices)
@@ -119,9 +120,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* s_empty = s_full + 1;
   uint64_t* g_full = s_full + 2;
   uint64_t* g_empty = s_full + 3;
-  uint64_t* c_full = s_full + 4;
-  uint64_t* c_empty = s_full + 5;
-  uint64_t* drain = s_full + 6;
+  uint64_t* c_full = s_full + 4;   // [2] per accumulator buffer
+  uint64_t* c_empty = s_full + 6;  // [2]
+  uint64_t* drain = s_full + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   // Per-tile live votes, a ring of 8 slots indexed by the CTA's tile counter.
@@ -142,8 +143,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(s_empty, BM);
     mbar_init(g_full, BM);
     mbar_init(g_empty, 1);
-    mbar_init(c_full, 1);
-    mbar_init(c_empty, BM);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&c_full[b], 1);
+      mbar_init(&c_empty[b], BM);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     for (int i = 0; i < 8; ++i) live_ring[i] = 0;
@@ -156,6 +159,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 32) {
     tma_prefetch_map(&tmE);
     tma_prefetch_map(&tmC);
+    tma_prefetch_map(&tmdE);
+    tma_prefetch_map(&tmdC);
   }
   tc_fence_before();
   __syncthreads();
@@ -172,7 +177,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int kt = 0;
       TileMap tm;
       tm.init(a);
-      for (int t = blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
+      // withhold_loads (test hook): no copy is issued; see the forward kernel.
+      for (int t = a.withhold_loads ? tm.T : blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
         int m, vt;
         tm.get(a, t, m, vt);
         // logit recompute slices, then (if the tile is live) the same slices
@@ -211,13 +217,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC_DC = idesc_bf16_f32(BM, 64, true, true);
       const uint32_t g_addr = smem_u32(sG);
       int stage = 0;
-      uint32_t phase = 0, sph = 0, gph = 0, cph = 0;
+      uint32_t phase = 0, sph = 0, gph = 0;
+      uint32_t cfill0 = 0u, cfill1 = 0u;  // fills of contraction buffers 0 / 1 so far
       int kt = 0;
       TileMap tm;
       tm.init(a);
       for (int t = blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
         if (!mbar_wait(s_empty, sph ^ 1u, wc)) goto mma_done;
         sph ^= 1u;
+        // buffer 1 lives in the logit tile's columns: wait until it is drained
+        if (!mbar_wait(&c_empty[1], (cfill1 & 1u) ^ 1u, wc)) goto mma_done;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
@@ -240,16 +249,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         if (live_ring[kt & 7]) {
           for (int kb = 0; kb < nkb; ++kb) {
+            const int b = kb & 1;
             if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
-            if (!mbar_wait(c_empty, cph ^ 1u, wc)) goto mma_done;
-            cph ^= 1u;
+            if (!mbar_wait(&c_empty[b], ((b ? cfill1 : cfill0) & 1u) ^ 1u, wc)) goto mma_done;
+            if (b) ++cfill1; else ++cfill0;
             tc_fence_after();
             const uint32_t e_addr = smem_u32(sA + stage * A_STAGE_BYTES);  // E[m-block, d-chunk]: 128 tok x 64 d
             const uint32_t c_addr = smem_u32(sB + stage * B_STAGE_BYTES);  // C[v-tile, d-chunk]: 256 voc x 64 d
             // dE chunk = G (128 tok x 256 voc, K-major) . Cchunk (K = voc rows, MN = d)
 #pragma unroll
             for (int k = 0; k < BN / 16; ++k)
-              umma_bf16(tmem_base + TM_DE,
+              umma_bf16(tmem_base + tm_de(b),
                         sdesc_sw128(g_addr + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024),
                         sdesc_sw128(c_addr + k * 2048, 16384, 1024), IDESC_DE, k != 0);
             // dC chunk, vocabulary half h = G^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
@@ -257,11 +267,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int h = 0; h < 2; ++h)
 #pragma unroll
               for (int k = 0; k < BM / 16; ++k)
-                umma_bf16(tmem_base + TM_DC + h * 64,
+                umma_bf16(tmem_base + tm_dc(b) + h * 64,
                           sdesc_sw128(g_addr + (2 * h) * (BM * 128) + k * 2048, BM * 128, 1024),
                           sdesc_sw128(e_addr + k * 2048, 16384, 1024), IDESC_DC, k != 0);
             umma_commit(&empty[stage]);
-            umma_commit(c_full);
+            umma_commit(&c_full[b]);
             if (++stage == BWD_STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -287,7 +297,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_addr = (uint32_t)(lane_grp * 32) << 16;
     const float eps = a.filter_eps;
     const bool filter_on = eps > 0.f;
-    uint32_t sph = 0, gph = 0, cph = 0;
+    uint32_t sph = 0, gph = 0;
+    uint32_t cfe0 = 0u, cfe1 = 0u;  // drains of contraction buffers 0 / 1 so far
     unsigned long long n_live = 0, n_dead = 0;
     uint8_t* g_row = sG + rib * 128;
     uint8_t* xb = sX + (warp - 2) * 4096;
@@ -359,46 +370,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         continue;
       }
       ++n_live;
-      const int vrow0 = vt * BN + rib;
-      const uint32_t rows_dE = __ballot_sync(0xffffffffu, valid);
       bool ok = true;
+      const int row0 = m * BM + lane_grp * 32;           // first dE row of this warp
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(c_full, cph, wc)) {
+        const int b = kb & 1;
+        if (!mbar_wait(&c_full[b], (b ? cfe1 : cfe0) & 1u, wc)) {
           ok = false;
           break;
         }
-        cph ^= 1u;
+        if (b) ++cfe1; else ++cfe0;
         tc_fence_after();
         const int d0 = kb * BK;
-        // dE rows of this warp: tokens m*128 + lane_grp*32 + r
+        // dE rows of this warp: tokens row0 .. row0 + 31
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
           float v[32];
-          tmem_ld32(tmem_base + lane_addr + TM_DE + q * 32, v);
-          const int c0 = d0 + q * 32;
-          if (c0 < a.D)
-            red_block32(xb, lane, v, a.dE + (size_t)(m * BM + lane_grp * 32) * a.D + c0, (size_t)a.D, rows_dE,
-                        min(32, a.D - c0));
+          tmem_ld32(tmem_base + lane_addr + tm_de(b) + q * 32, v);
+          if (d0 + q * 32 < a.D && row0 < a.N) tma_red_block32(xb, lane, v, &tmdE, d0 + q * 32, row0);
         }
-        // dC rows of this warp: vocabulary rows vt*256 + h*128 + lane_grp*32 + r
+        // dC rows of this warp: vocabulary rows vt*256 + h*128 + lane_grp*32 ..
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          const uint32_t rows_dC = __ballot_sync(0xffffffffu, vrow0 + h * BM < a.V);
+          const int vr0 = vt * BN + h * BM + lane_grp * 32;
 #pragma unroll 1
           for (int q = 0; q < 2; ++q) {
             float v[32];
-            tmem_ld32(tmem_base + lane_addr + TM_DC + h * 64 + q * 32, v);
-            const int c0 = d0 + q * 32;
-            if (c0 < a.D)
-              red_block32(xb, lane, v, a.dC + (size_t)(vt * BN + h * BM + lane_grp * 32) * a.D + c0, (size_t)a.D,
-                          rows_dC, min(32, a.D - c0));
+            tmem_ld32(tmem_base + lane_addr + tm_dc(b) + h * 64 + q * 32, v);
+            if (d0 + q * 32 < a.D && vr0 < a.V) tma_red_block32(xb, lane, v, &tmdC, d0 + q * 32, vr0);
           }
         }
         tc_fence_before();
-        mbar_arrive(c_empty);
+        mbar_arrive(&c_empty[b]);
       }
       if (!ok) break;
     }
+    if (lane == 0) bulk_wait_group0();  // every reduction issued by this warp has landed
     if (rib == 0) {
       atomicAdd(a.status + ST_LIVE_TILES, n_live);
       atomicAdd(a.status + ST_DEAD_TILES, n_dead);
@@ -419,12 +425,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 size_t bwd_smem_bytes() { return 1024 + (size_t)BWD_STAGES * STAGE_BYTES + G_BYTES + 4 * 4096 + 256; }
 
-cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const BwdArgs& a, int grid,
-                       cudaStream_t stream) {
+cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
+                       const CUtensorMap& tmdC, const BwdArgs& a, int grid, cudaStream_t stream) {
   const size_t smem = bwd_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  bwd_kernel<<<grid, NUM_THREADS, smem, stream>>>(tmE, tmC, a);
+  bwd_kernel<<<grid, NUM_THREADS, smem, stream>>>(tmE, tmC, tmdE, tmdC, a);
   return cudaGetLastError();
 }
 

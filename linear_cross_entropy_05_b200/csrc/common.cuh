@@ -50,10 +50,12 @@ struct FwdArgs {
   int n_vtile;     // ceil(V / BN)
   int n_split;     // vocabulary splits per token block
   int n_units;     // n_mblk * n_split
+  int group_m;     // token blocks per raster group (their E rows stay in L2)
   float2* partial; // [n_split][N]: (running max, sum of exp(z - max)) per split
   float* dbg_logits;           // optional [N][n_vtile * BN] raw logits (debug build entry only)
   unsigned long long* status;
   unsigned long long wait_limit_ns;
+  int withhold_loads;          // test hook: the TMA producer issues nothing
 };
 
 struct FinArgs {
@@ -95,7 +97,21 @@ struct BwdArgs {
   float* dC;            // [V][D] fp32, accumulated
   unsigned long long* status;
   unsigned long long wait_limit_ns;
+  int withhold_loads;   // test hook: the TMA producer issues nothing
 };
+
+// Work unit u -> (vocabulary split r, token block m).  Units are grouped by
+// group_m token blocks; inside a group the token block varies fastest, so the
+// CTAs running at the same time share a few splits (C tiles) and a bounded
+// set of E rows, both L2-resident.
+__host__ __device__ inline void unit_coords(int u, int n_mblk, int n_split, int group_m, int& r, int& m) {
+  const int gsz = group_m * n_split;
+  const int g = u / gsz;
+  const int rem = u - g * gsz;
+  const int gm = min(group_m, n_mblk - g * group_m);
+  r = rem / gm;
+  m = g * group_m + (rem - r * gm);
+}
 
 __host__ __device__ inline void split_range(int r, int n_vtile, int n_split, int& v0, int& v1) {
   v0 = (int)(((long long)r * n_vtile) / n_split);

@@ -6,7 +6,8 @@
 // the fly, with the matrix products and the reduction kept on chip.
 //
 // fwd_lse_kernel  persistent, warp-specialised tcgen05 kernel.  A work unit is
-//                 (token block m of 128 rows, vocabulary split r).  For every
+//                 (token block m of 128 rows, vocabulary split r), dealt in
+//                 groups of token blocks whose E rows fit in L2.  For every
 //                 256-wide vocabulary tile of the split the logit tile
 //                 S = E_m C_tile^T is accumulated in TMEM (double buffered),
 //                 and the epilogue warps fold it into a per-row running
@@ -78,8 +79,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0;  // stages armed at least once
-      for (int u = blockIdx.x; u < a.n_units; u += gridDim.x) {
-        const int r = u / a.n_mblk, m = u - r * a.n_mblk;
+      // withhold_loads (test hook): no copy is issued, so the MMA warp's first
+      // wait can only end by its time limit; that path must unwind cleanly.
+      for (int u = a.withhold_loads ? a.n_units : blockIdx.x; u < a.n_units; u += gridDim.x) {
+        int r, m;
+        unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m);
         int v0, v1;
         split_range(r, a.n_vtile, a.n_split, v0, v1);
         for (int vt = v0; vt < v1; ++vt) {
@@ -116,7 +120,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int u = blockIdx.x; u < a.n_units; u += gridDim.x) {
-        const int r = u / a.n_mblk;
+        int r, m;
+        unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m);
         int v0, v1;
         split_range(r, a.n_vtile, a.n_split, v0, v1);
         for (int vt = v0; vt < v1; ++vt) {
@@ -163,7 +168,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int u = blockIdx.x; u < a.n_units; u += gridDim.x) {
-      const int r = u / a.n_mblk, m = u - r * a.n_mblk;
+      int r, m;
+        unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m);
       int v0, v1;
       split_range(r, a.n_vtile, a.n_split, v0, v1);
       float mrun = -INFINITY, srun = 0.f;
