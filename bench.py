@@ -34,7 +34,8 @@ sys.path.insert(0, ROOT)
 METRIC = "CCE fwd+bwd tokens/s"
 UNIT = "tokens/s"
 IGN = -100
-BM, BN = 128, 256
+BM, BN = 128, 256      # logit tile (token block x vocabulary tile)
+FT = 128               # the gradient filter's unit: 128 tokens x FT vocabulary entries
 
 
 def log(*a):
@@ -198,7 +199,7 @@ def oracle_step(inp, rows, eps):
     y = inp["y"][rows]
     loss, lse = oracle.forward_f64(E64, C64, y, IGN)
     dl = np.full(len(rows), 1.0 / max(1, len(rows)))
-    dE, dC = oracle.backward_f64(E64, C64, y, lse, dl, IGN, filter_eps=eps, tile=(BM, BN))
+    dE, dC = oracle.backward_f64(E64, C64, y, lse, dl, IGN, filter_eps=eps, tile=(BM, FT))
     return loss
 
 
@@ -371,10 +372,10 @@ def run_gpu(args, w):
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = measured_peaks()
-    tile_flop = 2.0 * BM * BN * D
-    n_tiles = live + dead
+    unit_flop = 2.0 * BM * FT * D          # one 128 x 128 filter unit of logits
+    n_tiles = live + dead                  # filter units recomputed
     flop_fwd = 2.0 * N * D * V
-    flop_bwd = n_tiles * tile_flop + live * 2.0 * tile_flop
+    flop_bwd = n_tiles * unit_flop + live * 2.0 * unit_flop
     dominant = "bwd_kernel" if bwd_ms >= fwd_ms else "fwd_lse_kernel"
     dom_flop, dom_ms = (flop_bwd, bwd_ms) if dominant == "bwd_kernel" else (flop_fwd, fwd_ms)
     peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
@@ -454,9 +455,9 @@ def run_suite(args):
             torch.cuda.synchronize()
             tf += ev[0].elapsed_time(ev[1]) / reps
             tb += ev[1].elapsed_time(ev[2]) / reps
-        tile = 2.0 * BM * BN * D
+        unit = 2.0 * BM * FT * D
         visited = st["live_tiles"] + st["dead_tiles"]
-        executed = 2.0 * N * D * V + visited * tile + st["live_tiles"] * 2.0 * tile
+        executed = 2.0 * N * D * V + visited * unit + st["live_tiles"] * 2.0 * unit
         print(json.dumps({
             "workload": w.name, "N": N, "D": D, "V": V, "filter_eps": w.filter_eps,
             "fwd_ms": tf, "fwd_tokens_per_s": N / tf * 1e3, "fwd_frac_of_peak": 2.0 * N * D * V / tf / 1e9 / peak,

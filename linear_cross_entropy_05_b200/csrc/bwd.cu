@@ -3,12 +3,13 @@
 //
 // Cut Cross-Entropy abstract, sentences 4 and 9: the logits are never stored,
 // so the backward pass recomputes each 128 x 256 logit tile S = E_m C_v^T in
-// TMEM, forms P = exp(S - lse) and D = P - onehot(y) in registers, and skips
-// the tile when every |D| is below filter_eps (gradient work under numerical
-// precision).  Live tiles are written as G = dloss * D in bf16 to shared
-// memory and contracted on the tensor cores:
-//     dE[m-block, d-chunk] += G   . C[v-tile, d-chunk]     (M=128, N=64, K=256)
-//     dC[v-tile,  d-chunk] += G^T . E[m-block, d-chunk]    (2 x M=128, N=64, K=128)
+// TMEM and forms P = exp(S - lse) and D = P - onehot(y) in registers.  The
+// filter works on 128 x 128 units (two per logit tile): a unit whose every
+// |D| is below filter_eps is dropped (gradient work under numerical
+// precision).  G = dloss * D goes to shared memory in bf16 and the live units
+// are contracted on the tensor cores:
+//     dE[m-block, d-chunk] += sum over live halves h of G_h . C_h[d-chunk]   (M=128, N=64, K=128 each)
+//     dC[v-half h, d-chunk] += G_h^T . E[m-block, d-chunk]                  (M=128, N=64, K=128)
 // The C and E slices are the same TMA tiles the recompute streams (128-byte
 // swizzled rows of 64 d values); read K-major for S and MN-major for the
 // contractions.  Partial products are added to fp32 dE/dC by the TMA engine
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (pass == 1) {
             if (!mbar_wait(g_full, gph, wc)) goto producer_done;
             gph ^= 1u;
-            if (!live_ring[kt & 7]) break;
+            if (live_ring[kt & 7] == 0) break;
           }
           for (int kb = 0; kb < nkb; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
@@ -247,7 +248,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(g_full, gph, wc)) goto mma_done;
         gph ^= 1u;
         tc_fence_after();
-        if (live_ring[kt & 7]) {
+        const int hmask = live_ring[kt & 7];  // bit h: 128-column half h is live
+        if (hmask) {
           for (int kb = 0; kb < nkb; ++kb) {
             const int b = kb & 1;
             if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
@@ -256,20 +258,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint32_t e_addr = smem_u32(sA + stage * A_STAGE_BYTES);  // E[m-block, d-chunk]: 128 tok x 64 d
             const uint32_t c_addr = smem_u32(sB + stage * B_STAGE_BYTES);  // C[v-tile, d-chunk]: 256 voc x 64 d
-            // dE chunk = G (128 tok x 256 voc, K-major) . Cchunk (K = voc rows, MN = d)
+            uint32_t acc_de = 0;
 #pragma unroll
-            for (int k = 0; k < BN / 16; ++k)
-              umma_bf16(tmem_base + tm_de(b),
-                        sdesc_sw128(g_addr + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024),
-                        sdesc_sw128(c_addr + k * 2048, 16384, 1024), IDESC_DE, k != 0);
-            // dC chunk, vocabulary half h = G^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
+            for (int h = 0; h < 2; ++h) {
+              if (!((hmask >> h) & 1)) continue;
+              // dE chunk += G_h (128 tok x 128 voc, K-major) . C_h chunk (K = voc rows, MN = d)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+              for (int k = 8 * h; k < 8 * h + 8; ++k) {
+                umma_bf16(tmem_base + tm_de(b),
+                          sdesc_sw128(g_addr + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024),
+                          sdesc_sw128(c_addr + k * 2048, 16384, 1024), IDESC_DE, acc_de);
+                acc_de = 1;
+              }
+              // dC chunk of half h = G_h^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
 #pragma unroll
               for (int k = 0; k < BM / 16; ++k)
                 umma_bf16(tmem_base + tm_dc(b) + h * 64,
                           sdesc_sw128(g_addr + (2 * h) * (BM * 128) + k * 2048, BM * 128, 1024),
                           sdesc_sw128(e_addr + k * 2048, 16384, 1024), IDESC_DC, k != 0);
+            }
             umma_commit(&empty[stage]);
             umma_commit(&c_full[b]);
             if (++stage == BWD_STAGES) {
@@ -326,7 +333,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       sph ^= 1u;
       if (!mbar_wait(g_empty, gph ^ 1u, wc)) break;
       tc_fence_after();
-      bool live = !filter_on;
+      // bit h: some |D| >= eps in the 128-column half h (every existing half
+      // when the filter is off)
+      const uint32_t halves = ncols > 128 ? 3u : 1u;
+      uint32_t live = filter_on ? 0u : halves;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float x[32];
@@ -341,7 +351,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             float p = ex2_approx(fmaf(x[j + q], LOG2E, -lse2));
             float d = (col == ycol) ? p - 1.f : p;
             d = (valid && col < ncols) ? d : 0.f;
-            live |= fabsf(d) >= eps;
+            live |= (filter_on && fabsf(d) >= eps ? 1u : 0u) << (c >> 2);
             g2[q] = dl * d;
           }
           pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
@@ -358,18 +368,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       mbar_arrive(s_empty);
       fence_proxy_async_smem();
-      if (__any_sync(0xffffffffu, live) && lane == 0) atomicOr(const_cast<int*>(&live_ring[kt & 7]), 1);
+      const uint32_t wmask = __reduce_or_sync(0xffffffffu, live);
+      if (wmask && lane == 0) atomicOr(const_cast<int*>(&live_ring[kt & 7]), (int)wmask);
       __syncwarp();
       if (rib == 0) live_ring[(kt + 4) & 7] = 0;
       mbar_arrive(g_full);
       if (!mbar_wait(g_full, gph, wc)) break;
       gph ^= 1u;
-      const bool live_any = live_ring[kt & 7] != 0;
-      if (!live_any) {
-        ++n_dead;
-        continue;
-      }
-      ++n_live;
+      const uint32_t hmask = (uint32_t)live_ring[kt & 7];
+      n_live += __popc(hmask);
+      n_dead += __popc(halves & ~hmask);
+      if (!hmask) continue;
       bool ok = true;
       const int row0 = m * BM + lane_grp * 32;           // first dE row of this warp
       for (int kb = 0; kb < nkb; ++kb) {
@@ -391,6 +400,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // dC rows of this warp: vocabulary rows vt*256 + h*128 + lane_grp*32 ..
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
+          if (!((hmask >> h) & 1)) continue;
           const int vr0 = vt * BN + h * BM + lane_grp * 32;
 #pragma unroll 1
           for (int q = 0; q < 2; ++q) {
