@@ -338,37 +338,58 @@ def run_gpu(args, w):
     step_ms = 1e3 * sec / K
 
     # ---- end to end through the public API with host buffers ----
+    # Every step copies its inputs (E, C, y, dloss) from pinned host memory
+    # and reads its per-token loss back.  Two device input buffers let step
+    # k+1's copy (on a copy stream) overlap step k's kernels.
     E_h = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).pin_memory()
     C_h = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).pin_memory()
     y_h = torch.from_numpy(inp["y"]).pin_memory()
     dl_h = torch.from_numpy(synth.mean_dloss(inp["y"])).pin_memory()
-    loss_h = torch.empty(N, dtype=torch.float32).pin_memory()
-    Ke = max(3, K // 4)
-
-    def e2e_step():
-        E.copy_(E_h, non_blocking=True)
-        C.copy_(C_h, non_blocking=True)
-        y.copy_(y_h, non_blocking=True)
-        dloss.copy_(dl_h, non_blocking=True)
-        step()
-        loss_h.copy_(loss, non_blocking=True)
-
     h2d = E_h.numel() * 2 + C_h.numel() * 2 + y_h.numel() * 8 + dl_h.numel() * 4
-    d2h = loss_h.numel() * 4
+    d2h = N * 4
     e2e_value = None
     if not args.no_e2e:
-        e2e_step()
+        Ke = max(3, K // 4)
+        bufs = [(E, C, y, dloss)]
+        bufs.append((torch.empty_like(E), torch.empty_like(C), torch.empty_like(y), torch.empty_like(dloss)))
+        loss_h = [torch.empty(N, dtype=torch.float32).pin_memory() for _ in range(2)]
+        copy_stream = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        consumed = [torch.cuda.Event() for _ in range(2)]
+        for b in range(2):
+            consumed[b].record(stream)
+
+        def e2e_run(steps):
+            for k in range(steps):
+                b = k % 2
+                Eb, Cb, yb, dlb = bufs[b]
+                with torch.cuda.stream(copy_stream):
+                    copy_stream.wait_event(consumed[b])
+                    Eb.copy_(E_h, non_blocking=True)
+                    Cb.copy_(C_h, non_blocking=True)
+                    yb.copy_(y_h, non_blocking=True)
+                    dlb.copy_(dl_h, non_blocking=True)
+                    copied[b].record(copy_stream)
+                stream.wait_event(copied[b])
+                L.forward(Eb, Cb, yb, IGN, workspace=ws_f, out=(loss, lse))
+                L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC))
+                loss_h[b].copy_(loss, non_blocking=True)
+                consumed[b].record(stream)
+
+        e2e_run(2)
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(Ke):
-            e2e_step()
+        e2e_run(Ke)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_value, _ = aggregate_throughput(dist, float(N * Ke), e0.elapsed_time(e1) / 1e3, dev)
+        if not np.isfinite(loss_h[(Ke - 1) % 2].numpy()).all():
+            raise RuntimeError("end-to-end loss read back non-finite values")
+        del bufs
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = measured_peaks()
@@ -391,7 +412,7 @@ def run_gpu(args, w):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded numpy PCG64; random-init classifier, Zipf labels)",
-            "config": config_of(w, world),
+            "config": dict(config_of(w, world), forward_kernel=args.fwd_variant),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
@@ -405,7 +426,9 @@ def run_gpu(args, w):
             "extra_hbm_bytes": int(extra_hbm),
             "materialised_logits_fp32_bytes": N * V * 4,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-            "gpu_launches": 3 * K,
+            # our kernels per step: fwd_lse + fwd_finalize, bwd_kernel, and with
+            # the filter on the four pre-pass kernels (cnorm, blocks, scan, scatter)
+            "gpu_launches": (3 + (4 if eps > 0 else 0)) * K,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -486,9 +509,14 @@ def main(argv=None):
                     help="workload name (the default is the headline Gemma-2-2B-shaped head)")
     ap.add_argument("--N", type=int, default=None, help="override tokens (profiling cases)")
     ap.add_argument("--V", type=int, default=None, help="override vocabulary (profiling cases)")
+    ap.add_argument("--fwd-variant", choices=["single", "pair"], default="single",
+                    help="forward kernel: single CTAs (default) or CTA pairs (A/B measurement)")
     ap.add_argument("--suite", action="store_true",
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
+    if args.fwd_variant == "pair":
+        import linear_cross_entropy_05_b200 as L
+        L.cce_debug_set_forward_variant(1)
     if args.suite:
         return run_suite(args)
     if args.warmup < 3:

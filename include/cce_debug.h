@@ -37,6 +37,15 @@ CCE_API void cce_debug_set_wait_limit_ns(uint64_t limit_ns);
  * it is on.  Process-wide; 0 turns it off. */
 CCE_API void cce_debug_withhold_loads(int on);
 
+/* Selects the forward logit/LSE kernel: 0 = one SM per 128 x 256 logit tile
+ * (the default), 1 = CTA pairs (two SMs per 256 x 256 tile through tcgen05
+ * cta_group::2, half the shared-memory operand traffic per SM).  Both give
+ * the same loss up to fp32 rounding order; the switch exists for A/B
+ * measurement (on the power-capped B200 the two run within a few percent).  The forward workspace size depends on
+ * the variant: query cce_forward_workspace_size after switching.
+ * Process-wide.  Returns CCE_ERR_INVALID_ARG for other values. */
+CCE_API cce_status_t cce_debug_set_forward_variant(int variant);
+
 /* Profiling hook.  While set, every launch of the selected kernel records
  * `start_event` on the call's stream immediately before the launch and
  * `stop_event` immediately after it, so the caller can time that kernel alone

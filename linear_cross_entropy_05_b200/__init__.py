@@ -23,7 +23,8 @@ from typing import Optional, Tuple
 
 from . import _native
 from ._native import (CCEError, cce_backward, cce_backward_workspace_size, cce_debug_forward_logits,
-                      cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns, cce_debug_withhold_loads, cce_forward, cce_forward_noalloc,
+                      cce_debug_set_forward_variant, cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns,
+                      cce_debug_withhold_loads, cce_forward, cce_forward_noalloc,
                       cce_forward_workspace_size, cce_read_status,
                       cce_status_string, cce_version, load_library)
 
@@ -32,7 +33,7 @@ IGNORE_INDEX = -100
 __all__ = [
     "CCEError", "IGNORE_INDEX", "cce_forward", "cce_forward_noalloc", "cce_backward", "cce_forward_workspace_size",
     "cce_backward_workspace_size", "cce_read_status", "cce_status_string", "cce_version",
-    "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "cce_debug_set_kernel_events", "cce_debug_withhold_loads",
+    "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "cce_debug_set_kernel_events", "cce_debug_withhold_loads", "cce_debug_set_forward_variant",
     "load_library",
     "forward", "backward", "read_status", "linear_cross_entropy", "Workspace",
 ]

@@ -62,6 +62,8 @@ def load_library():
         lib.cce_debug_set_wait_limit_ns.restype = None
         lib.cce_forward_noalloc.argtypes = [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp]
         lib.cce_forward_noalloc.restype = ctypes.c_int
+        lib.cce_debug_set_forward_variant.argtypes = [ctypes.c_int]
+        lib.cce_debug_set_forward_variant.restype = ctypes.c_int
         lib.cce_debug_withhold_loads.argtypes = [ctypes.c_int]
         lib.cce_debug_withhold_loads.restype = None
         lib.cce_debug_set_kernel_events.argtypes = [ctypes.c_int, c_vp, c_vp]
@@ -147,3 +149,8 @@ def cce_debug_set_kernel_events(kernel: int, start_event: int, stop_event: int) 
 
 def cce_debug_withhold_loads(on: bool) -> None:
     load_library().cce_debug_withhold_loads(1 if on else 0)
+
+
+def cce_debug_set_forward_variant(variant: int) -> None:
+    """0 = single-CTA forward kernel (default), 1 = CTA-pair forward kernel."""
+    _check(load_library().cce_debug_set_forward_variant(int(variant)), "cce_debug_set_forward_variant")

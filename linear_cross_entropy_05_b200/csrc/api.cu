@@ -18,6 +18,8 @@
 namespace cce {
 cudaError_t launch_fwd_lse(const CUtensorMap& tmE, const CUtensorMap& tmC, const FwdArgs& a, int grid,
                            cudaStream_t stream);
+cudaError_t launch_fwd_lse_pair(const CUtensorMap& tmE, const CUtensorMap& tmCh, const FwdArgs& a, int grid,
+                                cudaStream_t stream);
 cudaError_t launch_fwd_finalize(const void* E, const void* C, const int64_t* y, const FinArgs& a, float* loss,
                                 float* lse, cudaStream_t stream);
 cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
@@ -31,6 +33,9 @@ using namespace cce;
 namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
+
+// Forward kernel variant: 0 = single CTAs (default), 1 = CTA pairs (cta_group::2).
+std::atomic<int> g_fwd_variant{0};
 
 // Test hook: when set, the next launches' TMA producers issue no copies.
 std::atomic<int> g_withhold_loads{0};
@@ -140,7 +145,8 @@ bool make_map_f32(CUtensorMap* map, const void* base, int64_t rows, int64_t D) {
 }
 
 struct FwdPlan {
-  int n_mblk, n_vtile, n_split, grid;
+  bool pair;       // CTA-pair kernel: token blocks of 2 x BM rows, grid in pairs
+  int n_mblk, n_vtile, n_split, grid, group_m;
   size_t ws_bytes;
 };
 
@@ -148,11 +154,16 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
   if (!sizes_ok(N, D, V)) return false;
   DeviceInfo di = device_info();
   if (!di.ok || di.sms <= 0) return false;
-  p->n_mblk = (int)((N + BM - 1) / BM);
+  p->pair = g_fwd_variant.load() == 1 && di.sms >= 2;
+  const int rows = p->pair ? 2 * BM : BM;           // token rows per work unit
+  const int workers = p->pair ? di.sms / 2 : di.sms;  // CTA pairs or CTAs
+  p->n_mblk = (int)((N + rows - 1) / rows);
   p->n_vtile = (int)((V + BN - 1) / BN);
-  p->n_split = choose_splits(p->n_mblk, p->n_vtile, di.sms);
+  p->n_split = choose_splits(p->n_mblk, p->n_vtile, workers);
   const long long units = (long long)p->n_mblk * p->n_split;
-  p->grid = (int)std::min<long long>(units, di.sms);
+  p->grid = (int)std::min<long long>(units, workers) * (p->pair ? 2 : 1);
+  // keep at most ~48 MB of E rows in flight so they stay resident in the 126 MB L2
+  p->group_m = (int)std::max<int64_t>(1, std::min<int64_t>(p->n_mblk, (48ll << 20) / ((int64_t)rows * D * 2)));
   p->ws_bytes = STATUS_BYTES + align_up((size_t)p->n_split * (size_t)N * sizeof(float2), 256);
   return true;
 }
@@ -198,7 +209,7 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
   CUtensorMap tmE, tmC;
-  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN)) return CCE_ERR_CUDA;
+  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, p.pair ? BM : BN)) return CCE_ERR_CUDA;
 
   unsigned long long* status = reinterpret_cast<unsigned long long*>(ws);
   float2* partial = reinterpret_cast<float2*>(reinterpret_cast<char*>(ws) + STATUS_BYTES);
@@ -212,15 +223,16 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   a.n_vtile = p.n_vtile;
   a.n_split = p.n_split;
   a.n_units = p.n_mblk * p.n_split;
-  // keep at most ~48 MB of E rows in flight so they stay resident in the 126 MB L2
-  a.group_m = (int)std::max<int64_t>(1, std::min<int64_t>(p.n_mblk, (48ll << 20) / ((int64_t)BM * D * 2)));
+  a.group_m = p.group_m;
   a.partial = partial;
   a.dbg_logits = dbg_logits;
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.withhold_loads = g_withhold_loads.load();
   if (record_event(0, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
-  if (launch_fwd_lse(tmE, tmC, a, p.grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  const cudaError_t le =
+      p.pair ? launch_fwd_lse_pair(tmE, tmC, a, p.grid, stream) : launch_fwd_lse(tmE, tmC, a, p.grid, stream);
+  if (le != cudaSuccess) return CCE_ERR_CUDA;
   if (record_event(0, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
 
   FinArgs f;
@@ -269,6 +281,12 @@ void cce_debug_set_wait_limit_ns(uint64_t limit_ns) {
 }
 
 void cce_debug_withhold_loads(int on) { g_withhold_loads.store(on ? 1 : 0); }
+
+cce_status_t cce_debug_set_forward_variant(int variant) {
+  if (variant < 0 || variant > 1) return CCE_ERR_INVALID_ARG;
+  g_fwd_variant.store(variant);
+  return CCE_OK;
+}
 
 cce_status_t cce_debug_set_kernel_events(int kernel, void* start_event, void* stop_event) {
   if (kernel < 0 || kernel > 1) return CCE_ERR_INVALID_ARG;

@@ -16,6 +16,8 @@ constexpr int B_STAGE_BYTES = BN * BK * 2;  // C slice  [256 rows][64 d]
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int NUM_THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int FWD_STAGES = 4;
+constexpr int PAIR_STAGES = 6;                          // CTA-pair forward: E half + C half per stage
+constexpr int PAIR_STAGE_BYTES = 2 * A_STAGE_BYTES;     // [128][64] bf16 of E and of C
 constexpr int BWD_STAGES = 3;
 constexpr int G_BYTES = BM * BN * 2;        // bf16 softmax-gradient tile (4 swizzled K blocks)
 
@@ -46,7 +48,7 @@ constexpr int STATUS_BYTES = 256;
 
 struct FwdArgs {
   int N, D, V;
-  int n_mblk;      // ceil(N / BM)
+  int n_mblk;      // token blocks: ceil(N / BM), or ceil(N / 2BM) for the CTA-pair kernel
   int n_vtile;     // ceil(V / BN)
   int n_split;     // vocabulary splits per token block
   int n_units;     // n_mblk * n_split

@@ -25,6 +25,52 @@
 
 namespace cce {
 
+// Fold one 128 x 256 logit tile held in TMEM (this thread's lane = one token
+// row) into the row's running (max, sum exp(z - max)).  Columns >= V are
+// masked to -inf; DUMP additionally stores the raw logits (debug entry only).
+template <bool DUMP>
+__device__ __forceinline__ void lse_fold_tile(uint32_t tbase, int col0, int row, const FwdArgs& a, float& mrun,
+                                              float& srun) {
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    const int cbase = col0 + c * 32;
+    if (cbase >= a.V) break;  // uniform across the warp
+    float x[32];
+    tmem_ld32(tbase + (uint32_t)(c * 32), x);
+    if constexpr (DUMP) {
+      if (row < a.N) {
+        float* dst = a.dbg_logits + (size_t)row * ((size_t)a.n_vtile * BN) + cbase;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dst[j] = x[j];
+      }
+    }
+    const int nvalid = a.V - cbase;
+    if (nvalid < 32) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j >= nvalid) x[j] = -INFINITY;
+    }
+    float cm0 = x[0], cm1 = x[1];
+#pragma unroll
+    for (int j = 2; j < 32; j += 2) {
+      cm0 = fmaxf(cm0, x[j]);
+      cm1 = fmaxf(cm1, x[j + 1]);
+    }
+    const float mnew = fmaxf(mrun, fmaxf(cm0, cm1));
+    const float ms = mnew * LOG2E;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      s0 += ex2_approx(fmaf(x[j], LOG2E, -ms));
+      s1 += ex2_approx(fmaf(x[j + 1], LOG2E, -ms));
+      s2 += ex2_approx(fmaf(x[j + 2], LOG2E, -ms));
+      s3 += ex2_approx(fmaf(x[j + 3], LOG2E, -ms));
+    }
+    srun = srun * ex2_approx(fmaf(mrun, LOG2E, -ms)) + ((s0 + s1) + (s2 + s3));
+    mrun = mnew;
+  }
+}
+
 template <bool DUMP>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_lse_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
@@ -180,47 +226,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t tbase = tmem_base + lane_addr + (uint32_t)(acc * BN);
-        const int col0 = vt * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          const int cbase = col0 + c * 32;
-          if (cbase >= a.V) break;  // uniform across the warp
-          float x[32];
-          tmem_ld32(tbase + (uint32_t)(c * 32), x);
-          if constexpr (DUMP) {
-            const int row = m * BM + row_in_blk;
-            if (row < a.N) {
-              float* dst = a.dbg_logits + (size_t)row * ((size_t)a.n_vtile * BN) + cbase;
-#pragma unroll
-              for (int j = 0; j < 32; ++j) dst[j] = x[j];
-            }
-          }
-          const int nvalid = a.V - cbase;
-          if (nvalid < 32) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j >= nvalid) x[j] = -INFINITY;
-          }
-          float cm0 = x[0], cm1 = x[1];
-#pragma unroll
-          for (int j = 2; j < 32; j += 2) {
-            cm0 = fmaxf(cm0, x[j]);
-            cm1 = fmaxf(cm1, x[j + 1]);
-          }
-          const float mnew = fmaxf(mrun, fmaxf(cm0, cm1));
-          const float ms = mnew * LOG2E;
-          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            s0 += ex2_approx(fmaf(x[j], LOG2E, -ms));
-            s1 += ex2_approx(fmaf(x[j + 1], LOG2E, -ms));
-            s2 += ex2_approx(fmaf(x[j + 2], LOG2E, -ms));
-            s3 += ex2_approx(fmaf(x[j + 3], LOG2E, -ms));
-          }
-          srun = srun * ex2_approx(fmaf(mrun, LOG2E, -ms)) + ((s0 + s1) + (s2 + s3));
-          mrun = mnew;
-        }
+        lse_fold_tile<DUMP>(tmem_base + lane_addr + (uint32_t)(acc * BN), vt * BN, m * BM + row_in_blk, a, mrun,
+                            srun);
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
         if (++acc == 2) {
@@ -246,6 +253,203 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0 && blockIdx.x == 0 && !*abort_flag) {
     atomicAdd(a.status + ST_TILES, (unsigned long long)a.n_mblk * (unsigned long long)a.n_vtile);
   }
+}
+
+
+// ----------------------------------------------------------------------------
+// CTA-pair variant: a cluster of two CTAs on two SMs computes 256 x 256 logit
+// tiles with tcgen05.mma.cta_group::2 (M = 256 split over the pair).  Each CTA
+// loads its own 128 token rows of E and 128 vocabulary rows of C per stage
+// (32 KB instead of 48 KB per SM for the same MMA work, so 6 stages fit), and
+// each CTA's TMEM holds its 128 rows x 256 columns of every tile, which its own
+// epilogue folds exactly as in the single-CTA kernel.  Only the even (leader)
+// CTA issues UMMAs; its full barriers count both CTAs' copies, its commits
+// arrive on both CTAs' barriers, and both epilogues release the accumulator
+// on the leader's barrier.  No TMA multicast is used.
+// ----------------------------------------------------------------------------
+template <bool DUMP>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    fwd_lse_pair_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmCh,
+                        const FwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                                    // PAIR_STAGES x [128 tok][64 d]
+  uint8_t* sB = smem + PAIR_STAGES * A_STAGE_BYTES;      // PAIR_STAGES x [128 voc][64 d]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + PAIR_STAGES * A_STAGE_BYTES);
+  uint64_t* full = bars;                      // leader: both CTAs' copies landed
+  uint64_t* empty = bars + PAIR_STAGES;       // each CTA: stage free again
+  uint64_t* tfull = bars + 2 * PAIR_STAGES;   // each CTA: accumulator ready
+  uint64_t* tempty = tfull + 2;               // leader: both epilogues done with the accumulator
+  uint64_t* drain = tempty + 2;               // leader: UMMA drain at exit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_map(&tmE);
+    tma_prefetch_map(&tmCh);
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, a.wait_limit_ns};
+  const int nkb = (a.D + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int stage = 0;
+      uint32_t phase = 0, armed = 0;
+      for (int u = a.withhold_loads ? a.n_units : pair; u < a.n_units; u += n_pairs) {
+        int r, m2;
+        unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m2);
+        int v0, v1;
+        split_range(r, a.n_vtile, a.n_split, v0, v1);
+        for (int vt = v0; vt < v1; ++vt) {
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
+            tma_load_2d_pair(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m2 * (2 * BM) + rank * BM);
+            tma_load_2d_pair(sB + stage * A_STAGE_BYTES, &tmCh, &full[stage], kb * BK, vt * BN + rank * BM);
+            armed |= 1u << stage;
+            if (++stage == PAIR_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    producer_done:
+      // The leader's full barriers count both CTAs' copies: once they have
+      // completed, nothing is in flight (the cluster sync below holds the
+      // peer until then).
+      if (leader) {
+        int dummy = 0;
+        WaitCtl exit_wc{&dummy, a.wait_limit_ns};
+        for (int s = 0; s < PAIR_STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (s < stage) ? phase : (phase ^ 1u), exit_wc);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- UMMA issuer (leader only) ----------------
+      constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, false, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int u = pair; u < a.n_units; u += n_pairs) {
+        int r, m2;
+        unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m2);
+        int v0, v1;
+        split_range(r, a.n_vtile, a.n_split, v0, v1);
+        for (int vt = v0; vt < v1; ++vt) {
+          if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, wc)) goto mma_done;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
+            const uint32_t b_addr = smem_u32(sB + stage * A_STAGE_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16_pair(d_tmem, sdesc_sw128(a_addr + k * 32, 16, 1024), sdesc_sw128(b_addr + k * 32, 16, 1024),
+                             IDESC, (kb | k) != 0);
+            umma_commit_pair_mc(&empty[stage], 0x3);
+            if (++stage == PAIR_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          umma_commit_pair_mc(&tfull[acc], 0x3);
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
+      }
+    mma_done:
+      umma_commit_pair_mc(drain, 0x1);
+      {
+        int dummy = 0;
+        WaitCtl exit_wc{&dummy, a.wait_limit_ns};
+        mbar_wait(drain, 0, exit_wc);
+      }
+    }
+  } else {
+    // ---------------- epilogue: 4 warps per CTA, one TMEM lane (token row) each ----------------
+    const int lane_grp = warp & 3;
+    const int row_in_blk = lane_grp * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(lane_grp * 32) << 16;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = pair; u < a.n_units; u += n_pairs) {
+      int r, m2;
+      unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m2);
+      int v0, v1;
+      split_range(r, a.n_vtile, a.n_split, v0, v1);
+      const int row = m2 * (2 * BM) + (int)rank * BM + row_in_blk;
+      float mrun = -INFINITY, srun = 0.f;
+      bool ok = true;
+      for (int vt = v0; vt < v1; ++vt) {
+        if (!mbar_wait(&tfull[acc], acc_phase, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        lse_fold_tile<DUMP>(tmem_base + lane_addr + (uint32_t)(acc * BN), vt * BN, row, a, mrun, srun);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (row < a.N) a.partial[(size_t)r * a.N + row] = make_float2(mrun, srun);
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no remote arrival or copy can target an exited CTA
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status + ST_FLAGS, SF_TIMEOUT);
+  if (threadIdx.x == 0 && blockIdx.x == 0 && !*abort_flag)
+    atomicAdd(a.status + ST_TILES, (unsigned long long)(a.N + BM - 1) / BM * (unsigned long long)a.n_vtile);
 }
 
 // One warp per token row.
@@ -308,6 +512,25 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const __nv_bfloat16* 
 }
 
 size_t fwd_smem_bytes() { return 1024 + (size_t)FWD_STAGES * STAGE_BYTES + 256; }
+size_t fwd_pair_smem_bytes() { return 1024 + (size_t)PAIR_STAGES * PAIR_STAGE_BYTES + 256; }
+
+// grid: an even number of CTAs (pairs)
+cudaError_t launch_fwd_lse_pair(const CUtensorMap& tmE, const CUtensorMap& tmCh, const FwdArgs& a, int grid,
+                                cudaStream_t stream) {
+  const size_t smem = fwd_pair_smem_bytes();
+  if (a.dbg_logits) {
+    cudaError_t e =
+        cudaFuncSetAttribute(fwd_lse_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    fwd_lse_pair_kernel<true><<<grid, NUM_THREADS, smem, stream>>>(tmE, tmCh, a);
+  } else {
+    cudaError_t e =
+        cudaFuncSetAttribute(fwd_lse_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    fwd_lse_pair_kernel<false><<<grid, NUM_THREADS, smem, stream>>>(tmE, tmCh, a);
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_fwd_lse(const CUtensorMap& tmE, const CUtensorMap& tmC, const FwdArgs& a, int grid,
                            cudaStream_t stream) {

@@ -31,16 +31,20 @@ def test_withheld_loads_end_with_timeout_status_and_a_usable_context():
     L.cce_debug_set_wait_limit_ns(20_000_000)       # 20 ms per wait
     L.cce_debug_withhold_loads(True)
     try:
-        ws = L.Workspace()
-        L.forward(E, C, y, IGN, workspace=ws)
-        st = L.read_status(ws)
-        assert st["status"] == CCE_ERR_TIMEOUT and st["flags"] & 1
+        for variant in (0, 1):   # single-CTA and CTA-pair forward kernels
+            L.cce_debug_set_forward_variant(variant)
+            ws = L.Workspace()
+            L.forward(E, C, y, IGN, workspace=ws)
+            st = L.read_status(ws)
+            assert st["status"] == CCE_ERR_TIMEOUT and st["flags"] & 1
+        L.cce_debug_set_forward_variant(0)
         for eps in (0.0, 2.0 ** -12):
             ws = L.Workspace()
             L.backward(E, C, y, torch.from_numpy(lse).cuda(), dl, eps, IGN, workspace=ws)
             st = L.read_status(ws)
             assert st["status"] == CCE_ERR_TIMEOUT and st["flags"] & 1
     finally:
+        L.cce_debug_set_forward_variant(0)
         L.cce_debug_withhold_loads(False)
         L.cce_debug_set_wait_limit_ns(1_000_000_000)
     torch.cuda.synchronize()

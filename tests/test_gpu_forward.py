@@ -40,7 +40,8 @@ def test_forward_matches_oracle(w):
     assert (loss[inp["y"] == IGN] == 0).all()
 
 
-def test_raw_logit_tiles_match_definition():
+@pytest.mark.parametrize("variant", [0, 1], ids=["single-cta", "cta-pair"])
+def test_raw_logit_tiles_match_definition(variant):
     import torch
     import linear_cross_entropy_05_b200 as L
     w = synth.TINY.with_sizes(N=300, V=4096 + 77, D=264)
@@ -52,10 +53,14 @@ def test_raw_logit_tiles_match_definition():
     loss = torch.empty(N, device="cuda")
     lse = torch.empty(N, device="cuda")
     ws = L.Workspace()
-    buf = ws.get(L.cce_forward_workspace_size(N, D, V))
-    L.cce_debug_forward_logits(E.data_ptr(), C.data_ptr(), y.data_ptr(), N, D, V, IGN, loss.data_ptr(),
-                               lse.data_ptr(), logits.data_ptr(), buf.data_ptr(), buf.numel(),
-                               torch.cuda.current_stream().cuda_stream)
+    L.cce_debug_set_forward_variant(variant)
+    try:
+        buf = ws.get(L.cce_forward_workspace_size(N, D, V))
+        L.cce_debug_forward_logits(E.data_ptr(), C.data_ptr(), y.data_ptr(), N, D, V, IGN, loss.data_ptr(),
+                                   lse.data_ptr(), logits.data_ptr(), buf.data_ptr(), buf.numel(),
+                                   torch.cuda.current_stream().cuda_stream)
+    finally:
+        L.cce_debug_set_forward_variant(0)
     g = logits.cpu().numpy()
     z = oracle.logits(oracle.bf16_bits_to_f64(inp["E"]), oracle.bf16_bits_to_f64(inp["C"]))
     # bf16 x bf16 products are exact in fp32; only the fp32 accumulation rounds
@@ -168,3 +173,25 @@ def test_library_allocates_no_device_memory():
     assert ws.buf.numel() == max(fwd, bwd)
     assert fwd <= 512 + 64 * 8 * w.N
     assert bwd <= 4096 + 8 * w.N + 3 * 4 * (w.V // 256 + 64) + 2 * 4 * (w.N // 128 + 64)
+
+
+@pytest.mark.parametrize("w", [synth.TINY.with_sizes(N=300, V=4096 + 77, D=264),
+                               synth.TINY.with_sizes(N=129, V=257, D=8),
+                               synth.GEMMA2_2B.with_sizes(N=1000, V=20000)],
+                         ids=["ragged", "minimal", "gemma-shaped"])
+def test_cta_pair_forward_variant_matches_oracle(w):
+    # the CTA-pair forward kernel (tcgen05 cta_group::2) is selectable for A/B
+    # measurement and must give the same losses as the default kernel
+    import linear_cross_entropy_05_b200 as L
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    L.cce_debug_set_forward_variant(1)
+    try:
+        loss1, lse1, st = gpu_forward(E, C, y)
+    finally:
+        L.cce_debug_set_forward_variant(0)
+    assert st["status"] == 0
+    loss0, lse0, st = gpu_forward(E, C, y)
+    ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    assert np.abs(loss1 - ol).max() <= LOSS_ABS and np.abs(lse1 - olse).max() <= LOSS_ABS
+    assert np.abs(loss0 - loss1).max() <= 1e-4
