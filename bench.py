@@ -203,14 +203,22 @@ def oracle_step(inp, rows, eps):
     return loss
 
 
-def cpu_baseline(inp, w, rows_n: int):
+def cpu_baseline(inp, w, rows_n: int, gpu_loss=None):
+    """Time the oracle on the first rows_n tokens; if the GPU's per-token
+    losses are given, also report their largest deviation from the oracle's
+    on those tokens (the same oracle run, no extra work)."""
     rows = np.arange(rows_n)
     t0 = time.perf_counter()
-    oracle_step(inp, rows, w.filter_eps)
+    oloss = oracle_step(inp, rows, w.filter_eps)
     dt = time.perf_counter() - t0
-    return {"value": rows_n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"fp64 oracle forward+backward (tile filter {w.filter_eps:g}) on the first {rows_n} tokens "
-                      f"of the {w.name} workload (full V={w.V}, D={w.D}); {dt:.2f} s"}
+    out = {"value": rows_n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+           "sample": f"fp64 oracle forward+backward (tile filter {w.filter_eps:g}) on the first {rows_n} tokens "
+                     f"of the {w.name} workload (full V={w.V}, D={w.D}); {dt:.2f} s"}
+    if gpu_loss is not None:
+        keep = inp["y"][rows] != IGN
+        err = np.abs(np.asarray(gpu_loss[:rows_n], dtype=np.float64) - oloss)[keep]
+        out["parity_loss_max_abs_err"] = float(err.max()) if err.size else 0.0
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -280,9 +288,14 @@ def run_gpu(args, w):
     eps = w.filter_eps
     stream = torch.cuda.current_stream()
 
+    gkw = dict(deterministic=args.deterministic, bf16_grads=args.bf16_grads)
+    if args.bf16_grads:
+        dE = torch.empty((N, D), device=dev, dtype=torch.bfloat16)
+        dC = torch.empty((V, D), device=dev, dtype=torch.bfloat16)
+
     def step():
         L.forward(E, C, y, IGN, workspace=ws_f, out=(loss, lse))
-        L.backward(E, C, y, lse, dloss, eps, IGN, workspace=ws_b, out=(dE, dC))
+        L.backward(E, C, y, lse, dloss, eps, IGN, workspace=ws_b, out=(dE, dC), **gkw)
 
     # warm-up (also loads the module) and status check
     for _ in range(max(3, args.warmup)):
@@ -372,7 +385,7 @@ def run_gpu(args, w):
                     copied[b].record(copy_stream)
                 stream.wait_event(copied[b])
                 L.forward(Eb, Cb, yb, IGN, workspace=ws_f, out=(loss, lse))
-                L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC))
+                L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC), **gkw)
                 loss_h[b].copy_(loss, non_blocking=True)
                 consumed[b].record(stream)
 
@@ -407,12 +420,16 @@ def run_gpu(args, w):
 
     out = None
     if rank == 0:
-        cpu = cpu_baseline(inp, w, args.cpu_rows) if world == 1 and not args.no_cpu_baseline else None
+        cpu = (cpu_baseline(inp, w, args.cpu_rows, gpu_loss=loss.cpu().numpy())
+               if world == 1 and not args.no_cpu_baseline else None)
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded numpy PCG64; random-init classifier, Zipf labels)",
-            "config": dict(config_of(w, world), forward_kernel=args.fwd_variant),
+            "config": dict(config_of(w, world), forward_kernel=args.fwd_variant,
+                           backward_accumulation=("fixed-point int64" if (args.deterministic or args.bf16_grads)
+                                                  else "fp32 atomic (TMA reduce-add)"),
+                           grad_dtype="bf16" if args.bf16_grads else "fp32"),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
@@ -509,6 +526,9 @@ def main(argv=None):
                     help="workload name (the default is the headline Gemma-2-2B-shaped head)")
     ap.add_argument("--N", type=int, default=None, help="override tokens (profiling cases)")
     ap.add_argument("--V", type=int, default=None, help="override vocabulary (profiling cases)")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="bitwise reproducible backward (fixed-point accumulation)")
+    ap.add_argument("--bf16-grads", action="store_true", help="bf16 dE/dC outputs (fixed-point accumulation)")
     ap.add_argument("--fwd-variant", choices=["single", "pair"], default="single",
                     help="forward kernel: single CTAs (default) or CTA pairs (A/B measurement)")
     ap.add_argument("--suite", action="store_true",

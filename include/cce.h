@@ -139,6 +139,35 @@ CCE_API cce_status_t cce_backward(const void* E, const void* C, const int64_t* y
 CCE_API cce_status_t cce_forward_noalloc(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D,
                                          int64_t V, int64_t ignore_index, float* loss, float* lse, void* stream);
 
+/* Options of cce_backward_ex (bit flags). */
+typedef enum {
+  CCE_BWD_DEFAULT = 0,
+  /* Bitwise reproducible dE/dC: every per-tile partial product (fp32, from
+   * the tensor cores) is rounded once to a 64-bit fixed-point value whose
+   * power-of-two scale puts a bound on the largest possible gradient entry
+   * (from max|dloss|, max_v|C_v|, max_i|E_i| and N) just under 2^61, and
+   * accumulated with integer adds, whose result does not depend on the order
+   * in which the tiles finish; a final pass converts to the output type.
+   * Needs an extra (N + V) * D * 8 bytes of workspace. */
+  CCE_BWD_DETERMINISTIC = 1,
+  /* dE and dC are written as bf16 (round to nearest even) instead of fp32;
+   * implies CCE_BWD_DETERMINISTIC (the accumulation is the same). */
+  CCE_BWD_BF16_GRADS = 2
+} cce_backward_flags_t;
+
+/* Workspace bytes for cce_backward_ex with these flags (0 if the sizes or
+ * flags are invalid). */
+CCE_API size_t cce_backward_workspace_size_ex(int64_t N, int64_t D, int64_t V, unsigned flags);
+
+/* cce_backward with options (see cce_backward_flags_t).  dE and dC are fp32
+ * unless CCE_BWD_BF16_GRADS is set, then bf16 (raw 16-bit storage).  With
+ * flags == 0 this is exactly cce_backward.  Same filter semantics, parity and
+ * error behaviour as cce_backward. */
+CCE_API cce_status_t cce_backward_ex(const void* E, const void* C, const int64_t* y, const float* lse,
+                                     const float* dloss, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
+                                     float filter_eps, unsigned flags, void* dE, void* dC, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then copies the status block of `workspace` (as left
  * by the last call that used it) into *out.  Returns CCE_ERR_TIMEOUT or
  * CCE_ERR_BAD_LABEL if the corresponding flag is set, else CCE_OK. */

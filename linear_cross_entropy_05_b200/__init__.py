@@ -22,7 +22,8 @@ import os
 from typing import Optional, Tuple
 
 from . import _native
-from ._native import (CCEError, cce_backward, cce_backward_workspace_size, cce_debug_forward_logits,
+from ._native import (CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCEError, cce_backward, cce_backward_ex,
+                      cce_backward_workspace_size, cce_backward_workspace_size_ex, cce_debug_forward_logits,
                       cce_debug_set_forward_variant, cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns,
                       cce_debug_withhold_loads, cce_forward, cce_forward_noalloc,
                       cce_forward_workspace_size, cce_read_status,
@@ -31,7 +32,8 @@ from ._native import (CCEError, cce_backward, cce_backward_workspace_size, cce_d
 IGNORE_INDEX = -100
 
 __all__ = [
-    "CCEError", "IGNORE_INDEX", "cce_forward", "cce_forward_noalloc", "cce_backward", "cce_forward_workspace_size",
+    "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "cce_forward",
+    "cce_forward_noalloc", "cce_backward", "cce_backward_ex", "cce_backward_workspace_size_ex", "cce_forward_workspace_size",
     "cce_backward_workspace_size", "cce_read_status", "cce_status_string", "cce_version",
     "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "cce_debug_set_kernel_events", "cce_debug_withhold_loads", "cce_debug_set_forward_variant",
     "load_library",
@@ -101,8 +103,11 @@ def forward(E, C, y, ignore_index: int = IGNORE_INDEX, workspace: Optional[Works
 
 
 def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = IGNORE_INDEX,
-             workspace: Optional[Workspace] = None, stream=None, out=None):
-    """dE [N, D] and dC [V, D] (fp32) of sum_i dloss[i] * loss[i]."""
+             workspace: Optional[Workspace] = None, stream=None, out=None, deterministic: bool = False,
+             bf16_grads: bool = False):
+    """dE [N, D] and dC [V, D] of sum_i dloss[i] * loss[i]: fp32, or bf16 with
+    bf16_grads; deterministic=True gives bitwise reproducible gradients
+    (fixed-point accumulation, extra (N + V) * D * 8 bytes of workspace)."""
     torch = _torch()
     _check_inputs(E, C, y)
     N, D = E.shape
@@ -110,16 +115,20 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     for t, n in ((lse, "lse"), (dloss, "dloss")):
         if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.shape != (N,):
             raise ValueError(f"{n} must be a contiguous CUDA float32 tensor of shape [N]")
+    flags = (CCE_BWD_DETERMINISTIC if deterministic else 0) | (CCE_BWD_BF16_GRADS if bf16_grads else 0)
+    gdt = torch.bfloat16 if bf16_grads else torch.float32
     if out is None:
-        dE = torch.empty((N, D), dtype=torch.float32, device=E.device)
-        dC = torch.empty((V, D), dtype=torch.float32, device=E.device)
+        dE = torch.empty((N, D), dtype=gdt, device=E.device)
+        dC = torch.empty((V, D), dtype=gdt, device=E.device)
     else:
         dE, dC = out
-    ws_bytes = cce_backward_workspace_size(N, D, V)
+        if dE.dtype != gdt or dC.dtype != gdt:
+            raise TypeError(f"dE and dC must be {gdt}")
+    ws_bytes = cce_backward_workspace_size_ex(N, D, V, flags)
     ws = (workspace or Workspace(E.device)).get(ws_bytes)
-    cce_backward(E.data_ptr(), C.data_ptr(), y.data_ptr(), lse.data_ptr(), dloss.data_ptr(), N, D, V,
-                 ignore_index, float(filter_eps), dE.data_ptr(), dC.data_ptr(), ws.data_ptr(), ws.numel(),
-                 _stream_ptr(stream))
+    cce_backward_ex(E.data_ptr(), C.data_ptr(), y.data_ptr(), lse.data_ptr(), dloss.data_ptr(), N, D, V,
+                    ignore_index, float(filter_eps), flags, dE.data_ptr(), dC.data_ptr(), ws.data_ptr(), ws.numel(),
+                    _stream_ptr(stream))
     return dE, dC
 
 

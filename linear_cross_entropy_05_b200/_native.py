@@ -49,6 +49,11 @@ def load_library():
         lib.cce_backward.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_vp, c_vp,
                                      c_vp, c_size, c_vp]
         lib.cce_backward.restype = ctypes.c_int
+        lib.cce_backward_workspace_size_ex.argtypes = [c_i64, c_i64, c_i64, ctypes.c_uint]
+        lib.cce_backward_workspace_size_ex.restype = c_size
+        lib.cce_backward_ex.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, ctypes.c_uint,
+                                        c_vp, c_vp, c_vp, c_size, c_vp]
+        lib.cce_backward_ex.restype = ctypes.c_int
         lib.cce_read_status.argtypes = [c_vp, c_vp, ctypes.POINTER(CCECounters)]
         lib.cce_read_status.restype = ctypes.c_int
         lib.cce_status_string.argtypes = [ctypes.c_int]
@@ -119,6 +124,24 @@ def cce_backward(E: int, C: int, y: int, lse: int, dloss: int, N: int, D: int, V
                                      workspace_bytes, stream)
     if check:
         _check(st, "cce_backward")
+    return st
+
+
+CCE_BWD_DETERMINISTIC = 1
+CCE_BWD_BF16_GRADS = 2
+
+
+def cce_backward_workspace_size_ex(N: int, D: int, V: int, flags: int) -> int:
+    return int(load_library().cce_backward_workspace_size_ex(N, D, V, flags))
+
+
+def cce_backward_ex(E: int, C: int, y: int, lse: int, dloss: int, N: int, D: int, V: int, ignore_index: int,
+                    filter_eps: float, flags: int, dE: int, dC: int, workspace: int, workspace_bytes: int,
+                    stream: int, check: bool = True) -> int:
+    st = load_library().cce_backward_ex(E, C, y, lse, dloss, N, D, V, ignore_index, filter_eps, flags, dE, dC,
+                                        workspace, workspace_bytes, stream)
+    if check:
+        _check(st, "cce_backward_ex")
     return st
 
 

@@ -26,6 +26,10 @@ cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUt
                        const CUtensorMap& tmdC, const BwdArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
                         int sms, cudaStream_t stream);
+cudaError_t launch_cnorm(const void* C, const PrepArgs& p, int sms, cudaStream_t stream);
+cudaError_t launch_fixed_prep(const void* E, const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream);
+cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
+                                bool bf16, int sms, cudaStream_t stream);
 }  // namespace cce
 
 using namespace cce;
@@ -173,9 +177,13 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
 struct BwdPlan {
   int n_mblk, n_vtile;
   size_t off_hdr, off_count, off_offset, off_cursor, off_flat, off_nonflat, off_list, zero_bytes, ws_bytes;
+  size_t off_accE, off_accC;  // fixed-point accumulators (deterministic mode only)
 };
 
-bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p) {
+constexpr unsigned kBwdFlagsAll = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS;
+
+bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags = 0) {
+  if (flags & ~kBwdFlagsAll) return false;
   if (!sizes_ok(N, D, V)) return false;
   p->n_mblk = (int)((N + BM - 1) / BM);
   p->n_vtile = (int)((V + BN - 1) / BN);
@@ -191,6 +199,12 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p) {
   p->off_nonflat = p->off_flat + mb4;
   p->off_list = p->off_nonflat + mb4;
   p->ws_bytes = p->off_list + align_up((size_t)N * sizeof(int2), 256);
+  p->off_accE = p->off_accC = 0;
+  if (flags) {
+    p->off_accE = p->ws_bytes;
+    p->off_accC = p->off_accE + align_up((size_t)N * D * 8, 256);
+    p->ws_bytes = p->off_accC + align_up((size_t)V * D * 8, 256);
+  }
   return true;
 }
 
@@ -295,32 +309,49 @@ cce_status_t cce_debug_set_kernel_events(int kernel, void* start_event, void* st
   return CCE_OK;
 }
 
-cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
-                          int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, float* dE,
-                          float* dC, void* workspace, size_t workspace_bytes, void* stream_) {
+}  // extern "C"
+
+namespace {
+
+cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
+                           int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, unsigned flags,
+                           void* dE, void* dC, void* workspace, size_t workspace_bytes, void* stream_) {
   if (!E || !C || !y || !lse || !dloss || !dE || !dC || !workspace) return CCE_ERR_INVALID_ARG;
+  if (flags & ~kBwdFlagsAll) return CCE_ERR_INVALID_ARG;
+  const bool fixed = flags != 0;
+  const bool bf16_out = (flags & CCE_BWD_BF16_GRADS) != 0;
   if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
   if (!(filter_eps == filter_eps)) return CCE_ERR_INVALID_ARG;  // NaN
   if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(lse, 4) || !aligned(dloss, 4) ||
       !aligned(dE, 16) || !aligned(dC, 16) || !aligned(workspace, 256))
     return CCE_ERR_MISALIGNED;
   BwdPlan bp;
-  if (!plan_backward(N, D, V, &bp)) return CCE_ERR_INVALID_ARG;
+  if (!plan_backward(N, D, V, &bp, flags)) return CCE_ERR_INVALID_ARG;
   DeviceInfo di = device_info();
   if (!di.ok) return CCE_ERR_UNSUPPORTED_DEVICE;
   if (workspace_bytes < bp.ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
   CUtensorMap tmE, tmC, tmdE, tmdC;
+  // (in fixed-point mode the fp32 maps are built but the kernel reduces into
+  // the int64 accumulators instead; dE/dC may then hold bf16)
   if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN) || !make_map_f32(&tmdE, dE, N, D) ||
       !make_map_f32(&tmdC, dC, V, D))
     return CCE_ERR_CUDA;
   char* ws = reinterpret_cast<char*>(workspace);
   unsigned long long* status = reinterpret_cast<unsigned long long*>(ws);
+  unsigned long long* accE = fixed ? reinterpret_cast<unsigned long long*>(ws + bp.off_accE) : nullptr;
+  unsigned long long* accC = fixed ? reinterpret_cast<unsigned long long*>(ws + bp.off_accC) : nullptr;
   const bool filter_on = filter_eps > 0.f;
-  if (cudaMemsetAsync(ws, 0, filter_on ? bp.zero_bytes : STATUS_BYTES, stream) != cudaSuccess) return CCE_ERR_CUDA;
-  if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
-  if (cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, (filter_on || fixed) ? bp.zero_bytes : STATUS_BYTES, stream) != cudaSuccess)
+    return CCE_ERR_CUDA;
+  if (fixed) {
+    if (cudaMemsetAsync(accE, 0, (size_t)N * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  } else {
+    if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
+  }
 
   BwdArgs a;
   a.N = (int)N;
@@ -339,13 +370,15 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
   a.y = y;
   a.lse = lse;
   a.dloss = dloss;
-  a.dE = dE;
-  a.dC = dC;
+  a.dE = reinterpret_cast<float*>(dE);
+  a.dC = reinterpret_cast<float*>(dC);
+  a.accE = accE;
+  a.accC = accC;
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.withhold_loads = g_withhold_loads.load();
 
-  if (filter_on) {
+  if (filter_on || fixed) {
     PrepArgs pp;
     pp.N = (int)N;
     pp.D = (int)D;
@@ -362,13 +395,48 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
     pp.nonflat = reinterpret_cast<int*>(ws + bp.off_nonflat);
     pp.list = reinterpret_cast<int2*>(ws + bp.off_list);
     pp.status = status;
-    if (launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (filter_on) {
+      if (launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    } else {
+      if (launch_cnorm(C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    }
+    if (fixed && launch_fixed_prep(E, dloss, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
   }
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (launch_bwd(tmE, tmC, tmdE, tmdC, a, grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (fixed) {
+    const unsigned* hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);
+    if (launch_fixed_to_out(accE, dE, (size_t)N * D, hdr, (int)N, bf16_out, di.sms, stream) != cudaSuccess ||
+        launch_fixed_to_out(accC, dC, (size_t)V * D, hdr, (int)N, bf16_out, di.sms, stream) != cudaSuccess)
+      return CCE_ERR_CUDA;
+  }
   return CCE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t cce_backward_workspace_size_ex(int64_t N, int64_t D, int64_t V, unsigned flags) {
+  BwdPlan p;
+  if (!plan_backward(N, D, V, &p, flags)) return 0;
+  return p.ws_bytes;
+}
+
+cce_status_t cce_backward_ex(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
+                             int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, unsigned flags,
+                             void* dE, void* dC, void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_impl(E, C, y, lse, dloss, N, D, V, ignore_index, filter_eps, flags, dE, dC, workspace,
+                       workspace_bytes, stream);
+}
+
+cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
+                          int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, float* dE,
+                          float* dC, void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_impl(E, C, y, lse, dloss, N, D, V, ignore_index, filter_eps, 0u, dE, dC, workspace,
+                       workspace_bytes, stream);
 }
 
 cce_status_t cce_read_status(const void* workspace, void* stream, cce_counters_t* out) {

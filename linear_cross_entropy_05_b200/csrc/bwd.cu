@@ -99,6 +99,32 @@ struct TileMap {
   }
 };
 
+// Deterministic-mode counterpart of tma_red_block32: the 32 x 32 block is
+// staged the same way, read back one row at a time (lane = column), each value
+// rounded to fixed point round(x * scale) and added to the int64 accumulator
+// with a 64-bit integer atomic (a warp covers 256 contiguous bytes per row).
+// Integer addition is associative, so the totals do not depend on the order
+// in which CTAs deliver their tiles.
+__device__ __forceinline__ void fixed_red_block32(uint8_t* xb, int lane, const float (&v)[32],
+                                                  unsigned long long* base, size_t ld, uint32_t row_ok, int ncols,
+                                                  float scale) {
+  if (lane == 0) bulk_wait_group_read0();  // a bulk copy may still be reading the buffer
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(xb + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+  const bool col_ok = lane < ncols;
+#pragma unroll 4
+  for (int r = 0; r < 32; ++r) {
+    const float x = *reinterpret_cast<const float*>(xb + r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + (lane & 3) * 4);
+    if (((row_ok >> r) & 1u) && col_ok)
+      atomicAdd(base + (size_t)r * ld + lane, (unsigned long long)__float2ll_rn(x * scale));
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -309,6 +335,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     unsigned long long n_live = 0, n_dead = 0;
     uint8_t* g_row = sG + rib * 128;
     uint8_t* xb = sX + (warp - 2) * 4096;
+    const bool fixed = a.accE != nullptr;
+    float fx_scale = 0.f;
+    if (fixed)
+      fx_scale = ldexpf(1.f, fixed_point_exponent(__uint_as_float(a.hdr[HDR_CMAX]), __uint_as_float(a.hdr[HDR_EMAX]),
+                                                  __uint_as_float(a.hdr[HDR_DLMAX]), a.N));
     const int sw = rib & 7;
     int kt = 0;
     TileMap tm;
@@ -381,6 +412,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!hmask) continue;
       bool ok = true;
       const int row0 = m * BM + lane_grp * 32;           // first dE row of this warp
+      const uint32_t rows_valid = __ballot_sync(0xffffffffu, valid);  // kept tokens among those rows
       for (int kb = 0; kb < nkb; ++kb) {
         const int b = kb & 1;
         if (!mbar_wait(&c_full[b], (b ? cfe1 : cfe0) & 1u, wc)) {
@@ -395,7 +427,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int q = 0; q < 2; ++q) {
           float v[32];
           tmem_ld32(tmem_base + lane_addr + tm_de(b) + q * 32, v);
-          if (d0 + q * 32 < a.D && row0 < a.N) tma_red_block32(xb, lane, v, &tmdE, d0 + q * 32, row0);
+          if (d0 + q * 32 < a.D && row0 < a.N) {
+            if (fixed)
+              fixed_red_block32(xb, lane, v, a.accE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D, rows_valid,
+                                min(32, a.D - (d0 + q * 32)), fx_scale);
+            else
+              tma_red_block32(xb, lane, v, &tmdE, d0 + q * 32, row0);
+          }
         }
         // dC rows of this warp: vocabulary rows vt*256 + h*128 + lane_grp*32 ..
 #pragma unroll 1
@@ -406,7 +444,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int q = 0; q < 2; ++q) {
             float v[32];
             tmem_ld32(tmem_base + lane_addr + tm_dc(b) + h * 64 + q * 32, v);
-            if (d0 + q * 32 < a.D && vr0 < a.V) tma_red_block32(xb, lane, v, &tmdC, d0 + q * 32, vr0);
+            if (d0 + q * 32 < a.D && vr0 < a.V) {
+              if (fixed)
+                fixed_red_block32(xb, lane, v, a.accC + (size_t)vr0 * a.D + d0 + q * 32, (size_t)a.D,
+                                  __ballot_sync(0xffffffffu, vr0 + lane < a.V), min(32, a.D - (d0 + q * 32)),
+                                  fx_scale);
+              else
+                tma_red_block32(xb, lane, v, &tmdC, d0 + q * 32, vr0);
+            }
           }
         }
         tc_fence_before();

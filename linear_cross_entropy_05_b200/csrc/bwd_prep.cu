@@ -177,6 +177,59 @@ __global__ void __launch_bounds__(128) prep_scatter_kernel(const int64_t* __rest
   }
 }
 
+// Deterministic mode: max_i |E_i| and max_i |dloss_i| for the fixed-point
+// scale (maxima do not depend on the order of the atomics).
+__global__ void __launch_bounds__(256) prep_fixed_kernel(const __nv_bfloat16* __restrict__ E,
+                                                         const float* __restrict__ dloss, PrepArgs p) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  float emax = 0.f;
+  for (int i = gw; i < p.N; i += nw) emax = fmaxf(emax, warp_row_norm(E + (size_t)i * p.D, p.D, lane));
+  if (lane == 0) atomicMax(p.hdr + HDR_EMAX, __float_as_uint(emax));
+  float dmax = 0.f;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.N; i += gridDim.x * blockDim.x)
+    dmax = fmaxf(dmax, fabsf(dloss[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+  if (lane == 0) atomicMax(p.hdr + HDR_DLMAX, __float_as_uint(dmax));
+}
+
+// Deterministic mode: int64 fixed-point accumulators -> fp32 or bf16 output.
+__global__ void __launch_bounds__(256) fixed_to_out_kernel(const unsigned long long* __restrict__ acc, void* out,
+                                                           size_t n, const unsigned* __restrict__ hdr, int N,
+                                                           int bf16) {
+  const int s = fixed_point_exponent(__uint_as_float(hdr[HDR_CMAX]), __uint_as_float(hdr[HDR_EMAX]),
+                                     __uint_as_float(hdr[HDR_DLMAX]), N);
+  const double inv = ldexp(1.0, -s);
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; 2 * i < n; i += stride) {
+    const ulonglong2 q = reinterpret_cast<const ulonglong2*>(acc)[i];   // n is even (D % 8 == 0)
+    const double x0 = (double)(long long)q.x * inv, x1 = (double)(long long)q.y * inv;
+    if (bf16) {
+      reinterpret_cast<__nv_bfloat162*>(out)[i] = __halves2bfloat162(__double2bfloat16(x0), __double2bfloat16(x1));
+    } else {
+      reinterpret_cast<float2*>(out)[i] = make_float2((float)x0, (float)x1);
+    }
+  }
+}
+
+cudaError_t launch_fixed_prep(const void* E, const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream) {
+  prep_fixed_kernel<<<sms * 4, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E), dloss, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
+                                bool bf16, int sms, cudaStream_t stream) {
+  fixed_to_out_kernel<<<sms * 8, 256, 0, stream>>>(acc, out, n, hdr, N, bf16 ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cnorm(const void* C, const PrepArgs& p, int sms, cudaStream_t stream) {
+  prep_cnorm_kernel<<<sms * 8, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(C), p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
                         int sms, cudaStream_t stream) {
   const int cgrid = sms * 8;

@@ -38,6 +38,8 @@ enum PrepHeader : int {
   HDR_NNF = 1,   // token blocks that are not flat (visited densely)
   HDR_L = 2,     // label tiles of flat blocks (list length)
   HDR_T = 3,     // tiles to visit: L + NNF * n_vtile
+  HDR_EMAX = 4,  // max_i |E_i| as float bits (fixed-point accumulation)
+  HDR_DLMAX = 5, // max_i |dloss_i| as float bits (fixed-point accumulation)
 };
 constexpr int HDR_BYTES = 256;
 enum StatusFlag : unsigned long long {
@@ -97,10 +99,32 @@ struct BwdArgs {
   const float* dloss;
   float* dE;            // [N][D] fp32, accumulated
   float* dC;            // [V][D] fp32, accumulated
+  // fixed-point accumulation (deterministic mode): when accE is non-null the
+  // contributions go to these int64 buffers instead of dE/dC
+  unsigned long long* accE;  // [N][D]
+  unsigned long long* accC;  // [V][D]
   unsigned long long* status;
   unsigned long long wait_limit_ns;
   int withhold_loads;   // test hook: the TMA producer issues nothing
 };
+
+// Fixed-point exponent s: contributions are stored as round(x * 2^s) in int64.
+// Every gradient entry is bounded by
+//   |dE_id| <= max_i|dloss_i| * 2 * max_v|C_v|   and
+//   |dC_vd| <= sum_i |dloss_i| * max_i|E_i| <= N * max|dloss| * max|E_i|,
+// so with B = 2 * max of both (and a factor 2 of headroom) the final sums stay
+// inside +-2^62 when s = 61 - ceil(log2 B).  Integer wrap-around in between
+// cancels, so only the final value needs the bound.
+__host__ __device__ inline int fixed_point_exponent(float cmax, float emax, float dlmax, int N) {
+  const float b1 = 2.f * dlmax * cmax;
+  const float b2 = (float)N * dlmax * emax;
+  float B = 2.f * fmaxf(b1, b2);
+  if (!(B > 0.f)) return 60;                  // nothing to accumulate
+  int e = 0;
+  frexpf(B, &e);                              // B < 2^e
+  int s = 61 - e;
+  return s < -60 ? -60 : (s > 100 ? 100 : s);
+}
 
 // Work unit u -> (vocabulary split r, token block m).  Units are grouped by
 // group_m token blocks; inside a group the token block varies fastest, so the

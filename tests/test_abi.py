@@ -130,3 +130,22 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "libcce.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         _native.load_library()
+
+
+def test_backward_ex_workspace_and_flags(lib):
+    _cpu_only()
+    from linear_cross_entropy_05_b200 import (cce_backward_ex, cce_backward_workspace_size,
+                                              cce_backward_workspace_size_ex)
+    up = lambda x: (x + 255) // 256 * 256
+    N, D, V = 8192, 2304, 256000
+    base = cce_backward_workspace_size(N, D, V)
+    assert cce_backward_workspace_size_ex(N, D, V, 0) == base
+    for flags in (1, 2, 3):   # deterministic / bf16 outputs: int64 accumulators for dE and dC
+        assert cce_backward_workspace_size_ex(N, D, V, flags) == base + up(8 * N * D) + up(8 * V * D)
+    assert cce_backward_workspace_size_ex(N, D, V, 4) == 0   # unknown flag
+    P = 1 << 20
+    args = [P, P, P, P, P, 256, 256, 4096, -100, 0.0, 0, P, P, P, 1 << 30, 0]
+    args[10] = 8
+    assert cce_backward_ex(*args, check=False) == 1          # unknown flag: rejected on the host
+    args[10] = 3
+    assert cce_backward_ex(*args, check=False) == 4          # valid, but no device here

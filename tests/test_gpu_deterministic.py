@@ -1,0 +1,90 @@
+"""Deterministic (fixed-point accumulated) backward and bf16 gradient outputs."""
+import numpy as np
+import pytest
+
+import oracle
+from linear_cross_entropy_05_b200 import synth
+
+from _gpu_helpers import GRAD_REL_FILTER_OFF, GRAD_REL_FILTER_ON, IGN, gpu_forward, rel_fro, to_dev
+
+pytestmark = pytest.mark.gpu
+
+EPS = synth.EPS_BF16_FILTER
+CASES = [
+    (synth.TINY.with_sizes(N=300, V=4096 + 77, D=264), 0.0),
+    (synth.GEMMA2_2B.with_sizes(N=1000, V=20000), EPS),
+    (synth.LLAMA3_8B.with_sizes(N=700, V=9000), EPS),
+    (synth.SMALL_LARGE_VOCAB.with_sizes(N=1500, V=20000), 0.0),
+]
+
+
+def _bwd(E, C, y, lse, dl, eps, **kw):
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    ws = L.Workspace()
+    dE, dC = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws, **kw)
+    st = L.read_status(ws)
+    assert st["status"] == 0 and st["flags"] == 0
+    return dE, dC, st
+
+
+@pytest.mark.parametrize("w,eps", CASES, ids=[c[0].name + ("-filter" if c[1] else "") for c in CASES])
+def test_deterministic_backward_is_bitwise_reproducible_and_matches_oracle(w, eps):
+    import torch
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    dloss = synth.random_dloss(8, w.N)
+    dl = torch.from_numpy(dloss).cuda()
+    lse_t = torch.from_numpy(lse).cuda()
+    a = _bwd(E, C, y, lse_t, dl, eps, deterministic=True)
+    b = _bwd(E, C, y, lse_t, dl, eps, deterministic=True)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])       # same bits
+    assert a[2]["live_tiles"] == b[2]["live_tiles"]
+    ref = _bwd(E, C, y, lse_t, dl, eps)                               # atomic fp32 accumulation
+    assert rel_fro(a[0].cpu().numpy(), ref[0].cpu().numpy()) < 1e-5
+    assert rel_fro(a[1].cpu().numpy(), ref[1].cpu().numpy()) < 1e-5
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    oE, oC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps)
+    assert rel_fro(a[0].cpu().numpy(), oE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(a[1].cpu().numpy(), oC) <= GRAD_REL_FILTER_OFF
+
+
+@pytest.mark.parametrize("w,eps", CASES[:2], ids=["ragged", "gemma-shaped-filter"])
+def test_bf16_gradient_outputs(w, eps):
+    import torch
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    dloss = synth.random_dloss(9, w.N)
+    dl = torch.from_numpy(dloss).cuda()
+    lse_t = torch.from_numpy(lse).cuda()
+    gE, gC, _ = _bwd(E, C, y, lse_t, dl, eps, bf16_grads=True)
+    assert gE.dtype == torch.bfloat16 and gC.dtype == torch.bfloat16
+    fE, fC, _ = _bwd(E, C, y, lse_t, dl, eps, deterministic=True)
+    # the bf16 outputs are the deterministic fp32 results rounded once
+    assert torch.equal(gE, fE.to(torch.bfloat16)) or rel_fro(gE.float().cpu().numpy(), fE.cpu().numpy()) < 4e-3
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    oE, oC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps)
+    tol = GRAD_REL_FILTER_OFF if eps <= 0 else GRAD_REL_FILTER_ON
+    assert rel_fro(gE.float().cpu().numpy(), oE) <= tol
+    assert rel_fro(gC.float().cpu().numpy(), oC) <= tol
+
+
+def test_deterministic_scale_edges():
+    # all-zero upstream gradient: exact zeros; a large dloss scale stays in range
+    import torch
+    w = synth.GEMMA2_2B.with_sizes(N=500, V=6000, D=256)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    lse_t = torch.from_numpy(lse).cuda()
+    z = torch.zeros(w.N, device="cuda")
+    dE, dC, _ = _bwd(E, C, y, lse_t, z, 0.0, deterministic=True)
+    assert (dE == 0).all() and (dC == 0).all()
+    big = torch.full((w.N,), 1e4, device="cuda")
+    dE, dC, _ = _bwd(E, C, y, lse_t, big, 0.0, deterministic=True)
+    rE, rC, _ = _bwd(E, C, y, lse_t, big, 0.0)
+    assert torch.isfinite(dE).all() and torch.isfinite(dC).all()
+    assert rel_fro(dE.cpu().numpy(), rE.cpu().numpy()) < 1e-5
+    assert rel_fro(dC.cpu().numpy(), rC.cpu().numpy()) < 1e-5
