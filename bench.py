@@ -526,6 +526,9 @@ def main(argv=None):
                     help="workload name (the default is the headline Gemma-2-2B-shaped head)")
     ap.add_argument("--N", type=int, default=None, help="override tokens (profiling cases)")
     ap.add_argument("--V", type=int, default=None, help="override vocabulary (profiling cases)")
+    ap.add_argument("--bwd-variant", type=int, choices=[0, 1, 2], default=0,
+                    help="backward kernel: 0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 buffers, "
+                         "2 = 2 stages / 8 epilogue warps")
     ap.add_argument("--deterministic", action="store_true",
                     help="bitwise reproducible backward (fixed-point accumulation)")
     ap.add_argument("--bf16-grads", action="store_true", help="bf16 dE/dC outputs (fixed-point accumulation)")
@@ -534,9 +537,10 @@ def main(argv=None):
     ap.add_argument("--suite", action="store_true",
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
-    if args.fwd_variant == "pair":
+    if args.fwd_variant == "pair" or args.bwd_variant:
         import linear_cross_entropy_05_b200 as L
-        L.cce_debug_set_forward_variant(1)
+        L.cce_debug_set_forward_variant(1 if args.fwd_variant == "pair" else 0)
+        L.cce_debug_set_backward_variant(args.bwd_variant)
     if args.suite:
         return run_suite(args)
     if args.warmup < 3:

@@ -168,6 +168,41 @@ CCE_API cce_status_t cce_backward_ex(const void* E, const void* C, const int64_t
                                      float filter_eps, unsigned flags, void* dE, void* dC, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* ---- Vocabulary-parallel form (e.g. one classifier shard per GPU) ----
+ * The log-sum-exp decomposes over any partition of the vocabulary:
+ *   lse = M + log sum_r s_r exp(m_r - M),  M = max_r m_r,
+ * where (m_r, s_r) are the max and the sum of exp(z - m_r) over shard r.  So
+ * each shard computes 3 floats per token, the shards exchange them (an
+ * all-gather of 12 bytes per token per shard, NCCL on multi-GPU), and every
+ * shard merges them into the same lse and loss.  Given that lse, each shard's
+ * backward yields its own rows of dC exactly and its share of dE; the full dE
+ * is the sum of the shares (an all-reduce).  Labels are always global ids.
+ * Workspaces: cce_forward_workspace_size / cce_backward_workspace_size with
+ * V = V_shard. */
+
+/* Forward on the classifier rows C_shard = C[v_offset : v_offset + V_shard].
+ *   stats [3][N] fp32 out: row 0 = max_v z_iv over the shard, row 1 =
+ *   sum_v exp(z_iv - max), row 2 = z_{i, y_i} if v_offset <= y_i <
+ *   v_offset + V_shard, else 0. */
+CCE_API cce_status_t cce_forward_shard(const void* E, const void* C_shard, const int64_t* y, int64_t N, int64_t D,
+                                       int64_t V_shard, int64_t v_offset, int64_t ignore_index, float* stats,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Merges R shards' stats ([R][3][N] fp32, device) into loss and lse (fp32
+ * [N]).  V_total: the full vocabulary size (labels outside [0, V_total) that
+ * are not ignore_index give a NaN loss). */
+CCE_API cce_status_t cce_merge_shards(const float* stats, int R, int64_t N, const int64_t* y, int64_t V_total,
+                                      int64_t ignore_index, float* loss, float* lse, void* stream);
+
+/* Backward for one shard, given the merged (global) lse: dC_shard [V_shard x
+ * D] is the exact gradient of the shard's classifier rows; dE_partial [N x D]
+ * is this shard's share of dE (sum the shares over shards).  Same filter as
+ * cce_backward (the tile grid starts at the shard's first row). */
+CCE_API cce_status_t cce_backward_shard(const void* E, const void* C_shard, const int64_t* y, const float* lse,
+                                        const float* dloss, int64_t N, int64_t D, int64_t V_shard,
+                                        int64_t v_offset, int64_t ignore_index, float filter_eps, float* dE_partial,
+                                        float* dC_shard, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then copies the status block of `workspace` (as left
  * by the last call that used it) into *out.  Returns CCE_ERR_TIMEOUT or
  * CCE_ERR_BAD_LABEL if the corresponding flag is set, else CCE_OK. */

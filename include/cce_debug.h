@@ -46,6 +46,15 @@ CCE_API void cce_debug_withhold_loads(int on);
  * Process-wide.  Returns CCE_ERR_INVALID_ARG for other values. */
 CCE_API cce_status_t cce_debug_set_forward_variant(int variant);
 
+/* Selects the backward kernel's buffering: 0 = three operand pipeline stages
+ * and one 4 KB reduction staging buffer per epilogue warp (the default),
+ * 1 = two stages and two staging buffers (the staging of a block overlaps the
+ * bulk read of the previous one), 2 = two stages and eight epilogue warps
+ * (two per TMEM lane group, splitting the gradient columns and the
+ * reduction pieces).  Same results; for A/B measurement.
+ * Process-wide.  Returns CCE_ERR_INVALID_ARG for other values. */
+CCE_API cce_status_t cce_debug_set_backward_variant(int variant);
+
 /* Profiling hook.  While set, every launch of the selected kernel records
  * `start_event` on the call's stream immediately before the launch and
  * `stop_event` immediately after it, so the caller can time that kernel alone

@@ -23,8 +23,9 @@ from typing import Optional, Tuple
 
 from . import _native
 from ._native import (CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCEError, cce_backward, cce_backward_ex,
-                      cce_backward_workspace_size, cce_backward_workspace_size_ex, cce_debug_forward_logits,
-                      cce_debug_set_forward_variant, cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns,
+                      cce_backward_shard, cce_backward_workspace_size, cce_backward_workspace_size_ex,
+                      cce_forward_shard, cce_merge_shards, cce_debug_forward_logits,
+                      cce_debug_set_backward_variant, cce_debug_set_forward_variant, cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns,
                       cce_debug_withhold_loads, cce_forward, cce_forward_noalloc,
                       cce_forward_workspace_size, cce_read_status,
                       cce_status_string, cce_version, load_library)
@@ -33,9 +34,12 @@ IGNORE_INDEX = -100
 
 __all__ = [
     "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "cce_forward",
-    "cce_forward_noalloc", "cce_backward", "cce_backward_ex", "cce_backward_workspace_size_ex", "cce_forward_workspace_size",
+    "cce_forward_noalloc", "cce_backward", "cce_backward_ex", "cce_backward_workspace_size_ex",
+    "cce_forward_shard", "cce_merge_shards", "cce_backward_shard", "forward_shard", "merge_shards",
+    "backward_shard", "vocab_parallel_forward_backward", "cce_forward_workspace_size",
     "cce_backward_workspace_size", "cce_read_status", "cce_status_string", "cce_version",
     "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "cce_debug_set_kernel_events", "cce_debug_withhold_loads", "cce_debug_set_forward_variant",
+    "cce_debug_set_backward_variant",
     "load_library",
     "forward", "backward", "read_status", "linear_cross_entropy", "Workspace",
 ]
@@ -146,3 +150,83 @@ def linear_cross_entropy(E, C, y, ignore_index: int = IGNORE_INDEX, filter_eps: 
     autograd support; the N x V logits are never materialised."""
     from ._autograd import LinearCrossEntropy
     return LinearCrossEntropy.apply(E, C, y, ignore_index, filter_eps)
+
+
+# ---------------------------------------------------------------------------
+# vocabulary-parallel form (one classifier shard per rank)
+# ---------------------------------------------------------------------------
+
+def forward_shard(E, C_shard, y, v_offset: int, ignore_index: int = IGNORE_INDEX,
+                  workspace: Optional[Workspace] = None, stream=None):
+    """Per-token (max, sum exp, target logit or 0) over the shard C_shard =
+    C[v_offset : v_offset + V_shard]: a float32 tensor [3, N]."""
+    torch = _torch()
+    _check_inputs(E, C_shard, y)
+    N, D = E.shape
+    V = C_shard.shape[0]
+    stats = torch.empty((3, N), dtype=torch.float32, device=E.device)
+    ws = (workspace or Workspace(E.device)).get(cce_forward_workspace_size(N, D, V))
+    cce_forward_shard(E.data_ptr(), C_shard.data_ptr(), y.data_ptr(), N, D, V, int(v_offset), ignore_index,
+                      stats.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    return stats
+
+
+def merge_shards(stats, y, V_total: int, ignore_index: int = IGNORE_INDEX, stream=None):
+    """stats [R, 3, N] (all shards) -> (loss, lse), fp32 [N]."""
+    torch = _torch()
+    stats = stats.contiguous()
+    R, three, N = stats.shape
+    if three != 3 or y.shape != (N,):
+        raise ValueError("stats must be [R, 3, N] and y [N]")
+    loss = torch.empty(N, dtype=torch.float32, device=stats.device)
+    lse = torch.empty(N, dtype=torch.float32, device=stats.device)
+    cce_merge_shards(stats.data_ptr(), R, N, y.data_ptr(), int(V_total), ignore_index, loss.data_ptr(),
+                     lse.data_ptr(), _stream_ptr(stream))
+    return loss, lse
+
+
+def backward_shard(E, C_shard, y, lse, dloss, v_offset: int, filter_eps: float = 0.0,
+                   ignore_index: int = IGNORE_INDEX, workspace: Optional[Workspace] = None, stream=None):
+    """(dE share, dC_shard) for one shard given the merged lse."""
+    torch = _torch()
+    _check_inputs(E, C_shard, y)
+    N, D = E.shape
+    V = C_shard.shape[0]
+    dE = torch.empty((N, D), dtype=torch.float32, device=E.device)
+    dC = torch.empty((V, D), dtype=torch.float32, device=E.device)
+    ws = (workspace or Workspace(E.device)).get(cce_backward_workspace_size(N, D, V))
+    cce_backward_shard(E.data_ptr(), C_shard.data_ptr(), y.data_ptr(), lse.data_ptr(), dloss.data_ptr(), N, D, V,
+                       int(v_offset), ignore_index, float(filter_eps), dE.data_ptr(), dC.data_ptr(), ws.data_ptr(),
+                       ws.numel(), _stream_ptr(stream))
+    return dE, dC
+
+
+def vocab_parallel_forward_backward(E, C_shard, y, v_offset: int, V_total: int, dloss=None,
+                                    filter_eps: float = 2.0 ** -12, ignore_index: int = IGNORE_INDEX, group=None):
+    """One vocabulary-parallel step on this rank's classifier shard.
+
+    Collectives (torch.distributed, NCCL on GPUs): an all-gather of the
+    [3, N] shard statistics (12 bytes per token per rank) and an all-reduce
+    of the dE shares.  Returns (loss, lse, dE, dC_shard); loss, lse and dE
+    are identical on every rank.  dloss defaults to the mean over kept
+    tokens.  Without an initialised process group this is the single-shard
+    case.
+    """
+    torch = _torch()
+    import torch.distributed as dist
+    stats = forward_shard(E, C_shard, y, v_offset, ignore_index)
+    if dist.is_available() and dist.is_initialized():
+        world = dist.get_world_size(group)
+        gathered = [torch.empty_like(stats) for _ in range(world)]
+        dist.all_gather(gathered, stats, group=group)
+        all_stats = torch.stack(gathered)
+    else:
+        all_stats = stats[None]
+    loss, lse = merge_shards(all_stats, y, V_total, ignore_index)
+    if dloss is None:
+        keep = (y != ignore_index).to(torch.float32)
+        dloss = keep / keep.sum().clamp_min(1.0)
+    dE, dC = backward_shard(E, C_shard, y, lse, dloss.contiguous(), v_offset, filter_eps, ignore_index)
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(dE, group=group)
+    return loss, lse, dE, dC

@@ -54,6 +54,14 @@ def load_library():
         lib.cce_backward_ex.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, ctypes.c_uint,
                                         c_vp, c_vp, c_vp, c_size, c_vp]
         lib.cce_backward_ex.restype = ctypes.c_int
+        lib.cce_forward_shard.argtypes = [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_size,
+                                          c_vp]
+        lib.cce_forward_shard.restype = ctypes.c_int
+        lib.cce_merge_shards.argtypes = [c_vp, ctypes.c_int, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp]
+        lib.cce_merge_shards.restype = ctypes.c_int
+        lib.cce_backward_shard.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_f32,
+                                           c_vp, c_vp, c_vp, c_size, c_vp]
+        lib.cce_backward_shard.restype = ctypes.c_int
         lib.cce_read_status.argtypes = [c_vp, c_vp, ctypes.POINTER(CCECounters)]
         lib.cce_read_status.restype = ctypes.c_int
         lib.cce_status_string.argtypes = [ctypes.c_int]
@@ -69,6 +77,8 @@ def load_library():
         lib.cce_forward_noalloc.restype = ctypes.c_int
         lib.cce_debug_set_forward_variant.argtypes = [ctypes.c_int]
         lib.cce_debug_set_forward_variant.restype = ctypes.c_int
+        lib.cce_debug_set_backward_variant.argtypes = [ctypes.c_int]
+        lib.cce_debug_set_backward_variant.restype = ctypes.c_int
         lib.cce_debug_withhold_loads.argtypes = [ctypes.c_int]
         lib.cce_debug_withhold_loads.restype = None
         lib.cce_debug_set_kernel_events.argtypes = [ctypes.c_int, c_vp, c_vp]
@@ -145,6 +155,34 @@ def cce_backward_ex(E: int, C: int, y: int, lse: int, dloss: int, N: int, D: int
     return st
 
 
+def cce_forward_shard(E: int, C_shard: int, y: int, N: int, D: int, V_shard: int, v_offset: int,
+                      ignore_index: int, stats: int, workspace: int, workspace_bytes: int, stream: int,
+                      check: bool = True) -> int:
+    st = load_library().cce_forward_shard(E, C_shard, y, N, D, V_shard, v_offset, ignore_index, stats, workspace,
+                                          workspace_bytes, stream)
+    if check:
+        _check(st, "cce_forward_shard")
+    return st
+
+
+def cce_merge_shards(stats: int, R: int, N: int, y: int, V_total: int, ignore_index: int, loss: int, lse: int,
+                     stream: int, check: bool = True) -> int:
+    st = load_library().cce_merge_shards(stats, R, N, y, V_total, ignore_index, loss, lse, stream)
+    if check:
+        _check(st, "cce_merge_shards")
+    return st
+
+
+def cce_backward_shard(E: int, C_shard: int, y: int, lse: int, dloss: int, N: int, D: int, V_shard: int,
+                       v_offset: int, ignore_index: int, filter_eps: float, dE_partial: int, dC_shard: int,
+                       workspace: int, workspace_bytes: int, stream: int, check: bool = True) -> int:
+    st = load_library().cce_backward_shard(E, C_shard, y, lse, dloss, N, D, V_shard, v_offset, ignore_index,
+                                           filter_eps, dE_partial, dC_shard, workspace, workspace_bytes, stream)
+    if check:
+        _check(st, "cce_backward_shard")
+    return st
+
+
 def cce_read_status(workspace: int, stream: int):
     c = CCECounters()
     st = load_library().cce_read_status(workspace, stream, ctypes.byref(c))
@@ -177,3 +215,8 @@ def cce_debug_withhold_loads(on: bool) -> None:
 def cce_debug_set_forward_variant(variant: int) -> None:
     """0 = single-CTA forward kernel (default), 1 = CTA-pair forward kernel."""
     _check(load_library().cce_debug_set_forward_variant(int(variant)), "cce_debug_set_forward_variant")
+
+
+def cce_debug_set_backward_variant(variant: int) -> None:
+    """0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 staging buffers."""
+    _check(load_library().cce_debug_set_backward_variant(int(variant)), "cce_debug_set_backward_variant")

@@ -22,12 +22,14 @@ cudaError_t launch_fwd_lse_pair(const CUtensorMap& tmE, const CUtensorMap& tmCh,
                                 cudaStream_t stream);
 cudaError_t launch_fwd_finalize(const void* E, const void* C, const int64_t* y, const FinArgs& a, float* loss,
                                 float* lse, cudaStream_t stream);
+cudaError_t launch_merge_shards(const float* stats, int R, int N, const int64_t* y, long long V_total,
+                                long long ignore_index, float* loss, float* lse, cudaStream_t stream);
 cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
-                       const CUtensorMap& tmdC, const BwdArgs& a, int grid, cudaStream_t stream);
+                       const CUtensorMap& tmdC, const BwdArgs& a, int grid, int variant, cudaStream_t stream);
 cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
                         int sms, cudaStream_t stream);
-cudaError_t launch_cnorm(const void* C, const PrepArgs& p, int sms, cudaStream_t stream);
-cudaError_t launch_fixed_prep(const void* E, const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream);
+cudaError_t launch_norms(const void* E, const void* C, const PrepArgs& p, int sms, cudaStream_t stream);
+cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
                                 bool bf16, int sms, cudaStream_t stream);
 }  // namespace cce
@@ -40,6 +42,8 @@ std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
 
 // Forward kernel variant: 0 = single CTAs (default), 1 = CTA pairs (cta_group::2).
 std::atomic<int> g_fwd_variant{0};
+// Backward kernel variant: 0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 buffers.
+std::atomic<int> g_bwd_variant{0};
 
 // Test hook: when set, the next launches' TMA producers issue no copies.
 std::atomic<int> g_withhold_loads{0};
@@ -176,7 +180,8 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
 // [n_vtile] | blk_flat, nonflat [n_mblk] | list [N] int2.  O(N + V/256).
 struct BwdPlan {
   int n_mblk, n_vtile;
-  size_t off_hdr, off_count, off_offset, off_cursor, off_flat, off_nonflat, off_list, zero_bytes, ws_bytes;
+  size_t off_hdr, off_count, off_offset, off_cursor, off_flat, off_nonflat, off_list, off_enorm, zero_bytes,
+      ws_bytes;
   size_t off_accE, off_accC;  // fixed-point accumulators (deterministic mode only)
 };
 
@@ -198,7 +203,8 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
   p->off_flat = p->zero_bytes;
   p->off_nonflat = p->off_flat + mb4;
   p->off_list = p->off_nonflat + mb4;
-  p->ws_bytes = p->off_list + align_up((size_t)N * sizeof(int2), 256);
+  p->off_enorm = p->off_list + align_up((size_t)N * sizeof(int2), 256);
+  p->ws_bytes = p->off_enorm + align_up((size_t)N * sizeof(float), 256);
   p->off_accE = p->off_accC = 0;
   if (flags) {
     p->off_accE = p->ws_bytes;
@@ -208,13 +214,17 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
   return true;
 }
 
+// shard_stats != nullptr: C is the vocabulary shard starting at global id
+// v_offset; per-token (max, sum exp, target) go to shard_stats [3][N] and
+// loss / lse are not written.
 cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
                           int64_t ignore_index, float* loss, float* lse, float* dbg_logits, void* ws,
-                          size_t ws_bytes, void* stream_) {
-  if (!E || !C || !y || !loss || !lse || !ws) return CCE_ERR_INVALID_ARG;
-  if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
+                          size_t ws_bytes, void* stream_, float* shard_stats = nullptr, int64_t v_offset = 0) {
+  if (!E || !C || !y || !ws) return CCE_ERR_INVALID_ARG;
+  if (!shard_stats && (!loss || !lse)) return CCE_ERR_INVALID_ARG;
+  if (!sizes_ok(N, D, V) || v_offset < 0) return CCE_ERR_INVALID_ARG;
   if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(loss, 4) || !aligned(lse, 4) ||
-      !aligned(ws, 256))
+      !aligned(shard_stats, 4) || !aligned(ws, 256))
     return CCE_ERR_MISALIGNED;
   if (!device_info().ok) return CCE_ERR_UNSUPPORTED_DEVICE;
   FwdPlan p;
@@ -257,6 +267,8 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   f.ignore_index = ignore_index;
   f.partial = partial;
   f.status = status;
+  f.shard_stats = shard_stats;
+  f.v_offset = v_offset;
   if (launch_fwd_finalize(E, C, y, f, loss, lse, stream) != cudaSuccess) return CCE_ERR_CUDA;
   return CCE_OK;
 }
@@ -302,6 +314,12 @@ cce_status_t cce_debug_set_forward_variant(int variant) {
   return CCE_OK;
 }
 
+cce_status_t cce_debug_set_backward_variant(int variant) {
+  if (variant < 0 || variant > 2) return CCE_ERR_INVALID_ARG;
+  g_bwd_variant.store(variant);
+  return CCE_OK;
+}
+
 cce_status_t cce_debug_set_kernel_events(int kernel, void* start_event, void* stop_event) {
   if (kernel < 0 || kernel > 1) return CCE_ERR_INVALID_ARG;
   g_events[kernel][0].store(start_event);
@@ -313,10 +331,14 @@ cce_status_t cce_debug_set_kernel_events(int kernel, void* start_event, void* st
 
 namespace {
 
+// shard: C is the vocabulary shard starting at global label id v_offset;
+// dC is that shard's gradient and dE this shard's share of the full dE.
 cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
                            int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, unsigned flags,
-                           void* dE, void* dC, void* workspace, size_t workspace_bytes, void* stream_) {
+                           void* dE, void* dC, void* workspace, size_t workspace_bytes, void* stream_,
+                           bool shard = false, int64_t v_offset = 0) {
   if (!E || !C || !y || !lse || !dloss || !dE || !dC || !workspace) return CCE_ERR_INVALID_ARG;
+  if (v_offset < 0) return CCE_ERR_INVALID_ARG;
   if (flags & ~kBwdFlagsAll) return CCE_ERR_INVALID_ARG;
   const bool fixed = flags != 0;
   const bool bf16_out = (flags & CCE_BWD_BF16_GRADS) != 0;
@@ -362,6 +384,8 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.n_tiles = bp.n_mblk * bp.n_vtile;
   a.group_m = std::min(a.n_mblk, 64);
   a.list_mode = filter_on ? 1 : 0;
+  a.shard_mode = shard ? 1 : 0;
+  a.v_offset = v_offset;
   a.hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);
   a.list = reinterpret_cast<const int2*>(ws + bp.off_list);
   a.nonflat = reinterpret_cast<const int*>(ws + bp.off_nonflat);
@@ -386,6 +410,8 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     pp.n_mblk = bp.n_mblk;
     pp.n_vtile = bp.n_vtile;
     pp.ignore_index = ignore_index;
+    pp.shard_mode = shard ? 1 : 0;
+    pp.v_offset = v_offset;
     pp.log_eps = logf(filter_eps);
     pp.hdr = reinterpret_cast<unsigned*>(ws + bp.off_hdr);
     pp.count = reinterpret_cast<unsigned*>(ws + bp.off_count);
@@ -394,17 +420,15 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     pp.blk_flat = reinterpret_cast<int*>(ws + bp.off_flat);
     pp.nonflat = reinterpret_cast<int*>(ws + bp.off_nonflat);
     pp.list = reinterpret_cast<int2*>(ws + bp.off_list);
+    pp.enorm = reinterpret_cast<float*>(ws + bp.off_enorm);
     pp.status = status;
-    if (filter_on) {
-      if (launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
-    } else {
-      if (launch_cnorm(C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
-    }
-    if (fixed && launch_fixed_prep(E, dloss, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (launch_norms(E, C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (filter_on && launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (fixed && launch_fixed_prep(dloss, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
   }
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
-  if (launch_bwd(tmE, tmC, tmdE, tmdC, a, grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (launch_bwd(tmE, tmC, tmdE, tmdC, a, grid, g_bwd_variant.load(), stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (fixed) {
     const unsigned* hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);
@@ -437,6 +461,33 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
                           float* dC, void* workspace, size_t workspace_bytes, void* stream) {
   return backward_impl(E, C, y, lse, dloss, N, D, V, ignore_index, filter_eps, 0u, dE, dC, workspace,
                        workspace_bytes, stream);
+}
+
+cce_status_t cce_forward_shard(const void* E, const void* C_shard, const int64_t* y, int64_t N, int64_t D,
+                               int64_t V_shard, int64_t v_offset, int64_t ignore_index, float* stats,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!stats) return CCE_ERR_INVALID_ARG;
+  return forward_impl(E, C_shard, y, N, D, V_shard, ignore_index, nullptr, nullptr, nullptr, workspace,
+                      workspace_bytes, stream, stats, v_offset);
+}
+
+cce_status_t cce_merge_shards(const float* stats, int R, int64_t N, const int64_t* y, int64_t V_total,
+                              int64_t ignore_index, float* loss, float* lse, void* stream) {
+  if (!stats || !y || !loss || !lse || R <= 0 || N <= 0 || N > INT_MAX || V_total <= 0) return CCE_ERR_INVALID_ARG;
+  if (!aligned(stats, 4) || !aligned(y, 8) || !aligned(loss, 4) || !aligned(lse, 4)) return CCE_ERR_MISALIGNED;
+  if (!device_info().ok) return CCE_ERR_UNSUPPORTED_DEVICE;
+  if (launch_merge_shards(stats, R, (int)N, y, V_total, ignore_index, loss, lse,
+                          reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return CCE_ERR_CUDA;
+  return CCE_OK;
+}
+
+cce_status_t cce_backward_shard(const void* E, const void* C_shard, const int64_t* y, const float* lse,
+                                const float* dloss, int64_t N, int64_t D, int64_t V_shard, int64_t v_offset,
+                                int64_t ignore_index, float filter_eps, float* dE_partial, float* dC_shard,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_impl(E, C_shard, y, lse, dloss, N, D, V_shard, ignore_index, filter_eps, 0u, dE_partial,
+                       dC_shard, workspace, workspace_bytes, stream, true, v_offset);
 }
 
 cce_status_t cce_read_status(const void* workspace, void* stream, cce_counters_t* out) {

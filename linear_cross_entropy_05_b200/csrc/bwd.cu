@@ -48,13 +48,16 @@ __device__ __forceinline__ void tile_coords(int t, int n_mblk, int n_vtile, int 
 }
 
 // Adds a 32 x 32 fp32 block held one row per lane (32 consecutive columns
-// each) to global memory through the TMA engine: the block is written to the
-// warp's 4 KB staging buffer in the 128-byte-swizzled layout of a {32, 32}
-// fp32 box and reduced into the tensor at (x = column, y = row) by one bulk
-// tensor reduce-add.  Rows/columns past the tensor's extent are clipped.
+// each) to global memory through the TMA engine: the block is written to one
+// of the warp's NXB 4 KB staging buffers (used in rotation) in the
+// 128-byte-swizzled layout of a {32, 32} fp32 box and reduced into the tensor
+// at (x = column, y = row) by one bulk tensor reduce-add.  Rows/columns past
+// the tensor's extent are clipped.
+template <int NXB>
 __device__ __forceinline__ void tma_red_block32(uint8_t* xb, int lane, const float (&v)[32], const CUtensorMap* map,
                                                 int x, int y) {
-  if (lane == 0) bulk_wait_group_read0();  // the previous block has left the buffer
+  // the block issued NXB pieces ago (which used this buffer) has left it
+  if (lane == 0) bulk_wait_group_read<NXB - 1>();
   __syncwarp();
 #pragma unroll
   for (int q = 0; q < 8; ++q)
@@ -131,19 +134,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 }  // namespace
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// NST: operand pipeline stages; NXB: reduction staging buffers per epilogue
+// warp; EPG: epilogue warps per TMEM lane group (1 or 2; with 2, the two
+// warps of a lane group split the softmax-gradient columns by 128-column half
+// and deal the reduction pieces of each chunk between them).
+template <int NST, int NXB, int EPG>
+__global__ void __launch_bounds__(64 + 128 * EPG, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
                const __grid_constant__ CUtensorMap tmdE, const __grid_constant__ CUtensorMap tmdC, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;                                   // BWD_STAGES x [128][64] bf16 (E slices)
-  uint8_t* sB = smem + BWD_STAGES * A_STAGE_BYTES;      // BWD_STAGES x [256][64] bf16 (C slices)
-  uint8_t* sG = sB + BWD_STAGES * B_STAGE_BYTES;        // 4 x [128][64] bf16, swizzled (G tile)
-  uint8_t* sX = sG + G_BYTES;                           // 4 x 4 KB reduction staging (one per epilogue warp)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 4 * 4096);
+  uint8_t* sA = smem;                                   // NST x [128][64] bf16 (E slices)
+  uint8_t* sB = smem + NST * A_STAGE_BYTES;      // NST x [256][64] bf16 (C slices)
+  uint8_t* sG = sB + NST * B_STAGE_BYTES;        // 4 x [128][64] bf16, swizzled (G tile)
+  uint8_t* sX = sG + G_BYTES;                           // 4*EPG x NXB x 4 KB reduction staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 4 * EPG * NXB * 4096);
+  constexpr int NEPI = 128 * EPG;                       // epilogue threads
   uint64_t* full = bars;
-  uint64_t* empty = bars + BWD_STAGES;
-  uint64_t* s_full = bars + 2 * BWD_STAGES;
+  uint64_t* empty = bars + NST;
+  uint64_t* s_full = bars + 2 * NST;
   uint64_t* s_empty = s_full + 1;
   uint64_t* g_full = s_full + 2;
   uint64_t* g_empty = s_full + 3;
@@ -162,17 +171,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < BWD_STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_empty, BM);
-    mbar_init(g_full, BM);
+    mbar_init(s_empty, NEPI);
+    mbar_init(g_full, NEPI);
     mbar_init(g_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&c_full[b], 1);
-      mbar_init(&c_empty[b], BM);
+      mbar_init(&c_empty[b], NEPI);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -222,7 +231,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
             tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
             armed |= 1u << stage;
-            if (++stage == BWD_STAGES) {
+            if (++stage == NST) {
               stage = 0;
               phase ^= 1u;
             }
@@ -232,7 +241,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     producer_done : {
       int dummy = 0;
       WaitCtl exit_wc{&dummy, a.wait_limit_ns};
-      for (int s = 0; s < BWD_STAGES; ++s)
+      for (int s = 0; s < NST; ++s)
         if (armed & (1u << s)) mbar_wait(&full[s], (s < stage) ? phase : (phase ^ 1u), exit_wc);
     }
     }
@@ -265,7 +274,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             umma_bf16(tmem_base + TM_S, sdesc_sw128(a_addr + k * 32, 16, 1024),
                       sdesc_sw128(b_addr + k * 32, 16, 1024), IDESC_S, (kb | k) != 0);
           umma_commit(&empty[stage]);
-          if (++stage == BWD_STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
@@ -305,7 +314,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             umma_commit(&empty[stage]);
             umma_commit(&c_full[b]);
-            if (++stage == BWD_STAGES) {
+            if (++stage == NST) {
               stage = 0;
               phase ^= 1u;
             }
@@ -326,6 +335,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- epilogue ----------------
     const int lane_grp = warp & 3;
+    const int ew = warp - 2;               // epilogue warp 0 .. 4*EPG-1
+    const int hsel = ew >> 2;              // with EPG = 2: the 128-column half this warp forms G for
     const int rib = lane_grp * 32 + lane;  // row inside the tile (token, or vocab for dC)
     const uint32_t lane_addr = (uint32_t)(lane_grp * 32) << 16;
     const float eps = a.filter_eps;
@@ -334,7 +345,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t cfe0 = 0u, cfe1 = 0u;  // drains of contraction buffers 0 / 1 so far
     unsigned long long n_live = 0, n_dead = 0;
     uint8_t* g_row = sG + rib * 128;
-    uint8_t* xb = sX + (warp - 2) * 4096;
+    uint8_t* const xb0 = sX + ew * NXB * 4096;
+    int xbi = 0;  // next staging buffer of this warp (rotation over NXB)
+    auto next_xb = [&]() -> uint8_t* {
+      uint8_t* p = xb0 + xbi * 4096;
+      xbi = (xbi + 1 == NXB) ? 0 : xbi + 1;
+      return p;
+    };
     const bool fixed = a.accE != nullptr;
     float fx_scale = 0.f;
     if (fixed)
@@ -351,13 +368,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool valid = row < a.N;
       long long yl = valid ? a.y[row] : a.ignore_index;
       if (yl == a.ignore_index) valid = false;
-      if (valid && (yl < 0 || yl >= a.V)) {
+      if (a.shard_mode) {
+        // vocabulary shard: labels are global ids; a label outside the shard
+        // contributes no one-hot entry here but the token's softmax row does
+        yl -= a.v_offset;
+      } else if (valid && (yl < 0 || yl >= a.V)) {
         valid = false;
         atomicOr(a.status + ST_FLAGS, SF_BAD_LABEL);
       }
       const float lse2 = valid ? a.lse[row] * LOG2E : 0.f;
       const float dl = valid ? a.dloss[row] : 0.f;
-      const int ycol = valid ? (int)(yl - (long long)vt * BN) : -1;  // may fall outside [0, BN)
+      const long long yrel = yl - (long long)vt * BN;
+      const int ycol = (valid && yrel >= 0 && yrel < BN) ? (int)yrel : -1;
       const int ncols = min(BN, a.V - vt * BN);
 
       if (!mbar_wait(s_full, sph, wc)) break;
@@ -368,8 +390,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // when the filter is off)
       const uint32_t halves = ncols > 128 ? 3u : 1u;
       uint32_t live = filter_on ? 0u : halves;
+      constexpr int NC = (BN / 32) / EPG;  // 32-column chunks of S handled by this warp
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = hsel * NC; c < hsel * NC + NC; ++c) {
         float x[32];
         tmem_ld32(tmem_base + lane_addr + TM_S + c * 32, x);
         uint32_t pk[16];
@@ -422,35 +445,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (b) ++cfe1; else ++cfe0;
         tc_fence_after();
         const int d0 = kb * BK;
-        // dE rows of this warp: tokens row0 .. row0 + 31
+        // Reduction pieces of this chunk (32 rows of this lane group x 32
+        // columns each): dE q0, dE q1, then dC q0, q1 of every live half.
+        // With EPG = 2 the pieces alternate between the two warps.
+        int piece = 0;
 #pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 2; ++q, ++piece) {
+          const bool mine = (piece % EPG) == hsel;
           float v[32];
-          tmem_ld32(tmem_base + lane_addr + tm_de(b) + q * 32, v);
-          if (d0 + q * 32 < a.D && row0 < a.N) {
+          if (mine) tmem_ld32(tmem_base + lane_addr + tm_de(b) + q * 32, v);
+          if (mine && d0 + q * 32 < a.D && row0 < a.N) {
             if (fixed)
-              fixed_red_block32(xb, lane, v, a.accE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D, rows_valid,
-                                min(32, a.D - (d0 + q * 32)), fx_scale);
+              fixed_red_block32(next_xb(), lane, v, a.accE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D,
+                                rows_valid, min(32, a.D - (d0 + q * 32)), fx_scale);
             else
-              tma_red_block32(xb, lane, v, &tmdE, d0 + q * 32, row0);
+              tma_red_block32<NXB>(next_xb(), lane, v, &tmdE, d0 + q * 32, row0);
           }
         }
-        // dC rows of this warp: vocabulary rows vt*256 + h*128 + lane_grp*32 ..
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           if (!((hmask >> h) & 1)) continue;
           const int vr0 = vt * BN + h * BM + lane_grp * 32;
 #pragma unroll 1
-          for (int q = 0; q < 2; ++q) {
+          for (int q = 0; q < 2; ++q, ++piece) {
+            const bool mine = (piece % EPG) == hsel;
             float v[32];
-            tmem_ld32(tmem_base + lane_addr + tm_dc(b) + h * 64 + q * 32, v);
-            if (d0 + q * 32 < a.D && vr0 < a.V) {
+            if (mine) tmem_ld32(tmem_base + lane_addr + tm_dc(b) + h * 64 + q * 32, v);
+            if (mine && d0 + q * 32 < a.D && vr0 < a.V) {
               if (fixed)
-                fixed_red_block32(xb, lane, v, a.accC + (size_t)vr0 * a.D + d0 + q * 32, (size_t)a.D,
+                fixed_red_block32(next_xb(), lane, v, a.accC + (size_t)vr0 * a.D + d0 + q * 32, (size_t)a.D,
                                   __ballot_sync(0xffffffffu, vr0 + lane < a.V), min(32, a.D - (d0 + q * 32)),
                                   fx_scale);
               else
-                tma_red_block32(xb, lane, v, &tmdC, d0 + q * 32, vr0);
+                tma_red_block32<NXB>(next_xb(), lane, v, &tmdC, d0 + q * 32, vr0);
             }
           }
         }
@@ -460,7 +487,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
     }
     if (lane == 0) bulk_wait_group0();  // every reduction issued by this warp has landed
-    if (rib == 0) {
+    if (rib == 0 && hsel == 0) {
       atomicAdd(a.status + ST_LIVE_TILES, n_live);
       atomicAdd(a.status + ST_DEAD_TILES, n_dead);
       atomicAdd(a.status + ST_TILES, n_live + n_dead);
@@ -478,15 +505,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status + ST_FLAGS, SF_TIMEOUT);
 }
 
-size_t bwd_smem_bytes() { return 1024 + (size_t)BWD_STAGES * STAGE_BYTES + G_BYTES + 4 * 4096 + 256; }
+template <int NST, int NXB, int EPG>
+size_t bwd_smem_bytes() {
+  return 1024 + (size_t)NST * STAGE_BYTES + G_BYTES + (size_t)4 * EPG * NXB * 4096 + 256;
+}
 
-cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
-                       const CUtensorMap& tmdC, const BwdArgs& a, int grid, cudaStream_t stream) {
-  const size_t smem = bwd_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int NST, int NXB, int EPG>
+cudaError_t launch_bwd_t(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
+                         const CUtensorMap& tmdC, const BwdArgs& a, int grid, cudaStream_t stream) {
+  const size_t smem = bwd_smem_bytes<NST, NXB, EPG>();
+  cudaError_t e =
+      cudaFuncSetAttribute(bwd_kernel<NST, NXB, EPG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  bwd_kernel<<<grid, NUM_THREADS, smem, stream>>>(tmE, tmC, tmdE, tmdC, a);
+  bwd_kernel<NST, NXB, EPG><<<grid, 64 + 128 * EPG, smem, stream>>>(tmE, tmC, tmdE, tmdC, a);
   return cudaGetLastError();
+}
+
+// variant 0: 3 operand stages, one staging buffer, 4 epilogue warps (default);
+// variant 1: 2 stages, two staging buffers per warp (staging overlaps the bulk
+//            read of the previous block);
+// variant 2: 2 stages, 8 epilogue warps (two per TMEM lane group).
+cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
+                       const CUtensorMap& tmdC, const BwdArgs& a, int grid, int variant, cudaStream_t stream) {
+  if (variant == 1) return launch_bwd_t<2, 2, 1>(tmE, tmC, tmdE, tmdC, a, grid, stream);
+  if (variant == 2) return launch_bwd_t<2, 1, 2>(tmE, tmC, tmdE, tmdC, a, grid, stream);
+  return launch_bwd_t<BWD_STAGES, 1, 1>(tmE, tmC, tmdE, tmdC, a, grid, stream);
 }
 
 }  // namespace cce

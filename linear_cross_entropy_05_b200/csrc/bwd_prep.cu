@@ -14,7 +14,8 @@
 //
 // Kernels (stream order):
 //   prep_cnorm    max_v |C_v| (fp32, atomicMax on the float's bits)
-//   prep_blocks   per token block: row norms, flatness, label-tile counts
+//   prep_enorm    |E_i| per token (and the maximum)
+//   prep_blocks   per token block: flatness, label-tile counts
 //   prep_scan     exclusive scan of the per-vocabulary-tile counts; totals
 //   prep_scatter  label tiles of flat blocks, ordered by vocabulary tile so
 //                 concurrent CTAs share C tiles in L2
@@ -64,41 +65,49 @@ __global__ void __launch_bounds__(256) prep_cnorm_kernel(const __nv_bfloat16* __
   if (lane == 0) atomicMax(p.hdr + HDR_CMAX, __float_as_uint(mx));  // non-negative: bit order = value order
 }
 
+// |E_i| for every token (one warp per row, all SMs), and their maximum.
+__global__ void __launch_bounds__(256) prep_enorm_kernel(const __nv_bfloat16* __restrict__ E, PrepArgs p) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  float mx = 0.f;
+  for (int i = gw; i < p.N; i += nw) {
+    const float n = warp_row_norm(E + (size_t)i * p.D, p.D, lane);
+    if (lane == 0) p.enorm[i] = n;
+    mx = fmaxf(mx, n);
+  }
+  if (lane == 0) atomicMax(p.hdr + HDR_EMAX, __float_as_uint(mx));
+}
+
 // One CTA (128 threads) per token block.
-__global__ void __launch_bounds__(128) prep_blocks_kernel(const __nv_bfloat16* __restrict__ E,
-                                                          const int64_t* __restrict__ y,
+__global__ void __launch_bounds__(128) prep_blocks_kernel(const int64_t* __restrict__ y,
                                                           const float* __restrict__ lse, PrepArgs p) {
-  __shared__ float nrm[BM];
   __shared__ int tl[BM];
   const int m = blockIdx.x;
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  for (int rr = 0; rr < 32; ++rr) {
-    const int r = warp * 32 + rr;
-    const int row = m * BM + r;
-    float n = 0.f;
-    if (row < p.N) n = warp_row_norm(E + (size_t)row * p.D, p.D, lane);
-    if (lane == 0) nrm[r] = n;
-  }
-  __syncthreads();
+  const int t = threadIdx.x;
   const int row = m * BM + t;
   long long yl = row < p.N ? y[row] : p.ignore_index;
-  const bool valid = row < p.N && label_ok(yl, p.ignore_index, p.V);
-  if (row < p.N && yl != p.ignore_index && !valid) atomicOr(p.status + ST_FLAGS, SF_BAD_LABEL);
+  // kept token (its softmax row matters for flatness) and, separately, whether
+  // its label has a column in this C (always, unless C is a vocabulary shard)
+  const bool valid = row < p.N && (p.shard_mode ? yl != p.ignore_index : label_ok(yl, p.ignore_index, p.V));
+  if (!p.shard_mode && row < p.N && yl != p.ignore_index && !valid) atomicOr(p.status + ST_FLAGS, SF_BAD_LABEL);
+  const long long ylocal = yl - (p.shard_mode ? p.v_offset : 0);
+  const bool has_col = valid && ylocal >= 0 && ylocal < p.V;
   const float cmax = __uint_as_float(p.hdr[HDR_CMAX]);
   // Margins cover the fp32 rounding of the norms, of the recomputed logits and
   // of the exp2 in the exact test.
   const float margin = 1.0f / 1024.0f;
   bool flat = true;
-  if (valid) flat = nrm[t] * cmax * (1.0f + margin) + margin < lse[row] + p.log_eps - margin;
+  if (valid) flat = p.enorm[row] * cmax * (1.0f + margin) + margin < lse[row] + p.log_eps - margin;
   const int all_flat = __syncthreads_and(flat);
   if (t == 0) p.blk_flat[m] = all_flat;
   if (!all_flat) {
     if (t == 0) p.nonflat[atomicAdd(p.hdr + HDR_NNF, 1u)] = m;
     return;
   }
-  tl[t] = valid ? (int)(yl / BN) : -1;
+  tl[t] = has_col ? (int)(ylocal / BN) : -1;
   __syncthreads();
-  bool owner = valid;
+  bool owner = has_col;
   for (int j = 0; j < t && owner; ++j) owner = tl[j] != tl[t];
   if (owner) atomicAdd(p.count + tl[t], 1u);
 }
@@ -165,10 +174,11 @@ __global__ void __launch_bounds__(128) prep_scatter_kernel(const int64_t* __rest
   const int t = threadIdx.x;
   const int row = m * BM + t;
   const long long yl = row < p.N ? y[row] : p.ignore_index;
-  const bool valid = row < p.N && label_ok(yl, p.ignore_index, p.V);
-  tl[t] = valid ? (int)(yl / BN) : -1;
+  const long long ylocal = yl - (p.shard_mode ? p.v_offset : 0);
+  const bool has_col = row < p.N && yl != p.ignore_index && ylocal >= 0 && ylocal < p.V;
+  tl[t] = has_col ? (int)(ylocal / BN) : -1;
   __syncthreads();
-  bool owner = valid;
+  bool owner = has_col;
   for (int j = 0; j < t && owner; ++j) owner = tl[j] != tl[t];
   if (owner) {
     const int v = tl[t];
@@ -177,16 +187,10 @@ __global__ void __launch_bounds__(128) prep_scatter_kernel(const int64_t* __rest
   }
 }
 
-// Deterministic mode: max_i |E_i| and max_i |dloss_i| for the fixed-point
-// scale (maxima do not depend on the order of the atomics).
-__global__ void __launch_bounds__(256) prep_fixed_kernel(const __nv_bfloat16* __restrict__ E,
-                                                         const float* __restrict__ dloss, PrepArgs p) {
+// Deterministic mode: max_i |dloss_i| for the fixed-point scale (max_i |E_i|
+// comes from prep_enorm; maxima do not depend on the order of the atomics).
+__global__ void __launch_bounds__(256) prep_fixed_kernel(const float* __restrict__ dloss, PrepArgs p) {
   const int lane = threadIdx.x & 31;
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  float emax = 0.f;
-  for (int i = gw; i < p.N; i += nw) emax = fmaxf(emax, warp_row_norm(E + (size_t)i * p.D, p.D, lane));
-  if (lane == 0) atomicMax(p.hdr + HDR_EMAX, __float_as_uint(emax));
   float dmax = 0.f;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.N; i += gridDim.x * blockDim.x)
     dmax = fmaxf(dmax, fabsf(dloss[i]));
@@ -214,8 +218,8 @@ __global__ void __launch_bounds__(256) fixed_to_out_kernel(const unsigned long l
   }
 }
 
-cudaError_t launch_fixed_prep(const void* E, const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream) {
-  prep_fixed_kernel<<<sms * 4, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E), dloss, p);
+cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream) {
+  prep_fixed_kernel<<<sms, 256, 0, stream>>>(dloss, p);
   return cudaGetLastError();
 }
 
@@ -225,16 +229,18 @@ cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t
   return cudaGetLastError();
 }
 
-cudaError_t launch_cnorm(const void* C, const PrepArgs& p, int sms, cudaStream_t stream) {
+// Norm pre-pass shared by the filter and the fixed-point scale: max_v |C_v|,
+// |E_i| per token and max_i |E_i|.
+cudaError_t launch_norms(const void* E, const void* C, const PrepArgs& p, int sms, cudaStream_t stream) {
   prep_cnorm_kernel<<<sms * 8, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(C), p);
+  prep_enorm_kernel<<<sms * 4, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E), p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
                         int sms, cudaStream_t stream) {
-  const int cgrid = sms * 8;
-  prep_cnorm_kernel<<<cgrid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(C), p);
-  prep_blocks_kernel<<<p.n_mblk, 128, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E), y, lse, p);
+  // expects launch_norms to have run
+  prep_blocks_kernel<<<p.n_mblk, 128, 0, stream>>>(y, lse, p);
   prep_scan_kernel<<<1, 1024, 0, stream>>>(p);
   prep_scatter_kernel<<<p.n_mblk, 128, 0, stream>>>(y, p);
   return cudaGetLastError();

@@ -67,11 +67,18 @@ struct FinArgs {
   long long ignore_index;
   const float2* partial;
   unsigned long long* status;
+  // vocabulary shard (C holds rows v_offset .. v_offset + V - 1 of the full
+  // classifier): write per-token (max, sum exp(z - max), target logit or 0)
+  // to shard_stats [3][N] instead of loss / lse
+  float* shard_stats;
+  long long v_offset;
 };
 
 struct PrepArgs {
   int N, D, V, n_mblk, n_vtile;
   long long ignore_index;
+  int shard_mode;         // labels are global ids; C is the shard [v_offset, v_offset + V)
+  long long v_offset;
   float log_eps;          // ln(filter_eps)
   unsigned* hdr;          // PrepHeader words
   unsigned* count;        // [n_vtile] label tiles per vocabulary tile
@@ -80,6 +87,7 @@ struct PrepArgs {
   int* blk_flat;          // [n_mblk]
   int* nonflat;           // [n_mblk] ids of blocks that are not flat
   int2* list;             // [<= N] (token block, vocabulary tile), vocabulary-major
+  float* enorm;           // [N] |E_i|
   unsigned long long* status;
 };
 
@@ -89,6 +97,8 @@ struct BwdArgs {
   int n_tiles;          // tiles to visit (dense mode)
   int group_m;          // token blocks per raster group (dense mode)
   int list_mode;        // 1: visit the pre-pass list (hdr, list, nonflat)
+  int shard_mode;       // 1: C is a vocabulary shard starting at global id v_offset
+  long long v_offset;
   const unsigned* hdr;
   const int2* list;
   const int* nonflat;

@@ -475,6 +475,40 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const __nv_bfloat16* 
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   const float L = M + logf(s);
 
+  if (a.shard_stats) {
+    // vocabulary shard: (max, sum exp(z - max)) over the shard and the target
+    // logit if the label falls in it (0 otherwise; exactly one shard owns it)
+    const long long tg = y[row];
+    const long long tl = tg - a.v_offset;
+    float z = 0.f;
+    if (tg != a.ignore_index && tl >= 0 && tl < a.V) {
+      const uint4* er = reinterpret_cast<const uint4*>(E + (size_t)row * a.D);
+      const uint4* cr = reinterpret_cast<const uint4*>(C + (size_t)tl * a.D);
+      float z0 = 0.f, z1 = 0.f;
+      for (int i = lane; i < (a.D >> 3); i += 32) {
+        const uint4 ev = __ldg(er + i), cv = __ldg(cr + i);
+        const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&ev);
+        const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&cv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 ef = __bfloat1622float2(e2[j]);
+          const float2 cf = __bfloat1622float2(c2[j]);
+          z0 = fmaf(ef.x, cf.x, z0);
+          z1 = fmaf(ef.y, cf.y, z1);
+        }
+      }
+      z = z0 + z1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    }
+    if (lane == 0) {
+      a.shard_stats[row] = M;
+      a.shard_stats[(size_t)a.N + row] = s;
+      a.shard_stats[2 * (size_t)a.N + row] = z;
+    }
+    return;
+  }
+
   const long long t = y[row];
   float out;
   if (t == a.ignore_index) {
@@ -509,6 +543,46 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const __nv_bfloat16* 
     lse[row] = L;
     loss[row] = out;
   }
+}
+
+// Merge R vocabulary shards' (max, sum exp, target) statistics into the
+// per-token loss and lse: lse = M + log sum_r s_r exp(m_r - M), M = max_r m_r;
+// the target logit is the sum over shards (only the owner contributes).
+__global__ void __launch_bounds__(256) merge_shards_kernel(const float* __restrict__ stats, int R, int N,
+                                                           const int64_t* __restrict__ y, long long V_total,
+                                                           long long ignore_index, float* __restrict__ loss,
+                                                           float* __restrict__ lse, unsigned long long* status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  const size_t sh = 3 * (size_t)N;
+  float M = -INFINITY;
+  for (int r = 0; r < R; ++r) M = fmaxf(M, stats[r * sh + i]);
+  float s = 0.f, z = 0.f;
+  for (int r = 0; r < R; ++r) {
+    const float m = stats[r * sh + i];
+    if (m != -INFINITY) s += stats[r * sh + N + i] * expf(m - M);
+    z += stats[r * sh + 2 * (size_t)N + i];
+  }
+  const float L = M + logf(s);
+  const long long t = y[i];
+  float out;
+  if (t == ignore_index) {
+    out = 0.f;
+  } else if (t >= 0 && t < V_total) {
+    out = L - z;
+  } else {
+    out = __int_as_float(0x7fc00000);
+    if (status) atomicOr(status + ST_FLAGS, SF_BAD_LABEL);
+  }
+  lse[i] = L;
+  loss[i] = out;
+}
+
+cudaError_t launch_merge_shards(const float* stats, int R, int N, const int64_t* y, long long V_total,
+                                long long ignore_index, float* loss, float* lse, cudaStream_t stream) {
+  merge_shards_kernel<<<(N + 255) / 256, 256, 0, stream>>>(stats, R, N, y, V_total, ignore_index, loss, lse,
+                                                           nullptr);
+  return cudaGetLastError();
 }
 
 size_t fwd_smem_bytes() { return 1024 + (size_t)FWD_STAGES * STAGE_BYTES + 256; }

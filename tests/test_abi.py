@@ -116,10 +116,11 @@ def test_workspace_size_without_device_is_zero(lib):
     from linear_cross_entropy_05_b200 import cce_backward_workspace_size, cce_forward_workspace_size
     assert cce_forward_workspace_size(8192, 2304, 256000) == 0
     assert cce_forward_workspace_size(0, 8, 8) == 0
-    # status 256 + header 256 + 3 x [V/256] u32 + 2 x [N/128] i32 + N int2, each rounded to 256 bytes
+    # status 256 + header 256 + 3 x [V/256] u32 + 2 x [N/128] i32 + N int2 + N f32,
+    # each rounded to 256 bytes
     up = lambda x: (x + 255) // 256 * 256
     for N, V in ((8192, 256000), (300, 4173), (65536, 262144)):
-        want = 512 + 3 * up(4 * (-(-V // 256))) + 2 * up(4 * (-(-N // 128))) + up(8 * N)
+        want = 512 + 3 * up(4 * (-(-V // 256))) + 2 * up(4 * (-(-N // 128))) + up(8 * N) + up(4 * N)
         assert cce_backward_workspace_size(N, 2304, V) == want
     assert cce_backward_workspace_size(8192, 2305, 256000) == 0
 
@@ -149,3 +150,17 @@ def test_backward_ex_workspace_and_flags(lib):
     assert cce_backward_ex(*args, check=False) == 1          # unknown flag: rejected on the host
     args[10] = 3
     assert cce_backward_ex(*args, check=False) == 4          # valid, but no device here
+
+
+def test_shard_entry_points_validate_on_the_host(lib):
+    _cpu_only()
+    from linear_cross_entropy_05_b200 import cce_backward_shard, cce_forward_shard, cce_merge_shards
+    P = 1 << 20
+    assert cce_forward_shard(P, P, P, 256, 256, 4096, 0, -100, 0, P, 1 << 20, 0, check=False) == 1   # no stats
+    assert cce_forward_shard(P, P, P, 256, 256, 4096, -1, -100, P, P, 1 << 20, 0, check=False) == 1  # offset < 0
+    assert cce_forward_shard(P, P, P, 256, 256, 4096, 4096, -100, P, P, 1 << 20, 0, check=False) == 4
+    assert cce_merge_shards(P, 0, 256, P, 8192, -100, P, P, 0, check=False) == 1                      # R = 0
+    assert cce_merge_shards(P, 2, 256, P + 4, 8192, -100, P, P, 0, check=False) == 2                  # y misaligned
+    assert cce_merge_shards(P, 2, 256, P, 8192, -100, P, P, 0, check=False) == 4
+    assert cce_backward_shard(P, P, P, P, P, 256, 256, 4096, -5, -100, 0.0, P, P, P, 1 << 20, 0,
+                              check=False) == 1

@@ -178,3 +178,46 @@ def test_autograd_wrapper_matches_oracle():
     # the wrapper returns bf16 gradients (the dtype of E and C)
     assert rel_fro(E.grad.float().cpu().numpy(), rE) <= 1e-2
     assert rel_fro(C.grad.float().cpu().numpy(), rC) <= 1e-2
+
+
+@pytest.mark.parametrize("variant", [1, 2], ids=["2stages-2buffers", "8-epilogue-warps"])
+@pytest.mark.parametrize("eps", [0.0, EPS], ids=["filter-off", "filter-on"])
+def test_backward_kernel_variants_match_oracle(variant, eps):
+    # the alternative buffering / epilogue-warp layouts (selectable for A/B
+    # measurement) must give the default kernel's results
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=700, V=12000 + 77)
+    L.cce_debug_set_backward_variant(variant)
+    try:
+        inp, dloss, olse, gE, gC, st = _run(w, eps)
+    finally:
+        L.cce_debug_set_backward_variant(0)
+    assert st["status"] == 0
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=TILE)
+    assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
+
+
+@pytest.mark.parametrize("eps", [0.0, EPS], ids=["filter-off", "filter-on"])
+def test_labels_at_vocabulary_edges(eps):
+    # labels 0 and V-1 (the last, ragged vocabulary tile) and a token block
+    # whose labels all fall in one tile
+    w = synth.GEMMA2_2B.with_sizes(N=300, V=5000 + 77, D=256)
+    inp = synth.make_inputs(w)
+    y = inp["y"]
+    y[:40] = 0
+    y[40:80] = w.V - 1
+    y[128:256] = w.V - 1
+    E, C, yd = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, yd)
+    ol, olse = oracle.forward(inp["E"], inp["C"], y, IGN)
+    assert np.abs(loss - ol).max() <= 1e-2
+    dloss = synth.random_dloss(12, w.N)
+    dE, dC, st = gpu_backward(E, C, yd, lse, dloss, eps)
+    assert st["status"] == 0
+    fE, fC = oracle.backward(inp["E"], inp["C"], y, olse, dloss, IGN, filter_eps=eps, tile=TILE)
+    assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
+    # the label rows of dC carry the one-hot part
+    gC = dC.cpu().numpy()
+    assert rel_fro(gC[[0, w.V - 1]], fC[[0, w.V - 1]]) <= GRAD_REL_FILTER_OFF

@@ -1,0 +1,101 @@
+"""Vocabulary-parallel form: shards of C on one GPU, merged, against the
+unsharded path and the oracle.  (Each shard would live on its own GPU; the
+exchange is an all-gather of the [3, N] statistics and an all-reduce of dE.)"""
+import numpy as np
+import pytest
+
+import oracle
+from linear_cross_entropy_05_b200 import synth
+
+from _gpu_helpers import GRAD_REL_FILTER_OFF, GRAD_REL_FILTER_ON, IGN, LOSS_ABS, gpu_backward, gpu_forward, \
+    rel_fro, to_dev
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    (synth.GEMMA2_2B.with_sizes(N=1000, V=20077), [0, 7001, 14500, 20077]),
+    (synth.LLAMA3_8B.with_sizes(N=700, V=9000), [0, 4096, 9000]),
+    (synth.TINY.with_sizes(N=300, V=4173, D=264), [0, 1, 2000, 4173]),     # a one-row shard
+]
+
+
+def _shards(w, bounds, C):
+    return [(bounds[k], C[bounds[k]:bounds[k + 1]].contiguous()) for k in range(len(bounds) - 1)]
+
+
+@pytest.mark.parametrize("w,bounds", CASES, ids=[c[0].name for c in CASES])
+def test_sharded_forward_merge_matches_unsharded(w, bounds):
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    stats = torch.stack([L.forward_shard(E, Cs, y, off, IGN) for off, Cs in _shards(w, bounds, C)])
+    loss, lse = L.merge_shards(stats, y, w.V, IGN)
+    ref_loss, ref_lse, _ = gpu_forward(E, C, y)
+    assert np.abs(loss.cpu().numpy() - ref_loss).max() <= 1e-4
+    assert np.abs(lse.cpu().numpy() - ref_lse).max() <= 1e-4
+    ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    assert np.abs(loss.cpu().numpy() - ol).max() <= LOSS_ABS
+    assert (loss.cpu().numpy()[inp["y"] == IGN] == 0).all()
+
+
+@pytest.mark.parametrize("eps", [0.0, synth.EPS_BF16_FILTER], ids=["filter-off", "filter-on"])
+@pytest.mark.parametrize("w,bounds", CASES[:2], ids=[c[0].name for c in CASES[:2]])
+def test_sharded_backward_assembles_the_full_gradient(w, bounds, eps):
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, _ = gpu_forward(E, C, y)
+    lse_t = torch.from_numpy(lse).cuda()
+    dloss = synth.random_dloss(21, w.N)
+    dl = torch.from_numpy(dloss).cuda()
+    dE = torch.zeros_like(E, dtype=torch.float32)
+    dCs = []
+    for off, Cs in _shards(w, bounds, C):
+        dEp, dCp = L.backward_shard(E, Cs, y, lse_t, dl, off, eps, IGN)
+        dE += dEp
+        dCs.append(dCp)
+    dC = torch.cat(dCs)
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    if eps == 0.0:
+        rE, rC, _ = gpu_backward(E, C, y, lse, dloss, 0.0)
+        assert rel_fro(dE.cpu().numpy(), rE.cpu().numpy()) < 1e-5
+        assert rel_fro(dC.cpu().numpy(), rC.cpu().numpy()) < 1e-5
+        oE, oC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
+        assert rel_fro(dE.cpu().numpy(), oE) <= GRAD_REL_FILTER_OFF
+        assert rel_fro(dC.cpu().numpy(), oC) <= GRAD_REL_FILTER_OFF
+    else:
+        # each shard's filter grid starts at its own first row; against the
+        # exact gradient the spec bar applies
+        xE, xC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
+        assert rel_fro(dE.cpu().numpy(), xE) <= GRAD_REL_FILTER_ON
+        assert rel_fro(dC.cpu().numpy(), xC) <= GRAD_REL_FILTER_ON
+
+
+def test_single_shard_helper_equals_unsharded_path():
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=600, V=9000)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, dE, dC = L.vocab_parallel_forward_backward(E, C, y, 0, w.V, filter_eps=0.0)
+    rl, rlse, _ = gpu_forward(E, C, y)
+    rE, rC, _ = gpu_backward(E, C, y, rlse, synth.mean_dloss(inp["y"]), 0.0)
+    assert np.abs(loss.cpu().numpy() - rl).max() <= 1e-5
+    assert rel_fro(dE.cpu().numpy(), rE.cpu().numpy()) < 1e-5
+    assert rel_fro(dC.cpu().numpy(), rC.cpu().numpy()) < 1e-5
+
+
+def test_merge_flags_labels_outside_the_full_vocabulary():
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.TINY.with_sizes(N=200, V=3000, D=64)
+    inp = synth.make_inputs(w)
+    inp["y"][5] = 3000
+    inp["y"][6] = IGN
+    E, C, y = to_dev(inp)
+    stats = torch.stack([L.forward_shard(E, C[:1500].contiguous(), y, 0), L.forward_shard(E, C[1500:].contiguous(), y, 1500)])
+    loss, lse = L.merge_shards(stats, y, w.V, IGN)
+    l = loss.cpu().numpy()
+    assert np.isnan(l[5]) and l[6] == 0.0 and np.isfinite(np.delete(l, 5)).all()
