@@ -35,7 +35,7 @@ METRIC = "CCE fwd+bwd tokens/s"
 UNIT = "tokens/s"
 IGN = -100
 BM, BN = 128, 256      # logit tile (token block x vocabulary tile)
-FT = 128               # the gradient filter's unit: 128 tokens x FT vocabulary entries
+FT = 64                # the gradient filter's unit: 128 tokens x FT vocabulary entries
 
 
 def log(*a):
@@ -406,7 +406,7 @@ def run_gpu(args, w):
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = measured_peaks()
-    unit_flop = 2.0 * BM * FT * D          # one 128 x 128 filter unit of logits
+    unit_flop = 2.0 * BM * FT * D          # one 128 x 64 filter unit of logits
     n_tiles = live + dead                  # filter units recomputed
     flop_fwd = 2.0 * N * D * V
     flop_bwd = n_tiles * unit_flop + live * 2.0 * unit_flop

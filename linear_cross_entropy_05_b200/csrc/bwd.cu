@@ -4,12 +4,13 @@
 // Cut Cross-Entropy abstract, sentences 4 and 9: the logits are never stored,
 // so the backward pass recomputes each 128 x 256 logit tile S = E_m C_v^T in
 // TMEM and forms P = exp(S - lse) and D = P - onehot(y) in registers.  The
-// filter works on 128 x 128 units (two per logit tile): a unit whose every
-// |D| is below filter_eps is dropped (gradient work under numerical
-// precision).  G = dloss * D goes to shared memory in bf16 and the live units
-// are contracted on the tensor cores:
-//     dE[m-block, d-chunk] += sum over live halves h of G_h . C_h[d-chunk]   (M=128, N=64, K=128 each)
-//     dC[v-half h, d-chunk] += G_h^T . E[m-block, d-chunk]                  (M=128, N=64, K=128)
+// filter works on 128 x 64 units (four per logit tile, one per 64-column
+// K block of G): a unit whose every |D| is below filter_eps is dropped
+// (gradient work under numerical precision).  G = dloss * D goes to shared
+// memory in bf16 and the live units are contracted on the tensor cores:
+//     dE[m-block, d-chunk] += sum over live quarters q of G_q . C_q[d-chunk]   (M=128, N=64, K=64 each)
+//     dC[v-half h, d-chunk] += G_h^T . E[m-block, d-chunk]  for halves with a live quarter (M=128, N=64, K=128)
+// and only the dC rows of live quarters are added to global memory.
 // The C and E slices are the same TMA tiles the recompute streams (128-byte
 // swizzled rows of 64 d values); read K-major for S and MN-major for the
 // contractions.  Partial products are added to fp32 dE/dC by the TMA engine
@@ -283,8 +284,8 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         if (!mbar_wait(g_full, gph, wc)) goto mma_done;
         gph ^= 1u;
         tc_fence_after();
-        const int hmask = live_ring[kt & 7];  // bit h: 128-column half h is live
-        if (hmask) {
+        const int qmask = live_ring[kt & 7];  // bit q: 64-column quarter q is live
+        if (qmask) {
           for (int kb = 0; kb < nkb; ++kb) {
             const int b = kb & 1;
             if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
@@ -295,16 +296,20 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
             const uint32_t c_addr = smem_u32(sB + stage * B_STAGE_BYTES);  // C[v-tile, d-chunk]: 256 voc x 64 d
             uint32_t acc_de = 0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (!((hmask >> h) & 1)) continue;
-              // dE chunk += G_h (128 tok x 128 voc, K-major) . C_h chunk (K = voc rows, MN = d)
+            for (int q = 0; q < 4; ++q) {
+              if (!((qmask >> q) & 1)) continue;
+              // dE chunk += G_q (128 tok x 64 voc, K-major) . C_q chunk (K = voc rows, MN = d)
 #pragma unroll
-              for (int k = 8 * h; k < 8 * h + 8; ++k) {
+              for (int k = 4 * q; k < 4 * q + 4; ++k) {
                 umma_bf16(tmem_base + tm_de(b),
                           sdesc_sw128(g_addr + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024),
                           sdesc_sw128(c_addr + k * 2048, 16384, 1024), IDESC_DE, acc_de);
                 acc_de = 1;
               }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (!((qmask >> (2 * h)) & 3)) continue;
               // dC chunk of half h = G_h^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
 #pragma unroll
               for (int k = 0; k < BM / 16; ++k)
@@ -386,10 +391,10 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       sph ^= 1u;
       if (!mbar_wait(g_empty, gph ^ 1u, wc)) break;
       tc_fence_after();
-      // bit h: some |D| >= eps in the 128-column half h (every existing half
-      // when the filter is off)
-      const uint32_t halves = ncols > 128 ? 3u : 1u;
-      uint32_t live = filter_on ? 0u : halves;
+      // bit q: some |D| >= eps in the 64-column quarter q (every existing
+      // quarter when the filter is off)
+      const uint32_t quarters = (1u << ((ncols + 63) >> 6)) - 1u;
+      uint32_t live = filter_on ? 0u : quarters;
       constexpr int NC = (BN / 32) / EPG;  // 32-column chunks of S handled by this warp
 #pragma unroll 1
       for (int c = hsel * NC; c < hsel * NC + NC; ++c) {
@@ -405,7 +410,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
             float p = ex2_approx(fmaf(x[j + q], LOG2E, -lse2));
             float d = (col == ycol) ? p - 1.f : p;
             d = (valid && col < ncols) ? d : 0.f;
-            live |= (filter_on && fabsf(d) >= eps ? 1u : 0u) << (c >> 2);
+            live |= (filter_on && fabsf(d) >= eps ? 1u : 0u) << (c >> 1);
             g2[q] = dl * d;
           }
           pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
@@ -429,10 +434,10 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       mbar_arrive(g_full);
       if (!mbar_wait(g_full, gph, wc)) break;
       gph ^= 1u;
-      const uint32_t hmask = (uint32_t)live_ring[kt & 7];
-      n_live += __popc(hmask);
-      n_dead += __popc(halves & ~hmask);
-      if (!hmask) continue;
+      const uint32_t qmask = (uint32_t)live_ring[kt & 7];
+      n_live += __popc(qmask);
+      n_dead += __popc(quarters & ~qmask);
+      if (!qmask) continue;
       bool ok = true;
       const int row0 = m * BM + lane_grp * 32;           // first dE row of this warp
       const uint32_t rows_valid = __ballot_sync(0xffffffffu, valid);  // kept tokens among those rows
@@ -464,11 +469,13 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         }
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          if (!((hmask >> h) & 1)) continue;
+          if (!((qmask >> (2 * h)) & 3u)) continue;
           const int vr0 = vt * BN + h * BM + lane_grp * 32;
+          // this warp's 32 vocabulary rows lie in quarter 2h + lane_grp/2
+          const bool rows_live = (qmask >> (2 * h + (lane_grp >> 1))) & 1u;
 #pragma unroll 1
           for (int q = 0; q < 2; ++q, ++piece) {
-            const bool mine = (piece % EPG) == hsel;
+            const bool mine = (piece % EPG) == hsel && rows_live;
             float v[32];
             if (mine) tmem_ld32(tmem_base + lane_addr + tm_dc(b) + h * 64 + q * 32, v);
             if (mine && d0 + q * 32 < a.D && vr0 < a.V) {

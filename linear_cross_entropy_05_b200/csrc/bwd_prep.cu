@@ -1,13 +1,13 @@
 // Backward pre-pass: the list of logit tiles the backward must recompute.
 //
 // The gradient filter (Cut Cross-Entropy abstract, sentence 9) drops a
-// 128 x 128 unit when every |P - onehot| < eps.  For a token i and a column v
+// 128 x 64 unit when every |P - onehot| < eps.  For a token i and a column v
 // that is not its label, P_iv = exp(E_i.C_v - lse_i) and, by Cauchy-Schwarz,
 // E_i.C_v <= |E_i| |C_v|.  So if |E_i| * max_v |C_v| < lse_i + ln(eps) for every
 // kept token of a 128-token block, every unit of that block that holds none
 // of its labels is dead, and its logits need not be recomputed at all.  Such
 // a block is "flat"; only the 128 x 256 logit tiles holding its labels are
-// visited (and their two units still tested exactly).  Blocks that are not
+// visited (and their four units still tested exactly).  Blocks that are not
 // flat are visited densely.  The visited set therefore covers every live
 // unit, and the gradients equal those of the dense recompute with the same
 // filter.
@@ -116,17 +116,20 @@ __global__ void __launch_bounds__(128) prep_blocks_kernel(const int64_t* __restr
 __global__ void __launch_bounds__(1024) prep_scan_kernel(PrepArgs p) {
   __shared__ unsigned warp_sums[32];
   __shared__ unsigned carry_s;
-  __shared__ unsigned long long halves_s;  // 128-column filter units inside the listed tiles
+  __shared__ unsigned long long units_s;  // 64-column filter units inside the listed tiles
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   if (t == 0) {
     carry_s = 0;
-    halves_s = 0;
+    units_s = 0;
   }
   __syncthreads();
   for (int base = 0; base < p.n_vtile; base += 1024) {
     const int i = base + t;
     const unsigned x = i < p.n_vtile ? p.count[i] : 0u;
-    if (x) atomicAdd(&halves_s, (unsigned long long)x * ((long long)i * BN + BN / 2 < p.V ? 2ull : 1ull));
+    if (x) {
+      const long long rem = (long long)p.V - (long long)i * BN;  // columns of tile i inside V
+      atomicAdd(&units_s, (unsigned long long)x * (unsigned long long)min(4ll, (rem + 63) / 64));
+    }
     unsigned incl = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -158,11 +161,10 @@ __global__ void __launch_bounds__(1024) prep_scan_kernel(PrepArgs p) {
     const unsigned long long T = (unsigned long long)L + (unsigned long long)nnf * (unsigned long long)p.n_vtile;
     p.hdr[HDR_L] = L;
     p.hdr[HDR_T] = (unsigned)T;
-    // pruned filter units (128 tokens x 128 vocabulary): all units minus
+    // pruned filter units (128 tokens x 64 vocabulary): all units minus
     // those inside the tiles that will be recomputed
-    const unsigned long long n_vhalf = ((unsigned long long)p.V + 127ull) / 128ull;
-    p.status[ST_PRUNED] =
-        (unsigned long long)p.n_mblk * n_vhalf - (halves_s + (unsigned long long)nnf * n_vhalf);
+    const unsigned long long n_vq = ((unsigned long long)p.V + 63ull) / 64ull;
+    p.status[ST_PRUNED] = (unsigned long long)p.n_mblk * n_vq - (units_s + (unsigned long long)nnf * n_vq);
   }
 }
 

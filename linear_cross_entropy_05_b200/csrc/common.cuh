@@ -27,7 +27,7 @@ constexpr float LN2 = 0.6931471805599453f;
 // Status block at the head of every workspace (8 x u64, zeroed per call).
 enum StatusWord : int {
   ST_FLAGS = 0,        // bit mask of StatusFlag
-  ST_LIVE_TILES = 1,   // backward: 128x128 filter units whose contraction ran
+  ST_LIVE_TILES = 1,   // backward: 128x64 filter units whose contraction ran
   ST_DEAD_TILES = 2,   // backward: filter units recomputed and found negligible
   ST_TILES = 3,        // forward: 128x256 logit tiles; backward: filter units tested
   ST_PRUNED = 4,       // backward: filter units proven negligible without recomputing them

@@ -20,7 +20,7 @@ plain definition):
 The backward recomputation and the gradient filter follow the abstract's
 sentence 9 (skip gradient work whose contribution is below numerical
 precision).  The filter is read at tile granularity: a (Bn x Bv) tile of G,
-anchored at (0, 0) (128 x 128 unless stated), is dropped iff every entry has
+anchored at (0, 0) (128 x 64 unless stated), is dropped iff every entry has
 |P - onehot| < eps; ignored rows and out-of-range rows/columns count as zero.
 eps <= 0 disables it.
 
@@ -160,7 +160,7 @@ def tile_live_map_f64(Dm_rows: np.ndarray, row0: int, Bn: int, Bv: int, eps: flo
 
 
 def backward_f64(E64, C64, y, lse, dloss, ignore_index: int, filter_eps: float = 0.0,
-                 tile=(128, 128), return_live: bool = False):
+                 tile=(128, 64), return_live: bool = False):
     """Full dE (N x D) and dC (V x D) in fp64 from the given per-token lse.
 
     With filter_eps > 0 the tiles of G that are not live (see module doc) are
@@ -191,7 +191,7 @@ def backward_f64(E64, C64, y, lse, dloss, ignore_index: int, filter_eps: float =
 
 
 def backward(E_bits, C_bits, y, lse, dloss, ignore_index: int, filter_eps: float = 0.0,
-             tile=(128, 128), return_live: bool = False):
+             tile=(128, 64), return_live: bool = False):
     """backward_f64 on bf16 bit-pattern inputs (lse from the oracle's forward)."""
     return backward_f64(bf16_bits_to_f64(E_bits), bf16_bits_to_f64(C_bits), y,
                         np.asarray(lse, dtype=np.float64), np.asarray(dloss), ignore_index,
@@ -200,7 +200,7 @@ def backward(E_bits, C_bits, y, lse, dloss, ignore_index: int, filter_eps: float
 
 def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
                      rows_dE: Sequence[int], rows_dC: Sequence[int],
-                     filter_eps: float = 0.0, tile=(128, 128)):
+                     filter_eps: float = 0.0, tile=(128, 64)):
     """Selected rows of dE and of dC without forming the full gradients.
 
     rows_dE: token rows i; dE[i] = sum_v G[i, v] C[v] needs only row i's lse.
@@ -285,7 +285,7 @@ def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
 
 
 def tile_live_map(E_bits, C_bits, y, lse, ignore_index: int, filter_eps: float,
-                  tile=(128, 128)):
+                  tile=(128, 64)):
     """Tile live map (N/Bn x V/Bv, ceil) for bf16 inputs and the given lse."""
     E64 = bf16_bits_to_f64(E_bits)
     C64 = bf16_bits_to_f64(C_bits)

@@ -13,7 +13,7 @@ from _gpu_helpers import (GRAD_REL_FILTER_OFF, GRAD_REL_FILTER_ON, IGN, gpu_back
 pytestmark = pytest.mark.gpu
 
 EPS = synth.EPS_BF16_FILTER
-TILE = (128, 128)   # the filter's unit: 128 tokens x 128 vocabulary entries
+TILE = (128, 64)    # the filter's unit: 128 tokens x 64 vocabulary entries
 
 CASES_OFF = [
     synth.TINY,
@@ -48,7 +48,7 @@ def _run(w, eps, dloss_seed=99):
 def test_backward_filter_off_matches_exact_gradient(w):
     inp, dloss, olse, gE, gC, st = _run(w, 0.0)
     assert st["status"] == 0 and st["flags"] == 0
-    n_tiles = -(-w.N // 128) * -(-w.V // 128)
+    n_tiles = -(-w.N // 128) * -(-w.V // 64)
     assert st["live_tiles"] == n_tiles and st["dead_tiles"] == 0 and st["pruned_tiles"] == 0
     rE, rC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
     if w.V == 1:  # one class: the gradient is exactly zero
@@ -85,7 +85,7 @@ def test_filter_threshold_edges():
     inp, dloss, olse, gE, gC, st = _run(w, 0.5)
     live_o = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, 0.5, TILE)
     assert st["live_tiles"] == int(live_o.sum())
-    yt = {(i // 128, int(inp["y"][i]) // 128) for i in range(w.N)}
+    yt = {(i // 128, int(inp["y"][i]) // 64) for i in range(w.N)}
     assert st["live_tiles"] == len(yt)
     inp, dloss, olse, gE, gC, st = _run(w, 2.0)
     assert st["live_tiles"] == 0 and (gE == 0).all() and (gC == 0).all()
@@ -109,8 +109,8 @@ def test_non_flat_blocks_are_recomputed_densely():
     _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
     fE, fC, live = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=TILE,
                                    return_live=True)
-    nvh = -(-w.V // 128)
-    label_tiles = {(i // 128, int(inp["y"][i]) // 128) for i in range(w.N)}
+    nvh = -(-w.V // 64)
+    label_tiles = {(i // 128, int(inp["y"][i]) // 64) for i in range(w.N)}
     assert int(live.sum()) > len(label_tiles)            # the peaky blocks have live non-label tiles
     assert st["live_tiles"] + st["dead_tiles"] >= 2 * nvh  # blocks 1 and 2 visited in full
     assert abs(st["live_tiles"] - int(live.sum())) <= 2
