@@ -24,7 +24,7 @@ cudaError_t launch_fwd_finalize(const void* E, const void* C, const int64_t* y, 
                                 float* lse, cudaStream_t stream);
 cudaError_t launch_merge_shards(const float* stats, int R, int N, const int64_t* y, long long V_total,
                                 long long ignore_index, float* loss, float* lse, cudaStream_t stream);
-cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
+cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmCq, const CUtensorMap& tmdE,
                        const CUtensorMap& tmdC, const BwdArgs& a, int grid, int variant, cudaStream_t stream);
 cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
                         int sms, cudaStream_t stream);
@@ -354,10 +354,11 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   if (workspace_bytes < bp.ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
-  CUtensorMap tmE, tmC, tmdE, tmdC;
+  CUtensorMap tmE, tmC, tmCq, tmdE, tmdC;
   // (in fixed-point mode the fp32 maps are built but the kernel reduces into
   // the int64 accumulators instead; dE/dC may then hold bf16)
-  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN) || !make_map_f32(&tmdE, dE, N, D) ||
+  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN) || !make_map(&tmCq, C, V, D, 64) ||
+      !make_map_f32(&tmdE, dE, N, D) ||
       !make_map_f32(&tmdC, dC, V, D))
     return CCE_ERR_CUDA;
   char* ws = reinterpret_cast<char*>(workspace);
@@ -428,7 +429,7 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   }
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
-  if (launch_bwd(tmE, tmC, tmdE, tmdC, a, grid, g_bwd_variant.load(), stream) != cudaSuccess) return CCE_ERR_CUDA;
+  if (launch_bwd(tmE, tmC, tmCq, tmdE, tmdC, a, grid, g_bwd_variant.load(), stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (fixed) {
     const unsigned* hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);

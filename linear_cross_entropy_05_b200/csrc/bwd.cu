@@ -142,6 +142,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <int NST, int NXB, int EPG>
 __global__ void __launch_bounds__(64 + 128 * EPG, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
+               const __grid_constant__ CUtensorMap tmCq,
                const __grid_constant__ CUtensorMap tmdE, const __grid_constant__ CUtensorMap tmdC, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
   if (threadIdx.x == 32) {
     tma_prefetch_map(&tmE);
     tma_prefetch_map(&tmC);
+    tma_prefetch_map(&tmCq);
     tma_prefetch_map(&tmdE);
     tma_prefetch_map(&tmdC);
   }
@@ -218,24 +220,40 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       for (int t = a.withhold_loads ? tm.T : blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
         int m, vt;
         tm.get(a, t, m, vt);
-        // logit recompute slices, then (if the tile is live) the same slices
-        // again as operands of the two contractions
-        for (int pass = 0; pass < 2; ++pass) {
-          if (pass == 1) {
-            if (!mbar_wait(g_full, gph, wc)) goto producer_done;
-            gph ^= 1u;
-            if (live_ring[kt & 7] == 0) break;
+        // logit recompute slices (d ascending); then, if the tile has a live
+        // quarter, the operands of the two contractions with d descending, so
+        // that the slices fetched last (most likely still in L2) come first:
+        // the E slice, and of the C slice only the 64-row quarters that are
+        // live (their dE products are the only ones that read C)
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
+          tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
+          armed |= 1u << stage;
+          if (++stage == NST) {
+            stage = 0;
+            phase ^= 1u;
           }
-          for (int kb = 0; kb < nkb; ++kb) {
-            if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
-            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-            tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
-            tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
-            armed |= 1u << stage;
-            if (++stage == NST) {
-              stage = 0;
-              phase ^= 1u;
-            }
+        }
+        if (!mbar_wait(g_full, gph, wc)) goto producer_done;
+        gph ^= 1u;
+        const int qmask = live_ring[kt & 7];
+        if (qmask == 0) continue;
+        const uint32_t bytes = A_STAGE_BYTES + (uint32_t)__popc(qmask) * QUARTER_BYTES;
+        for (int kb = nkb - 1; kb >= 0; --kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if ((qmask >> q) & 1)
+              tma_load_2d(sB + stage * B_STAGE_BYTES + q * QUARTER_BYTES, &tmCq, &full[stage], kb * BK,
+                          vt * BN + q * 64);
+          armed |= 1u << stage;
+          if (++stage == NST) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
       }
@@ -449,7 +467,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         }
         if (b) ++cfe1; else ++cfe0;
         tc_fence_after();
-        const int d0 = kb * BK;
+        const int d0 = (nkb - 1 - kb) * BK;  // the contraction pass runs d descending
         // Reduction pieces of this chunk (32 rows of this lane group x 32
         // columns each): dE q0, dE q1, then dC q0, q1 of every live half.
         // With EPG = 2 the pieces alternate between the two warps.
@@ -518,13 +536,13 @@ size_t bwd_smem_bytes() {
 }
 
 template <int NST, int NXB, int EPG>
-cudaError_t launch_bwd_t(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
+cudaError_t launch_bwd_t(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmCq, const CUtensorMap& tmdE,
                          const CUtensorMap& tmdC, const BwdArgs& a, int grid, cudaStream_t stream) {
   const size_t smem = bwd_smem_bytes<NST, NXB, EPG>();
   cudaError_t e =
       cudaFuncSetAttribute(bwd_kernel<NST, NXB, EPG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  bwd_kernel<NST, NXB, EPG><<<grid, 64 + 128 * EPG, smem, stream>>>(tmE, tmC, tmdE, tmdC, a);
+  bwd_kernel<NST, NXB, EPG><<<grid, 64 + 128 * EPG, smem, stream>>>(tmE, tmC, tmCq, tmdE, tmdC, a);
   return cudaGetLastError();
 }
 
@@ -532,11 +550,11 @@ cudaError_t launch_bwd_t(const CUtensorMap& tmE, const CUtensorMap& tmC, const C
 // variant 1: 2 stages, two staging buffers per warp (staging overlaps the bulk
 //            read of the previous block);
 // variant 2: 2 stages, 8 epilogue warps (two per TMEM lane group).
-cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmdE,
+cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmCq, const CUtensorMap& tmdE,
                        const CUtensorMap& tmdC, const BwdArgs& a, int grid, int variant, cudaStream_t stream) {
-  if (variant == 1) return launch_bwd_t<2, 2, 1>(tmE, tmC, tmdE, tmdC, a, grid, stream);
-  if (variant == 2) return launch_bwd_t<2, 1, 2>(tmE, tmC, tmdE, tmdC, a, grid, stream);
-  return launch_bwd_t<BWD_STAGES, 1, 1>(tmE, tmC, tmdE, tmdC, a, grid, stream);
+  if (variant == 1) return launch_bwd_t<2, 2, 1>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
+  if (variant == 2) return launch_bwd_t<2, 1, 2>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
+  return launch_bwd_t<BWD_STAGES, 1, 1>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
 }
 
 }  // namespace cce

@@ -14,6 +14,7 @@ constexpr int BK = 64;
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // E slice  [128 rows][64 d]
 constexpr int B_STAGE_BYTES = BN * BK * 2;  // C slice  [256 rows][64 d]
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int QUARTER_BYTES = 64 * BK * 2;   // C slice [64 rows][64 d]: one filter unit's rows
 constexpr int NUM_THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int FWD_STAGES = 4;
 constexpr int PAIR_STAGES = 6;                          // CTA-pair forward: E half + C half per stage
