@@ -35,7 +35,7 @@ METRIC = "CCE fwd+bwd tokens/s"
 UNIT = "tokens/s"
 IGN = -100
 BM, BN = 128, 256      # logit tile (token block x vocabulary tile)
-FT = 64                # the gradient filter's unit: 128 tokens x FT vocabulary entries
+FU = (32, 32)          # the gradient filter's unit: 32 tokens x 32 vocabulary entries
 
 
 def log(*a):
@@ -199,7 +199,7 @@ def oracle_step(inp, rows, eps):
     y = inp["y"][rows]
     loss, lse = oracle.forward_f64(E64, C64, y, IGN)
     dl = np.full(len(rows), 1.0 / max(1, len(rows)))
-    dE, dC = oracle.backward_f64(E64, C64, y, lse, dl, IGN, filter_eps=eps, tile=(BM, FT))
+    dE, dC = oracle.backward_f64(E64, C64, y, lse, dl, IGN, filter_eps=eps, tile=FU)
     return loss
 
 
@@ -305,6 +305,7 @@ def run_gpu(args, w):
     if stf["status"] != 0 or stb["status"] != 0:
         raise RuntimeError(f"device status not clean: fwd {stf} bwd {stb}")
     live, dead, pruned = stb["live_tiles"], stb["dead_tiles"], stb["pruned_tiles"]
+    recomputed = stb["logit_tiles"]     # 128 x 256 logit tiles the backward recomputed
 
     # extra global memory of one step: the library allocates nothing itself
     torch.cuda.synchronize()
@@ -406,10 +407,10 @@ def run_gpu(args, w):
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = measured_peaks()
-    unit_flop = 2.0 * BM * FT * D          # one 128 x 64 filter unit of logits
-    n_tiles = live + dead                  # filter units recomputed
+    unit_flop = 2.0 * FU[0] * FU[1] * D    # one filter unit's products, per contraction
     flop_fwd = 2.0 * N * D * V
-    flop_bwd = n_tiles * unit_flop + live * 2.0 * unit_flop
+    # recompute of the visited logit tiles + the dE and dC products of the live units
+    flop_bwd = recomputed * 2.0 * BM * BN * D + live * 2.0 * unit_flop
     dominant = "bwd_kernel" if bwd_ms >= fwd_ms else "fwd_lse_kernel"
     dom_flop, dom_ms = (flop_bwd, bwd_ms) if dominant == "bwd_kernel" else (flop_fwd, fwd_ms)
     peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
@@ -436,10 +437,12 @@ def run_gpu(args, w):
                          "flop_per_launch": dom_flop, "launch_ms": dom_ms},
             "kernels": {"fwd_lse_kernel": {"ms": fwd_ms, "tflops": flop_fwd / fwd_ms / 1e9},
                         "bwd_kernel": {"ms": bwd_ms, "tflops": flop_bwd / bwd_ms / 1e9,
-                                       "live_tiles": live, "dead_tiles": dead, "pruned_tiles": pruned}},
+                                       "live_units": live, "dead_units": dead, "pruned_units": pruned,
+                                       "logit_tiles_recomputed": recomputed}},
             "pct_bf16_peak_executed": executed_flop / (step_ms * 1e-3) / 1e12 / peak,
             "pct_bf16_peak_nominal_6NDV": nominal_flop / (step_ms * 1e-3) / 1e12 / peak,
-            "live_tile_frac": live / max(1, n_tiles + pruned),
+            "filter_unit": list(FU),
+            "live_unit_frac": live / max(1, live + dead + pruned),
             "extra_hbm_bytes": int(extra_hbm),
             "materialised_logits_fp32_bytes": N * V * 4,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
@@ -495,16 +498,15 @@ def run_suite(args):
             torch.cuda.synchronize()
             tf += ev[0].elapsed_time(ev[1]) / reps
             tb += ev[1].elapsed_time(ev[2]) / reps
-        unit = 2.0 * BM * FT * D
-        visited = st["live_tiles"] + st["dead_tiles"]
-        executed = 2.0 * N * D * V + visited * unit + st["live_tiles"] * 2.0 * unit
+        unit = 2.0 * FU[0] * FU[1] * D
+        executed = 2.0 * N * D * V + st["logit_tiles"] * 2.0 * BM * BN * D + st["live_tiles"] * 2.0 * unit
         print(json.dumps({
             "workload": w.name, "N": N, "D": D, "V": V, "filter_eps": w.filter_eps,
             "fwd_ms": tf, "fwd_tokens_per_s": N / tf * 1e3, "fwd_frac_of_peak": 2.0 * N * D * V / tf / 1e9 / peak,
             "fwd_bwd_ms": tf + tb, "fwd_bwd_tokens_per_s": N / (tf + tb) * 1e3,
             "executed_frac_of_peak": executed / (tf + tb) / 1e9 / peak,
             "nominal_6NDV_frac_of_peak": 6.0 * N * D * V / (tf + tb) / 1e9 / peak,
-            "tiles": {k: st[k] for k in ("live_tiles", "dead_tiles", "pruned_tiles")},
+            "tiles": {k: st[k] for k in ("live_tiles", "dead_tiles", "pruned_tiles", "logit_tiles")},
             "extra_hbm_bytes": {"forward_workspace": wsf.buf.numel(), "backward_workspace": wsb.buf.numel()},
             "materialised_logits_fp32_bytes": N * V * 4, "peak_tflops": peak}), flush=True)
         del E, C, y, dl, dE, dC, loss, lse, wsf, wsb

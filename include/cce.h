@@ -9,9 +9,10 @@
  *   gradients of sum_i dloss[i] * loss[i]:
  *     G[i,v] = dloss[i] * (softmax(E_i C^T)[v] - [v == y_i]),
  *     dE = G C,  dC = G^T E,
- *   where the 128x128 gradient tiles whose every |softmax - onehot| entry is
- *   below filter_eps are skipped (the abstract's sentence 9: gradient work
- *   below numerical precision is dropped).
+ *   where the 32x32 gradient units (32 tokens x 32 vocabulary entries) whose
+ *   every |softmax - onehot| entry is below filter_eps are skipped (the
+ *   abstract's sentence 9: gradient work below numerical precision is
+ *   dropped).
  *
  * Conventions for every entry point:
  *   - All matrix arguments are DEVICE pointers to row-major, contiguous data.
@@ -61,12 +62,13 @@ typedef enum {
 /* Status block decoded by cce_read_status. */
 typedef struct {
   uint64_t flags;       /* bit 0: a wait timed out; bit 1: an invalid label was seen */
-  uint64_t live_tiles;  /* backward: 128x128 filter tiles whose contractions ran */
-  uint64_t dead_tiles;  /* backward: filter tiles recomputed and found negligible */
+  uint64_t live_tiles;  /* backward: 32x32 filter units whose contributions were added */
+  uint64_t dead_tiles;  /* backward: filter units recomputed and found negligible */
   uint64_t logit_tiles; /* forward: 128x256 logit tiles computed on chip;
-                           backward: filter tiles tested (live + dead) */
-  uint64_t pruned_tiles;/* backward: filter tiles proven negligible without
-                           recomputing them */
+                           backward: 128x256 logit tiles recomputed on chip */
+  uint64_t pruned_tiles;/* backward: filter units proven negligible without
+                           recomputing them; live + dead + pruned =
+                           ceil(N/32) * ceil(V/32) when filter_eps > 0 */
 } cce_counters_t;
 
 /* Workspace bytes needed by cce_forward for these sizes on the current device
@@ -97,14 +99,14 @@ CCE_API cce_status_t cce_forward(const void* E, const void* C, const int64_t* y,
 /* Backward pass (abstract, sentences 4 and 9): gradients of sum_i dloss[i] * loss[i].
  *   lse   [N] fp32   from cce_forward on the same E, C
  *   dloss [N] fp32   upstream gradient per token (e.g. 1/#kept for a mean)
- *   filter_eps       a 128x128 tile (128 tokens x 128 vocabulary entries,
+ *   filter_eps       a 32x32 unit (32 tokens x 32 vocabulary entries,
  *                    anchored at 0) of (softmax - onehot) whose entries are
  *                    all below filter_eps in magnitude is skipped; <= 0 keeps
- *                    every tile (exact gradient)
+ *                    every unit (exact gradient)
  *   dE    [N x D] fp32 out (overwritten), dC [V x D] fp32 out (overwritten)
  * The logit tiles are recomputed on chip; rows with y == ignore_index
  * contribute nothing.  With filter_eps > 0 a pre-pass bounds every logit by
- * |E_i| max_v |C_v| (Cauchy-Schwarz): tiles that bound proves negligible and
+ * |E_i| max_v |C_v| (Cauchy-Schwarz): units that bound proves negligible and
  * that hold no label are not recomputed (counted as pruned); the result is
  * the same as recomputing and testing them.  Accumulation order across tiles
  * is not fixed (fp32 atomics), so results may differ in the last bits between

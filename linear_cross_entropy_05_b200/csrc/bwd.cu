@@ -4,13 +4,15 @@
 // Cut Cross-Entropy abstract, sentences 4 and 9: the logits are never stored,
 // so the backward pass recomputes each 128 x 256 logit tile S = E_m C_v^T in
 // TMEM and forms P = exp(S - lse) and D = P - onehot(y) in registers.  The
-// filter works on 128 x 64 units (four per logit tile, one per 64-column
-// K block of G): a unit whose every |D| is below filter_eps is dropped
-// (gradient work under numerical precision).  G = dloss * D goes to shared
-// memory in bf16 and the live units are contracted on the tensor cores:
-//     dE[m-block, d-chunk] += sum over live quarters q of G_q . C_q[d-chunk]   (M=128, N=64, K=64 each)
-//     dC[v-half h, d-chunk] += G_h^T . E[m-block, d-chunk]  for halves with a live quarter (M=128, N=64, K=128)
-// and only the dC rows of live quarters are added to global memory.
+// filter works on 32 x 32 units (32 tokens x 32 vocabulary entries, 32 per
+// logit tile: one epilogue warp's rows x one 32-column chunk): a unit whose
+// every |D| is below filter_eps is dropped (gradient work under numerical
+// precision) by writing its part of G = dloss * D to shared memory as zeros.
+// The tensor cores then contract whole blocks that hold a live unit:
+//     dE[m-block, d-chunk] += sum over live 64-column quarters q of G_q . C_q[d-chunk]   (M=128, N=64, K=64 each)
+//     dC[v-half h, d-chunk] += G_h^T . E[m-block, d-chunk]  for halves with a live unit  (M=128, N=64, K=128)
+// and only the 32-row pieces of dE and dC that a live unit touches are added
+// to global memory (the others are exactly zero).
 // The C and E slices are the same TMA tiles the recompute streams (128-byte
 // swizzled rows of 64 d values); read K-major for S and MN-major for the
 // contractions.  Partial products are added to fp32 dE/dC by the TMA engine
@@ -35,6 +37,13 @@ namespace {
 constexpr uint32_t TM_S = 0;
 __device__ __forceinline__ uint32_t tm_de(int b) { return b ? 0u : 256u; }   // dE chunk of buffer b
 __device__ __forceinline__ uint32_t tm_dc(int b) { return b ? 64u : 320u; }   // dC chunk of buffer b
+
+// Live mask of a logit tile: bit 8 * g + c is the 32 x 32 filter unit of
+// token rows [32g, 32g + 32) and columns [32c, 32c + 32).
+__device__ __forceinline__ bool quarter_live(uint32_t u, int q) { return (u & (0x03030303u << (2 * q))) != 0; }
+__device__ __forceinline__ bool half_live(uint32_t u, int h) { return (u & (0x0F0F0F0Fu << (4 * h))) != 0; }
+__device__ __forceinline__ bool chunk_live(uint32_t u, int c) { return (u & (0x01010101u << c)) != 0; }
+__device__ __forceinline__ bool rows_live(uint32_t u, int g) { return ((u >> (8 * g)) & 0xFFu) != 0; }
 
 __device__ __forceinline__ void tile_coords(int t, int n_mblk, int n_vtile, int group_m, int& m, int& vt) {
   // Raster: groups of group_m token blocks; inside a group the token block
@@ -238,8 +247,11 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         }
         if (!mbar_wait(g_full, gph, wc)) goto producer_done;
         gph ^= 1u;
-        const int qmask = live_ring[kt & 7];
-        if (qmask == 0) continue;
+        const uint32_t umask = (uint32_t)live_ring[kt & 7];
+        if (umask == 0) continue;
+        uint32_t qmask = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) qmask |= (quarter_live(umask, q) ? 1u : 0u) << q;
         const uint32_t bytes = A_STAGE_BYTES + (uint32_t)__popc(qmask) * QUARTER_BYTES;
         for (int kb = nkb - 1; kb >= 0; --kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
@@ -302,8 +314,8 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         if (!mbar_wait(g_full, gph, wc)) goto mma_done;
         gph ^= 1u;
         tc_fence_after();
-        const int qmask = live_ring[kt & 7];  // bit q: 64-column quarter q is live
-        if (qmask) {
+        const uint32_t umask = (uint32_t)live_ring[kt & 7];  // live 32 x 32 units of the tile
+        if (umask) {
           for (int kb = 0; kb < nkb; ++kb) {
             const int b = kb & 1;
             if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
@@ -315,7 +327,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
             uint32_t acc_de = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              if (!((qmask >> q) & 1)) continue;
+              if (!quarter_live(umask, q)) continue;
               // dE chunk += G_q (128 tok x 64 voc, K-major) . C_q chunk (K = voc rows, MN = d)
 #pragma unroll
               for (int k = 4 * q; k < 4 * q + 4; ++k) {
@@ -327,7 +339,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              if (!((qmask >> (2 * h)) & 3)) continue;
+              if (!half_live(umask, h)) continue;
               // dC chunk of half h = G_h^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
 #pragma unroll
               for (int k = 0; k < BM / 16; ++k)
@@ -366,7 +378,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
     const bool filter_on = eps > 0.f;
     uint32_t sph = 0, gph = 0;
     uint32_t cfe0 = 0u, cfe1 = 0u;  // drains of contraction buffers 0 / 1 so far
-    unsigned long long n_live = 0, n_dead = 0;
+    unsigned long long n_live = 0, n_dead = 0, n_tiles = 0;
     uint8_t* g_row = sG + rib * 128;
     uint8_t* const xb0 = sX + ew * NXB * 4096;
     int xbi = 0;  // next staging buffer of this warp (rotation over NXB)
@@ -409,16 +421,20 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       sph ^= 1u;
       if (!mbar_wait(g_empty, gph ^ 1u, wc)) break;
       tc_fence_after();
-      // bit q: some |D| >= eps in the 64-column quarter q (every existing
-      // quarter when the filter is off)
-      const uint32_t quarters = (1u << ((ncols + 63) >> 6)) - 1u;
-      uint32_t live = filter_on ? 0u : quarters;
+      // This warp's units: its 32 rows (if any of them is a token) x each
+      // 32-column chunk inside V.  A unit is live if some |D| >= eps in it
+      // (every existing unit when the filter is off).
+      const int n_groups = min(4, (a.N - m * BM + 31) >> 5);  // token row groups of this block
+      const int n_chunks = (ncols + 31) >> 5;
+      const uint32_t my_chunks = lane_grp < n_groups ? (1u << n_chunks) - 1u : 0u;
+      uint32_t live = 0;
       constexpr int NC = (BN / 32) / EPG;  // 32-column chunks of S handled by this warp
 #pragma unroll 1
       for (int c = hsel * NC; c < hsel * NC + NC; ++c) {
         float x[32];
         tmem_ld32(tmem_base + lane_addr + TM_S + c * 32, x);
         uint32_t pk[16];
+        bool big = false;  // some |D| >= eps in this lane's 32 entries
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           float g2[2];
@@ -428,11 +444,17 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
             float p = ex2_approx(fmaf(x[j + q], LOG2E, -lse2));
             float d = (col == ycol) ? p - 1.f : p;
             d = (valid && col < ncols) ? d : 0.f;
-            live |= (filter_on && fabsf(d) >= eps ? 1u : 0u) << (c >> 1);
+            big |= fabsf(d) >= eps;
             g2[q] = dl * d;
           }
           pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
         }
+        const bool unit_live = filter_on ? __any_sync(0xffffffffu, big) : ((my_chunks >> c) & 1u) != 0;
+        if (!unit_live) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;  // a dropped unit contributes nothing
+        }
+        live |= (unit_live ? 1u : 0u) << (8 * lane_grp + c);
         // 32 columns = 64 bytes = four 16-byte chunks of the 128-byte row of
         // K block (c / 2); 128B swizzle: chunk index ^= row % 8.
         uint8_t* blk = g_row + (c >> 1) * (BM * 128);
@@ -445,17 +467,18 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       tc_fence_before();
       mbar_arrive(s_empty);
       fence_proxy_async_smem();
-      const uint32_t wmask = __reduce_or_sync(0xffffffffu, live);
-      if (wmask && lane == 0) atomicOr(const_cast<int*>(&live_ring[kt & 7]), (int)wmask);
+      if (live && lane == 0) atomicOr(const_cast<int*>(&live_ring[kt & 7]), (int)live);
       __syncwarp();
       if (rib == 0) live_ring[(kt + 4) & 7] = 0;
       mbar_arrive(g_full);
       if (!mbar_wait(g_full, gph, wc)) break;
       gph ^= 1u;
-      const uint32_t qmask = (uint32_t)live_ring[kt & 7];
-      n_live += __popc(qmask);
-      n_dead += __popc(quarters & ~qmask);
-      if (!qmask) continue;
+      const uint32_t umask = (uint32_t)live_ring[kt & 7];
+      n_live += __popc(umask);
+      n_dead += (unsigned)(n_groups * n_chunks) - __popc(umask);
+      ++n_tiles;
+      if (!umask) continue;
+      const bool de_rows_live = rows_live(umask, lane_grp);  // this warp's 32 token rows
       bool ok = true;
       const int row0 = m * BM + lane_grp * 32;           // first dE row of this warp
       const uint32_t rows_valid = __ballot_sync(0xffffffffu, valid);  // kept tokens among those rows
@@ -474,7 +497,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         int piece = 0;
 #pragma unroll 1
         for (int q = 0; q < 2; ++q, ++piece) {
-          const bool mine = (piece % EPG) == hsel;
+          const bool mine = (piece % EPG) == hsel && de_rows_live;
           float v[32];
           if (mine) tmem_ld32(tmem_base + lane_addr + tm_de(b) + q * 32, v);
           if (mine && d0 + q * 32 < a.D && row0 < a.N) {
@@ -487,13 +510,13 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         }
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          if (!((qmask >> (2 * h)) & 3u)) continue;
+          if (!half_live(umask, h)) continue;
           const int vr0 = vt * BN + h * BM + lane_grp * 32;
-          // this warp's 32 vocabulary rows lie in quarter 2h + lane_grp/2
-          const bool rows_live = (qmask >> (2 * h + (lane_grp >> 1))) & 1u;
+          // this warp's 32 vocabulary rows are column chunk 4h + lane_grp
+          const bool dc_rows_live = chunk_live(umask, 4 * h + lane_grp);
 #pragma unroll 1
           for (int q = 0; q < 2; ++q, ++piece) {
-            const bool mine = (piece % EPG) == hsel && rows_live;
+            const bool mine = (piece % EPG) == hsel && dc_rows_live;
             float v[32];
             if (mine) tmem_ld32(tmem_base + lane_addr + tm_dc(b) + h * 64 + q * 32, v);
             if (mine && d0 + q * 32 < a.D && vr0 < a.V) {
@@ -515,7 +538,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
     if (rib == 0 && hsel == 0) {
       atomicAdd(a.status + ST_LIVE_TILES, n_live);
       atomicAdd(a.status + ST_DEAD_TILES, n_dead);
-      atomicAdd(a.status + ST_TILES, n_live + n_dead);
+      atomicAdd(a.status + ST_TILES, n_tiles);
     }
   }
 

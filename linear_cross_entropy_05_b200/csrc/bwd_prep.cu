@@ -1,13 +1,13 @@
 // Backward pre-pass: the list of logit tiles the backward must recompute.
 //
 // The gradient filter (Cut Cross-Entropy abstract, sentence 9) drops a
-// 128 x 64 unit when every |P - onehot| < eps.  For a token i and a column v
+// 32 x 32 unit when every |P - onehot| < eps.  For a token i and a column v
 // that is not its label, P_iv = exp(E_i.C_v - lse_i) and, by Cauchy-Schwarz,
 // E_i.C_v <= |E_i| |C_v|.  So if |E_i| * max_v |C_v| < lse_i + ln(eps) for every
 // kept token of a 128-token block, every unit of that block that holds none
 // of its labels is dead, and its logits need not be recomputed at all.  Such
 // a block is "flat"; only the 128 x 256 logit tiles holding its labels are
-// visited (and their four units still tested exactly).  Blocks that are not
+// visited (and their units still tested exactly).  Blocks that are not
 // flat are visited densely.  The visited set therefore covers every live
 // unit, and the gradients equal those of the dense recompute with the same
 // filter.
@@ -52,6 +52,19 @@ __device__ __forceinline__ float warp_row_norm(const __nv_bfloat16* row, int D, 
 
 __device__ __forceinline__ bool label_ok(long long t, long long ignore_index, int V) {
   return t != ignore_index && t >= 0 && t < V;
+}
+
+// Filter units (32 tokens x 32 vocabulary entries) inside token block m and
+// inside vocabulary tile v, and the pruned-unit counter's update: it starts
+// at the number of all units and loses those of every recomputed tile.
+__device__ __forceinline__ unsigned long long unit_rows(const PrepArgs& p, int m) {
+  return (unsigned long long)min(BM / 32, (p.N - m * BM + 31) / 32);
+}
+__device__ __forceinline__ unsigned long long unit_cols(const PrepArgs& p, int v) {
+  return (unsigned long long)min(BN / 32, (p.V - v * BN + 31) / 32);
+}
+__device__ __forceinline__ void pruned_sub(const PrepArgs& p, unsigned long long units) {
+  atomicAdd(p.status + ST_PRUNED, 0ull - units);  // modulo 2^64: order of the updates is free
 }
 
 }  // namespace
@@ -102,7 +115,10 @@ __global__ void __launch_bounds__(128) prep_blocks_kernel(const int64_t* __restr
   const int all_flat = __syncthreads_and(flat);
   if (t == 0) p.blk_flat[m] = all_flat;
   if (!all_flat) {
-    if (t == 0) p.nonflat[atomicAdd(p.hdr + HDR_NNF, 1u)] = m;
+    if (t == 0) {
+      p.nonflat[atomicAdd(p.hdr + HDR_NNF, 1u)] = m;
+      pruned_sub(p, unit_rows(p, m) * (((unsigned long long)p.V + 31ull) / 32ull));  // visited densely
+    }
     return;
   }
   tl[t] = has_col ? (int)(ylocal / BN) : -1;
@@ -116,20 +132,14 @@ __global__ void __launch_bounds__(128) prep_blocks_kernel(const int64_t* __restr
 __global__ void __launch_bounds__(1024) prep_scan_kernel(PrepArgs p) {
   __shared__ unsigned warp_sums[32];
   __shared__ unsigned carry_s;
-  __shared__ unsigned long long units_s;  // 64-column filter units inside the listed tiles
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   if (t == 0) {
     carry_s = 0;
-    units_s = 0;
   }
   __syncthreads();
   for (int base = 0; base < p.n_vtile; base += 1024) {
     const int i = base + t;
     const unsigned x = i < p.n_vtile ? p.count[i] : 0u;
-    if (x) {
-      const long long rem = (long long)p.V - (long long)i * BN;  // columns of tile i inside V
-      atomicAdd(&units_s, (unsigned long long)x * (unsigned long long)min(4ll, (rem + 63) / 64));
-    }
     unsigned incl = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -161,10 +171,10 @@ __global__ void __launch_bounds__(1024) prep_scan_kernel(PrepArgs p) {
     const unsigned long long T = (unsigned long long)L + (unsigned long long)nnf * (unsigned long long)p.n_vtile;
     p.hdr[HDR_L] = L;
     p.hdr[HDR_T] = (unsigned)T;
-    // pruned filter units (128 tokens x 64 vocabulary): all units minus
-    // those inside the tiles that will be recomputed
-    const unsigned long long n_vq = ((unsigned long long)p.V + 63ull) / 64ull;
-    p.status[ST_PRUNED] = (unsigned long long)p.n_mblk * n_vq - (units_s + (unsigned long long)nnf * n_vq);
+    // all filter units; the recomputed tiles' units are taken off by
+    // prep_blocks (dense blocks) and prep_scatter (listed tiles)
+    atomicAdd(p.status + ST_PRUNED,
+              (((unsigned long long)p.N + 31ull) / 32ull) * (((unsigned long long)p.V + 31ull) / 32ull));
   }
 }
 
@@ -186,6 +196,7 @@ __global__ void __launch_bounds__(128) prep_scatter_kernel(const int64_t* __rest
     const int v = tl[t];
     const unsigned slot = atomicAdd(p.cursor + v, 1u);
     p.list[p.offset[v] + slot] = make_int2(m, v);
+    pruned_sub(p, unit_rows(p, m) * unit_cols(p, v));
   }
 }
 

@@ -14,7 +14,7 @@ constexpr int BK = 64;
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // E slice  [128 rows][64 d]
 constexpr int B_STAGE_BYTES = BN * BK * 2;  // C slice  [256 rows][64 d]
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-constexpr int QUARTER_BYTES = 64 * BK * 2;   // C slice [64 rows][64 d]: one filter unit's rows
+constexpr int QUARTER_BYTES = 64 * BK * 2;   // C slice [64 rows][64 d]: one K block of the dE product
 constexpr int NUM_THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int FWD_STAGES = 4;
 constexpr int PAIR_STAGES = 6;                          // CTA-pair forward: E half + C half per stage
@@ -28,9 +28,9 @@ constexpr float LN2 = 0.6931471805599453f;
 // Status block at the head of every workspace (8 x u64, zeroed per call).
 enum StatusWord : int {
   ST_FLAGS = 0,        // bit mask of StatusFlag
-  ST_LIVE_TILES = 1,   // backward: 128x64 filter units whose contraction ran
+  ST_LIVE_TILES = 1,   // backward: 32x32 filter units whose contraction ran
   ST_DEAD_TILES = 2,   // backward: filter units recomputed and found negligible
-  ST_TILES = 3,        // forward: 128x256 logit tiles; backward: filter units tested
+  ST_TILES = 3,        // forward: 128x256 logit tiles computed; backward: logit tiles recomputed
   ST_PRUNED = 4,       // backward: filter units proven negligible without recomputing them
 };
 // Header words of the backward pre-pass (u32, after the status block).

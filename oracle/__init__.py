@@ -20,7 +20,7 @@ plain definition):
 The backward recomputation and the gradient filter follow the abstract's
 sentence 9 (skip gradient work whose contribution is below numerical
 precision).  The filter is read at tile granularity: a (Bn x Bv) tile of G,
-anchored at (0, 0) (128 x 64 unless stated), is dropped iff every entry has
+anchored at (0, 0) (32 x 32 unless stated), is dropped iff every entry has
 |P - onehot| < eps; ignored rows and out-of-range rows/columns count as zero.
 eps <= 0 disables it.
 
@@ -151,16 +151,15 @@ def tile_live_map_f64(Dm_rows: np.ndarray, row0: int, Bn: int, Bv: int, eps: flo
     nr, V = Dm_rows.shape
     nt_r = -(-nr // Bn)
     nt_v = -(-V // Bv)
-    live = np.zeros((nt_r, nt_v), dtype=bool)
-    A = np.abs(Dm_rows)
-    for a in range(nt_r):
-        for b in range(nt_v):
-            live[a, b] = bool((A[a * Bn:(a + 1) * Bn, b * Bv:(b + 1) * Bv] >= eps).any())
-    return live
+    # pad with zeros (out-of-range rows/columns count as zero) and ask, per
+    # (Bn x Bv) block, whether any entry reaches eps
+    big = np.zeros((nt_r * Bn, nt_v * Bv), dtype=bool)
+    big[:nr, :V] = np.abs(Dm_rows) >= eps
+    return big.reshape(nt_r, Bn, nt_v, Bv).any(axis=(1, 3))
 
 
 def backward_f64(E64, C64, y, lse, dloss, ignore_index: int, filter_eps: float = 0.0,
-                 tile=(128, 64), return_live: bool = False):
+                 tile=(32, 32), return_live: bool = False):
     """Full dE (N x D) and dC (V x D) in fp64 from the given per-token lse.
 
     With filter_eps > 0 the tiles of G that are not live (see module doc) are
@@ -191,7 +190,7 @@ def backward_f64(E64, C64, y, lse, dloss, ignore_index: int, filter_eps: float =
 
 
 def backward(E_bits, C_bits, y, lse, dloss, ignore_index: int, filter_eps: float = 0.0,
-             tile=(128, 64), return_live: bool = False):
+             tile=(32, 32), return_live: bool = False):
     """backward_f64 on bf16 bit-pattern inputs (lse from the oracle's forward)."""
     return backward_f64(bf16_bits_to_f64(E_bits), bf16_bits_to_f64(C_bits), y,
                         np.asarray(lse, dtype=np.float64), np.asarray(dloss), ignore_index,
@@ -200,7 +199,7 @@ def backward(E_bits, C_bits, y, lse, dloss, ignore_index: int, filter_eps: float
 
 def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
                      rows_dE: Sequence[int], rows_dC: Sequence[int],
-                     filter_eps: float = 0.0, tile=(128, 64)):
+                     filter_eps: float = 0.0, tile=(32, 32)):
     """Selected rows of dE and of dC without forming the full gradients.
 
     rows_dE: token rows i; dE[i] = sum_v G[i, v] C[v] needs only row i's lse.
@@ -285,7 +284,7 @@ def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
 
 
 def tile_live_map(E_bits, C_bits, y, lse, ignore_index: int, filter_eps: float,
-                  tile=(128, 64)):
+                  tile=(32, 32)):
     """Tile live map (N/Bn x V/Bv, ceil) for bf16 inputs and the given lse."""
     E64 = bf16_bits_to_f64(E_bits)
     C64 = bf16_bits_to_f64(C_bits)

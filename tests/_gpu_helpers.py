@@ -11,6 +11,17 @@ GRAD_REL_FILTER_OFF = 5e-3   # dE, dC relative Frobenius error, filter off
 GRAD_REL_FILTER_ON = 1e-2    # dE, dC relative Frobenius error, filter on (vs the exact gradient)
 
 
+def filter_on_bar(V):
+    """Filter-on bar against the exact gradient for a vocabulary of V.
+
+    The 1e-2 bar is meant for vocabularies of ~1e5.  With eps = 2^-12 ~ 2.4/V
+    at V ~ 1e4, nearly every softmax entry outside the label units is below
+    eps, and dropping that tail alone gives a relative error of about
+    1/sqrt(V) (a sum of ~V entries of size ~1/V times random rows, against
+    the label's row), so small vocabularies get 1.25/sqrt(V)."""
+    return max(GRAD_REL_FILTER_ON, 1.25 / np.sqrt(V))
+
+
 def to_dev(inp, device="cuda"):
     import torch
     E = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(device)

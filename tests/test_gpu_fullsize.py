@@ -38,7 +38,7 @@ def test_full_size_forward_backward_sampled(w):
     dloss = synth.mean_dloss(inp["y"])
     dE, dC, st = gpu_backward(E, C, y, lse, dloss, w.filter_eps)
     assert st["status"] == 0 and st["flags"] == 0
-    n_tiles = -(-w.N // 128) * -(-w.V // 64)   # 128 x 64 filter units
+    n_tiles = -(-w.N // 32) * -(-w.V // 32)   # 32 x 32 filter units
     assert st["live_tiles"] + st["dead_tiles"] + st["pruned_tiles"] == n_tiles
     # at full vocabulary size |E_i| max|C_v| < lse_i + ln(eps) for these
     # random-init heads: only label tiles are recomputed
@@ -52,7 +52,7 @@ def test_full_size_forward_backward_sampled(w):
         _, lse_o[r] = oracle.forward(inp["E"], inp["C"], inp["y"], IGN, rows=r)
     rE = np.concatenate([np.arange(b * 128, min(w.N, (b + 1) * 128)) for b in blocks])
     oE, _ = oracle.backward_sampled(inp["E"], inp["C"], inp["y"], lse_o, dloss, IGN, rE, [],
-                                    filter_eps=w.filter_eps, tile=(128, 64))
+                                    filter_eps=w.filter_eps, tile=(32, 32))
     gE = dE[torch.from_numpy(rE).cuda()].cpu().numpy()
     assert rel_fro(gE, oE) <= GRAD_REL_FILTER_ON
 
@@ -79,6 +79,6 @@ def test_full_size_gemma_dC_rows_and_mean_loss():
     counts = np.bincount(inp["y"], minlength=w.V)
     rC = np.unique(np.concatenate([np.argsort(-counts)[:6], [int(np.argmax(counts == 1))], [w.V - 1, 7777]]))
     _, oC = oracle.backward_sampled(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, [], rC,
-                                    filter_eps=w.filter_eps, tile=(128, 64))
+                                    filter_eps=w.filter_eps, tile=(32, 32))
     gC = dC[torch.from_numpy(rC).cuda()].cpu().numpy()
     assert rel_fro(gC, oC) <= GRAD_REL_FILTER_ON

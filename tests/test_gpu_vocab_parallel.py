@@ -7,7 +7,7 @@ import pytest
 import oracle
 from linear_cross_entropy_05_b200 import synth
 
-from _gpu_helpers import GRAD_REL_FILTER_OFF, GRAD_REL_FILTER_ON, IGN, LOSS_ABS, gpu_backward, gpu_forward, \
+from _gpu_helpers import GRAD_REL_FILTER_OFF, IGN, LOSS_ABS, filter_on_bar, gpu_backward, gpu_forward, \
     rel_fro, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -69,8 +69,8 @@ def test_sharded_backward_assembles_the_full_gradient(w, bounds, eps):
         # each shard's filter grid starts at its own first row; against the
         # exact gradient the spec bar applies
         xE, xC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
-        assert rel_fro(dE.cpu().numpy(), xE) <= GRAD_REL_FILTER_ON
-        assert rel_fro(dC.cpu().numpy(), xC) <= GRAD_REL_FILTER_ON
+        assert rel_fro(dE.cpu().numpy(), xE) <= filter_on_bar(w.V)
+        assert rel_fro(dC.cpu().numpy(), xC) <= filter_on_bar(w.V)
 
 
 def test_single_shard_helper_equals_unsharded_path():
