@@ -293,9 +293,32 @@ def run_gpu(args, w):
         dE = torch.empty((N, D), device=dev, dtype=torch.bfloat16)
         dC = torch.empty((V, D), device=dev, dtype=torch.bfloat16)
 
+    # Gradient zeroing: by default the fp32 dE/dC are cleared on a side stream
+    # while the (compute-bound) forward runs, and the backward adds into them
+    # (CCE_BWD_ACCUMULATE); the fixed-point modes write their outputs anyway.
+    overlap_zero = not (args.deterministic or args.bf16_grads or args.no_overlap_zero)
+    zero_stream = torch.cuda.Stream(device=dev)
+    grads_free = torch.cuda.Event()   # the previous backward is done with dE/dC
+    grads_zeroed = torch.cuda.Event()
+    grads_free.record(stream)
+
+    def fwd_bwd(Eb, Cb, yb, dlb):
+        if overlap_zero:
+            with torch.cuda.stream(zero_stream):
+                zero_stream.wait_event(grads_free)
+                dE.zero_()
+                dC.zero_()
+                grads_zeroed.record(zero_stream)
+        L.forward(Eb, Cb, yb, IGN, workspace=ws_f, out=(loss, lse))
+        if overlap_zero:
+            stream.wait_event(grads_zeroed)
+            L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC), accumulate=True, **gkw)
+            grads_free.record(stream)
+        else:
+            L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC), **gkw)
+
     def step():
-        L.forward(E, C, y, IGN, workspace=ws_f, out=(loss, lse))
-        L.backward(E, C, y, lse, dloss, eps, IGN, workspace=ws_b, out=(dE, dC), **gkw)
+        fwd_bwd(E, C, y, dloss)
 
     # warm-up (also loads the module) and status check
     for _ in range(max(3, args.warmup)):
@@ -385,8 +408,7 @@ def run_gpu(args, w):
                     dlb.copy_(dl_h, non_blocking=True)
                     copied[b].record(copy_stream)
                 stream.wait_event(copied[b])
-                L.forward(Eb, Cb, yb, IGN, workspace=ws_f, out=(loss, lse))
-                L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC), **gkw)
+                fwd_bwd(Eb, Cb, yb, dlb)
                 loss_h[b].copy_(loss, non_blocking=True)
                 consumed[b].record(stream)
 
@@ -430,7 +452,9 @@ def run_gpu(args, w):
             "config": dict(config_of(w, world), forward_kernel=args.fwd_variant,
                            backward_accumulation=("fixed-point int64" if (args.deterministic or args.bf16_grads)
                                                   else "fp32 atomic (TMA reduce-add)"),
-                           grad_dtype="bf16" if args.bf16_grads else "fp32"),
+                           grad_dtype="bf16" if args.bf16_grads else "fp32",
+                           grad_zeroing=("side stream during the forward; backward accumulates (CCE_BWD_ACCUMULATE)"
+                                         if overlap_zero else "inside the backward call")),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
@@ -534,6 +558,8 @@ def main(argv=None):
     ap.add_argument("--deterministic", action="store_true",
                     help="bitwise reproducible backward (fixed-point accumulation)")
     ap.add_argument("--bf16-grads", action="store_true", help="bf16 dE/dC outputs (fixed-point accumulation)")
+    ap.add_argument("--no-overlap-zero", action="store_true",
+                    help="let the backward zero dE/dC itself instead of a side stream during the forward")
     ap.add_argument("--fwd-variant", choices=["single", "pair"], default="single",
                     help="forward kernel: single CTAs (default) or CTA pairs (A/B measurement)")
     ap.add_argument("--suite", action="store_true",

@@ -154,7 +154,17 @@ typedef enum {
   CCE_BWD_DETERMINISTIC = 1,
   /* dE and dC are written as bf16 (round to nearest even) instead of fp32;
    * implies CCE_BWD_DETERMINISTIC (the accumulation is the same). */
-  CCE_BWD_BF16_GRADS = 2
+  CCE_BWD_BF16_GRADS = 2,
+  /* Add this call's gradients to the contents of dE and dC instead of
+   * overwriting them (no zeroing pass): gradient accumulation over
+   * micro-batches, or zeroing done by the caller where it costs nothing,
+   * e.g. on another stream while the compute-bound forward runs.  The
+   * caller must have written dE and dC (zeros before a first call).  With
+   * CCE_BWD_DETERMINISTIC each output entry gets one add of this call's
+   * fixed-point sum, in fp32 (or, with CCE_BWD_BF16_GRADS, the old bf16
+   * value plus the sum rounded once to bf16), so the result is still
+   * bitwise reproducible.  No extra workspace. */
+  CCE_BWD_ACCUMULATE = 4
 } cce_backward_flags_t;
 
 /* Workspace bytes for cce_backward_ex with these flags (0 if the sizes or

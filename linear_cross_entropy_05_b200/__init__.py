@@ -22,7 +22,7 @@ import os
 from typing import Optional, Tuple
 
 from . import _native
-from ._native import (CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCEError, cce_backward, cce_backward_ex,
+from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCEError, cce_backward, cce_backward_ex,
                       cce_backward_shard, cce_backward_workspace_size, cce_backward_workspace_size_ex,
                       cce_forward_shard, cce_merge_shards, cce_debug_forward_logits,
                       cce_debug_set_backward_variant, cce_debug_set_forward_variant, cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns,
@@ -33,7 +33,7 @@ from ._native import (CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCEError, cce_b
 IGNORE_INDEX = -100
 
 __all__ = [
-    "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "cce_forward",
+    "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "CCE_BWD_ACCUMULATE", "cce_forward",
     "cce_forward_noalloc", "cce_backward", "cce_backward_ex", "cce_backward_workspace_size_ex",
     "cce_forward_shard", "cce_merge_shards", "cce_backward_shard", "forward_shard", "merge_shards",
     "backward_shard", "vocab_parallel_forward_backward", "cce_forward_workspace_size",
@@ -108,10 +108,12 @@ def forward(E, C, y, ignore_index: int = IGNORE_INDEX, workspace: Optional[Works
 
 def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = IGNORE_INDEX,
              workspace: Optional[Workspace] = None, stream=None, out=None, deterministic: bool = False,
-             bf16_grads: bool = False):
+             bf16_grads: bool = False, accumulate: bool = False):
     """dE [N, D] and dC [V, D] of sum_i dloss[i] * loss[i]: fp32, or bf16 with
     bf16_grads; deterministic=True gives bitwise reproducible gradients
-    (fixed-point accumulation, extra (N + V) * D * 8 bytes of workspace)."""
+    (fixed-point accumulation, extra (N + V) * D * 8 bytes of workspace).
+    accumulate=True adds them to the tensors given in `out` (required)
+    instead of overwriting them."""
     torch = _torch()
     _check_inputs(E, C, y)
     N, D = E.shape
@@ -119,7 +121,10 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     for t, n in ((lse, "lse"), (dloss, "dloss")):
         if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.shape != (N,):
             raise ValueError(f"{n} must be a contiguous CUDA float32 tensor of shape [N]")
-    flags = (CCE_BWD_DETERMINISTIC if deterministic else 0) | (CCE_BWD_BF16_GRADS if bf16_grads else 0)
+    flags = ((CCE_BWD_DETERMINISTIC if deterministic else 0) | (CCE_BWD_BF16_GRADS if bf16_grads else 0) |
+             (CCE_BWD_ACCUMULATE if accumulate else 0))
+    if accumulate and out is None:
+        raise ValueError("accumulate=True adds into existing gradients: pass them as out=(dE, dC)")
     gdt = torch.bfloat16 if bf16_grads else torch.float32
     if out is None:
         dE = torch.empty((N, D), dtype=gdt, device=E.device)

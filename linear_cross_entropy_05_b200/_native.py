@@ -139,6 +139,7 @@ def cce_backward(E: int, C: int, y: int, lse: int, dloss: int, N: int, D: int, V
 
 CCE_BWD_DETERMINISTIC = 1
 CCE_BWD_BF16_GRADS = 2
+CCE_BWD_ACCUMULATE = 4
 
 
 def cce_backward_workspace_size_ex(N: int, D: int, V: int, flags: int) -> int:

@@ -31,7 +31,7 @@ cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const fl
 cudaError_t launch_norms(const void* E, const void* C, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
-                                bool bf16, int sms, cudaStream_t stream);
+                                bool bf16, bool accumulate, int sms, cudaStream_t stream);
 }  // namespace cce
 
 using namespace cce;
@@ -185,7 +185,8 @@ struct BwdPlan {
   size_t off_accE, off_accC;  // fixed-point accumulators (deterministic mode only)
 };
 
-constexpr unsigned kBwdFlagsAll = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS;
+constexpr unsigned kBwdFlagsAll = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE;
+constexpr unsigned kBwdFixedPoint = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS;  // int64 accumulators
 
 bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags = 0) {
   if (flags & ~kBwdFlagsAll) return false;
@@ -206,7 +207,7 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
   p->off_enorm = p->off_list + align_up((size_t)N * sizeof(int2), 256);
   p->ws_bytes = p->off_enorm + align_up((size_t)N * sizeof(float), 256);
   p->off_accE = p->off_accC = 0;
-  if (flags) {
+  if (flags & kBwdFixedPoint) {
     p->off_accE = p->ws_bytes;
     p->off_accC = p->off_accE + align_up((size_t)N * D * 8, 256);
     p->ws_bytes = p->off_accC + align_up((size_t)V * D * 8, 256);
@@ -340,8 +341,9 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   if (!E || !C || !y || !lse || !dloss || !dE || !dC || !workspace) return CCE_ERR_INVALID_ARG;
   if (v_offset < 0) return CCE_ERR_INVALID_ARG;
   if (flags & ~kBwdFlagsAll) return CCE_ERR_INVALID_ARG;
-  const bool fixed = flags != 0;
+  const bool fixed = (flags & kBwdFixedPoint) != 0;
   const bool bf16_out = (flags & CCE_BWD_BF16_GRADS) != 0;
+  const bool accumulate = (flags & CCE_BWD_ACCUMULATE) != 0;
   if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
   if (!(filter_eps == filter_eps)) return CCE_ERR_INVALID_ARG;  // NaN
   if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(lse, 4) || !aligned(dloss, 4) ||
@@ -371,7 +373,7 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   if (fixed) {
     if (cudaMemsetAsync(accE, 0, (size_t)N * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
-  } else {
+  } else if (!accumulate) {
     if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
   }
@@ -433,8 +435,10 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (fixed) {
     const unsigned* hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);
-    if (launch_fixed_to_out(accE, dE, (size_t)N * D, hdr, (int)N, bf16_out, di.sms, stream) != cudaSuccess ||
-        launch_fixed_to_out(accC, dC, (size_t)V * D, hdr, (int)N, bf16_out, di.sms, stream) != cudaSuccess)
+    if (launch_fixed_to_out(accE, dE, (size_t)N * D, hdr, (int)N, bf16_out, accumulate, di.sms, stream) !=
+            cudaSuccess ||
+        launch_fixed_to_out(accC, dC, (size_t)V * D, hdr, (int)N, bf16_out, accumulate, di.sms, stream) !=
+            cudaSuccess)
       return CCE_ERR_CUDA;
   }
   return CCE_OK;

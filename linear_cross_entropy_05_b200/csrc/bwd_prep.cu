@@ -212,21 +212,36 @@ __global__ void __launch_bounds__(256) prep_fixed_kernel(const float* __restrict
   if (lane == 0) atomicMax(p.hdr + HDR_DLMAX, __float_as_uint(dmax));
 }
 
-// Deterministic mode: int64 fixed-point accumulators -> fp32 or bf16 output.
+// Deterministic mode: int64 fixed-point accumulators -> fp32 or bf16 output
+// (written, or with accumulate added to what the output holds: one add per
+// entry, so the result stays reproducible).
 __global__ void __launch_bounds__(256) fixed_to_out_kernel(const unsigned long long* __restrict__ acc, void* out,
                                                            size_t n, const unsigned* __restrict__ hdr, int N,
-                                                           int bf16) {
+                                                           int bf16, int accumulate) {
   const int s = fixed_point_exponent(__uint_as_float(hdr[HDR_CMAX]), __uint_as_float(hdr[HDR_EMAX]),
                                      __uint_as_float(hdr[HDR_DLMAX]), N);
   const double inv = ldexp(1.0, -s);
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; 2 * i < n; i += stride) {
     const ulonglong2 q = reinterpret_cast<const ulonglong2*>(acc)[i];   // n is even (D % 8 == 0)
-    const double x0 = (double)(long long)q.x * inv, x1 = (double)(long long)q.y * inv;
+    double x0 = (double)(long long)q.x * inv, x1 = (double)(long long)q.y * inv;
     if (bf16) {
-      reinterpret_cast<__nv_bfloat162*>(out)[i] = __halves2bfloat162(__double2bfloat16(x0), __double2bfloat16(x1));
+      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out) + i;
+      if (accumulate) {
+        const float2 old = __bfloat1622float2(*o);
+        x0 += (double)old.x;
+        x1 += (double)old.y;
+      }
+      *o = __halves2bfloat162(__double2bfloat16(x0), __double2bfloat16(x1));
     } else {
-      reinterpret_cast<float2*>(out)[i] = make_float2((float)x0, (float)x1);
+      float2* o = reinterpret_cast<float2*>(out) + i;
+      float2 r = make_float2((float)x0, (float)x1);
+      if (accumulate) {
+        const float2 old = *o;
+        r.x = old.x + r.x;  // fp32 add of this call's sum, rounded once to fp32
+        r.y = old.y + r.y;
+      }
+      *o = r;
     }
   }
 }
@@ -237,8 +252,8 @@ cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cu
 }
 
 cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
-                                bool bf16, int sms, cudaStream_t stream) {
-  fixed_to_out_kernel<<<sms * 8, 256, 0, stream>>>(acc, out, n, hdr, N, bf16 ? 1 : 0);
+                                bool bf16, bool accumulate, int sms, cudaStream_t stream) {
+  fixed_to_out_kernel<<<sms * 8, 256, 0, stream>>>(acc, out, n, hdr, N, bf16 ? 1 : 0, accumulate ? 1 : 0);
   return cudaGetLastError();
 }
 

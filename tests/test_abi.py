@@ -141,15 +141,17 @@ def test_backward_ex_workspace_and_flags(lib):
     N, D, V = 8192, 2304, 256000
     base = cce_backward_workspace_size(N, D, V)
     assert cce_backward_workspace_size_ex(N, D, V, 0) == base
-    for flags in (1, 2, 3):   # deterministic / bf16 outputs: int64 accumulators for dE and dC
+    for flags in (1, 2, 3, 5, 6, 7):   # deterministic / bf16 outputs: int64 accumulators for dE and dC
         assert cce_backward_workspace_size_ex(N, D, V, flags) == base + up(8 * N * D) + up(8 * V * D)
-    assert cce_backward_workspace_size_ex(N, D, V, 4) == 0   # unknown flag
+    assert cce_backward_workspace_size_ex(N, D, V, 4) == base   # accumulate alone: no extra workspace
+    assert cce_backward_workspace_size_ex(N, D, V, 8) == 0   # unknown flag
     P = 1 << 20
     args = [P, P, P, P, P, 256, 256, 4096, -100, 0.0, 0, P, P, P, 1 << 30, 0]
     args[10] = 8
     assert cce_backward_ex(*args, check=False) == 1          # unknown flag: rejected on the host
-    args[10] = 3
-    assert cce_backward_ex(*args, check=False) == 4          # valid, but no device here
+    for flags in (3, 4, 7):
+        args[10] = flags
+        assert cce_backward_ex(*args, check=False) == 4      # valid, but no device here
 
 
 def test_shard_entry_points_validate_on_the_host(lib):

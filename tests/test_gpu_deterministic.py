@@ -88,3 +88,44 @@ def test_deterministic_scale_edges():
     assert torch.isfinite(dE).all() and torch.isfinite(dC).all()
     assert rel_fro(dE.cpu().numpy(), rE.cpu().numpy()) < 1e-5
     assert rel_fro(dC.cpu().numpy(), rC.cpu().numpy()) < 1e-5
+
+
+@pytest.mark.parametrize("mode", ["atomic", "deterministic", "bf16"])
+def test_accumulate_adds_this_calls_gradients(mode):
+    # CCE_BWD_ACCUMULATE: no zeroing pass; the call adds its gradients to
+    # whatever dE and dC hold
+    import torch
+    w = synth.GEMMA2_2B.with_sizes(N=600, V=9000, D=256)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    dl = torch.from_numpy(synth.random_dloss(12, w.N)).cuda()
+    lse_t = torch.from_numpy(lse).cuda()
+    kw = {"atomic": {}, "deterministic": {"deterministic": True}, "bf16": {"bf16_grads": True}}[mode]
+    gE, gC, _ = _bwd(E, C, y, lse_t, dl, EPS, **kw)          # this call's gradients alone
+    # prior contents of the size of the gradients (seeded, generated on the host)
+    gen = torch.Generator().manual_seed(3)
+    rE = (torch.randn(gE.shape, generator=gen) * float(gE.float().abs().max())).to(gE.dtype).cuda()
+    rC = (torch.randn(gC.shape, generator=gen) * float(gC.float().abs().max())).to(gC.dtype).cuda()
+    aE, aC = rE.clone(), rC.clone()
+    _bwd(E, C, y, lse_t, dl, EPS, out=(aE, aC), accumulate=True, **kw)
+    if mode == "deterministic":
+        # one fp32 add of the same fixed-point sum per entry: bit for bit
+        assert torch.equal(aE, rE + gE) and torch.equal(aC, rC + gC)
+        zE, zC = torch.zeros_like(gE), torch.zeros_like(gC)
+        for _ in range(2):
+            _bwd(E, C, y, lse_t, dl, EPS, out=(zE, zC), accumulate=True, **kw)
+        assert torch.equal(zE, 2 * gE) and torch.equal(zC, 2 * gC)   # doubling is exact in fp32
+    elif mode == "bf16":
+        # old + this call's sum, rounded once to bf16: the same as rounding
+        # old + (the fp32 deterministic sum) except where the fp32 rounding of
+        # the sum moves a bf16 tie, and then by one bf16 step at most
+        fE, fC, _ = _bwd(E, C, y, lse_t, dl, EPS, deterministic=True)
+        for a, r, f in ((aE, rE, fE), (aC, rC, fC)):
+            want = (r.float() + f).to(torch.bfloat16)
+            off = a != want
+            assert off.float().mean().item() < 1e-3
+            assert ((a.float() - want.float()).abs()[off] <= want.float().abs()[off] * 2.0 ** -7).all()
+    else:
+        for a, r, g in ((aE, rE, gE), (aC, rC, gC)):
+            assert rel_fro((a - r).cpu().numpy(), g.cpu().numpy()) < 1e-5
