@@ -37,6 +37,19 @@ CCE_API void cce_debug_set_wait_limit_ns(uint64_t limit_ns);
  * it is on.  Process-wide; 0 turns it off. */
 CCE_API void cce_debug_withhold_loads(int on);
 
+/* Profiling hook for the backward kernel's per-tile timeline.  While set,
+ * every backward launch writes, for each CTA b (one per SM) and each of its
+ * first tiles_per_cta tiles k, four u64 at trace[(b * tiles_per_cta + k) * 4]:
+ * the GPU's globaltimer (ns) when the CTA's epilogue starts on the tile, when
+ * the tile's recomputed logits are complete in tensor memory, when its
+ * softmax-gradient tile and live mask are published, and the 32-bit live
+ * mask; after its last tile the CTA writes the end time into word 0 of the
+ * next entry (if < tiles_per_cta).  `trace` is a device buffer owned by the
+ * caller with room for (number of SMs) * tiles_per_cta * 32 bytes; the
+ * library does not clear it.  NULL turns the hook off.  Process-wide.
+ * Returns CCE_ERR_INVALID_ARG for tiles_per_cta outside [1, 2^20]. */
+CCE_API cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta);
+
 /* Selects the forward logit/LSE kernel: 0 = one SM per 128 x 256 logit tile
  * (the default), 1 = CTA pairs (two SMs per 256 x 256 tile through tcgen05
  * cta_group::2, half the shared-memory operand traffic per SM).  Both give

@@ -83,6 +83,8 @@ def load_library():
         lib.cce_debug_withhold_loads.restype = None
         lib.cce_debug_set_kernel_events.argtypes = [ctypes.c_int, c_vp, c_vp]
         lib.cce_debug_set_kernel_events.restype = ctypes.c_int
+        lib.cce_debug_set_backward_trace.argtypes = [c_vp, c_i64]
+        lib.cce_debug_set_backward_trace.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -219,5 +221,13 @@ def cce_debug_set_forward_variant(variant: int) -> None:
 
 
 def cce_debug_set_backward_variant(variant: int) -> None:
-    """0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 staging buffers."""
+    """0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 staging buffers,
+    2 = 2 stages / eight epilogue warps."""
     _check(load_library().cce_debug_set_backward_variant(int(variant)), "cce_debug_set_backward_variant")
+
+
+def cce_debug_set_backward_trace(trace: int, tiles_per_cta: int) -> None:
+    """Per-tile globaltimer stamps of every backward launch into the device
+    buffer `trace` (u64 [SMs][tiles_per_cta][4]); trace = 0 turns it off."""
+    _check(load_library().cce_debug_set_backward_trace(trace or None, int(tiles_per_cta)),
+           "cce_debug_set_backward_trace")

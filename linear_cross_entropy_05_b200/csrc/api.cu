@@ -47,6 +47,8 @@ std::atomic<int> g_bwd_variant{0};
 
 // Test hook: when set, the next launches' TMA producers issue no copies.
 std::atomic<int> g_withhold_loads{0};
+std::atomic<unsigned long long*> g_bwd_trace{nullptr};
+std::atomic<int> g_bwd_trace_cap{0};
 
 // Optional per-kernel timing events (debug hook): [kernel][0 = start, 1 = stop].
 std::atomic<void*> g_events[2][2] = {{{nullptr}, {nullptr}}, {{nullptr}, {nullptr}}};
@@ -309,6 +311,13 @@ void cce_debug_set_wait_limit_ns(uint64_t limit_ns) {
 
 void cce_debug_withhold_loads(int on) { g_withhold_loads.store(on ? 1 : 0); }
 
+cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta) {
+  if (trace && (tiles_per_cta <= 0 || tiles_per_cta > (1 << 20))) return CCE_ERR_INVALID_ARG;
+  g_bwd_trace_cap.store(trace ? (int)tiles_per_cta : 0);
+  g_bwd_trace.store(reinterpret_cast<unsigned long long*>(trace));
+  return CCE_OK;
+}
+
 cce_status_t cce_debug_set_forward_variant(int variant) {
   if (variant < 0 || variant > 1) return CCE_ERR_INVALID_ARG;
   g_fwd_variant.store(variant);
@@ -404,6 +413,8 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.withhold_loads = g_withhold_loads.load();
+  a.trace = g_bwd_trace.load();
+  a.trace_cap = g_bwd_trace_cap.load();
 
   if (filter_on || fixed) {
     PrepArgs pp;

@@ -177,6 +177,15 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
   // every role after it; the epilogue clears slot (kt+4)%8 at tile kt, long
   // after its last reader (tile kt-4) and before its next writer (tile kt+4).
   volatile int* live_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  // Work items are handed out at run time (a global counter), so CTAs that
+  // draw cheap tiles take more of them.  The producer draws the CTA's kt-th
+  // item, writes it to tile_ring[kt%8] (-1: no more work) and arrives on
+  // tile_full[kt%2]; the MMA and epilogue roles wait on that barrier (phase
+  // kt/2) before reading the slot.  The producer cannot run two tiles ahead
+  // of either role (it needs tile kt's live mask before tile kt+1), so
+  // neither barrier can complete twice between a role's waits.
+  volatile int* tile_ring = live_ring + 8;
+  uint64_t* tile_full = reinterpret_cast<uint64_t*>(tmem_slot + 20);  // [2], 8-byte aligned
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -195,6 +204,8 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       mbar_init(&c_empty[b], NEPI);
     }
     mbar_init(drain, 1);
+    mbar_init(&tile_full[0], 1);
+    mbar_init(&tile_full[1], 1);
     *abort_flag = 0;
     for (int i = 0; i < 8; ++i) live_ring[i] = 0;
     fence_mbar_init();
@@ -225,8 +236,14 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       int kt = 0;
       TileMap tm;
       tm.init(a);
-      // withhold_loads (test hook): no copy is issued; see the forward kernel.
-      for (int t = a.withhold_loads ? tm.T : blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
+      // withhold_loads (test hook): tiles are handed out but no copy is
+      // issued, so the other roles wait on data that never comes.
+      for (;; ++kt) {
+        const unsigned long long drawn = atomicAdd(a.status + ST_NEXT_TILE, 1ull);
+        const int t = drawn < (unsigned long long)tm.T ? (int)drawn : -1;
+        tile_ring[kt & 7] = t;
+        mbar_arrive(&tile_full[kt & 1]);
+        if (t < 0) break;
         int m, vt;
         tm.get(a, t, m, vt);
         // logit recompute slices (d ascending); then, if the tile has a live
@@ -236,10 +253,12 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         // live (their dE products are the only ones that read C)
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
-          tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
-          armed |= 1u << stage;
+          if (!a.withhold_loads) {
+            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+            tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
+            tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
+            armed |= 1u << stage;
+          }
           if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
@@ -286,10 +305,9 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       int stage = 0;
       uint32_t phase = 0, sph = 0, gph = 0;
       uint32_t cfill0 = 0u, cfill1 = 0u;  // fills of contraction buffers 0 / 1 so far
-      int kt = 0;
-      TileMap tm;
-      tm.init(a);
-      for (int t = blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
+      for (int kt = 0;; ++kt) {
+        if (!mbar_wait(&tile_full[kt & 1], (uint32_t)(kt >> 1) & 1u, wc)) goto mma_done;
+        if (tile_ring[kt & 7] < 0) break;
         if (!mbar_wait(s_empty, sph ^ 1u, wc)) goto mma_done;
         sph ^= 1u;
         // buffer 1 lives in the logit tile's columns: wait until it is drained
@@ -396,7 +414,13 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
     int kt = 0;
     TileMap tm;
     tm.init(a);
-    for (int t = blockIdx.x; t < tm.T; t += gridDim.x, ++kt) {
+    const bool tracer = a.trace != nullptr && ew == 0 && lane == 0;
+    unsigned long long* trace_cta = a.trace ? a.trace + (size_t)blockIdx.x * a.trace_cap * 4 : nullptr;
+    for (;; ++kt) {
+      if (tracer && kt < a.trace_cap) trace_cta[kt * 4 + 0] = global_timer_ns();
+      if (!mbar_wait(&tile_full[kt & 1], (uint32_t)(kt >> 1) & 1u, wc)) break;
+      const int t = tile_ring[kt & 7];
+      if (t < 0) break;
       int m, vt;
       tm.get(a, t, m, vt);
       const int row = m * BM + rib;
@@ -419,6 +443,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
 
       if (!mbar_wait(s_full, sph, wc)) break;
       sph ^= 1u;
+      if (tracer && kt < a.trace_cap) trace_cta[kt * 4 + 1] = global_timer_ns();
       if (!mbar_wait(g_empty, gph ^ 1u, wc)) break;
       tc_fence_after();
       // This warp's units: its 32 rows (if any of them is a token) x each
@@ -474,6 +499,10 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       if (!mbar_wait(g_full, gph, wc)) break;
       gph ^= 1u;
       const uint32_t umask = (uint32_t)live_ring[kt & 7];
+      if (tracer && kt < a.trace_cap) {
+        trace_cta[kt * 4 + 2] = global_timer_ns();
+        trace_cta[kt * 4 + 3] = umask;
+      }
       n_live += __popc(umask);
       n_dead += (unsigned)(n_groups * n_chunks) - __popc(umask);
       ++n_tiles;
@@ -535,6 +564,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       if (!ok) break;
     }
     if (lane == 0) bulk_wait_group0();  // every reduction issued by this warp has landed
+    if (tracer && kt < a.trace_cap) trace_cta[kt * 4 + 0] = global_timer_ns();  // end of the last tile
     if (rib == 0 && hsel == 0) {
       atomicAdd(a.status + ST_LIVE_TILES, n_live);
       atomicAdd(a.status + ST_DEAD_TILES, n_dead);

@@ -32,6 +32,7 @@ enum StatusWord : int {
   ST_DEAD_TILES = 2,   // backward: filter units recomputed and found negligible
   ST_TILES = 3,        // forward: 128x256 logit tiles computed; backward: logit tiles recomputed
   ST_PRUNED = 4,       // backward: filter units proven negligible without recomputing them
+  ST_NEXT_TILE = 5,    // backward: next work item to hand out (CTAs take tiles as they free up)
 };
 // Header words of the backward pre-pass (u32, after the status block).
 enum PrepHeader : int {
@@ -117,6 +118,11 @@ struct BwdArgs {
   unsigned long long* status;
   unsigned long long wait_limit_ns;
   int withhold_loads;   // test hook: the TMA producer issues nothing
+  // profiling hook: per CTA and tile, globaltimer stamps (ns) at the start of
+  // the tile, when its logits are in TMEM and when its gradient tile and
+  // live mask are published; [grid][trace_cap][4] u64, null when off
+  unsigned long long* trace;
+  int trace_cap;
 };
 
 // Fixed-point exponent s: contributions are stored as round(x * 2^s) in int64.
