@@ -50,12 +50,13 @@ CCE_API void cce_debug_withhold_loads(int on);
  * Returns CCE_ERR_INVALID_ARG for tiles_per_cta outside [1, 2^20]. */
 CCE_API cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta);
 
-/* Selects the forward logit/LSE kernel: 0 = one SM per 128 x 256 logit tile
- * (the default), 1 = CTA pairs (two SMs per 256 x 256 tile through tcgen05
- * cta_group::2, half the shared-memory operand traffic per SM).  Both give
- * the same loss up to fp32 rounding order; the switch exists for A/B
- * measurement (on the power-capped B200 the two run within a few percent).  The forward workspace size depends on
- * the variant: query cce_forward_workspace_size after switching.
+/* Selects the forward logit/LSE kernel: 1 = CTA pairs (two SMs per 256 x 256
+ * logit tile through tcgen05 cta_group::2, two thirds of the operand traffic
+ * per SM; the default), 0 = one SM per 128 x 256 logit tile.  Both give the
+ * same loss up to fp32 rounding order; the switch exists for A/B measurement
+ * (on the power-capped B200 the pairs are ~3 % faster on the Gemma-2-2B
+ * head in long runs).  The forward workspace size depends on the variant:
+ * query cce_forward_workspace_size after switching.
  * Process-wide.  Returns CCE_ERR_INVALID_ARG for other values. */
 CCE_API cce_status_t cce_debug_set_forward_variant(int variant);
 

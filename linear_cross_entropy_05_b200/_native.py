@@ -216,7 +216,7 @@ def cce_debug_withhold_loads(on: bool) -> None:
 
 
 def cce_debug_set_forward_variant(variant: int) -> None:
-    """0 = single-CTA forward kernel (default), 1 = CTA-pair forward kernel."""
+    """1 = CTA-pair forward kernel (default), 0 = single-CTA forward kernel."""
     _check(load_library().cce_debug_set_forward_variant(int(variant)), "cce_debug_set_forward_variant")
 
 

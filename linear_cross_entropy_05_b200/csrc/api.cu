@@ -40,8 +40,8 @@ namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
 
-// Forward kernel variant: 0 = single CTAs (default), 1 = CTA pairs (cta_group::2).
-std::atomic<int> g_fwd_variant{0};
+// Forward kernel variant: 1 = CTA pairs (cta_group::2, the default), 0 = single CTAs.
+std::atomic<int> g_fwd_variant{1};
 // Backward kernel variant: 0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 buffers.
 std::atomic<int> g_bwd_variant{0};
 

@@ -10,6 +10,8 @@ MEAN_REL = 1e-4          # mean loss, relative
 GRAD_REL_FILTER_OFF = 5e-3   # dE, dC relative Frobenius error, filter off
 GRAD_REL_FILTER_ON = 1e-2    # dE, dC relative Frobenius error, filter on (vs the exact gradient)
 
+DEFAULT_FWD_VARIANT = 1      # the library's default forward kernel: CTA pairs (tcgen05 cta_group::2)
+
 
 def filter_on_bar(V):
     """Filter-on bar against the exact gradient for a vocabulary of V.

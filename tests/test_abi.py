@@ -13,7 +13,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _declared_symbols():
     names = set()
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
-        src = open(h).read()
+        with open(h) as f:
+            src = f.read()
         names |= set(re.findall(r"CCE_API\s+[\w\s\*]+?\b(cce_\w+)\s*\(", src))
     return sorted(names)
 

@@ -38,7 +38,7 @@ def _worker(rank, world, port, out):
 def test_aggregate_over_two_gloo_ranks():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
     for r in range(world):

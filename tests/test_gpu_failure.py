@@ -12,7 +12,7 @@ import pytest
 import oracle
 from linear_cross_entropy_05_b200 import synth
 
-from _gpu_helpers import IGN, LOSS_ABS, gpu_backward, gpu_forward, rel_fro, to_dev
+from _gpu_helpers import DEFAULT_FWD_VARIANT, IGN, LOSS_ABS, gpu_backward, gpu_forward, rel_fro, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -37,14 +37,14 @@ def test_withheld_loads_end_with_timeout_status_and_a_usable_context():
             L.forward(E, C, y, IGN, workspace=ws)
             st = L.read_status(ws)
             assert st["status"] == CCE_ERR_TIMEOUT and st["flags"] & 1
-        L.cce_debug_set_forward_variant(0)
+        L.cce_debug_set_forward_variant(DEFAULT_FWD_VARIANT)
         for eps in (0.0, 2.0 ** -12):
             ws = L.Workspace()
             L.backward(E, C, y, torch.from_numpy(lse).cuda(), dl, eps, IGN, workspace=ws)
             st = L.read_status(ws)
             assert st["status"] == CCE_ERR_TIMEOUT and st["flags"] & 1
     finally:
-        L.cce_debug_set_forward_variant(0)
+        L.cce_debug_set_forward_variant(DEFAULT_FWD_VARIANT)
         L.cce_debug_withhold_loads(False)
         L.cce_debug_set_wait_limit_ns(1_000_000_000)
     torch.cuda.synchronize()

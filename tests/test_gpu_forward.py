@@ -7,7 +7,7 @@ import pytest
 import oracle
 from linear_cross_entropy_05_b200 import synth
 
-from _gpu_helpers import IGN, LOSS_ABS, MEAN_REL, gpu_forward, mean_of, to_dev
+from _gpu_helpers import DEFAULT_FWD_VARIANT, IGN, LOSS_ABS, MEAN_REL, gpu_forward, mean_of, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -60,7 +60,7 @@ def test_raw_logit_tiles_match_definition(variant):
                                    lse.data_ptr(), logits.data_ptr(), buf.data_ptr(), buf.numel(),
                                    torch.cuda.current_stream().cuda_stream)
     finally:
-        L.cce_debug_set_forward_variant(0)
+        L.cce_debug_set_forward_variant(DEFAULT_FWD_VARIANT)
     g = logits.cpu().numpy()
     z = oracle.logits(oracle.bf16_bits_to_f64(inp["E"]), oracle.bf16_bits_to_f64(inp["C"]))
     # bf16 x bf16 products are exact in fp32; only the fp32 accumulation rounds
@@ -179,17 +179,17 @@ def test_library_allocates_no_device_memory():
                                synth.TINY.with_sizes(N=129, V=257, D=8),
                                synth.GEMMA2_2B.with_sizes(N=1000, V=20000)],
                          ids=["ragged", "minimal", "gemma-shaped"])
-def test_cta_pair_forward_variant_matches_oracle(w):
-    # the CTA-pair forward kernel (tcgen05 cta_group::2) is selectable for A/B
-    # measurement and must give the same losses as the default kernel
+def test_single_cta_forward_variant_matches_oracle(w):
+    # the single-CTA forward kernel is selectable for A/B measurement and must
+    # give the same losses as the default CTA-pair kernel (tcgen05 cta_group::2)
     import linear_cross_entropy_05_b200 as L
     inp = synth.make_inputs(w)
     E, C, y = to_dev(inp)
-    L.cce_debug_set_forward_variant(1)
+    L.cce_debug_set_forward_variant(0)
     try:
         loss1, lse1, st = gpu_forward(E, C, y)
     finally:
-        L.cce_debug_set_forward_variant(0)
+        L.cce_debug_set_forward_variant(DEFAULT_FWD_VARIANT)
     assert st["status"] == 0
     loss0, lse0, st = gpu_forward(E, C, y)
     ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)

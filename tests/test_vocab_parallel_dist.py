@@ -105,7 +105,7 @@ def test_two_rank_vocab_parallel_step_matches_unsharded_oracle(bounds):
     import oracle
     from linear_cross_entropy_05_b200 import synth
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, _free_port(), bounds, out), nprocs=world, join=True,
                        start_method="spawn")
