@@ -20,10 +20,11 @@
 //
 // Roles (192 threads): warp 0 TMA producer, warp 1 UMMA issuer, warps 2-5
 // epilogue (one TMEM lane = one token row / one vocabulary row per thread).
-// TMEM columns: [0,256) logit tile; contraction accumulators double-buffered:
-// buffer 0 = dE chunk [256,320) + dC chunk [320,448), buffer 1 = dE [0,64) +
-// dC [64,192) (inside the logit tile's columns, free once the epilogue has
-// read the tile; the next tile's logits wait until buffer 1 is drained).
+// TMEM columns: [0,256) logit tile; [256,512) two contraction buffers of a
+// dE chunk and one half's dC chunk each.  Because the two never overlap, the
+// next tile's logits are recomputed while this tile's products drain: once a
+// tile's gradient tile is published, the operand stream interleaves its
+// contraction slices with the next tile's recompute slices.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -35,8 +36,11 @@ namespace cce {
 
 namespace {
 constexpr uint32_t TM_S = 0;
-__device__ __forceinline__ uint32_t tm_de(int b) { return b ? 0u : 256u; }   // dE chunk of buffer b
-__device__ __forceinline__ uint32_t tm_dc(int b) { return b ? 64u : 320u; }   // dC chunk of buffer b
+// Contraction accumulators, double-buffered beside the logit tile: buffer b =
+// TMEM columns [256 + 128 b, 384 + 128 b): a dE chunk (64 columns) then one
+// half's dC chunk (64 columns).
+__device__ __forceinline__ uint32_t tm_de(int b) { return 256u + 128u * (uint32_t)b; }
+__device__ __forceinline__ uint32_t tm_dc(int b) { return 320u + 128u * (uint32_t)b; }
 
 // Live mask of a logit tile: bit 8 * g + c is the 32 x 32 filter unit of
 // token rows [32g, 32g + 32) and columns [32c, 32c + 32).
@@ -233,60 +237,83 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       // ---------------- TMA producer ----------------
       int stage = 0;
       uint32_t phase = 0, gph = 0, armed = 0;
-      int kt = 0;
       TileMap tm;
       tm.init(a);
       // withhold_loads (test hook): tiles are handed out but no copy is
       // issued, so the other roles wait on data that never comes.
-      for (;; ++kt) {
+      //
+      // Stage order (the MMA warp consumes the ring in the same order): the
+      // first tile's recompute slices (d ascending); then, per tile kt, once
+      // its live mask is known, its contraction slices (d descending, so the
+      // slices fetched last, most likely still in L2, come first: the E
+      // slice and only the live 64-row quarters of the C slice, the only C
+      // rows its dE products read) interleaved one to one with the next
+      // tile's recompute slices, so that the next logits are computed while
+      // this tile's partial products drain.
+      auto draw = [&](int k) -> int {
         const unsigned long long drawn = atomicAdd(a.status + ST_NEXT_TILE, 1ull);
         const int t = drawn < (unsigned long long)tm.T ? (int)drawn : -1;
-        tile_ring[kt & 7] = t;
-        mbar_arrive(&tile_full[kt & 1]);
-        if (t < 0) break;
-        int m, vt;
+        tile_ring[k & 7] = t;
+        mbar_arrive(&tile_full[k & 1]);
+        return t;
+      };
+      auto advance = [&]() {
+        if (++stage == NST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+      auto load_s = [&](int m, int vt, int kb) {  // one recompute slice (stage already free)
+        if (a.withhold_loads) return;
+        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+        tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
+        tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
+        armed |= 1u << stage;
+      };
+      int t = draw(0);
+      int m = 0, vt = 0;
+      if (t >= 0) {
         tm.get(a, t, m, vt);
-        // logit recompute slices (d ascending); then, if the tile has a live
-        // quarter, the operands of the two contractions with d descending, so
-        // that the slices fetched last (most likely still in L2) come first:
-        // the E slice, and of the C slice only the 64-row quarters that are
-        // live (their dE products are the only ones that read C)
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
-          if (!a.withhold_loads) {
-            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-            tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
-            tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
-            armed |= 1u << stage;
-          }
-          if (++stage == NST) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          load_s(m, vt, kb);
+          advance();
         }
+      }
+      for (int kt = 0; t >= 0; ++kt) {
         if (!mbar_wait(g_full, gph, wc)) goto producer_done;
         gph ^= 1u;
         const uint32_t umask = (uint32_t)live_ring[kt & 7];
-        if (umask == 0) continue;
+        const int tn = draw(kt + 1);
+        int mn = 0, vtn = 0;
+        if (tn >= 0) tm.get(a, tn, mn, vtn);
         uint32_t qmask = 0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) qmask |= (quarter_live(umask, q) ? 1u : 0u) << q;
-        const uint32_t bytes = A_STAGE_BYTES + (uint32_t)__popc(qmask) * QUARTER_BYTES;
-        for (int kb = nkb - 1; kb >= 0; --kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
+        const uint32_t c_bytes = A_STAGE_BYTES + (uint32_t)__popc(qmask) * QUARTER_BYTES;
+        for (int j = 0; j < nkb; ++j) {
+          if (umask) {
+            const int kb = nkb - 1 - j;
+            if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
+            mbar_arrive_expect_tx(&full[stage], c_bytes);
+            tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if ((qmask >> q) & 1)
-              tma_load_2d(sB + stage * B_STAGE_BYTES + q * QUARTER_BYTES, &tmCq, &full[stage], kb * BK,
-                          vt * BN + q * 64);
-          armed |= 1u << stage;
-          if (++stage == NST) {
-            stage = 0;
-            phase ^= 1u;
+            for (int q = 0; q < 4; ++q)
+              if ((qmask >> q) & 1)
+                tma_load_2d(sB + stage * B_STAGE_BYTES + q * QUARTER_BYTES, &tmCq, &full[stage], kb * BK,
+                            vt * BN + q * 64);
+            armed |= 1u << stage;
+            advance();
+          }
+          if (tn >= 0) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
+            load_s(mn, vtn, j);
+            advance();
           }
         }
+        t = tn;
+        m = mn;
+        vt = vtn;
       }
     producer_done : {
       int dummy = 0;
@@ -305,77 +332,104 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       int stage = 0;
       uint32_t phase = 0, sph = 0, gph = 0;
       uint32_t cfill0 = 0u, cfill1 = 0u;  // fills of contraction buffers 0 / 1 so far
-      for (int kt = 0;; ++kt) {
-        if (!mbar_wait(&tile_full[kt & 1], (uint32_t)(kt >> 1) & 1u, wc)) goto mma_done;
-        if (tile_ring[kt & 7] < 0) break;
+      int fb = 0;                         // contraction buffer of the next fill
+      auto advance = [&]() {
+        if (++stage == NST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+      // one k-block of the logit tile S = E_m C_vt^T into TMEM columns [0, 256)
+      auto s_block = [&](int kb) {
+        const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
+        const uint32_t b_addr = smem_u32(sB + stage * B_STAGE_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          umma_bf16(tmem_base + TM_S, sdesc_sw128(a_addr + k * 32, 16, 1024),
+                    sdesc_sw128(b_addr + k * 32, 16, 1024), IDESC_S, (kb | k) != 0);
+        umma_commit(&empty[stage]);
+      };
+      int t = -1;
+      if (!mbar_wait(&tile_full[0], 0u, wc)) goto mma_done;
+      t = tile_ring[0];
+      if (t >= 0) {
         if (!mbar_wait(s_empty, sph ^ 1u, wc)) goto mma_done;
         sph ^= 1u;
-        // buffer 1 lives in the logit tile's columns: wait until it is drained
-        if (!mbar_wait(&c_empty[1], (cfill1 & 1u) ^ 1u, wc)) goto mma_done;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * B_STAGE_BYTES);
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_bf16(tmem_base + TM_S, sdesc_sw128(a_addr + k * 32, 16, 1024),
-                      sdesc_sw128(b_addr + k * 32, 16, 1024), IDESC_S, (kb | k) != 0);
-          umma_commit(&empty[stage]);
-          if (++stage == NST) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          s_block(kb);
+          advance();
         }
         umma_commit(s_full);
+      }
+      for (int kt = 0; t >= 0; ++kt) {
         if (!mbar_wait(g_full, gph, wc)) goto mma_done;
         gph ^= 1u;
         tc_fence_after();
         const uint32_t umask = (uint32_t)live_ring[kt & 7];  // live 32 x 32 units of the tile
-        if (umask) {
-          for (int kb = 0; kb < nkb; ++kb) {
-            const int b = kb & 1;
+        if (!mbar_wait(&tile_full[(kt + 1) & 1], (uint32_t)((kt + 1) >> 1) & 1u, wc)) goto mma_done;
+        const int tn = tile_ring[(kt + 1) & 7];
+        if (tn >= 0) {
+          // the epilogue has read this tile's logits: the next tile may overwrite them
+          if (!mbar_wait(s_empty, sph ^ 1u, wc)) goto mma_done;
+          sph ^= 1u;
+          tc_fence_after();
+        }
+        // Contraction fills per 64-wide d slice: the first holds the dE chunk
+        // (every live quarter) and the dC chunk of the first live half, the
+        // second (only when both halves are live) the dC chunk of half 1.
+        const int h_first = half_live(umask, 0) ? 0 : 1;
+        const bool both = half_live(umask, 0) && half_live(umask, 1);
+        for (int j = 0; j < nkb; ++j) {
+          if (umask) {
             if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
-            if (!mbar_wait(&c_empty[b], ((b ? cfill1 : cfill0) & 1u) ^ 1u, wc)) goto mma_done;
-            if (b) ++cfill1; else ++cfill0;
-            tc_fence_after();
             const uint32_t e_addr = smem_u32(sA + stage * A_STAGE_BYTES);  // E[m-block, d-chunk]: 128 tok x 64 d
-            const uint32_t c_addr = smem_u32(sB + stage * B_STAGE_BYTES);  // C[v-tile, d-chunk]: 256 voc x 64 d
-            uint32_t acc_de = 0;
+            const uint32_t c_addr = smem_u32(sB + stage * B_STAGE_BYTES);  // C[v-tile, d-chunk]: live quarters
+            for (int f = 0; f < (both ? 2 : 1); ++f) {
+              const int b = fb;
+              fb ^= 1;
+              if (!mbar_wait(&c_empty[b], ((b ? cfill1 : cfill0) & 1u) ^ 1u, wc)) goto mma_done;
+              if (b) ++cfill1; else ++cfill0;
+              tc_fence_after();
+              if (f == 0) {
+                uint32_t acc_de = 0;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (!quarter_live(umask, q)) continue;
-              // dE chunk += G_q (128 tok x 64 voc, K-major) . C_q chunk (K = voc rows, MN = d)
+                for (int q = 0; q < 4; ++q) {
+                  if (!quarter_live(umask, q)) continue;
+                  // dE chunk += G_q (128 tok x 64 voc, K-major) . C_q chunk (K = voc rows, MN = d)
 #pragma unroll
-              for (int k = 4 * q; k < 4 * q + 4; ++k) {
-                umma_bf16(tmem_base + tm_de(b),
-                          sdesc_sw128(g_addr + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024),
-                          sdesc_sw128(c_addr + k * 2048, 16384, 1024), IDESC_DE, acc_de);
-                acc_de = 1;
+                  for (int k = 4 * q; k < 4 * q + 4; ++k) {
+                    umma_bf16(tmem_base + tm_de(b),
+                              sdesc_sw128(g_addr + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024),
+                              sdesc_sw128(c_addr + k * 2048, 16384, 1024), IDESC_DE, acc_de);
+                    acc_de = 1;
+                  }
+                }
               }
-            }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (!half_live(umask, h)) continue;
+              const int h = f == 0 ? h_first : 1;
               // dC chunk of half h = G_h^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
 #pragma unroll
               for (int k = 0; k < BM / 16; ++k)
-                umma_bf16(tmem_base + tm_dc(b) + h * 64,
+                umma_bf16(tmem_base + tm_dc(b),
                           sdesc_sw128(g_addr + (2 * h) * (BM * 128) + k * 2048, BM * 128, 1024),
                           sdesc_sw128(e_addr + k * 2048, 16384, 1024), IDESC_DC, k != 0);
+              umma_commit(&c_full[b]);
             }
             umma_commit(&empty[stage]);
-            umma_commit(&c_full[b]);
-            if (++stage == NST) {
-              stage = 0;
-              phase ^= 1u;
-            }
+            advance();
           }
-          umma_commit(g_empty);
-        } else {
-          mbar_arrive(g_empty);
+          if (tn >= 0) {
+            if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
+            tc_fence_after();
+            s_block(j);
+            advance();
+          }
         }
+        umma_commit(g_empty);  // this tile's gradient tile may be overwritten once these products are done
+        if (tn >= 0) umma_commit(s_full);
+        t = tn;
       }
     mma_done:
       umma_commit(drain);
@@ -396,6 +450,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
     const bool filter_on = eps > 0.f;
     uint32_t sph = 0, gph = 0;
     uint32_t cfe0 = 0u, cfe1 = 0u;  // drains of contraction buffers 0 / 1 so far
+    int fb = 0;                     // contraction buffer of the next fill
     unsigned long long n_live = 0, n_dead = 0, n_tiles = 0;
     uint8_t* g_row = sG + rib * 128;
     uint8_t* const xb0 = sX + ew * NXB * 4096;
@@ -511,35 +566,41 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       bool ok = true;
       const int row0 = m * BM + lane_grp * 32;           // first dE row of this warp
       const uint32_t rows_valid = __ballot_sync(0xffffffffu, valid);  // kept tokens among those rows
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int b = kb & 1;
-        if (!mbar_wait(&c_full[b], (b ? cfe1 : cfe0) & 1u, wc)) {
-          ok = false;
-          break;
-        }
-        if (b) ++cfe1; else ++cfe0;
-        tc_fence_after();
-        const int d0 = (nkb - 1 - kb) * BK;  // the contraction pass runs d descending
-        // Reduction pieces of this chunk (32 rows of this lane group x 32
-        // columns each): dE q0, dE q1, then dC q0, q1 of every live half.
-        // With EPG = 2 the pieces alternate between the two warps.
+      // the fills of each d slice, in the MMA warp's order (see there)
+      const int h_first = half_live(umask, 0) ? 0 : 1;
+      const bool both = half_live(umask, 0) && half_live(umask, 1);
+      for (int j = 0; j < nkb && ok; ++j) {
+        const int d0 = (nkb - 1 - j) * BK;  // the contraction pass runs d descending
+        // Reduction pieces of this slice (32 rows of this lane group x 32
+        // columns each): dE q0, dE q1 and dC q0, q1 of the first live half,
+        // then dC q0, q1 of half 1 if both are live.  With EPG = 2 the
+        // pieces alternate between the two warps of the lane group.
         int piece = 0;
-#pragma unroll 1
-        for (int q = 0; q < 2; ++q, ++piece) {
-          const bool mine = (piece % EPG) == hsel && de_rows_live;
-          float v[32];
-          if (mine) tmem_ld32(tmem_base + lane_addr + tm_de(b) + q * 32, v);
-          if (mine && d0 + q * 32 < a.D && row0 < a.N) {
-            if (fixed)
-              fixed_red_block32(next_xb(), lane, v, a.accE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D,
-                                rows_valid, min(32, a.D - (d0 + q * 32)), fx_scale);
-            else
-              tma_red_block32<NXB>(next_xb(), lane, v, &tmdE, d0 + q * 32, row0);
+        for (int f = 0; f < (both ? 2 : 1); ++f) {
+          const int b = fb;
+          fb ^= 1;
+          if (!mbar_wait(&c_full[b], (b ? cfe1 : cfe0) & 1u, wc)) {
+            ok = false;
+            break;
           }
-        }
+          if (b) ++cfe1; else ++cfe0;
+          tc_fence_after();
+          if (f == 0) {
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          if (!half_live(umask, h)) continue;
+            for (int q = 0; q < 2; ++q, ++piece) {
+              const bool mine = (piece % EPG) == hsel && de_rows_live;
+              float v[32];
+              if (mine) tmem_ld32(tmem_base + lane_addr + tm_de(b) + q * 32, v);
+              if (mine && d0 + q * 32 < a.D && row0 < a.N) {
+                if (fixed)
+                  fixed_red_block32(next_xb(), lane, v, a.accE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D,
+                                    rows_valid, min(32, a.D - (d0 + q * 32)), fx_scale);
+                else
+                  tma_red_block32<NXB>(next_xb(), lane, v, &tmdE, d0 + q * 32, row0);
+              }
+            }
+          }
+          const int h = f == 0 ? h_first : 1;
           const int vr0 = vt * BN + h * BM + lane_grp * 32;
           // this warp's 32 vocabulary rows are column chunk 4h + lane_grp
           const bool dc_rows_live = chunk_live(umask, 4 * h + lane_grp);
@@ -547,7 +608,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
           for (int q = 0; q < 2; ++q, ++piece) {
             const bool mine = (piece % EPG) == hsel && dc_rows_live;
             float v[32];
-            if (mine) tmem_ld32(tmem_base + lane_addr + tm_dc(b) + h * 64 + q * 32, v);
+            if (mine) tmem_ld32(tmem_base + lane_addr + tm_dc(b) + q * 32, v);
             if (mine && d0 + q * 32 < a.D && vr0 < a.V) {
               if (fixed)
                 fixed_red_block32(next_xb(), lane, v, a.accC + (size_t)vr0 * a.D + d0 + q * 32, (size_t)a.D,
@@ -557,9 +618,9 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
                 tma_red_block32<NXB>(next_xb(), lane, v, &tmdC, d0 + q * 32, vr0);
             }
           }
+          tc_fence_before();
+          mbar_arrive(&c_empty[b]);
         }
-        tc_fence_before();
-        mbar_arrive(&c_empty[b]);
       }
       if (!ok) break;
     }
