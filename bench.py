@@ -553,9 +553,9 @@ def main(argv=None):
                     help="workload name (the default is the headline Gemma-2-2B-shaped head)")
     ap.add_argument("--N", type=int, default=None, help="override tokens (profiling cases)")
     ap.add_argument("--V", type=int, default=None, help="override vocabulary (profiling cases)")
-    ap.add_argument("--bwd-variant", type=int, choices=[0, 1, 2], default=0,
+    ap.add_argument("--bwd-variant", type=int, choices=[0, 1, 2, 3], default=0,
                     help="backward kernel: 0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 buffers, "
-                         "2 = 2 stages / 8 epilogue warps")
+                         "2 = 2 stages / 8 epilogue warps, 3 = as 0 with load/store-path reductions")
     ap.add_argument("--deterministic", action="store_true",
                     help="bitwise reproducible backward (fixed-point accumulation)")
     ap.add_argument("--bf16-grads", action="store_true", help="bf16 dE/dC outputs (fixed-point accumulation)")

@@ -65,7 +65,9 @@ CCE_API cce_status_t cce_debug_set_forward_variant(int variant);
  * 1 = two stages and two staging buffers (the staging of a block overlaps the
  * bulk read of the previous one), 2 = two stages and eight epilogue warps
  * (two per TMEM lane group, splitting the gradient columns and the
- * reduction pieces).  Same results; for A/B measurement.
+ * reduction pieces), 3 = as 0 but the fp32 reductions go through vector
+ * atomics (red.global.add.v4.f32) instead of the TMA engine.  Same results
+ * up to fp32 summation order; for A/B measurement.
  * Process-wide.  Returns CCE_ERR_INVALID_ARG for other values. */
 CCE_API cce_status_t cce_debug_set_backward_variant(int variant);
 

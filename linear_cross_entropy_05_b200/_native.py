@@ -222,7 +222,7 @@ def cce_debug_set_forward_variant(variant: int) -> None:
 
 def cce_debug_set_backward_variant(variant: int) -> None:
     """0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 staging buffers,
-    2 = 2 stages / eight epilogue warps."""
+    2 = 2 stages / eight epilogue warps, 3 = as 0 with load/store-path reductions."""
     _check(load_library().cce_debug_set_backward_variant(int(variant)), "cce_debug_set_backward_variant")
 
 

@@ -325,7 +325,7 @@ cce_status_t cce_debug_set_forward_variant(int variant) {
 }
 
 cce_status_t cce_debug_set_backward_variant(int variant) {
-  if (variant < 0 || variant > 2) return CCE_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 3) return CCE_ERR_INVALID_ARG;
   g_bwd_variant.store(variant);
   return CCE_OK;
 }

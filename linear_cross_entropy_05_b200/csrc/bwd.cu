@@ -85,6 +85,29 @@ __device__ __forceinline__ void tma_red_block32(uint8_t* xb, int lane, const flo
   }
 }
 
+// The same 32 x 32 fp32 block added with vector atomics on the load/store
+// path instead of the TMA engine: staged in the same swizzled layout, then
+// each warp instruction `red.global.add.v4.f32` covers four rows x 128
+// contiguous bytes.  nrows / ncols clip the block at the tensor's edge
+// (ncols is a multiple of 8).
+__device__ __forceinline__ void lsu_red_block32(uint8_t* xb, int lane, const float (&v)[32], float* base, size_t ld,
+                                                int nrows, int ncols) {
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(xb + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+  const int c4 = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = i * 4 + (lane >> 3);
+    const float4 x = *reinterpret_cast<const float4*>(xb + r * 128 + ((c4 ^ (r & 7)) << 4));
+    if (r < nrows && c4 * 4 < ncols) red_add_v4(base + (size_t)r * ld + c4 * 4, x.x, x.y, x.z, x.w);
+  }
+  __syncwarp();
+}
+
 // Work item t -> (token block m, vocabulary tile vt).  Dense mode rasters the
 // whole grid; list mode visits the pre-pass list (label tiles of flat blocks,
 // vocabulary-major), then every tile of each block that is not flat.
@@ -149,10 +172,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }  // namespace
 
 // NST: operand pipeline stages; NXB: reduction staging buffers per epilogue
-// warp; EPG: epilogue warps per TMEM lane group (1 or 2; with 2, the two
+// warp; RED: 0 = fp32 reductions by the TMA engine (bulk tensor reduce-add),
+// 1 = by vector atomics on the load/store path; EPG: epilogue warps per TMEM lane group (1 or 2; with 2, the two
 // warps of a lane group split the softmax-gradient columns by 128-column half
 // and deal the reduction pieces of each chunk between them).
-template <int NST, int NXB, int EPG>
+template <int NST, int NXB, int EPG, int RED>
 __global__ void __launch_bounds__(64 + 128 * EPG, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
                const __grid_constant__ CUtensorMap tmCq,
@@ -290,22 +314,39 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         uint32_t qmask = 0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) qmask |= (quarter_live(umask, q) ? 1u : 0u) << q;
-        const uint32_t c_bytes = A_STAGE_BYTES + (uint32_t)__popc(qmask) * QUARTER_BYTES;
-        for (int j = 0; j < nkb; ++j) {
-          if (umask) {
-            const int kb = nkb - 1 - j;
+        const uint32_t c_bytes = A_STAGE_BYTES + (uint32_t)__popc(qmask) * QUARTER_BYTES;  // one d slice
+        // A tile with a single live quarter needs 24 KB per d slice: two
+        // slices share one stage (E of the second slice at B + 8 KB, the
+        // quarters at B + 0 and B + 24 KB), halving its contraction stages.
+        const int cpack = __popc(qmask) == 1 ? 2 : 1;
+        const int q1 = __ffs(qmask) - 1;
+        const int n_cst = umask ? (nkb + cpack - 1) / cpack : 0;
+        const int n_sst = tn >= 0 ? nkb : 0;
+        for (int j = 0; j < max(n_cst, n_sst); ++j) {
+          if (j < n_cst) {
+            const int kb0 = nkb - 1 - cpack * j;
+            const int ns = (cpack == 2 && kb0 >= 1) ? 2 : 1;  // d slices in this stage
             if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
-            mbar_arrive_expect_tx(&full[stage], c_bytes);
-            tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
+            mbar_arrive_expect_tx(&full[stage], (uint32_t)ns * c_bytes);
+            uint8_t* b_st = sB + stage * B_STAGE_BYTES;
+            tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb0 * BK, m * BM);
+            if (cpack == 2) {
+              tma_load_2d(b_st, &tmCq, &full[stage], kb0 * BK, vt * BN + q1 * 64);
+              if (ns == 2) {
+                tma_load_2d(b_st + QUARTER_BYTES, &tmE, &full[stage], (kb0 - 1) * BK, m * BM);
+                tma_load_2d(b_st + QUARTER_BYTES + A_STAGE_BYTES, &tmCq, &full[stage], (kb0 - 1) * BK,
+                            vt * BN + q1 * 64);
+              }
+            } else {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if ((qmask >> q) & 1)
-                tma_load_2d(sB + stage * B_STAGE_BYTES + q * QUARTER_BYTES, &tmCq, &full[stage], kb * BK,
-                            vt * BN + q * 64);
+              for (int q = 0; q < 4; ++q)
+                if ((qmask >> q) & 1)
+                  tma_load_2d(b_st + q * QUARTER_BYTES, &tmCq, &full[stage], kb0 * BK, vt * BN + q * 64);
+            }
             armed |= 1u << stage;
             advance();
           }
-          if (tn >= 0) {
+          if (j < n_sst) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
             load_s(mn, vtn, j);
             advance();
@@ -382,45 +423,61 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         // second (only when both halves are live) the dC chunk of half 1.
         const int h_first = half_live(umask, 0) ? 0 : 1;
         const bool both = half_live(umask, 0) && half_live(umask, 1);
-        for (int j = 0; j < nkb; ++j) {
-          if (umask) {
+        uint32_t qmask = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) qmask |= (quarter_live(umask, q) ? 1u : 0u) << q;
+        // stage packing as in the producer: one live quarter -> two d slices per stage
+        const int cpack = __popc(qmask) == 1 ? 2 : 1;
+        const int n_cst = umask ? (nkb + cpack - 1) / cpack : 0;
+        const int n_sst = tn >= 0 ? nkb : 0;
+        for (int j = 0; j < max(n_cst, n_sst); ++j) {
+          if (j < n_cst) {
+            const int kb0 = nkb - 1 - cpack * j;
+            const int ns = (cpack == 2 && kb0 >= 1) ? 2 : 1;
             if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
-            const uint32_t e_addr = smem_u32(sA + stage * A_STAGE_BYTES);  // E[m-block, d-chunk]: 128 tok x 64 d
-            const uint32_t c_addr = smem_u32(sB + stage * B_STAGE_BYTES);  // C[v-tile, d-chunk]: live quarters
-            for (int f = 0; f < (both ? 2 : 1); ++f) {
-              const int b = fb;
-              fb ^= 1;
-              if (!mbar_wait(&c_empty[b], ((b ? cfill1 : cfill0) & 1u) ^ 1u, wc)) goto mma_done;
-              if (b) ++cfill1; else ++cfill0;
-              tc_fence_after();
-              if (f == 0) {
-                uint32_t acc_de = 0;
+            const uint32_t a_st = smem_u32(sA + stage * A_STAGE_BYTES);
+            const uint32_t b_st = smem_u32(sB + stage * B_STAGE_BYTES);
+            for (int sl = 0; sl < ns; ++sl) {
+              // E[m-block, d slice]: 128 tok x 64 d; C rows of the live quarters
+              const uint32_t e_addr = sl == 0 ? a_st : b_st + QUARTER_BYTES;
+              const uint32_t c_base = sl == 0 ? b_st : b_st + QUARTER_BYTES + A_STAGE_BYTES;
+              for (int f = 0; f < (both ? 2 : 1); ++f) {
+                const int b = fb;
+                fb ^= 1;
+                if (!mbar_wait(&c_empty[b], ((b ? cfill1 : cfill0) & 1u) ^ 1u, wc)) goto mma_done;
+                if (b) ++cfill1; else ++cfill0;
+                tc_fence_after();
+                if (f == 0) {
+                  uint32_t acc_de = 0;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  if (!quarter_live(umask, q)) continue;
-                  // dE chunk += G_q (128 tok x 64 voc, K-major) . C_q chunk (K = voc rows, MN = d)
+                  for (int q = 0; q < 4; ++q) {
+                    if (!quarter_live(umask, q)) continue;
+                    // C rows of quarter q: packed stages hold the single live quarter at c_base
+                    const uint32_t cq = cpack == 2 ? c_base : c_base + q * QUARTER_BYTES;
+                    // dE chunk += G_q (128 tok x 64 voc, K-major) . C_q chunk (K = voc rows, MN = d)
 #pragma unroll
-                  for (int k = 4 * q; k < 4 * q + 4; ++k) {
-                    umma_bf16(tmem_base + tm_de(b),
-                              sdesc_sw128(g_addr + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024),
-                              sdesc_sw128(c_addr + k * 2048, 16384, 1024), IDESC_DE, acc_de);
-                    acc_de = 1;
+                    for (int k = 0; k < 4; ++k) {
+                      umma_bf16(tmem_base + tm_de(b),
+                                sdesc_sw128(g_addr + q * (BM * 128) + k * 32, 16, 1024),
+                                sdesc_sw128(cq + k * 2048, 16384, 1024), IDESC_DE, acc_de);
+                      acc_de = 1;
+                    }
                   }
                 }
-              }
-              const int h = f == 0 ? h_first : 1;
-              // dC chunk of half h = G_h^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
+                const int h = f == 0 ? h_first : 1;
+                // dC chunk of half h = G_h^T (MN = voc, K = tok) . Echunk (K = tok rows, MN = d)
 #pragma unroll
-              for (int k = 0; k < BM / 16; ++k)
-                umma_bf16(tmem_base + tm_dc(b),
-                          sdesc_sw128(g_addr + (2 * h) * (BM * 128) + k * 2048, BM * 128, 1024),
-                          sdesc_sw128(e_addr + k * 2048, 16384, 1024), IDESC_DC, k != 0);
-              umma_commit(&c_full[b]);
+                for (int k = 0; k < BM / 16; ++k)
+                  umma_bf16(tmem_base + tm_dc(b),
+                            sdesc_sw128(g_addr + (2 * h) * (BM * 128) + k * 2048, BM * 128, 1024),
+                            sdesc_sw128(e_addr + k * 2048, 16384, 1024), IDESC_DC, k != 0);
+                umma_commit(&c_full[b]);
+              }
             }
             umma_commit(&empty[stage]);
             advance();
           }
-          if (tn >= 0) {
+          if (j < n_sst) {
             if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
             tc_fence_after();
             s_block(j);
@@ -595,6 +652,9 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
                 if (fixed)
                   fixed_red_block32(next_xb(), lane, v, a.accE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D,
                                     rows_valid, min(32, a.D - (d0 + q * 32)), fx_scale);
+                else if (RED == 1)
+                  lsu_red_block32(next_xb(), lane, v, a.dE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D,
+                                  min(32, a.N - row0), min(32, a.D - (d0 + q * 32)));
                 else
                   tma_red_block32<NXB>(next_xb(), lane, v, &tmdE, d0 + q * 32, row0);
               }
@@ -614,6 +674,9 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
                 fixed_red_block32(next_xb(), lane, v, a.accC + (size_t)vr0 * a.D + d0 + q * 32, (size_t)a.D,
                                   __ballot_sync(0xffffffffu, vr0 + lane < a.V), min(32, a.D - (d0 + q * 32)),
                                   fx_scale);
+              else if (RED == 1)
+                lsu_red_block32(next_xb(), lane, v, a.dC + (size_t)vr0 * a.D + d0 + q * 32, (size_t)a.D,
+                                min(32, a.V - vr0), min(32, a.D - (d0 + q * 32)));
               else
                 tma_red_block32<NXB>(next_xb(), lane, v, &tmdC, d0 + q * 32, vr0);
             }
@@ -644,31 +707,33 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
   if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status + ST_FLAGS, SF_TIMEOUT);
 }
 
-template <int NST, int NXB, int EPG>
+template <int NST, int NXB, int EPG, int RED>
 size_t bwd_smem_bytes() {
   return 1024 + (size_t)NST * STAGE_BYTES + G_BYTES + (size_t)4 * EPG * NXB * 4096 + 256;
 }
 
-template <int NST, int NXB, int EPG>
+template <int NST, int NXB, int EPG, int RED>
 cudaError_t launch_bwd_t(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmCq, const CUtensorMap& tmdE,
                          const CUtensorMap& tmdC, const BwdArgs& a, int grid, cudaStream_t stream) {
-  const size_t smem = bwd_smem_bytes<NST, NXB, EPG>();
+  const size_t smem = bwd_smem_bytes<NST, NXB, EPG, RED>();
   cudaError_t e =
-      cudaFuncSetAttribute(bwd_kernel<NST, NXB, EPG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(bwd_kernel<NST, NXB, EPG, RED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  bwd_kernel<NST, NXB, EPG><<<grid, 64 + 128 * EPG, smem, stream>>>(tmE, tmC, tmCq, tmdE, tmdC, a);
+  bwd_kernel<NST, NXB, EPG, RED><<<grid, 64 + 128 * EPG, smem, stream>>>(tmE, tmC, tmCq, tmdE, tmdC, a);
   return cudaGetLastError();
 }
 
 // variant 0: 3 operand stages, one staging buffer, 4 epilogue warps (default);
 // variant 1: 2 stages, two staging buffers per warp (staging overlaps the bulk
 //            read of the previous block);
-// variant 2: 2 stages, 8 epilogue warps (two per TMEM lane group).
+// variant 2: 2 stages, 8 epilogue warps (two per TMEM lane group);
+// variant 3: as 0 with the fp32 reductions on the load/store path.
 cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUtensorMap& tmCq, const CUtensorMap& tmdE,
                        const CUtensorMap& tmdC, const BwdArgs& a, int grid, int variant, cudaStream_t stream) {
-  if (variant == 1) return launch_bwd_t<2, 2, 1>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
-  if (variant == 2) return launch_bwd_t<2, 1, 2>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
-  return launch_bwd_t<BWD_STAGES, 1, 1>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
+  if (variant == 1) return launch_bwd_t<2, 2, 1, 0>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
+  if (variant == 2) return launch_bwd_t<2, 1, 2, 0>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
+  if (variant == 3) return launch_bwd_t<BWD_STAGES, 1, 1, 1>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
+  return launch_bwd_t<BWD_STAGES, 1, 1, 0>(tmE, tmC, tmCq, tmdE, tmdC, a, grid, stream);
 }
 
 }  // namespace cce

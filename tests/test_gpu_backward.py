@@ -185,7 +185,7 @@ def test_autograd_wrapper_matches_oracle():
     assert rel_fro(C.grad.float().cpu().numpy(), rC) <= 1e-2
 
 
-@pytest.mark.parametrize("variant", [1, 2], ids=["2stages-2buffers", "8-epilogue-warps"])
+@pytest.mark.parametrize("variant", [1, 2, 3], ids=["2stages-2buffers", "8-epilogue-warps", "lsu-reductions"])
 @pytest.mark.parametrize("eps", [0.0, EPS], ids=["filter-off", "filter-on"])
 def test_backward_kernel_variants_match_oracle(variant, eps):
     # the alternative buffering / epilogue-warp layouts (selectable for A/B
