@@ -191,8 +191,8 @@ def blas_threads():
 
 def oracle_step(inp, rows, eps):
     """The oracle's forward + backward for the token rows `rows` (a whole
-    number of 128-row blocks): loss/lse for those rows, then their full
-    contribution to dE and dC (tile filter applied)."""
+    number of 32-row filter units): loss/lse for those rows, then their full
+    contribution to dE and dC (unit filter applied)."""
     import oracle
     E64 = oracle.bf16_bits_to_f64(inp["E"][rows])
     C64 = oracle.bf16_bits_to_f64(inp["C"])
@@ -232,9 +232,18 @@ def run_reference(args, w):
     from linear_cross_entropy_05_b200 import synth
     log(f"[reference] generating {w.name} ...")
     inp = synth.make_inputs(w)
-    rows_n = args.ref_rows
+    rows_n = max(32, args.ref_rows // 32 * 32)
+    # size the per-step sample so that warm-up + timed steps stay within the
+    # time budget: the first warm-up step calibrates (the oracle's cost is
+    # linear in the number of token rows)
+    t_cal = time.perf_counter()
+    oracle_step(inp, np.arange(rows_n), w.filter_eps)
+    t_cal = time.perf_counter() - t_cal
+    total_steps = args.steps + max(0, args.warmup - 1)
+    if total_steps * t_cal > args.ref_budget_s:
+        rows_n = max(32, int(rows_n * args.ref_budget_s / (total_steps * t_cal)) // 32 * 32)
     rows = np.arange(rows_n)
-    for _ in range(args.warmup):
+    for _ in range(args.warmup - 1):
         oracle_step(inp, rows, w.filter_eps)
     t0 = time.perf_counter()
     for _ in range(args.steps):
@@ -547,6 +556,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["cce", "reference"], default="cce")
     ap.add_argument("--cpu-rows", type=int, default=1024, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=128, help="tokens per step of the reference (oracle) arm")
+    ap.add_argument("--ref-budget-s", type=float, default=150.0,
+                    help="the reference arm shrinks its per-step sample (to >= 32 tokens) to stay within this time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--workload", default="gemma2-2b-head",
