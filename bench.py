@@ -393,7 +393,7 @@ def run_gpu(args, w):
     dl_h = torch.from_numpy(synth.mean_dloss(inp["y"])).pin_memory()
     h2d = E_h.numel() * 2 + C_h.numel() * 2 + y_h.numel() * 8 + dl_h.numel() * 4
     d2h = N * 4
-    e2e_value = None
+    e2e_value = e2e_resident = None
     if not args.no_e2e:
         Ke = max(3, K // 4)
         bufs = [(E, C, y, dloss)]
@@ -405,35 +405,43 @@ def run_gpu(args, w):
         for b in range(2):
             consumed[b].record(stream)
 
-        def e2e_run(steps):
+        def e2e_run(steps, copy_c=True):
             for k in range(steps):
                 b = k % 2
                 Eb, Cb, yb, dlb = bufs[b]
                 with torch.cuda.stream(copy_stream):
                     copy_stream.wait_event(consumed[b])
                     Eb.copy_(E_h, non_blocking=True)
-                    Cb.copy_(C_h, non_blocking=True)
+                    if copy_c:
+                        Cb.copy_(C_h, non_blocking=True)
                     yb.copy_(y_h, non_blocking=True)
                     dlb.copy_(dl_h, non_blocking=True)
                     copied[b].record(copy_stream)
                 stream.wait_event(copied[b])
-                fwd_bwd(Eb, Cb, yb, dlb)
+                fwd_bwd(Eb, Cb if copy_c else C, yb, dlb)
                 loss_h[b].copy_(loss, non_blocking=True)
                 consumed[b].record(stream)
 
-        e2e_run(2)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        e2e_run(Ke)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_value, _ = aggregate_throughput(dist, float(N * Ke), e0.elapsed_time(e1) / 1e3, dev)
-        if not np.isfinite(loss_h[(Ke - 1) % 2].numpy()).all():
-            raise RuntimeError("end-to-end loss read back non-finite values")
+        def e2e_time(copy_c):
+            e2e_run(2, copy_c)
+            torch.cuda.synchronize()
+            if dist is not None:
+                dist.barrier()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            e2e_run(Ke, copy_c)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            v, _ = aggregate_throughput(dist, float(N * Ke), e0.elapsed_time(e1) / 1e3, dev)
+            if not np.isfinite(loss_h[(Ke - 1) % 2].numpy()).all():
+                raise RuntimeError("end-to-end loss read back non-finite values")
+            return v
+
+        e2e_value = e2e_time(True)
+        # the same with the classifier C resident on the device (a training
+        # step's weights): only E, y and dloss cross the host link each step
+        e2e_resident = e2e_time(False)
         del bufs
 
     # ---- roofline of the dominant kernel ----
@@ -479,7 +487,11 @@ def run_gpu(args, w):
             "live_unit_frac": live / max(1, live + dead + pruned),
             "extra_hbm_bytes": int(extra_hbm),
             "materialised_logits_fp32_bytes": N * V * 4,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "inputs_copied": "E, C, y, dloss every step",
+                    "weights_resident": {"value": e2e_resident, "unit": UNIT,
+                                         "h2d_bytes_per_step": int(h2d - C_h.numel() * 2),
+                                         "inputs_copied": "E, y, dloss every step; C uploaded once"}},
             # our kernels per step: fwd_lse + fwd_finalize, bwd_kernel, and with
             # the filter on the four pre-pass kernels (cnorm, blocks, scan, scatter)
             "gpu_launches": (3 + (4 if eps > 0 else 0)) * K,

@@ -226,3 +226,35 @@ def test_labels_at_vocabulary_edges(eps):
     # the label rows of dC carry the one-hot part
     gC = dC.cpu().numpy()
     assert rel_fro(gC[[0, w.V - 1]], fC[[0, w.V - 1]]) <= GRAD_REL_FILTER_OFF
+
+
+def test_trace_hook_and_run_time_tile_dealing():
+    # CTAs draw work items from a global counter: over all CTAs every logit
+    # tile is drawn exactly once, each tile's stamps are ordered, and the
+    # traced live masks add up to the live-unit counter
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=1000, V=20000)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cap = 64
+    tr = torch.zeros(sms * cap * 4, dtype=torch.int64, device="cuda")
+    L.cce_debug_set_backward_trace(tr.data_ptr(), cap)
+    try:
+        dE, dC, st = gpu_backward(E, C, y, lse, synth.random_dloss(6, w.N), EPS)
+    finally:
+        L.cce_debug_set_backward_trace(0, 1)
+    assert st["status"] == 0
+    t = tr.view(sms, cap, 4).cpu().numpy()
+    tiles, live = 0, 0
+    for b in range(sms):
+        k = 0
+        while k < cap - 1 and t[b, k, 1] > 0:
+            assert t[b, k, 0] <= t[b, k, 1] <= t[b, k, 2] <= t[b, k + 1, 0]
+            live += bin(int(t[b, k, 3]) & 0xFFFFFFFF).count("1")
+            k += 1
+        tiles += k
+    assert tiles == st["logit_tiles"] > 0
+    assert live == st["live_tiles"]
