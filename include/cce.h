@@ -11,8 +11,8 @@
  *     dE = G C,  dC = G^T E,
  *   where the 32x32 gradient units (32 tokens x 32 vocabulary entries) whose
  *   every |softmax - onehot| entry is below filter_eps are skipped (the
- *   abstract's sentence 9: gradient work below numerical precision is
- *   dropped).
+ *   abstract's sentence 9: gradient terms too small to matter at the
+ *   working precision are left out).
  *
  * Conventions for every entry point:
  *   - All matrix arguments are DEVICE pointers to row-major, contiguous data.

@@ -6,8 +6,9 @@
 // TMEM and forms P = exp(S - lse) and D = P - onehot(y) in registers.  The
 // filter works on 32 x 32 units (32 tokens x 32 vocabulary entries, 32 per
 // logit tile: one epilogue warp's rows x one 32-column chunk): a unit whose
-// every |D| is below filter_eps is dropped (gradient work under numerical
-// precision) by writing its part of G = dloss * D to shared memory as zeros.
+// every |D| is below filter_eps is dropped (gradient terms too small to
+// matter at the working precision) by writing its part of G = dloss * D to
+// shared memory as zeros.
 // The tensor cores then contract whole blocks that hold a live unit:
 //     dE[m-block, d-chunk] += sum over live 64-column quarters q of G_q . C_q[d-chunk]   (M=128, N=64, K=64 each)
 //     dC[v-half h, d-chunk] += G_h^T . E[m-block, d-chunk]  for halves with a live unit  (M=128, N=64, K=128)

@@ -263,20 +263,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// OR-reduce a predicate over `nthreads` threads on named barrier `id`.
-__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
-  uint32_t out;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, %2, %3, q;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(out)
-      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-      : "memory");
-  return out != 0;
-}
-__device__ __forceinline__ void bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 __device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(gaddr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
