@@ -506,6 +506,75 @@ def run_gpu(args, w):
     return 0
 
 
+def run_memory(args, w):
+    """Classifier-head training step through the autograd wrapper: peak extra
+    device memory and time of `linear_cross_entropy(E, C, y).backward()`
+    against the same step with materialised logits (E C^T in bf16, then
+    torch's fp32 cross-entropy), the usual head a user would replace.  The
+    torch step is a comparison only; it runs nothing of this library.  One
+    JSON object (documentation, not the contract line)."""
+    import torch
+    import torch.nn.functional as F
+    import linear_cross_entropy_05_b200 as L
+    from linear_cross_entropy_05_b200 import synth
+    dev = torch.device("cuda", 0)
+    inp = synth.make_inputs(w)
+    E0 = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(dev)
+    C0 = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.from_numpy(inp["y"]).to(dev)
+
+    def cce_step(E, C):
+        return L.linear_cross_entropy(E, C, y, IGN, w.filter_eps)
+
+    def torch_step(E, C):
+        return F.cross_entropy((E @ C.t()).float(), y, ignore_index=IGN)
+
+    def measure(step, reps=5):
+        E = E0.clone().requires_grad_(True)
+        C = C0.clone().requires_grad_(True)
+        out = {}
+        for i in range(reps + 1):
+            E.grad = None
+            C.grad = None
+            torch.cuda.synchronize()
+            base = torch.cuda.memory_allocated(dev)
+            torch.cuda.reset_peak_memory_stats(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            loss = step(E, C)
+            loss.backward()
+            e1.record()
+            torch.cuda.synchronize()
+            if i == 0:        # first call: module load / allocator warm-up
+                continue
+            out.setdefault("ms", []).append(e0.elapsed_time(e1))
+            out["peak_extra_bytes"] = max(out.get("peak_extra_bytes", 0),
+                                          torch.cuda.max_memory_allocated(dev) - base)
+        out["loss"] = float(loss)
+        out["dE"], out["dC"] = E.grad.float(), C.grad.float()
+        out["ms"] = float(np.median(out["ms"]))
+        return out
+
+    a = measure(cce_step)
+    b = measure(torch_step)
+    rel = lambda x, r: float((x - r).norm() / r.norm())
+    grads = (w.N + w.V) * w.D * 2
+    res = {
+        "mode": "memory", "workload": w.name, "N": w.N, "D": w.D, "V": w.V, "filter_eps": w.filter_eps,
+        "gradient_bytes_bf16": grads,
+        "cce": {"peak_extra_bytes": int(a["peak_extra_bytes"]), "ms_per_step": a["ms"],
+                "tokens_per_s": w.N / a["ms"] * 1e3},
+        "materialised_torch": {"peak_extra_bytes": int(b["peak_extra_bytes"]), "ms_per_step": b["ms"],
+                               "tokens_per_s": w.N / b["ms"] * 1e3,
+                               "what": "logits = E @ C^T (bf16), F.cross_entropy(logits.float()), backward"},
+        "loss_abs_diff": abs(a["loss"] - b["loss"]),
+        "dE_rel_diff": rel(a["dE"], b["dE"]), "dC_rel_diff": rel(a["dC"], b["dC"]),
+    }
+    print(json.dumps(res), flush=True)
+    return 0
+
+
 def run_suite(args):
     """Per-workload table (not the contract line): fwd-only and fwd+bwd time,
     executed tensor fraction, tiles visited, extra global memory against the
@@ -586,6 +655,8 @@ def main(argv=None):
                     help="let the backward zero dE/dC itself instead of a side stream during the forward")
     ap.add_argument("--fwd-variant", choices=["single", "pair"], default="pair",
                     help="forward kernel: CTA pairs (default) or single CTAs (A/B measurement)")
+    ap.add_argument("--memory", action="store_true",
+                    help="classifier-head training step: peak memory and time, CCE vs materialised logits")
     ap.add_argument("--suite", action="store_true",
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
@@ -595,6 +666,10 @@ def main(argv=None):
         L.cce_debug_set_backward_variant(args.bwd_variant)
     if args.suite:
         return run_suite(args)
+    if args.memory:
+        from linear_cross_entropy_05_b200 import synth
+        w = synth.WORKLOADS[args.workload]
+        return run_memory(args, w.with_sizes(N=args.N, V=args.V) if (args.N or args.V) else w)
     if args.warmup < 3:
         args.warmup = 3
     from linear_cross_entropy_05_b200 import synth
