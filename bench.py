@@ -189,13 +189,15 @@ def blas_threads():
         return os.cpu_count()
 
 
-def oracle_step(inp, rows, eps):
+def oracle_step(inp, rows, eps, C64=None):
     """The oracle's forward + backward for the token rows `rows` (a whole
     number of 32-row filter units): loss/lse for those rows, then their full
-    contribution to dE and dC (unit filter applied)."""
+    contribution to dE and dC (unit filter applied).  C64: the classifier
+    already decoded to fp64 (resident input), else decoded here."""
     import oracle
     E64 = oracle.bf16_bits_to_f64(inp["E"][rows])
-    C64 = oracle.bf16_bits_to_f64(inp["C"])
+    if C64 is None:
+        C64 = oracle.bf16_bits_to_f64(inp["C"])
     y = inp["y"][rows]
     loss, lse = oracle.forward_f64(E64, C64, y, IGN)
     dl = np.full(len(rows), 1.0 / max(1, len(rows)))
@@ -232,26 +234,30 @@ def run_reference(args, w):
     from linear_cross_entropy_05_b200 import synth
     log(f"[reference] generating {w.name} ...")
     inp = synth.make_inputs(w)
+    import oracle
+    # the classifier is a resident input (decoded to fp64 once, as the GPU
+    # arm keeps C on the device); every step decodes its token rows
+    C64 = oracle.bf16_bits_to_f64(inp["C"])
     rows_n = max(32, args.ref_rows // 32 * 32)
     # size the per-step sample so that warm-up + timed steps stay within the
     # time budget: the first warm-up step calibrates (the oracle's cost is
     # linear in the number of token rows)
     t_cal = time.perf_counter()
-    oracle_step(inp, np.arange(rows_n), w.filter_eps)
+    oracle_step(inp, np.arange(rows_n), w.filter_eps, C64)
     t_cal = time.perf_counter() - t_cal
     total_steps = args.steps + max(0, args.warmup - 1)
     if total_steps * t_cal > args.ref_budget_s:
         rows_n = max(32, int(rows_n * args.ref_budget_s / (total_steps * t_cal)) // 32 * 32)
     rows = np.arange(rows_n)
     for _ in range(args.warmup - 1):
-        oracle_step(inp, rows, w.filter_eps)
+        oracle_step(inp, rows, w.filter_eps, C64)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(inp, rows, w.filter_eps)
+        oracle_step(inp, rows, w.filter_eps, C64)
     dt = time.perf_counter() - t0
     value = rows_n * args.steps / dt
-    sample = (f"each step: fp64 oracle forward+backward (tile filter {w.filter_eps:g}) on {rows_n} tokens of the "
-              f"{w.name} workload (full V={w.V}, D={w.D})")
+    sample = (f"each step: fp64 oracle forward+backward (unit filter {w.filter_eps:g}) on {rows_n} tokens of the "
+              f"{w.name} workload (full V={w.V}, D={w.D}; classifier decoded to fp64 once, outside the steps)")
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
