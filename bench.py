@@ -158,11 +158,18 @@ def measured_peaks():
 
 
 def kernel_source_hash(which: str) -> str:
+    """Hash of the code of a kernel's sources, comments and blank lines
+    removed (a comment edit does not change the kernel the counters came from)."""
+    import re
     base = os.path.join(ROOT, "linear_cross_entropy_05_b200", "csrc")
     h = hashlib.sha256()
     for f in (f"{which}.cu", "common.cuh", "ptx.cuh"):
-        with open(os.path.join(base, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(base, f)) as fh:
+            src = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        for line in src.splitlines():
+            line = line.split("//", 1)[0].rstrip()
+            if line.strip():
+                h.update(line.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

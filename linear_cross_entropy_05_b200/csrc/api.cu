@@ -42,7 +42,8 @@ std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
 
 // Forward kernel variant: 1 = CTA pairs (cta_group::2, the default), 0 = single CTAs.
 std::atomic<int> g_fwd_variant{1};
-// Backward kernel variant: 0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 buffers.
+// Backward kernel variant: 0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 buffers,
+// 2 = 2 stages / 8 epilogue warps, 3 = as 0 with load/store-path reductions.
 std::atomic<int> g_bwd_variant{0};
 
 // Test hook: when set, the next launches' TMA producers issue no copies.

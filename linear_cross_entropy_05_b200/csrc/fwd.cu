@@ -13,6 +13,9 @@
 //                 and the epilogue warps fold it into a per-row running
 //                 (max, sum exp(z - max)).  One (max, sum) pair per row and
 //                 split goes to the workspace; logits never leave the SM.
+// fwd_lse_pair_kernel  the same on clusters of two CTAs (the default): one
+//                 256 x 256 logit tile per pair through tcgen05 cta_group::2,
+//                 each CTA loading 128 rows of E and 128 rows of C per slice.
 // fwd_finalize    one warp per token: merges the split partials into lse,
 //                 forms the correct-token logit E_i . C_{y_i} with coalesced
 //                 16-byte loads, and writes loss = lse - z_y (0 if ignored).
