@@ -258,3 +258,34 @@ def test_trace_hook_and_run_time_tile_dealing():
         tiles += k
     assert tiles == st["logit_tiles"] > 0
     assert live == st["live_tiles"]
+
+
+@pytest.mark.parametrize("side", [-1, 1], ids=["eps-just-below-P", "eps-just-above-P"])
+def test_filter_decision_at_the_threshold(side):
+    # one softmax entry P sits 1 % away from eps: its 32 x 32 unit must be
+    # live when eps < P and dead when eps > P (every other entry of that unit
+    # is ~1/V, far below eps), exactly as the oracle's unit filter decides
+    w = synth.TINY.with_sizes(N=64, V=300, D=16)
+    inp = synth.make_inputs(w)
+    E = np.zeros((w.N, w.D), np.float32)
+    C = np.zeros((w.V, w.D), np.float32)
+    E[5, 0] = 1.0
+    C[200, 0] = 1.125                    # bf16-exact logit z[5, 200] = 1.125, all others 0
+    inp["E"] = synth.round_to_bf16_bits(E)
+    inp["C"] = synth.round_to_bf16_bits(C)
+    inp["y"] = np.zeros(w.N, np.int64)   # every label in column 0 (unit column 0)
+    ea = np.exp(1.125)
+    P = ea / (ea + w.V - 1)
+    eps = P * (1.0 + 0.01 * side)
+    Ed, Cd, yd = to_dev(inp)
+    loss, lse, st = gpu_forward(Ed, Cd, yd)
+    dloss = synth.random_dloss(7, w.N)
+    dE, dC, st = gpu_backward(Ed, Cd, yd, lse, dloss, eps)
+    assert st["status"] == 0
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    fE, fC, live = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=TILE,
+                                   return_live=True)
+    assert bool(live[0, 200 // 32]) == (side < 0)
+    assert st["live_tiles"] == int(live.sum()) == 2 + (side < 0)   # two label units (+ the edge unit)
+    assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF

@@ -99,3 +99,31 @@ def test_merge_flags_labels_outside_the_full_vocabulary():
     loss, lse = L.merge_shards(stats, y, w.V, IGN)
     l = loss.cpu().numpy()
     assert np.isnan(l[5]) and l[6] == 0.0 and np.isfinite(np.delete(l, 5)).all()
+
+
+def test_merge_of_hand_made_statistics():
+    # lse = M + log sum_r s_r exp(m_r - M) and loss = lse - sum_r t_r, with
+    # shards that hold nothing for a token (m = -inf, s = 0) and an ignored
+    # token; float32-exact inputs against fp64
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    inf = np.inf
+    m = np.array([[1.0, 2.0, -inf, 0.5, 30.0],
+                  [3.0, -inf, -inf, 0.25, -20.0],
+                  [-2.0, 1.5, 4.0, 0.5, 29.0]], dtype=np.float32)
+    s = np.array([[1.5, 2.0, 0.0, 1.0, 3.0],
+                  [2.5, 0.0, 0.0, 7.0, 1.0],
+                  [1.0, 4.0, 9.0, 1.0, 2.0]], dtype=np.float32)
+    t = np.array([[0.75, 0.0, 0.0, 0.0, 0.0],
+                  [0.0, 0.0, 0.0, 0.125, 0.0],
+                  [0.0, 1.0, 3.5, 0.0, 28.0]], dtype=np.float32)
+    y = np.array([3, 9, 7, 0, IGN], dtype=np.int64)
+    stats = torch.from_numpy(np.stack([m, s, t], axis=1)).cuda()        # [R, 3, N]
+    loss, lse = L.merge_shards(stats, torch.from_numpy(y).cuda(), 10, IGN)
+    m64, s64, t64 = m.astype(np.float64), s.astype(np.float64), t.astype(np.float64)
+    M = m64.max(axis=0)
+    want_lse = M + np.log((s64 * np.exp(m64 - M)).sum(axis=0))
+    want_loss = np.where(y != IGN, want_lse - t64.sum(axis=0), 0.0)
+    assert np.abs(lse.cpu().numpy() - want_lse).max() <= 1e-5 * np.abs(want_lse).max()
+    assert np.abs(loss.cpu().numpy() - want_loss).max() <= 1e-5 * np.abs(want_loss).max()
+    assert loss.cpu().numpy()[4] == 0
