@@ -266,10 +266,10 @@ def run_reference(args, w):
     sample = (f"each step: fp64 oracle forward+backward (unit filter {w.filter_eps:g}) on {rows_n} tokens of the "
               f"{w.name} workload (full V={w.V}, D={w.D}; classifier decoded to fp64 once, outside the steps)")
     out = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, ws), "gpu_launches": 0,
+        "config": config_of(w, ws), "gpu_launches": 0, "device": f"host cores (rank 0 of {ws})",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
