@@ -1,0 +1,56 @@
+"""Host-side helpers of bench.py: which peak the roofline divides by, and when
+a stored DRAM-traffic figure still belongs to the kernel being timed."""
+import importlib.util
+import json
+import os
+import shutil
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench(monkeypatch, root):
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    monkeypatch.setattr(b, "ROOT", str(root))
+    return b
+
+
+def _copy_sources(tmp_path):
+    dst = tmp_path / "linear_cross_entropy_05_b200" / "csrc"
+    shutil.copytree(os.path.join(ROOT, "linear_cross_entropy_05_b200", "csrc"), dst)
+    return dst
+
+
+def test_peaks_come_from_the_measured_file_else_the_stated_fallback(monkeypatch, tmp_path):
+    b = _bench(monkeypatch, tmp_path)
+    peaks, src = b.measured_peaks()
+    assert src == "fallback" and peaks["bf16_tflops_sustained"] == 1400.0 and peaks["hbm_gbs"] == 6650.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"bf16_tflops": 1.0, "bf16_tflops_sustained": 2.0}))
+    peaks, src = b.measured_peaks()
+    assert src == "measured" and peaks["bf16_tflops_sustained"] == 2.0
+
+
+def test_source_hash_follows_code_not_comments(monkeypatch, tmp_path):
+    csrc = _copy_sources(tmp_path)
+    b = _bench(monkeypatch, tmp_path)
+    h0 = b.kernel_source_hash("bwd")
+    f = csrc / "bwd.cu"
+    src = f.read_text()
+    f.write_text("// a new comment line\n" + src.replace("namespace cce {", "namespace cce {  /* inline note */", 1))
+    assert b.kernel_source_hash("bwd") == h0
+    assert b.kernel_source_hash("fwd") != h0          # another kernel's files
+    f.write_text(src.replace("constexpr uint32_t TM_S = 0;", "constexpr uint32_t TM_S = 1;", 1))
+    assert b.kernel_source_hash("bwd") != h0          # a code change invalidates stored counters
+
+
+def test_stored_traffic_is_reported_only_for_the_same_kernel_code(monkeypatch, tmp_path):
+    _copy_sources(tmp_path)
+    b = _bench(monkeypatch, tmp_path)
+    (tmp_path / "profiles").mkdir()
+    store = {"bwd_kernel": {"w": {"dram_bytes_per_launch": 123.0, "source_hash": b.kernel_source_hash("bwd")}},
+             "fwd_lse_kernel": {"w": {"dram_bytes_per_launch": 7.0, "source_hash": "0000000000000000"}}}
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(store))
+    assert b.ncu_traffic("bwd_kernel", "w") == 123.0
+    assert b.ncu_traffic("fwd_lse_kernel", "w") is None   # captured on other code
+    assert b.ncu_traffic("bwd_kernel", "other-workload") is None
