@@ -668,15 +668,19 @@ def main(argv=None):
                     help="let the backward zero dE/dC itself instead of a side stream during the forward")
     ap.add_argument("--fwd-variant", choices=["single", "pair"], default="pair",
                     help="forward kernel: CTA pairs (default) or single CTAs (A/B measurement)")
+    ap.add_argument("--prefetch", type=int, nargs=2, default=None, metavar=("FWD", "BWD"),
+                    help="L2 prefetch distances in K slices for the forward / backward operand streams (A/B)")
     ap.add_argument("--memory", action="store_true",
                     help="classifier-head training step: peak memory and time, CCE vs materialised logits")
     ap.add_argument("--suite", action="store_true",
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
-    if args.impl == "cce" and (args.fwd_variant != "pair" or args.bwd_variant):
+    if args.impl == "cce" and (args.fwd_variant != "pair" or args.bwd_variant or args.prefetch):
         import linear_cross_entropy_05_b200 as L
         L.cce_debug_set_forward_variant(1 if args.fwd_variant == "pair" else 0)
         L.cce_debug_set_backward_variant(args.bwd_variant)
+        if args.prefetch:
+            L.cce_debug_set_prefetch(*args.prefetch)
     if args.suite:
         return run_suite(args)
     if args.memory:

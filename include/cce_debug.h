@@ -37,6 +37,14 @@ CCE_API void cce_debug_set_wait_limit_ns(uint64_t limit_ns);
  * it is on.  Process-wide; 0 turns it off. */
 CCE_API void cce_debug_withhold_loads(int on);
 
+/* L2 prefetch distances, in 64-wide K slices, of the operand streams of the
+ * forward and backward kernels: while loading slice k into shared memory the
+ * TMA producer also asks for slice k + distance to be brought into L2
+ * (`cp.async.bulk.prefetch.tensor`, a hint with no completion).  0 turns the
+ * prefetch off.  Same results; for A/B measurement.  Process-wide.  Returns
+ * CCE_ERR_INVALID_ARG outside [0, 64]. */
+CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
+
 /* Profiling hook for the backward kernel's per-tile timeline.  While set,
  * every backward launch writes, for each CTA b (one per SM) and each of its
  * first tiles_per_cta tiles k, four u64 at trace[(b * tiles_per_cta + k) * 4]:

@@ -25,7 +25,7 @@ from . import _native
 from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCEError, cce_backward, cce_backward_ex,
                       cce_backward_shard, cce_backward_workspace_size, cce_backward_workspace_size_ex,
                       cce_forward_shard, cce_merge_shards, cce_debug_forward_logits,
-                      cce_debug_set_backward_trace, cce_debug_set_backward_variant, cce_debug_set_forward_variant, cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns,
+                      cce_debug_set_backward_trace, cce_debug_set_backward_variant, cce_debug_set_prefetch, cce_debug_set_forward_variant, cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns,
                       cce_debug_withhold_loads, cce_forward, cce_forward_noalloc,
                       cce_forward_workspace_size, cce_read_status,
                       cce_status_string, cce_version, load_library)
@@ -39,7 +39,7 @@ __all__ = [
     "backward_shard", "vocab_parallel_forward_backward", "cce_forward_workspace_size",
     "cce_backward_workspace_size", "cce_read_status", "cce_status_string", "cce_version",
     "cce_debug_forward_logits", "cce_debug_set_wait_limit_ns", "cce_debug_set_kernel_events", "cce_debug_withhold_loads", "cce_debug_set_forward_variant",
-    "cce_debug_set_backward_variant", "cce_debug_set_backward_trace",
+    "cce_debug_set_backward_variant", "cce_debug_set_backward_trace", "cce_debug_set_prefetch",
     "load_library",
     "forward", "backward", "read_status", "linear_cross_entropy", "Workspace",
 ]

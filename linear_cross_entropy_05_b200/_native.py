@@ -83,6 +83,8 @@ def load_library():
         lib.cce_debug_withhold_loads.restype = None
         lib.cce_debug_set_kernel_events.argtypes = [ctypes.c_int, c_vp, c_vp]
         lib.cce_debug_set_kernel_events.restype = ctypes.c_int
+        lib.cce_debug_set_prefetch.argtypes = [ctypes.c_int, ctypes.c_int]
+        lib.cce_debug_set_prefetch.restype = ctypes.c_int
         lib.cce_debug_set_backward_trace.argtypes = [c_vp, c_i64]
         lib.cce_debug_set_backward_trace.restype = ctypes.c_int
         _lib = lib
@@ -224,6 +226,11 @@ def cce_debug_set_backward_variant(variant: int) -> None:
     """0 = 3 stages / 1 staging buffer (default), 1 = 2 stages / 2 staging buffers,
     2 = 2 stages / eight epilogue warps, 3 = as 0 with load/store-path reductions."""
     _check(load_library().cce_debug_set_backward_variant(int(variant)), "cce_debug_set_backward_variant")
+
+
+def cce_debug_set_prefetch(fwd_slices: int, bwd_slices: int) -> None:
+    """L2 prefetch distances (64-wide K slices) of the forward / backward operand streams; 0 = off."""
+    _check(load_library().cce_debug_set_prefetch(int(fwd_slices), int(bwd_slices)), "cce_debug_set_prefetch")
 
 
 def cce_debug_set_backward_trace(trace: int, tiles_per_cta: int) -> None:

@@ -48,6 +48,8 @@ std::atomic<int> g_bwd_variant{0};
 
 // Test hook: when set, the next launches' TMA producers issue no copies.
 std::atomic<int> g_withhold_loads{0};
+std::atomic<int> g_fwd_pf{0};  // L2 prefetch distances (K slices) of the forward / backward operand streams
+std::atomic<int> g_bwd_pf{0};
 std::atomic<unsigned long long*> g_bwd_trace{nullptr};
 std::atomic<int> g_bwd_trace_cap{0};
 
@@ -257,6 +259,7 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.withhold_loads = g_withhold_loads.load();
+  a.pf = g_fwd_pf.load();
   if (record_event(0, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   const cudaError_t le =
       p.pair ? launch_fwd_lse_pair(tmE, tmC, a, p.grid, stream) : launch_fwd_lse(tmE, tmC, a, p.grid, stream);
@@ -311,6 +314,13 @@ void cce_debug_set_wait_limit_ns(uint64_t limit_ns) {
 }
 
 void cce_debug_withhold_loads(int on) { g_withhold_loads.store(on ? 1 : 0); }
+
+cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices) {
+  if (fwd_slices < 0 || fwd_slices > 64 || bwd_slices < 0 || bwd_slices > 64) return CCE_ERR_INVALID_ARG;
+  g_fwd_pf.store(fwd_slices);
+  g_bwd_pf.store(bwd_slices);
+  return CCE_OK;
+}
 
 cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta) {
   if (trace && (tiles_per_cta <= 0 || tiles_per_cta > (1 << 20))) return CCE_ERR_INVALID_ARG;
@@ -414,6 +424,7 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.withhold_loads = g_withhold_loads.load();
+  a.pf = g_bwd_pf.load();
   a.trace = g_bwd_trace.load();
   a.trace_cap = g_bwd_trace_cap.load();
 

@@ -294,6 +294,10 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
         tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
         armed |= 1u << stage;
+        if (a.pf && kb + a.pf < nkb) {  // L2 prefetch of the slices a.pf ahead
+          tma_prefetch_l2_2d(&tmE, (kb + a.pf) * BK, m * BM);
+          tma_prefetch_l2_2d(&tmC, (kb + a.pf) * BK, vt * BN);
+        }
       };
       int t = draw(0);
       int m = 0, vt = 0;
@@ -345,6 +349,14 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
                   tma_load_2d(b_st + q * QUARTER_BYTES, &tmCq, &full[stage], kb0 * BK, vt * BN + q * 64);
             }
             armed |= 1u << stage;
+            for (int sl = 0; a.pf && sl < ns; ++sl) {  // L2 prefetch of the contraction slices a.pf further on
+              const int kp = kb0 - sl - a.pf * cpack;         // (d descending)
+              if (kp < 0) break;
+              tma_prefetch_l2_2d(&tmE, kp * BK, m * BM);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if ((qmask >> q) & 1) tma_prefetch_l2_2d(&tmCq, kp * BK, vt * BN + q * 64);
+            }
             advance();
           }
           if (j < n_sst) {

@@ -62,6 +62,7 @@ struct FwdArgs {
   unsigned long long* status;
   unsigned long long wait_limit_ns;
   int withhold_loads;          // test hook: the TMA producer issues nothing
+  int pf;                      // L2 prefetch distance of the C stream in K slices (0: off)
 };
 
 struct FinArgs {
@@ -118,6 +119,7 @@ struct BwdArgs {
   unsigned long long* status;
   unsigned long long wait_limit_ns;
   int withhold_loads;   // test hook: the TMA producer issues nothing
+  int pf;               // L2 prefetch distance of the operand streams in K slices (0: off)
   // profiling hook: per CTA and tile, globaltimer stamps (ns) at the start of
   // the tile, when its logits are in TMEM and when its gradient tile and
   // live mask are published; [grid][trace_cap][4] u64, null when off

@@ -142,6 +142,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
             tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
             armed |= 1u << stage;
+            if (a.pf) {  // L2 prefetch of the C slice a.pf slices ahead in this unit's stream
+              const int s2 = (vt - v0) * nkb + kb + a.pf;
+              if (s2 < (v1 - v0) * nkb) tma_prefetch_l2_2d(&tmC, (s2 % nkb) * BK, (v0 + s2 / nkb) * BN);
+            }
             if (++stage == FWD_STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -339,6 +343,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d_pair(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m2 * (2 * BM) + rank * BM);
             tma_load_2d_pair(sB + stage * A_STAGE_BYTES, &tmCh, &full[stage], kb * BK, vt * BN + rank * BM);
             armed |= 1u << stage;
+            if (a.pf) {  // L2 prefetch of this CTA's C rows a.pf slices ahead in the unit's stream
+              const int s2 = (vt - v0) * nkb + kb + a.pf;
+              if (s2 < (v1 - v0) * nkb)
+                tma_prefetch_l2_2d(&tmCh, (s2 % nkb) * BK, (v0 + s2 / nkb) * BN + rank * BM);
+            }
             if (++stage == PAIR_STAGES) {
               stage = 0;
               phase ^= 1u;
