@@ -485,7 +485,8 @@ def run_gpu(args, w):
                                                   else "fp32 atomic (TMA reduce-add)"),
                            grad_dtype="bf16" if args.bf16_grads else "fp32",
                            grad_zeroing=("side stream during the forward; backward accumulates (CCE_BWD_ACCUMULATE)"
-                                         if overlap_zero else "inside the backward call")),
+                                         if overlap_zero else "inside the backward call"),
+                           l2_prefetch_slices=list(args.prefetch) if args.prefetch else [0, 0]),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
