@@ -148,6 +148,22 @@ class ClockSampler:
 # helpers
 # ---------------------------------------------------------------------------
 
+def launches_per_step(eps: float, fixed_point: bool) -> int:
+    """Kernels of this library launched by one forward + backward call pair:
+    forward logit/LSE kernel and finalize; backward kernel; the norm pass
+    (classifier and token norms) when the filter or the fixed-point mode
+    needs it; the candidate-tile pre-pass (blocks, scan, scatter) with the
+    filter on; the dloss maximum and two conversion passes in fixed point."""
+    n = 2 + 1
+    if eps > 0 or fixed_point:
+        n += 2
+    if eps > 0:
+        n += 3
+    if fixed_point:
+        n += 3
+    return n
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -508,7 +524,7 @@ def run_gpu(args, w):
                                          "inputs_copied": "E, y, dloss every step; C uploaded once"}},
             # our kernels per step: fwd_lse + fwd_finalize, bwd_kernel, and with
             # the filter on the four pre-pass kernels (cnorm, blocks, scan, scatter)
-            "gpu_launches": (3 + (4 if eps > 0 else 0)) * K,
+            "gpu_launches": launches_per_step(eps, args.deterministic or args.bf16_grads) * K,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
