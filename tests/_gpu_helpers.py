@@ -4,7 +4,7 @@ import numpy as np
 
 IGN = -100
 
-# Tolerances (the spec bar for this path)
+# Tolerances (the parity bar of this path)
 LOSS_ABS = 1e-2          # per-token loss, absolute
 MEAN_REL = 1e-4          # mean loss, relative
 GRAD_REL_FILTER_OFF = 5e-3   # dE, dC relative Frobenius error, filter off

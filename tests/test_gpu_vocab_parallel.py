@@ -67,7 +67,7 @@ def test_sharded_backward_assembles_the_full_gradient(w, bounds, eps):
         assert rel_fro(dC.cpu().numpy(), oC) <= GRAD_REL_FILTER_OFF
     else:
         # each shard's filter grid starts at its own first row; against the
-        # exact gradient the spec bar applies
+        # exact gradient the filter-on bar applies
         xE, xC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
         assert rel_fro(dE.cpu().numpy(), xE) <= filter_on_bar(w.V)
         assert rel_fro(dC.cpu().numpy(), xC) <= filter_on_bar(w.V)
