@@ -536,6 +536,58 @@ def run_gpu(args, w):
     return 0
 
 
+def run_trace(args, w):
+    """Per-tile timeline of one backward launch (cce_debug_set_backward_trace):
+    per CTA and tile, how long the epilogue waited for the recomputed logits,
+    how long it took to form and publish the gradient tile, and how long the
+    contraction and its drain took until the next tile.  One JSON object
+    (documentation, not the contract line)."""
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    from linear_cross_entropy_05_b200 import synth
+    dev = torch.device("cuda", 0)
+    inp = synth.make_inputs(w)
+    E = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(dev)
+    C = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.from_numpy(inp["y"]).to(dev)
+    dl = torch.from_numpy(synth.mean_dloss(inp["y"])).to(dev)
+    wf, wb = L.Workspace(dev), L.Workspace(dev)
+    loss, lse = L.forward(E, C, y, IGN, workspace=wf)
+    dE = torch.empty((w.N, w.D), device=dev)
+    dC = torch.empty((w.V, w.D), device=dev)
+    for _ in range(3):
+        L.backward(E, C, y, lse, dl, w.filter_eps, IGN, workspace=wb, out=(dE, dC))
+    cap = 256
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tr = torch.zeros(sms * cap * 4, dtype=torch.int64, device=dev)
+    L.cce_debug_set_backward_trace(tr.data_ptr(), cap)
+    try:
+        L.backward(E, C, y, lse, dl, w.filter_eps, IGN, workspace=wb, out=(dE, dC))
+        torch.cuda.synchronize()
+    finally:
+        L.cce_debug_set_backward_trace(0, 1)
+    st = L.read_status(wb)
+    t = tr.view(sms, cap, 4).cpu().numpy().astype(np.int64)
+    t0 = t[:, 0, 0][t[:, 0, 0] > 0].min()
+    S, G, Cc, ntiles, ends = [], [], [], [], []
+    for b in range(sms):
+        k = 0
+        while k < cap - 1 and t[b, k, 1] > 0:
+            S.append(t[b, k, 1] - t[b, k, 0])
+            G.append(t[b, k, 2] - t[b, k, 1])
+            Cc.append(t[b, k + 1, 0] - t[b, k, 2])
+            k += 1
+        ntiles.append(k)
+        ends.append(t[b, k, 0] - t0)
+    us = lambda x: float(np.mean(x) / 1e3) if x else None
+    print(json.dumps({
+        "mode": "trace", "workload": w.name, "N": w.N, "D": w.D, "V": w.V, "filter_eps": w.filter_eps,
+        "status": st, "ctas": sms, "tiles_per_cta_mean": float(np.mean(ntiles)), "tiles_per_cta_max": int(max(ntiles)),
+        "kernel_span_us": float(max(ends) / 1e3), "first_cta_end_us": float(min(ends) / 1e3),
+        "wait_for_logits_us": us(S), "gradient_tile_us": us(G), "contraction_and_drain_us": us(Cc)}), flush=True)
+    return 0
+
+
 def run_memory(args, w):
     """Classifier-head training step through the autograd wrapper: peak extra
     device memory and time of `linear_cross_entropy(E, C, y).backward()`
@@ -687,6 +739,8 @@ def main(argv=None):
                     help="forward kernel: CTA pairs (default) or single CTAs (A/B measurement)")
     ap.add_argument("--prefetch", type=int, nargs=2, default=None, metavar=("FWD", "BWD"),
                     help="L2 prefetch distances in K slices for the forward / backward operand streams (A/B)")
+    ap.add_argument("--trace", action="store_true",
+                    help="per-tile timeline of one backward launch (recompute wait, gradient tile, contraction)")
     ap.add_argument("--memory", action="store_true",
                     help="classifier-head training step: peak memory and time, CCE vs materialised logits")
     ap.add_argument("--suite", action="store_true",
@@ -700,10 +754,11 @@ def main(argv=None):
             L.cce_debug_set_prefetch(*args.prefetch)
     if args.suite:
         return run_suite(args)
-    if args.memory:
+    if args.memory or args.trace:
         from linear_cross_entropy_05_b200 import synth
         w = synth.WORKLOADS[args.workload]
-        return run_memory(args, w.with_sizes(N=args.N, V=args.V) if (args.N or args.V) else w)
+        w = w.with_sizes(N=args.N, V=args.V) if (args.N or args.V) else w
+        return run_memory(args, w) if args.memory else run_trace(args, w)
     if args.warmup < 3:
         args.warmup = 3
     from linear_cross_entropy_05_b200 import synth
