@@ -325,35 +325,43 @@ def run_gpu(args, w):
     ws_b = L.Workspace(dev)
     eps = w.filter_eps
     stream = torch.cuda.current_stream()
+    ws_b.get(L.cce_backward_workspace_size_ex(
+        N, D, V, (L.CCE_BWD_DETERMINISTIC if args.deterministic else 0) |
+        (L.CCE_BWD_BF16_GRADS if args.bf16_grads else 0)))   # allocated before the side stream uses it
 
     gkw = dict(deterministic=args.deterministic, bf16_grads=args.bf16_grads)
     if args.bf16_grads:
         dE = torch.empty((N, D), device=dev, dtype=torch.bfloat16)
         dC = torch.empty((V, D), device=dev, dtype=torch.bfloat16)
 
-    # Gradient zeroing: by default the fp32 dE/dC are cleared on a side stream
-    # while the (compute-bound) forward runs, and the backward adds into them
-    # (CCE_BWD_ACCUMULATE); the fixed-point modes write their outputs anyway.
+    # Side stream during the (tensor-bound) forward: the classifier-only part
+    # of the backward's pre-pass (cce_backward_prepare: max_v |C_v|, one read
+    # of C) and, by default, the clearing of the fp32 dE/dC, into which the
+    # backward then adds (CCE_BWD_ACCUMULATE); the fixed-point modes write
+    # their outputs anyway.
     overlap_zero = not (args.deterministic or args.bf16_grads or args.no_overlap_zero)
-    zero_stream = torch.cuda.Stream(device=dev)
-    grads_free = torch.cuda.Event()   # the previous backward is done with dE/dC
-    grads_zeroed = torch.cuda.Event()
-    grads_free.record(stream)
+    # (the classifier bound is used only by the filter and the fixed-point modes)
+    prepare = not args.no_prepare and (eps > 0 or args.deterministic or args.bf16_grads)
+    side_stream = torch.cuda.Stream(device=dev)
+    side_done = torch.cuda.Event()
 
     def fwd_bwd(Eb, Cb, yb, dlb):
-        if overlap_zero:
-            with torch.cuda.stream(zero_stream):
-                zero_stream.wait_event(grads_free)
-                dE.zero_()
-                dC.zero_()
-                grads_zeroed.record(zero_stream)
+        if overlap_zero or prepare:
+            with torch.cuda.stream(side_stream):
+                # after the previous backward (dE/dC and the backward workspace
+                # are free) and after this step's inputs have arrived
+                side_stream.wait_stream(stream)
+                if prepare:
+                    L.backward_prepare(Cb, N, ws_b, stream=side_stream, **gkw)
+                if overlap_zero:
+                    dE.zero_()
+                    dC.zero_()
+                side_done.record(side_stream)
         L.forward(Eb, Cb, yb, IGN, workspace=ws_f, out=(loss, lse))
-        if overlap_zero:
-            stream.wait_event(grads_zeroed)
-            L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC), accumulate=True, **gkw)
-            grads_free.record(stream)
-        else:
-            L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC), **gkw)
+        if overlap_zero or prepare:
+            stream.wait_event(side_done)
+        L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC), accumulate=overlap_zero,
+                   prepared=prepare, **gkw)
 
     def step():
         fwd_bwd(E, C, y, dloss)
@@ -411,6 +419,36 @@ def run_gpu(args, w):
     fwd_ms = float(np.mean([a.elapsed_time(b) for a, b in ev[0]]))
     bwd_ms = float(np.mean([a.elapsed_time(b) for a, b in ev[1]]))
     step_ms = 1e3 * sec / K
+
+    # ---- the dense backward (filter off), outside the timed region ----
+    # Every 32 x 32 unit is live: recompute of every logit tile plus both
+    # full contractions, 6 N D V flops.  This is the path of a head whose
+    # softmax is not sparse (a trained model); timed per launch through the
+    # kernel-event hook on the same inputs.
+    dense = None
+    if not args.no_dense and not (args.deterministic or args.bf16_grads):
+        ws_d = L.Workspace(dev)
+        evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
+        L.backward(E, C, y, lse, dloss, 0.0, IGN, workspace=ws_d, out=(dE, dC))   # warm-up
+        for a_, b_ in evd:
+            a_.record(stream)
+            b_.record(stream)
+        torch.cuda.synchronize()
+        clocks_d = ClockSampler(local)
+        clocks_d.start()
+        time.sleep(0.3)
+        for a_, b_ in evd:
+            L.cce_debug_set_kernel_events(1, a_.cuda_event, b_.cuda_event)
+            L.backward(E, C, y, lse, dloss, 0.0, IGN, workspace=ws_d, out=(dE, dC))
+        torch.cuda.synchronize()
+        L.cce_debug_set_kernel_events(1, 0, 0)
+        clk_d = clocks_d.stop()
+        std = L.read_status(ws_d)
+        dense = {"ms": float(np.mean([a_.elapsed_time(b_) for a_, b_ in evd])), "launches": len(evd),
+                 "flop_per_launch": 6.0 * N * D * V, "status": std["status"],
+                 "live_units": std["live_tiles"], "logit_tiles_recomputed": std["logit_tiles"],
+                 "clocks": {"sm_mhz": clk_d["sm_mhz"], "reasons": clk_d["reasons"]}}
+        del ws_d
 
     # ---- end to end through the public API with host buffers ----
     # Every step copies its inputs (E, C, y, dloss) from pinned host memory
@@ -482,11 +520,19 @@ def run_gpu(args, w):
     fwd_name = "fwd_lse_pair_kernel" if args.fwd_variant == "pair" else "fwd_lse_kernel"
     dominant = "bwd_kernel" if bwd_ms >= fwd_ms else fwd_name
     dom_flop, dom_ms = (flop_bwd, bwd_ms) if dominant == "bwd_kernel" else (flop_fwd, fwd_ms)
-    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    # The timed region is well under a second of work per launch, so the
+    # kernels are held to the burst figure; the sustained one (a seconds-long
+    # cuBLAS loop that settles at a lower clock under the power cap) is
+    # reported beside it, with the SM clock sampled during the timed region.
+    peak = float(peaks["bf16_tflops"])
+    peak_sus = float(peaks.get("bf16_tflops_sustained") or peak)
     achieved = dom_flop / (dom_ms * 1e-3) / 1e12
     traffic = ncu_traffic(dominant, w.name)
     executed_flop = flop_fwd + flop_bwd
-    nominal_flop = 6.0 * N * D * V
+    if dense is not None:
+        dense["tflops"] = dense["flop_per_launch"] / dense["ms"] / 1e9
+        dense["frac_of_burst_peak"] = dense["tflops"] / peak
+        dense["frac_of_sustained_peak"] = dense["tflops"] / peak_sus
 
     out = None
     if rank == 0:
@@ -502,17 +548,26 @@ def run_gpu(args, w):
                            grad_dtype="bf16" if args.bf16_grads else "fp32",
                            grad_zeroing=("side stream during the forward; backward accumulates (CCE_BWD_ACCUMULATE)"
                                          if overlap_zero else "inside the backward call"),
+                           classifier_norm=("cce_backward_prepare on the side stream during the forward"
+                                            if prepare else "inside the backward call"),
                            l2_prefetch_slices=list(args.prefetch) if args.prefetch else [0, 0]),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                         "peak_source": f"{peak_src} bf16_tflops (burst: the timed region is under a second)",
+                         "frac_sustained": achieved / peak_sus, "peak_sustained": peak_sus,
+                         "sm_mhz_median": clk["sm_mhz"],
                          "flop_per_launch": dom_flop, "launch_ms": dom_ms},
-            "kernels": {fwd_name: {"ms": fwd_ms, "tflops": flop_fwd / fwd_ms / 1e9},
+            "kernels": {fwd_name: {"ms": fwd_ms, "tflops": flop_fwd / fwd_ms / 1e9,
+                                   "frac_of_burst_peak": flop_fwd / fwd_ms / 1e9 / peak},
                         "bwd_kernel": {"ms": bwd_ms, "tflops": flop_bwd / bwd_ms / 1e9,
+                                       "frac_of_burst_peak": flop_bwd / bwd_ms / 1e9 / peak,
                                        "live_units": live, "dead_units": dead, "pruned_units": pruned,
-                                       "logit_tiles_recomputed": recomputed}},
+                                       "logit_tiles_recomputed": recomputed},
+                        "bwd_dense": dense},
+            # flops the tensor cores executed in a step (forward, recomputed
+            # tiles, live units' contractions) over the step time, against the
+            # burst peak; pruned units are not counted
             "pct_bf16_peak_executed": executed_flop / (step_ms * 1e-3) / 1e12 / peak,
-            "pct_bf16_peak_nominal_6NDV": nominal_flop / (step_ms * 1e-3) / 1e12 / peak,
             "filter_unit": list(FU),
             "live_unit_frac": live / max(1, live + dead + pruned),
             "extra_hbm_bytes": int(extra_hbm),
@@ -666,7 +721,7 @@ def run_suite(args):
     from linear_cross_entropy_05_b200 import synth
     dev = torch.device("cuda", 0)
     peaks, _ = measured_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    peak = float(peaks["bf16_tflops"])   # burst: every call here is timed alone
     cases = [synth.TINY, synth.GEMMA2_2B, synth.LLAMA3_8B, synth.SMALL_LARGE_VOCAB,
              synth.SMALL_LARGE_VOCAB.__class__(**{**synth.SMALL_LARGE_VOCAB.__dict__, "filter_eps": 0.0,
                                                    "name": "small-model-large-vocab[filter off]"})] + \
@@ -702,7 +757,7 @@ def run_suite(args):
             "fwd_ms": tf, "fwd_tokens_per_s": N / tf * 1e3, "fwd_frac_of_peak": 2.0 * N * D * V / tf / 1e9 / peak,
             "fwd_bwd_ms": tf + tb, "fwd_bwd_tokens_per_s": N / (tf + tb) * 1e3,
             "executed_frac_of_peak": executed / (tf + tb) / 1e9 / peak,
-            "nominal_6NDV_frac_of_peak": 6.0 * N * D * V / (tf + tb) / 1e9 / peak,
+            "bwd_ms": tb, "bwd_executed_frac_of_peak": (executed - 2.0 * N * D * V) / tb / 1e9 / peak,
             "tiles": {k: st[k] for k in ("live_tiles", "dead_tiles", "pruned_tiles", "logit_tiles")},
             "extra_hbm_bytes": {"forward_workspace": wsf.buf.numel(), "backward_workspace": wsb.buf.numel()},
             "materialised_logits_fp32_bytes": N * V * 4, "peak_tflops": peak}), flush=True)
@@ -735,6 +790,10 @@ def main(argv=None):
     ap.add_argument("--bf16-grads", action="store_true", help="bf16 dE/dC outputs (fixed-point accumulation)")
     ap.add_argument("--no-overlap-zero", action="store_true",
                     help="let the backward zero dE/dC itself instead of a side stream during the forward")
+    ap.add_argument("--no-prepare", action="store_true",
+                    help="let the backward compute max_v |C_v| itself instead of cce_backward_prepare on the side "
+                         "stream during the forward")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense (filter-off) backward measurement")
     ap.add_argument("--fwd-variant", choices=["single", "pair"], default="pair",
                     help="forward kernel: CTA pairs (default) or single CTAs (A/B measurement)")
     ap.add_argument("--prefetch", type=int, nargs=2, default=None, metavar=("FWD", "BWD"),

@@ -22,7 +22,8 @@ import os
 from typing import Optional, Tuple
 
 from . import _native
-from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCEError, cce_backward, cce_backward_ex,
+from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCE_BWD_PREPARED, CCEError,
+                      cce_backward, cce_backward_ex, cce_backward_prepare,
                       cce_backward_shard, cce_backward_workspace_size, cce_backward_workspace_size_ex,
                       cce_forward_shard, cce_merge_shards, cce_debug_forward_logits,
                       cce_debug_set_backward_trace, cce_debug_set_backward_variant, cce_debug_set_prefetch, cce_debug_set_forward_variant, cce_debug_set_kernel_events, cce_debug_set_wait_limit_ns,
@@ -33,7 +34,8 @@ from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINIS
 IGNORE_INDEX = -100
 
 __all__ = [
-    "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "CCE_BWD_ACCUMULATE", "cce_forward",
+    "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "CCE_BWD_ACCUMULATE",
+    "CCE_BWD_PREPARED", "cce_backward_prepare", "backward_prepare", "cce_forward",
     "cce_forward_noalloc", "cce_backward", "cce_backward_ex", "cce_backward_workspace_size_ex",
     "cce_forward_shard", "cce_merge_shards", "cce_backward_shard", "forward_shard", "merge_shards",
     "backward_shard", "vocab_parallel_forward_backward", "cce_forward_workspace_size",
@@ -106,14 +108,29 @@ def forward(E, C, y, ignore_index: int = IGNORE_INDEX, workspace: Optional[Works
     return loss, lse
 
 
+def backward_prepare(C, N: int, workspace: Workspace, deterministic: bool = False, bf16_grads: bool = False,
+                     stream=None):
+    """The classifier-only part of the backward's pre-pass (max_v |C_v|) into
+    `workspace`, sized for the backward call that will use it; that call then
+    passes prepared=True.  Can run on another stream while the forward runs."""
+    torch = _torch()
+    if C.dtype != torch.bfloat16 or not C.is_cuda or not C.is_contiguous() or C.dim() != 2:
+        raise ValueError("C must be a contiguous CUDA bfloat16 tensor [V, D]")
+    V, D = C.shape
+    flags = (CCE_BWD_DETERMINISTIC if deterministic else 0) | (CCE_BWD_BF16_GRADS if bf16_grads else 0)
+    ws = workspace.get(cce_backward_workspace_size_ex(N, D, V, flags))
+    cce_backward_prepare(C.data_ptr(), N, D, V, ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+
+
 def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = IGNORE_INDEX,
              workspace: Optional[Workspace] = None, stream=None, out=None, deterministic: bool = False,
-             bf16_grads: bool = False, accumulate: bool = False):
+             bf16_grads: bool = False, accumulate: bool = False, prepared: bool = False):
     """dE [N, D] and dC [V, D] of sum_i dloss[i] * loss[i]: fp32, or bf16 with
     bf16_grads; deterministic=True gives bitwise reproducible gradients
     (fixed-point accumulation, extra (N + V) * D * 8 bytes of workspace).
     accumulate=True adds them to the tensors given in `out` (required)
-    instead of overwriting them."""
+    instead of overwriting them.  prepared=True: backward_prepare already ran
+    on `workspace` for this C."""
     torch = _torch()
     _check_inputs(E, C, y)
     N, D = E.shape
@@ -122,7 +139,9 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
         if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.shape != (N,):
             raise ValueError(f"{n} must be a contiguous CUDA float32 tensor of shape [N]")
     flags = ((CCE_BWD_DETERMINISTIC if deterministic else 0) | (CCE_BWD_BF16_GRADS if bf16_grads else 0) |
-             (CCE_BWD_ACCUMULATE if accumulate else 0))
+             (CCE_BWD_ACCUMULATE if accumulate else 0) | (CCE_BWD_PREPARED if prepared else 0))
+    if prepared and workspace is None:
+        raise ValueError("prepared=True needs the workspace that backward_prepare filled")
     if accumulate and out is None:
         raise ValueError("accumulate=True adds into existing gradients: pass them as out=(dE, dC)")
     gdt = torch.bfloat16 if bf16_grads else torch.float32

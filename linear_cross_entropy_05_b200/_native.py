@@ -54,6 +54,8 @@ def load_library():
         lib.cce_backward_ex.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, ctypes.c_uint,
                                         c_vp, c_vp, c_vp, c_size, c_vp]
         lib.cce_backward_ex.restype = ctypes.c_int
+        lib.cce_backward_prepare.argtypes = [c_vp, c_i64, c_i64, c_i64, c_vp, c_size, c_vp]
+        lib.cce_backward_prepare.restype = ctypes.c_int
         lib.cce_forward_shard.argtypes = [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_size,
                                           c_vp]
         lib.cce_forward_shard.restype = ctypes.c_int
@@ -144,6 +146,15 @@ def cce_backward(E: int, C: int, y: int, lse: int, dloss: int, N: int, D: int, V
 CCE_BWD_DETERMINISTIC = 1
 CCE_BWD_BF16_GRADS = 2
 CCE_BWD_ACCUMULATE = 4
+CCE_BWD_PREPARED = 8
+
+
+def cce_backward_prepare(C: int, N: int, D: int, V: int, workspace: int, workspace_bytes: int, stream: int,
+                         check: bool = True) -> int:
+    st = load_library().cce_backward_prepare(C, N, D, V, workspace, workspace_bytes, stream)
+    if check:
+        _check(st, "cce_backward_prepare")
+    return st
 
 
 def cce_backward_workspace_size_ex(N: int, D: int, V: int, flags: int) -> int:

@@ -28,7 +28,8 @@ cudaError_t launch_bwd(const CUtensorMap& tmE, const CUtensorMap& tmC, const CUt
                        const CUtensorMap& tmdC, const BwdArgs& a, int grid, int variant, cudaStream_t stream);
 cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
                         int sms, cudaStream_t stream);
-cudaError_t launch_norms(const void* E, const void* C, const PrepArgs& p, int sms, cudaStream_t stream);
+cudaError_t launch_cnorm(const void* C, const PrepArgs& p, int sms, cudaStream_t stream);
+cudaError_t launch_enorm(const void* E, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
                                 bool bf16, bool accumulate, int sms, cudaStream_t stream);
@@ -190,7 +191,7 @@ struct BwdPlan {
   size_t off_accE, off_accC;  // fixed-point accumulators (deterministic mode only)
 };
 
-constexpr unsigned kBwdFlagsAll = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE;
+constexpr unsigned kBwdFlagsAll = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE | CCE_BWD_PREPARED;
 constexpr unsigned kBwdFixedPoint = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS;  // int64 accumulators
 
 bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags = 0) {
@@ -388,8 +389,16 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   unsigned long long* accE = fixed ? reinterpret_cast<unsigned long long*>(ws + bp.off_accE) : nullptr;
   unsigned long long* accC = fixed ? reinterpret_cast<unsigned long long*>(ws + bp.off_accC) : nullptr;
   const bool filter_on = filter_eps > 0.f;
-  if (cudaMemsetAsync(ws, 0, (filter_on || fixed) ? bp.zero_bytes : STATUS_BYTES, stream) != cudaSuccess)
+  const bool prepared = (flags & CCE_BWD_PREPARED) != 0;
+  if (prepared && (filter_on || fixed)) {
+    // keep max_v |C_v| (header word HDR_CMAX) from cce_backward_prepare
+    const size_t keep0 = bp.off_hdr + HDR_CMAX * sizeof(unsigned), keep1 = keep0 + sizeof(unsigned);
+    if (cudaMemsetAsync(ws, 0, keep0, stream) != cudaSuccess ||
+        cudaMemsetAsync(ws + keep1, 0, bp.zero_bytes - keep1, stream) != cudaSuccess)
+      return CCE_ERR_CUDA;
+  } else if (cudaMemsetAsync(ws, 0, (filter_on || fixed) ? bp.zero_bytes : STATUS_BYTES, stream) != cudaSuccess) {
     return CCE_ERR_CUDA;
+  }
   if (fixed) {
     if (cudaMemsetAsync(accE, 0, (size_t)N * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
@@ -448,7 +457,8 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     pp.list = reinterpret_cast<int2*>(ws + bp.off_list);
     pp.enorm = reinterpret_cast<float*>(ws + bp.off_enorm);
     pp.status = status;
-    if (launch_norms(E, C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (!prepared && launch_cnorm(C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (launch_enorm(E, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (filter_on && launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (fixed && launch_fixed_prep(dloss, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
   }
@@ -489,6 +499,29 @@ cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const 
                           float* dC, void* workspace, size_t workspace_bytes, void* stream) {
   return backward_impl(E, C, y, lse, dloss, N, D, V, ignore_index, filter_eps, 0u, dE, dC, workspace,
                        workspace_bytes, stream);
+}
+
+cce_status_t cce_backward_prepare(const void* C, int64_t N, int64_t D, int64_t V, void* workspace,
+                                  size_t workspace_bytes, void* stream_) {
+  if (!C || !workspace) return CCE_ERR_INVALID_ARG;
+  if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
+  if (!aligned(C, 16) || !aligned(workspace, 256)) return CCE_ERR_MISALIGNED;
+  BwdPlan bp;
+  if (!plan_backward(N, D, V, &bp)) return CCE_ERR_INVALID_ARG;
+  DeviceInfo di = device_info();
+  if (!di.ok) return CCE_ERR_UNSUPPORTED_DEVICE;
+  if (workspace_bytes < bp.ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  char* ws = reinterpret_cast<char*>(workspace);
+  unsigned* hdr = reinterpret_cast<unsigned*>(ws + bp.off_hdr);
+  if (cudaMemsetAsync(hdr + HDR_CMAX, 0, sizeof(unsigned), stream) != cudaSuccess) return CCE_ERR_CUDA;
+  PrepArgs pp{};
+  pp.N = (int)N;
+  pp.D = (int)D;
+  pp.V = (int)V;
+  pp.hdr = hdr;
+  if (launch_cnorm(C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  return CCE_OK;
 }
 
 cce_status_t cce_forward_shard(const void* E, const void* C_shard, const int64_t* y, int64_t N, int64_t D,

@@ -257,17 +257,22 @@ cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t
   return cudaGetLastError();
 }
 
-// Norm pre-pass shared by the filter and the fixed-point scale: max_v |C_v|,
-// |E_i| per token and max_i |E_i|.
-cudaError_t launch_norms(const void* E, const void* C, const PrepArgs& p, int sms, cudaStream_t stream) {
+// Norm pre-pass shared by the filter and the fixed-point scale: max_v |C_v|
+// (launch_cnorm; HDR_CMAX must start at zero), |E_i| per token and
+// max_i |E_i| (launch_enorm).
+cudaError_t launch_cnorm(const void* C, const PrepArgs& p, int sms, cudaStream_t stream) {
   prep_cnorm_kernel<<<sms * 8, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(C), p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_enorm(const void* E, const PrepArgs& p, int sms, cudaStream_t stream) {
   prep_enorm_kernel<<<sms * 4, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E), p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const float* lse, const PrepArgs& p,
                         int sms, cudaStream_t stream) {
-  // expects launch_norms to have run
+  // expects launch_cnorm and launch_enorm to have run
   prep_blocks_kernel<<<p.n_mblk, 128, 0, stream>>>(y, lse, p);
   prep_scan_kernel<<<1, 1024, 0, stream>>>(p);
   prep_scatter_kernel<<<p.n_mblk, 128, 0, stream>>>(y, p);

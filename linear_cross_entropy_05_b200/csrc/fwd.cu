@@ -473,6 +473,24 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const __nv_bfloat16* 
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= a.N) return;
 
+  // A bounded wait of the logit kernel gave up: some partials were never
+  // written (the workspace may hold an earlier call's values), so every
+  // output of this call is NaN rather than a plausible wrong number.
+  if (a.status[ST_FLAGS] & SF_TIMEOUT) {
+    if (lane == 0) {
+      const float qnan = __int_as_float(0x7fc00000);
+      if (a.shard_stats) {
+        a.shard_stats[row] = qnan;
+        a.shard_stats[(size_t)a.N + row] = qnan;
+        a.shard_stats[2 * (size_t)a.N + row] = qnan;
+      } else {
+        lse[row] = qnan;
+        loss[row] = qnan;
+      }
+    }
+    return;
+  }
+
   // merge the per-split (max, sum) pairs: lse = M + log(sum_r s_r exp(m_r - M))
   float M = -INFINITY;
   for (int r = lane; r < a.n_split; r += 32) M = fmaxf(M, a.partial[(size_t)r * a.N + row].x);

@@ -23,25 +23,55 @@ constexpr size_t kNoallocScratchBytes = size_t(8) << 20;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-// Device address of the array, looked up once per device.  The name
-// g_noalloc_scratch is only a host-side stand-in in host code: a kernel given
-// &g_noalloc_scratch would fault (or, where the GPU can reach host memory,
-// silently use the wrong memory), so the address comes from
-// cudaGetSymbolAddress with the device current.
+// Device address of the array, looked up once per device and CUDA context.
+// The name g_noalloc_scratch is only a host-side stand-in in host code: a
+// kernel given &g_noalloc_scratch would fault (or, where the GPU can reach
+// host memory, silently use the wrong memory), so the address comes from
+// cudaGetSymbolAddress with the device current.  The cached address belongs
+// to the context the module was loaded into: when the device's current
+// context is another one (after cudaDeviceReset, or a context the caller
+// created), the module is loaded anew there and the address is looked up
+// again.
 struct ScratchSlot {
-  std::once_flag once;
+  std::mutex mu;
+  void* ctx = nullptr;  // context the cached address belongs to
   void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
 };
 constexpr int kMaxDevices = 64;
 ScratchSlot g_slots[kMaxDevices];
 
+typedef int (*CtxGetCurrentFn)(void**);  // CUresult cuCtxGetCurrent(CUcontext*)
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 cce_status_t device_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CCE_ERR_CUDA;
+  // make the device's primary context current (cudaSetDevice initialises
+  // it if needed), then identify it
+  if (cudaSetDevice(dev) != cudaSuccess) return CCE_ERR_CUDA;
+  CtxGetCurrentFn get = ctx_get_current();
+  void* ctx = nullptr;
+  if (!get || get(&ctx) != 0 || ctx == nullptr) return CCE_ERR_CUDA;
   ScratchSlot& s = g_slots[dev];
-  std::call_once(s.once, [&s] { s.err = cudaGetSymbolAddress(&s.ptr, g_noalloc_scratch); });
-  if (s.err != cudaSuccess || s.ptr == nullptr) return CCE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(s.mu);
+  if (s.ptr == nullptr || s.ctx != ctx) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return CCE_ERR_CUDA;
+    s.ptr = p;
+    s.ctx = ctx;
+  }
   *out = s.ptr;
   return CCE_OK;
 }

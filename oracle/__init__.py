@@ -232,11 +232,12 @@ def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
             for k in np.nonzero((rows_dE >= b0) & (rows_dE < b1))[0]:
                 out_dE[k] = np.where(mask, G[int(rows_dE[k]) - b0], 0.0) @ C64
     else:
-        for k, i in enumerate(rows_dE):
-            z = logits(E64[int(i):int(i) + 1], C64)
-            _, _, G = softmax_grad_f64(z, lse_all[int(i):int(i) + 1], y[int(i):int(i) + 1],
-                                       dloss[int(i):int(i) + 1], ignore_index)
-            out_dE[k] = G[0] @ C64
+        # the requested rows, a few at a time (one matrix product per group)
+        for k0 in range(0, rows_dE.shape[0], 64):
+            sel = rows_dE[k0:k0 + 64]
+            z = logits(E64[sel], C64)
+            _, _, G = softmax_grad_f64(z, lse_all[sel], y[sel], dloss[sel], ignore_index)
+            out_dE[k0:k0 + sel.shape[0]] = G @ C64
 
     # dC rows: the column v of G over all tokens.  With filtering, the column
     # tile of v must be evaluated in full for each token block.

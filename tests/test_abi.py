@@ -145,14 +145,25 @@ def test_backward_ex_workspace_and_flags(lib):
     for flags in (1, 2, 3, 5, 6, 7):   # deterministic / bf16 outputs: int64 accumulators for dE and dC
         assert cce_backward_workspace_size_ex(N, D, V, flags) == base + up(8 * N * D) + up(8 * V * D)
     assert cce_backward_workspace_size_ex(N, D, V, 4) == base   # accumulate alone: no extra workspace
-    assert cce_backward_workspace_size_ex(N, D, V, 8) == 0   # unknown flag
+    assert cce_backward_workspace_size_ex(N, D, V, 8) == base   # prepared: no extra workspace
+    assert cce_backward_workspace_size_ex(N, D, V, 16) == 0     # unknown flag
     P = 1 << 20
     args = [P, P, P, P, P, 256, 256, 4096, -100, 0.0, 0, P, P, P, 1 << 30, 0]
-    args[10] = 8
+    args[10] = 16
     assert cce_backward_ex(*args, check=False) == 1          # unknown flag: rejected on the host
-    for flags in (3, 4, 7):
+    for flags in (3, 4, 7, 8, 15):
         args[10] = flags
         assert cce_backward_ex(*args, check=False) == 4      # valid, but no device here
+
+
+def test_backward_prepare_validates_on_the_host(lib):
+    _cpu_only()
+    from linear_cross_entropy_05_b200 import cce_backward_prepare
+    P = 1 << 20
+    assert cce_backward_prepare(0, 256, 256, 4096, P, 1 << 30, 0, check=False) == 1        # null C
+    assert cce_backward_prepare(P, 256, 260, 4096, P, 1 << 30, 0, check=False) == 1        # D % 8 != 0
+    assert cce_backward_prepare(P + 8, 256, 256, 4096, P, 1 << 30, 0, check=False) == 2    # misaligned C
+    assert cce_backward_prepare(P, 256, 256, 4096, P, 1 << 30, 0, check=False) == 4        # valid, no device
 
 
 def test_shard_entry_points_validate_on_the_host(lib):

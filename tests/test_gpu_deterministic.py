@@ -129,3 +129,34 @@ def test_accumulate_adds_this_calls_gradients(mode):
     else:
         for a, r, g in ((aE, rE, gE), (aC, rC, gC)):
             assert rel_fro((a - r).cpu().numpy(), g.cpu().numpy()) < 1e-5
+
+
+@pytest.mark.parametrize("eps", [0.0, synth.EPS_BF16_FILTER])
+def test_prepared_backward_equals_unprepared(eps):
+    """cce_backward_prepare on a second stream while the forward runs, then
+    the backward with CCE_BWD_PREPARED: the same bits (deterministic mode) and
+    the same filter counters as a backward that computes max_v |C_v| itself."""
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=900, V=20000)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    dl = torch.from_numpy(synth.random_dloss(5, w.N)).cuda()
+    ws_f, ws_a, ws_b = L.Workspace(), L.Workspace(), L.Workspace()
+    side = torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    ready = torch.cuda.Event()
+    side.wait_stream(main)
+    L.backward_prepare(C, w.N, ws_b, deterministic=True, stream=side)
+    ready.record(side)
+    loss, lse = L.forward(E, C, y, IGN, workspace=ws_f)
+    main.wait_event(ready)
+    dE_p, dC_p = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws_b, deterministic=True, prepared=True)
+    st_p = L.read_status(ws_b)
+    dE, dC = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws_a, deterministic=True)
+    st = L.read_status(ws_a)
+    assert st_p["status"] == 0 and st["status"] == 0
+    for k in ("live_tiles", "dead_tiles", "pruned_tiles", "logit_tiles"):
+        assert st_p[k] == st[k]
+    assert torch.equal(dE_p.view(torch.int32), dE.view(torch.int32))
+    assert torch.equal(dC_p.view(torch.int32), dC.view(torch.int32))

@@ -34,9 +34,11 @@ def test_withheld_loads_end_with_timeout_status_and_a_usable_context():
         for variant in (0, 1):   # single-CTA and CTA-pair forward kernels
             L.cce_debug_set_forward_variant(variant)
             ws = L.Workspace()
-            L.forward(E, C, y, IGN, workspace=ws)
+            l_t, s_t = L.forward(E, C, y, IGN, workspace=ws)
             st = L.read_status(ws)
             assert st["status"] == CCE_ERR_TIMEOUT and st["flags"] & 1
+            # partials were never written: the call's outputs are NaN, not stale values
+            assert torch.isnan(l_t).all() and torch.isnan(s_t).all()
         L.cce_debug_set_forward_variant(DEFAULT_FWD_VARIANT)
         for eps in (0.0, 2.0 ** -12):
             ws = L.Workspace()

@@ -260,6 +260,63 @@ def test_tile_filter_against_brute_force(eps):
     np.testing.assert_allclose(dC, dC_b, rtol=1e-12, atol=1e-14)
 
 
+def _decode_bits(bits):
+    # bf16 is the upper half of an fp32 (decoding pinned by test_bf16_decode_known_patterns)
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def _tile_map_case():
+    rng = np.random.default_rng(21)
+    N, D, V, Bn, Bv = 13, 3, 19, 2, 3          # ragged in both directions
+    E_bits = _bits(rng.standard_normal((N, D)) * 3.0)
+    C_bits = _bits(rng.standard_normal((V, D)) * 3.0)
+    y = rng.integers(0, V, N)
+    y[[2, 9]] = IGN
+    return E_bits, C_bits, y, Bn, Bv
+
+
+@pytest.mark.parametrize("rows_per_block", [None, 1, 5])
+@pytest.mark.parametrize("eps", [0.03, 0.1])
+def test_tile_live_map_against_brute_force(monkeypatch, rows_per_block, eps):
+    """oracle.tile_live_map (bf16 inputs, the caller's lse) against a
+    brute-force enumeration of |P - onehot| >= eps per tile; rows_per_block
+    forces the oracle's row blocking to cut the rows every 2 or 4 tokens (not
+    only at the end), so a wrong block boundary shows."""
+    E_bits, C_bits, y, Bn, Bv = _tile_map_case()
+    E, C = _decode_bits(E_bits), _decode_bits(C_bits)
+    lse_b, live_b, _, _ = _brute_filtered(E, C, y, np.ones(len(y)), eps, Bn, Bv)
+    if rows_per_block is not None:
+        monkeypatch.setattr(oracle, "_rows_per_block", lambda V, budget_elems=0: rows_per_block)
+    live = oracle.tile_live_map(E_bits, C_bits, y, lse_b, IGN, eps, tile=(Bn, Bv))
+    assert live.shape == live_b.shape == (7, 7)
+    assert (live == live_b).all()
+    assert 0 < live.sum() < live.size
+
+
+@pytest.mark.parametrize("mutation", ["scaled_difference", "rows_shifted", "columns_shifted"])
+def test_tile_live_map_pin_catches_planted_mistakes(monkeypatch, mutation):
+    E_bits, C_bits, y, Bn, Bv = _tile_map_case()
+    E, C = _decode_bits(E_bits), _decode_bits(C_bits)
+    eps = 0.03
+    lse_b, live_b, _, _ = _brute_filtered(E, C, y, np.ones(len(y)), eps, Bn, Bv)
+    real_sg = oracle.softmax_grad_f64
+    real_map = oracle.tile_live_map_f64
+    if mutation == "scaled_difference":     # liveness decided on dloss-scaled entries (dloss = 0.3)
+        monkeypatch.setattr(oracle, "softmax_grad_f64",
+                            lambda z, lse, yy, dl, ign: tuple(x * (0.3 if k else 1.0)
+                                                               for k, x in enumerate(real_sg(z, lse, yy, dl, ign))))
+    elif mutation == "rows_shifted":        # tile rows anchored one token late
+        monkeypatch.setattr(oracle, "tile_live_map_f64",
+                            lambda Dm, r0, bn, bv, e: real_map(np.vstack([np.zeros((1, Dm.shape[1])), Dm])[:-1],
+                                                               r0, bn, bv, e))
+    elif mutation == "columns_shifted":     # vocabulary tiles anchored one column late
+        monkeypatch.setattr(oracle, "tile_live_map_f64",
+                            lambda Dm, r0, bn, bv, e: real_map(np.hstack([np.zeros((Dm.shape[0], 1)), Dm])[:, :-1],
+                                                               r0, bn, bv, e))
+    live = oracle.tile_live_map(E_bits, C_bits, y, lse_b, IGN, eps, tile=(Bn, Bv))
+    assert live.shape != live_b.shape or not (live == live_b).all(), f"{mutation} went unnoticed"
+
+
 def test_sampled_backward_matches_full():
     w = synth.TINY.with_sizes(N=300, V=1000, D=64)
     inp = synth.make_inputs(w)
