@@ -87,6 +87,29 @@ def aggregate_throughput(dist, tokens_local: float, seconds_local: float, device
     return tok / tmax, tmax
 
 
+def aggregate_shared_batch(dist, tokens: float, seconds_local: float, device):
+    """Throughput of one batch processed jointly by all ranks (the
+    vocabulary-parallel mode: every rank works on the same tokens, each on
+    its classifier shard): tokens / max time over ranks."""
+    tmax = reduce_max(dist, seconds_local, device)
+    return tokens / tmax, tmax
+
+
+def vocab_shard(V: int, world: int, rank: int, tile: int = 256):
+    """Contiguous classifier shard [v_offset, v_offset + V_shard) of `rank`:
+    whole 256-row vocabulary tiles dealt as evenly as possible (the first
+    V_tiles % world ranks get one tile more), the ragged last tile with the
+    last rank."""
+    n_t = -(-V // tile)
+    if n_t < world:
+        raise ValueError(f"{V} vocabulary rows make {n_t} tiles: fewer than the {world} ranks")
+    base, extra = divmod(n_t, world)
+    t0 = rank * base + min(rank, extra)
+    t1 = t0 + base + (1 if rank < extra else 0)
+    v0, v1 = min(V, t0 * tile), min(V, t1 * tile)
+    return v0, v1 - v0
+
+
 # ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
@@ -429,7 +452,8 @@ def run_gpu(args, w):
     if not args.no_dense and not (args.deterministic or args.bf16_grads):
         ws_d = L.Workspace(dev)
         evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
-        L.backward(E, C, y, lse, dloss, 0.0, IGN, workspace=ws_d, out=(dE, dC))   # warm-up
+        stripes = not args.dense_fused
+        L.backward(E, C, y, lse, dloss, 0.0, IGN, workspace=ws_d, out=(dE, dC), stripes=stripes)   # warm-up
         for a_, b_ in evd:
             a_.record(stream)
             b_.record(stream)
@@ -439,12 +463,15 @@ def run_gpu(args, w):
         time.sleep(0.3)
         for a_, b_ in evd:
             L.cce_debug_set_kernel_events(1, a_.cuda_event, b_.cuda_event)
-            L.backward(E, C, y, lse, dloss, 0.0, IGN, workspace=ws_d, out=(dE, dC))
+            L.backward(E, C, y, lse, dloss, 0.0, IGN, workspace=ws_d, out=(dE, dC), stripes=stripes)
         torch.cuda.synchronize()
         L.cce_debug_set_kernel_events(1, 0, 0)
         clk_d = clocks_d.stop()
         std = L.read_status(ws_d)
-        dense = {"ms": float(np.mean([a_.elapsed_time(b_) for a_, b_ in evd])), "launches": len(evd),
+        dense = {"path": ("softmax-gradient stripes (CCE_BWD_STRIPES)" if stripes else
+                          "fused per-tile contractions with fp32 reduce-adds"),
+                 "workspace_bytes": int(ws_d.buf.numel()),
+                 "ms": float(np.mean([a_.elapsed_time(b_) for a_, b_ in evd])), "launches": len(evd),
                  "flop_per_launch": 6.0 * N * D * V, "status": std["status"],
                  "live_units": std["live_tiles"], "logit_tiles_recomputed": std["logit_tiles"],
                  "clocks": {"sm_mhz": clk_d["sm_mhz"], "reasons": clk_d["reasons"]}}
@@ -582,6 +609,77 @@ def run_gpu(args, w):
             "gpu_launches": launches_per_step(eps, args.deterministic or args.bf16_grads) * K,
             "clocks": clk,
             "cpu_baseline": cpu,
+        }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+def run_vocab_parallel(args, w):
+    """The vocabulary-parallel form on N ranks (one GPU each, NCCL): rank r
+    holds the classifier shard C[v_offset : v_offset + V_r] and runs
+    vocab_parallel_forward_backward on the whole batch (forward on its shard,
+    all-gather of 12 bytes per token, merge, backward on its shard,
+    all-reduce of the dE shares).  The batch is shared, so the throughput is
+    N tokens / max time over ranks ("scaling": "strong").  No TMA multicast:
+    every load of the kernels reads this GPU's own memory."""
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl")
+    import linear_cross_entropy_05_b200 as L
+    from linear_cross_entropy_05_b200 import synth
+    inp = synth.make_inputs(w)
+    N, D, V = w.N, w.D, w.V
+    v0, Vr = vocab_shard(V, world, rank)
+    E = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(dev)
+    C_sh = torch.from_numpy(inp["C"][v0:v0 + Vr].view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.from_numpy(inp["y"]).to(dev)
+    dloss = torch.from_numpy(synth.mean_dloss(inp["y"])).to(dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return L.vocab_parallel_forward_backward(E, C_sh, y, v0, V, dloss=dloss, filter_eps=w.filter_eps)
+
+    for _ in range(max(3, args.warmup)):
+        loss, lse, dE, dC = step()
+    torch.cuda.synchronize()
+    K = args.steps
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(K):
+        loss, lse, dE, dC = step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    value, sec = aggregate_shared_batch(dist, float(N * K), t0.elapsed_time(t1) / 1e3, dev)
+    finite = bool(torch.isfinite(loss).all())
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sec / K, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded numpy PCG64; random-init classifier, Zipf labels)",
+            "config": dict(config_of(w, world), parallelism=f"vocab{world}", global_batch=N,
+                           shard_rows=[vocab_shard(V, world, r)[1] for r in range(world)],
+                           collectives="all-gather of [3, N] fp32 shard statistics; all-reduce of dE (N x D fp32)"),
+            # per step: shard forward (logit kernel + finalize), the merge, and the
+            # shard backward's kernels (as in a one-GPU step)
+            "gpu_launches": (launches_per_step(w.filter_eps, False) + 1) * K,
+            "clocks": clk, "loss_finite": finite, "e2e": None, "cpu_baseline": None,
         }
     if dist is not None:
         dist.barrier()
@@ -794,6 +892,8 @@ def main(argv=None):
                     help="let the backward compute max_v |C_v| itself instead of cce_backward_prepare on the side "
                          "stream during the forward")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense (filter-off) backward measurement")
+    ap.add_argument("--dense-fused", action="store_true",
+                    help="measure the dense backward on the fused per-tile kernel instead of the stripe kernel")
     ap.add_argument("--fwd-variant", choices=["single", "pair"], default="pair",
                     help="forward kernel: CTA pairs (default) or single CTAs (A/B measurement)")
     ap.add_argument("--prefetch", type=int, nargs=2, default=None, metavar=("FWD", "BWD"),
@@ -802,6 +902,9 @@ def main(argv=None):
                     help="per-tile timeline of one backward launch (recompute wait, gradient tile, contraction)")
     ap.add_argument("--memory", action="store_true",
                     help="classifier-head training step: peak memory and time, CCE vs materialised logits")
+    ap.add_argument("--vocab-parallel", action="store_true",
+                    help="vocabulary-parallel form over the launched ranks (classifier sharded by rows, NCCL "
+                         "exchange) instead of independent replicas")
     ap.add_argument("--suite", action="store_true",
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
@@ -826,6 +929,8 @@ def main(argv=None):
         w = w.with_sizes(N=args.N, V=args.V)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.vocab_parallel:
+        return run_vocab_parallel(args, w)
     return run_gpu(args, w)
 
 

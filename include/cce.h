@@ -175,7 +175,23 @@ typedef enum {
    * N, D, V (e.g. on a second stream while the forward ran): the backward
    * skips its own pass over C and uses the stored max_v |C_v|.  Same result
    * as without the flag.  No extra workspace. */
-  CCE_BWD_PREPARED = 8
+  CCE_BWD_PREPARED = 8,
+  /* With filter_eps <= 0 (every unit kept: the exact gradient), run the
+   * dense backward through stripes of the softmax gradient: the vocabulary
+   * is taken 2048 rows at a time; per stripe the logit tiles are recomputed
+   * on chip and G = dloss (softmax - onehot) is stored in bf16 into one of
+   * three stripe buffers in the workspace, then dC of the stripe's rows =
+   * G^T E is formed with every token as the reduction dimension (each entry
+   * written once) and dE += G C of the stripe (one bulk reduce-add per
+   * 256 x 256 dE tile and stripe).  Only these stripes of G ever exist in
+   * global memory: 3 x min(N, 16384) x 2048 x 2 bytes (100 MB at N = 8192),
+   * whatever V; tokens beyond 16384 are taken in further launches whose dC
+   * contributions are added.  Far less fp32 reduction traffic than adding
+   * every logit tile's partial products, so the tensor cores set the pace.
+   * Same result as without the flag up to fp32 summation order.  Ignored
+   * when filter_eps > 0 or with the fixed-point flags.  Needs the workspace
+   * of cce_backward_workspace_size_ex with this flag. */
+  CCE_BWD_STRIPES = 16
 } cce_backward_flags_t;
 
 /* The part of the backward's pre-pass that depends on the classifier alone:

@@ -58,6 +58,17 @@ CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
  * Returns CCE_ERR_INVALID_ARG for tiles_per_cta outside [1, 2^20]. */
 CCE_API cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta);
 
+/* Host-only view of the task order of the stripe backward (CCE_BWD_STRIPES)
+ * for a launch of n_m2 256-token blocks, n_vtile 256-row vocabulary tiles,
+ * n_dc 256-wide d-chunks, vt_per_s tiles per stripe and nbuf stripe
+ * buffers: writes min(total + 1, max_tasks) task descriptors, four int32
+ * each (kind: -1 end, 0 recompute-and-store G, 1 dC tile, 2 dE tile;
+ * stripe; then (token block, vocabulary tile), (vocabulary tile, d-chunk)
+ * or (token block, d-chunk)), into out (host memory; may be NULL) and
+ * returns the number of tasks, or -1 for invalid sizes.  Runs no kernel. */
+CCE_API int64_t cce_debug_stripe_schedule(int n_m2, int n_vtile, int n_dc, int vt_per_s, int nbuf, int32_t* out,
+                                          int64_t max_tasks);
+
 /* Selects the forward logit/LSE kernel: 1 = CTA pairs (two SMs per 256 x 256
  * logit tile through tcgen05 cta_group::2, two thirds of the operand traffic
  * per SM; the default), 0 = one SM per 128 x 256 logit tile.  Both give the

@@ -22,7 +22,8 @@ import os
 from typing import Optional, Tuple
 
 from . import _native
-from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCE_BWD_PREPARED, CCEError,
+from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCE_BWD_PREPARED,
+                      CCE_BWD_STRIPES, CCEError, cce_debug_stripe_schedule,
                       cce_backward, cce_backward_ex, cce_backward_prepare,
                       cce_backward_shard, cce_backward_workspace_size, cce_backward_workspace_size_ex,
                       cce_forward_shard, cce_merge_shards, cce_debug_forward_logits,
@@ -35,7 +36,8 @@ IGNORE_INDEX = -100
 
 __all__ = [
     "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "CCE_BWD_ACCUMULATE",
-    "CCE_BWD_PREPARED", "cce_backward_prepare", "backward_prepare", "cce_forward",
+    "CCE_BWD_PREPARED", "CCE_BWD_STRIPES", "cce_debug_stripe_schedule", "cce_backward_prepare",
+    "backward_prepare", "cce_forward",
     "cce_forward_noalloc", "cce_backward", "cce_backward_ex", "cce_backward_workspace_size_ex",
     "cce_forward_shard", "cce_merge_shards", "cce_backward_shard", "forward_shard", "merge_shards",
     "backward_shard", "vocab_parallel_forward_backward", "cce_forward_workspace_size",
@@ -124,13 +126,17 @@ def backward_prepare(C, N: int, workspace: Workspace, deterministic: bool = Fals
 
 def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = IGNORE_INDEX,
              workspace: Optional[Workspace] = None, stream=None, out=None, deterministic: bool = False,
-             bf16_grads: bool = False, accumulate: bool = False, prepared: bool = False):
+             bf16_grads: bool = False, accumulate: bool = False, prepared: bool = False,
+             stripes: Optional[bool] = None):
     """dE [N, D] and dC [V, D] of sum_i dloss[i] * loss[i]: fp32, or bf16 with
     bf16_grads; deterministic=True gives bitwise reproducible gradients
     (fixed-point accumulation, extra (N + V) * D * 8 bytes of workspace).
     accumulate=True adds them to the tensors given in `out` (required)
     instead of overwriting them.  prepared=True: backward_prepare already ran
-    on `workspace` for this C."""
+    on `workspace` for this C.  stripes (default: on when filter_eps <= 0
+    and neither deterministic nor bf16_grads): the dense backward through
+    softmax-gradient stripes (CCE_BWD_STRIPES), which needs a larger
+    workspace (about 12 KB per token, at most ~200 MB)."""
     torch = _torch()
     _check_inputs(E, C, y)
     N, D = E.shape
@@ -140,6 +146,10 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
             raise ValueError(f"{n} must be a contiguous CUDA float32 tensor of shape [N]")
     flags = ((CCE_BWD_DETERMINISTIC if deterministic else 0) | (CCE_BWD_BF16_GRADS if bf16_grads else 0) |
              (CCE_BWD_ACCUMULATE if accumulate else 0) | (CCE_BWD_PREPARED if prepared else 0))
+    if stripes is None:
+        stripes = filter_eps <= 0 and not (deterministic or bf16_grads)
+    if stripes:
+        flags |= CCE_BWD_STRIPES
     if prepared and workspace is None:
         raise ValueError("prepared=True needs the workspace that backward_prepare filled")
     if accumulate and out is None:
@@ -153,6 +163,8 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
         if dE.dtype != gdt or dC.dtype != gdt:
             raise TypeError(f"dE and dC must be {gdt}")
     ws_bytes = cce_backward_workspace_size_ex(N, D, V, flags)
+    if prepared and (workspace.buf is None or workspace.buf.numel() < ws_bytes):
+        raise ValueError("prepared=True: the workspace backward_prepare filled is smaller than this call needs")
     ws = (workspace or Workspace(E.device)).get(ws_bytes)
     cce_backward_ex(E.data_ptr(), C.data_ptr(), y.data_ptr(), lse.data_ptr(), dloss.data_ptr(), N, D, V,
                     ignore_index, float(filter_eps), flags, dE.data_ptr(), dC.data_ptr(), ws.data_ptr(), ws.numel(),

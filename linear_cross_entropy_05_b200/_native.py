@@ -87,6 +87,8 @@ def load_library():
         lib.cce_debug_set_kernel_events.restype = ctypes.c_int
         lib.cce_debug_set_prefetch.argtypes = [ctypes.c_int, ctypes.c_int]
         lib.cce_debug_set_prefetch.restype = ctypes.c_int
+        lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 5 + [c_vp, c_i64]
+        lib.cce_debug_stripe_schedule.restype = c_i64
         lib.cce_debug_set_backward_trace.argtypes = [c_vp, c_i64]
         lib.cce_debug_set_backward_trace.restype = ctypes.c_int
         _lib = lib
@@ -147,6 +149,7 @@ CCE_BWD_DETERMINISTIC = 1
 CCE_BWD_BF16_GRADS = 2
 CCE_BWD_ACCUMULATE = 4
 CCE_BWD_PREPARED = 8
+CCE_BWD_STRIPES = 16
 
 
 def cce_backward_prepare(C: int, N: int, D: int, V: int, workspace: int, workspace_bytes: int, stream: int,
@@ -249,3 +252,16 @@ def cce_debug_set_backward_trace(trace: int, tiles_per_cta: int) -> None:
     buffer `trace` (u64 [SMs][tiles_per_cta][4]); trace = 0 turns it off."""
     _check(load_library().cce_debug_set_backward_trace(trace or None, int(tiles_per_cta)),
            "cce_debug_set_backward_trace")
+
+
+def cce_debug_stripe_schedule(n_m2: int, n_vtile: int, n_dc: int, vt_per_s: int, nbuf: int):
+    """Task order of the stripe backward (host-side decode, no kernel):
+    an int32 array [tasks + 1, 4] of (kind, stripe, a, b); kind -1 ends it."""
+    import numpy as np
+    lib = load_library()
+    total = int(lib.cce_debug_stripe_schedule(n_m2, n_vtile, n_dc, vt_per_s, nbuf, None, 0))
+    if total < 0:
+        raise CCEError(1, "cce_debug_stripe_schedule: invalid sizes")
+    out = np.zeros((total + 1, 4), dtype=np.int32)
+    lib.cce_debug_stripe_schedule(n_m2, n_vtile, n_dc, vt_per_s, nbuf, out.ctypes.data, total + 1)
+    return out

@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcce.so")
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "bwd_prep.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "bwd_prep.cu", "bwd_stripe.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "ptx.cuh"]
 INCLUDE = [os.path.join(ROOT, "include", "cce.h"), os.path.join(ROOT, "include", "cce_debug.h")]
 

@@ -31,6 +31,7 @@ cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const fl
 cudaError_t launch_cnorm(const void* C, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_enorm(const void* E, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream);
+cudaError_t launch_bwd_stripe(const CUtensorMap* maps, const StripeArgs& a, void* G, int grid, cudaStream_t stream);
 cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
                                 bool bf16, bool accumulate, int sms, cudaStream_t stream);
 }  // namespace cce
@@ -184,14 +185,54 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
 
 // Backward workspace: status | pre-pass header | count, offset, cursor
 // [n_vtile] | blk_flat, nonflat [n_mblk] | list [N] int2.  O(N + V/256).
+// Stripe backward (CCE_BWD_STRIPES, filter off): 256-token blocks per launch
+// (token super-block; dC gathers the super-blocks by reduce-adds) and
+// vocabulary tiles per stripe.
+constexpr int kStripeMaxM2 = 64;     // 16384 tokens per launch
+constexpr int kStripeVtiles = 8;     // 2048 vocabulary columns per stripe
+constexpr int kStripeBuffers = 3;
+
+struct StripeLayout {
+  StripePlan p;          // of a full super-block
+  int n_sb;              // super-blocks (launches)
+  int Ns_pad, Vs;
+  size_t off_ctr, ctr_bytes, off_G, G_bytes, bytes;
+  size_t n_doneA_v, n_doneA_ms, n_doneBC;
+};
+
+StripeLayout plan_stripes(int64_t N, int64_t D, int64_t V, size_t base) {
+  StripeLayout L{};
+  const int n_m2_total = (int)((N + 255) / 256);
+  L.p.n_m2 = std::min(n_m2_total, kStripeMaxM2);
+  L.p.n_vtile = (int)((V + BN - 1) / BN);
+  L.p.n_dc = (int)((D + 255) / 256);
+  L.p.vt_per_s = std::min(L.p.n_vtile, kStripeVtiles);
+  L.p.n_s = (L.p.n_vtile + L.p.vt_per_s - 1) / L.p.vt_per_s;
+  L.p.nbuf = std::min(L.p.n_s, kStripeBuffers);
+  L.n_sb = (n_m2_total + L.p.n_m2 - 1) / L.p.n_m2;
+  L.Ns_pad = L.p.n_m2 * 256;
+  L.Vs = L.p.vt_per_s * BN;
+  L.n_doneA_v = (size_t)L.p.n_vtile;
+  L.n_doneA_ms = (size_t)L.p.n_s * L.p.n_m2;
+  L.n_doneBC = (size_t)L.p.n_s;
+  L.off_ctr = base;
+  L.ctr_bytes = align_up(8 + 4 * (L.n_doneA_v + L.n_doneA_ms + L.n_doneBC), 256);
+  L.off_G = L.off_ctr + L.ctr_bytes;
+  L.G_bytes = align_up((size_t)L.p.nbuf * L.Ns_pad * L.Vs * 2, 256);
+  L.bytes = L.off_G + L.G_bytes;
+  return L;
+}
+
 struct BwdPlan {
   int n_mblk, n_vtile;
   size_t off_hdr, off_count, off_offset, off_cursor, off_flat, off_nonflat, off_list, off_enorm, zero_bytes,
       ws_bytes;
   size_t off_accE, off_accC;  // fixed-point accumulators (deterministic mode only)
+  StripeLayout stripes;       // CCE_BWD_STRIPES only
 };
 
-constexpr unsigned kBwdFlagsAll = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE | CCE_BWD_PREPARED;
+constexpr unsigned kBwdFlagsAll =
+    CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE | CCE_BWD_PREPARED | CCE_BWD_STRIPES;
 constexpr unsigned kBwdFixedPoint = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS;  // int64 accumulators
 
 bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags = 0) {
@@ -217,6 +258,11 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
     p->off_accE = p->ws_bytes;
     p->off_accC = p->off_accE + align_up((size_t)N * D * 8, 256);
     p->ws_bytes = p->off_accC + align_up((size_t)V * D * 8, 256);
+  }
+  p->stripes = StripeLayout{};
+  if (flags & CCE_BWD_STRIPES) {
+    p->stripes = plan_stripes(N, D, V, p->ws_bytes);
+    p->ws_bytes = p->stripes.bytes;
   }
   return true;
 }
@@ -330,6 +376,29 @@ cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta
   return CCE_OK;
 }
 
+int64_t cce_debug_stripe_schedule(int n_m2, int n_vtile, int n_dc, int vt_per_s, int nbuf, int32_t* out,
+                                  int64_t max_tasks) {
+  if (n_m2 <= 0 || n_vtile <= 0 || n_dc <= 0 || vt_per_s <= 0 || nbuf <= 0) return -1;
+  StripePlan p{};
+  p.n_m2 = n_m2;
+  p.n_vtile = n_vtile;
+  p.n_dc = n_dc;
+  p.vt_per_s = vt_per_s;
+  p.n_s = (n_vtile + vt_per_s - 1) / vt_per_s;
+  p.nbuf = std::min(nbuf, p.n_s);
+  const long long total = stripe_total(p);
+  if (out) {
+    for (long long t = 0; t < total + 1 && t < max_tasks; ++t) {
+      const StripeTaskDesc d = stripe_decode(p, t);
+      out[4 * t + 0] = d.type;
+      out[4 * t + 1] = d.s;
+      out[4 * t + 2] = d.a;
+      out[4 * t + 3] = d.b;
+    }
+  }
+  return total;
+}
+
 cce_status_t cce_debug_set_forward_variant(int variant) {
   if (variant < 0 || variant > 1) return CCE_ERR_INVALID_ARG;
   g_fwd_variant.store(variant);
@@ -352,6 +421,55 @@ cce_status_t cce_debug_set_kernel_events(int kernel, void* start_event, void* st
 }  // extern "C"
 
 namespace {
+
+// Dense backward through softmax-gradient stripes (bwd_stripe.cu): one
+// launch per token super-block; a: the common backward arguments.
+cce_status_t backward_stripes(const void* E, const void* C, void* dE, void* dC, const BwdPlan& bp, const BwdArgs& a,
+                              bool accumulate, int sms, char* ws, cudaStream_t stream) {
+  const StripeLayout& L = bp.stripes;
+  void* G = ws + L.off_G;
+  CUtensorMap maps[9];
+  const int64_t Grows = (int64_t)L.p.nbuf * L.Ns_pad;
+  if (!make_map(&maps[0], E, a.N, a.D, 128) || !make_map(&maps[1], C, a.V, a.D, 128) ||
+      !make_map(&maps[2], G, Grows, L.Vs, 32) || !make_map(&maps[3], G, Grows, L.Vs, 128) ||
+      !make_map(&maps[4], G, Grows, L.Vs, 64) || !make_map(&maps[5], E, a.N, a.D, 64) ||
+      !make_map(&maps[6], C, a.V, a.D, 64) || !make_map_f32(&maps[7], dE, a.N, a.D) ||
+      !make_map_f32(&maps[8], dC, a.V, a.D))
+    return CCE_ERR_CUDA;
+  unsigned char* ctr = reinterpret_cast<unsigned char*>(ws + L.off_ctr);
+  StripeArgs sa{};
+  sa.N = a.N;
+  sa.D = a.D;
+  sa.V = a.V;
+  sa.Vs = L.Vs;
+  sa.ignore_index = a.ignore_index;
+  sa.shard_mode = a.shard_mode;
+  sa.v_offset = a.v_offset;
+  sa.y = a.y;
+  sa.lse = a.lse;
+  sa.dloss = a.dloss;
+  sa.next = reinterpret_cast<unsigned long long*>(ctr);
+  sa.doneA_v = reinterpret_cast<unsigned*>(ctr + 8);
+  sa.doneA_ms = sa.doneA_v + L.n_doneA_v;
+  sa.doneBC = sa.doneA_ms + L.n_doneA_ms;
+  sa.status = a.status;
+  sa.wait_limit_ns = a.wait_limit_ns;
+  sa.withhold_loads = a.withhold_loads;
+  const int grid = sms & ~1;
+  const int n_m2_total = (a.N + 255) / 256;
+  if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  for (int sb = 0; sb < L.n_sb; ++sb) {
+    sa.p = L.p;
+    sa.p.n_m2 = std::min(L.p.n_m2, n_m2_total - sb * L.p.n_m2);
+    sa.tok0 = sb * L.p.n_m2 * 256;
+    sa.Ns_pad = sa.p.n_m2 * 256;   // buffer row stride of this launch
+    sa.dC_add = (accumulate || sb > 0) ? 1 : 0;
+    if (cudaMemsetAsync(ctr, 0, L.ctr_bytes, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (launch_bwd_stripe(maps, sa, G, grid, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  }
+  if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  return CCE_OK;
+}
 
 // shard: C is the vocabulary shard starting at global label id v_offset;
 // dC is that shard's gradient and dE this shard's share of the full dE.
@@ -403,8 +521,11 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     if (cudaMemsetAsync(accE, 0, (size_t)N * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
   } else if (!accumulate) {
+    const bool stripes = (flags & CCE_BWD_STRIPES) && !(filter_eps > 0.f);
     if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
-    if (cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
+    // (the stripe path writes every entry of dC)
+    if (!stripes && cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess)
+      return CCE_ERR_CUDA;
   }
 
   BwdArgs a;
@@ -462,6 +583,8 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     if (filter_on && launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (fixed && launch_fixed_prep(dloss, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
   }
+  if ((flags & CCE_BWD_STRIPES) && !filter_on && !fixed)
+    return backward_stripes(E, C, dE, dC, bp, a, accumulate, di.sms, ws, stream);
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (launch_bwd(tmE, tmC, tmCq, tmdE, tmdC, a, grid, g_bwd_variant.load(), stream) != cudaSuccess) return CCE_ERR_CUDA;

@@ -1,0 +1,526 @@
+// CCE backward with every gradient unit kept (filter off): the dense path,
+// through stripes of the softmax gradient.
+//
+// Cut Cross-Entropy abstract, sentences 4 and 9: the logits are recomputed,
+// never stored; the backward forms G = dloss * (softmax - onehot) and
+// contracts it into dE = G C and dC = G^T E.  When nothing is filtered every
+// logit tile contributes to both products, and adding each tile's fp32
+// partial products to dE and dC ((256 + 256) x D values per 256 x 256 tile)
+// would move far more bytes through L2 than the tensor cores need time for.
+// Instead the vocabulary is processed in stripes of Vs = vt_per_s * 256
+// columns; for each stripe (task kinds, see StripePlan in common.cuh):
+//   A  recompute the logit tiles of the stripe (E C^T on the tensor cores,
+//      tcgen05 cta_group::2, as in the forward), form G in registers and
+//      store it in bf16 into a stripe buffer in global memory (L2-resident:
+//      nbuf x 256-row blocks x Vs columns);
+//   B  dC[stripe rows] = G^T E with the whole token range as the reduction
+//      dimension: each dC tile is written exactly once;
+//   C  dE += G C[stripe rows]: one bulk reduce-add of a 256 x 256 dE tile per
+//      stripe instead of one per logit tile.
+// So the logits never exist in global memory: only nbuf stripes of G do,
+// O(N) bytes for a fixed stripe width (Vs = 2048: 12 KB per token with three
+// buffers), against N x V x 4 bytes of fp32 logits.
+//
+// One persistent kernel runs all three kinds on clusters of two CTAs.  Tasks
+// are drawn in a fixed global order from a counter by the leader CTA's
+// producer thread, which also waits (bounded) until the task's inputs are
+// complete (counters in global memory, released by the epilogues that wrote
+// them), then hands the task to both CTAs through a small ring in shared
+// memory.  Roles per CTA (192 threads): warp 0 TMA producer, warp 1 UMMA
+// issuer (leader CTA only), warps 2-5 epilogue.  Each CTA stages 32 KB of
+// operands per 64-wide K slice (5 stages) and double-buffers a 128 x 256 fp32
+// accumulator in TMEM, so the epilogue of one task overlaps the MMAs of the
+// next.  No TMA multicast: every load reads this GPU's memory.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace cce {
+
+namespace {
+
+constexpr int SP_STAGES = 5;
+constexpr int SP_STAGE_BYTES = 32768;          // per CTA: two 16 KB operand regions
+constexpr int SP_STAGING_PER_WARP = 16384;     // epilogue staging (bf16 G boxes or fp32 blocks)
+constexpr int SP_RING = 4;                     // task hand-off slots
+constexpr int SP_CONSUMERS = 10;               // leader: MMA + 4 epilogue warps; peer: producer + 4 epilogue warps
+
+struct StripeMaps {
+  CUtensorMap eA;    // E   bf16 [N][D]        box {64, 128}: A tasks, K-major token rows
+  CUtensorMap cA;    // C   bf16 [V][D]        box {64, 128}: A tasks, K-major vocabulary rows
+  CUtensorMap gSt;   // G   bf16 [nbuf*Ns][Vs] box {64, 32}:  A tasks store one warp's rows
+  CUtensorMap gK;    // G   bf16               box {64, 128}: C tasks, K-major token rows
+  CUtensorMap gM;    // G   bf16               box {64, 64}:  B tasks, vocabulary-contiguous (MN-major)
+  CUtensorMap eM;    // E   bf16               box {64, 64}:  B tasks, d-contiguous (MN-major)
+  CUtensorMap cM;    // C   bf16               box {64, 64}:  C tasks, d-contiguous (MN-major)
+  CUtensorMap dE;    // dE  fp32 [N][D]        box {32, 32}: reduce-add
+  CUtensorMap dC;    // dC  fp32 [V][D]        box {32, 32}: store / reduce-add
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// A 32 x 32 fp32 block held one row per lane goes to global memory through
+// the TMA engine: written into a 4 KB staging buffer in the 128-byte-swizzled
+// layout of a {32, 32} fp32 box, then stored or reduce-added at (x, y).
+__device__ __forceinline__ void stage_f32_block(uint8_t* xb, int lane, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(xb + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+}  // namespace
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    bwd_stripe_kernel(const __grid_constant__ StripeMaps mp, const StripeArgs a, __nv_bfloat16* G) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;                                          // SP_STAGES x 32 KB
+  uint8_t* staging = smem + SP_STAGES * SP_STAGE_BYTES;            // 4 x 16 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + 4 * SP_STAGING_PER_WARP);
+  uint64_t* full = bars;                          // leader: both CTAs' copies of a stage landed
+  uint64_t* empty = bars + SP_STAGES;             // each CTA: stage free again
+  uint64_t* tfull = bars + 2 * SP_STAGES;         // each CTA: accumulator ready [2]
+  uint64_t* tempty = tfull + 2;                   // leader: both epilogues done with it [2]
+  uint64_t* drain = tempty + 2;                   // leader: UMMA drain at exit
+  uint64_t* task_full = drain + 1;                // each CTA [SP_RING]
+  uint64_t* task_empty = task_full + SP_RING;     // leader [SP_RING]
+  // each CTA [SP_RING], 16-byte aligned (written with 16-byte stores)
+  int4* task_slot = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(task_empty + SP_RING) + 15) & ~uintptr_t(15));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(task_slot + SP_RING);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const StripePlan& P = a.p;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SP_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);
+    }
+    mbar_init(drain, 1);
+    for (int r = 0; r < SP_RING; ++r) {
+      mbar_init(&task_full[r], 1);
+      mbar_init(&task_empty[r], SP_CONSUMERS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_map(&mp.eA);
+    tma_prefetch_map(&mp.cA);
+    tma_prefetch_map(&mp.gSt);
+    tma_prefetch_map(&mp.gK);
+    tma_prefetch_map(&mp.gM);
+    tma_prefetch_map(&mp.eM);
+    tma_prefetch_map(&mp.cM);
+    tma_prefetch_map(&mp.dE);
+    tma_prefetch_map(&mp.dC);
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, a.wait_limit_ns};
+  const uint32_t task_empty_leader0 = mapa_shared(smem_u32(&task_empty[0]), 0);
+
+  // Reads task k from this CTA's ring, then frees the slot on the leader
+  // (one arrival per consumer).  With whole_warp, lane 0 waits and reads and
+  // the warp follows its outcome, so the lanes never part ways on a wait.
+  auto take_task = [&](int k, StripeTaskDesc& t, bool whole_warp) -> bool {
+    const int slot = k & (SP_RING - 1);
+    int4 d = make_int4(TASK_END, 0, 0, 0);
+    int ok = 1;
+    if (!whole_warp || lane == 0) {
+      ok = mbar_wait_cluster(&task_full[slot], (uint32_t)(k / SP_RING) & 1u, wc) ? 1 : 0;
+      if (ok) {
+        const volatile int* vs = reinterpret_cast<const volatile int*>(&task_slot[slot]);
+        d = make_int4(vs[0], vs[1], vs[2], vs[3]);
+        mbar_arrive_cluster(task_empty_leader0 + (uint32_t)(slot * 8));
+      }
+    }
+    if (whole_warp) {
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      d.x = __shfl_sync(0xffffffffu, d.x, 0);
+      d.y = __shfl_sync(0xffffffffu, d.y, 0);
+      d.z = __shfl_sync(0xffffffffu, d.z, 0);
+      d.w = __shfl_sync(0xffffffffu, d.w, 0);
+    }
+    t = StripeTaskDesc{d.x, d.y, d.z, d.w};
+    return ok != 0;
+  };
+  // Bounded wait taken by lane 0 for the whole warp (warp-uniform outcome).
+  auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait(bar, parity, wc) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+  };
+  auto k_steps = [&](const StripeTaskDesc& t) -> int {
+    if (t.type == TASK_A) return (a.D + BK - 1) / BK;
+    if (t.type == TASK_B) return a.Ns_pad / BK;
+    return stripe_tiles(P, t.s) * (BN / BK);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- producer (both CTAs); the leader also deals the tasks ----------------
+      int stage = 0;
+      uint32_t phase = 0, armed = 0;
+      const long long total = stripe_total(P);
+      for (int k = 0;; ++k) {
+        StripeTaskDesc t;
+        if (leader) {
+          const int slot = k & (SP_RING - 1);
+          if (!mbar_wait(&task_empty[slot], ((uint32_t)(k / SP_RING) & 1u) ^ 1u, wc)) goto producer_done;
+          const unsigned long long drawn = atomicAdd(a.next, 1ull);
+          t = drawn < (unsigned long long)total ? stripe_decode(P, (long long)drawn)
+                                                : StripeTaskDesc{TASK_END, 0, 0, 0};
+          // wait until the task's inputs are complete (bounded)
+          if (t.type != TASK_END) {
+            const unsigned* ctr = nullptr;
+            unsigned want = 0;
+            if (t.type == TASK_A) {
+              if (t.s >= P.nbuf) {
+                const int s0 = t.s - P.nbuf;
+                ctr = a.doneBC + s0;
+                want = 8u * (unsigned)(stripe_nB(P, s0) + stripe_nC(P));
+              }
+            } else if (t.type == TASK_B) {
+              ctr = a.doneA_v + t.a;
+              want = 8u * (unsigned)P.n_m2;
+            } else {
+              ctr = a.doneA_ms + (size_t)t.s * P.n_m2 + t.a;
+              want = 8u * (unsigned)stripe_tiles(P, t.s);
+            }
+            if (ctr != nullptr && ld_acquire_gpu(ctr) < want) {
+              const uint64_t t0 = global_timer_ns();
+              bool ok = false;
+              while (true) {
+                __nanosleep(256);
+                if (ld_acquire_gpu(ctr) >= want) {
+                  ok = true;
+                  break;
+                }
+                if (*abort_flag) break;
+                if (global_timer_ns() - t0 > a.wait_limit_ns) {
+                  *abort_flag = 1;
+                  break;
+                }
+              }
+              if (!ok) goto producer_done;
+            }
+            fence_proxy_async_global();  // the inputs were written by other CTAs' bulk stores
+          }
+          const int4 d = make_int4(t.type, t.s, t.a, t.b);
+          task_slot[slot] = d;
+          st_shared_cluster_v4(mapa_shared(smem_u32(&task_slot[slot]), 1), d);
+          mbar_arrive(&task_full[slot]);
+          mbar_arrive_release_cluster(mapa_shared(smem_u32(&task_full[slot]), 1));
+        } else {
+          if (!take_task(k, t, false)) goto producer_done;
+          fence_proxy_async_global();
+        }
+        if (t.type == TASK_END) break;
+        const int nk = k_steps(t);
+        const int r = (int)rank;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
+          uint8_t* X = stages + stage * SP_STAGE_BYTES;
+          uint8_t* Y = X + 16384;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * SP_STAGE_BYTES);
+          if (!a.withhold_loads) {
+            if (t.type == TASK_A) {
+              // X = E[token rows of this CTA][64 d], Y = C[vocabulary rows of this CTA][64 d]
+              tma_load_2d_pair(X, &mp.eA, &full[stage], kb * BK, a.tok0 + t.a * 256 + r * 128);
+              tma_load_2d_pair(Y, &mp.cA, &full[stage], kb * BK, t.b * BN + r * 128);
+            } else if (t.type == TASK_B) {
+              // X = G[64 tokens][this CTA's 128 vocabulary columns] (two 64-column boxes),
+              // Y = E[64 tokens][this CTA's 128 d columns]
+              const int gcol = (t.a - t.s * P.vt_per_s) * BN + r * 128;
+              const int grow = (t.s % P.nbuf) * a.Ns_pad + kb * BK;
+              tma_load_2d_pair(X, &mp.gM, &full[stage], gcol, grow);
+              tma_load_2d_pair(X + 8192, &mp.gM, &full[stage], gcol + 64, grow);
+              const int d0 = t.b * 256 + r * 128;
+              tma_load_2d_pair(Y, &mp.eM, &full[stage], d0, a.tok0 + kb * BK);
+              tma_load_2d_pair(Y + 8192, &mp.eM, &full[stage], d0 + 64, a.tok0 + kb * BK);
+            } else {
+              // X = G[this CTA's 128 token rows][64 stripe columns],
+              // Y = C[64 stripe rows][this CTA's 128 d columns]
+              tma_load_2d_pair(X, &mp.gK, &full[stage], kb * BK,
+                               (t.s % P.nbuf) * a.Ns_pad + t.a * 256 + r * 128);
+              const int v0 = t.s * P.vt_per_s * BN + kb * BK;
+              const int d0 = t.b * 256 + r * 128;
+              tma_load_2d_pair(Y, &mp.cM, &full[stage], d0, v0);
+              tma_load_2d_pair(Y + 8192, &mp.cM, &full[stage], d0 + 64, v0);
+            }
+            armed |= 1u << stage;
+          }
+          if (++stage == SP_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:
+      if (leader) {
+        int dummy = 0;
+        WaitCtl exit_wc{&dummy, a.wait_limit_ns};
+        for (int s = 0; s < SP_STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (s < stage) ? phase : (phase ^ 1u), exit_wc);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- UMMA issuer (leader) ----------------
+      constexpr uint32_t IDESC_A = idesc_bf16_f32(2 * BM, BN, false, false);
+      constexpr uint32_t IDESC_B = idesc_bf16_f32(2 * BM, BN, true, true);
+      constexpr uint32_t IDESC_C = idesc_bf16_f32(2 * BM, BN, false, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int k = 0;; ++k) {
+        StripeTaskDesc t;
+        if (!take_task(k, t, false)) goto mma_done;
+        if (t.type == TASK_END) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, wc)) goto mma_done;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const int nk = k_steps(t);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
+          tc_fence_after();
+          const uint32_t xa = smem_u32(stages + stage * SP_STAGE_BYTES);
+          const uint32_t ya = xa + 16384;
+#pragma unroll
+          for (int k16 = 0; k16 < BK / 16; ++k16) {
+            const uint32_t acc_on = (kb | k16) != 0;
+            if (t.type == TASK_A) {
+              umma_bf16_pair(d_tmem, sdesc_sw128(xa + k16 * 32, 16, 1024), sdesc_sw128(ya + k16 * 32, 16, 1024),
+                             IDESC_A, acc_on);
+            } else if (t.type == TASK_B) {
+              // A = G^T (M = vocabulary, 64-column groups 8 KB apart; K = tokens, 128 B rows)
+              // B = E (N = d, 64-column groups 8 KB apart; K = tokens)
+              umma_bf16_pair(d_tmem, sdesc_sw128(xa + k16 * 2048, 8192, 1024),
+                             sdesc_sw128(ya + k16 * 2048, 8192, 1024), IDESC_B, acc_on);
+            } else {
+              // A = G (K-major token rows), B = C (N = d groups 8 KB apart; K = vocabulary rows)
+              umma_bf16_pair(d_tmem, sdesc_sw128(xa + k16 * 32, 16, 1024),
+                             sdesc_sw128(ya + k16 * 2048, 8192, 1024), IDESC_C, acc_on);
+            }
+          }
+          umma_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == SP_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        umma_commit_pair_mc(&tfull[acc], 0x3);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    mma_done:
+      umma_commit_pair_mc(drain, 0x1);
+      {
+        int dummy = 0;
+        WaitCtl exit_wc{&dummy, a.wait_limit_ns};
+        mbar_wait(drain, 0, exit_wc);
+      }
+    }
+  } else {
+    // ---------------- epilogue: 4 warps per CTA, one TMEM lane (row) per thread ----------------
+    const int ew = warp & 3;  // TMEM lane group of this warp
+    const uint32_t lane_addr = (uint32_t)(ew * 32) << 16;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    uint8_t* stg = staging + ew * SP_STAGING_PER_WARP;
+    const int r = (int)rank;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    unsigned long long n_tiles = 0, n_units = 0;
+    for (int k = 0;; ++k) {
+      StripeTaskDesc t;
+      if (!take_task(k, t, true)) break;
+      if (t.type == TASK_END) break;
+      if (!warp_wait(&tfull[acc], acc_phase)) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + lane_addr + (uint32_t)(acc * BN);
+      if (t.type == TASK_A) {
+        // row = token; columns = the 256 vocabulary entries of tile t.b
+        const int row = a.tok0 + t.a * 256 + r * 128 + ew * 32 + lane;
+        bool valid = row < a.N;
+        long long yl = valid ? a.y[row] : a.ignore_index;
+        if (yl == a.ignore_index) valid = false;
+        if (a.shard_mode) {
+          yl -= a.v_offset;
+        } else if (valid && (yl < 0 || yl >= a.V)) {
+          valid = false;
+          atomicOr(a.status + ST_FLAGS, SF_BAD_LABEL);
+        }
+        const float lse2 = valid ? a.lse[row] * LOG2E : 0.f;
+        const float dl = valid ? a.dloss[row] : 0.f;
+        const long long yrel = yl - (long long)t.b * BN;
+        const int ycol = (valid && yrel >= 0 && yrel < BN) ? (int)yrel : -1;
+        const int ncols = min(BN, a.V - t.b * BN);
+        const int sw = lane & 7;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float x[32];
+          tmem_ld32(tacc + (uint32_t)(c * 32), x);
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float g2[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int col = c * 32 + j + q;
+              const float p = ex2_approx(fmaf(x[j + q], LOG2E, -lse2));
+              float d = (col == ycol) ? p - 1.f : p;
+              d = (valid && col < ncols) ? d : 0.f;
+              g2[q] = dl * d;
+            }
+            pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
+          }
+          // box q = c / 2 (64 columns), this lane's 128-byte row, 128B swizzle
+          uint8_t* rowp = stg + (c >> 1) * 4096 + lane * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = ((c & 1) * 4 + q) ^ sw;
+            *reinterpret_cast<uint4*>(rowp + chunk * 16) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int gcol = (t.b - t.s * P.vt_per_s) * BN;
+          const int grow = (t.s % P.nbuf) * a.Ns_pad + t.a * 256 + r * 128 + ew * 32;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tma_store_2d(&mp.gSt, stg + q * 4096, gcol + q * 64, grow);
+          bulk_commit_group();
+          bulk_wait_group0();
+          fence_proxy_async_global();
+          red_release_gpu_add(a.doneA_v + t.b, 1u);
+          red_release_gpu_add(a.doneA_ms + (size_t)t.s * P.n_m2 + t.a, 1u);
+          if (ew == 0) {
+            const int rows_here = a.N - (a.tok0 + t.a * 256 + r * 128);
+            if (rows_here > 0) {
+              n_tiles += 1;
+              n_units += (unsigned long long)min(4, (rows_here + 31) / 32) * (unsigned long long)((ncols + 31) / 32);
+            }
+          }
+        }
+        __syncwarp();
+      } else {
+        // B: rows = vocabulary (dC), C: rows = tokens (dE); 256 d columns of chunk t.b
+        const bool isB = t.type == TASK_B;
+        const int row0 = isB ? t.a * BN + r * 128 + ew * 32 : a.tok0 + t.a * 256 + r * 128 + ew * 32;
+        const int rows_lim = isB ? a.V : a.N;
+        const CUtensorMap* map = isB ? &mp.dC : &mp.dE;
+        const bool add = isB ? (a.dC_add != 0) : true;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tacc + (uint32_t)(c * 32), v);
+          const int x0 = t.b * 256 + c * 32;
+          if (row0 < rows_lim && x0 < a.D) {
+            // Two staging buffers in turn: the block staged here two pieces ago
+            // has been read once at most one group is still reading.  (Pieces
+            // are skipped only from some c on, so the turn never breaks.)
+            uint8_t* xb = stg + (c & 1) * 4096;
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            stage_f32_block(xb, lane, v);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (add)
+                tma_reduce_add_2d(map, xb, x0, row0);
+              else
+                tma_store_2d(map, xb, x0, row0);
+              bulk_commit_group();
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        if (lane == 0) {
+          bulk_wait_group0();
+          fence_proxy_async_global();
+          red_release_gpu_add(a.doneBC + t.s, 1u);
+        }
+        __syncwarp();
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (lane == 0) bulk_wait_group0();
+    if (ew == 0 && lane == 0) {
+      atomicAdd(a.status + ST_TILES, n_tiles);
+      atomicAdd(a.status + ST_LIVE_TILES, n_units);
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no remote arrival or copy can target an exited CTA
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status + ST_FLAGS, SF_TIMEOUT);
+}
+
+size_t bwd_stripe_smem_bytes() {
+  return 1024 + (size_t)SP_STAGES * SP_STAGE_BYTES + 4 * (size_t)SP_STAGING_PER_WARP + 512;
+}
+
+// maps: the nine tensor maps in the order of StripeMaps; grid: an even number of CTAs.
+cudaError_t launch_bwd_stripe(const CUtensorMap* maps, const StripeArgs& a, void* G, int grid, cudaStream_t stream) {
+  StripeMaps mp;
+  mp.eA = maps[0];
+  mp.cA = maps[1];
+  mp.gSt = maps[2];
+  mp.gK = maps[3];
+  mp.gM = maps[4];
+  mp.eM = maps[5];
+  mp.cM = maps[6];
+  mp.dE = maps[7];
+  mp.dC = maps[8];
+  const size_t smem = bwd_stripe_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(bwd_stripe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  bwd_stripe_kernel<<<grid, NUM_THREADS, smem, stream>>>(mp, a, reinterpret_cast<__nv_bfloat16*>(G));
+  return cudaGetLastError();
+}
+
+}  // namespace cce

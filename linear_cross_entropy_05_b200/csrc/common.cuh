@@ -127,6 +127,128 @@ struct BwdArgs {
   int trace_cap;
 };
 
+// ----------------------------------------------------------------------------
+// Dense backward through softmax-gradient stripes (filter off).
+//
+// The vocabulary is cut into stripes of vt_per_s 256-wide tiles.  For each
+// stripe s three kinds of 256 x 256 CTA-pair tasks run:
+//   A(s): (token block m2 of 256, vocabulary tile vt of the stripe): recompute
+//         the logit tile, form G = dloss (softmax - onehot) and store it in
+//         bf16 into stripe buffer s % nbuf;
+//   B(s): (vt of the stripe, d-chunk dc of 256): dC[vt, dc] = G[:, vt]^T E[:, dc]
+//         over every token of the launch (written once);
+//   C(s): (m2, dc): dE[m2, dc] += G[m2, stripe] C[stripe, dc].
+// Global task order: A(0); then for s = 1 .. n_s - 1: A(s), B(s-1), C(s-1);
+// then B(n_s - 1), C(n_s - 1).  Every task depends only on tasks earlier in
+// this order (B(s), C(s) on A(s); A(s) on B(s - nbuf), C(s - nbuf), which
+// free its buffer), so CTA pairs that take tasks in this order always make
+// progress.
+// ----------------------------------------------------------------------------
+struct StripePlan {
+  int n_m2;      // 256-token blocks of this launch
+  int n_vtile;   // 256-wide vocabulary tiles (all of V)
+  int n_dc;      // 256-wide d-chunks
+  int vt_per_s;  // vocabulary tiles per stripe
+  int n_s;       // stripes
+  int nbuf;      // stripe buffers (<= n_s)
+};
+enum StripeTask : int { TASK_END = -1, TASK_A = 0, TASK_B = 1, TASK_C = 2 };
+struct StripeTaskDesc {
+  int type, s, a, b;  // A: a = m2, b = vt; B: a = vt, b = dc; C: a = m2, b = dc
+};
+
+__host__ __device__ inline int stripe_tiles(const StripePlan& p, int s) {
+  const int t = p.n_vtile - s * p.vt_per_s;
+  return t < p.vt_per_s ? t : p.vt_per_s;
+}
+__host__ __device__ inline long long stripe_nA(const StripePlan& p, int s) {
+  return (long long)p.n_m2 * stripe_tiles(p, s);
+}
+__host__ __device__ inline long long stripe_nB(const StripePlan& p, int s) {
+  return (long long)stripe_tiles(p, s) * p.n_dc;
+}
+__host__ __device__ inline long long stripe_nC(const StripePlan& p) { return (long long)p.n_m2 * p.n_dc; }
+__host__ __device__ inline long long stripe_total(const StripePlan& p) {
+  long long t = 0;
+  for (int s = 0; s < p.n_s; ++s) t += stripe_nA(p, s) + stripe_nB(p, s) + stripe_nC(p);
+  return t;
+}
+
+// Inside A(s): the token block varies fastest, so the pairs running at the
+// same time share a vocabulary tile of C; inside B(s) and C(s) the d-chunk
+// varies fastest (pairs share the stripe columns, resp. the token rows, of G).
+__host__ __device__ inline StripeTaskDesc stripe_A(const StripePlan& p, int s, long long k) {
+  return StripeTaskDesc{TASK_A, s, (int)(k % p.n_m2), s * p.vt_per_s + (int)(k / p.n_m2)};
+}
+__host__ __device__ inline StripeTaskDesc stripe_BC(const StripePlan& p, int s, long long k) {
+  const long long nB = stripe_nB(p, s);
+  if (k < nB) return StripeTaskDesc{TASK_B, s, s * p.vt_per_s + (int)(k / p.n_dc), (int)(k % p.n_dc)};
+  k -= nB;
+  return StripeTaskDesc{TASK_C, s, (int)(k / p.n_dc), (int)(k % p.n_dc)};
+}
+
+// Task t of the global order.  Every stripe but the last has the same task
+// counts, so the position is found without walking the stripes.
+__host__ __device__ inline StripeTaskDesc stripe_decode(const StripePlan& p, long long t) {
+  if (t < 0) return StripeTaskDesc{TASK_END, 0, 0, 0};
+  const long long nA = stripe_nA(p, 0);
+  if (p.n_s == 1) {
+    if (t < nA) return stripe_A(p, 0, t);
+    t -= nA;
+    if (t < stripe_nB(p, 0) + stripe_nC(p)) return stripe_BC(p, 0, t);
+    return StripeTaskDesc{TASK_END, 0, 0, 0};
+  }
+  if (t < nA) return stripe_A(p, 0, t);
+  t -= nA;
+  // groups g = 1 .. n_s - 2: A(g) (full), then B/C(g - 1) (full)
+  const long long nBCf = stripe_nB(p, 0) + stripe_nC(p);
+  const long long gsz = nA + nBCf;
+  const long long full_groups = p.n_s - 2;
+  if (t < full_groups * gsz) {
+    const int g = 1 + (int)(t / gsz);
+    const long long k = t % gsz;
+    return k < nA ? stripe_A(p, g, k) : stripe_BC(p, g - 1, k - nA);
+  }
+  t -= full_groups * gsz;
+  const int L = p.n_s - 1;  // the last stripe (possibly narrower)
+  const long long nAL = stripe_nA(p, L);
+  if (t < nAL) return stripe_A(p, L, t);
+  t -= nAL;
+  const long long nBCp = stripe_nB(p, L - 1) + stripe_nC(p);
+  if (t < nBCp) return stripe_BC(p, L - 1, t);
+  t -= nBCp;
+  if (t < stripe_nB(p, L) + stripe_nC(p)) return stripe_BC(p, L, t);
+  return StripeTaskDesc{TASK_END, 0, 0, 0};
+}
+
+// Counters of the stripe backward (u32, zeroed per launch): one arrival per
+// epilogue warp (4 per CTA, 8 per pair) for each finished task.
+//   doneA_v[n_vtile]        A tasks of vocabulary tile vt
+//   doneA_ms[n_s][n_m2]     A tasks of token block m2 in stripe s
+//   doneBC[n_s]             B and C tasks of stripe s
+//   next                    the next task to hand out
+struct StripeArgs {
+  StripePlan p;
+  int N, D, V;
+  int tok0;              // first token of this launch (token super-block)
+  int Ns_pad;            // rows of one stripe buffer: n_m2 * 256
+  int Vs;                // columns of one stripe buffer: vt_per_s * 256
+  int dC_add;            // 1: B tasks add into dC (later super-blocks, or accumulation)
+  long long ignore_index;
+  int shard_mode;        // labels are global ids; C is the shard [v_offset, v_offset + V)
+  long long v_offset;
+  const int64_t* y;
+  const float* lse;
+  const float* dloss;
+  unsigned* doneA_v;
+  unsigned* doneA_ms;
+  unsigned* doneBC;
+  unsigned long long* next;
+  unsigned long long* status;
+  unsigned long long wait_limit_ns;
+  int withhold_loads;    // test hook: the TMA producers issue nothing
+};
+
 // Fixed-point exponent s: contributions are stored as round(x * 2^s) in int64.
 // Every gradient entry is bounded by
 //   |dE_id| <= max_i|dloss_i| * 2 * max_v|C_v|   and

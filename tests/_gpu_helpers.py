@@ -52,13 +52,15 @@ def gpu_forward(E, C, y, ws=None):
     return loss.cpu().numpy(), lse.cpu().numpy(), st
 
 
-def gpu_backward(E, C, y, lse, dloss_np, eps, ws=None):
+def gpu_backward(E, C, y, lse, dloss_np, eps, ws=None, stripes=None):
+    """stripes: None = the binding's default (the stripe backward when the
+    filter is off), True / False to force either dense path."""
     import torch
     import linear_cross_entropy_05_b200 as L
     ws = ws or L.Workspace(E.device)
     dl = torch.from_numpy(np.asarray(dloss_np, dtype=np.float32)).to(E.device)
     if not torch.is_tensor(lse):
         lse = torch.from_numpy(np.asarray(lse, dtype=np.float32)).to(E.device)
-    dE, dC = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws)
+    dE, dC = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws, stripes=stripes)
     st = L.read_status(ws)
     return dE, dC, st

@@ -47,6 +47,58 @@ def test_aggregate_over_two_gloo_ranks():
         assert value == pytest.approx((1000.0 + 2000.0) / 1.5)
 
 
+def _worker_shared(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist = bench.init_dist("gloo")
+    # vocabulary-parallel: both ranks work on the same 8192 tokens
+    value, tmax = bench.aggregate_shared_batch(dist, 8192.0, 0.25 + 0.25 * rank, "cpu")
+    shard = bench.vocab_shard(256000, world, rank)
+    out[rank] = (value, tmax, shard)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_vocab_parallel_aggregate_over_two_gloo_ranks():
+    world = 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker_shared, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+    shards = []
+    for r in range(world):
+        value, tmax, shard = out[r]
+        assert tmax == pytest.approx(0.5)
+        assert value == pytest.approx(8192.0 / 0.5)     # the shared batch is counted once
+        shards.append(shard)
+    assert shards[0][0] == 0 and shards[0][0] + shards[0][1] == shards[1][0]
+    assert shards[1][0] + shards[1][1] == 256000
+
+
+@pytest.mark.parametrize("V,world", [(256000, 8), (151936, 3), (4096 + 77, 2), (513, 3), (128256, 5)])
+def test_vocab_shards_cover_the_vocabulary_in_whole_tiles(V, world):
+    sys.path.insert(0, ROOT)
+    import bench
+    shards = [bench.vocab_shard(V, world, r) for r in range(world)]
+    pos = 0
+    for v0, n in shards:
+        assert v0 == pos and n >= 0
+        assert v0 % 256 == 0
+        pos += n
+    assert pos == V
+    sizes = [-(-n // 256) for _, n in shards]
+    assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+
+
+def test_vocab_shards_need_a_tile_per_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    with pytest.raises(ValueError):
+        bench.vocab_shard(300, 4, 0)
+
+
 def test_single_process_aggregate_is_identity():
     sys.path.insert(0, ROOT)
     import bench

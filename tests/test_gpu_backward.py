@@ -33,20 +33,23 @@ CASES_ON = [
 ]
 
 
-def _run(w, eps, dloss_seed=99):
+def _run(w, eps, dloss_seed=99, stripes=None):
     inp = synth.make_inputs(w)
     E, C, y = to_dev(inp)
     loss, lse, st = gpu_forward(E, C, y)
     assert st["status"] == 0
     dloss = synth.random_dloss(dloss_seed, w.N)
-    dE, dC, st = gpu_backward(E, C, y, lse, dloss, eps)
+    dE, dC, st = gpu_backward(E, C, y, lse, dloss, eps, stripes=stripes)
     _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
     return inp, dloss, olse, dE.cpu().numpy(), dC.cpu().numpy(), st
 
 
+@pytest.mark.parametrize("stripes", [True, False], ids=["stripes", "fused-tiles"])
 @pytest.mark.parametrize("w", CASES_OFF, ids=[w.name for w in CASES_OFF])
-def test_backward_filter_off_matches_exact_gradient(w):
-    inp, dloss, olse, gE, gC, st = _run(w, 0.0)
+def test_backward_filter_off_matches_exact_gradient(w, stripes):
+    # both dense paths: softmax-gradient stripes (the default with the filter
+    # off) and the fused per-tile kernel
+    inp, dloss, olse, gE, gC, st = _run(w, 0.0, stripes=stripes)
     assert st["status"] == 0 and st["flags"] == 0
     n_tiles = -(-w.N // 32) * -(-w.V // 32)
     assert st["live_tiles"] == n_tiles and st["dead_tiles"] == 0 and st["pruned_tiles"] == 0
@@ -194,7 +197,7 @@ def test_backward_kernel_variants_match_oracle(variant, eps):
     w = synth.GEMMA2_2B.with_sizes(N=700, V=12000 + 77)
     L.cce_debug_set_backward_variant(variant)
     try:
-        inp, dloss, olse, gE, gC, st = _run(w, eps)
+        inp, dloss, olse, gE, gC, st = _run(w, eps, stripes=False)
     finally:
         L.cce_debug_set_backward_variant(0)
     assert st["status"] == 0
