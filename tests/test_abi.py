@@ -146,12 +146,19 @@ def test_backward_ex_workspace_and_flags(lib):
         assert cce_backward_workspace_size_ex(N, D, V, flags) == base + up(8 * N * D) + up(8 * V * D)
     assert cce_backward_workspace_size_ex(N, D, V, 4) == base   # accumulate alone: no extra workspace
     assert cce_backward_workspace_size_ex(N, D, V, 8) == base   # prepared: no extra workspace
-    assert cce_backward_workspace_size_ex(N, D, V, 16) == 0     # unknown flag
+    # stripes: counters + three bf16 stripe buffers of 8192 tokens x 2048 columns
+    n_vt, n_s = -(-V // 256), -(-V // 2048)
+    ctr = up(8 + 4 * (n_vt + n_s * 32 + n_s))
+    assert cce_backward_workspace_size_ex(N, D, V, 16) == base + ctr + up(3 * 8192 * 2048 * 2)
+    # token super-blocks of 16384 bound the stripe buffers whatever N
+    big = cce_backward_workspace_size_ex(65536, 2048, 262144, 16) - cce_backward_workspace_size(65536, 2048, 262144)
+    assert big < 3 * 16384 * 2048 * 2 + (1 << 20)
+    assert cce_backward_workspace_size_ex(N, D, V, 32) == 0     # unknown flag
     P = 1 << 20
     args = [P, P, P, P, P, 256, 256, 4096, -100, 0.0, 0, P, P, P, 1 << 30, 0]
-    args[10] = 16
+    args[10] = 32
     assert cce_backward_ex(*args, check=False) == 1          # unknown flag: rejected on the host
-    for flags in (3, 4, 7, 8, 15):
+    for flags in (3, 4, 7, 8, 15, 16, 31):
         args[10] = flags
         assert cce_backward_ex(*args, check=False) == 4      # valid, but no device here
 
