@@ -577,7 +577,8 @@ def run_gpu(args, w):
                                          if overlap_zero else "inside the backward call"),
                            classifier_norm=("cce_backward_prepare on the side stream during the forward"
                                             if prepare else "inside the backward call"),
-                           l2_prefetch_slices=list(args.prefetch) if args.prefetch else [0, 0]),
+                           l2_prefetch_slices=list(args.prefetch) if args.prefetch else [0, 0],
+                           reduce_prefetch_slices=args.reduce_prefetch),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops (burst: the timed region is under a second)",
@@ -741,6 +742,82 @@ def run_trace(args, w):
     return 0
 
 
+def run_trace_stripes(args, w):
+    """Per-task timeline of one dense (filter-off) stripe backward launch
+    through the trace hook: per task kind, the time between the completions
+    of consecutive accumulators of a CTA pair (the tensor cores' time per
+    task, bubbles included), how long the pair's producer waited for the
+    task's inputs, and how often a task was handed out only after the
+    previous accumulator was complete (a pipeline bubble).  One JSON object
+    (documentation, not the contract line)."""
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    from linear_cross_entropy_05_b200 import synth
+    dev = torch.device("cuda", 0)
+    inp = synth.make_inputs(w)
+    E = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(dev)
+    C = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.from_numpy(inp["y"]).to(dev)
+    dl = torch.from_numpy(synth.mean_dloss(inp["y"])).to(dev)
+    wf, wb = L.Workspace(dev), L.Workspace(dev)
+    loss, lse = L.forward(E, C, y, IGN, workspace=wf)
+    dE = torch.empty((w.N, w.D), device=dev)
+    dC = torch.empty((w.V, w.D), device=dev)
+    for _ in range(2):
+        L.backward(E, C, y, lse, dl, 0.0, IGN, workspace=wb, out=(dE, dC), stripes=True)
+    cap = 4096
+    pairs = torch.cuda.get_device_properties(dev).multi_processor_count // 2
+    tr = torch.zeros(pairs * cap * 4, dtype=torch.int64, device=dev)
+    L.cce_debug_set_backward_trace(tr.data_ptr(), cap)
+    try:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        L.backward(E, C, y, lse, dl, 0.0, IGN, workspace=wb, out=(dE, dC), stripes=True)
+        e1.record()
+        torch.cuda.synchronize()
+    finally:
+        L.cce_debug_set_backward_trace(0, 1)
+    st = L.read_status(wb)
+    t = tr.view(pairs, cap, 4).cpu().numpy().astype(np.int64)
+    names = {0: "A recompute + G store", 1: "B dC tile", 2: "C dE tile"}
+    per = {k: {"n": 0, "acc_interval_us": [], "dep_wait_us": [], "epilogue_us": [], "bubbles": 0} for k in names}
+    t_first = t[:, 0, 0][t[:, 0, 0] > 0].min()
+    ends = []
+    for p in range(pairs):
+        k = 0
+        while k < cap and t[p, k, 0] > 0:
+            kind = int(t[p, k, 3] & 0xFF)
+            d = per[kind]
+            d["n"] += 1
+            d["dep_wait_us"].append((t[p, k, 3] >> 8) / 1e3)
+            if t[p, k, 2] > 0 and t[p, k, 1] > 0:
+                d["epilogue_us"].append((t[p, k, 2] - t[p, k, 1]) / 1e3)
+            if k > 0 and t[p, k, 1] > 0 and t[p, k - 1, 1] > 0:
+                d["acc_interval_us"].append((t[p, k, 1] - t[p, k - 1, 1]) / 1e3)
+                if t[p, k, 0] > t[p, k - 1, 1]:
+                    d["bubbles"] += 1
+            k += 1
+        if k:
+            ends.append((t[p, k - 1, 2] - t_first) / 1e3)
+    flop = {0: 2.0 * 256 * 256 * w.D, 1: 2.0 * 256 * 256 * -(-w.N // 256) * 256,
+            2: 2.0 * 256 * 256 * min(2048, -(-w.V // 256) * 256)}
+    peaks, _ = measured_peaks()
+    pair_peak = float(peaks["bf16_tflops"]) * 1e12 / pairs
+    out = {"mode": "trace-stripes", "workload": w.name, "N": w.N, "D": w.D, "V": w.V, "status": st,
+           "launch_ms": e0.elapsed_time(e1), "pairs": pairs, "first_pair_done_us": float(min(ends)),
+           "last_pair_done_us": float(max(ends)), "kinds": {}}
+    for k, nm in names.items():
+        d = per[k]
+        out["kinds"][nm] = {
+            "tasks": d["n"], "acc_interval_us_mean": float(np.mean(d["acc_interval_us"])) if d["acc_interval_us"] else None,
+            "at_burst_peak_us": flop[k] / pair_peak * 1e6,
+            "dep_wait_us_mean": float(np.mean(d["dep_wait_us"])) if d["dep_wait_us"] else None,
+            "epilogue_us_mean": float(np.mean(d["epilogue_us"])) if d["epilogue_us"] else None,
+            "handed_out_after_previous_done": d["bubbles"]}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def run_memory(args, w):
     """Classifier-head training step through the autograd wrapper: peak extra
     device memory and time of `linear_cross_entropy(E, C, y).backward()`
@@ -898,8 +975,12 @@ def main(argv=None):
                     help="forward kernel: CTA pairs (default) or single CTAs (A/B measurement)")
     ap.add_argument("--prefetch", type=int, nargs=2, default=None, metavar=("FWD", "BWD"),
                     help="L2 prefetch distances in K slices for the forward / backward operand streams (A/B)")
+    ap.add_argument("--reduce-prefetch", type=int, default=None, metavar="SLICES",
+                    help="L2 prefetch distance of the filtered backward's reduction targets (A/B; 0 = off)")
     ap.add_argument("--trace", action="store_true",
                     help="per-tile timeline of one backward launch (recompute wait, gradient tile, contraction)")
+    ap.add_argument("--dense-trace", action="store_true",
+                    help="with --trace: per-task timeline of the dense stripe backward (filter off)")
     ap.add_argument("--memory", action="store_true",
                     help="classifier-head training step: peak memory and time, CCE vs materialised logits")
     ap.add_argument("--vocab-parallel", action="store_true",
@@ -908,19 +989,24 @@ def main(argv=None):
     ap.add_argument("--suite", action="store_true",
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
-    if args.impl == "cce" and (args.fwd_variant != "pair" or args.bwd_variant or args.prefetch):
+    if args.impl == "cce" and (args.fwd_variant != "pair" or args.bwd_variant or args.prefetch or
+                               args.reduce_prefetch is not None):
         import linear_cross_entropy_05_b200 as L
         L.cce_debug_set_forward_variant(1 if args.fwd_variant == "pair" else 0)
         L.cce_debug_set_backward_variant(args.bwd_variant)
         if args.prefetch:
             L.cce_debug_set_prefetch(*args.prefetch)
+        if args.reduce_prefetch is not None:
+            L.cce_debug_set_reduce_prefetch(args.reduce_prefetch)
     if args.suite:
         return run_suite(args)
     if args.memory or args.trace:
         from linear_cross_entropy_05_b200 import synth
         w = synth.WORKLOADS[args.workload]
         w = w.with_sizes(N=args.N, V=args.V) if (args.N or args.V) else w
-        return run_memory(args, w) if args.memory else run_trace(args, w)
+        if args.memory:
+            return run_memory(args, w)
+        return run_trace_stripes(args, w) if args.dense_trace else run_trace(args, w)
     if args.warmup < 3:
         args.warmup = 3
     from linear_cross_entropy_05_b200 import synth

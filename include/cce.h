@@ -124,8 +124,10 @@ CCE_API cce_status_t cce_backward(const void* E, const void* C, const int64_t* y
  * cudaMalloc -- and so cannot supply the workspace cce_forward needs.
  * Inputs, outputs and results are those of cce_forward.  The scratch (status
  * block and per-split partials) lives in a static 8 MiB device array inside
- * the library, which every GPU that loads the library holds until the process
- * exits.
+ * the library, which every GPU that loads this part of the library holds
+ * until the process exits (with CUDA's lazy module loading the array is
+ * created at the first call on the device, not by the call itself; later
+ * calls change nothing in the device's free memory).
  *   - Problems whose forward workspace (cce_forward_workspace_size) exceeds
  *     8 MiB are rejected with CCE_ERR_WORKSPACE_TOO_SMALL before anything is
  *     launched (e.g. N = 65536 tokens, V = 262144); invalid sizes or no sm_100
@@ -189,8 +191,13 @@ typedef enum {
    * contributions are added.  Far less fp32 reduction traffic than adding
    * every logit tile's partial products, so the tensor cores set the pace.
    * Same result as without the flag up to fp32 summation order.  Ignored
-   * when filter_eps > 0 or with the fixed-point flags.  Needs the workspace
-   * of cce_backward_workspace_size_ex with this flag. */
+   * when filter_eps > 0.  With CCE_BWD_DETERMINISTIC the reduce-adds into
+   * each dE tile happen in stripe order (and dC is written once per tile),
+   * so the fp32 result is bitwise reproducible without the int64
+   * accumulators; that combination requires filter_eps <= 0
+   * (CCE_ERR_INVALID_ARG otherwise) and is not available with
+   * CCE_BWD_BF16_GRADS (the workspace size query returns 0).  Needs the
+   * workspace of cce_backward_workspace_size_ex with this flag. */
   CCE_BWD_STRIPES = 16
 } cce_backward_flags_t;
 

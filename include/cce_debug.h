@@ -45,6 +45,15 @@ CCE_API void cce_debug_withhold_loads(int on);
  * CCE_ERR_INVALID_ARG outside [0, 64]. */
 CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
 
+/* L2 prefetch distance, in 64-wide K slices, of the fp32 dE / dC rows that
+ * the filtered backward kernel's bulk reduce-adds add into: while loading
+ * the operands of contraction slice k, its TMA producer asks for the live
+ * 32-row pieces of slice k - distance (the pass runs d descending) to be
+ * brought into L2, so the reductions find their lines there.  0 turns it
+ * off.  Same results; for A/B measurement.  Process-wide.  Returns
+ * CCE_ERR_INVALID_ARG outside [0, 64]. */
+CCE_API cce_status_t cce_debug_set_reduce_prefetch(int slices);
+
 /* Profiling hook for the backward kernel's per-tile timeline.  While set,
  * every backward launch writes, for each CTA b (one per SM) and each of its
  * first tiles_per_cta tiles k, four u64 at trace[(b * tiles_per_cta + k) * 4]:
@@ -54,7 +63,13 @@ CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
  * mask; after its last tile the CTA writes the end time into word 0 of the
  * next entry (if < tiles_per_cta).  `trace` is a device buffer owned by the
  * caller with room for (number of SMs) * tiles_per_cta * 32 bytes; the
- * library does not clear it.  NULL turns the hook off.  Process-wide.
+ * library does not clear it.  The dense stripe backward (CCE_BWD_STRIPES)
+ * writes through the same hook, per CTA pair p (leader CTA) and task k, at
+ * trace[(p * tiles_per_cta + k) * 4]: the time the task was handed out, the
+ * time its accumulator was complete, the time its epilogue finished, and the
+ * task kind (0 recompute and store G, 1 dC tile, 2 dE tile) | (ns spent
+ * waiting for the task's inputs << 8).  NULL turns the hook off.
+ * Process-wide.
  * Returns CCE_ERR_INVALID_ARG for tiles_per_cta outside [1, 2^20]. */
 CCE_API cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta);
 

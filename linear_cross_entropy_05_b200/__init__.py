@@ -23,7 +23,7 @@ from typing import Optional, Tuple
 
 from . import _native
 from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCE_BWD_PREPARED,
-                      CCE_BWD_STRIPES, CCEError, cce_debug_stripe_schedule,
+                      CCE_BWD_STRIPES, CCEError, cce_debug_stripe_schedule, cce_debug_set_reduce_prefetch,
                       cce_backward, cce_backward_ex, cce_backward_prepare,
                       cce_backward_shard, cce_backward_workspace_size, cce_backward_workspace_size_ex,
                       cce_forward_shard, cce_merge_shards, cce_debug_forward_logits,
@@ -36,7 +36,8 @@ IGNORE_INDEX = -100
 
 __all__ = [
     "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "CCE_BWD_ACCUMULATE",
-    "CCE_BWD_PREPARED", "CCE_BWD_STRIPES", "cce_debug_stripe_schedule", "cce_backward_prepare",
+    "CCE_BWD_PREPARED", "CCE_BWD_STRIPES", "cce_debug_stripe_schedule", "cce_debug_set_reduce_prefetch",
+    "cce_backward_prepare",
     "backward_prepare", "cce_forward",
     "cce_forward_noalloc", "cce_backward", "cce_backward_ex", "cce_backward_workspace_size_ex",
     "cce_forward_shard", "cce_merge_shards", "cce_backward_shard", "forward_shard", "merge_shards",
@@ -134,9 +135,10 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     accumulate=True adds them to the tensors given in `out` (required)
     instead of overwriting them.  prepared=True: backward_prepare already ran
     on `workspace` for this C.  stripes (default: on when filter_eps <= 0
-    and neither deterministic nor bf16_grads): the dense backward through
-    softmax-gradient stripes (CCE_BWD_STRIPES), which needs a larger
-    workspace (about 12 KB per token, at most ~200 MB)."""
+    and not bf16_grads): the dense backward through softmax-gradient stripes
+    (CCE_BWD_STRIPES), which needs a larger workspace (about 12 KB per
+    token, at most ~200 MB); with deterministic=True it sums in a fixed
+    order instead of using the int64 fixed-point accumulators."""
     torch = _torch()
     _check_inputs(E, C, y)
     N, D = E.shape
@@ -147,7 +149,7 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     flags = ((CCE_BWD_DETERMINISTIC if deterministic else 0) | (CCE_BWD_BF16_GRADS if bf16_grads else 0) |
              (CCE_BWD_ACCUMULATE if accumulate else 0) | (CCE_BWD_PREPARED if prepared else 0))
     if stripes is None:
-        stripes = filter_eps <= 0 and not (deterministic or bf16_grads)
+        stripes = filter_eps <= 0 and not bf16_grads
     if stripes:
         flags |= CCE_BWD_STRIPES
     if prepared and workspace is None:

@@ -87,6 +87,8 @@ def load_library():
         lib.cce_debug_set_kernel_events.restype = ctypes.c_int
         lib.cce_debug_set_prefetch.argtypes = [ctypes.c_int, ctypes.c_int]
         lib.cce_debug_set_prefetch.restype = ctypes.c_int
+        lib.cce_debug_set_reduce_prefetch.argtypes = [ctypes.c_int]
+        lib.cce_debug_set_reduce_prefetch.restype = ctypes.c_int
         lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 5 + [c_vp, c_i64]
         lib.cce_debug_stripe_schedule.restype = c_i64
         lib.cce_debug_set_backward_trace.argtypes = [c_vp, c_i64]
@@ -265,3 +267,9 @@ def cce_debug_stripe_schedule(n_m2: int, n_vtile: int, n_dc: int, vt_per_s: int,
     out = np.zeros((total + 1, 4), dtype=np.int32)
     lib.cce_debug_stripe_schedule(n_m2, n_vtile, n_dc, vt_per_s, nbuf, out.ctypes.data, total + 1)
     return out
+
+
+def cce_debug_set_reduce_prefetch(slices: int) -> None:
+    """L2 prefetch distance (64-wide K slices) of the filtered backward's
+    reduction targets (live dE / dC rows); 0 = off."""
+    _check(load_library().cce_debug_set_reduce_prefetch(int(slices)), "cce_debug_set_reduce_prefetch")

@@ -33,7 +33,10 @@ cudaError_t launch_enorm(const void* E, const PrepArgs& p, int sms, cudaStream_t
 cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_bwd_stripe(const CUtensorMap* maps, const StripeArgs& a, void* G, int grid, cudaStream_t stream);
 cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
-                                bool bf16, bool accumulate, int sms, cudaStream_t stream);
+                                bool bf16, bool accumulate, const unsigned* count, int D, int sms,
+                                cudaStream_t stream);
+cudaError_t launch_clear_visited_rows(unsigned long long* acc, int V, int D, const unsigned* count,
+                                      const unsigned* hdr, int sms, cudaStream_t stream);
 }  // namespace cce
 
 using namespace cce;
@@ -52,6 +55,7 @@ std::atomic<int> g_bwd_variant{0};
 std::atomic<int> g_withhold_loads{0};
 std::atomic<int> g_fwd_pf{0};  // L2 prefetch distances (K slices) of the forward / backward operand streams
 std::atomic<int> g_bwd_pf{0};
+std::atomic<int> g_bwd_red_pf{0};  // L2 prefetch distance (K slices) of the backward's reduction targets
 std::atomic<unsigned long long*> g_bwd_trace{nullptr};
 std::atomic<int> g_bwd_trace_cap{0};
 
@@ -159,6 +163,22 @@ bool make_map_f32(CUtensorMap* map, const void* base, int64_t rows, int64_t D) {
   return r == CUDA_SUCCESS;
 }
 
+// int64 fixed-point accumulator [rows][D] as {16, 32} boxes of u64 with
+// 128-byte swizzle (16 values = one 128-byte row): the target of the
+// deterministic backward's bulk reduce-adds.
+bool make_map_u64(CUtensorMap* map, const void* base, int64_t rows, int64_t D) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 8};
+  cuuint32_t box[2] = {16, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 struct FwdPlan {
   bool pair;       // CTA-pair kernel: token blocks of 2 x BM rows, grid in pairs
   int n_mblk, n_vtile, n_split, grid, group_m;
@@ -197,7 +217,7 @@ struct StripeLayout {
   int n_sb;              // super-blocks (launches)
   int Ns_pad, Vs;
   size_t off_ctr, ctr_bytes, off_G, G_bytes, bytes;
-  size_t n_doneA_v, n_doneA_ms, n_doneBC;
+  size_t n_doneA_v, n_doneA_ms, n_doneBC, n_doneC;
 };
 
 StripeLayout plan_stripes(int64_t N, int64_t D, int64_t V, size_t base) {
@@ -215,8 +235,9 @@ StripeLayout plan_stripes(int64_t N, int64_t D, int64_t V, size_t base) {
   L.n_doneA_v = (size_t)L.p.n_vtile;
   L.n_doneA_ms = (size_t)L.p.n_s * L.p.n_m2;
   L.n_doneBC = (size_t)L.p.n_s;
+  L.n_doneC = (size_t)L.p.n_m2 * L.p.n_dc;
   L.off_ctr = base;
-  L.ctr_bytes = align_up(8 + 4 * (L.n_doneA_v + L.n_doneA_ms + L.n_doneBC), 256);
+  L.ctr_bytes = align_up(8 + 4 * (L.n_doneA_v + L.n_doneA_ms + L.n_doneBC + L.n_doneC), 256);
   L.off_G = L.off_ctr + L.ctr_bytes;
   L.G_bytes = align_up((size_t)L.p.nbuf * L.Ns_pad * L.Vs * 2, 256);
   L.bytes = L.off_G + L.G_bytes;
@@ -234,6 +255,14 @@ struct BwdPlan {
 constexpr unsigned kBwdFlagsAll =
     CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE | CCE_BWD_PREPARED | CCE_BWD_STRIPES;
 constexpr unsigned kBwdFixedPoint = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS;  // int64 accumulators
+
+// Whether these flags take the int64 fixed-point accumulation.  With
+// CCE_BWD_STRIPES the deterministic mode is served by the stripe kernel's
+// fixed reduction order instead (filter off only, fp32 outputs).
+bool uses_fixed_point(unsigned flags) {
+  if (flags & CCE_BWD_BF16_GRADS) return true;
+  return (flags & CCE_BWD_DETERMINISTIC) && !(flags & CCE_BWD_STRIPES);
+}
 
 bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags = 0) {
   if (flags & ~kBwdFlagsAll) return false;
@@ -254,7 +283,8 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
   p->off_enorm = p->off_list + align_up((size_t)N * sizeof(int2), 256);
   p->ws_bytes = p->off_enorm + align_up((size_t)N * sizeof(float), 256);
   p->off_accE = p->off_accC = 0;
-  if (flags & kBwdFixedPoint) {
+  if ((flags & CCE_BWD_STRIPES) && (flags & CCE_BWD_BF16_GRADS)) return false;  // not combined
+  if (uses_fixed_point(flags)) {
     p->off_accE = p->ws_bytes;
     p->off_accC = p->off_accE + align_up((size_t)N * D * 8, 256);
     p->ws_bytes = p->off_accC + align_up((size_t)V * D * 8, 256);
@@ -369,6 +399,12 @@ cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices) {
   return CCE_OK;
 }
 
+cce_status_t cce_debug_set_reduce_prefetch(int slices) {
+  if (slices < 0 || slices > 64) return CCE_ERR_INVALID_ARG;
+  g_bwd_red_pf.store(slices);
+  return CCE_OK;
+}
+
 cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta) {
   if (trace && (tiles_per_cta <= 0 || tiles_per_cta > (1 << 20))) return CCE_ERR_INVALID_ARG;
   g_bwd_trace_cap.store(trace ? (int)tiles_per_cta : 0);
@@ -425,7 +461,7 @@ namespace {
 // Dense backward through softmax-gradient stripes (bwd_stripe.cu): one
 // launch per token super-block; a: the common backward arguments.
 cce_status_t backward_stripes(const void* E, const void* C, void* dE, void* dC, const BwdPlan& bp, const BwdArgs& a,
-                              bool accumulate, int sms, char* ws, cudaStream_t stream) {
+                              bool accumulate, bool ordered, int sms, char* ws, cudaStream_t stream) {
   const StripeLayout& L = bp.stripes;
   void* G = ws + L.off_G;
   CUtensorMap maps[9];
@@ -452,9 +488,13 @@ cce_status_t backward_stripes(const void* E, const void* C, void* dE, void* dC, 
   sa.doneA_v = reinterpret_cast<unsigned*>(ctr + 8);
   sa.doneA_ms = sa.doneA_v + L.n_doneA_v;
   sa.doneBC = sa.doneA_ms + L.n_doneA_ms;
+  sa.doneC = sa.doneBC + L.n_doneBC;
+  sa.ordered = ordered ? 1 : 0;
   sa.status = a.status;
   sa.wait_limit_ns = a.wait_limit_ns;
   sa.withhold_loads = a.withhold_loads;
+  sa.trace = a.trace;
+  sa.trace_cap = a.trace_cap;
   const int grid = sms & ~1;
   const int n_m2_total = (a.N + 255) / 256;
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
@@ -480,9 +520,11 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   if (!E || !C || !y || !lse || !dloss || !dE || !dC || !workspace) return CCE_ERR_INVALID_ARG;
   if (v_offset < 0) return CCE_ERR_INVALID_ARG;
   if (flags & ~kBwdFlagsAll) return CCE_ERR_INVALID_ARG;
-  const bool fixed = (flags & kBwdFixedPoint) != 0;
+  const bool fixed = uses_fixed_point(flags);
   const bool bf16_out = (flags & CCE_BWD_BF16_GRADS) != 0;
   const bool accumulate = (flags & CCE_BWD_ACCUMULATE) != 0;
+  // deterministic through the stripe kernel's fixed reduction order: filter off only
+  if ((flags & CCE_BWD_STRIPES) && (flags & CCE_BWD_DETERMINISTIC) && filter_eps > 0.f) return CCE_ERR_INVALID_ARG;
   if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
   if (!(filter_eps == filter_eps)) return CCE_ERR_INVALID_ARG;  // NaN
   if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(lse, 4) || !aligned(dloss, 4) ||
@@ -496,16 +538,17 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
   CUtensorMap tmE, tmC, tmCq, tmdE, tmdC;
-  // (in fixed-point mode the fp32 maps are built but the kernel reduces into
-  // the int64 accumulators instead; dE/dC may then hold bf16)
-  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN) || !make_map(&tmCq, C, V, D, 64) ||
-      !make_map_f32(&tmdE, dE, N, D) ||
-      !make_map_f32(&tmdC, dC, V, D))
-    return CCE_ERR_CUDA;
   char* ws = reinterpret_cast<char*>(workspace);
   unsigned long long* status = reinterpret_cast<unsigned long long*>(ws);
   unsigned long long* accE = fixed ? reinterpret_cast<unsigned long long*>(ws + bp.off_accE) : nullptr;
   unsigned long long* accC = fixed ? reinterpret_cast<unsigned long long*>(ws + bp.off_accC) : nullptr;
+  // the reduction targets: fp32 dE / dC, or in fixed-point mode the int64
+  // accumulators (dE / dC may then hold bf16)
+  const bool red_maps_ok = fixed ? (make_map_u64(&tmdE, accE, N, D) && make_map_u64(&tmdC, accC, V, D))
+                                 : (make_map_f32(&tmdE, dE, N, D) && make_map_f32(&tmdC, dC, V, D));
+  if (!make_map(&tmE, E, N, D, BM) || !make_map(&tmC, C, V, D, BN) || !make_map(&tmCq, C, V, D, 64) ||
+      !red_maps_ok)
+    return CCE_ERR_CUDA;
   const bool filter_on = filter_eps > 0.f;
   const bool prepared = (flags & CCE_BWD_PREPARED) != 0;
   if (prepared && (filter_on || fixed)) {
@@ -519,7 +562,8 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   }
   if (fixed) {
     if (cudaMemsetAsync(accE, 0, (size_t)N * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
-    if (cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    // with the filter on only visited vocabulary tiles are cleared, after the pre-pass
+    if (!filter_on && cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
   } else if (!accumulate) {
     const bool stripes = (flags & CCE_BWD_STRIPES) && !(filter_eps > 0.f);
     if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
@@ -555,6 +599,7 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.withhold_loads = g_withhold_loads.load();
   a.pf = g_bwd_pf.load();
+  a.red_pf = g_bwd_red_pf.load();
   a.trace = g_bwd_trace.load();
   a.trace_cap = g_bwd_trace_cap.load();
 
@@ -582,19 +627,24 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     if (launch_enorm(E, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (filter_on && launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (fixed && launch_fixed_prep(dloss, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    if (fixed && filter_on &&
+        launch_clear_visited_rows(accC, (int)V, (int)D, pp.count, pp.hdr, di.sms, stream) != cudaSuccess)
+      return CCE_ERR_CUDA;
   }
   if ((flags & CCE_BWD_STRIPES) && !filter_on && !fixed)
-    return backward_stripes(E, C, dE, dC, bp, a, accumulate, di.sms, ws, stream);
+    return backward_stripes(E, C, dE, dC, bp, a, accumulate, (flags & CCE_BWD_DETERMINISTIC) != 0, di.sms, ws,
+                            stream);
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (launch_bwd(tmE, tmC, tmCq, tmdE, tmdC, a, grid, g_bwd_variant.load(), stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (fixed) {
     const unsigned* hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);
-    if (launch_fixed_to_out(accE, dE, (size_t)N * D, hdr, (int)N, bf16_out, accumulate, di.sms, stream) !=
-            cudaSuccess ||
-        launch_fixed_to_out(accC, dC, (size_t)V * D, hdr, (int)N, bf16_out, accumulate, di.sms, stream) !=
-            cudaSuccess)
+    const unsigned* count = filter_on ? reinterpret_cast<const unsigned*>(ws + bp.off_count) : nullptr;
+    if (launch_fixed_to_out(accE, dE, (size_t)N * D, hdr, (int)N, bf16_out, accumulate, nullptr, (int)D, di.sms,
+                            stream) != cudaSuccess ||
+        launch_fixed_to_out(accC, dC, (size_t)V * D, hdr, (int)N, bf16_out, accumulate, count, (int)D, di.sms,
+                            stream) != cudaSuccess)
       return CCE_ERR_CUDA;
   }
   return CCE_OK;

@@ -166,6 +166,35 @@ __device__ __forceinline__ void fixed_red_block32(uint8_t* xb, int lane, const f
   __syncwarp();
 }
 
+// Deterministic mode through the TMA engine: the 32 x 32 block, each value
+// rounded once to 64-bit fixed point round(x * scale), is added to the int64
+// accumulator by two bulk tensor reduce-adds (the map's element type is u64
+// and its box {16, 32}: 128-byte rows, 128-byte swizzle), the halves staged
+// in turn in the warp's 4 KB buffer.  Integer addition is associative, so
+// the totals do not depend on the order in which the operations land.
+// Columns from ncols on lie past the tensor and are not sent.
+__device__ __forceinline__ void tma_fixed_block32(uint8_t* xb, int lane, const float (&v)[32], const CUtensorMap* map,
+                                                  int x, int y, int ncols, float scale) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (16 * h >= ncols) break;
+    if (lane == 0) bulk_wait_group_read0();  // the buffer's previous contents have been read
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const long long a0 = __float2ll_rn(v[16 * h + 2 * q] * scale);
+      const long long a1 = __float2ll_rn(v[16 * h + 2 * q + 1] * scale);
+      *reinterpret_cast<longlong2*>(xb + lane * 128 + ((q ^ (lane & 7)) << 4)) = make_longlong2(a0, a1);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_reduce_add_2d(map, xb, x + 16 * h, y);
+      bulk_commit_group();
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -327,10 +356,33 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
         const int q1 = __ffs(qmask) - 1;
         const int n_cst = umask ? (nkb + cpack - 1) / cpack : 0;
         const int n_sst = tn >= 0 ? nkb : 0;
+        // L2 prefetch of the fp32 dE / dC rows this tile's reductions add
+        // into (the live 32-row pieces of d slice kb), a.red_pf slices ahead
+        // of the slice being loaded, so the reduce-adds find their lines in
+        // L2 instead of filling them from DRAM one by one.
+        auto pf_red = [&](int kb) {
+          if (kb < 0 || kb >= nkb) return;
+#pragma unroll 1
+          for (int q = 0; q < 2; ++q) {
+            const int x = kb * BK + q * 32;
+            if (x >= a.D) break;
+#pragma unroll 1
+            for (int g = 0; g < 4; ++g)
+              if (rows_live(umask, g) && m * BM + 32 * g < a.N) tma_prefetch_l2_2d(&tmdE, x, m * BM + 32 * g);
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c)
+              if (chunk_live(umask, c) && vt * BN + 32 * c < a.V) tma_prefetch_l2_2d(&tmdC, x, vt * BN + 32 * c);
+          }
+        };
+        const bool red_pf = a.red_pf > 0 && umask != 0u && a.accE == nullptr && RED == 0;
+        if (red_pf)
+          for (int i = 0; i < a.red_pf; ++i) pf_red(nkb - 1 - i);
         for (int j = 0; j < max(n_cst, n_sst); ++j) {
           if (j < n_cst) {
             const int kb0 = nkb - 1 - cpack * j;
             const int ns = (cpack == 2 && kb0 >= 1) ? 2 : 1;  // d slices in this stage
+            if (red_pf)
+              for (int sl = 0; sl < ns; ++sl) pf_red(kb0 - sl - a.red_pf);
             if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
             mbar_arrive_expect_tx(&full[stage], (uint32_t)ns * c_bytes);
             uint8_t* b_st = sB + stage * B_STAGE_BYTES;
@@ -662,7 +714,10 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
               float v[32];
               if (mine) tmem_ld32(tmem_base + lane_addr + tm_de(b) + q * 32, v);
               if (mine && d0 + q * 32 < a.D && row0 < a.N) {
-                if (fixed)
+                if (fixed && RED == 0)
+                  tma_fixed_block32(next_xb(), lane, v, &tmdE, d0 + q * 32, row0, min(32, a.D - (d0 + q * 32)),
+                                    fx_scale);
+                else if (fixed)
                   fixed_red_block32(next_xb(), lane, v, a.accE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D,
                                     rows_valid, min(32, a.D - (d0 + q * 32)), fx_scale);
                 else if (RED == 1)
@@ -683,7 +738,10 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
             float v[32];
             if (mine) tmem_ld32(tmem_base + lane_addr + tm_dc(b) + q * 32, v);
             if (mine && d0 + q * 32 < a.D && vr0 < a.V) {
-              if (fixed)
+              if (fixed && RED == 0)
+                tma_fixed_block32(next_xb(), lane, v, &tmdC, d0 + q * 32, vr0, min(32, a.D - (d0 + q * 32)),
+                                  fx_scale);
+              else if (fixed)
                 fixed_red_block32(next_xb(), lane, v, a.accC + (size_t)vr0 * a.D + d0 + q * 32, (size_t)a.D,
                                   __ballot_sync(0xffffffffu, vr0 + lane < a.V), min(32, a.D - (d0 + q * 32)),
                                   fx_scale);

@@ -67,6 +67,14 @@ __device__ __forceinline__ void pruned_sub(const PrepArgs& p, unsigned long long
   atomicAdd(p.status + ST_PRUNED, 0ull - units);  // modulo 2^64: order of the updates is free
 }
 
+// Vocabulary tile v can receive a gradient only if the backward visits it:
+// with the filter on, when some token block is not flat (every tile is
+// visited) or some flat block has a label in v.  Rows of the other tiles
+// of dC are exactly zero.
+__device__ __forceinline__ bool vtile_visited(const unsigned* count, const unsigned* hdr, int all, int v) {
+  return all || hdr[HDR_NNF] != 0u || count[v] != 0u;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(256) prep_cnorm_kernel(const __nv_bfloat16* __restrict__ C, PrepArgs p) {
@@ -215,15 +223,21 @@ __global__ void __launch_bounds__(256) prep_fixed_kernel(const float* __restrict
 // Deterministic mode: int64 fixed-point accumulators -> fp32 or bf16 output
 // (written, or with accumulate added to what the output holds: one add per
 // entry, so the result stays reproducible).
+// count / D: when count is non-null the accumulator is dC and only the rows
+// of visited vocabulary tiles (vtile_visited) were cleared and accumulated;
+// the others are exactly zero and are not read.
 __global__ void __launch_bounds__(256) fixed_to_out_kernel(const unsigned long long* __restrict__ acc, void* out,
                                                            size_t n, const unsigned* __restrict__ hdr, int N,
-                                                           int bf16, int accumulate) {
+                                                           int bf16, int accumulate,
+                                                           const unsigned* __restrict__ count, int D) {
   const int s = fixed_point_exponent(__uint_as_float(hdr[HDR_CMAX]), __uint_as_float(hdr[HDR_EMAX]),
                                      __uint_as_float(hdr[HDR_DLMAX]), N);
   const double inv = ldexp(1.0, -s);
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; 2 * i < n; i += stride) {
-    const ulonglong2 q = reinterpret_cast<const ulonglong2*>(acc)[i];   // n is even (D % 8 == 0)
+    const bool live_row = count == nullptr || vtile_visited(count, hdr, 0, (int)((2 * i) / (size_t)D) / BN);
+    const ulonglong2 q = live_row ? reinterpret_cast<const ulonglong2*>(acc)[i]   // n is even (D % 8 == 0)
+                                  : make_ulonglong2(0ull, 0ull);
     double x0 = (double)(long long)q.x * inv, x1 = (double)(long long)q.y * inv;
     if (bf16) {
       __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out) + i;
@@ -246,14 +260,33 @@ __global__ void __launch_bounds__(256) fixed_to_out_kernel(const unsigned long l
   }
 }
 
+// Fixed-point dC accumulator: clear the rows of visited vocabulary tiles only.
+__global__ void __launch_bounds__(256) clear_visited_rows_kernel(unsigned long long* __restrict__ acc, int V, int D,
+                                                                 const unsigned* __restrict__ count,
+                                                                 const unsigned* __restrict__ hdr) {
+  const size_t n2 = (size_t)V * D / 2;  // D is even
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += stride) {
+    const int row = (int)((2 * i) / (size_t)D);
+    if (vtile_visited(count, hdr, 0, row / BN)) reinterpret_cast<ulonglong2*>(acc)[i] = make_ulonglong2(0ull, 0ull);
+  }
+}
+
+cudaError_t launch_clear_visited_rows(unsigned long long* acc, int V, int D, const unsigned* count,
+                                      const unsigned* hdr, int sms, cudaStream_t stream) {
+  clear_visited_rows_kernel<<<sms * 8, 256, 0, stream>>>(acc, V, D, count, hdr);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream) {
   prep_fixed_kernel<<<sms, 256, 0, stream>>>(dloss, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
-                                bool bf16, bool accumulate, int sms, cudaStream_t stream) {
-  fixed_to_out_kernel<<<sms * 8, 256, 0, stream>>>(acc, out, n, hdr, N, bf16 ? 1 : 0, accumulate ? 1 : 0);
+                                bool bf16, bool accumulate, const unsigned* count, int D, int sms,
+                                cudaStream_t stream) {
+  fixed_to_out_kernel<<<sms * 8, 256, 0, stream>>>(acc, out, n, hdr, N, bf16 ? 1 : 0, accumulate ? 1 : 0, count, D);
   return cudaGetLastError();
 }
 

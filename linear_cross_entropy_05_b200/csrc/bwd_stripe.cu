@@ -28,7 +28,7 @@
 // them), then hands the task to both CTAs through a small ring in shared
 // memory.  Roles per CTA (192 threads): warp 0 TMA producer, warp 1 UMMA
 // issuer (leader CTA only), warps 2-5 epilogue.  Each CTA stages 32 KB of
-// operands per 64-wide K slice (5 stages) and double-buffers a 128 x 256 fp32
+// operands per 64-wide K slice (6 stages) and double-buffers a 128 x 256 fp32
 // accumulator in TMEM, so the epilogue of one task overlaps the MMAs of the
 // next.  No TMA multicast: every load reads this GPU's memory.
 #include <cuda.h>
@@ -42,9 +42,9 @@ namespace cce {
 
 namespace {
 
-constexpr int SP_STAGES = 5;
+constexpr int SP_STAGES = 6;
 constexpr int SP_STAGE_BYTES = 32768;          // per CTA: two 16 KB operand regions
-constexpr int SP_STAGING_PER_WARP = 16384;     // epilogue staging (bf16 G boxes or fp32 blocks)
+constexpr int SP_STAGING_PER_WARP = 8192;      // epilogue staging: two 4 KB boxes (bf16 G or fp32 blocks)
 constexpr int SP_RING = 4;                     // task hand-off slots
 constexpr int SP_CONSUMERS = 10;               // leader: MMA + 4 epilogue warps; peer: producer + 4 epilogue warps
 
@@ -82,7 +82,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;                                          // SP_STAGES x 32 KB
-  uint8_t* staging = smem + SP_STAGES * SP_STAGE_BYTES;            // 4 x 16 KB
+  uint8_t* staging = smem + SP_STAGES * SP_STAGE_BYTES;            // 4 x 8 KB
   uint64_t* bars = reinterpret_cast<uint64_t*>(staging + 4 * SP_STAGING_PER_WARP);
   uint64_t* full = bars;                          // leader: both CTAs' copies of a stage landed
   uint64_t* empty = bars + SP_STAGES;             // each CTA: stage free again
@@ -186,37 +186,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0;
       const long long total = stripe_total(P);
+      unsigned long long* trace = (a.trace && leader) ? a.trace + (size_t)(blockIdx.x >> 1) * a.trace_cap * 4 : nullptr;
+      // The leader draws task k+1 while it issues task k's loads, and reads
+      // the counter of its inputs a few stages before the end of task k, so
+      // neither round trip stalls the operand stream between tasks.
+      unsigned long long drawn_next = leader ? atomicAdd(a.next, 1ull) : 0ull;
+      StripeTaskDesc t_next{TASK_END, 0, 0, 0};
+      const unsigned* dep_ctr = nullptr;
+      unsigned dep_want = 0, dep_seen = 0;
+      bool next_known = false;
+      auto look_ahead = [&]() {
+        t_next = drawn_next < (unsigned long long)total ? stripe_decode(P, (long long)drawn_next)
+                                                        : StripeTaskDesc{TASK_END, 0, 0, 0};
+        dep_ctr = nullptr;
+        dep_want = 0;
+        if (t_next.type == TASK_A) {
+          if (t_next.s >= P.nbuf) {
+            const int s0 = t_next.s - P.nbuf;
+            dep_ctr = a.doneBC + s0;
+            dep_want = 8u * (unsigned)(stripe_nB(P, s0) + stripe_nC(P));
+          }
+        } else if (t_next.type == TASK_B) {
+          dep_ctr = a.doneA_v + t_next.a;
+          dep_want = 8u * (unsigned)P.n_m2;
+        } else if (t_next.type == TASK_C) {
+          dep_ctr = a.doneA_ms + (size_t)t_next.s * P.n_m2 + t_next.a;
+          dep_want = 8u * (unsigned)stripe_tiles(P, t_next.s);
+        }
+        dep_seen = dep_ctr ? ld_acquire_gpu(dep_ctr) : dep_want;
+        next_known = true;
+      };
       for (int k = 0;; ++k) {
         StripeTaskDesc t;
         if (leader) {
           const int slot = k & (SP_RING - 1);
           if (!mbar_wait(&task_empty[slot], ((uint32_t)(k / SP_RING) & 1u) ^ 1u, wc)) goto producer_done;
-          const unsigned long long drawn = atomicAdd(a.next, 1ull);
-          t = drawn < (unsigned long long)total ? stripe_decode(P, (long long)drawn)
-                                                : StripeTaskDesc{TASK_END, 0, 0, 0};
+          const uint64_t t_dep0 = trace ? global_timer_ns() : 0;
+          if (!next_known) look_ahead();
+          t = t_next;
+          next_known = false;
           // wait until the task's inputs are complete (bounded)
           if (t.type != TASK_END) {
-            const unsigned* ctr = nullptr;
-            unsigned want = 0;
-            if (t.type == TASK_A) {
-              if (t.s >= P.nbuf) {
-                const int s0 = t.s - P.nbuf;
-                ctr = a.doneBC + s0;
-                want = 8u * (unsigned)(stripe_nB(P, s0) + stripe_nC(P));
-              }
-            } else if (t.type == TASK_B) {
-              ctr = a.doneA_v + t.a;
-              want = 8u * (unsigned)P.n_m2;
-            } else {
-              ctr = a.doneA_ms + (size_t)t.s * P.n_m2 + t.a;
-              want = 8u * (unsigned)stripe_tiles(P, t.s);
-            }
-            if (ctr != nullptr && ld_acquire_gpu(ctr) < want) {
+            if (dep_seen < dep_want) {
               const uint64_t t0 = global_timer_ns();
               bool ok = false;
               while (true) {
                 __nanosleep(256);
-                if (ld_acquire_gpu(ctr) >= want) {
+                if (ld_acquire_gpu(dep_ctr) >= dep_want) {
                   ok = true;
                   break;
                 }
@@ -235,6 +251,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           st_shared_cluster_v4(mapa_shared(smem_u32(&task_slot[slot]), 1), d);
           mbar_arrive(&task_full[slot]);
           mbar_arrive_release_cluster(mapa_shared(smem_u32(&task_full[slot]), 1));
+          if (t.type != TASK_END) drawn_next = atomicAdd(a.next, 1ull);
+          if (trace && k < a.trace_cap && t.type != TASK_END) {
+            const uint64_t now = global_timer_ns();
+            trace[k * 4 + 0] = now;
+            trace[k * 4 + 3] = (unsigned long long)t.type | ((now - t_dep0) << 8);
+          }
         } else {
           if (!take_task(k, t, false)) goto producer_done;
           fence_proxy_async_global();
@@ -242,7 +264,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (t.type == TASK_END) break;
         const int nk = k_steps(t);
         const int r = (int)rank;
+        if (t.type == TASK_C && !a.withhold_loads) {
+          // the dE rows this task's epilogue will add into: into L2 while it computes
+          const int row0 = a.tok0 + t.a * 256 + r * 128;
+#pragma unroll 1
+          for (int g = 0; g < 4; ++g)
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c)
+              if (row0 + 32 * g < a.N && t.b * 256 + 32 * c < a.D)
+                tma_prefetch_l2_2d(&mp.dE, t.b * 256 + 32 * c, row0 + 32 * g);
+        }
         for (int kb = 0; kb < nk; ++kb) {
+          if (leader && kb == (nk > SP_STAGES ? nk - SP_STAGES : 0)) look_ahead();
           if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
           uint8_t* X = stages + stage * SP_STAGE_BYTES;
           uint8_t* Y = X + 16384;
@@ -359,12 +392,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     unsigned long long n_tiles = 0, n_units = 0;
+    unsigned long long* trace =
+        (a.trace && leader && ew == 0 && lane == 0) ? a.trace + (size_t)(blockIdx.x >> 1) * a.trace_cap * 4 : nullptr;
     for (int k = 0;; ++k) {
       StripeTaskDesc t;
       if (!take_task(k, t, true)) break;
       if (t.type == TASK_END) break;
       if (!warp_wait(&tfull[acc], acc_phase)) break;
       tc_fence_after();
+      if (trace && k < a.trace_cap) trace[k * 4 + 1] = global_timer_ns();
       const uint32_t tacc = tmem_base + lane_addr + (uint32_t)(acc * BN);
       if (t.type == TASK_A) {
         // row = token; columns = the 256 vocabulary entries of tile t.b
@@ -384,8 +420,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int ycol = (valid && yrel >= 0 && yrel < BN) ? (int)yrel : -1;
         const int ncols = min(BN, a.V - t.b * BN);
         const int sw = lane & 7;
+        const int gcol = (t.b - t.s * P.vt_per_s) * BN;
+        const int grow = (t.s % P.nbuf) * a.Ns_pad + t.a * 256 + r * 128 + ew * 32;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
+          if (c == 4) {
+            // the first 128 columns are stored: reuse their two staging boxes
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+          }
           float x[32];
           tmem_ld32(tacc + (uint32_t)(c * 32), x);
           uint32_t pk[16];
@@ -402,26 +445,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             }
             pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
           }
-          // box q = c / 2 (64 columns), this lane's 128-byte row, 128B swizzle
-          uint8_t* rowp = stg + (c >> 1) * 4096 + lane * 128;
+          // box (c / 2) % 2 of the staging (64 columns each), this lane's
+          // 128-byte row, 128B swizzle
+          uint8_t* rowp = stg + ((c >> 1) & 1) * 4096 + lane * 128;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int chunk = ((c & 1) * 4 + q) ^ sw;
             *reinterpret_cast<uint4*>(rowp + chunk * 16) =
                 make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
+          if (c == 7) {
+            // every column read from TMEM: the accumulator may be reused
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+          }
+          if (c == 3 || c == 7) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const int h = c >> 2;  // 128-column half
+              tma_store_2d(&mp.gSt, stg, gcol + h * 128, grow);
+              tma_store_2d(&mp.gSt, stg + 4096, gcol + h * 128 + 64, grow);
+              bulk_commit_group();
+            }
+          }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-        fence_proxy_async_smem();
-        __syncwarp();
         if (lane == 0) {
-          const int gcol = (t.b - t.s * P.vt_per_s) * BN;
-          const int grow = (t.s % P.nbuf) * a.Ns_pad + t.a * 256 + r * 128 + ew * 32;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tma_store_2d(&mp.gSt, stg + q * 4096, gcol + q * 64, grow);
-          bulk_commit_group();
           bulk_wait_group0();
           fence_proxy_async_global();
           red_release_gpu_add(a.doneA_v + t.b, 1u);
@@ -442,6 +492,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int rows_lim = isB ? a.V : a.N;
         const CUtensorMap* map = isB ? &mp.dC : &mp.dE;
         const bool add = isB ? (a.dC_add != 0) : true;
+        unsigned* tile_ctr = isB ? nullptr : a.doneC + (size_t)t.a * P.n_dc + t.b;
+        if (!isB && a.ordered && t.s > 0) {
+          // Ordered mode: this dE tile's reduce-adds follow those of the
+          // previous stripe, so every entry is summed in stripe order and the
+          // result does not depend on timing (bitwise reproducible).
+          int ok = 1;
+          if (lane == 0) {
+            const unsigned want = 8u * (unsigned)t.s;
+            if (ld_acquire_gpu(tile_ctr) < want) {
+              const uint64_t t0 = global_timer_ns();
+              ok = 0;
+              while (true) {
+                __nanosleep(128);
+                if (ld_acquire_gpu(tile_ctr) >= want) {
+                  ok = 1;
+                  break;
+                }
+                if (*abort_flag) break;
+                if (global_timer_ns() - t0 > a.wait_limit_ns) {
+                  *abort_flag = 1;
+                  break;
+                }
+              }
+            }
+            fence_proxy_async_global();
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          __syncwarp();
+          if (!ok) break;
+        }
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
@@ -473,9 +553,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           bulk_wait_group0();
           fence_proxy_async_global();
           red_release_gpu_add(a.doneBC + t.s, 1u);
+          if (tile_ctr) red_release_gpu_add(tile_ctr, 1u);
         }
         __syncwarp();
       }
+      if (trace && k < a.trace_cap) trace[k * 4 + 2] = global_timer_ns();
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;

@@ -120,6 +120,7 @@ struct BwdArgs {
   unsigned long long wait_limit_ns;
   int withhold_loads;   // test hook: the TMA producer issues nothing
   int pf;               // L2 prefetch distance of the operand streams in K slices (0: off)
+  int red_pf;           // L2 prefetch distance, in K slices, of the dE/dC rows the reductions add into (0: off)
   // profiling hook: per CTA and tile, globaltimer stamps (ns) at the start of
   // the tile, when its logits are in TMEM and when its gradient tile and
   // live mask are published; [grid][trace_cap][4] u64, null when off
@@ -226,6 +227,7 @@ __host__ __device__ inline StripeTaskDesc stripe_decode(const StripePlan& p, lon
 //   doneA_v[n_vtile]        A tasks of vocabulary tile vt
 //   doneA_ms[n_s][n_m2]     A tasks of token block m2 in stripe s
 //   doneBC[n_s]             B and C tasks of stripe s
+//   doneC[n_m2][n_dc]       C tasks of each dE tile (ordered mode)
 //   next                    the next task to hand out
 struct StripeArgs {
   StripePlan p;
@@ -243,7 +245,15 @@ struct StripeArgs {
   unsigned* doneA_v;
   unsigned* doneA_ms;
   unsigned* doneBC;
+  unsigned* doneC;       // [n_m2][n_dc] C tasks of each dE tile (ordered mode)
   unsigned long long* next;
+  int ordered;           // 1: the stripes' reduce-adds into a dE tile happen in stripe order
+  // profiling hook: per CTA pair and task, globaltimer stamps (ns) when the
+  // task was handed out, when its accumulator was complete and when its
+  // epilogue finished, then the task kind | (ns spent waiting for its inputs
+  // << 8); [pairs][trace_cap][4] u64, null when off
+  unsigned long long* trace;
+  int trace_cap;
   unsigned long long* status;
   unsigned long long wait_limit_ns;
   int withhold_loads;    // test hook: the TMA producers issue nothing

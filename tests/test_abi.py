@@ -147,9 +147,12 @@ def test_backward_ex_workspace_and_flags(lib):
     assert cce_backward_workspace_size_ex(N, D, V, 4) == base   # accumulate alone: no extra workspace
     assert cce_backward_workspace_size_ex(N, D, V, 8) == base   # prepared: no extra workspace
     # stripes: counters + three bf16 stripe buffers of 8192 tokens x 2048 columns
-    n_vt, n_s = -(-V // 256), -(-V // 2048)
-    ctr = up(8 + 4 * (n_vt + n_s * 32 + n_s))
+    n_vt, n_s, n_dc = -(-V // 256), -(-V // 2048), -(-D // 256)
+    ctr = up(8 + 4 * (n_vt + n_s * 32 + n_s + 32 * n_dc))
     assert cce_backward_workspace_size_ex(N, D, V, 16) == base + ctr + up(3 * 8192 * 2048 * 2)
+    # deterministic with stripes: fixed stripe order, no int64 accumulators
+    assert cce_backward_workspace_size_ex(N, D, V, 17) == base + ctr + up(3 * 8192 * 2048 * 2)
+    assert cce_backward_workspace_size_ex(N, D, V, 18) == 0     # bf16 outputs and stripes do not combine
     # token super-blocks of 16384 bound the stripe buffers whatever N
     big = cce_backward_workspace_size_ex(65536, 2048, 262144, 16) - cce_backward_workspace_size(65536, 2048, 262144)
     assert big < 3 * 16384 * 2048 * 2 + (1 << 20)
@@ -158,7 +161,7 @@ def test_backward_ex_workspace_and_flags(lib):
     args = [P, P, P, P, P, 256, 256, 4096, -100, 0.0, 0, P, P, P, 1 << 30, 0]
     args[10] = 32
     assert cce_backward_ex(*args, check=False) == 1          # unknown flag: rejected on the host
-    for flags in (3, 4, 7, 8, 15, 16, 31):
+    for flags in (3, 4, 7, 8, 15, 16, 17, 21):
         args[10] = flags
         assert cce_backward_ex(*args, check=False) == 4      # valid, but no device here
 

@@ -292,3 +292,19 @@ def test_filter_decision_at_the_threshold(side):
     assert st["live_tiles"] == int(live.sum()) == 2 + (side < 0)   # two label units (+ the edge unit)
     assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
+
+
+@pytest.mark.parametrize("slices", [2, 6])
+def test_reduce_prefetch_keeps_the_results(slices):
+    # the L2 prefetch of the reduction targets is a hint: same gradients
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=1000, V=20000)
+    L.cce_debug_set_reduce_prefetch(slices)
+    try:
+        inp, dloss, olse, gE, gC, st = _run(w, EPS)
+    finally:
+        L.cce_debug_set_reduce_prefetch(0)
+    assert st["status"] == 0
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=TILE)
+    assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF

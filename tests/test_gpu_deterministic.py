@@ -28,8 +28,12 @@ def _bwd(E, C, y, lse, dl, eps, **kw):
     return dE, dC, st
 
 
+@pytest.mark.parametrize("stripes", [None, False], ids=["default-path", "fixed-point"])
 @pytest.mark.parametrize("w,eps", CASES, ids=[c[0].name + ("-filter" if c[1] else "") for c in CASES])
-def test_deterministic_backward_is_bitwise_reproducible_and_matches_oracle(w, eps):
+def test_deterministic_backward_is_bitwise_reproducible_and_matches_oracle(w, eps, stripes):
+    # with the filter off the default path is the stripe kernel summing in
+    # stripe order; stripes=False (and the filter on) take the int64
+    # fixed-point accumulation
     import torch
     inp = synth.make_inputs(w)
     E, C, y = to_dev(inp)
@@ -37,8 +41,8 @@ def test_deterministic_backward_is_bitwise_reproducible_and_matches_oracle(w, ep
     dloss = synth.random_dloss(8, w.N)
     dl = torch.from_numpy(dloss).cuda()
     lse_t = torch.from_numpy(lse).cuda()
-    a = _bwd(E, C, y, lse_t, dl, eps, deterministic=True)
-    b = _bwd(E, C, y, lse_t, dl, eps, deterministic=True)
+    a = _bwd(E, C, y, lse_t, dl, eps, deterministic=True, stripes=stripes)
+    b = _bwd(E, C, y, lse_t, dl, eps, deterministic=True, stripes=stripes)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])       # same bits
     assert a[2]["live_tiles"] == b[2]["live_tiles"]
     ref = _bwd(E, C, y, lse_t, dl, eps)                               # atomic fp32 accumulation
@@ -61,7 +65,7 @@ def test_bf16_gradient_outputs(w, eps):
     lse_t = torch.from_numpy(lse).cuda()
     gE, gC, _ = _bwd(E, C, y, lse_t, dl, eps, bf16_grads=True)
     assert gE.dtype == torch.bfloat16 and gC.dtype == torch.bfloat16
-    fE, fC, _ = _bwd(E, C, y, lse_t, dl, eps, deterministic=True)
+    fE, fC, _ = _bwd(E, C, y, lse_t, dl, eps, deterministic=True, stripes=False)
     # the bf16 outputs are the deterministic fp32 results rounded once
     assert torch.equal(gE, fE.to(torch.bfloat16)) or rel_fro(gE.float().cpu().numpy(), fE.cpu().numpy()) < 4e-3
     _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
@@ -151,9 +155,11 @@ def test_prepared_backward_equals_unprepared(eps):
     ready.record(side)
     loss, lse = L.forward(E, C, y, IGN, workspace=ws_f)
     main.wait_event(ready)
-    dE_p, dC_p = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws_b, deterministic=True, prepared=True)
+    # (the fixed-point path, which uses max_v |C_v| with the filter on or off)
+    dE_p, dC_p = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws_b, deterministic=True, prepared=True,
+                            stripes=False)
     st_p = L.read_status(ws_b)
-    dE, dC = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws_a, deterministic=True)
+    dE, dC = L.backward(E, C, y, lse, dl, eps, IGN, workspace=ws_a, deterministic=True, stripes=False)
     st = L.read_status(ws_a)
     assert st_p["status"] == 0 and st["status"] == 0
     for k in ("live_tiles", "dead_tiles", "pruned_tiles", "logit_tiles"):
