@@ -360,9 +360,10 @@ def run_gpu(args, w):
     # Side stream during the (tensor-bound) forward: the classifier-only part
     # of the backward's pre-pass (cce_backward_prepare: max_v |C_v|, one read
     # of C) and, by default, the clearing of the fp32 dE/dC, into which the
-    # backward then adds (CCE_BWD_ACCUMULATE); the fixed-point modes write
-    # their outputs anyway.
-    overlap_zero = not (args.deterministic or args.bf16_grads or args.no_overlap_zero)
+    # backward then adds (CCE_BWD_ACCUMULATE; in the deterministic mode the
+    # conversion pass then adds once per entry and leaves the rows of
+    # unvisited vocabulary tiles alone); the bf16 outputs are written anyway.
+    overlap_zero = not (args.bf16_grads or args.no_overlap_zero)
     # (the classifier bound is used only by the filter and the fixed-point modes)
     prepare = not args.no_prepare and (eps > 0 or args.deterministic or args.bf16_grads)
     side_stream = torch.cuda.Stream(device=dev)

@@ -45,6 +45,16 @@ CCE_API void cce_debug_withhold_loads(int on);
  * CCE_ERR_INVALID_ARG outside [0, 64]. */
 CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
 
+/* Tuning knobs of the dense stripe backward (CCE_BWD_STRIPES), for A/B
+ * measurement: tokens_per_launch (a multiple of 256, at most 16384; 0 = the
+ * default 16384) bounds the tokens one launch takes (fewer tokens per launch
+ * keep the stripe buffers, E and dE of a launch in L2, at the cost of adding
+ * dC over more launches); dE_prefetch (0 or 1, default 0) asks for the dE
+ * rows of each dE-tile task in L2 when the task starts.  Same results up to
+ * fp32 summation order.  Process-wide.  Returns CCE_ERR_INVALID_ARG for other
+ * values. */
+CCE_API cce_status_t cce_debug_set_stripe_params(int tokens_per_launch, int dE_prefetch);
+
 /* L2 prefetch distance, in 64-wide K slices, of the fp32 dE / dC rows that
  * the filtered backward kernel's bulk reduce-adds add into: while loading
  * the operands of contraction slice k, its TMA producer asks for the live

@@ -87,6 +87,8 @@ def load_library():
         lib.cce_debug_set_kernel_events.restype = ctypes.c_int
         lib.cce_debug_set_prefetch.argtypes = [ctypes.c_int, ctypes.c_int]
         lib.cce_debug_set_prefetch.restype = ctypes.c_int
+        lib.cce_debug_set_stripe_params.argtypes = [ctypes.c_int, ctypes.c_int]
+        lib.cce_debug_set_stripe_params.restype = ctypes.c_int
         lib.cce_debug_set_reduce_prefetch.argtypes = [ctypes.c_int]
         lib.cce_debug_set_reduce_prefetch.restype = ctypes.c_int
         lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 5 + [c_vp, c_i64]
@@ -273,3 +275,10 @@ def cce_debug_set_reduce_prefetch(slices: int) -> None:
     """L2 prefetch distance (64-wide K slices) of the filtered backward's
     reduction targets (live dE / dC rows); 0 = off."""
     _check(load_library().cce_debug_set_reduce_prefetch(int(slices)), "cce_debug_set_reduce_prefetch")
+
+
+def cce_debug_set_stripe_params(tokens_per_launch: int = 0, dE_prefetch: int = 0) -> None:
+    """Stripe backward knobs (A/B): tokens per launch (multiple of 256, <= 16384;
+    0 = default) and the L2 prefetch of dE rows for dE-tile tasks (0/1)."""
+    _check(load_library().cce_debug_set_stripe_params(int(tokens_per_launch), int(dE_prefetch)),
+           "cce_debug_set_stripe_params")

@@ -208,9 +208,11 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
 // Stripe backward (CCE_BWD_STRIPES, filter off): 256-token blocks per launch
 // (token super-block; dC gathers the super-blocks by reduce-adds) and
 // vocabulary tiles per stripe.
-constexpr int kStripeMaxM2 = 64;     // 16384 tokens per launch
+constexpr int kStripeMaxM2 = 64;     // 16384 tokens per launch (upper bound; workspace sized for it)
 constexpr int kStripeVtiles = 8;     // 2048 vocabulary columns per stripe
 constexpr int kStripeBuffers = 3;
+std::atomic<int> g_stripe_m2{kStripeMaxM2};  // token blocks per launch actually used (A/B knob)
+std::atomic<int> g_stripe_dE_pf{0};          // L2 prefetch of the dE rows of dE-tile tasks (measured: no gain)
 
 struct StripeLayout {
   StripePlan p;          // of a full super-block
@@ -399,6 +401,15 @@ cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices) {
   return CCE_OK;
 }
 
+cce_status_t cce_debug_set_stripe_params(int tokens_per_launch, int dE_prefetch) {
+  if (tokens_per_launch < 0 || tokens_per_launch > kStripeMaxM2 * 256 || tokens_per_launch % 256 != 0 ||
+      dE_prefetch < 0 || dE_prefetch > 1)
+    return CCE_ERR_INVALID_ARG;
+  g_stripe_m2.store(tokens_per_launch ? tokens_per_launch / 256 : kStripeMaxM2);
+  g_stripe_dE_pf.store(dE_prefetch);
+  return CCE_OK;
+}
+
 cce_status_t cce_debug_set_reduce_prefetch(int slices) {
   if (slices < 0 || slices > 64) return CCE_ERR_INVALID_ARG;
   g_bwd_red_pf.store(slices);
@@ -495,13 +506,16 @@ cce_status_t backward_stripes(const void* E, const void* C, void* dE, void* dC, 
   sa.withhold_loads = a.withhold_loads;
   sa.trace = a.trace;
   sa.trace_cap = a.trace_cap;
+  sa.dE_prefetch = g_stripe_dE_pf.load();
   const int grid = sms & ~1;
   const int n_m2_total = (a.N + 255) / 256;
+  const int m2_per_launch = std::max(1, std::min(L.p.n_m2, g_stripe_m2.load()));
+  const int n_sb = (n_m2_total + m2_per_launch - 1) / m2_per_launch;
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
-  for (int sb = 0; sb < L.n_sb; ++sb) {
+  for (int sb = 0; sb < n_sb; ++sb) {
     sa.p = L.p;
-    sa.p.n_m2 = std::min(L.p.n_m2, n_m2_total - sb * L.p.n_m2);
-    sa.tok0 = sb * L.p.n_m2 * 256;
+    sa.p.n_m2 = std::min(m2_per_launch, n_m2_total - sb * m2_per_launch);
+    sa.tok0 = sb * m2_per_launch * 256;
     sa.Ns_pad = sa.p.n_m2 * 256;   // buffer row stride of this launch
     sa.dC_add = (accumulate || sb > 0) ? 1 : 0;
     if (cudaMemsetAsync(ctr, 0, L.ctr_bytes, stream) != cudaSuccess) return CCE_ERR_CUDA;

@@ -236,6 +236,7 @@ __global__ void __launch_bounds__(256) fixed_to_out_kernel(const unsigned long l
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; 2 * i < n; i += stride) {
     const bool live_row = count == nullptr || vtile_visited(count, hdr, 0, (int)((2 * i) / (size_t)D) / BN);
+    if (!live_row && accumulate) continue;  // adds nothing: the output keeps its contents
     const ulonglong2 q = live_row ? reinterpret_cast<const ulonglong2*>(acc)[i]   // n is even (D % 8 == 0)
                                   : make_ulonglong2(0ull, 0ull);
     double x0 = (double)(long long)q.x * inv, x1 = (double)(long long)q.y * inv;

@@ -264,7 +264,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (t.type == TASK_END) break;
         const int nk = k_steps(t);
         const int r = (int)rank;
-        if (t.type == TASK_C && !a.withhold_loads) {
+        if (t.type == TASK_C && a.dE_prefetch && !a.withhold_loads) {
           // the dE rows this task's epilogue will add into: into L2 while it computes
           const int row0 = a.tok0 + t.a * 256 + r * 128;
 #pragma unroll 1

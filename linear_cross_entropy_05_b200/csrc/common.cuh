@@ -248,6 +248,7 @@ struct StripeArgs {
   unsigned* doneC;       // [n_m2][n_dc] C tasks of each dE tile (ordered mode)
   unsigned long long* next;
   int ordered;           // 1: the stripes' reduce-adds into a dE tile happen in stripe order
+  int dE_prefetch;       // 1: dE-tile tasks ask for their dE rows in L2 when they start
   // profiling hook: per CTA pair and task, globaltimer stamps (ns) when the
   // task was handed out, when its accumulator was complete and when its
   // epilogue finished, then the task kind | (ns spent waiting for its inputs
