@@ -27,8 +27,9 @@
 // complete (counters in global memory, released by the epilogues that wrote
 // them), then hands the task to both CTAs through a small ring in shared
 // memory.  Roles per CTA (192 threads): warp 0 TMA producer, warp 1 UMMA
-// issuer (leader CTA only), warps 2-5 epilogue.  Each CTA stages 32 KB of
-// operands per 64-wide K slice (6 stages) and double-buffers a 128 x 256 fp32
+// issuer (leader CTA only), warps 2-9 epilogue (two per TMEM lane group, one
+// per 128-column half).  Each CTA stages 32 KB of
+// operands per 64-wide K slice (5 stages) and double-buffers a 128 x 256 fp32
 // accumulator in TMEM, so the epilogue of one task overlaps the MMAs of the
 // next.  No TMA multicast: every load reads this GPU's memory.
 #include <cuda.h>
@@ -42,11 +43,19 @@ namespace cce {
 
 namespace {
 
-constexpr int SP_STAGES = 6;
+constexpr int SP_STAGES = 5;
 constexpr int SP_STAGE_BYTES = 32768;          // per CTA: two 16 KB operand regions
+constexpr int SP_EPI_WARPS = 8;                // two per TMEM lane group, one per 128-column half
+constexpr int SP_THREADS = 64 + 32 * SP_EPI_WARPS;
 constexpr int SP_STAGING_PER_WARP = 8192;      // epilogue staging: two 4 KB boxes (bf16 G or fp32 blocks)
 constexpr int SP_RING = 4;                     // task hand-off slots
-constexpr int SP_CONSUMERS = 10;               // leader: MMA + 4 epilogue warps; peer: producer + 4 epilogue warps
+constexpr int SP_CONSUMERS = 2 + 2 * SP_EPI_WARPS;  // leader: MMA + epilogue warps; peer: producer + epilogue warps
+constexpr unsigned SP_DONE = 2 * SP_EPI_WARPS; // completion arrivals per task (epilogue warps of both CTAs)
+
+// d-columns of a dC / dE task's chunk: 256, or 128 for a last chunk that
+// narrow (D = 896: three chunks of 256 and one of 128), so the tensor cores
+// do not multiply columns that lie past D.
+__device__ __forceinline__ int chunk_width(int D, int dc) { return D - dc * 256 <= 128 ? 128 : 256; }
 
 struct StripeMaps {
   CUtensorMap eA;    // E   bf16 [N][D]        box {64, 128}: A tasks, K-major token rows
@@ -77,13 +86,13 @@ __device__ __forceinline__ void stage_f32_block(uint8_t* xb, int lane, const flo
 
 }  // namespace
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
     bwd_stripe_kernel(const __grid_constant__ StripeMaps mp, const StripeArgs a, __nv_bfloat16* G) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;                                          // SP_STAGES x 32 KB
-  uint8_t* staging = smem + SP_STAGES * SP_STAGE_BYTES;            // 4 x 8 KB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + 4 * SP_STAGING_PER_WARP);
+  uint8_t* staging = smem + SP_STAGES * SP_STAGE_BYTES;            // SP_EPI_WARPS x 8 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + SP_EPI_WARPS * SP_STAGING_PER_WARP);
   uint64_t* full = bars;                          // leader: both CTAs' copies of a stage landed
   uint64_t* empty = bars + SP_STAGES;             // each CTA: stage free again
   uint64_t* tfull = bars + 2 * SP_STAGES;         // each CTA: accumulator ready [2]
@@ -109,7 +118,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);
+      mbar_init(&tempty[b], 2 * SP_EPI_WARPS);
     }
     mbar_init(drain, 1);
     for (int r = 0; r < SP_RING; ++r) {
@@ -204,14 +213,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           if (t_next.s >= P.nbuf) {
             const int s0 = t_next.s - P.nbuf;
             dep_ctr = a.doneBC + s0;
-            dep_want = 8u * (unsigned)(stripe_nB(P, s0) + stripe_nC(P));
+            dep_want = SP_DONE * (unsigned)(stripe_nB(P, s0) + stripe_nC(P));
           }
         } else if (t_next.type == TASK_B) {
           dep_ctr = a.doneA_v + t_next.a;
-          dep_want = 8u * (unsigned)P.n_m2;
+          dep_want = SP_DONE * (unsigned)P.n_m2;
         } else if (t_next.type == TASK_C) {
           dep_ctr = a.doneA_ms + (size_t)t_next.s * P.n_m2 + t_next.a;
-          dep_want = 8u * (unsigned)stripe_tiles(P, t_next.s);
+          dep_want = SP_DONE * (unsigned)stripe_tiles(P, t_next.s);
         }
         dep_seen = dep_ctr ? ld_acquire_gpu(dep_ctr) : dep_want;
         next_known = true;
@@ -274,12 +283,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               if (row0 + 32 * g < a.N && t.b * 256 + 32 * c < a.D)
                 tma_prefetch_l2_2d(&mp.dE, t.b * 256 + 32 * c, row0 + 32 * g);
         }
+        // B / C tasks: this CTA's half of the chunk's d columns, in 64-wide boxes
+        const int nd = t.type == TASK_A ? 256 : chunk_width(a.D, t.b);
+        const int half_boxes = nd / 128;                 // 2, or 1 for a 128-wide chunk
+        const uint32_t cta_bytes = 16384u + (t.type == TASK_A ? 16384u : 8192u * (uint32_t)half_boxes);
         for (int kb = 0; kb < nk; ++kb) {
           if (leader && kb == (nk > SP_STAGES ? nk - SP_STAGES : 0)) look_ahead();
           if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
           uint8_t* X = stages + stage * SP_STAGE_BYTES;
           uint8_t* Y = X + 16384;
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * SP_STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2u * cta_bytes);
           if (!a.withhold_loads) {
             if (t.type == TASK_A) {
               // X = E[token rows of this CTA][64 d], Y = C[vocabulary rows of this CTA][64 d]
@@ -292,18 +305,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               const int grow = (t.s % P.nbuf) * a.Ns_pad + kb * BK;
               tma_load_2d_pair(X, &mp.gM, &full[stage], gcol, grow);
               tma_load_2d_pair(X + 8192, &mp.gM, &full[stage], gcol + 64, grow);
-              const int d0 = t.b * 256 + r * 128;
+              const int d0 = t.b * 256 + r * (nd / 2);
               tma_load_2d_pair(Y, &mp.eM, &full[stage], d0, a.tok0 + kb * BK);
-              tma_load_2d_pair(Y + 8192, &mp.eM, &full[stage], d0 + 64, a.tok0 + kb * BK);
+              if (half_boxes == 2) tma_load_2d_pair(Y + 8192, &mp.eM, &full[stage], d0 + 64, a.tok0 + kb * BK);
             } else {
               // X = G[this CTA's 128 token rows][64 stripe columns],
               // Y = C[64 stripe rows][this CTA's 128 d columns]
               tma_load_2d_pair(X, &mp.gK, &full[stage], kb * BK,
                                (t.s % P.nbuf) * a.Ns_pad + t.a * 256 + r * 128);
               const int v0 = t.s * P.vt_per_s * BN + kb * BK;
-              const int d0 = t.b * 256 + r * 128;
+              const int d0 = t.b * 256 + r * (nd / 2);
               tma_load_2d_pair(Y, &mp.cM, &full[stage], d0, v0);
-              tma_load_2d_pair(Y + 8192, &mp.cM, &full[stage], d0 + 64, v0);
+              if (half_boxes == 2) tma_load_2d_pair(Y + 8192, &mp.cM, &full[stage], d0 + 64, v0);
             }
             armed |= 1u << stage;
           }
@@ -327,6 +340,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC_A = idesc_bf16_f32(2 * BM, BN, false, false);
       constexpr uint32_t IDESC_B = idesc_bf16_f32(2 * BM, BN, true, true);
       constexpr uint32_t IDESC_C = idesc_bf16_f32(2 * BM, BN, false, true);
+      constexpr uint32_t IDESC_B128 = idesc_bf16_f32(2 * BM, 128, true, true);
+      constexpr uint32_t IDESC_C128 = idesc_bf16_f32(2 * BM, 128, false, true);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -339,6 +354,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         const int nk = k_steps(t);
+        const bool narrow = t.type != TASK_A && chunk_width(a.D, t.b) == 128;
+        const uint32_t idesc_b = narrow ? IDESC_B128 : IDESC_B;
+        const uint32_t idesc_c = narrow ? IDESC_C128 : IDESC_C;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, wc)) goto mma_done;
           tc_fence_after();
@@ -354,11 +372,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               // A = G^T (M = vocabulary, 64-column groups 8 KB apart; K = tokens, 128 B rows)
               // B = E (N = d, 64-column groups 8 KB apart; K = tokens)
               umma_bf16_pair(d_tmem, sdesc_sw128(xa + k16 * 2048, 8192, 1024),
-                             sdesc_sw128(ya + k16 * 2048, 8192, 1024), IDESC_B, acc_on);
+                             sdesc_sw128(ya + k16 * 2048, 8192, 1024), idesc_b, acc_on);
             } else {
               // A = G (K-major token rows), B = C (N = d groups 8 KB apart; K = vocabulary rows)
               umma_bf16_pair(d_tmem, sdesc_sw128(xa + k16 * 32, 16, 1024),
-                             sdesc_sw128(ya + k16 * 2048, 8192, 1024), IDESC_C, acc_on);
+                             sdesc_sw128(ya + k16 * 2048, 8192, 1024), idesc_c, acc_on);
             }
           }
           umma_commit_pair_mc(&empty[stage], 0x3);
@@ -382,18 +400,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
-    // ---------------- epilogue: 4 warps per CTA, one TMEM lane (row) per thread ----------------
-    const int ew = warp & 3;  // TMEM lane group of this warp
-    const uint32_t lane_addr = (uint32_t)(ew * 32) << 16;
+    // ---------------- epilogue: 8 warps per CTA, one TMEM lane (row) per thread ----------------
+    // Warp w may only read TMEM lanes 32 (w % 4) .. +31; warps 2-5 take the
+    // first 128 accumulator columns and warps 6-9 the last 128, so each lane
+    // group has one warp per half.
+    const int lg = warp & 3;                 // TMEM lane group of this warp
+    const int hsel = (warp - 2) >> 2;        // 128-column half of this warp
+    const uint32_t lane_addr = (uint32_t)(lg * 32) << 16;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-    uint8_t* stg = staging + ew * SP_STAGING_PER_WARP;
+    uint8_t* stg = staging + (warp - 2) * SP_STAGING_PER_WARP;
     const int r = (int)rank;
     int acc = 0;
     uint32_t acc_phase = 0;
     unsigned long long n_tiles = 0, n_units = 0;
-    unsigned long long* trace =
-        (a.trace && leader && ew == 0 && lane == 0) ? a.trace + (size_t)(blockIdx.x >> 1) * a.trace_cap * 4 : nullptr;
+    unsigned long long* trace = (a.trace && leader && warp == 2 && lane == 0)
+                                    ? a.trace + (size_t)(blockIdx.x >> 1) * a.trace_cap * 4
+                                    : nullptr;
     for (int k = 0;; ++k) {
       StripeTaskDesc t;
       if (!take_task(k, t, true)) break;
@@ -403,8 +426,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       if (trace && k < a.trace_cap) trace[k * 4 + 1] = global_timer_ns();
       const uint32_t tacc = tmem_base + lane_addr + (uint32_t)(acc * BN);
       if (t.type == TASK_A) {
-        // row = token; columns = the 256 vocabulary entries of tile t.b
-        const int row = a.tok0 + t.a * 256 + r * 128 + ew * 32 + lane;
+        // row = token; columns = this warp's 128 of the 256 vocabulary entries of tile t.b
+        const int row = a.tok0 + t.a * 256 + r * 128 + lg * 32 + lane;
         bool valid = row < a.N;
         long long yl = valid ? a.y[row] : a.ignore_index;
         if (yl == a.ignore_index) valid = false;
@@ -420,15 +443,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int ycol = (valid && yrel >= 0 && yrel < BN) ? (int)yrel : -1;
         const int ncols = min(BN, a.V - t.b * BN);
         const int sw = lane & 7;
-        const int gcol = (t.b - t.s * P.vt_per_s) * BN;
-        const int grow = (t.s % P.nbuf) * a.Ns_pad + t.a * 256 + r * 128 + ew * 32;
+        const int gcol = (t.b - t.s * P.vt_per_s) * BN + hsel * 128;
+        const int grow = (t.s % P.nbuf) * a.Ns_pad + t.a * 256 + r * 128 + lg * 32;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          if (c == 4) {
-            // the first 128 columns are stored: reuse their two staging boxes
-            if (lane == 0) bulk_wait_group_read0();
-            __syncwarp();
-          }
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = hsel * 4 + cc;  // 32-column chunk of the accumulator
           float x[32];
           tmem_ld32(tacc + (uint32_t)(c * 32), x);
           uint32_t pk[16];
@@ -445,38 +464,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             }
             pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
           }
-          // box (c / 2) % 2 of the staging (64 columns each), this lane's
-          // 128-byte row, 128B swizzle
-          uint8_t* rowp = stg + ((c >> 1) & 1) * 4096 + lane * 128;
+          // staging box cc / 2 (64 columns), this lane's 128-byte row, 128B swizzle
+          uint8_t* rowp = stg + (cc >> 1) * 4096 + lane * 128;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int chunk = ((c & 1) * 4 + q) ^ sw;
+            const int chunk = ((cc & 1) * 4 + q) ^ sw;
             *reinterpret_cast<uint4*>(rowp + chunk * 16) =
                 make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
-          if (c == 7) {
-            // every column read from TMEM: the accumulator may be reused
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-          }
-          if (c == 3 || c == 7) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              const int h = c >> 2;  // 128-column half
-              tma_store_2d(&mp.gSt, stg, gcol + h * 128, grow);
-              tma_store_2d(&mp.gSt, stg + 4096, gcol + h * 128 + 64, grow);
-              bulk_commit_group();
-            }
-          }
         }
+        // every column this warp needs is read from TMEM
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        fence_proxy_async_smem();
+        __syncwarp();
         if (lane == 0) {
+          tma_store_2d(&mp.gSt, stg, gcol, grow);
+          tma_store_2d(&mp.gSt, stg + 4096, gcol + 64, grow);
+          bulk_commit_group();
           bulk_wait_group0();
           fence_proxy_async_global();
           red_release_gpu_add(a.doneA_v + t.b, 1u);
           red_release_gpu_add(a.doneA_ms + (size_t)t.s * P.n_m2 + t.a, 1u);
-          if (ew == 0) {
+          if (lg == 0 && hsel == 0) {
             const int rows_here = a.N - (a.tok0 + t.a * 256 + r * 128);
             if (rows_here > 0) {
               n_tiles += 1;
@@ -486,12 +497,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         __syncwarp();
       } else {
-        // B: rows = vocabulary (dC), C: rows = tokens (dE); 256 d columns of chunk t.b
+        // B: rows = vocabulary (dC), C: rows = tokens (dE); this warp's half
+        // of the chunk's d columns
         const bool isB = t.type == TASK_B;
-        const int row0 = isB ? t.a * BN + r * 128 + ew * 32 : a.tok0 + t.a * 256 + r * 128 + ew * 32;
+        const int row0 = isB ? t.a * BN + r * 128 + lg * 32 : a.tok0 + t.a * 256 + r * 128 + lg * 32;
         const int rows_lim = isB ? a.V : a.N;
         const CUtensorMap* map = isB ? &mp.dC : &mp.dE;
         const bool add = isB ? (a.dC_add != 0) : true;
+        const int nd = chunk_width(a.D, t.b);
         unsigned* tile_ctr = isB ? nullptr : a.doneC + (size_t)t.a * P.n_dc + t.b;
         if (!isB && a.ordered && t.s > 0) {
           // Ordered mode: this dE tile's reduce-adds follow those of the
@@ -499,7 +512,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           // result does not depend on timing (bitwise reproducible).
           int ok = 1;
           if (lane == 0) {
-            const unsigned want = 8u * (unsigned)t.s;
+            const unsigned want = SP_DONE * (unsigned)t.s;
             if (ld_acquire_gpu(tile_ctr) < want) {
               const uint64_t t0 = global_timer_ns();
               ok = 0;
@@ -523,7 +536,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           if (!ok) break;
         }
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = hsel * 4 + cc;
+          if (c * 32 >= nd) break;  // a 128-wide chunk fills only the first half
           float v[32];
           tmem_ld32(tacc + (uint32_t)(c * 32), v);
           const int x0 = t.b * 256 + c * 32;
@@ -531,7 +546,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // Two staging buffers in turn: the block staged here two pieces ago
             // has been read once at most one group is still reading.  (Pieces
             // are skipped only from some c on, so the turn never breaks.)
-            uint8_t* xb = stg + (c & 1) * 4096;
+            uint8_t* xb = stg + (cc & 1) * 4096;
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
             stage_f32_block(xb, lane, v);
@@ -564,7 +579,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
     }
     if (lane == 0) bulk_wait_group0();
-    if (ew == 0 && lane == 0) {
+    if (lg == 0 && hsel == 0 && lane == 0) {
       atomicAdd(a.status + ST_TILES, n_tiles);
       atomicAdd(a.status + ST_LIVE_TILES, n_units);
     }
@@ -583,7 +598,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 }
 
 size_t bwd_stripe_smem_bytes() {
-  return 1024 + (size_t)SP_STAGES * SP_STAGE_BYTES + 4 * (size_t)SP_STAGING_PER_WARP + 512;
+  return 1024 + (size_t)SP_STAGES * SP_STAGE_BYTES + (size_t)SP_EPI_WARPS * SP_STAGING_PER_WARP + 512;
 }
 
 // maps: the nine tensor maps in the order of StripeMaps; grid: an even number of CTAs.
@@ -601,7 +616,7 @@ cudaError_t launch_bwd_stripe(const CUtensorMap* maps, const StripeArgs& a, void
   const size_t smem = bwd_stripe_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(bwd_stripe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  bwd_stripe_kernel<<<grid, NUM_THREADS, smem, stream>>>(mp, a, reinterpret_cast<__nv_bfloat16*>(G));
+  bwd_stripe_kernel<<<grid, SP_THREADS, smem, stream>>>(mp, a, reinterpret_cast<__nv_bfloat16*>(G));
   return cudaGetLastError();
 }
 
