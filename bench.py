@@ -579,7 +579,7 @@ def run_gpu(args, w):
                            classifier_norm=("cce_backward_prepare on the side stream during the forward"
                                             if prepare else "inside the backward call"),
                            l2_prefetch_slices=list(args.prefetch) if args.prefetch else [0, 0],
-                           reduce_prefetch_slices=args.reduce_prefetch),
+                           reduce_prefetch_slices=args.reduce_prefetch, l2_hints=bool(args.l2_hints)),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops (burst: the timed region is under a second)",
@@ -978,6 +978,8 @@ def main(argv=None):
                     help="L2 prefetch distances in K slices for the forward / backward operand streams (A/B)")
     ap.add_argument("--reduce-prefetch", type=int, default=None, metavar="SLICES",
                     help="L2 prefetch distance of the filtered backward's reduction targets (A/B; 0 = off)")
+    ap.add_argument("--l2-hints", action="store_true",
+                    help="L2 eviction priorities in the filtered backward (A/B)")
     ap.add_argument("--trace", action="store_true",
                     help="per-tile timeline of one backward launch (recompute wait, gradient tile, contraction)")
     ap.add_argument("--dense-trace", action="store_true",
@@ -991,7 +993,7 @@ def main(argv=None):
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
     if args.impl == "cce" and (args.fwd_variant != "pair" or args.bwd_variant or args.prefetch or
-                               args.reduce_prefetch is not None):
+                               args.reduce_prefetch is not None or args.l2_hints):
         import linear_cross_entropy_05_b200 as L
         L.cce_debug_set_forward_variant(1 if args.fwd_variant == "pair" else 0)
         L.cce_debug_set_backward_variant(args.bwd_variant)
@@ -999,6 +1001,8 @@ def main(argv=None):
             L.cce_debug_set_prefetch(*args.prefetch)
         if args.reduce_prefetch is not None:
             L.cce_debug_set_reduce_prefetch(args.reduce_prefetch)
+        if args.l2_hints:
+            L.cce_debug_set_l2_hints(True)
     if args.suite:
         return run_suite(args)
     if args.memory or args.trace:

@@ -64,6 +64,14 @@ CCE_API cce_status_t cce_debug_set_stripe_params(int tokens_per_launch, int dE_p
  * CCE_ERR_INVALID_ARG outside [0, 64]. */
 CCE_API cce_status_t cce_debug_set_reduce_prefetch(int slices);
 
+/* L2 eviction priorities in the filtered backward kernel: while on, its TMA
+ * producer loads the classifier slices with an evict-first cache policy and
+ * its epilogue adds into dE with an evict-last policy, so the streamed
+ * classifier leaves L2 before the dE rows the reductions keep returning to.
+ * Hints only: same results.  For A/B measurement; 0 (the default) is off.
+ * Process-wide.  Returns CCE_ERR_INVALID_ARG for values other than 0, 1. */
+CCE_API cce_status_t cce_debug_set_l2_hints(int on);
+
 /* Profiling hook for the backward kernel's per-tile timeline.  While set,
  * every backward launch writes, for each CTA b (one per SM) and each of its
  * first tiles_per_cta tiles k, four u64 at trace[(b * tiles_per_cta + k) * 4]:

@@ -89,6 +89,8 @@ def load_library():
         lib.cce_debug_set_prefetch.restype = ctypes.c_int
         lib.cce_debug_set_stripe_params.argtypes = [ctypes.c_int, ctypes.c_int]
         lib.cce_debug_set_stripe_params.restype = ctypes.c_int
+        lib.cce_debug_set_l2_hints.argtypes = [ctypes.c_int]
+        lib.cce_debug_set_l2_hints.restype = ctypes.c_int
         lib.cce_debug_set_reduce_prefetch.argtypes = [ctypes.c_int]
         lib.cce_debug_set_reduce_prefetch.restype = ctypes.c_int
         lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 5 + [c_vp, c_i64]
@@ -282,3 +284,9 @@ def cce_debug_set_stripe_params(tokens_per_launch: int = 0, dE_prefetch: int = 0
     0 = default) and the L2 prefetch of dE rows for dE-tile tasks (0/1)."""
     _check(load_library().cce_debug_set_stripe_params(int(tokens_per_launch), int(dE_prefetch)),
            "cce_debug_set_stripe_params")
+
+
+def cce_debug_set_l2_hints(on: bool) -> None:
+    """L2 eviction priorities in the filtered backward (evict-first classifier
+    slices, evict-last dE reductions); A/B knob, off by default."""
+    _check(load_library().cce_debug_set_l2_hints(1 if on else 0), "cce_debug_set_l2_hints")

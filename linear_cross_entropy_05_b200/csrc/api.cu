@@ -56,6 +56,7 @@ std::atomic<int> g_withhold_loads{0};
 std::atomic<int> g_fwd_pf{0};  // L2 prefetch distances (K slices) of the forward / backward operand streams
 std::atomic<int> g_bwd_pf{0};
 std::atomic<int> g_bwd_red_pf{0};  // L2 prefetch distance (K slices) of the backward's reduction targets
+std::atomic<int> g_bwd_l2_hints{0};  // L2 eviction priorities in the filtered backward (A/B)
 std::atomic<unsigned long long*> g_bwd_trace{nullptr};
 std::atomic<int> g_bwd_trace_cap{0};
 
@@ -256,8 +257,6 @@ struct BwdPlan {
 
 constexpr unsigned kBwdFlagsAll =
     CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE | CCE_BWD_PREPARED | CCE_BWD_STRIPES;
-constexpr unsigned kBwdFixedPoint = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS;  // int64 accumulators
-
 // Whether these flags take the int64 fixed-point accumulation.  With
 // CCE_BWD_STRIPES the deterministic mode is served by the stripe kernel's
 // fixed reduction order instead (filter off only, fp32 outputs).
@@ -413,6 +412,12 @@ cce_status_t cce_debug_set_stripe_params(int tokens_per_launch, int dE_prefetch)
 cce_status_t cce_debug_set_reduce_prefetch(int slices) {
   if (slices < 0 || slices > 64) return CCE_ERR_INVALID_ARG;
   g_bwd_red_pf.store(slices);
+  return CCE_OK;
+}
+
+cce_status_t cce_debug_set_l2_hints(int on) {
+  if (on < 0 || on > 1) return CCE_ERR_INVALID_ARG;
+  g_bwd_l2_hints.store(on);
   return CCE_OK;
 }
 
@@ -614,6 +619,7 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.withhold_loads = g_withhold_loads.load();
   a.pf = g_bwd_pf.load();
   a.red_pf = g_bwd_red_pf.load();
+  a.l2_hints = g_bwd_l2_hints.load();
   a.trace = g_bwd_trace.load();
   a.trace_cap = g_bwd_trace_cap.load();
 

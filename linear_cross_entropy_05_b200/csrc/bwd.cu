@@ -70,7 +70,7 @@ __device__ __forceinline__ void tile_coords(int t, int n_mblk, int n_vtile, int 
 // the tensor's extent are clipped.
 template <int NXB>
 __device__ __forceinline__ void tma_red_block32(uint8_t* xb, int lane, const float (&v)[32], const CUtensorMap* map,
-                                                int x, int y) {
+                                                int x, int y, uint64_t policy = 0) {
   // the block issued NXB pieces ago (which used this buffer) has left it
   if (lane == 0) bulk_wait_group_read<NXB - 1>();
   __syncwarp();
@@ -81,7 +81,10 @@ __device__ __forceinline__ void tma_red_block32(uint8_t* xb, int lane, const flo
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    tma_reduce_add_2d(map, xb, x, y);
+    if (policy)
+      tma_reduce_add_2d_hint(map, xb, x, y, policy);
+    else
+      tma_reduce_add_2d(map, xb, x, y);
     bulk_commit_group();
   }
 }
@@ -317,11 +320,21 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
           phase ^= 1u;
         }
       };
+      // With a.l2_hints the C slices (streamed, shared only by the CTAs on the
+      // same vocabulary tile at about the same time) leave L2 first, so the
+      // dE rows the reductions keep returning to stay there.
+      const uint64_t pol_c = a.l2_hints ? l2_policy_evict_first() : 0ull;
+      auto load_c = [&](void* dst, const CUtensorMap* map, int x, int y) {
+        if (pol_c)
+          tma_load_2d_hint(dst, map, &full[stage], x, y, pol_c);
+        else
+          tma_load_2d(dst, map, &full[stage], x, y);
+      };
       auto load_s = [&](int m, int vt, int kb) {  // one recompute slice (stage already free)
         if (a.withhold_loads) return;
         mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
         tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m * BM);
-        tma_load_2d(sB + stage * B_STAGE_BYTES, &tmC, &full[stage], kb * BK, vt * BN);
+        load_c(sB + stage * B_STAGE_BYTES, &tmC, kb * BK, vt * BN);
         armed |= 1u << stage;
         if (a.pf && kb + a.pf < nkb) {  // L2 prefetch of the slices a.pf ahead
           tma_prefetch_l2_2d(&tmE, (kb + a.pf) * BK, m * BM);
@@ -388,17 +401,15 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
             uint8_t* b_st = sB + stage * B_STAGE_BYTES;
             tma_load_2d(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb0 * BK, m * BM);
             if (cpack == 2) {
-              tma_load_2d(b_st, &tmCq, &full[stage], kb0 * BK, vt * BN + q1 * 64);
+              load_c(b_st, &tmCq, kb0 * BK, vt * BN + q1 * 64);
               if (ns == 2) {
                 tma_load_2d(b_st + QUARTER_BYTES, &tmE, &full[stage], (kb0 - 1) * BK, m * BM);
-                tma_load_2d(b_st + QUARTER_BYTES + A_STAGE_BYTES, &tmCq, &full[stage], (kb0 - 1) * BK,
-                            vt * BN + q1 * 64);
+                load_c(b_st + QUARTER_BYTES + A_STAGE_BYTES, &tmCq, (kb0 - 1) * BK, vt * BN + q1 * 64);
               }
             } else {
 #pragma unroll
               for (int q = 0; q < 4; ++q)
-                if ((qmask >> q) & 1)
-                  tma_load_2d(b_st + q * QUARTER_BYTES, &tmCq, &full[stage], kb0 * BK, vt * BN + q * 64);
+                if ((qmask >> q) & 1) load_c(b_st + q * QUARTER_BYTES, &tmCq, kb0 * BK, vt * BN + q * 64);
             }
             armed |= 1u << stage;
             for (int sl = 0; a.pf && sl < ns; ++sl) {  // L2 prefetch of the contraction slices a.pf further on
@@ -583,6 +594,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
       return p;
     };
     const bool fixed = a.accE != nullptr;
+    const uint64_t pol_de = a.l2_hints ? l2_policy_evict_last() : 0ull;
     float fx_scale = 0.f;
     if (fixed)
       fx_scale = ldexpf(1.f, fixed_point_exponent(__uint_as_float(a.hdr[HDR_CMAX]), __uint_as_float(a.hdr[HDR_EMAX]),
@@ -724,7 +736,7 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
                   lsu_red_block32(next_xb(), lane, v, a.dE + (size_t)row0 * a.D + d0 + q * 32, (size_t)a.D,
                                   min(32, a.N - row0), min(32, a.D - (d0 + q * 32)));
                 else
-                  tma_red_block32<NXB>(next_xb(), lane, v, &tmdE, d0 + q * 32, row0);
+                  tma_red_block32<NXB>(next_xb(), lane, v, &tmdE, d0 + q * 32, row0, pol_de);
               }
             }
           }

@@ -121,6 +121,7 @@ struct BwdArgs {
   int withhold_loads;   // test hook: the TMA producer issues nothing
   int pf;               // L2 prefetch distance of the operand streams in K slices (0: off)
   int red_pf;           // L2 prefetch distance, in K slices, of the dE/dC rows the reductions add into (0: off)
+  int l2_hints;         // 1: C slices loaded evict-first, dE reduce-adds evict-last (keeps dE in L2)
   // profiling hook: per CTA and tile, globaltimer stamps (ns) at the start of
   // the tile, when its logits are in TMEM and when its gradient tile and
   // live mask are published; [grid][trace_cap][4] u64, null when off

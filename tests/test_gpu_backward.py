@@ -308,3 +308,19 @@ def test_reduce_prefetch_keeps_the_results(slices):
     fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=TILE)
     assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
+
+
+@pytest.mark.parametrize("eps", [0.0, EPS], ids=["filter-off", "filter-on"])
+def test_l2_hints_keep_the_results(eps):
+    # eviction priorities are hints: the fused kernel's gradients are unchanged
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=800, V=12000)
+    L.cce_debug_set_l2_hints(True)
+    try:
+        inp, dloss, olse, gE, gC, st = _run(w, eps, stripes=False)
+    finally:
+        L.cce_debug_set_l2_hints(False)
+    assert st["status"] == 0
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=TILE)
+    assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
