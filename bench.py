@@ -35,7 +35,8 @@ METRIC = "CCE fwd+bwd tokens/s"
 UNIT = "tokens/s"
 IGN = -100
 BM, BN = 128, 256      # logit tile (token block x vocabulary tile)
-FU = (32, 32)          # the gradient filter's unit: 32 tokens x 32 vocabulary entries
+FU = (32, 32)          # the unit of skipped work: 32 tokens x 32 vocabulary entries (the filter itself
+                       # drops single entries)
 
 
 def log(*a):
@@ -237,8 +238,8 @@ def blas_threads():
 
 def oracle_step(inp, rows, eps, C64=None):
     """The oracle's forward + backward for the token rows `rows` (a whole
-    number of 32-row filter units): loss/lse for those rows, then their full
-    contribution to dE and dC (unit filter applied).  C64: the classifier
+    number of 32-row units): loss/lse for those rows, then their full
+    contribution to dE and dC (entry filter applied).  C64: the classifier
     already decoded to fp64 (resident input), else decoded here."""
     import oracle
     E64 = oracle.bf16_bits_to_f64(inp["E"][rows])
@@ -247,7 +248,7 @@ def oracle_step(inp, rows, eps, C64=None):
     y = inp["y"][rows]
     loss, lse = oracle.forward_f64(E64, C64, y, IGN)
     dl = np.full(len(rows), 1.0 / max(1, len(rows)))
-    dE, dC = oracle.backward_f64(E64, C64, y, lse, dl, IGN, filter_eps=eps, tile=FU)
+    dE, dC = oracle.backward_f64(E64, C64, y, lse, dl, IGN, filter_eps=eps, tile=(1, 1))
     return loss
 
 
@@ -398,6 +399,7 @@ def run_gpu(args, w):
     if stf["status"] != 0 or stb["status"] != 0:
         raise RuntimeError(f"device status not clean: fwd {stf} bwd {stb}")
     live, dead, pruned = stb["live_tiles"], stb["dead_tiles"], stb["pruned_tiles"]
+    flat = stb["flat_units"]            # live units formed by the flat-row kernel (no tensor-core work)
     recomputed = stb["logit_tiles"]     # 128 x 256 logit tiles the backward recomputed
 
     # extra global memory of one step: the library allocates nothing itself
@@ -543,8 +545,9 @@ def run_gpu(args, w):
     peaks, peak_src = measured_peaks()
     unit_flop = 2.0 * FU[0] * FU[1] * D    # one filter unit's products, per contraction
     flop_fwd = 2.0 * N * D * V
-    # recompute of the visited logit tiles + the dE and dC products of the live units
-    flop_bwd = recomputed * 2.0 * BM * BN * D + live * 2.0 * unit_flop
+    # recompute of the visited logit tiles + the dE and dC products of the live
+    # units the tile kernel contracted (the flat-row kernel's are not tensor work)
+    flop_bwd = recomputed * 2.0 * BM * BN * D + (live - flat) * 2.0 * unit_flop
     fwd_name = "fwd_lse_pair_kernel" if args.fwd_variant == "pair" else "fwd_lse_kernel"
     dominant = "bwd_kernel" if bwd_ms >= fwd_ms else fwd_name
     dom_flop, dom_ms = (flop_bwd, bwd_ms) if dominant == "bwd_kernel" else (flop_fwd, fwd_ms)
@@ -591,6 +594,7 @@ def run_gpu(args, w):
                         "bwd_kernel": {"ms": bwd_ms, "tflops": flop_bwd / bwd_ms / 1e9,
                                        "frac_of_burst_peak": flop_bwd / bwd_ms / 1e9 / peak,
                                        "live_units": live, "dead_units": dead, "pruned_units": pruned,
+                                       "flat_units": flat,
                                        "logit_tiles_recomputed": recomputed},
                         "bwd_dense": dense},
             # flops the tensor cores executed in a step (forward, recomputed
@@ -927,14 +931,15 @@ def run_suite(args):
             tf += ev[0].elapsed_time(ev[1]) / reps
             tb += ev[1].elapsed_time(ev[2]) / reps
         unit = 2.0 * FU[0] * FU[1] * D
-        executed = 2.0 * N * D * V + st["logit_tiles"] * 2.0 * BM * BN * D + st["live_tiles"] * 2.0 * unit
+        executed = (2.0 * N * D * V + st["logit_tiles"] * 2.0 * BM * BN * D +
+                    (st["live_tiles"] - st["flat_units"]) * 2.0 * unit)
         print(json.dumps({
             "workload": w.name, "N": N, "D": D, "V": V, "filter_eps": w.filter_eps,
             "fwd_ms": tf, "fwd_tokens_per_s": N / tf * 1e3, "fwd_frac_of_peak": 2.0 * N * D * V / tf / 1e9 / peak,
             "fwd_bwd_ms": tf + tb, "fwd_bwd_tokens_per_s": N / (tf + tb) * 1e3,
             "executed_frac_of_peak": executed / (tf + tb) / 1e9 / peak,
             "bwd_ms": tb, "bwd_executed_frac_of_peak": (executed - 2.0 * N * D * V) / tb / 1e9 / peak,
-            "tiles": {k: st[k] for k in ("live_tiles", "dead_tiles", "pruned_tiles", "logit_tiles")},
+            "tiles": {k: st[k] for k in ("live_tiles", "dead_tiles", "pruned_tiles", "logit_tiles", "flat_units")},
             "extra_hbm_bytes": {"forward_workspace": wsf.buf.numel(), "backward_workspace": wsb.buf.numel()},
             "materialised_logits_fp32_bytes": N * V * 4, "peak_tflops": peak}), flush=True)
         del E, C, y, dl, dE, dC, loss, lse, wsf, wsb

@@ -9,10 +9,9 @@
  *   gradients of sum_i dloss[i] * loss[i]:
  *     G[i,v] = dloss[i] * (softmax(E_i C^T)[v] - [v == y_i]),
  *     dE = G C,  dC = G^T E,
- *   where the 32x32 gradient units (32 tokens x 32 vocabulary entries) whose
- *   every |softmax - onehot| entry is below filter_eps are skipped (the
- *   abstract's sentence 9: gradient terms too small to matter at the
- *   working precision are left out).
+ *   where every entry of G whose |softmax - onehot| is below filter_eps is
+ *   left out (the abstract's sentence 9: gradient elements too small to
+ *   matter at the working precision are skipped).
  *
  * Conventions for every entry point:
  *   - All matrix arguments are DEVICE pointers to row-major, contiguous data.
@@ -62,13 +61,19 @@ typedef enum {
 /* Status block decoded by cce_read_status. */
 typedef struct {
   uint64_t flags;       /* bit 0: a wait timed out; bit 1: an invalid label was seen */
-  uint64_t live_tiles;  /* backward: 32x32 filter units whose contributions were added */
-  uint64_t dead_tiles;  /* backward: filter units recomputed and found negligible */
+  uint64_t live_tiles;  /* backward: 32x32 units (tokens x vocabulary rows) holding at
+                           least one gradient entry that was added */
+  uint64_t dead_tiles;  /* backward: units recomputed and found to hold no entry
+                           at or above the filter threshold */
   uint64_t logit_tiles; /* forward: 128x256 logit tiles computed on chip;
                            backward: 128x256 logit tiles recomputed on chip */
-  uint64_t pruned_tiles;/* backward: filter units proven negligible without
-                           recomputing them; live + dead + pruned =
-                           ceil(N/32) * ceil(V/32) when filter_eps > 0 */
+  uint64_t pruned_tiles;/* backward: units proven negligible without recomputing
+                           them; live + dead + pruned = ceil(N/32) * ceil(V/32)
+                           when filter_eps > 0 */
+  uint64_t flat_units;  /* backward: the live units that lie in flat token blocks
+                           and were formed one correct-token entry at a time,
+                           without recomputing a logit tile (included in
+                           live_tiles).  Added in version 102. */
 } cce_counters_t;
 
 /* Workspace bytes needed by cce_forward for these sizes on the current device
@@ -101,18 +106,19 @@ CCE_API cce_status_t cce_forward(const void* E, const void* C, const int64_t* y,
 /* Backward pass (abstract, sentences 4 and 9): gradients of sum_i dloss[i] * loss[i].
  *   lse   [N] fp32   from cce_forward on the same E, C
  *   dloss [N] fp32   upstream gradient per token (e.g. 1/#kept for a mean)
- *   filter_eps       a 32x32 unit (32 tokens x 32 vocabulary entries,
- *                    anchored at 0) of (softmax - onehot) whose entries are
- *                    all below filter_eps in magnitude is skipped; <= 0 keeps
- *                    every unit (exact gradient)
+ *   filter_eps       an entry of (softmax - onehot) below filter_eps in
+ *                    magnitude is left out of G; <= 0 keeps every entry
+ *                    (exact gradient)
  *   dE    [N x D] fp32 out (overwritten), dC [V x D] fp32 out (overwritten)
  * The logit tiles are recomputed on chip; rows with y == ignore_index
  * contribute nothing.  With filter_eps > 0 a pre-pass bounds every logit by
- * |E_i| max_v |C_v| (Cauchy-Schwarz): units that bound proves negligible and
- * that hold no label are not recomputed (counted as pruned); the result is
- * the same as recomputing and testing them.  Accumulation order across tiles
- * is not fixed (fp32 atomics), so results may differ in the last bits between
- * runs. */
+ * |E_i| max_v |C_v| (Cauchy-Schwarz).  In a 128-token block where that bound
+ * puts every softmax probability below filter_eps, only the correct-token
+ * entries can survive: they are formed one token at a time (one dot product
+ * each) and no logit tile of the block is recomputed.  Other blocks are
+ * recomputed tile by tile and tested entry by entry.  The result is the same
+ * as testing every entry.  Accumulation order across tiles is not fixed
+ * (fp32 atomics), so results may differ in the last bits between runs. */
 CCE_API cce_status_t cce_backward(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
                           int64_t N, int64_t D, int64_t V, int64_t ignore_index, float filter_eps, float* dE,
                           float* dC, void* workspace, size_t workspace_bytes, void* stream);
@@ -178,7 +184,7 @@ typedef enum {
    * skips its own pass over C and uses the stored max_v |C_v|.  Same result
    * as without the flag.  No extra workspace. */
   CCE_BWD_PREPARED = 8,
-  /* With filter_eps <= 0 (every unit kept: the exact gradient), run the
+  /* With filter_eps <= 0 (every entry kept: the exact gradient), run the
    * dense backward through stripes of the softmax gradient: the vocabulary
    * is taken 2048 rows at a time; per stripe the logit tiles are recomputed
    * on chip and G = dloss (softmax - onehot) is stored in bf16 into one of

@@ -182,7 +182,7 @@ def read_status(workspace: Workspace, stream=None, raise_on_flag: bool = False) 
     if raise_on_flag and st != 0:
         raise CCEError(st, cce_status_string(st))
     return {"status": st, "flags": c[0], "live_tiles": c[1], "dead_tiles": c[2], "logit_tiles": c[3],
-            "pruned_tiles": c[4]}
+            "pruned_tiles": c[4], "flat_units": c[5]}
 
 
 def linear_cross_entropy(E, C, y, ignore_index: int = IGNORE_INDEX, filter_eps: float = 2.0 ** -12):

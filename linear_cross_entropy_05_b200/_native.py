@@ -20,7 +20,7 @@ c_f32 = ctypes.c_float
 class CCECounters(ctypes.Structure):
     _fields_ = [("flags", ctypes.c_uint64), ("live_tiles", ctypes.c_uint64),
                 ("dead_tiles", ctypes.c_uint64), ("logit_tiles", ctypes.c_uint64),
-                ("pruned_tiles", ctypes.c_uint64)]
+                ("pruned_tiles", ctypes.c_uint64), ("flat_units", ctypes.c_uint64)]
 
 
 class CCEError(RuntimeError):
@@ -211,7 +211,7 @@ def cce_backward_shard(E: int, C_shard: int, y: int, lse: int, dloss: int, N: in
 def cce_read_status(workspace: int, stream: int):
     c = CCECounters()
     st = load_library().cce_read_status(workspace, stream, ctypes.byref(c))
-    return st, (c.flags, c.live_tiles, c.dead_tiles, c.logit_tiles, c.pruned_tiles)
+    return st, (c.flags, c.live_tiles, c.dead_tiles, c.logit_tiles, c.pruned_tiles, c.flat_units)
 
 
 def cce_debug_forward_logits(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: int, loss: int,

@@ -37,6 +37,8 @@ cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t
                                 cudaStream_t stream);
 cudaError_t launch_clear_visited_rows(unsigned long long* acc, int V, int D, const unsigned* count,
                                       const unsigned* hdr, int sms, cudaStream_t stream);
+cudaError_t launch_flat_rows(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
+                             const FlatArgs& f, cudaStream_t stream);
 }  // namespace cce
 
 using namespace cce;
@@ -650,6 +652,26 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     if (fixed && filter_on &&
         launch_clear_visited_rows(accC, (int)V, (int)D, pp.count, pp.hdr, di.sms, stream) != cudaSuccess)
       return CCE_ERR_CUDA;
+    if (filter_on) {
+      // the label entries of the flat blocks (their other entries are all below eps)
+      FlatArgs fa;
+      fa.N = (int)N;
+      fa.D = (int)D;
+      fa.V = (int)V;
+      fa.ignore_index = ignore_index;
+      fa.shard_mode = shard ? 1 : 0;
+      fa.v_offset = v_offset;
+      fa.filter_eps = filter_eps;
+      fa.accumulate = accumulate ? 1 : 0;
+      fa.blk_flat = pp.blk_flat;
+      fa.hdr = pp.hdr;
+      fa.dE = reinterpret_cast<float*>(dE);
+      fa.dC = reinterpret_cast<float*>(dC);
+      fa.accE = accE;
+      fa.accC = accC;
+      fa.status = status;
+      if (launch_flat_rows(E, C, y, lse, dloss, fa, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    }
   }
   if ((flags & CCE_BWD_STRIPES) && !filter_on && !fixed)
     return backward_stripes(E, C, dE, dC, bp, a, accumulate, (flags & CCE_BWD_DETERMINISTIC) != 0, di.sms, ws,
@@ -748,13 +770,14 @@ cce_status_t cce_read_status(const void* workspace, void* stream, cce_counters_t
   if (!workspace || !out) return CCE_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return CCE_ERR_CUDA;
-  unsigned long long h[5];
+  unsigned long long h[8];
   if (cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return CCE_ERR_CUDA;
   out->flags = h[ST_FLAGS];
   out->live_tiles = h[ST_LIVE_TILES];
   out->dead_tiles = h[ST_DEAD_TILES];
   out->logit_tiles = h[ST_TILES];
   out->pruned_tiles = h[ST_PRUNED];
+  out->flat_units = h[ST_FLAT];
   if (h[ST_FLAGS] & SF_TIMEOUT) return CCE_ERR_TIMEOUT;
   if (h[ST_FLAGS] & SF_BAD_LABEL) return CCE_ERR_BAD_LABEL;
   return CCE_OK;
@@ -774,6 +797,6 @@ const char* cce_status_string(cce_status_t s) {
   return "CCE_ERR_UNKNOWN";
 }
 
-int cce_version(void) { return 101; }
+int cce_version(void) { return 102; }
 
 }  // extern "C"

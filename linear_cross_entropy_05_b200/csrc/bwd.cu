@@ -4,12 +4,12 @@
 // Cut Cross-Entropy abstract, sentences 4 and 9: the logits are never stored,
 // so the backward pass recomputes each 128 x 256 logit tile S = E_m C_v^T in
 // TMEM and forms P = exp(S - lse) and D = P - onehot(y) in registers.  The
-// filter works on 32 x 32 units (32 tokens x 32 vocabulary entries, 32 per
-// logit tile: one epilogue warp's rows x one 32-column chunk): a unit whose
-// every |D| is below filter_eps is dropped (gradient terms too small to
-// matter at the working precision) by writing its part of G = dloss * D to
-// shared memory as zeros.
-// The tensor cores then contract whole blocks that hold a live unit:
+// filter drops every entry with |D| below filter_eps (gradient elements too
+// small to matter at the working precision) by writing it to the shared
+// memory tile of G = dloss * D as zero.  The skipping of work is coarser:
+// 32 x 32 units (one epilogue warp's 32 rows x one 32-column chunk, 32 per
+// logit tile) left with no entry are "dead", and
+// the tensor cores contract only whole blocks that hold a live unit:
 //     dE[m-block, d-chunk] += sum over live 64-column quarters q of G_q . C_q[d-chunk]   (M=128, N=64, K=64 each)
 //     dC[v-half h, d-chunk] += G_h^T . E[m-block, d-chunk]  for halves with a live unit  (M=128, N=64, K=128)
 // and only the 32-row pieces of dE and dC that a live unit touches are added
@@ -658,8 +658,11 @@ __global__ void __launch_bounds__(64 + 128 * EPG, 1)
             float p = ex2_approx(fmaf(x[j + q], LOG2E, -lse2));
             float d = (col == ycol) ? p - 1.f : p;
             d = (valid && col < ncols) ? d : 0.f;
-            big |= fabsf(d) >= eps;
-            g2[q] = dl * d;
+            // entries below the threshold are dropped one by one (with the
+            // filter off eps <= 0 keeps every entry)
+            const bool keep = fabsf(d) >= eps;
+            big |= keep;
+            g2[q] = keep ? dl * d : 0.f;
           }
           pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
         }

@@ -1,28 +1,30 @@
 // Backward pre-pass: the list of logit tiles the backward must recompute.
 //
-// The gradient filter (Cut Cross-Entropy abstract, sentence 9) drops a
-// 32 x 32 unit when every |P - onehot| < eps.  For a token i and a column v
-// that is not its label, P_iv = exp(E_i.C_v - lse_i) and, by Cauchy-Schwarz,
-// E_i.C_v <= |E_i| |C_v|.  So if |E_i| * max_v |C_v| < lse_i + ln(eps) for every
-// kept token of a 128-token block, every unit of that block that holds none
-// of its labels is dead, and its logits need not be recomputed at all.  Such
-// a block is "flat"; only the 128 x 256 logit tiles holding its labels are
-// visited (and their units still tested exactly).  Blocks that are not
-// flat are visited densely.  The visited set therefore covers every live
-// unit, and the gradients equal those of the dense recompute with the same
-// filter.
+// The gradient filter (Cut Cross-Entropy abstract, sentence 9) drops every
+// entry of the softmax gradient with |P - onehot| < eps.  For a token i and a
+// column v that is not its label, P_iv = exp(E_i.C_v - lse_i) and, by
+// Cauchy-Schwarz, E_i.C_v <= |E_i| |C_v|.  So if |E_i| * max_v |C_v| <
+// lse_i + ln(eps) for every kept token of a 128-token block, every entry of
+// that block's rows except the label entries is dropped, and no logit of the
+// block needs to be recomputed: the label entry P_iy - 1 needs only the
+// correct-token logit E_i . C_y and lse_i.  Such a block is "flat"; its
+// tokens go to the flat-row kernel.  Blocks that are not flat are visited
+// densely by the tile kernel, which tests every entry.  The result equals
+// that of the dense recompute with the same filter.
 //
 // Kernels (stream order):
 //   prep_cnorm    max_v |C_v| (fp32, atomicMax on the float's bits)
 //   prep_enorm    |E_i| per token (and the maximum)
 //   prep_blocks   per token block: flatness, label-tile counts
-//   prep_scan     exclusive scan of the per-vocabulary-tile counts; totals
-//   prep_scatter  label tiles of flat blocks, ordered by vocabulary tile so
-//                 concurrent CTAs share C tiles in L2
+//   prep_scan     totals: the tiles to visit (every tile of each block that
+//                 is not flat)
+//   flat_rows     the label entries of the flat blocks' tokens, formed
+//                 directly (no logit tile is recomputed for a flat block)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace cce {
 
@@ -59,9 +61,6 @@ __device__ __forceinline__ bool label_ok(long long t, long long ignore_index, in
 // at the number of all units and loses those of every recomputed tile.
 __device__ __forceinline__ unsigned long long unit_rows(const PrepArgs& p, int m) {
   return (unsigned long long)min(BM / 32, (p.N - m * BM + 31) / 32);
-}
-__device__ __forceinline__ unsigned long long unit_cols(const PrepArgs& p, int v) {
-  return (unsigned long long)min(BN / 32, (p.V - v * BN + 31) / 32);
 }
 __device__ __forceinline__ void pruned_sub(const PrepArgs& p, unsigned long long units) {
   atomicAdd(p.status + ST_PRUNED, 0ull - units);  // modulo 2^64: order of the updates is free
@@ -174,10 +173,12 @@ __global__ void __launch_bounds__(1024) prep_scan_kernel(PrepArgs p) {
     __syncthreads();
   }
   if (t == 0) {
-    const unsigned L = carry_s;
+    // The label tiles of flat blocks are not visited: their only entries
+    // above the threshold are the label entries, which the flat-row kernel
+    // forms directly.  The list holds the non-flat blocks only.
     const unsigned nnf = p.hdr[HDR_NNF];
-    const unsigned long long T = (unsigned long long)L + (unsigned long long)nnf * (unsigned long long)p.n_vtile;
-    p.hdr[HDR_L] = L;
+    const unsigned long long T = (unsigned long long)nnf * (unsigned long long)p.n_vtile;
+    p.hdr[HDR_L] = 0u;
     p.hdr[HDR_T] = (unsigned)T;
     // all filter units; the recomputed tiles' units are taken off by
     // prep_blocks (dense blocks) and prep_scatter (listed tiles)
@@ -186,26 +187,116 @@ __global__ void __launch_bounds__(1024) prep_scan_kernel(PrepArgs p) {
   }
 }
 
-// One CTA (128 threads) per token block: place the flat block's label tiles.
-__global__ void __launch_bounds__(128) prep_scatter_kernel(const int64_t* __restrict__ y, PrepArgs p) {
-  __shared__ int tl[BM];
-  const int m = blockIdx.x;
-  if (!p.blk_flat[m]) return;
-  const int t = threadIdx.x;
-  const int row = m * BM + t;
-  const long long yl = row < p.N ? y[row] : p.ignore_index;
-  const long long ylocal = yl - (p.shard_mode ? p.v_offset : 0);
-  const bool has_col = row < p.N && yl != p.ignore_index && ylocal >= 0 && ylocal < p.V;
-  tl[t] = has_col ? (int)(ylocal / BN) : -1;
-  __syncthreads();
-  bool owner = has_col;
-  for (int j = 0; j < t && owner; ++j) owner = tl[j] != tl[t];
-  if (owner) {
-    const int v = tl[t];
-    const unsigned slot = atomicAdd(p.cursor + v, 1u);
-    p.list[p.offset[v] + slot] = make_int2(m, v);
-    pruned_sub(p, unit_rows(p, m) * unit_cols(p, v));
+// Flat token blocks: one CTA (32 warps) per 32-token row group, one warp per
+// token.  A kept token whose label column lies in this C has
+//   z = E_i . C_y,  p = exp(z - lse_i),  d = p - 1,
+// its only entry with |d| >= filter_eps (the pre-pass proved all others
+// below it); if |d| >= eps, G = dloss_i d adds G C_y to dE_i (the warp owns
+// the row) and G E_i to dC_y (atomically: tokens share labels).  The live
+// 32 x 32 units of the row group are its distinct live label chunks; they
+// move from the pruned to the live count.
+__global__ void __launch_bounds__(1024) flat_rows_kernel(const __nv_bfloat16* __restrict__ E,
+                                                         const __nv_bfloat16* __restrict__ C,
+                                                         const int64_t* __restrict__ y,
+                                                         const float* __restrict__ lse,
+                                                         const float* __restrict__ dloss, FlatArgs f) {
+  __shared__ int chunk_of[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g0 = blockIdx.x * 32;              // first token of the row group
+  if (!f.blk_flat[g0 / BM]) return;            // whole CTA: a row group lies in one token block
+  const int row = g0 + warp;
+  int live_chunk = -1;
+  if (row < f.N) {
+    const long long yg = y[row];
+    const long long yl = yg - (f.shard_mode ? f.v_offset : 0);
+    if (yg != f.ignore_index && yl >= 0 && yl < f.V) {
+      const uint4* er = reinterpret_cast<const uint4*>(E + (size_t)row * f.D);
+      const uint4* cr = reinterpret_cast<const uint4*>(C + (size_t)yl * f.D);
+      const int nvec = f.D >> 3;
+      float z0 = 0.f, z1 = 0.f;
+      for (int i = lane; i < nvec; i += 32) {
+        const uint4 ev = __ldg(er + i), cv = __ldg(cr + i);
+        const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&ev);
+        const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&cv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 ef = __bfloat1622float2(e2[j]);
+          const float2 cf = __bfloat1622float2(c2[j]);
+          z0 = fmaf(ef.x, cf.x, z0);
+          z1 = fmaf(ef.y, cf.y, z1);
+        }
+      }
+      float z = z0 + z1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      const float d = expf(z - lse[row]) - 1.f;
+      if (fabsf(d) >= f.filter_eps) {
+        live_chunk = (int)(yl >> 5);
+        const float g = dloss[row] * d;
+        const bool fixed = f.accE != nullptr;
+        const float scale =
+            fixed ? ldexpf(1.f, fixed_point_exponent(__uint_as_float(f.hdr[HDR_CMAX]), __uint_as_float(f.hdr[HDR_EMAX]),
+                                                     __uint_as_float(f.hdr[HDR_DLMAX]), f.N))
+                  : 0.f;
+        for (int i = lane; i < nvec; i += 32) {
+          const uint4 ev = __ldg(er + i), cv = __ldg(cr + i);
+          const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&ev);
+          const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&cv);
+          float ce[8], ee[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 cf = __bfloat1622float2(c2[j]);
+            const float2 ef = __bfloat1622float2(e2[j]);
+            ce[2 * j] = g * cf.x;
+            ce[2 * j + 1] = g * cf.y;
+            ee[2 * j] = g * ef.x;
+            ee[2 * j + 1] = g * ef.y;
+          }
+          const size_t oe = (size_t)row * f.D + 8 * (size_t)i, oc = (size_t)yl * f.D + 8 * (size_t)i;
+          if (fixed) {
+            // this warp owns dE_i (the accumulator starts at zero); dC_y is shared
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              f.accE[oe + j] = (unsigned long long)__float2ll_rn(ce[j] * scale);
+              atomicAdd(f.accC + oc + j, (unsigned long long)__float2ll_rn(ee[j] * scale));
+            }
+          } else {
+            float4* de = reinterpret_cast<float4*>(f.dE + oe);
+            float4 a0 = make_float4(ce[0], ce[1], ce[2], ce[3]), a1 = make_float4(ce[4], ce[5], ce[6], ce[7]);
+            if (f.accumulate) {
+              const float4 o0 = de[0], o1 = de[1];
+              a0 = make_float4(o0.x + a0.x, o0.y + a0.y, o0.z + a0.z, o0.w + a0.w);
+              a1 = make_float4(o1.x + a1.x, o1.y + a1.y, o1.z + a1.z, o1.w + a1.w);
+            }
+            de[0] = a0;
+            de[1] = a1;
+            red_add_v4(f.dC + oc, ee[0], ee[1], ee[2], ee[3]);
+            red_add_v4(f.dC + oc + 4, ee[4], ee[5], ee[6], ee[7]);
+          }
+        }
+      }
+    }
   }
+  if (lane == 0) chunk_of[warp] = live_chunk;
+  __syncthreads();
+  if (warp == 0) {
+    const int c = chunk_of[lane];
+    const unsigned same = __match_any_sync(0xffffffffu, c);
+    const bool first = (__ffs(same) - 1) == lane;  // one lane per distinct chunk
+    const unsigned n = __popc(__ballot_sync(0xffffffffu, first && c >= 0));
+    if (lane == 0 && n) {
+      atomicAdd(f.status + ST_LIVE_TILES, (unsigned long long)n);
+      atomicAdd(f.status + ST_FLAT, (unsigned long long)n);
+      atomicAdd(f.status + ST_PRUNED, 0ull - (unsigned long long)n);
+    }
+  }
+}
+
+cudaError_t launch_flat_rows(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
+                             const FlatArgs& f, cudaStream_t stream) {
+  flat_rows_kernel<<<(f.N + 31) / 32, 1024, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E),
+                                                         reinterpret_cast<const __nv_bfloat16*>(C), y, lse, dloss, f);
+  return cudaGetLastError();
 }
 
 // Deterministic mode: max_i |dloss_i| for the fixed-point scale (max_i |E_i|
@@ -309,7 +400,6 @@ cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const fl
   // expects launch_cnorm and launch_enorm to have run
   prep_blocks_kernel<<<p.n_mblk, 128, 0, stream>>>(y, lse, p);
   prep_scan_kernel<<<1, 1024, 0, stream>>>(p);
-  prep_scatter_kernel<<<p.n_mblk, 128, 0, stream>>>(y, p);
   return cudaGetLastError();
 }
 

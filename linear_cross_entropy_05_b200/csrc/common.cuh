@@ -33,6 +33,7 @@ enum StatusWord : int {
   ST_TILES = 3,        // forward: 128x256 logit tiles computed; backward: logit tiles recomputed
   ST_PRUNED = 4,       // backward: filter units proven negligible without recomputing them
   ST_NEXT_TILE = 5,    // backward: next work item to hand out (CTAs take tiles as they free up)
+  ST_FLAT = 6,         // backward: live units of flat blocks, formed without recomputing a tile
 };
 // Header words of the backward pre-pass (u32, after the status block).
 enum PrepHeader : int {
@@ -91,6 +92,25 @@ struct PrepArgs {
   int* nonflat;           // [n_mblk] ids of blocks that are not flat
   int2* list;             // [<= N] (token block, vocabulary tile), vocabulary-major
   float* enorm;           // [N] |E_i|
+  unsigned long long* status;
+};
+
+// Flat token blocks (the pre-pass proved every non-label entry of their
+// softmax rows below filter_eps): the only entry left per kept token is its
+// label entry, handled without recomputing any logit tile.
+struct FlatArgs {
+  int N, D, V;
+  long long ignore_index;
+  int shard_mode;
+  long long v_offset;
+  float filter_eps;
+  int accumulate;              // dE rows are added to instead of written
+  const int* blk_flat;         // [n_mblk] from the pre-pass
+  const unsigned* hdr;         // pre-pass header (fixed-point scale)
+  float* dE;                   // fp32 [N][D] (unless accE)
+  float* dC;                   // fp32 [V][D] (unless accC)
+  unsigned long long* accE;    // fixed-point accumulators (deterministic mode) or null
+  unsigned long long* accC;
   unsigned long long* status;
 };
 

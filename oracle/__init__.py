@@ -18,11 +18,14 @@ plain definition):
     dE        = G @ C,    dC = G^T @ E
 
 The backward recomputation and the gradient filter follow the abstract's
-sentence 9 (skip gradient work whose contribution is below numerical
-precision).  The filter is read at tile granularity: a (Bn x Bv) tile of G,
-anchored at (0, 0) (32 x 32 unless stated), is dropped iff every entry has
-|P - onehot| < eps; ignored rows and out-of-range rows/columns count as zero.
-eps <= 0 disables it.
+sentence 9 (skip the elements of the gradient computation whose contribution
+is below numerical precision).  The filter is written for any tile of the
+gradient: a (Bn x Bv) tile of G, anchored at (0, 0), is dropped iff every
+entry has |P - onehot| < eps; ignored rows and out-of-range rows/columns
+count as zero; eps <= 0 disables it.  The default tile is (1, 1): every
+element is kept or dropped on its own, which is the reading the library
+computes.  Larger tiles (32 x 32 is one unit of the library's work
+skipping) give the unit liveness the library counts.
 
 Everything is float64 on the bf16-rounded inputs decoded exactly.  The only
 blocking is over token rows (to bound memory); each row block materialises its
@@ -159,7 +162,7 @@ def tile_live_map_f64(Dm_rows: np.ndarray, row0: int, Bn: int, Bv: int, eps: flo
 
 
 def backward_f64(E64, C64, y, lse, dloss, ignore_index: int, filter_eps: float = 0.0,
-                 tile=(32, 32), return_live: bool = False):
+                 tile=(1, 1), return_live: bool = False):
     """Full dE (N x D) and dC (V x D) in fp64 from the given per-token lse.
 
     With filter_eps > 0 the tiles of G that are not live (see module doc) are
@@ -190,7 +193,7 @@ def backward_f64(E64, C64, y, lse, dloss, ignore_index: int, filter_eps: float =
 
 
 def backward(E_bits, C_bits, y, lse, dloss, ignore_index: int, filter_eps: float = 0.0,
-             tile=(32, 32), return_live: bool = False):
+             tile=(1, 1), return_live: bool = False):
     """backward_f64 on bf16 bit-pattern inputs (lse from the oracle's forward)."""
     return backward_f64(bf16_bits_to_f64(E_bits), bf16_bits_to_f64(C_bits), y,
                         np.asarray(lse, dtype=np.float64), np.asarray(dloss), ignore_index,
@@ -199,7 +202,7 @@ def backward(E_bits, C_bits, y, lse, dloss, ignore_index: int, filter_eps: float
 
 def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
                      rows_dE: Sequence[int], rows_dC: Sequence[int],
-                     filter_eps: float = 0.0, tile=(32, 32)):
+                     filter_eps: float = 0.0, tile=(1, 1)):
     """Selected rows of dE and of dC without forming the full gradients.
 
     rows_dE: token rows i; dE[i] = sum_v G[i, v] C[v] needs only row i's lse.
@@ -222,15 +225,24 @@ def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
     # the token's tile block, so evaluate the whole block when filtering.
     out_dE = np.zeros((rows_dE.shape[0], E64.shape[1]), dtype=np.float64)
     if filter_eps > 0.0:
-        # one evaluation per token block holding requested rows
-        for b in sorted({int(i) // Bn for i in rows_dE}):
-            b0, b1 = b * Bn, min(N, (b + 1) * Bn)
-            z = logits(E64[b0:b1], C64)
-            _, Dm, G = softmax_grad_f64(z, lse_all[b0:b1], y[b0:b1], dloss[b0:b1], ignore_index)
-            live = tile_live_map_f64(Dm, b0, Bn, Bv, filter_eps)
-            mask = np.repeat(live[0], Bv)[:V]
-            for k in np.nonzero((rows_dE >= b0) & (rows_dE < b1))[0]:
-                out_dE[k] = np.where(mask, G[int(rows_dE[k]) - b0], 0.0) @ C64
+        # the token blocks holding requested rows, a few at a time (one matrix
+        # product per group); each block's tile mask is its own
+        blocks = sorted({int(i) // Bn for i in rows_dE})
+        per = max(1, 64 // Bn)
+        for g0 in range(0, len(blocks), per):
+            grp = blocks[g0:g0 + per]
+            spans = [(b * Bn, min(N, (b + 1) * Bn)) for b in grp]
+            rows_all = np.concatenate([np.arange(b0, b1) for b0, b1 in spans])
+            z = logits(E64[rows_all], C64)
+            _, Dm, G = softmax_grad_f64(z, lse_all[rows_all], y[rows_all], dloss[rows_all], ignore_index)
+            pos = 0
+            for b0, b1 in spans:
+                n = b1 - b0
+                live = tile_live_map_f64(Dm[pos:pos + n], b0, Bn, Bv, filter_eps)
+                mask = np.repeat(live[0], Bv)[:V]
+                for k in np.nonzero((rows_dE >= b0) & (rows_dE < b1))[0]:
+                    out_dE[k] = np.where(mask, G[pos + int(rows_dE[k]) - b0], 0.0) @ C64
+                pos += n
     else:
         # the requested rows, a few at a time (one matrix product per group)
         for k0 in range(0, rows_dE.shape[0], 64):
@@ -263,7 +275,9 @@ def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
                     hit = np.nonzero(cols == t)[0]
                     if hit.size:
                         Dm[k, hit[0]] -= 1.0
-            if filter_eps > 0.0:
+            if filter_eps > 0.0 and Bn == 1 and Bv == 1:
+                Dm = np.where(np.abs(Dm) >= filter_eps, Dm, 0.0)   # element by element
+            elif filter_eps > 0.0:
                 A = np.abs(Dm)
                 pos = 0
                 for t in tiles:
@@ -274,6 +288,7 @@ def backward_sampled(E_bits, C_bits, y, lse_all, dloss, ignore_index: int,
                         if not (blk >= filter_eps).any():
                             Dm[a0 - r0:a1 - r0, pos:pos + w] = 0.0
                     pos += w
+            if filter_eps > 0.0:
                 colpos = {int(c): j for j, c in enumerate(cols)}
                 take = np.array([colpos[int(v)] for v in rows_dC])
                 Dsel = Dm[:, take]

@@ -13,7 +13,8 @@ from _gpu_helpers import (GRAD_REL_FILTER_OFF, IGN, filter_on_bar, gpu_backward,
 pytestmark = pytest.mark.gpu
 
 EPS = synth.EPS_BF16_FILTER
-TILE = (32, 32)     # the filter's unit: 32 tokens x 32 vocabulary entries
+UNIT = (32, 32)     # the unit of skipped work the kernels count: 32 tokens x 32 vocabulary entries
+ELEM = (1, 1)       # the filter itself: every entry kept or dropped on its own
 
 CASES_OFF = [
     synth.TINY,
@@ -68,15 +69,15 @@ def test_backward_filter_off_matches_exact_gradient(w, stripes):
 def test_backward_filter_on(w):
     inp, dloss, olse, gE, gC, st = _run(w, EPS)
     assert st["status"] == 0 and st["flags"] == 0
-    fE, fC, live = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=TILE,
-                                   return_live=True)
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=ELEM)
+    live = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, EPS, UNIT)
     xE, xC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
-    # same tiles dropped as the oracle's tile filter (the decision sits at
-    # |P - onehot| = eps; fp32 vs fp64 may flip a tile exactly at the edge)
+    # same live units as the oracle's (the decision sits at |P - onehot| =
+    # eps; fp32 vs fp64 may flip a unit exactly at the edge)
     assert abs(st["live_tiles"] - int(live.sum())) <= max(1, live.size // 1000)
     assert st["live_tiles"] + st["dead_tiles"] + st["pruned_tiles"] == live.size
-    # tight against the unit-filtered oracle; the filter-on bar against the
-    # exact gradient
+    # tight against the element-filtered oracle; the filter-on bar against
+    # the exact gradient
     assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
     bar = filter_on_bar(w.V)
@@ -89,12 +90,15 @@ def test_filter_threshold_edges():
     # eps above 1 kills every tile
     w = synth.GEMMA2_2B.with_sizes(N=512, V=8192, D=256)
     inp, dloss, olse, gE, gC, st = _run(w, 0.5)
-    live_o = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, 0.5, TILE)
+    live_o = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, 0.5, UNIT)
     assert st["live_tiles"] == int(live_o.sum())
     yt = {(i // 32, int(inp["y"][i]) // 32) for i in range(w.N)}
     assert st["live_tiles"] == len(yt)
-    # every block is flat here: only the logit tiles holding labels are recomputed
-    assert st["logit_tiles"] == len({(i // 128, int(inp["y"][i]) // 256) for i in range(w.N)})
+    # every block is flat here: the label entries are formed directly and no
+    # logit tile is recomputed
+    assert st["logit_tiles"] == 0 and st["flat_units"] == st["live_tiles"]
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=0.5, tile=ELEM)
+    assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF and rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
     inp, dloss, olse, gE, gC, st = _run(w, 2.0)
     assert st["live_tiles"] == 0 and (gE == 0).all() and (gC == 0).all()
 
@@ -115,12 +119,15 @@ def test_non_flat_blocks_are_recomputed_densely():
     dE, dC, st = gpu_backward(Ed, Cd, yd, lse, dloss, EPS)
     assert st["status"] == 0
     _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
-    fE, fC, live = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=TILE,
-                                   return_live=True)
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=ELEM)
+    live = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, EPS, UNIT)
     nvu = -(-w.V // 32)
     label_tiles = {(i // 32, int(inp["y"][i]) // 32) for i in range(w.N)}
     assert int(live.sum()) > len(label_tiles)            # the peaky blocks have live non-label tiles
     assert st["live_tiles"] + st["dead_tiles"] >= 2 * 4 * nvu  # blocks 1 and 2 visited in full
+    # the other blocks are flat: their label units come from the flat-row kernel
+    assert 0 < st["flat_units"] < st["live_tiles"]
+    assert st["logit_tiles"] % -(-w.V // 256) == 0 and st["logit_tiles"] >= 2 * -(-w.V // 256)
     assert abs(st["live_tiles"] - int(live.sum())) <= max(2, live.size // 1000)
     assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
@@ -201,7 +208,7 @@ def test_backward_kernel_variants_match_oracle(variant, eps):
     finally:
         L.cce_debug_set_backward_variant(0)
     assert st["status"] == 0
-    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=TILE)
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=ELEM)
     assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
 
@@ -223,7 +230,7 @@ def test_labels_at_vocabulary_edges(eps):
     dloss = synth.random_dloss(12, w.N)
     dE, dC, st = gpu_backward(E, C, yd, lse, dloss, eps)
     assert st["status"] == 0
-    fE, fC = oracle.backward(inp["E"], inp["C"], y, olse, dloss, IGN, filter_eps=eps, tile=TILE)
+    fE, fC = oracle.backward(inp["E"], inp["C"], y, olse, dloss, IGN, filter_eps=eps, tile=ELEM)
     assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
     # the label rows of dC carry the one-hot part
@@ -239,6 +246,9 @@ def test_trace_hook_and_run_time_tile_dealing():
     import linear_cross_entropy_05_b200 as L
     w = synth.GEMMA2_2B.with_sizes(N=1000, V=20000)
     inp = synth.make_inputs(w)
+    E64 = oracle.bf16_bits_to_f64(inp["E"])
+    E64[256:384] *= 120.0        # a peaky block, which the pre-pass cannot clear: its tiles are recomputed
+    inp["E"] = synth.round_to_bf16_bits(E64.astype(np.float32))
     E, C, y = to_dev(inp)
     loss, lse, st = gpu_forward(E, C, y)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
@@ -260,7 +270,9 @@ def test_trace_hook_and_run_time_tile_dealing():
             k += 1
         tiles += k
     assert tiles == st["logit_tiles"] > 0
-    assert live == st["live_tiles"]
+    # the traced masks hold the units the tile kernel formed; the flat-row
+    # kernel forms the rest
+    assert live + st["flat_units"] == st["live_tiles"]
 
 
 @pytest.mark.parametrize("side", [-1, 1], ids=["eps-just-below-P", "eps-just-above-P"])
@@ -286,8 +298,8 @@ def test_filter_decision_at_the_threshold(side):
     dE, dC, st = gpu_backward(Ed, Cd, yd, lse, dloss, eps)
     assert st["status"] == 0
     _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
-    fE, fC, live = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=TILE,
-                                   return_live=True)
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=ELEM)
+    live = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, eps, UNIT)
     assert bool(live[0, 200 // 32]) == (side < 0)
     assert st["live_tiles"] == int(live.sum()) == 2 + (side < 0)   # two label units (+ the edge unit)
     assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
@@ -305,7 +317,7 @@ def test_reduce_prefetch_keeps_the_results(slices):
     finally:
         L.cce_debug_set_reduce_prefetch(0)
     assert st["status"] == 0
-    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=TILE)
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=ELEM)
     assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
 
@@ -321,6 +333,6 @@ def test_l2_hints_keep_the_results(eps):
     finally:
         L.cce_debug_set_l2_hints(False)
     assert st["status"] == 0
-    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=TILE)
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=ELEM)
     assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF

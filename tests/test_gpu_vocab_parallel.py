@@ -66,8 +66,12 @@ def test_sharded_backward_assembles_the_full_gradient(w, bounds, eps):
         assert rel_fro(dE.cpu().numpy(), oE) <= GRAD_REL_FILTER_OFF
         assert rel_fro(dC.cpu().numpy(), oC) <= GRAD_REL_FILTER_OFF
     else:
-        # each shard's filter grid starts at its own first row; against the
-        # exact gradient the filter-on bar applies
+        # the filter decides entry by entry, so the shards together drop
+        # exactly the entries the unsharded filter drops: tight against the
+        # element-filtered oracle, and the filter-on bar against the exact one
+        fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=(1, 1))
+        assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
+        assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
         xE, xC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN)
         assert rel_fro(dE.cpu().numpy(), xE) <= filter_on_bar(w.V)
         assert rel_fro(dC.cpu().numpy(), xC) <= filter_on_bar(w.V)

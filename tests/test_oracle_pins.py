@@ -241,9 +241,11 @@ def _brute_filtered(E, C, y, dloss, eps, Bn, Bv):
 
 
 @pytest.mark.parametrize("eps", [0.02, 0.1])
-def test_tile_filter_against_brute_force(eps):
+@pytest.mark.parametrize("tile", [(2, 4), (1, 1)], ids=["2x4-tiles", "elements"])
+def test_tile_filter_against_brute_force(eps, tile):
     rng = np.random.default_rng(8)
-    N, D, V, Bn, Bv = 7, 3, 11, 2, 4
+    N, D, V = 7, 3, 11
+    Bn, Bv = tile
     E = rng.standard_normal((N, D)) * 1.5
     C = rng.standard_normal((V, D)) * 1.5
     y = rng.integers(0, V, N)
@@ -317,6 +319,33 @@ def test_tile_live_map_pin_catches_planted_mistakes(monkeypatch, mutation):
     assert live.shape != live_b.shape or not (live == live_b).all(), f"{mutation} went unnoticed"
 
 
+def test_element_filter_defaults_and_keeps_only_large_entries():
+    # the default filter works element by element: the filtered G equals the
+    # exact G with every |P - onehot| < eps entry set to zero
+    rng = np.random.default_rng(13)
+    N, D, V = 6, 4, 9
+    E = rng.standard_normal((N, D))
+    C = rng.standard_normal((V, D))
+    y = rng.integers(0, V, N)
+    y[2] = IGN
+    dloss = rng.random(N) + 0.5
+    _, lse = oracle.forward_f64(E, C, y, IGN)
+    eps = 0.05
+    z = E @ C.T
+    P = np.exp(z - lse[:, None])
+    Dm = P.copy()
+    for i in range(N):
+        if y[i] == IGN:
+            Dm[i] = 0.0
+        else:
+            Dm[i, y[i]] -= 1.0
+    G = np.where(np.abs(Dm) >= eps, Dm, 0.0) * dloss[:, None]
+    assert 0 < (np.abs(Dm) >= eps).sum() < Dm.size - N   # the case really drops entries
+    dE, dC = oracle.backward_f64(E, C, y, lse, dloss, IGN, filter_eps=eps)
+    np.testing.assert_allclose(dE, G @ C, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(dC, G.T @ E, rtol=1e-12, atol=1e-15)
+
+
 def test_sampled_backward_matches_full():
     w = synth.TINY.with_sizes(N=300, V=1000, D=64)
     inp = synth.make_inputs(w)
@@ -326,7 +355,7 @@ def test_sampled_backward_matches_full():
     loss, lse = oracle.forward(E, C, y, IGN)
     loss_s, lse_s = oracle.forward(E, C, y, IGN, rows=[5, 299, 3])
     np.testing.assert_allclose(loss_s, loss[[5, 299, 3]], rtol=1e-14)
-    for eps, tile in ((0.0, (128, 256)), (2e-3, (128, 256)), (1e-3, (64, 128))):
+    for eps, tile in ((0.0, (128, 256)), (2e-3, (128, 256)), (1e-3, (64, 128)), (1e-3, (1, 1)), (3e-4, (1, 1))):
         dE, dC = oracle.backward(E, C, y, lse, dloss, IGN, filter_eps=eps, tile=tile)
         rE = [0, 129, 299, 3]
         rC = [0, 255, 256, 999, int(y[7])]
