@@ -174,10 +174,12 @@ class ClockSampler:
 
 def launches_per_step(eps: float, fixed_point: bool) -> int:
     """Kernels of this library launched by one forward + backward call pair:
-    forward logit/LSE kernel and finalize; backward kernel; the norm pass
-    (classifier and token norms) when the filter or the fixed-point mode
-    needs it; the candidate-tile pre-pass (blocks, scan, scatter) with the
-    filter on; the dloss maximum and two conversion passes in fixed point."""
+    forward logit/LSE kernel and finalize; backward tile kernel (or the
+    stripe kernel, one launch up to 16384 tokens); the norm pass (classifier
+    and token norms) when the filter or the fixed-point mode needs it; with
+    the filter on the pre-pass (blocks, scan) and the flat-row kernel; the
+    dloss maximum and two conversion passes in fixed point; and with both,
+    the clearing of the dC accumulator rows that can receive a gradient."""
     n = 2 + 1
     if eps > 0 or fixed_point:
         n += 2
@@ -185,6 +187,8 @@ def launches_per_step(eps: float, fixed_point: bool) -> int:
         n += 3
     if fixed_point:
         n += 3
+    if eps > 0 and fixed_point:
+        n += 1
     return n
 
 
@@ -398,6 +402,8 @@ def run_gpu(args, w):
     stb = L.read_status(ws_b)
     if stf["status"] != 0 or stb["status"] != 0:
         raise RuntimeError(f"device status not clean: fwd {stf} bwd {stb}")
+    # vocabulary splits of the forward (its workspace holds N (max, sum) pairs per split)
+    fwd_splits = (L.cce_forward_workspace_size(N, D, V) - 256) // (8 * N)
     live, dead, pruned = stb["live_tiles"], stb["dead_tiles"], stb["pruned_tiles"]
     flat = stb["flat_units"]            # live units formed by the flat-row kernel (no tensor-core work)
     recomputed = stb["logit_tiles"]     # 128 x 256 logit tiles the backward recomputed
@@ -582,7 +588,9 @@ def run_gpu(args, w):
                            classifier_norm=("cce_backward_prepare on the side stream during the forward"
                                             if prepare else "inside the backward call"),
                            l2_prefetch_slices=list(args.prefetch) if args.prefetch else [0, 0],
-                           reduce_prefetch_slices=args.reduce_prefetch, l2_hints=bool(args.l2_hints)),
+                           reduce_prefetch_slices=args.reduce_prefetch, l2_hints=bool(args.l2_hints),
+                           forward_splits=fwd_splits,
+                           forward_schedule=list(args.fwd_schedule) if args.fwd_schedule else None),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops (burst: the timed region is under a second)",
@@ -985,6 +993,10 @@ def main(argv=None):
                     help="L2 prefetch distance of the filtered backward's reduction targets (A/B; 0 = off)")
     ap.add_argument("--l2-hints", action="store_true",
                     help="L2 eviction priorities in the filtered backward (A/B)")
+    ap.add_argument("--fwd-schedule", type=int, nargs=3, default=None, metavar=("SPLITS", "GROUP_M", "L2_HINTS"),
+                    help="forward schedule (A/B): vocabulary splits per token block and token blocks per raster "
+                         "group (0 = chosen per shape), L2 hints of the pair kernel (bit 0: E evict_last, bit 1: C "
+                         "evict_first)")
     ap.add_argument("--trace", action="store_true",
                     help="per-tile timeline of one backward launch (recompute wait, gradient tile, contraction)")
     ap.add_argument("--dense-trace", action="store_true",
@@ -998,7 +1010,7 @@ def main(argv=None):
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
     if args.impl == "cce" and (args.fwd_variant != "pair" or args.bwd_variant or args.prefetch or
-                               args.reduce_prefetch is not None or args.l2_hints):
+                               args.reduce_prefetch is not None or args.l2_hints or args.fwd_schedule):
         import linear_cross_entropy_05_b200 as L
         L.cce_debug_set_forward_variant(1 if args.fwd_variant == "pair" else 0)
         L.cce_debug_set_backward_variant(args.bwd_variant)
@@ -1008,6 +1020,8 @@ def main(argv=None):
             L.cce_debug_set_reduce_prefetch(args.reduce_prefetch)
         if args.l2_hints:
             L.cce_debug_set_l2_hints(True)
+        if args.fwd_schedule:
+            L.cce_debug_set_forward_schedule(*args.fwd_schedule)
     if args.suite:
         return run_suite(args)
     if args.memory or args.trace:

@@ -83,9 +83,8 @@ typedef struct {
 CCE_API size_t cce_forward_workspace_size(int64_t N, int64_t D, int64_t V);
 
 /* Workspace bytes needed by cce_backward: the status block plus the
- * candidate-tile pre-pass (O(N + V/256): one (block, tile) pair per token at
- * most, a few words per 128-token block and per 256-row vocabulary tile).
- * Returns 0 if the sizes are invalid. */
+ * pre-pass (O(N + V/32): one norm per token, a few words per 128-token
+ * block, one bit per vocabulary row).  Returns 0 if the sizes are invalid. */
 CCE_API size_t cce_backward_workspace_size(int64_t N, int64_t D, int64_t V);
 
 /* Forward pass (abstract, sentences 4-6): per-token loss and log-sum-exp.

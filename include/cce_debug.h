@@ -45,6 +45,19 @@ CCE_API void cce_debug_withhold_loads(int on);
  * CCE_ERR_INVALID_ARG outside [0, 64]. */
 CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
 
+/* Schedule knobs of the forward logit/LSE kernels, for A/B measurement.
+ * n_split (0..64; 0 = chosen per shape: the fewest splits that minimise the
+ * most-loaded worker's vocabulary tiles) is the number of vocabulary ranges
+ * per token block, i.e. of (max, sum) partials per token; group_m (>= 0; 0 =
+ * chosen per shape, ~48 MB of E rows) is the number of token blocks per
+ * raster group; l2_hints (0..3, default 0; CTA-pair kernel only) gives the
+ * E slices the evict_last L2 policy (bit 0) and the C slices evict_first
+ * (bit 1).  Same loss and lse up to fp32 rounding order.  The forward
+ * workspace size depends on n_split: query cce_forward_workspace_size after
+ * changing it.  Process-wide.  Returns CCE_ERR_INVALID_ARG for other
+ * values. */
+CCE_API cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hints);
+
 /* Tuning knobs of the dense stripe backward (CCE_BWD_STRIPES), for A/B
  * measurement: tokens_per_launch (a multiple of 256, at most 16384; 0 = the
  * default 16384) bounds the tokens one launch takes (fewer tokens per launch

@@ -91,6 +91,8 @@ def load_library():
         lib.cce_debug_set_stripe_params.restype = ctypes.c_int
         lib.cce_debug_set_l2_hints.argtypes = [ctypes.c_int]
         lib.cce_debug_set_l2_hints.restype = ctypes.c_int
+        lib.cce_debug_set_forward_schedule.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.cce_debug_set_forward_schedule.restype = ctypes.c_int
         lib.cce_debug_set_reduce_prefetch.argtypes = [ctypes.c_int]
         lib.cce_debug_set_reduce_prefetch.restype = ctypes.c_int
         lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 5 + [c_vp, c_i64]
@@ -290,3 +292,11 @@ def cce_debug_set_l2_hints(on: bool) -> None:
     """L2 eviction priorities in the filtered backward (evict-first classifier
     slices, evict-last dE reductions); A/B knob, off by default."""
     _check(load_library().cce_debug_set_l2_hints(1 if on else 0), "cce_debug_set_l2_hints")
+
+
+def cce_debug_set_forward_schedule(n_split: int = 0, group_m: int = 0, l2_hints: int = 0) -> None:
+    """Forward schedule knobs (A/B): vocabulary splits per token block, token
+    blocks per raster group (0 = chosen per shape) and L2 eviction hints of
+    the CTA-pair kernel (bit 0: E evict_last, bit 1: C evict_first)."""
+    _check(load_library().cce_debug_set_forward_schedule(int(n_split), int(group_m), int(l2_hints)),
+           "cce_debug_set_forward_schedule")

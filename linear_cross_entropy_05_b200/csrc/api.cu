@@ -4,12 +4,15 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <array>
 #include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <vector>
 
 #include "../../include/cce.h"
 #include "../../include/cce_debug.h"
@@ -32,10 +35,10 @@ cudaError_t launch_cnorm(const void* C, const PrepArgs& p, int sms, cudaStream_t
 cudaError_t launch_enorm(const void* E, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cudaStream_t stream);
 cudaError_t launch_bwd_stripe(const CUtensorMap* maps, const StripeArgs& a, void* G, int grid, cudaStream_t stream);
-cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
-                                bool bf16, bool accumulate, const unsigned* count, int D, int sms,
+cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, int rows, int D, const unsigned* hdr,
+                                int N, bool bf16, bool accumulate, const unsigned* rowbits, int sms,
                                 cudaStream_t stream);
-cudaError_t launch_clear_visited_rows(unsigned long long* acc, int V, int D, const unsigned* count,
+cudaError_t launch_clear_visited_rows(unsigned long long* acc, int V, int D, const unsigned* rowbits,
                                       const unsigned* hdr, int sms, cudaStream_t stream);
 cudaError_t launch_flat_rows(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
                              const FlatArgs& f, cudaStream_t stream);
@@ -56,6 +59,9 @@ std::atomic<int> g_bwd_variant{0};
 // Test hook: when set, the next launches' TMA producers issue no copies.
 std::atomic<int> g_withhold_loads{0};
 std::atomic<int> g_fwd_pf{0};  // L2 prefetch distances (K slices) of the forward / backward operand streams
+std::atomic<int> g_fwd_split{0};     // forward vocabulary splits per token block (0: chosen per shape)
+std::atomic<int> g_fwd_group_m{0};   // forward token blocks per raster group (0: chosen per shape)
+std::atomic<int> g_fwd_l2_hints{0};  // forward CTA-pair kernel: L2 eviction priorities (A/B)
 std::atomic<int> g_bwd_pf{0};
 std::atomic<int> g_bwd_red_pf{0};  // L2 prefetch distance (K slices) of the backward's reduction targets
 std::atomic<int> g_bwd_l2_hints{0};  // L2 eviction priorities in the filtered backward (A/B)
@@ -119,20 +125,47 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // Vocabulary splits per 128-row token block.  Work units (block, split) are
 // dealt to the persistent CTAs round-robin; pick the split count that
 // minimises (units per CTA) x (tiles per unit).
-int choose_splits(int n_mblk, int n_vtile, int grid_max) {
+// Largest number of vocabulary tiles any worker gets when the n_mblk * s
+// work units are dealt round-robin (unit u to worker u % workers, as the
+// forward kernels take them) and unit_coords maps a unit to its split.
+long long max_worker_tiles(int n_mblk, int n_vtile, int s, int workers, int group_m) {
+  std::vector<long long> load((size_t)workers, 0);
+  const int units = n_mblk * s;
+  for (int u = 0; u < units; ++u) {
+    int r, m;
+    unit_coords(u, n_mblk, s, group_m, r, m);
+    int v0, v1;
+    split_range(r, n_vtile, s, v0, v1);
+    load[(size_t)(u % workers)] += v1 - v0;
+  }
+  return *std::max_element(load.begin(), load.end());
+}
+
+// Splits per token block: the fewest that minimise the most-loaded worker's
+// vocabulary tiles (the kernel's duration).  Memoised per shape: the search
+// is O(64 * n_mblk * 64).
+int choose_splits(int n_mblk, int n_vtile, int workers, int group_m) {
+  static std::mutex mu;
+  static std::map<std::array<int, 4>, int> memo;
+  const std::array<int, 4> key{n_mblk, n_vtile, workers, group_m};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = memo.find(key);
+    if (it != memo.end()) return it->second;
+  }
   long long best = LLONG_MAX;
   int best_s = 1;
   const int smax = std::min(64, n_vtile);
   for (int s = 1; s <= smax; ++s) {
-    const long long units = (long long)n_mblk * s;
-    const long long per_cta = (units + grid_max - 1) / grid_max;
-    const long long tiles = (n_vtile + s - 1) / s;
-    const long long cost = per_cta * tiles;
+    const long long cost = max_worker_tiles(n_mblk, n_vtile, s, workers, group_m);
     if (cost < best) {
       best = cost;
       best_s = s;
     }
   }
+  std::lock_guard<std::mutex> lk(mu);
+  if (memo.size() > 256) memo.clear();
+  memo[key] = best_s;
   return best_s;
 }
 
@@ -197,17 +230,19 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
   const int workers = p->pair ? di.sms / 2 : di.sms;  // CTA pairs or CTAs
   p->n_mblk = (int)((N + rows - 1) / rows);
   p->n_vtile = (int)((V + BN - 1) / BN);
-  p->n_split = choose_splits(p->n_mblk, p->n_vtile, workers);
-  const long long units = (long long)p->n_mblk * p->n_split;
-  p->grid = (int)std::min<long long>(units, workers) * (p->pair ? 2 : 1);
   // keep at most ~48 MB of E rows in flight so they stay resident in the 126 MB L2
   p->group_m = (int)std::max<int64_t>(1, std::min<int64_t>(p->n_mblk, (48ll << 20) / ((int64_t)rows * D * 2)));
+  if (g_fwd_group_m.load() > 0) p->group_m = std::min(p->n_mblk, g_fwd_group_m.load());
+  p->n_split = g_fwd_split.load() > 0 ? std::min(p->n_vtile, g_fwd_split.load())
+                                      : choose_splits(p->n_mblk, p->n_vtile, workers, p->group_m);
+  const long long units = (long long)p->n_mblk * p->n_split;
+  p->grid = (int)std::min<long long>(units, workers) * (p->pair ? 2 : 1);
   p->ws_bytes = STATUS_BYTES + align_up((size_t)p->n_split * (size_t)N * sizeof(float2), 256);
   return true;
 }
 
-// Backward workspace: status | pre-pass header | count, offset, cursor
-// [n_vtile] | blk_flat, nonflat [n_mblk] | list [N] int2.  O(N + V/256).
+// Backward workspace: status | pre-pass header | dC row bits [ceil(V/32)] |
+// blk_flat, nonflat [n_mblk] | |E_i| [N].  O(N + V/32).
 // Stripe backward (CCE_BWD_STRIPES, filter off): 256-token blocks per launch
 // (token super-block; dC gathers the super-blocks by reduce-adds) and
 // vocabulary tiles per stripe.
@@ -251,8 +286,7 @@ StripeLayout plan_stripes(int64_t N, int64_t D, int64_t V, size_t base) {
 
 struct BwdPlan {
   int n_mblk, n_vtile;
-  size_t off_hdr, off_count, off_offset, off_cursor, off_flat, off_nonflat, off_list, off_enorm, zero_bytes,
-      ws_bytes;
+  size_t off_hdr, off_rowbits, off_flat, off_nonflat, off_enorm, zero_bytes, ws_bytes;
   size_t off_accE, off_accC;  // fixed-point accumulators (deterministic mode only)
   StripeLayout stripes;       // CCE_BWD_STRIPES only
 };
@@ -273,17 +307,13 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
   p->n_mblk = (int)((N + BM - 1) / BM);
   p->n_vtile = (int)((V + BN - 1) / BN);
   if ((int64_t)p->n_mblk * p->n_vtile >= ((int64_t)1 << 31)) return false;
-  const size_t vt4 = align_up((size_t)p->n_vtile * 4, 256);
   const size_t mb4 = align_up((size_t)p->n_mblk * 4, 256);
   p->off_hdr = STATUS_BYTES;
-  p->off_count = p->off_hdr + HDR_BYTES;
-  p->off_offset = p->off_count + vt4;
-  p->off_cursor = p->off_offset + vt4;
-  p->zero_bytes = p->off_cursor + vt4;  // status, header, count, offset, cursor start at zero
+  p->off_rowbits = p->off_hdr + HDR_BYTES;
+  p->zero_bytes = p->off_rowbits + align_up((size_t)((V + 31) / 32) * 4, 256);  // status, header, row bits
   p->off_flat = p->zero_bytes;
   p->off_nonflat = p->off_flat + mb4;
-  p->off_list = p->off_nonflat + mb4;
-  p->off_enorm = p->off_list + align_up((size_t)N * sizeof(int2), 256);
+  p->off_enorm = p->off_nonflat + mb4;
   p->ws_bytes = p->off_enorm + align_up((size_t)N * sizeof(float), 256);
   p->off_accE = p->off_accC = 0;
   if ((flags & CCE_BWD_STRIPES) && (flags & CCE_BWD_BF16_GRADS)) return false;  // not combined
@@ -340,6 +370,7 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.withhold_loads = g_withhold_loads.load();
   a.pf = g_fwd_pf.load();
+  a.l2_hints = g_fwd_l2_hints.load();
   if (record_event(0, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   const cudaError_t le =
       p.pair ? launch_fwd_lse_pair(tmE, tmC, a, p.grid, stream) : launch_fwd_lse(tmE, tmC, a, p.grid, stream);
@@ -399,6 +430,14 @@ cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices) {
   if (fwd_slices < 0 || fwd_slices > 64 || bwd_slices < 0 || bwd_slices > 64) return CCE_ERR_INVALID_ARG;
   g_fwd_pf.store(fwd_slices);
   g_bwd_pf.store(bwd_slices);
+  return CCE_OK;
+}
+
+cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hints) {
+  if (n_split < 0 || n_split > 64 || group_m < 0 || l2_hints < 0 || l2_hints > 3) return CCE_ERR_INVALID_ARG;
+  g_fwd_split.store(n_split);
+  g_fwd_group_m.store(group_m);
+  g_fwd_l2_hints.store(l2_hints);
   return CCE_OK;
 }
 
@@ -605,7 +644,6 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.shard_mode = shard ? 1 : 0;
   a.v_offset = v_offset;
   a.hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);
-  a.list = reinterpret_cast<const int2*>(ws + bp.off_list);
   a.nonflat = reinterpret_cast<const int*>(ws + bp.off_nonflat);
   a.filter_eps = filter_eps;
   a.ignore_index = ignore_index;
@@ -637,12 +675,9 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     pp.v_offset = v_offset;
     pp.log_eps = logf(filter_eps);
     pp.hdr = reinterpret_cast<unsigned*>(ws + bp.off_hdr);
-    pp.count = reinterpret_cast<unsigned*>(ws + bp.off_count);
-    pp.offset = reinterpret_cast<unsigned*>(ws + bp.off_offset);
-    pp.cursor = reinterpret_cast<unsigned*>(ws + bp.off_cursor);
+    pp.rowbits = reinterpret_cast<unsigned*>(ws + bp.off_rowbits);
     pp.blk_flat = reinterpret_cast<int*>(ws + bp.off_flat);
     pp.nonflat = reinterpret_cast<int*>(ws + bp.off_nonflat);
-    pp.list = reinterpret_cast<int2*>(ws + bp.off_list);
     pp.enorm = reinterpret_cast<float*>(ws + bp.off_enorm);
     pp.status = status;
     if (!prepared && launch_cnorm(C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
@@ -650,7 +685,7 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     if (filter_on && launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (fixed && launch_fixed_prep(dloss, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (fixed && filter_on &&
-        launch_clear_visited_rows(accC, (int)V, (int)D, pp.count, pp.hdr, di.sms, stream) != cudaSuccess)
+        launch_clear_visited_rows(accC, (int)V, (int)D, pp.rowbits, pp.hdr, di.sms, stream) != cudaSuccess)
       return CCE_ERR_CUDA;
     if (filter_on) {
       // the label entries of the flat blocks (their other entries are all below eps)
@@ -682,10 +717,10 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   if (record_event(1, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (fixed) {
     const unsigned* hdr = reinterpret_cast<const unsigned*>(ws + bp.off_hdr);
-    const unsigned* count = filter_on ? reinterpret_cast<const unsigned*>(ws + bp.off_count) : nullptr;
-    if (launch_fixed_to_out(accE, dE, (size_t)N * D, hdr, (int)N, bf16_out, accumulate, nullptr, (int)D, di.sms,
+    const unsigned* rowbits = filter_on ? reinterpret_cast<const unsigned*>(ws + bp.off_rowbits) : nullptr;
+    if (launch_fixed_to_out(accE, dE, (int)N, (int)D, hdr, (int)N, bf16_out, accumulate, nullptr, di.sms,
                             stream) != cudaSuccess ||
-        launch_fixed_to_out(accC, dC, (size_t)V * D, hdr, (int)N, bf16_out, accumulate, count, (int)D, di.sms,
+        launch_fixed_to_out(accC, dC, (int)V, (int)D, hdr, (int)N, bf16_out, accumulate, rowbits, di.sms,
                             stream) != cudaSuccess)
       return CCE_ERR_CUDA;
   }

@@ -113,32 +113,25 @@ __device__ __forceinline__ void lsu_red_block32(uint8_t* xb, int lane, const flo
 }
 
 // Work item t -> (token block m, vocabulary tile vt).  Dense mode rasters the
-// whole grid; list mode visits the pre-pass list (label tiles of flat blocks,
-// vocabulary-major), then every tile of each block that is not flat.
+// whole grid; list mode visits every tile of each token block that is not
+// flat, vocabulary-major (the flat blocks are handled by the flat-row kernel).
 struct TileMap {
-  int T, L, nnf;
+  int T, nnf;
   __device__ __forceinline__ void init(const BwdArgs& a) {
     if (a.list_mode) {
       T = (int)a.hdr[HDR_T];
-      L = (int)a.hdr[HDR_L];
       nnf = (int)a.hdr[HDR_NNF];
     } else {
       T = a.n_tiles;
-      L = 0;
       nnf = 0;
     }
   }
   __device__ __forceinline__ void get(const BwdArgs& a, int t, int& m, int& vt) const {
     if (!a.list_mode) {
       tile_coords(t, a.n_mblk, a.n_vtile, a.group_m, m, vt);
-    } else if (t < L) {
-      const int2 e = a.list[t];
-      m = e.x;
-      vt = e.y;
     } else {
-      const int k = t - L;
-      vt = k / nnf;
-      m = a.nonflat[k - vt * nnf];
+      vt = t / nnf;
+      m = a.nonflat[t - vt * nnf];
     }
   }
 };

@@ -15,8 +15,9 @@
 // Kernels (stream order):
 //   prep_cnorm    max_v |C_v| (fp32, atomicMax on the float's bits)
 //   prep_enorm    |E_i| per token (and the maximum)
-//   prep_blocks   per token block: flatness, label-tile counts
-//   prep_scan     totals: the tiles to visit (every tile of each block that
+//   prep_blocks   per token block: flatness; marks the dC rows (labels)
+//                 that flat blocks can touch
+//   prep_totals   totals: the tiles to visit (every tile of each block that
 //                 is not flat)
 //   flat_rows     the label entries of the flat blocks' tokens, formed
 //                 directly (no logit tile is recomputed for a flat block)
@@ -66,12 +67,11 @@ __device__ __forceinline__ void pruned_sub(const PrepArgs& p, unsigned long long
   atomicAdd(p.status + ST_PRUNED, 0ull - units);  // modulo 2^64: order of the updates is free
 }
 
-// Vocabulary tile v can receive a gradient only if the backward visits it:
-// with the filter on, when some token block is not flat (every tile is
-// visited) or some flat block has a label in v.  Rows of the other tiles
-// of dC are exactly zero.
-__device__ __forceinline__ bool vtile_visited(const unsigned* count, const unsigned* hdr, int all, int v) {
-  return all || hdr[HDR_NNF] != 0u || count[v] != 0u;
+// Row v of dC can receive a gradient only if some token block is not flat
+// (its tiles are all visited) or v is the label of a kept token of a flat
+// block (rowbits).  The other rows of dC are exactly zero.
+__device__ __forceinline__ bool row_visited(const unsigned* rowbits, const unsigned* hdr, int v) {
+  return hdr[HDR_NNF] != 0u || ((rowbits[v >> 5] >> (v & 31)) & 1u) != 0u;
 }
 
 }  // namespace
@@ -102,7 +102,6 @@ __global__ void __launch_bounds__(256) prep_enorm_kernel(const __nv_bfloat16* __
 // One CTA (128 threads) per token block.
 __global__ void __launch_bounds__(128) prep_blocks_kernel(const int64_t* __restrict__ y,
                                                           const float* __restrict__ lse, PrepArgs p) {
-  __shared__ int tl[BM];
   const int m = blockIdx.x;
   const int t = threadIdx.x;
   const int row = m * BM + t;
@@ -128,63 +127,20 @@ __global__ void __launch_bounds__(128) prep_blocks_kernel(const int64_t* __restr
     }
     return;
   }
-  tl[t] = has_col ? (int)(ylocal / BN) : -1;
-  __syncthreads();
-  bool owner = has_col;
-  for (int j = 0; j < t && owner; ++j) owner = tl[j] != tl[t];
-  if (owner) atomicAdd(p.count + tl[t], 1u);
+  // flat block: the flat-row kernel touches row ylocal of dC
+  if (has_col) atomicOr(p.rowbits + (ylocal >> 5), 1u << (ylocal & 31));
 }
 
-// Single CTA: exclusive scan of count[] -> offset[]; totals into the header.
-__global__ void __launch_bounds__(1024) prep_scan_kernel(PrepArgs p) {
-  __shared__ unsigned warp_sums[32];
-  __shared__ unsigned carry_s;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  if (t == 0) {
-    carry_s = 0;
-  }
-  __syncthreads();
-  for (int base = 0; base < p.n_vtile; base += 1024) {
-    const int i = base + t;
-    const unsigned x = i < p.n_vtile ? p.count[i] : 0u;
-    unsigned incl = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned n = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += n;
-    }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      unsigned ws = warp_sums[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned n = __shfl_up_sync(0xffffffffu, ws, o);
-        if (lane >= o) ws += n;
-      }
-      warp_sums[lane] = ws;  // inclusive over warps
-    }
-    __syncthreads();
-    const unsigned carry = carry_s;
-    const unsigned excl = carry + (warp ? warp_sums[warp - 1] : 0u) + incl - x;
-    if (i < p.n_vtile) p.offset[i] = excl;
-    __syncthreads();
-    if (t == 1023) carry_s = carry + warp_sums[31];
-    __syncthreads();
-  }
-  if (t == 0) {
-    // The label tiles of flat blocks are not visited: their only entries
-    // above the threshold are the label entries, which the flat-row kernel
-    // forms directly.  The list holds the non-flat blocks only.
-    const unsigned nnf = p.hdr[HDR_NNF];
-    const unsigned long long T = (unsigned long long)nnf * (unsigned long long)p.n_vtile;
-    p.hdr[HDR_L] = 0u;
-    p.hdr[HDR_T] = (unsigned)T;
-    // all filter units; the recomputed tiles' units are taken off by
-    // prep_blocks (dense blocks) and prep_scatter (listed tiles)
-    atomicAdd(p.status + ST_PRUNED,
-              (((unsigned long long)p.N + 31ull) / 32ull) * (((unsigned long long)p.V + 31ull) / 32ull));
-  }
+// Totals into the header once every block is classified: the tiles to visit
+// are every tile of each block that is not flat (vocabulary-major), and the
+// pruned-unit counter starts from all units (prep_blocks took off the dense
+// blocks' units, flat_rows takes off the flat blocks' live label units).
+__global__ void prep_totals_kernel(PrepArgs p) {
+  if (threadIdx.x != 0) return;
+  const unsigned nnf = p.hdr[HDR_NNF];
+  p.hdr[HDR_T] = (unsigned)((unsigned long long)nnf * (unsigned long long)p.n_vtile);
+  atomicAdd(p.status + ST_PRUNED,
+            (((unsigned long long)p.N + 31ull) / 32ull) * (((unsigned long long)p.V + 31ull) / 32ull));
 }
 
 // Flat token blocks: one CTA (32 warps) per 32-token row group, one warp per
@@ -313,60 +269,70 @@ __global__ void __launch_bounds__(256) prep_fixed_kernel(const float* __restrict
 
 // Deterministic mode: int64 fixed-point accumulators -> fp32 or bf16 output
 // (written, or with accumulate added to what the output holds: one add per
-// entry, so the result stays reproducible).
-// count / D: when count is non-null the accumulator is dC and only the rows
-// of visited vocabulary tiles (vtile_visited) were cleared and accumulated;
-// the others are exactly zero and are not read.
+// entry, so the result stays reproducible).  The n values are `rows` rows of
+// D.  When rowbits is non-null the accumulator is dC and only its visited
+// rows (row_visited) were cleared and accumulated: the others are exactly
+// zero and are not read (written as zeros, or left alone when accumulating).
+// One warp per row.
 __global__ void __launch_bounds__(256) fixed_to_out_kernel(const unsigned long long* __restrict__ acc, void* out,
-                                                           size_t n, const unsigned* __restrict__ hdr, int N,
+                                                           int rows, int D, const unsigned* __restrict__ hdr, int N,
                                                            int bf16, int accumulate,
-                                                           const unsigned* __restrict__ count, int D) {
+                                                           const unsigned* __restrict__ rowbits) {
   const int s = fixed_point_exponent(__uint_as_float(hdr[HDR_CMAX]), __uint_as_float(hdr[HDR_EMAX]),
                                      __uint_as_float(hdr[HDR_DLMAX]), N);
   const double inv = ldexp(1.0, -s);
-  const size_t stride = (size_t)gridDim.x * blockDim.x;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; 2 * i < n; i += stride) {
-    const bool live_row = count == nullptr || vtile_visited(count, hdr, 0, (int)((2 * i) / (size_t)D) / BN);
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int h = D >> 1;  // value pairs per row (D is even)
+  for (int row = gw; row < rows; row += nw) {
+    const bool live_row = rowbits == nullptr || row_visited(rowbits, hdr, row);
     if (!live_row && accumulate) continue;  // adds nothing: the output keeps its contents
-    const ulonglong2 q = live_row ? reinterpret_cast<const ulonglong2*>(acc)[i]   // n is even (D % 8 == 0)
-                                  : make_ulonglong2(0ull, 0ull);
-    double x0 = (double)(long long)q.x * inv, x1 = (double)(long long)q.y * inv;
-    if (bf16) {
-      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out) + i;
-      if (accumulate) {
-        const float2 old = __bfloat1622float2(*o);
-        x0 += (double)old.x;
-        x1 += (double)old.y;
+    const ulonglong2* a2 = reinterpret_cast<const ulonglong2*>(acc + (size_t)row * D);
+    for (int j = lane; j < h; j += 32) {
+      const ulonglong2 q = live_row ? a2[j] : make_ulonglong2(0ull, 0ull);
+      double x0 = (double)(long long)q.x * inv, x1 = (double)(long long)q.y * inv;
+      const size_t i = (size_t)row * h + j;
+      if (bf16) {
+        __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out) + i;
+        if (accumulate) {
+          const float2 old = __bfloat1622float2(*o);
+          x0 += (double)old.x;
+          x1 += (double)old.y;
+        }
+        *o = __halves2bfloat162(__double2bfloat16(x0), __double2bfloat16(x1));
+      } else {
+        float2* o = reinterpret_cast<float2*>(out) + i;
+        float2 r = make_float2((float)x0, (float)x1);
+        if (accumulate) {
+          const float2 old = *o;
+          r.x = old.x + r.x;  // fp32 add of this call's sum, rounded once to fp32
+          r.y = old.y + r.y;
+        }
+        *o = r;
       }
-      *o = __halves2bfloat162(__double2bfloat16(x0), __double2bfloat16(x1));
-    } else {
-      float2* o = reinterpret_cast<float2*>(out) + i;
-      float2 r = make_float2((float)x0, (float)x1);
-      if (accumulate) {
-        const float2 old = *o;
-        r.x = old.x + r.x;  // fp32 add of this call's sum, rounded once to fp32
-        r.y = old.y + r.y;
-      }
-      *o = r;
     }
   }
 }
 
-// Fixed-point dC accumulator: clear the rows of visited vocabulary tiles only.
+// Fixed-point dC accumulator: clear the visited rows only (one warp per row).
 __global__ void __launch_bounds__(256) clear_visited_rows_kernel(unsigned long long* __restrict__ acc, int V, int D,
-                                                                 const unsigned* __restrict__ count,
+                                                                 const unsigned* __restrict__ rowbits,
                                                                  const unsigned* __restrict__ hdr) {
-  const size_t n2 = (size_t)V * D / 2;  // D is even
-  const size_t stride = (size_t)gridDim.x * blockDim.x;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += stride) {
-    const int row = (int)((2 * i) / (size_t)D);
-    if (vtile_visited(count, hdr, 0, row / BN)) reinterpret_cast<ulonglong2*>(acc)[i] = make_ulonglong2(0ull, 0ull);
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int h = D >> 1;
+  for (int row = gw; row < V; row += nw) {
+    if (!row_visited(rowbits, hdr, row)) continue;
+    ulonglong2* a2 = reinterpret_cast<ulonglong2*>(acc + (size_t)row * D);
+    for (int j = lane; j < h; j += 32) a2[j] = make_ulonglong2(0ull, 0ull);
   }
 }
 
-cudaError_t launch_clear_visited_rows(unsigned long long* acc, int V, int D, const unsigned* count,
+cudaError_t launch_clear_visited_rows(unsigned long long* acc, int V, int D, const unsigned* rowbits,
                                       const unsigned* hdr, int sms, cudaStream_t stream) {
-  clear_visited_rows_kernel<<<sms * 8, 256, 0, stream>>>(acc, V, D, count, hdr);
+  clear_visited_rows_kernel<<<sms * 8, 256, 0, stream>>>(acc, V, D, rowbits, hdr);
   return cudaGetLastError();
 }
 
@@ -375,10 +341,11 @@ cudaError_t launch_fixed_prep(const float* dloss, const PrepArgs& p, int sms, cu
   return cudaGetLastError();
 }
 
-cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, size_t n, const unsigned* hdr, int N,
-                                bool bf16, bool accumulate, const unsigned* count, int D, int sms,
+cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, int rows, int D, const unsigned* hdr,
+                                int N, bool bf16, bool accumulate, const unsigned* rowbits, int sms,
                                 cudaStream_t stream) {
-  fixed_to_out_kernel<<<sms * 8, 256, 0, stream>>>(acc, out, n, hdr, N, bf16 ? 1 : 0, accumulate ? 1 : 0, count, D);
+  fixed_to_out_kernel<<<sms * 8, 256, 0, stream>>>(acc, out, rows, D, hdr, N, bf16 ? 1 : 0, accumulate ? 1 : 0,
+                                                   rowbits);
   return cudaGetLastError();
 }
 
@@ -399,7 +366,7 @@ cudaError_t launch_prep(const void* E, const void* C, const int64_t* y, const fl
                         int sms, cudaStream_t stream) {
   // expects launch_cnorm and launch_enorm to have run
   prep_blocks_kernel<<<p.n_mblk, 128, 0, stream>>>(y, lse, p);
-  prep_scan_kernel<<<1, 1024, 0, stream>>>(p);
+  prep_totals_kernel<<<1, 32, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -39,8 +39,7 @@ enum StatusWord : int {
 enum PrepHeader : int {
   HDR_CMAX = 0,  // max_v |C_v| as float bits
   HDR_NNF = 1,   // token blocks that are not flat (visited densely)
-  HDR_L = 2,     // label tiles of flat blocks (list length)
-  HDR_T = 3,     // tiles to visit: L + NNF * n_vtile
+  HDR_T = 3,     // tiles to visit: NNF * n_vtile (word 2 is unused)
   HDR_EMAX = 4,  // max_i |E_i| as float bits (fixed-point accumulation)
   HDR_DLMAX = 5, // max_i |dloss_i| as float bits (fixed-point accumulation)
 };
@@ -64,6 +63,7 @@ struct FwdArgs {
   unsigned long long wait_limit_ns;
   int withhold_loads;          // test hook: the TMA producer issues nothing
   int pf;                      // L2 prefetch distance of the C stream in K slices (0: off)
+  int l2_hints;                // CTA-pair kernel: bit 0 E slices evict_last, bit 1 C slices evict_first
 };
 
 struct FinArgs {
@@ -85,12 +85,9 @@ struct PrepArgs {
   long long v_offset;
   float log_eps;          // ln(filter_eps)
   unsigned* hdr;          // PrepHeader words
-  unsigned* count;        // [n_vtile] label tiles per vocabulary tile
-  unsigned* offset;       // [n_vtile] exclusive scan of count
-  unsigned* cursor;       // [n_vtile] fill cursors
+  unsigned* rowbits;      // [ceil(V / 32)] bit v: row v of dC is a label of a flat block's kept token
   int* blk_flat;          // [n_mblk]
   int* nonflat;           // [n_mblk] ids of blocks that are not flat
-  int2* list;             // [<= N] (token block, vocabulary tile), vocabulary-major
   float* enorm;           // [N] |E_i|
   unsigned long long* status;
 };
@@ -119,11 +116,10 @@ struct BwdArgs {
   int n_mblk, n_vtile;
   int n_tiles;          // tiles to visit (dense mode)
   int group_m;          // token blocks per raster group (dense mode)
-  int list_mode;        // 1: visit the pre-pass list (hdr, list, nonflat)
+  int list_mode;        // 1: visit the tiles of the blocks that are not flat (hdr, nonflat)
   int shard_mode;       // 1: C is a vocabulary shard starting at global id v_offset
   long long v_offset;
   const unsigned* hdr;
-  const int2* list;
   const int* nonflat;
   float filter_eps;     // <= 0: every tile is live
   long long ignore_index;

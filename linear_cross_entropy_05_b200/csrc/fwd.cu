@@ -331,6 +331,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       // ---------------- TMA producer (both CTAs) ----------------
       int stage = 0;
       uint32_t phase = 0, armed = 0;
+      // optional L2 eviction priorities: E (re-read for every vocabulary
+      // tile) kept, C (read by every token block in turn) evicted first
+      const uint64_t pol_e = l2_policy_evict_last(), pol_c = l2_policy_evict_first();
+      const bool hint_e = (a.l2_hints & 1) != 0, hint_c = (a.l2_hints & 2) != 0;
       for (int u = a.withhold_loads ? a.n_units : pair; u < a.n_units; u += n_pairs) {
         int r, m2;
         unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m2);
@@ -340,8 +344,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           for (int kb = 0; kb < nkb; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
             if (leader) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
-            tma_load_2d_pair(sA + stage * A_STAGE_BYTES, &tmE, &full[stage], kb * BK, m2 * (2 * BM) + rank * BM);
-            tma_load_2d_pair(sB + stage * A_STAGE_BYTES, &tmCh, &full[stage], kb * BK, vt * BN + rank * BM);
+            void* dA = sA + stage * A_STAGE_BYTES;
+            void* dB = sB + stage * A_STAGE_BYTES;
+            const int yE = m2 * (2 * BM) + rank * BM, yC = vt * BN + rank * BM;
+            if (hint_e)
+              tma_load_2d_pair_hint(dA, &tmE, &full[stage], kb * BK, yE, pol_e);
+            else
+              tma_load_2d_pair(dA, &tmE, &full[stage], kb * BK, yE);
+            if (hint_c)
+              tma_load_2d_pair_hint(dB, &tmCh, &full[stage], kb * BK, yC, pol_c);
+            else
+              tma_load_2d_pair(dB, &tmCh, &full[stage], kb * BK, yC);
             armed |= 1u << stage;
             if (a.pf) {  // L2 prefetch of this CTA's C rows a.pf slices ahead in the unit's stream
               const int s2 = (vt - v0) * nkb + kb + a.pf;

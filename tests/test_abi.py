@@ -117,11 +117,11 @@ def test_workspace_size_without_device_is_zero(lib):
     from linear_cross_entropy_05_b200 import cce_backward_workspace_size, cce_forward_workspace_size
     assert cce_forward_workspace_size(8192, 2304, 256000) == 0
     assert cce_forward_workspace_size(0, 8, 8) == 0
-    # status 256 + header 256 + 3 x [V/256] u32 + 2 x [N/128] i32 + N int2 + N f32,
+    # status 256 + header 256 + one bit per vocabulary row + 2 x [N/128] i32 + N f32,
     # each rounded to 256 bytes
     up = lambda x: (x + 255) // 256 * 256
     for N, V in ((8192, 256000), (300, 4173), (65536, 262144)):
-        want = 512 + 3 * up(4 * (-(-V // 256))) + 2 * up(4 * (-(-N // 128))) + up(8 * N) + up(4 * N)
+        want = 512 + up(4 * (-(-V // 32))) + 2 * up(4 * (-(-N // 128))) + up(4 * N)
         assert cce_backward_workspace_size(N, 2304, V) == want
     assert cce_backward_workspace_size(8192, 2305, 256000) == 0
 
@@ -188,3 +188,11 @@ def test_shard_entry_points_validate_on_the_host(lib):
     assert cce_merge_shards(P, 2, 256, P, 8192, -100, P, P, 0, check=False) == 4
     assert cce_backward_shard(P, P, P, P, P, 256, 256, 4096, -5, -100, 0.0, P, P, P, 1 << 20, 0,
                               check=False) == 1
+
+
+def test_forward_schedule_knob_validates_on_the_host(lib):
+    assert lib.cce_debug_set_forward_schedule(65, 0, 0) == 1       # more than 64 splits
+    assert lib.cce_debug_set_forward_schedule(0, -1, 0) == 1
+    assert lib.cce_debug_set_forward_schedule(0, 0, 4) == 1        # hint bits beyond E and C
+    assert lib.cce_debug_set_forward_schedule(37, 8, 3) == 0
+    assert lib.cce_debug_set_forward_schedule(0, 0, 0) == 0        # back to the per-shape choice

@@ -58,11 +58,12 @@ def test_stored_traffic_is_reported_only_for_the_same_kernel_code(monkeypatch, t
 
 def test_launch_count_matches_the_kernels_a_step_runs(monkeypatch, tmp_path):
     # one step = fwd_lse(_pair) + finalize, then with the filter on:
-    # cnorm, enorm, blocks, scan, scatter, bwd_kernel (the launch list of a
+    # cnorm, enorm, blocks, scan, flat_rows, bwd_kernel (the launch list of a
     # profiled step shows these eight); fixed point adds the dloss maximum
-    # and the two conversion passes
+    # and the two conversion passes, and with the filter on the clearing of
+    # the visited dC accumulator rows
     b = _bench(monkeypatch, tmp_path)
     assert b.launches_per_step(2.0 ** -12, False) == 8
     assert b.launches_per_step(0.0, False) == 3
     assert b.launches_per_step(0.0, True) == 8
-    assert b.launches_per_step(2.0 ** -12, True) == 11
+    assert b.launches_per_step(2.0 ** -12, True) == 12

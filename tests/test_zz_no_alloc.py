@@ -80,9 +80,10 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     import torch
     import linear_cross_entropy_05_b200 as L
     torch.cuda.init()
-    # the N = 65536 sweep needs ~20 MiB of partials; the static scratch is 8 MiB
-    assert L.cce_forward_workspace_size(65536, 2048, 262144) > (8 << 20)
-    st = L.cce_forward_noalloc(0, 0, 0, 65536, 2048, 262144, IGN, 0, 0, 0, check=False)
+    # 131072 tokens over a 262144-entry vocabulary need ~26 MB of partials;
+    # the static scratch is 8 MiB
+    assert L.cce_forward_workspace_size(131072, 2048, 262144) > (8 << 20)
+    st = L.cce_forward_noalloc(0, 0, 0, 131072, 2048, 262144, IGN, 0, 0, 0, check=False)
     assert st == CCE_ERR_WORKSPACE_TOO_SMALL  # nothing launched
 
 
