@@ -116,16 +116,45 @@ def vocab_shard(V: int, world: int, rank: int, tile: int = 256):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU sampled during a
+    timed region: through NVML every 2 ms when the bindings import (the
+    source nvidia-smi reads), else `nvidia-smi -lms 100`.  The GPU is found by
+    the PCI bus id of the CUDA device when torch exposes it (the NVML index
+    may differ from the CUDA index under CUDA_VISIBLE_DEVICES)."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.002
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.nvml = None
         self.lines = []
+        self.samples = []   # (sm MHz, power W, reasons bitmask) from NVML
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(self.gpu)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.upper())
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        try:
+            self.nvml = self._nvml_handle()
+        except Exception as e:
+            log("NVML unavailable, sampling with nvidia-smi:", e)
+            self.nvml = None
+        if self.nvml is not None:
+            self.stop_flag = False
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
@@ -136,11 +165,47 @@ class ClockSampler:
             log("clock sampler unavailable:", e)
             self.proc = None
 
+    def _poll_nvml(self):
+        nv, h = self.nvml
+        while not self.stop_flag:
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def _stop_nvml(self):
+        nv, h = self.nvml
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        try:
+            smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            smax = None
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        sm = [float(c) for c, _, _ in self.samples]
+        pw = [p for _, p, _ in self.samples]
+        reasons = sorted(n for n, b in bits.items() if any(r & b for _, _, r in self.samples))
+        cap = [bool(r & bits["sw_power_cap"]) for _, _, r in self.samples]
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "sm_mhz_min": min(sm) if sm else None, "sm_mhz_p90": float(np.percentile(sm, 90)) if sm else None,
+                "reasons": reasons, "samples": len(sm), "source": "nvml 2 ms",
+                "power_cap_frac": float(np.mean(cap)) if cap else None,
+                "power_w_max": max(pw) if pw else None}
+
     def stop(self):
+        if self.nvml is not None:
+            return self._stop_nvml()
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.proc.terminate()
@@ -165,7 +230,8 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm), "power_w_max": max(pw) if pw else None}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi 100 ms",
+                "power_w_max": max(pw) if pw else None}
 
 
 # ---------------------------------------------------------------------------
@@ -993,10 +1059,11 @@ def main(argv=None):
                     help="L2 prefetch distance of the filtered backward's reduction targets (A/B; 0 = off)")
     ap.add_argument("--l2-hints", action="store_true",
                     help="L2 eviction priorities in the filtered backward (A/B)")
-    ap.add_argument("--fwd-schedule", type=int, nargs=3, default=None, metavar=("SPLITS", "GROUP_M", "L2_HINTS"),
+    ap.add_argument("--fwd-schedule", type=int, nargs=4, default=None,
+                    metavar=("SPLITS", "GROUP_M", "L2_HINTS", "STAGES"),
                     help="forward schedule (A/B): vocabulary splits per token block and token blocks per raster "
                          "group (0 = chosen per shape), L2 hints of the pair kernel (bit 0: E evict_last, bit 1: C "
-                         "evict_first)")
+                         "evict_first), its operand stages (0 = default 7, or 6)")
     ap.add_argument("--trace", action="store_true",
                     help="per-tile timeline of one backward launch (recompute wait, gradient tile, contraction)")
     ap.add_argument("--dense-trace", action="store_true",

@@ -52,11 +52,13 @@ CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
  * chosen per shape, ~48 MB of E rows) is the number of token blocks per
  * raster group; l2_hints (0..3, default 0; CTA-pair kernel only) gives the
  * E slices the evict_last L2 policy (bit 0) and the C slices evict_first
- * (bit 1).  Same loss and lse up to fp32 rounding order.  The forward
+ * (bit 1); stages (0 = the default 7, or 6 or 7; CTA-pair kernel only) is
+ * the number of 32 KB operand stages per CTA (7 fill the 227 KB of shared
+ * memory; 1 % faster than 6 on the Gemma-2-2B-shaped head).  Same loss and lse up to fp32 rounding order.  The forward
  * workspace size depends on n_split: query cce_forward_workspace_size after
  * changing it.  Process-wide.  Returns CCE_ERR_INVALID_ARG for other
  * values. */
-CCE_API cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hints);
+CCE_API cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hints, int stages);
 
 /* Tuning knobs of the dense stripe backward (CCE_BWD_STRIPES), for A/B
  * measurement: tokens_per_launch (a multiple of 256, at most 16384; 0 = the

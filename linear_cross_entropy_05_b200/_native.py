@@ -91,7 +91,7 @@ def load_library():
         lib.cce_debug_set_stripe_params.restype = ctypes.c_int
         lib.cce_debug_set_l2_hints.argtypes = [ctypes.c_int]
         lib.cce_debug_set_l2_hints.restype = ctypes.c_int
-        lib.cce_debug_set_forward_schedule.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.cce_debug_set_forward_schedule.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         lib.cce_debug_set_forward_schedule.restype = ctypes.c_int
         lib.cce_debug_set_reduce_prefetch.argtypes = [ctypes.c_int]
         lib.cce_debug_set_reduce_prefetch.restype = ctypes.c_int
@@ -294,9 +294,10 @@ def cce_debug_set_l2_hints(on: bool) -> None:
     _check(load_library().cce_debug_set_l2_hints(1 if on else 0), "cce_debug_set_l2_hints")
 
 
-def cce_debug_set_forward_schedule(n_split: int = 0, group_m: int = 0, l2_hints: int = 0) -> None:
+def cce_debug_set_forward_schedule(n_split: int = 0, group_m: int = 0, l2_hints: int = 0, stages: int = 0) -> None:
     """Forward schedule knobs (A/B): vocabulary splits per token block, token
-    blocks per raster group (0 = chosen per shape) and L2 eviction hints of
-    the CTA-pair kernel (bit 0: E evict_last, bit 1: C evict_first)."""
-    _check(load_library().cce_debug_set_forward_schedule(int(n_split), int(group_m), int(l2_hints)),
+    blocks per raster group (0 = chosen per shape), L2 eviction hints of the
+    CTA-pair kernel (bit 0: E evict_last, bit 1: C evict_first) and its
+    operand stages per CTA (0 = default 7, or 6)."""
+    _check(load_library().cce_debug_set_forward_schedule(int(n_split), int(group_m), int(l2_hints), int(stages)),
            "cce_debug_set_forward_schedule")

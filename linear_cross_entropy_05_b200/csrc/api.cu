@@ -22,7 +22,7 @@ namespace cce {
 cudaError_t launch_fwd_lse(const CUtensorMap& tmE, const CUtensorMap& tmC, const FwdArgs& a, int grid,
                            cudaStream_t stream);
 cudaError_t launch_fwd_lse_pair(const CUtensorMap& tmE, const CUtensorMap& tmCh, const FwdArgs& a, int grid,
-                                cudaStream_t stream);
+                                int stages, cudaStream_t stream);
 cudaError_t launch_fwd_finalize(const void* E, const void* C, const int64_t* y, const FinArgs& a, float* loss,
                                 float* lse, cudaStream_t stream);
 cudaError_t launch_merge_shards(const float* stats, int R, int N, const int64_t* y, long long V_total,
@@ -62,6 +62,7 @@ std::atomic<int> g_fwd_pf{0};  // L2 prefetch distances (K slices) of the forwar
 std::atomic<int> g_fwd_split{0};     // forward vocabulary splits per token block (0: chosen per shape)
 std::atomic<int> g_fwd_group_m{0};   // forward token blocks per raster group (0: chosen per shape)
 std::atomic<int> g_fwd_l2_hints{0};  // forward CTA-pair kernel: L2 eviction priorities (A/B)
+std::atomic<int> g_fwd_stages{PAIR_STAGES_MAX};  // forward CTA-pair kernel: operand stages per CTA
 std::atomic<int> g_bwd_pf{0};
 std::atomic<int> g_bwd_red_pf{0};  // L2 prefetch distance (K slices) of the backward's reduction targets
 std::atomic<int> g_bwd_l2_hints{0};  // L2 eviction priorities in the filtered backward (A/B)
@@ -373,7 +374,8 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   a.l2_hints = g_fwd_l2_hints.load();
   if (record_event(0, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   const cudaError_t le =
-      p.pair ? launch_fwd_lse_pair(tmE, tmC, a, p.grid, stream) : launch_fwd_lse(tmE, tmC, a, p.grid, stream);
+      p.pair ? launch_fwd_lse_pair(tmE, tmC, a, p.grid, g_fwd_stages.load(), stream)
+             : launch_fwd_lse(tmE, tmC, a, p.grid, stream);
   if (le != cudaSuccess) return CCE_ERR_CUDA;
   if (record_event(0, 1, stream) != cudaSuccess) return CCE_ERR_CUDA;
 
@@ -433,11 +435,13 @@ cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices) {
   return CCE_OK;
 }
 
-cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hints) {
+cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hints, int stages) {
   if (n_split < 0 || n_split > 64 || group_m < 0 || l2_hints < 0 || l2_hints > 3) return CCE_ERR_INVALID_ARG;
+  if (stages != 0 && stages != PAIR_STAGES && stages != PAIR_STAGES_MAX) return CCE_ERR_INVALID_ARG;
   g_fwd_split.store(n_split);
   g_fwd_group_m.store(group_m);
   g_fwd_l2_hints.store(l2_hints);
+  g_fwd_stages.store(stages ? stages : PAIR_STAGES_MAX);
   return CCE_OK;
 }
 

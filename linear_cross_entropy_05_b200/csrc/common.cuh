@@ -17,7 +17,8 @@ constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int QUARTER_BYTES = 64 * BK * 2;   // C slice [64 rows][64 d]: one K block of the dE product
 constexpr int NUM_THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int FWD_STAGES = 4;
-constexpr int PAIR_STAGES = 6;                          // CTA-pair forward: E half + C half per stage
+constexpr int PAIR_STAGES = 6;                          // CTA-pair forward: E half + C half per stage (A/B)
+constexpr int PAIR_STAGES_MAX = 7;                      // the default: the most that fit in 227 KB of shared memory
 constexpr int PAIR_STAGE_BYTES = 2 * A_STAGE_BYTES;     // [128][64] bf16 of E and of C
 constexpr int BWD_STAGES = 3;
 constexpr int G_BYTES = BM * BN * 2;        // bf16 softmax-gradient tile (4 swizzled K blocks)

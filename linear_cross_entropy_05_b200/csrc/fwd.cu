@@ -267,25 +267,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // CTA-pair variant: a cluster of two CTAs on two SMs computes 256 x 256 logit
 // tiles with tcgen05.mma.cta_group::2 (M = 256 split over the pair).  Each CTA
 // loads its own 128 token rows of E and 128 vocabulary rows of C per stage
-// (32 KB instead of 48 KB per SM for the same MMA work, so 6 stages fit), and
+// (32 KB instead of 48 KB per SM for the same MMA work, so 7 stages fit), and
 // each CTA's TMEM holds its 128 rows x 256 columns of every tile, which its own
 // epilogue folds exactly as in the single-CTA kernel.  Only the even (leader)
 // CTA issues UMMAs; its full barriers count both CTAs' copies, its commits
 // arrive on both CTAs' barriers, and both epilogues release the accumulator
 // on the leader's barrier.  No TMA multicast is used.
 // ----------------------------------------------------------------------------
-template <bool DUMP>
+template <bool DUMP, int S>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     fwd_lse_pair_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmCh,
                         const FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;                                    // PAIR_STAGES x [128 tok][64 d]
-  uint8_t* sB = smem + PAIR_STAGES * A_STAGE_BYTES;      // PAIR_STAGES x [128 voc][64 d]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + PAIR_STAGES * A_STAGE_BYTES);
+  uint8_t* sA = smem;                                    // S x [128 tok][64 d]
+  uint8_t* sB = smem + S * A_STAGE_BYTES;      // S x [128 voc][64 d]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * A_STAGE_BYTES);
   uint64_t* full = bars;                      // leader: both CTAs' copies landed
-  uint64_t* empty = bars + PAIR_STAGES;       // each CTA: stage free again
-  uint64_t* tfull = bars + 2 * PAIR_STAGES;   // each CTA: accumulator ready
+  uint64_t* empty = bars + S;       // each CTA: stage free again
+  uint64_t* tfull = bars + 2 * S;   // each CTA: accumulator ready
   uint64_t* tempty = tfull + 2;               // leader: both epilogues done with the accumulator
   uint64_t* drain = tempty + 2;               // leader: UMMA drain at exit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -299,7 +299,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const int n_pairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < PAIR_STAGES; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -356,12 +356,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             else
               tma_load_2d_pair(dB, &tmCh, &full[stage], kb * BK, yC);
             armed |= 1u << stage;
-            if (a.pf) {  // L2 prefetch of this CTA's C rows a.pf slices ahead in the unit's stream
+            // L2 prefetch of this CTA's C rows a.pf slices ahead in the unit's
+            // stream, by the pair on the first token block of the raster group
+            // only (the other pairs on this split read the same rows)
+            if (a.pf && m2 % a.group_m == 0) {
               const int s2 = (vt - v0) * nkb + kb + a.pf;
               if (s2 < (v1 - v0) * nkb)
                 tma_prefetch_l2_2d(&tmCh, (s2 % nkb) * BK, (v0 + s2 / nkb) * BN + rank * BM);
             }
-            if (++stage == PAIR_STAGES) {
+            if (++stage == S) {
               stage = 0;
               phase ^= 1u;
             }
@@ -375,7 +378,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       if (leader) {
         int dummy = 0;
         WaitCtl exit_wc{&dummy, a.wait_limit_ns};
-        for (int s = 0; s < PAIR_STAGES; ++s)
+        for (int s = 0; s < S; ++s)
           if (armed & (1u << s)) mbar_wait(&full[s], (s < stage) ? phase : (phase ^ 1u), exit_wc);
       }
     }
@@ -406,7 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               umma_bf16_pair(d_tmem, sdesc_sw128(a_addr + k * 32, 16, 1024), sdesc_sw128(b_addr + k * 32, 16, 1024),
                              IDESC, (kb | k) != 0);
             umma_commit_pair_mc(&empty[stage], 0x3);
-            if (++stage == PAIR_STAGES) {
+            if (++stage == S) {
               stage = 0;
               phase ^= 1u;
             }
@@ -629,24 +632,30 @@ cudaError_t launch_merge_shards(const float* stats, int R, int N, const int64_t*
 }
 
 size_t fwd_smem_bytes() { return 1024 + (size_t)FWD_STAGES * STAGE_BYTES + 256; }
-size_t fwd_pair_smem_bytes() { return 1024 + (size_t)PAIR_STAGES * PAIR_STAGE_BYTES + 256; }
+size_t fwd_pair_smem_bytes(int stages) { return 1024 + (size_t)stages * PAIR_STAGE_BYTES + 256; }
 
-// grid: an even number of CTAs (pairs)
-cudaError_t launch_fwd_lse_pair(const CUtensorMap& tmE, const CUtensorMap& tmCh, const FwdArgs& a, int grid,
-                                cudaStream_t stream) {
-  const size_t smem = fwd_pair_smem_bytes();
-  if (a.dbg_logits) {
-    cudaError_t e =
-        cudaFuncSetAttribute(fwd_lse_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    fwd_lse_pair_kernel<true><<<grid, NUM_THREADS, smem, stream>>>(tmE, tmCh, a);
-  } else {
-    cudaError_t e =
-        cudaFuncSetAttribute(fwd_lse_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    fwd_lse_pair_kernel<false><<<grid, NUM_THREADS, smem, stream>>>(tmE, tmCh, a);
-  }
+namespace {
+template <bool DUMP, int S>
+cudaError_t launch_pair_stages(const CUtensorMap& tmE, const CUtensorMap& tmCh, const FwdArgs& a, int grid,
+                               cudaStream_t stream) {
+  const size_t smem = fwd_pair_smem_bytes(S);
+  cudaError_t e = cudaFuncSetAttribute(fwd_lse_pair_kernel<DUMP, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  fwd_lse_pair_kernel<DUMP, S><<<grid, NUM_THREADS, smem, stream>>>(tmE, tmCh, a);
   return cudaGetLastError();
+}
+}  // namespace
+
+// grid: an even number of CTAs (pairs); stages: PAIR_STAGES or PAIR_STAGES_MAX
+// operand stages per CTA (the latter fills the 227 KB of shared memory)
+cudaError_t launch_fwd_lse_pair(const CUtensorMap& tmE, const CUtensorMap& tmCh, const FwdArgs& a, int grid,
+                                int stages, cudaStream_t stream) {
+  if (stages == PAIR_STAGES_MAX)
+    return a.dbg_logits ? launch_pair_stages<true, PAIR_STAGES_MAX>(tmE, tmCh, a, grid, stream)
+                        : launch_pair_stages<false, PAIR_STAGES_MAX>(tmE, tmCh, a, grid, stream);
+  return a.dbg_logits ? launch_pair_stages<true, PAIR_STAGES>(tmE, tmCh, a, grid, stream)
+                      : launch_pair_stages<false, PAIR_STAGES>(tmE, tmCh, a, grid, stream);
 }
 
 cudaError_t launch_fwd_lse(const CUtensorMap& tmE, const CUtensorMap& tmC, const FwdArgs& a, int grid,

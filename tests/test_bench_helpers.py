@@ -67,3 +67,46 @@ def test_launch_count_matches_the_kernels_a_step_runs(monkeypatch, tmp_path):
     assert b.launches_per_step(0.0, False) == 3
     assert b.launches_per_step(0.0, True) == 8
     assert b.launches_per_step(2.0 ** -12, True) == 12
+
+
+def test_clock_sampler_reduces_nvml_samples(monkeypatch, tmp_path):
+    # a fake NVML: the clock falls under the power cap, one sample shows a
+    # thermal slowdown; the summary gives the median, the minimum and every
+    # reason seen
+    import sys
+    import types
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1, nvmlClocksEventReasonHwSlowdown=8, nvmlClocksEventReasonHwThermalSlowdown=64,
+        nvmlClocksEventReasonHwPowerBrakeSlowdown=128, nvmlClocksEventReasonSwThermalSlowdown=32,
+        nvmlClocksEventReasonSwPowerCap=4)
+    seq = [(1965, 0), (1965, 4), (1300, 4), (1250, 4), (1250, 4 | 32)]
+    state = {"i": 0}
+
+    def clock(h, which):
+        return seq[min(state["i"], len(seq) - 1)][0]
+
+    def reasons(h):
+        r = seq[min(state["i"], len(seq) - 1)][1]
+        state["i"] += 1
+        return r
+
+    fake.nvmlInit = lambda: None
+    fake.nvmlDeviceGetHandleByIndex = lambda i: "gpu"
+    fake.nvmlDeviceGetHandleByPciBusId = lambda bus: "gpu"
+    fake.nvmlDeviceGetClockInfo = clock
+    fake.nvmlDeviceGetPowerUsage = lambda h: 900000
+    fake.nvmlDeviceGetCurrentClocksEventReasons = reasons
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, which: 1965
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    b = _bench(monkeypatch, tmp_path)
+    cs = b.ClockSampler(0)
+    cs.PERIOD_S = 0.0005
+    cs.start()
+    import time
+    while state["i"] < len(seq):
+        time.sleep(0.001)
+    out = cs.stop()
+    # the last reading repeats after the sequence ends; compare on what was seen
+    assert out["sm_max_mhz"] == 1965 and out["sm_mhz_min"] == 1250
+    assert out["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+    assert out["sm_mhz"] <= 1300 and out["power_w_max"] == 900.0 and out["source"].startswith("nvml")

@@ -197,11 +197,13 @@ def test_single_cta_forward_variant_matches_oracle(w):
     assert np.abs(loss0 - loss1).max() <= 1e-4
 
 
-@pytest.mark.parametrize("sched", [(1, 1, 1), (37, 0, 3), (64, 2, 2), (5, 3, 0)],
-                         ids=["one-split-E-hint", "37-splits-both-hints", "64-splits-C-hint", "5-splits-groups-of-3"])
+@pytest.mark.parametrize("sched", [(1, 1, 1, 0), (37, 0, 3, 7), (64, 2, 2, 0), (5, 3, 0, 7), (0, 0, 0, 7)],
+                         ids=["one-split-E-hint", "37-splits-both-hints-7-stages", "64-splits-C-hint",
+                              "5-splits-groups-of-3-7-stages", "7-stages"])
 def test_forward_schedule_knobs_keep_the_result(sched):
-    # the split count (partials per token), the raster group and the L2
-    # hints change only the order of work: the loss stays the oracle's
+    # the split count (partials per token), the raster group, the L2 hints
+    # and the pipeline depth change only the order of work: the loss stays
+    # the oracle's
     import linear_cross_entropy_05_b200 as L
     w = synth.GEMMA2_2B.with_sizes(N=1000 + 300, V=20000 + 77, D=512)
     inp = synth.make_inputs(w)
@@ -210,7 +212,7 @@ def test_forward_schedule_knobs_keep_the_result(sched):
     try:
         loss, lse, st = gpu_forward(E, C, y)
     finally:
-        L.cce_debug_set_forward_schedule(0, 0, 0)
+        L.cce_debug_set_forward_schedule(0, 0, 0, 0)
     assert st["status"] == 0 and st["flags"] == 0
     ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
     assert np.abs(loss - ol).max() <= LOSS_ABS
