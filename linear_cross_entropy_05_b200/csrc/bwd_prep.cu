@@ -148,14 +148,23 @@ __global__ void prep_totals_kernel(PrepArgs p) {
 //   z = E_i . C_y,  p = exp(z - lse_i),  d = p - 1,
 // its only entry with |d| >= filter_eps (the pre-pass proved all others
 // below it); if |d| >= eps, G = dloss_i d adds G C_y to dE_i (the warp owns
-// the row) and G E_i to dC_y (atomically: tokens share labels).  The live
-// 32 x 32 units of the row group are its distinct live label chunks; they
-// move from the pruned to the live count.
+// the row: plain stores) and G E_i to dC_y.  Tokens share labels, so the dC
+// row is added with bulk reduce-adds: the warp writes 1 KB pieces of G E_i
+// (fp32, or int64 fixed point in the deterministic mode) into one of two
+// shared-memory buffers and one lane hands each piece to the TMA engine,
+// which adds it at L2 -- 9 operations per 2304-wide row instead of 576
+// vector (or 2304 64-bit) atomics.  The live 32 x 32 units of the row group
+// are its distinct live label chunks; they move from the pruned to the live
+// count.
+constexpr int FLAT_PIECE = 1024;                           // bytes per bulk reduce-add
+constexpr int FLAT_SMEM = 32 * 2 * FLAT_PIECE;             // two pieces per warp
+
 __global__ void __launch_bounds__(1024) flat_rows_kernel(const __nv_bfloat16* __restrict__ E,
                                                          const __nv_bfloat16* __restrict__ C,
                                                          const int64_t* __restrict__ y,
                                                          const float* __restrict__ lse,
                                                          const float* __restrict__ dloss, FlatArgs f) {
+  extern __shared__ __align__(128) uint8_t flat_smem[];
   __shared__ int chunk_of[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g0 = blockIdx.x * 32;              // first token of the row group
@@ -194,42 +203,85 @@ __global__ void __launch_bounds__(1024) flat_rows_kernel(const __nv_bfloat16* __
             fixed ? ldexpf(1.f, fixed_point_exponent(__uint_as_float(f.hdr[HDR_CMAX]), __uint_as_float(f.hdr[HDR_EMAX]),
                                                      __uint_as_float(f.hdr[HDR_DLMAX]), f.N))
                   : 0.f;
-        for (int i = lane; i < nvec; i += 32) {
-          const uint4 ev = __ldg(er + i), cv = __ldg(cr + i);
-          const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&ev);
-          const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&cv);
-          float ce[8], ee[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 cf = __bfloat1622float2(c2[j]);
-            const float2 ef = __bfloat1622float2(e2[j]);
-            ce[2 * j] = g * cf.x;
-            ce[2 * j + 1] = g * cf.y;
-            ee[2 * j] = g * ef.x;
-            ee[2 * j + 1] = g * ef.y;
+        // elements per piece: 256 fp32 or 128 int64; a lane takes 8 or 4 of them
+        const int per_piece = fixed ? FLAT_PIECE / 8 : FLAT_PIECE / 4;
+        const int per_lane = per_piece / 32;
+        uint8_t* wbuf = flat_smem + warp * 2 * FLAT_PIECE;
+        const int npieces = (f.D + per_piece - 1) / per_piece;
+        for (int c = 0; c < npieces; ++c) {
+          uint8_t* buf = wbuf + (c & 1) * FLAT_PIECE;
+          if (c >= 2) {
+            if (lane == 0) bulk_wait_group_read<1>();  // the reduce-add of piece c - 2 has read this buffer
+            __syncwarp();
           }
-          const size_t oe = (size_t)row * f.D + 8 * (size_t)i, oc = (size_t)yl * f.D + 8 * (size_t)i;
-          if (fixed) {
-            // this warp owns dE_i (the accumulator starts at zero); dC_y is shared
+          const int e0 = c * per_piece + lane * per_lane;  // this lane's first element
+          const int n_el = min(per_piece, f.D - c * per_piece);
+          if (e0 < f.D) {
+            const size_t oe = (size_t)row * f.D + e0;
+            if (fixed) {
+              const uint2 ev = *reinterpret_cast<const uint2*>(E + (size_t)row * f.D + e0);
+              const uint2 cv = *reinterpret_cast<const uint2*>(C + (size_t)yl * f.D + e0);
+              const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&ev);
+              const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&cv);
+              unsigned long long qe[4], qc[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              f.accE[oe + j] = (unsigned long long)__float2ll_rn(ce[j] * scale);
-              atomicAdd(f.accC + oc + j, (unsigned long long)__float2ll_rn(ee[j] * scale));
+              for (int j = 0; j < 2; ++j) {
+                const float2 ef = __bfloat1622float2(e2[j]);
+                const float2 cf = __bfloat1622float2(c2[j]);
+                qc[2 * j] = (unsigned long long)__float2ll_rn(g * ef.x * scale);
+                qc[2 * j + 1] = (unsigned long long)__float2ll_rn(g * ef.y * scale);
+                qe[2 * j] = (unsigned long long)__float2ll_rn(g * cf.x * scale);
+                qe[2 * j + 1] = (unsigned long long)__float2ll_rn(g * cf.y * scale);
+              }
+              // this warp owns dE_i (the accumulator starts at zero)
+              ulonglong2* ae = reinterpret_cast<ulonglong2*>(f.accE + oe);
+              ae[0] = make_ulonglong2(qe[0], qe[1]);
+              ae[1] = make_ulonglong2(qe[2], qe[3]);
+              ulonglong2* sb = reinterpret_cast<ulonglong2*>(buf + lane * per_lane * 8);
+              sb[0] = make_ulonglong2(qc[0], qc[1]);
+              sb[1] = make_ulonglong2(qc[2], qc[3]);
+            } else {
+              const uint4 ev = *reinterpret_cast<const uint4*>(E + (size_t)row * f.D + e0);
+              const uint4 cv = *reinterpret_cast<const uint4*>(C + (size_t)yl * f.D + e0);
+              const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&ev);
+              const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&cv);
+              float ce[8], ee[8];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float2 cf = __bfloat1622float2(c2[j]);
+                const float2 ef = __bfloat1622float2(e2[j]);
+                ce[2 * j] = g * cf.x;
+                ce[2 * j + 1] = g * cf.y;
+                ee[2 * j] = g * ef.x;
+                ee[2 * j + 1] = g * ef.y;
+              }
+              float4* de = reinterpret_cast<float4*>(f.dE + oe);
+              float4 a0 = make_float4(ce[0], ce[1], ce[2], ce[3]), a1 = make_float4(ce[4], ce[5], ce[6], ce[7]);
+              if (f.accumulate) {
+                const float4 o0 = de[0], o1 = de[1];
+                a0 = make_float4(o0.x + a0.x, o0.y + a0.y, o0.z + a0.z, o0.w + a0.w);
+                a1 = make_float4(o1.x + a1.x, o1.y + a1.y, o1.z + a1.z, o1.w + a1.w);
+              }
+              de[0] = a0;
+              de[1] = a1;
+              float4* sb = reinterpret_cast<float4*>(buf + lane * per_lane * 4);
+              sb[0] = make_float4(ee[0], ee[1], ee[2], ee[3]);
+              sb[1] = make_float4(ee[4], ee[5], ee[6], ee[7]);
             }
-          } else {
-            float4* de = reinterpret_cast<float4*>(f.dE + oe);
-            float4 a0 = make_float4(ce[0], ce[1], ce[2], ce[3]), a1 = make_float4(ce[4], ce[5], ce[6], ce[7]);
-            if (f.accumulate) {
-              const float4 o0 = de[0], o1 = de[1];
-              a0 = make_float4(o0.x + a0.x, o0.y + a0.y, o0.z + a0.z, o0.w + a0.w);
-              a1 = make_float4(o1.x + a1.x, o1.y + a1.y, o1.z + a1.z, o1.w + a1.w);
-            }
-            de[0] = a0;
-            de[1] = a1;
-            red_add_v4(f.dC + oc, ee[0], ee[1], ee[2], ee[3]);
-            red_add_v4(f.dC + oc + 4, ee[4], ee[5], ee[6], ee[7]);
+          }
+          fence_proxy_async_smem();  // the generic-proxy writes above, seen by the TMA engine
+          __syncwarp();
+          if (lane == 0) {
+            const size_t oc = (size_t)yl * f.D + (size_t)c * per_piece;
+            if (fixed)
+              bulk_reduce_add_u64(f.accC + oc, buf, (uint32_t)n_el * 8u);
+            else
+              bulk_reduce_add_f32(f.dC + oc, buf, (uint32_t)n_el * 4u);
+            bulk_commit_group();
           }
         }
+        if (lane == 0) bulk_wait_group0();  // sources read and adds done before the CTA exits
+        __syncwarp();
       }
     }
   }
@@ -250,8 +302,11 @@ __global__ void __launch_bounds__(1024) flat_rows_kernel(const __nv_bfloat16* __
 
 cudaError_t launch_flat_rows(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
                              const FlatArgs& f, cudaStream_t stream) {
-  flat_rows_kernel<<<(f.N + 31) / 32, 1024, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E),
-                                                         reinterpret_cast<const __nv_bfloat16*>(C), y, lse, dloss, f);
+  cudaError_t e = cudaFuncSetAttribute(flat_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FLAT_SMEM);
+  if (e != cudaSuccess) return e;
+  flat_rows_kernel<<<(f.N + 31) / 32, 1024, FLAT_SMEM, stream>>>(reinterpret_cast<const __nv_bfloat16*>(E),
+                                                                 reinterpret_cast<const __nv_bfloat16*>(C), y, lse,
+                                                                 dloss, f);
   return cudaGetLastError();
 }
 
