@@ -35,6 +35,7 @@ METRIC = "CCE fwd+bwd tokens/s"
 UNIT = "tokens/s"
 IGN = -100
 BM, BN = 128, 256      # logit tile (token block x vocabulary tile)
+STRIPE_COLS = 4096     # vocabulary columns per stripe of the dense backward (the library's default)
 FU = (32, 32)          # the unit of skipped work: 32 tokens x 32 vocabulary entries (the filter itself
                        # drops single entries)
 
@@ -879,7 +880,7 @@ def run_trace_stripes(args, w):
         if k:
             ends.append((t[p, k - 1, 2] - t_first) / 1e3)
     flop = {0: 2.0 * 256 * 256 * w.D, 1: 2.0 * 256 * 256 * -(-w.N // 256) * 256,
-            2: 2.0 * 256 * 256 * min(2048, -(-w.V // 256) * 256)}
+            2: 2.0 * 256 * 256 * min(STRIPE_COLS, -(-w.V // 256) * 256)}
     peaks, _ = measured_peaks()
     pair_peak = float(peaks["bf16_tflops"]) * 1e12 / pairs
     out = {"mode": "trace-stripes", "workload": w.name, "N": w.N, "D": w.D, "V": w.V, "status": st,

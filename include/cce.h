@@ -185,13 +185,13 @@ typedef enum {
   CCE_BWD_PREPARED = 8,
   /* With filter_eps <= 0 (every entry kept: the exact gradient), run the
    * dense backward through stripes of the softmax gradient: the vocabulary
-   * is taken 2048 rows at a time; per stripe the logit tiles are recomputed
+   * is taken 4096 rows at a time; per stripe the logit tiles are recomputed
    * on chip and G = dloss (softmax - onehot) is stored in bf16 into one of
    * three stripe buffers in the workspace, then dC of the stripe's rows =
    * G^T E is formed with every token as the reduction dimension (each entry
    * written once) and dE += G C of the stripe (one bulk reduce-add per
    * 256 x 256 dE tile and stripe).  Only these stripes of G ever exist in
-   * global memory: 3 x min(N, 16384) x 2048 x 2 bytes (100 MB at N = 8192),
+   * global memory: 3 x min(N, 16384) x 4096 x 2 bytes (201 MB at N = 8192),
    * whatever V; tokens beyond 16384 are taken in further launches whose dC
    * contributions are added.  Far less fp32 reduction traffic than adding
    * every logit tile's partial products, so the tensor cores set the pace.

@@ -65,10 +65,13 @@ CCE_API cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, in
  * default 16384) bounds the tokens one launch takes (fewer tokens per launch
  * keep the stripe buffers, E and dE of a launch in L2, at the cost of adding
  * dC over more launches); dE_prefetch (0 or 1, default 0) asks for the dE
- * rows of each dE-tile task in L2 when the task starts.  Same results up to
- * fp32 summation order.  Process-wide.  Returns CCE_ERR_INVALID_ARG for other
- * values. */
-CCE_API cce_status_t cce_debug_set_stripe_params(int tokens_per_launch, int dE_prefetch);
+ * rows of each dE-tile task in L2 when the task starts; vtiles_per_stripe
+ * (0..32; 0 = the default 8) sets the stripe width in 256-wide vocabulary
+ * tiles (wider stripes: fewer reduce-adds into dE, larger stripe buffers).
+ * Same results up to fp32 summation order.  The workspace size depends on
+ * the stripe width: query cce_backward_workspace_size_ex after changing it.
+ * Process-wide.  Returns CCE_ERR_INVALID_ARG for other values. */
+CCE_API cce_status_t cce_debug_set_stripe_params(int tokens_per_launch, int dE_prefetch, int vtiles_per_stripe);
 
 /* L2 prefetch distance, in 64-wide K slices, of the fp32 dE / dC rows that
  * the filtered backward kernel's bulk reduce-adds add into: while loading

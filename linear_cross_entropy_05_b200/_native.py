@@ -87,7 +87,7 @@ def load_library():
         lib.cce_debug_set_kernel_events.restype = ctypes.c_int
         lib.cce_debug_set_prefetch.argtypes = [ctypes.c_int, ctypes.c_int]
         lib.cce_debug_set_prefetch.restype = ctypes.c_int
-        lib.cce_debug_set_stripe_params.argtypes = [ctypes.c_int, ctypes.c_int]
+        lib.cce_debug_set_stripe_params.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
         lib.cce_debug_set_stripe_params.restype = ctypes.c_int
         lib.cce_debug_set_l2_hints.argtypes = [ctypes.c_int]
         lib.cce_debug_set_l2_hints.restype = ctypes.c_int
@@ -281,10 +281,12 @@ def cce_debug_set_reduce_prefetch(slices: int) -> None:
     _check(load_library().cce_debug_set_reduce_prefetch(int(slices)), "cce_debug_set_reduce_prefetch")
 
 
-def cce_debug_set_stripe_params(tokens_per_launch: int = 0, dE_prefetch: int = 0) -> None:
+def cce_debug_set_stripe_params(tokens_per_launch: int = 0, dE_prefetch: int = 0, vtiles_per_stripe: int = 0) -> None:
     """Stripe backward knobs (A/B): tokens per launch (multiple of 256, <= 16384;
-    0 = default) and the L2 prefetch of dE rows for dE-tile tasks (0/1)."""
-    _check(load_library().cce_debug_set_stripe_params(int(tokens_per_launch), int(dE_prefetch)),
+    0 = default), the L2 prefetch of dE rows for dE-tile tasks (0/1) and the
+    stripe width in 256-wide vocabulary tiles (0 = default 8, at most 32)."""
+    _check(load_library().cce_debug_set_stripe_params(int(tokens_per_launch), int(dE_prefetch),
+                                                      int(vtiles_per_stripe)),
            "cce_debug_set_stripe_params")
 
 

@@ -18,7 +18,7 @@
 //   C  dE += G C[stripe rows]: one bulk reduce-add of a 256 x 256 dE tile per
 //      stripe instead of one per logit tile.
 // So the logits never exist in global memory: only nbuf stripes of G do,
-// O(N) bytes for a fixed stripe width (Vs = 2048: 12 KB per token with three
+// O(N) bytes for a fixed stripe width (Vs = 4096: 24 KB per token with three
 // buffers), against N x V x 4 bytes of fp32 logits.
 //
 // One persistent kernel runs all three kinds on clusters of two CTAs.  Tasks

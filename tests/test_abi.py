@@ -146,16 +146,16 @@ def test_backward_ex_workspace_and_flags(lib):
         assert cce_backward_workspace_size_ex(N, D, V, flags) == base + up(8 * N * D) + up(8 * V * D)
     assert cce_backward_workspace_size_ex(N, D, V, 4) == base   # accumulate alone: no extra workspace
     assert cce_backward_workspace_size_ex(N, D, V, 8) == base   # prepared: no extra workspace
-    # stripes: counters + three bf16 stripe buffers of 8192 tokens x 2048 columns
-    n_vt, n_s, n_dc = -(-V // 256), -(-V // 2048), -(-D // 256)
+    # stripes: counters + three bf16 stripe buffers of 8192 tokens x 4096 columns
+    n_vt, n_s, n_dc = -(-V // 256), -(-V // 4096), -(-D // 256)
     ctr = up(8 + 4 * (n_vt + n_s * 32 + n_s + 32 * n_dc))
-    assert cce_backward_workspace_size_ex(N, D, V, 16) == base + ctr + up(3 * 8192 * 2048 * 2)
+    assert cce_backward_workspace_size_ex(N, D, V, 16) == base + ctr + up(3 * 8192 * 4096 * 2)
     # deterministic with stripes: fixed stripe order, no int64 accumulators
-    assert cce_backward_workspace_size_ex(N, D, V, 17) == base + ctr + up(3 * 8192 * 2048 * 2)
+    assert cce_backward_workspace_size_ex(N, D, V, 17) == base + ctr + up(3 * 8192 * 4096 * 2)
     assert cce_backward_workspace_size_ex(N, D, V, 18) == 0     # bf16 outputs and stripes do not combine
     # token super-blocks of 16384 bound the stripe buffers whatever N
     big = cce_backward_workspace_size_ex(65536, 2048, 262144, 16) - cce_backward_workspace_size(65536, 2048, 262144)
-    assert big < 3 * 16384 * 2048 * 2 + (1 << 20)
+    assert big < 3 * 16384 * 4096 * 2 + (1 << 20)
     assert cce_backward_workspace_size_ex(N, D, V, 32) == 0     # unknown flag
     P = 1 << 20
     args = [P, P, P, P, P, 256, 256, 4096, -100, 0.0, 0, P, P, P, 1 << 30, 0]
@@ -197,3 +197,11 @@ def test_forward_schedule_knob_validates_on_the_host(lib):
     assert lib.cce_debug_set_forward_schedule(0, 0, 0, 8) == 1        # 8 stages do not fit
     assert lib.cce_debug_set_forward_schedule(37, 8, 3, 7) == 0
     assert lib.cce_debug_set_forward_schedule(0, 0, 0, 0) == 0        # back to the defaults
+
+
+def test_stripe_knob_validates_on_the_host(lib):
+    assert lib.cce_debug_set_stripe_params(100, 0, 0) == 1          # not a multiple of 256
+    assert lib.cce_debug_set_stripe_params(0, 2, 0) == 1
+    assert lib.cce_debug_set_stripe_params(0, 0, 33) == 1           # wider than 32 tiles
+    assert lib.cce_debug_set_stripe_params(4096, 1, 16) == 0
+    assert lib.cce_debug_set_stripe_params(0, 0, 0) == 0            # back to the defaults

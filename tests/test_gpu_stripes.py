@@ -15,7 +15,7 @@ from _gpu_helpers import GRAD_REL_FILTER_OFF, IGN, gpu_forward, rel_fro, to_dev
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    synth.GEMMA2_2B.with_sizes(N=700, V=8 * 256 * 4 + 77, D=264),    # 5 stripes: buffers reused, ragged tail
+    synth.GEMMA2_2B.with_sizes(N=700, V=16 * 256 * 4 + 77, D=264),   # 5 stripes: buffers reused, ragged tail
     synth.LLAMA3_8B.with_sizes(N=16384 + 300, V=3000, D=64),          # two launches (token super-blocks)
     synth.SMALL_LARGE_VOCAB.with_sizes(N=513, V=2048, D=896),         # exactly one stripe
 ]
@@ -73,3 +73,28 @@ def test_stripe_backward_dC_written_once_and_accumulation():
     assert float((aE - (pE + dE1)).abs().max()) <= 1e-5
     assert float((aC - (pC + dC1)).abs().max()) <= 1e-5
     assert L.read_status(ws)["status"] == 0
+
+
+@pytest.mark.parametrize("vt", [1, 4, 8, 12], ids=["1-tile", "4-tiles", "8-tiles", "12-tiles"])
+def test_stripe_width_knob_keeps_the_result(vt):
+    # narrower and ragged stripe widths (the default is 16 tiles of 256):
+    # more stripes, more buffer reuse, the same gradient
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=600, V=9 * 256 + 77, D=264)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    dloss = synth.random_dloss(19, w.N)
+    L.cce_debug_set_stripe_params(0, 0, vt)
+    try:
+        ws = L.Workspace()
+        dE, dC = L.backward(E, C, y, torch.from_numpy(lse).cuda(), torch.from_numpy(dloss).cuda(), 0.0, IGN,
+                            workspace=ws, stripes=True)
+        st = L.read_status(ws)
+    finally:
+        L.cce_debug_set_stripe_params(0, 0, 0)
+    assert st["status"] == 0 and st["flags"] == 0
+    rE, rC = _exact(inp, dloss)
+    assert rel_fro(dE.cpu().numpy(), rE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(dC.cpu().numpy(), rC) <= GRAD_REL_FILTER_OFF
