@@ -46,7 +46,7 @@ CCE_API void cce_debug_withhold_loads(int on);
 CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
 
 /* Schedule knobs of the forward logit/LSE kernels, for A/B measurement.
- * n_split (0..64; 0 = chosen per shape: the fewest splits that minimise the
+ * n_split (0..256; 0 = chosen per shape: the fewest splits that minimise the
  * most-loaded worker's vocabulary tiles) is the number of vocabulary ranges
  * per token block, i.e. of (max, sum) partials per token; group_m (>= 0; 0 =
  * chosen per shape, ~48 MB of E rows) is the number of token blocks per

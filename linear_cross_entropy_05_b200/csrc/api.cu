@@ -437,7 +437,7 @@ cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices) {
 }
 
 cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hints, int stages) {
-  if (n_split < 0 || n_split > 64 || group_m < 0 || l2_hints < 0 || l2_hints > 3) return CCE_ERR_INVALID_ARG;
+  if (n_split < 0 || n_split > 256 || group_m < 0 || l2_hints < 0 || l2_hints > 3) return CCE_ERR_INVALID_ARG;
   if (stages != 0 && stages != PAIR_STAGES && stages != PAIR_STAGES_MAX) return CCE_ERR_INVALID_ARG;
   g_fwd_split.store(n_split);
   g_fwd_group_m.store(group_m);

@@ -191,7 +191,7 @@ def test_shard_entry_points_validate_on_the_host(lib):
 
 
 def test_forward_schedule_knob_validates_on_the_host(lib):
-    assert lib.cce_debug_set_forward_schedule(65, 0, 0, 0) == 1       # more than 64 splits
+    assert lib.cce_debug_set_forward_schedule(257, 0, 0, 0) == 1      # more than 256 splits
     assert lib.cce_debug_set_forward_schedule(0, -1, 0, 0) == 1
     assert lib.cce_debug_set_forward_schedule(0, 0, 4, 0) == 1        # hint bits beyond E and C
     assert lib.cce_debug_set_forward_schedule(0, 0, 0, 8) == 1        # 8 stages do not fit
