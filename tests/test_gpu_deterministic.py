@@ -15,6 +15,9 @@ CASES = [
     (synth.GEMMA2_2B.with_sizes(N=1000, V=20000), EPS),
     (synth.LLAMA3_8B.with_sizes(N=700, V=9000), EPS),
     (synth.SMALL_LARGE_VOCAB.with_sizes(N=1500, V=20000), 0.0),
+    # flat blocks with D = 264: the flat-row kernel's last dC piece is a
+    # ragged 8-value tail (fp32 and int64 bulk reduce-adds)
+    (synth.GEMMA2_2B.with_sizes(N=500, V=6000, D=264), EPS),
 ]
 
 
@@ -54,7 +57,7 @@ def test_deterministic_backward_is_bitwise_reproducible_and_matches_oracle(w, ep
     assert rel_fro(a[1].cpu().numpy(), oC) <= GRAD_REL_FILTER_OFF
 
 
-@pytest.mark.parametrize("w,eps", CASES[:2], ids=["ragged", "gemma-shaped-filter"])
+@pytest.mark.parametrize("w,eps", CASES[:2] + CASES[4:], ids=["ragged", "gemma-shaped-filter", "flat-D264-filter"])
 def test_bf16_gradient_outputs(w, eps):
     import torch
     inp = synth.make_inputs(w)
