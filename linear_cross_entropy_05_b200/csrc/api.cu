@@ -143,8 +143,9 @@ long long max_worker_tiles(int n_mblk, int n_vtile, int s, int workers, int grou
 }
 
 // Splits per token block: the fewest that minimise the most-loaded worker's
-// vocabulary tiles (the kernel's duration).  Memoised per shape: the search
-// is O(64 * n_mblk * 64).
+// vocabulary tiles (the kernel's duration).  The load is counted exactly
+// while a candidate has at most 2^16 units (every workload here), else
+// estimated as ceil(units / workers) * ceil(n_vtile / s).  Memoised per shape.
 int choose_splits(int n_mblk, int n_vtile, int workers, int group_m) {
   static std::mutex mu;
   static std::map<std::array<int, 4>, int> memo;
@@ -158,7 +159,9 @@ int choose_splits(int n_mblk, int n_vtile, int workers, int group_m) {
   int best_s = 1;
   const int smax = std::min(64, n_vtile);
   for (int s = 1; s <= smax; ++s) {
-    const long long cost = max_worker_tiles(n_mblk, n_vtile, s, workers, group_m);
+    const long long units = (long long)n_mblk * s;
+    const long long cost = units <= (1ll << 16) ? max_worker_tiles(n_mblk, n_vtile, s, workers, group_m)
+                                                : ((units + workers - 1) / workers) * ((n_vtile + s - 1) / s);
     if (cost < best) {
       best = cost;
       best_s = s;
