@@ -111,14 +111,26 @@ CCE_API cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles
 
 /* Host-only view of the task order of the stripe backward (CCE_BWD_STRIPES)
  * for a launch of n_m2 256-token blocks, n_vtile 256-row vocabulary tiles,
- * n_dc 256-wide d-chunks, vt_per_s tiles per stripe and nbuf stripe
- * buffers: writes min(total + 1, max_tasks) task descriptors, four int32
- * each (kind: -1 end, 0 recompute-and-store G, 1 dC tile, 2 dE tile;
- * stripe; then (token block, vocabulary tile), (vocabulary tile, d-chunk)
- * or (token block, d-chunk)), into out (host memory; may be NULL) and
- * returns the number of tasks, or -1 for invalid sizes.  Runs no kernel. */
-CCE_API int64_t cce_debug_stripe_schedule(int n_m2, int n_vtile, int n_dc, int vt_per_s, int nbuf, int32_t* out,
-                                          int64_t max_tasks);
+ * n_dc 256-wide d-chunks, vt_per_s tiles per stripe, nbuf stripe buffers
+ * and the order of cce_debug_set_stripe_order (order, group_m2, lag):
+ * writes min(total + 1, max_tasks) task descriptors, four int32 each (kind:
+ * -1 end, 0 recompute-and-store G, 1 dC tile, 2 dE tile; stripe; then
+ * (token block, vocabulary tile), (vocabulary tile, d-chunk) or (token
+ * block, d-chunk)), into out (host memory; may be NULL) and returns the
+ * number of tasks, or -1 for invalid arguments.  Runs no kernel. */
+CCE_API int64_t cce_debug_stripe_schedule(int n_m2, int n_vtile, int n_dc, int vt_per_s, int nbuf, int order,
+                                          int group_m2, int lag, int32_t* out, int64_t max_tasks);
+
+/* Task order of the stripe backward, for A/B measurement.  order 0 (the
+ * default): recompute tasks of stripe s, then the dC and dE tasks of stripe
+ * s - 1.  order 1: per stripe, the token blocks in groups of group_m2; each
+ * group's recompute tasks are followed by the dE tasks of the group lag
+ * groups earlier (their G rows still in L2), then the last groups' dE tasks
+ * and the stripe's dC tasks.  Same results up to fp32 summation order (bit
+ * for bit in the deterministic mode).  Process-wide.  Returns
+ * CCE_ERR_INVALID_ARG unless order is 0 or 1 and group_m2, lag are in
+ * [1, 64]. */
+CCE_API cce_status_t cce_debug_set_stripe_order(int order, int group_m2, int lag);
 
 /* Selects the forward logit/LSE kernel: 1 = CTA pairs (two SMs per 256 x 256
  * logit tile through tcgen05 cta_group::2, two thirds of the operand traffic

@@ -95,8 +95,10 @@ def load_library():
         lib.cce_debug_set_forward_schedule.restype = ctypes.c_int
         lib.cce_debug_set_reduce_prefetch.argtypes = [ctypes.c_int]
         lib.cce_debug_set_reduce_prefetch.restype = ctypes.c_int
-        lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 5 + [c_vp, c_i64]
+        lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 8 + [c_vp, c_i64]
         lib.cce_debug_stripe_schedule.restype = c_i64
+        lib.cce_debug_set_stripe_order.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.cce_debug_set_stripe_order.restype = ctypes.c_int
         lib.cce_debug_set_backward_trace.argtypes = [c_vp, c_i64]
         lib.cce_debug_set_backward_trace.restype = ctypes.c_int
         _lib = lib
@@ -262,17 +264,26 @@ def cce_debug_set_backward_trace(trace: int, tiles_per_cta: int) -> None:
            "cce_debug_set_backward_trace")
 
 
-def cce_debug_stripe_schedule(n_m2: int, n_vtile: int, n_dc: int, vt_per_s: int, nbuf: int):
+def cce_debug_stripe_schedule(n_m2: int, n_vtile: int, n_dc: int, vt_per_s: int, nbuf: int, order: int = 0,
+                              group_m2: int = 4, lag: int = 2):
     """Task order of the stripe backward (host-side decode, no kernel):
     an int32 array [tasks + 1, 4] of (kind, stripe, a, b); kind -1 ends it."""
     import numpy as np
     lib = load_library()
-    total = int(lib.cce_debug_stripe_schedule(n_m2, n_vtile, n_dc, vt_per_s, nbuf, None, 0))
+    total = int(lib.cce_debug_stripe_schedule(n_m2, n_vtile, n_dc, vt_per_s, nbuf, order, group_m2, lag, None, 0))
     if total < 0:
         raise CCEError(1, "cce_debug_stripe_schedule: invalid sizes")
     out = np.zeros((total + 1, 4), dtype=np.int32)
-    lib.cce_debug_stripe_schedule(n_m2, n_vtile, n_dc, vt_per_s, nbuf, out.ctypes.data, total + 1)
+    lib.cce_debug_stripe_schedule(n_m2, n_vtile, n_dc, vt_per_s, nbuf, order, group_m2, lag, out.ctypes.data,
+                                  total + 1)
     return out
+
+
+def cce_debug_set_stripe_order(order: int = 0, group_m2: int = 4, lag: int = 2) -> None:
+    """Stripe backward task order (A/B): 0 stripe-major, 1 interleaved with
+    groups of group_m2 token blocks and the dE tasks lag groups behind."""
+    _check(load_library().cce_debug_set_stripe_order(int(order), int(group_m2), int(lag)),
+           "cce_debug_set_stripe_order")
 
 
 def cce_debug_set_reduce_prefetch(slices: int) -> None:

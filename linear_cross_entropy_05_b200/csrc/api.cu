@@ -256,6 +256,9 @@ constexpr int kStripeBuffers = 3;
 std::atomic<int> g_stripe_m2{kStripeMaxM2};  // token blocks per launch actually used (A/B knob)
 std::atomic<int> g_stripe_dE_pf{0};          // L2 prefetch of the dE rows of dE-tile tasks (measured: no gain)
 std::atomic<int> g_stripe_vt{kStripeVtiles};  // vocabulary tiles per stripe (A/B knob)
+std::atomic<int> g_stripe_order{0};  // task order: 0 stripe-major, 1 interleaved (A/B knob)
+std::atomic<int> g_stripe_gm{4};     // interleaved order: token blocks per group
+std::atomic<int> g_stripe_lag{2};    // interleaved order: groups between A and C tasks
 
 struct StripeLayout {
   StripePlan p;          // of a full super-block
@@ -274,6 +277,9 @@ StripeLayout plan_stripes(int64_t N, int64_t D, int64_t V, size_t base) {
   L.p.vt_per_s = std::min(L.p.n_vtile, g_stripe_vt.load());
   L.p.n_s = (L.p.n_vtile + L.p.vt_per_s - 1) / L.p.vt_per_s;
   L.p.nbuf = std::min(L.p.n_s, kStripeBuffers);
+  L.p.order = g_stripe_order.load();
+  L.p.gm = g_stripe_gm.load();
+  L.p.lag = g_stripe_lag.load();
   L.n_sb = (n_m2_total + L.p.n_m2 - 1) / L.p.n_m2;
   L.Ns_pad = L.p.n_m2 * 256;
   L.Vs = L.p.vt_per_s * BN;
@@ -459,6 +465,14 @@ cce_status_t cce_debug_set_stripe_params(int tokens_per_launch, int dE_prefetch,
   return CCE_OK;
 }
 
+cce_status_t cce_debug_set_stripe_order(int order, int group_m2, int lag) {
+  if (order < 0 || order > 1 || group_m2 <= 0 || group_m2 > 64 || lag <= 0 || lag > 64) return CCE_ERR_INVALID_ARG;
+  g_stripe_order.store(order);
+  g_stripe_gm.store(group_m2);
+  g_stripe_lag.store(lag);
+  return CCE_OK;
+}
+
 cce_status_t cce_debug_set_reduce_prefetch(int slices) {
   if (slices < 0 || slices > 64) return CCE_ERR_INVALID_ARG;
   g_bwd_red_pf.store(slices);
@@ -478,9 +492,10 @@ cce_status_t cce_debug_set_backward_trace(uint64_t* trace, int64_t tiles_per_cta
   return CCE_OK;
 }
 
-int64_t cce_debug_stripe_schedule(int n_m2, int n_vtile, int n_dc, int vt_per_s, int nbuf, int32_t* out,
-                                  int64_t max_tasks) {
+int64_t cce_debug_stripe_schedule(int n_m2, int n_vtile, int n_dc, int vt_per_s, int nbuf, int order, int group_m2,
+                                  int lag, int32_t* out, int64_t max_tasks) {
   if (n_m2 <= 0 || n_vtile <= 0 || n_dc <= 0 || vt_per_s <= 0 || nbuf <= 0) return -1;
+  if (order < 0 || order > 1 || group_m2 <= 0 || lag <= 0) return -1;
   StripePlan p{};
   p.n_m2 = n_m2;
   p.n_vtile = n_vtile;
@@ -488,6 +503,9 @@ int64_t cce_debug_stripe_schedule(int n_m2, int n_vtile, int n_dc, int vt_per_s,
   p.vt_per_s = vt_per_s;
   p.n_s = (n_vtile + vt_per_s - 1) / vt_per_s;
   p.nbuf = std::min(nbuf, p.n_s);
+  p.order = order;
+  p.gm = group_m2;
+  p.lag = lag;
   const long long total = stripe_total(p);
   if (out) {
     for (long long t = 0; t < total + 1 && t < max_tasks; ++t) {

@@ -170,6 +170,9 @@ struct StripePlan {
   int vt_per_s;  // vocabulary tiles per stripe
   int n_s;       // stripes
   int nbuf;      // stripe buffers (<= n_s)
+  int order;     // 0: stripe-major (above); 1: interleaved (below)
+  int gm;        // order 1: token blocks per group
+  int lag;       // order 1: groups between a group's A tasks and its C tasks (>= 1)
 };
 enum StripeTask : int { TASK_END = -1, TASK_A = 0, TASK_B = 1, TASK_C = 2 };
 struct StripeTaskDesc {
@@ -206,10 +209,67 @@ __host__ __device__ inline StripeTaskDesc stripe_BC(const StripePlan& p, int s, 
   return StripeTaskDesc{TASK_C, s, (int)(k / p.n_dc), (int)(k % p.n_dc)};
 }
 
+// Interleaved order (order 1): each stripe is one run of tasks.  Its token
+// blocks are taken gm at a time; a group's A tasks (vocabulary tile outer,
+// token block inner, so the pairs running together share a C tile) are
+// followed by the C tasks of the group `lag` groups earlier, whose G rows
+// were written recently and are still in L2; the C tasks of the last `lag`
+// groups and then the stripe's B tasks close the run.  Every task still
+// comes after the tasks it reads: C(s, m2) after all A(s, m2, .), B(s, vt)
+// after all A(s, ., vt), A(s) after the B and C tasks of earlier stripes.
+__host__ __device__ inline int stripe_group_size(const StripePlan& p, int grp) {
+  const int r = p.n_m2 - grp * p.gm;
+  return r < p.gm ? r : p.gm;
+}
+__host__ __device__ inline StripeTaskDesc stripe_local_interleaved(const StripePlan& p, int s, long long k) {
+  const int T = stripe_tiles(p, s), nd = p.n_dc;
+  const int ng = (p.n_m2 + p.gm - 1) / p.gm;
+  const int L = p.lag < ng ? p.lag : ng;
+  const int vt0 = s * p.vt_per_s;
+  long long off = 0;
+  for (int grp = 0; grp < ng; ++grp) {
+    const int mc = stripe_group_size(p, grp);
+    const long long nA = (long long)T * mc;
+    if (k < off + nA) {
+      const long long i = k - off;
+      return StripeTaskDesc{TASK_A, s, grp * p.gm + (int)(i % mc), vt0 + (int)(i / mc)};
+    }
+    off += nA;
+    if (grp >= L) {
+      const int cg = grp - L;
+      const long long nC = (long long)stripe_group_size(p, cg) * nd;
+      if (k < off + nC) {
+        const long long i = k - off;
+        return StripeTaskDesc{TASK_C, s, cg * p.gm + (int)(i / nd), (int)(i % nd)};
+      }
+      off += nC;
+    }
+  }
+  for (int cg = ng - L; cg < ng; ++cg) {
+    const long long nC = (long long)stripe_group_size(p, cg) * nd;
+    if (k < off + nC) {
+      const long long i = k - off;
+      return StripeTaskDesc{TASK_C, s, cg * p.gm + (int)(i / nd), (int)(i % nd)};
+    }
+    off += nC;
+  }
+  const long long i = k - off;
+  return StripeTaskDesc{TASK_B, s, vt0 + (int)(i / nd), (int)(i % nd)};
+}
+
 // Task t of the global order.  Every stripe but the last has the same task
 // counts, so the position is found without walking the stripes.
 __host__ __device__ inline StripeTaskDesc stripe_decode(const StripePlan& p, long long t) {
   if (t < 0) return StripeTaskDesc{TASK_END, 0, 0, 0};
+  if (p.order == 1) {
+    const long long per = stripe_nA(p, 0) + stripe_nC(p) + stripe_nB(p, 0);
+    const long long full = (long long)(p.n_s - 1) * per;
+    if (t < full) return stripe_local_interleaved(p, (int)(t / per), t % per);
+    t -= full;
+    const int L = p.n_s - 1;
+    if (t < stripe_nA(p, L) + stripe_nC(p) + stripe_nB(p, L)) return stripe_local_interleaved(p, L, t);
+    return StripeTaskDesc{TASK_END, 0, 0, 0};
+  }
   const long long nA = stripe_nA(p, 0);
   if (p.n_s == 1) {
     if (t < nA) return stripe_A(p, 0, t);

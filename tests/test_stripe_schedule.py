@@ -32,10 +32,14 @@ PLANS = [
 ]
 
 
+ORDERS = [(0, 4, 2), (1, 4, 2), (1, 1, 1), (1, 3, 5), (1, 64, 1)]   # (order, token blocks per group, lag)
+
+
+@pytest.mark.parametrize("order", ORDERS, ids=[f"order{o}-g{g}-lag{l}" for o, g, l in ORDERS])
 @pytest.mark.parametrize("plan", PLANS, ids=[str(p) for p in PLANS])
-def test_stripe_schedule_is_complete_and_ordered(lib, plan):
+def test_stripe_schedule_is_complete_and_ordered(lib, plan, order):
     n_m2, n_vt, n_dc, vps, nbuf = plan
-    tasks = lib.cce_debug_stripe_schedule(*plan)
+    tasks = lib.cce_debug_stripe_schedule(*plan, *order)
     n_s = -(-n_vt // vps)
     nbuf = min(nbuf, n_s)
     assert tasks[-1][0] == END
@@ -68,9 +72,22 @@ def test_stripe_schedule_is_complete_and_ordered(lib, plan):
             for m2 in range(n_m2):
                 for dc in range(n_dc):
                     assert pos[(C, s0, m2, dc)] < i
+    # the deterministic mode sums each dE tile in stripe order
+    for s in range(1, n_s):
+        for m2 in range(n_m2):
+            for dc in range(n_dc):
+                assert pos[(C, s - 1, m2, dc)] < pos[(C, s, m2, dc)]
 
 
 def test_stripe_schedule_rejects_bad_sizes(lib):
     from linear_cross_entropy_05_b200._native import CCEError
     with pytest.raises(CCEError):
         lib.cce_debug_stripe_schedule(0, 4, 1, 8, 3)
+    with pytest.raises(CCEError):
+        lib.cce_debug_stripe_schedule(4, 4, 1, 8, 3, 1, 4, 0)     # lag 0: a dE task right after its inputs
+    from linear_cross_entropy_05_b200 import _native
+    lib_c = _native.load_library()
+    assert lib_c.cce_debug_set_stripe_order(2, 4, 2) == 1
+    assert lib_c.cce_debug_set_stripe_order(1, 0, 2) == 1
+    assert lib_c.cce_debug_set_stripe_order(1, 4, 2) == 0
+    assert lib_c.cce_debug_set_stripe_order(0, 4, 2) == 0
