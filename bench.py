@@ -676,7 +676,8 @@ def run_gpu(args, w):
             # tiles, live units' contractions) over the step time, against the
             # burst peak; pruned units are not counted
             "pct_bf16_peak_executed": executed_flop / (step_ms * 1e-3) / 1e12 / peak,
-            "filter_unit": list(FU),
+            "filter_unit": [1, 1],          # entries are kept or dropped one by one
+            "skip_unit": list(FU),          # live / dead / pruned counts are of these units
             "live_unit_frac": live / max(1, live + dead + pruned),
             "extra_hbm_bytes": int(extra_hbm),
             "materialised_logits_fp32_bytes": N * V * 4,
@@ -685,8 +686,7 @@ def run_gpu(args, w):
                     "weights_resident": {"value": e2e_resident, "unit": UNIT,
                                          "h2d_bytes_per_step": int(h2d - C_h.numel() * 2),
                                          "inputs_copied": "E, y, dloss every step; C uploaded once"}},
-            # our kernels per step: fwd_lse + fwd_finalize, bwd_kernel, and with
-            # the filter on the four pre-pass kernels (cnorm, blocks, scan, scatter)
+            # our kernels per step (launches_per_step lists them)
             "gpu_launches": launches_per_step(eps, args.deterministic or args.bf16_grads) * K,
             "clocks": clk,
             "cpu_baseline": cpu,
