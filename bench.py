@@ -259,6 +259,12 @@ def launches_per_step(eps: float, fixed_point: bool) -> int:
     return n
 
 
+def scale_bf16_bits(bits, scale):
+    """bf16 bit patterns times `scale`, rounded back to bf16."""
+    from linear_cross_entropy_05_b200 import synth
+    return synth.round_to_bf16_bits((bits.astype(np.uint32) << 16).view(np.float32) * np.float32(scale))
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -407,6 +413,10 @@ def run_gpu(args, w):
     t0 = time.perf_counter()
     inp = synth.make_inputs(w)
     log(f"[rank {rank}] generated {w.name} in {time.perf_counter() - t0:.1f} s")
+    if args.e_scale:
+        # stress variant (not one of the workloads): E scaled so that the
+        # softmax is peaky and token blocks are no longer flat
+        inp["E"] = scale_bf16_bits(inp["E"], args.e_scale)
     N, D, V = w.N, w.D, w.V
     E = torch.from_numpy(inp["E"].view(np.int16)).view(torch.bfloat16).to(dev)
     C = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).to(dev)
@@ -422,9 +432,12 @@ def run_gpu(args, w):
     stream = torch.cuda.current_stream()
     ws_b.get(L.cce_backward_workspace_size_ex(
         N, D, V, (L.CCE_BWD_DETERMINISTIC if args.deterministic else 0) |
-        (L.CCE_BWD_BF16_GRADS if args.bf16_grads else 0)))   # allocated before the side stream uses it
+        (L.CCE_BWD_BF16_GRADS if args.bf16_grads else 0) |
+        (L.CCE_BWD_STRIPES if args.bwd_stripes else 0)))   # allocated before the side stream uses it
 
     gkw = dict(deterministic=args.deterministic, bf16_grads=args.bf16_grads)
+    if args.bwd_stripes:
+        gkw["stripes"] = True
     if args.bf16_grads:
         dE = torch.empty((N, D), device=dev, dtype=torch.bfloat16)
         dC = torch.empty((V, D), device=dev, dtype=torch.bfloat16)
@@ -437,7 +450,8 @@ def run_gpu(args, w):
     # unvisited vocabulary tiles alone); the bf16 outputs are written anyway.
     overlap_zero = not (args.bf16_grads or args.no_overlap_zero)
     # (the classifier bound is used only by the filter and the fixed-point modes)
-    prepare = not args.no_prepare and (eps > 0 or args.deterministic or args.bf16_grads)
+    prepare = (not args.no_prepare and not args.bwd_stripes and
+               (eps > 0 or args.deterministic or args.bf16_grads))
     side_stream = torch.cuda.Stream(device=dev)
     side_done = torch.cuda.Event()
 
@@ -657,6 +671,9 @@ def run_gpu(args, w):
                            l2_prefetch_slices=list(args.prefetch) if args.prefetch else [0, 0],
                            reduce_prefetch_slices=args.reduce_prefetch, l2_hints=bool(args.l2_hints),
                            forward_splits=fwd_splits,
+                           e_scale=args.e_scale,
+                           backward_path=("stripes (CCE_BWD_STRIPES)" if args.bwd_stripes else
+                                          "pre-pass, flat rows, tile kernel" if eps > 0 else "stripes"),
                            forward_schedule=list(args.fwd_schedule) if args.fwd_schedule else None),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
@@ -1065,6 +1082,11 @@ def main(argv=None):
                     help="forward schedule (A/B): vocabulary splits per token block and token blocks per raster "
                          "group (0 = chosen per shape), L2 hints of the pair kernel (bit 0: E evict_last, bit 1: C "
                          "evict_first), its operand stages (0 = default 7, or 6)")
+    ap.add_argument("--e-scale", type=float, default=None, metavar="F",
+                    help="stress variant, not one of the workloads: E multiplied by F (a peaky softmax whose token "
+                         "blocks are not flat)")
+    ap.add_argument("--bwd-stripes", action="store_true",
+                    help="take the backward through the stripe kernel (CCE_BWD_STRIPES) also with the filter on")
     ap.add_argument("--trace", action="store_true",
                     help="per-tile timeline of one backward launch (recompute wait, gradient tile, contraction)")
     ap.add_argument("--dense-trace", action="store_true",

@@ -139,10 +139,13 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     accumulate=True adds them to the tensors given in `out` (required)
     instead of overwriting them.  prepared=True: backward_prepare already ran
     on `workspace` for this C.  stripes (default: on when filter_eps <= 0
-    and not bf16_grads): the dense backward through softmax-gradient stripes
-    (CCE_BWD_STRIPES), which needs a larger workspace (about 12 KB per
-    token, at most ~200 MB); with deterministic=True it sums in a fixed
-    order instead of using the int64 fixed-point accumulators."""
+    and not bf16_grads): the backward through softmax-gradient stripes
+    (CCE_BWD_STRIPES), which needs a larger workspace (about 24 KB per
+    token, at most ~400 MB); with deterministic=True it sums in a fixed
+    order instead of using the int64 fixed-point accumulators.  With
+    filter_eps > 0 it applies the same entry filter but skips no work: the
+    faster choice only when a large share of the gradient is above the
+    threshold (a peaky, non-flat softmax)."""
     torch = _torch()
     _check_inputs(E, C, y)
     N, D = E.shape

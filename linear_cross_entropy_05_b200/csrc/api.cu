@@ -580,6 +580,7 @@ cce_status_t backward_stripes(const void* E, const void* C, void* dE, void* dC, 
   sa.trace = a.trace;
   sa.trace_cap = a.trace_cap;
   sa.dE_prefetch = g_stripe_dE_pf.load();
+  sa.filter_eps = a.filter_eps;
   const int grid = sms & ~1;
   const int n_m2_total = (a.N + 255) / 256;
   const int m2_per_launch = std::max(1, std::min(L.p.n_m2, g_stripe_m2.load()));
@@ -610,8 +611,6 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   const bool fixed = uses_fixed_point(flags);
   const bool bf16_out = (flags & CCE_BWD_BF16_GRADS) != 0;
   const bool accumulate = (flags & CCE_BWD_ACCUMULATE) != 0;
-  // deterministic through the stripe kernel's fixed reduction order: filter off only
-  if ((flags & CCE_BWD_STRIPES) && (flags & CCE_BWD_DETERMINISTIC) && filter_eps > 0.f) return CCE_ERR_INVALID_ARG;
   if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
   if (!(filter_eps == filter_eps)) return CCE_ERR_INVALID_ARG;  // NaN
   if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(lse, 4) || !aligned(dloss, 4) ||
@@ -652,7 +651,7 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     // with the filter on only visited vocabulary tiles are cleared, after the pre-pass
     if (!filter_on && cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
   } else if (!accumulate) {
-    const bool stripes = (flags & CCE_BWD_STRIPES) && !(filter_eps > 0.f);
+    const bool stripes = (flags & CCE_BWD_STRIPES) != 0;
     if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
     // (the stripe path writes every entry of dC)
     if (!stripes && cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess)
@@ -690,6 +689,11 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.trace = g_bwd_trace.load();
   a.trace_cap = g_bwd_trace_cap.load();
 
+  // the stripe kernel applies the entry filter while it forms G and needs no
+  // pre-pass (it visits every tile)
+  if ((flags & CCE_BWD_STRIPES) && !fixed)
+    return backward_stripes(E, C, dE, dC, bp, a, accumulate, (flags & CCE_BWD_DETERMINISTIC) != 0, di.sms, ws,
+                            stream);
   if (filter_on || fixed) {
     PrepArgs pp;
     pp.N = (int)N;
@@ -735,9 +739,6 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
       if (launch_flat_rows(E, C, y, lse, dloss, fa, stream) != cudaSuccess) return CCE_ERR_CUDA;
     }
   }
-  if ((flags & CCE_BWD_STRIPES) && !filter_on && !fixed)
-    return backward_stripes(E, C, dE, dC, bp, a, accumulate, (flags & CCE_BWD_DETERMINISTIC) != 0, di.sms, ws,
-                            stream);
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   if (launch_bwd(tmE, tmC, tmCq, tmdE, tmdC, a, grid, g_bwd_variant.load(), stream) != cudaSuccess) return CCE_ERR_CUDA;

@@ -460,6 +460,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
               const float p = ex2_approx(fmaf(x[j + q], LOG2E, -lse2));
               float d = (col == ycol) ? p - 1.f : p;
               d = (valid && col < ncols) ? d : 0.f;
+              // the entry filter (eps <= 0 keeps every entry)
+              d = fabsf(d) >= a.filter_eps ? d : 0.f;
               g2[q] = dl * d;
             }
             pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);

@@ -336,6 +336,7 @@ struct StripeArgs {
   unsigned long long* status;
   unsigned long long wait_limit_ns;
   int withhold_loads;    // test hook: the TMA producers issue nothing
+  float filter_eps;      // > 0: entries of G with |P - onehot| below it are zeroed
 };
 
 // Fixed-point exponent s: contributions are stored as round(x * 2^s) in int64.
