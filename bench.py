@@ -239,16 +239,19 @@ class ClockSampler:
 # helpers
 # ---------------------------------------------------------------------------
 
-def launches_per_step(eps: float, fixed_point: bool) -> int:
+def launches_per_step(eps: float, fixed_point: bool, row_max: bool = False, stripes: bool = False) -> int:
     """Kernels of this library launched by one forward + backward call pair:
     forward logit/LSE kernel and finalize; backward tile kernel (or the
-    stripe kernel, one launch up to 16384 tokens); the norm pass (classifier
-    and token norms) when the filter or the fixed-point mode needs it; with
-    the filter on the pre-pass (blocks, scan) and the flat-row kernel; the
-    dloss maximum and two conversion passes in fixed point; and with both,
-    the clearing of the dC accumulator rows that can receive a gradient."""
+    stripe kernel, one launch up to 16384 tokens, and nothing else); the
+    norm pass (classifier and token norms) when the filter (without the
+    forward's row maxima) or the fixed-point mode needs it; with the filter
+    on the pre-pass (blocks, totals) and the flat-row kernel; the dloss
+    maximum and two conversion passes in fixed point; and with both, the
+    clearing of the dC accumulator rows that can receive a gradient."""
     n = 2 + 1
-    if eps > 0 or fixed_point:
+    if stripes and not fixed_point:
+        return n
+    if fixed_point or (eps > 0 and not row_max):
         n += 2
     if eps > 0:
         n += 3
@@ -450,8 +453,13 @@ def run_gpu(args, w):
     # unvisited vocabulary tiles alone); the bf16 outputs are written anyway.
     overlap_zero = not (args.bf16_grads or args.no_overlap_zero)
     # (the classifier bound is used only by the filter and the fixed-point modes)
+    # the forward's row maxima bound the logits for the filter's pre-pass
+    # (CCE_BWD_ROW_MAX); then only the fixed-point modes need max_v |C_v|
+    use_rows = eps > 0 and not args.bwd_stripes and not args.no_row_max
+    row_max = torch.empty(N, device=dev) if use_rows else None
+    fixed_mode = args.deterministic or args.bf16_grads
     prepare = (not args.no_prepare and not args.bwd_stripes and
-               (eps > 0 or args.deterministic or args.bf16_grads))
+               (fixed_mode or (eps > 0 and not use_rows)))
     side_stream = torch.cuda.Stream(device=dev)
     side_done = torch.cuda.Event()
 
@@ -467,11 +475,11 @@ def run_gpu(args, w):
                     dE.zero_()
                     dC.zero_()
                 side_done.record(side_stream)
-        L.forward(Eb, Cb, yb, IGN, workspace=ws_f, out=(loss, lse))
+        L.forward(Eb, Cb, yb, IGN, workspace=ws_f, out=(loss, lse), row_max=row_max)
         if overlap_zero or prepare:
             stream.wait_event(side_done)
         L.backward(Eb, Cb, yb, lse, dlb, eps, IGN, workspace=ws_b, out=(dE, dC), accumulate=overlap_zero,
-                   prepared=prepare, **gkw)
+                   prepared=prepare, row_max=row_max, **gkw)
 
     def step():
         fwd_bwd(E, C, y, dloss)
@@ -667,7 +675,10 @@ def run_gpu(args, w):
                            grad_zeroing=("side stream during the forward; backward accumulates (CCE_BWD_ACCUMULATE)"
                                          if overlap_zero else "inside the backward call"),
                            classifier_norm=("cce_backward_prepare on the side stream during the forward"
-                                            if prepare else "inside the backward call"),
+                                            if prepare else
+                                            "not needed (the forward's row maxima bound the logits)"
+                                            if use_rows and not fixed_mode else "inside the backward call"),
+                           row_max=use_rows,
                            l2_prefetch_slices=list(args.prefetch) if args.prefetch else [0, 0],
                            reduce_prefetch_slices=args.reduce_prefetch, l2_hints=bool(args.l2_hints),
                            forward_splits=fwd_splits,
@@ -704,7 +715,8 @@ def run_gpu(args, w):
                                          "h2d_bytes_per_step": int(h2d - C_h.numel() * 2),
                                          "inputs_copied": "E, y, dloss every step; C uploaded once"}},
             # our kernels per step (launches_per_step lists them)
-            "gpu_launches": launches_per_step(eps, args.deterministic or args.bf16_grads) * K,
+            "gpu_launches": launches_per_step(eps, args.deterministic or args.bf16_grads, use_rows,
+                                              args.bwd_stripes) * K,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -1085,6 +1097,9 @@ def main(argv=None):
     ap.add_argument("--e-scale", type=float, default=None, metavar="F",
                     help="stress variant, not one of the workloads: E multiplied by F (a peaky softmax whose token "
                          "blocks are not flat)")
+    ap.add_argument("--no-row-max", action="store_true",
+                    help="let the filter's pre-pass bound the logits by Cauchy-Schwarz instead of the forward's "
+                         "per-token maximum logits (A/B)")
     ap.add_argument("--bwd-stripes", action="store_true",
                     help="take the backward through the stripe kernel (CCE_BWD_STRIPES) also with the filter on")
     ap.add_argument("--trace", action="store_true",

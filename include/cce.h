@@ -210,8 +210,36 @@ typedef enum {
    * is not available with CCE_BWD_BF16_GRADS (the workspace size query
    * returns 0).  Needs the workspace of cce_backward_workspace_size_ex with
    * this flag. */
-  CCE_BWD_STRIPES = 16
+  CCE_BWD_STRIPES = 16,
+  /* With filter_eps > 0: cce_backward_prepare_rows has stored each token's
+   * largest logit max_v E_i . C_v (from cce_forward_ex) in this workspace for
+   * the same E, C and N.  The pre-pass then proves token blocks flat with
+   * that exact maximum instead of the Cauchy-Schwarz bound |E_i| max_v |C_v|
+   * (which can be far looser), and skips both norm passes unless the
+   * fixed-point modes need them.  The stored maxima serve one backward call;
+   * without a fresh cce_backward_prepare_rows the pre-pass treats every
+   * block as not flat (the exact, slower path).  Same result as without the
+   * flag.  Ignored with CCE_BWD_STRIPES or filter_eps <= 0.  No extra
+   * workspace. */
+  CCE_BWD_ROW_MAX = 32
 } cce_backward_flags_t;
+
+/* Forward pass that also writes row_max [N] fp32 (device; may be NULL): each
+ * token's largest logit max_v E_i . C_v, the maximum the log-sum-exp is
+ * taken around (also for ignored rows; NaN where loss is NaN after a wait
+ * gave up).  Otherwise the same as cce_forward. */
+CCE_API cce_status_t cce_forward_ex(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
+                                    int64_t ignore_index, float* loss, float* lse, float* row_max, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* Stores row_max [N] (device, fp32: each token's largest logit, from
+ * cce_forward_ex on the same E and C) in the backward workspace for the next
+ * cce_backward_ex with CCE_BWD_ROW_MAX (an asynchronous 4N-byte copy on
+ * stream).  Workspace as for cce_backward_workspace_size(N, D, V).  Returns
+ * CCE_ERR_INVALID_ARG / CCE_ERR_MISALIGNED / CCE_ERR_WORKSPACE_TOO_SMALL on
+ * the host. */
+CCE_API cce_status_t cce_backward_prepare_rows(const float* row_max, int64_t N, int64_t D, int64_t V,
+                                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* The part of the backward's pre-pass that depends on the classifier alone:
  * max_v |C_v| (one read of all of C, about 0.17 ms for a 256000 x 2304 bf16

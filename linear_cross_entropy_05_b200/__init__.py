@@ -23,7 +23,7 @@ from typing import Optional, Tuple
 
 from . import _native
 from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCE_BWD_PREPARED,
-                      CCE_BWD_STRIPES, CCEError, cce_debug_stripe_schedule, cce_debug_set_reduce_prefetch,
+                      CCE_BWD_STRIPES, CCE_BWD_ROW_MAX, CCEError, cce_forward_ex, cce_backward_prepare_rows, cce_debug_stripe_schedule, cce_debug_set_reduce_prefetch,
                       cce_debug_set_stripe_params, cce_debug_set_l2_hints, cce_debug_set_forward_schedule,
                       cce_debug_set_stripe_order,
                       cce_backward, cce_backward_ex, cce_backward_prepare,
@@ -51,6 +51,7 @@ __all__ = [
     "cce_debug_set_backward_variant", "cce_debug_set_backward_trace", "cce_debug_set_prefetch",
     "load_library",
     "forward", "backward", "read_status", "linear_cross_entropy", "Workspace",
+    "CCE_BWD_ROW_MAX", "cce_forward_ex", "cce_backward_prepare_rows",
 ]
 
 
@@ -95,8 +96,10 @@ def _stream_ptr(stream) -> int:
 
 
 def forward(E, C, y, ignore_index: int = IGNORE_INDEX, workspace: Optional[Workspace] = None,
-            stream=None, out=None) -> Tuple["object", "object"]:
-    """Per-token loss and log-sum-exp (fp32 tensors of shape [N])."""
+            stream=None, out=None, row_max=None) -> Tuple["object", "object"]:
+    """Per-token loss and log-sum-exp (fp32 tensors of shape [N]).  row_max:
+    an optional fp32 tensor [N] that receives each token's largest logit
+    (cce_forward_ex), for backward(..., row_max=...)."""
     torch = _torch()
     _check_inputs(E, C, y)
     N, D = E.shape
@@ -110,8 +113,15 @@ def forward(E, C, y, ignore_index: int = IGNORE_INDEX, workspace: Optional[Works
     if ws_bytes == 0:
         raise CCEError(1, "cce_forward_workspace_size: invalid sizes or no sm_100 device")
     ws = (workspace or Workspace(E.device)).get(ws_bytes)
-    cce_forward(E.data_ptr(), C.data_ptr(), y.data_ptr(), N, D, V, ignore_index, loss.data_ptr(),
-                lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    if row_max is not None:
+        if row_max.dtype != torch.float32 or not row_max.is_cuda or not row_max.is_contiguous() or \
+                row_max.shape != (N,):
+            raise ValueError("row_max must be a contiguous CUDA float32 tensor of shape [N]")
+        cce_forward_ex(E.data_ptr(), C.data_ptr(), y.data_ptr(), N, D, V, ignore_index, loss.data_ptr(),
+                       lse.data_ptr(), row_max.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    else:
+        cce_forward(E.data_ptr(), C.data_ptr(), y.data_ptr(), N, D, V, ignore_index, loss.data_ptr(),
+                    lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
     return loss, lse
 
 
@@ -132,7 +142,7 @@ def backward_prepare(C, N: int, workspace: Workspace, deterministic: bool = Fals
 def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = IGNORE_INDEX,
              workspace: Optional[Workspace] = None, stream=None, out=None, deterministic: bool = False,
              bf16_grads: bool = False, accumulate: bool = False, prepared: bool = False,
-             stripes: Optional[bool] = None):
+             stripes: Optional[bool] = None, row_max=None):
     """dE [N, D] and dC [V, D] of sum_i dloss[i] * loss[i]: fp32, or bf16 with
     bf16_grads; deterministic=True gives bitwise reproducible gradients
     (fixed-point accumulation, extra (N + V) * D * 8 bytes of workspace).
@@ -145,7 +155,10 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     order instead of using the int64 fixed-point accumulators.  With
     filter_eps > 0 it applies the same entry filter but skips no work: the
     faster choice only when a large share of the gradient is above the
-    threshold (a peaky, non-flat softmax)."""
+    threshold (a peaky, non-flat softmax).  row_max: the tokens' largest
+    logits from forward(..., row_max=...) on the same E and C; with the
+    filter on they replace the Cauchy-Schwarz bound in the pre-pass
+    (CCE_BWD_ROW_MAX), which finds more token blocks flat."""
     torch = _torch()
     _check_inputs(E, C, y)
     N, D = E.shape
@@ -159,6 +172,12 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
         stripes = filter_eps <= 0 and not bf16_grads
     if stripes:
         flags |= CCE_BWD_STRIPES
+    use_rows = row_max is not None and filter_eps > 0 and not stripes
+    if use_rows:
+        if row_max.dtype != torch.float32 or not row_max.is_cuda or not row_max.is_contiguous() or \
+                row_max.shape != (N,):
+            raise ValueError("row_max must be a contiguous CUDA float32 tensor of shape [N]")
+        flags |= CCE_BWD_ROW_MAX
     if prepared and workspace is None:
         raise ValueError("prepared=True needs the workspace that backward_prepare filled")
     if accumulate and out is None:
@@ -175,6 +194,8 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     if prepared and (workspace.buf is None or workspace.buf.numel() < ws_bytes):
         raise ValueError("prepared=True: the workspace backward_prepare filled is smaller than this call needs")
     ws = (workspace or Workspace(E.device)).get(ws_bytes)
+    if use_rows:
+        cce_backward_prepare_rows(row_max.data_ptr(), N, D, V, ws.data_ptr(), ws.numel(), _stream_ptr(stream))
     cce_backward_ex(E.data_ptr(), C.data_ptr(), y.data_ptr(), lse.data_ptr(), dloss.data_ptr(), N, D, V,
                     ignore_index, float(filter_eps), flags, dE.data_ptr(), dC.data_ptr(), ws.data_ptr(), ws.numel(),
                     _stream_ptr(stream))

@@ -56,6 +56,11 @@ def load_library():
         lib.cce_backward_ex.restype = ctypes.c_int
         lib.cce_backward_prepare.argtypes = [c_vp, c_i64, c_i64, c_i64, c_vp, c_size, c_vp]
         lib.cce_backward_prepare.restype = ctypes.c_int
+        lib.cce_backward_prepare_rows.argtypes = [c_vp, c_i64, c_i64, c_i64, c_vp, c_size, c_vp]
+        lib.cce_backward_prepare_rows.restype = ctypes.c_int
+        lib.cce_forward_ex.argtypes = [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_size,
+                                       c_vp]
+        lib.cce_forward_ex.restype = ctypes.c_int
         lib.cce_forward_shard.argtypes = [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_size,
                                           c_vp]
         lib.cce_forward_shard.restype = ctypes.c_int
@@ -135,6 +140,15 @@ def cce_forward(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: in
     return st
 
 
+def cce_forward_ex(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: int, loss: int, lse: int,
+                   row_max: int, workspace: int, workspace_bytes: int, stream: int, check: bool = True) -> int:
+    st = load_library().cce_forward_ex(E, C, y, N, D, V, ignore_index, loss, lse, row_max, workspace,
+                                       workspace_bytes, stream)
+    if check:
+        _check(st, "cce_forward_ex")
+    return st
+
+
 def cce_forward_noalloc(E: int, C: int, y: int, N: int, D: int, V: int, ignore_index: int, loss: int, lse: int,
                         stream: int, check: bool = True) -> int:
     """Forward pass without a workspace, for callers that cannot allocate
@@ -160,6 +174,15 @@ CCE_BWD_BF16_GRADS = 2
 CCE_BWD_ACCUMULATE = 4
 CCE_BWD_PREPARED = 8
 CCE_BWD_STRIPES = 16
+CCE_BWD_ROW_MAX = 32
+
+
+def cce_backward_prepare_rows(row_max: int, N: int, D: int, V: int, workspace: int, workspace_bytes: int,
+                              stream: int, check: bool = True) -> int:
+    st = load_library().cce_backward_prepare_rows(row_max, N, D, V, workspace, workspace_bytes, stream)
+    if check:
+        _check(st, "cce_backward_prepare_rows")
+    return st
 
 
 def cce_backward_prepare(C: int, N: int, D: int, V: int, workspace: int, workspace_bytes: int, stream: int,

@@ -246,7 +246,8 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
 }
 
 // Backward workspace: status | pre-pass header | dC row bits [ceil(V/32)] |
-// blk_flat, nonflat [n_mblk] | |E_i| [N].  O(N + V/32).
+// blk_flat, nonflat [n_mblk] | |E_i| [N] | the tokens' maximum logits [N]
+// (cce_backward_prepare_rows).  O(N + V/32).
 // Stripe backward (CCE_BWD_STRIPES, filter off): 256-token blocks per launch
 // (token super-block; dC gathers the super-blocks by reduce-adds) and
 // vocabulary tiles per stripe.
@@ -297,13 +298,13 @@ StripeLayout plan_stripes(int64_t N, int64_t D, int64_t V, size_t base) {
 
 struct BwdPlan {
   int n_mblk, n_vtile;
-  size_t off_hdr, off_rowbits, off_flat, off_nonflat, off_enorm, zero_bytes, ws_bytes;
+  size_t off_hdr, off_rowbits, off_flat, off_nonflat, off_enorm, off_rowmax, zero_bytes, ws_bytes;
   size_t off_accE, off_accC;  // fixed-point accumulators (deterministic mode only)
   StripeLayout stripes;       // CCE_BWD_STRIPES only
 };
 
-constexpr unsigned kBwdFlagsAll =
-    CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE | CCE_BWD_PREPARED | CCE_BWD_STRIPES;
+constexpr unsigned kBwdFlagsAll = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | CCE_BWD_ACCUMULATE |
+                                  CCE_BWD_PREPARED | CCE_BWD_STRIPES | CCE_BWD_ROW_MAX;
 // Whether these flags take the int64 fixed-point accumulation.  With
 // CCE_BWD_STRIPES the deterministic mode is served by the stripe kernel's
 // fixed reduction order instead (filter off only, fp32 outputs).
@@ -325,7 +326,8 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
   p->off_flat = p->zero_bytes;
   p->off_nonflat = p->off_flat + mb4;
   p->off_enorm = p->off_nonflat + mb4;
-  p->ws_bytes = p->off_enorm + align_up((size_t)N * sizeof(float), 256);
+  p->off_rowmax = p->off_enorm + align_up((size_t)N * sizeof(float), 256);
+  p->ws_bytes = p->off_rowmax + align_up((size_t)N * sizeof(float), 256);
   p->off_accE = p->off_accC = 0;
   if ((flags & CCE_BWD_STRIPES) && (flags & CCE_BWD_BF16_GRADS)) return false;  // not combined
   if (uses_fixed_point(flags)) {
@@ -346,12 +348,13 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
 // loss / lse are not written.
 cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
                           int64_t ignore_index, float* loss, float* lse, float* dbg_logits, void* ws,
-                          size_t ws_bytes, void* stream_, float* shard_stats = nullptr, int64_t v_offset = 0) {
+                          size_t ws_bytes, void* stream_, float* shard_stats = nullptr, int64_t v_offset = 0,
+                          float* row_max = nullptr) {
   if (!E || !C || !y || !ws) return CCE_ERR_INVALID_ARG;
   if (!shard_stats && (!loss || !lse)) return CCE_ERR_INVALID_ARG;
   if (!sizes_ok(N, D, V) || v_offset < 0) return CCE_ERR_INVALID_ARG;
   if (!aligned(E, 16) || !aligned(C, 16) || !aligned(y, 8) || !aligned(loss, 4) || !aligned(lse, 4) ||
-      !aligned(shard_stats, 4) || !aligned(ws, 256))
+      !aligned(shard_stats, 4) || !aligned(row_max, 4) || !aligned(ws, 256))
     return CCE_ERR_MISALIGNED;
   if (!device_info().ok) return CCE_ERR_UNSUPPORTED_DEVICE;
   FwdPlan p;
@@ -399,6 +402,7 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   f.status = status;
   f.shard_stats = shard_stats;
   f.v_offset = v_offset;
+  f.row_max = row_max;
   if (launch_fwd_finalize(E, C, y, f, loss, lse, stream) != cudaSuccess) return CCE_ERR_CUDA;
   return CCE_OK;
 }
@@ -423,6 +427,13 @@ cce_status_t cce_forward(const void* E, const void* C, const int64_t* y, int64_t
                          int64_t ignore_index, float* loss, float* lse, void* workspace, size_t workspace_bytes,
                          void* stream) {
   return forward_impl(E, C, y, N, D, V, ignore_index, loss, lse, nullptr, workspace, workspace_bytes, stream);
+}
+
+cce_status_t cce_forward_ex(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D, int64_t V,
+                            int64_t ignore_index, float* loss, float* lse, float* row_max, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return forward_impl(E, C, y, N, D, V, ignore_index, loss, lse, nullptr, workspace, workspace_bytes, stream,
+                      nullptr, 0, row_max);
 }
 
 cce_status_t cce_debug_forward_logits(const void* E, const void* C, const int64_t* y, int64_t N, int64_t D,
@@ -637,11 +648,18 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     return CCE_ERR_CUDA;
   const bool filter_on = filter_eps > 0.f;
   const bool prepared = (flags & CCE_BWD_PREPARED) != 0;
-  if (prepared && (filter_on || fixed)) {
-    // keep max_v |C_v| (header word HDR_CMAX) from cce_backward_prepare
-    const size_t keep0 = bp.off_hdr + HDR_CMAX * sizeof(unsigned), keep1 = keep0 + sizeof(unsigned);
-    if (cudaMemsetAsync(ws, 0, keep0, stream) != cudaSuccess ||
-        cudaMemsetAsync(ws + keep1, 0, bp.zero_bytes - keep1, stream) != cudaSuccess)
+  // the tokens' maximum logits from cce_backward_prepare_rows bound the
+  // logits exactly; the filter then needs neither |E_i| nor max_v |C_v|
+  const bool row_max = (flags & CCE_BWD_ROW_MAX) != 0 && filter_on && !(flags & CCE_BWD_STRIPES);
+  if ((prepared || row_max) && (filter_on || fixed)) {
+    // keep header words HDR_CMAX (cce_backward_prepare) and HDR_ROWMAX
+    // (cce_backward_prepare_rows); clear the rest
+    char* hdr0 = ws + bp.off_hdr;
+    if (cudaMemsetAsync(ws, 0, bp.off_hdr, stream) != cudaSuccess ||
+        (!prepared && cudaMemsetAsync(hdr0 + HDR_CMAX * 4, 0, 4, stream) != cudaSuccess) ||
+        cudaMemsetAsync(hdr0 + HDR_NNF * 4, 0, 4, stream) != cudaSuccess ||
+        (!row_max && cudaMemsetAsync(hdr0 + HDR_ROWMAX * 4, 0, 4, stream) != cudaSuccess) ||
+        cudaMemsetAsync(hdr0 + HDR_T * 4, 0, bp.zero_bytes - bp.off_hdr - HDR_T * 4, stream) != cudaSuccess)
       return CCE_ERR_CUDA;
   } else if (cudaMemsetAsync(ws, 0, (filter_on || fixed) ? bp.zero_bytes : STATUS_BYTES, stream) != cudaSuccess) {
     return CCE_ERR_CUDA;
@@ -710,9 +728,13 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     pp.blk_flat = reinterpret_cast<int*>(ws + bp.off_flat);
     pp.nonflat = reinterpret_cast<int*>(ws + bp.off_nonflat);
     pp.enorm = reinterpret_cast<float*>(ws + bp.off_enorm);
+    pp.row_max = row_max ? reinterpret_cast<const float*>(ws + bp.off_rowmax) : nullptr;
     pp.status = status;
-    if (!prepared && launch_cnorm(C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
-    if (launch_enorm(E, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    // the norms bound the logits (unless the row maxima do) and scale the
+    // fixed-point accumulation
+    if (!prepared && (fixed || !row_max) && launch_cnorm(C, pp, di.sms, stream) != cudaSuccess)
+      return CCE_ERR_CUDA;
+    if ((fixed || !row_max) && launch_enorm(E, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (filter_on && launch_prep(E, C, y, lse, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (fixed && launch_fixed_prep(dloss, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
     if (fixed && filter_on &&
@@ -799,6 +821,23 @@ cce_status_t cce_backward_prepare(const void* C, int64_t N, int64_t D, int64_t V
   pp.V = (int)V;
   pp.hdr = hdr;
   if (launch_cnorm(C, pp, di.sms, stream) != cudaSuccess) return CCE_ERR_CUDA;
+  return CCE_OK;
+}
+
+cce_status_t cce_backward_prepare_rows(const float* row_max, int64_t N, int64_t D, int64_t V, void* workspace,
+                                       size_t workspace_bytes, void* stream_) {
+  if (!row_max || !workspace) return CCE_ERR_INVALID_ARG;
+  if (!sizes_ok(N, D, V)) return CCE_ERR_INVALID_ARG;
+  if (!aligned(row_max, 4) || !aligned(workspace, 256)) return CCE_ERR_MISALIGNED;
+  BwdPlan bp;
+  if (!plan_backward(N, D, V, &bp)) return CCE_ERR_INVALID_ARG;
+  if (workspace_bytes < bp.ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  char* ws = reinterpret_cast<char*>(workspace);
+  if (cudaMemcpyAsync(ws + bp.off_rowmax, row_max, (size_t)N * sizeof(float), cudaMemcpyDeviceToDevice, stream) !=
+          cudaSuccess ||
+      cudaMemsetAsync(ws + bp.off_hdr + HDR_ROWMAX * 4, 0x01, 4, stream) != cudaSuccess)
+    return CCE_ERR_CUDA;
   return CCE_OK;
 }
 

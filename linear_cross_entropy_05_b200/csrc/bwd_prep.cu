@@ -3,8 +3,10 @@
 // The gradient filter (Cut Cross-Entropy abstract, sentence 9) drops every
 // entry of the softmax gradient with |P - onehot| < eps.  For a token i and a
 // column v that is not its label, P_iv = exp(E_i.C_v - lse_i) and, by
-// Cauchy-Schwarz, E_i.C_v <= |E_i| |C_v|.  So if |E_i| * max_v |C_v| <
-// lse_i + ln(eps) for every kept token of a 128-token block, every entry of
+// Cauchy-Schwarz, E_i.C_v <= |E_i| |C_v| (or, when the forward's maximum
+// logit of each token is at hand, E_i.C_v <= max_v E_i.C_v exactly).  So if
+// |E_i| * max_v |C_v| (or that maximum) < lse_i + ln(eps) for every kept
+// token of a 128-token block, every entry of
 // that block's rows except the label entries is dropped, and no logit of the
 // block needs to be recomputed: the label entry P_iy - 1 needs only the
 // correct-token logit E_i . C_y and lse_i.  Such a block is "flat"; its
@@ -112,12 +114,20 @@ __global__ void __launch_bounds__(128) prep_blocks_kernel(const int64_t* __restr
   if (!p.shard_mode && row < p.N && yl != p.ignore_index && !valid) atomicOr(p.status + ST_FLAGS, SF_BAD_LABEL);
   const long long ylocal = yl - (p.shard_mode ? p.v_offset : 0);
   const bool has_col = valid && ylocal >= 0 && ylocal < p.V;
-  const float cmax = __uint_as_float(p.hdr[HDR_CMAX]);
-  // Margins cover the fp32 rounding of the norms, of the recomputed logits and
-  // of the exp2 in the exact test.
+  // Margins cover the fp32 rounding of the norms (or of the forward's
+  // maximum against the backward's recomputed logits) and of the exp2 in
+  // the exact test.
   const float margin = 1.0f / 1024.0f;
   bool flat = true;
-  if (valid) flat = p.enorm[row] * cmax * (1.0f + margin) + margin < lse[row] + p.log_eps - margin;
+  if (p.row_max && p.hdr[HDR_ROWMAX] == 0u) {
+    flat = false;  // row maxima asked for but not stored for this call: visit every tile (exact, slower)
+  } else if (valid) {
+    // an upper bound of max_v E_i . C_v: the forward's exact maximum when
+    // given, else Cauchy-Schwarz
+    const float zmax = p.row_max ? p.row_max[row] + margin * (1.0f + fabsf(p.row_max[row]))
+                                 : p.enorm[row] * __uint_as_float(p.hdr[HDR_CMAX]) * (1.0f + margin) + margin;
+    flat = zmax < lse[row] + p.log_eps - margin;
+  }
   const int all_flat = __syncthreads_and(flat);
   if (t == 0) p.blk_flat[m] = all_flat;
   if (!all_flat) {
@@ -139,6 +149,7 @@ __global__ void prep_totals_kernel(PrepArgs p) {
   if (threadIdx.x != 0) return;
   const unsigned nnf = p.hdr[HDR_NNF];
   p.hdr[HDR_T] = (unsigned)((unsigned long long)nnf * (unsigned long long)p.n_vtile);
+  p.hdr[HDR_ROWMAX] = 0u;  // the row maxima serve one backward: the next needs cce_backward_prepare_rows again
   atomicAdd(p.status + ST_PRUNED,
             (((unsigned long long)p.N + 31ull) / 32ull) * (((unsigned long long)p.V + 31ull) / 32ull));
 }

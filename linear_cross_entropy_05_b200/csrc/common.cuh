@@ -40,7 +40,8 @@ enum StatusWord : int {
 enum PrepHeader : int {
   HDR_CMAX = 0,  // max_v |C_v| as float bits
   HDR_NNF = 1,   // token blocks that are not flat (visited densely)
-  HDR_T = 3,     // tiles to visit: NNF * n_vtile (word 2 is unused)
+  HDR_ROWMAX = 2,// nonzero: the workspace holds each token's maximum logit (cce_backward_prepare_rows)
+  HDR_T = 3,     // tiles to visit: NNF * n_vtile
   HDR_EMAX = 4,  // max_i |E_i| as float bits (fixed-point accumulation)
   HDR_DLMAX = 5, // max_i |dloss_i| as float bits (fixed-point accumulation)
 };
@@ -77,6 +78,7 @@ struct FinArgs {
   // to shard_stats [3][N] instead of loss / lse
   float* shard_stats;
   long long v_offset;
+  float* row_max;        // optional [N]: max_v z_iv, the largest logit of each token
 };
 
 struct PrepArgs {
@@ -90,6 +92,7 @@ struct PrepArgs {
   int* blk_flat;          // [n_mblk]
   int* nonflat;           // [n_mblk] ids of blocks that are not flat
   float* enorm;           // [N] |E_i|
+  const float* row_max;   // [N] max_v E_i . C_v from the forward, or null (then |E_i| max_v |C_v| bounds it)
   unsigned long long* status;
 };
 

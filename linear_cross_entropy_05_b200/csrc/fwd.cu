@@ -502,6 +502,7 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const __nv_bfloat16* 
       } else {
         lse[row] = qnan;
         loss[row] = qnan;
+        if (a.row_max) a.row_max[row] = qnan;
       }
     }
     return;
@@ -520,6 +521,7 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const __nv_bfloat16* 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   const float L = M + logf(s);
+  if (lane == 0 && a.row_max && !a.shard_stats) a.row_max[row] = M;
 
   if (a.shard_stats) {
     // vocabulary shard: (max, sum exp(z - max)) over the shard and the target

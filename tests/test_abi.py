@@ -117,11 +117,11 @@ def test_workspace_size_without_device_is_zero(lib):
     from linear_cross_entropy_05_b200 import cce_backward_workspace_size, cce_forward_workspace_size
     assert cce_forward_workspace_size(8192, 2304, 256000) == 0
     assert cce_forward_workspace_size(0, 8, 8) == 0
-    # status 256 + header 256 + one bit per vocabulary row + 2 x [N/128] i32 + N f32,
-    # each rounded to 256 bytes
+    # status 256 + header 256 + one bit per vocabulary row + 2 x [N/128] i32 + N f32
+    # (token norms) + N f32 (the tokens' maximum logits), each rounded to 256 bytes
     up = lambda x: (x + 255) // 256 * 256
     for N, V in ((8192, 256000), (300, 4173), (65536, 262144)):
-        want = 512 + up(4 * (-(-V // 32))) + 2 * up(4 * (-(-N // 128))) + up(4 * N)
+        want = 512 + up(4 * (-(-V // 32))) + 2 * up(4 * (-(-N // 128))) + 2 * up(4 * N)
         assert cce_backward_workspace_size(N, 2304, V) == want
     assert cce_backward_workspace_size(8192, 2305, 256000) == 0
 
@@ -156,12 +156,13 @@ def test_backward_ex_workspace_and_flags(lib):
     # token super-blocks of 16384 bound the stripe buffers whatever N
     big = cce_backward_workspace_size_ex(65536, 2048, 262144, 16) - cce_backward_workspace_size(65536, 2048, 262144)
     assert big < 3 * 16384 * 4096 * 2 + (1 << 20)
-    assert cce_backward_workspace_size_ex(N, D, V, 32) == 0     # unknown flag
+    assert cce_backward_workspace_size_ex(N, D, V, 32) == base  # row maxima: no extra workspace
+    assert cce_backward_workspace_size_ex(N, D, V, 64) == 0     # unknown flag
     P = 1 << 20
     args = [P, P, P, P, P, 256, 256, 4096, -100, 0.0, 0, P, P, P, 1 << 30, 0]
-    args[10] = 32
+    args[10] = 64
     assert cce_backward_ex(*args, check=False) == 1          # unknown flag: rejected on the host
-    for flags in (3, 4, 7, 8, 15, 16, 17, 21):
+    for flags in (3, 4, 7, 8, 15, 16, 17, 21, 32, 40):
         args[10] = flags
         assert cce_backward_ex(*args, check=False) == 4      # valid, but no device here
 
@@ -205,3 +206,16 @@ def test_stripe_knob_validates_on_the_host(lib):
     assert lib.cce_debug_set_stripe_params(0, 0, 33) == 1           # wider than 32 tiles
     assert lib.cce_debug_set_stripe_params(4096, 1, 16) == 0
     assert lib.cce_debug_set_stripe_params(0, 0, 0) == 0            # back to the defaults
+
+
+def test_row_max_entry_points_validate_on_the_host(lib):
+    _cpu_only()
+    from linear_cross_entropy_05_b200 import cce_backward_prepare_rows, cce_forward_ex
+    P = 1 << 20
+    assert cce_backward_prepare_rows(0, 4096, 256, 8192, P, 1 << 30, 0, check=False) == 1     # no row maxima
+    assert cce_backward_prepare_rows(P + 2, 4096, 256, 8192, P, 1 << 30, 0, check=False) == 2  # misaligned
+    assert cce_backward_prepare_rows(P, 4096, 255, 8192, P, 1 << 30, 0, check=False) == 1     # D % 8 != 0
+    assert cce_backward_prepare_rows(P, 4096, 256, 8192, P, 16, 0, check=False) == 3          # workspace too small
+    # the forward with row maxima validates like cce_forward (no device here)
+    assert cce_forward_ex(P, P, P, 4096, 256, 8192, -100, P, P, P + 2, P, 1 << 30, 0, check=False) == 2
+    assert cce_forward_ex(0, P, P, 4096, 256, 8192, -100, P, P, P, P, 1 << 30, 0, check=False) == 1

@@ -67,6 +67,11 @@ def test_launch_count_matches_the_kernels_a_step_runs(monkeypatch, tmp_path):
     assert b.launches_per_step(0.0, False) == 3
     assert b.launches_per_step(0.0, True) == 8
     assert b.launches_per_step(2.0 ** -12, True) == 12
+    # with the forward's row maxima the filter needs no norm pass (the
+    # fixed-point scale still does); the stripe path is one kernel
+    assert b.launches_per_step(2.0 ** -12, False, row_max=True) == 6
+    assert b.launches_per_step(2.0 ** -12, True, row_max=True) == 12
+    assert b.launches_per_step(2.0 ** -12, False, stripes=True) == 3
 
 
 def test_clock_sampler_reduces_nvml_samples(monkeypatch, tmp_path):

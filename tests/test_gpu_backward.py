@@ -336,3 +336,76 @@ def test_l2_hints_keep_the_results(eps):
     fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=ELEM)
     assert rel_fro(gE, fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(gC, fC) <= GRAD_REL_FILTER_OFF
+
+
+def test_row_max_bound_finds_flat_blocks_cauchy_schwarz_cannot():
+    # E scaled x10: the softmax is still spread out (max_v P ~ 1.7e-4 < eps),
+    # but |E_i| max_v |C_v| ~ 10 is far above lse + ln eps ~ 1.1, so the
+    # Cauchy-Schwarz pre-pass recomputes every tile; the forward's exact
+    # row maxima prove the blocks flat.  Both give the element-filtered
+    # gradient.  A peaky block (x120) stays non-flat either way.
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=900, V=12000 + 77, D=256)
+    inp = synth.make_inputs(w)
+    E64 = oracle.bf16_bits_to_f64(inp["E"]) * 10.0
+    E64[256:384] *= 12.0                    # one block with a peaky softmax
+    inp["E"] = synth.round_to_bf16_bits(E64.astype(np.float32))
+    E, C, y = to_dev(inp)
+    rm = torch.empty(w.N, device="cuda")
+    loss, lse = L.forward(E, C, y, IGN, row_max=rm)
+    dloss = synth.random_dloss(23, w.N)
+    dl = torch.from_numpy(dloss).cuda()
+    n_vt = -(-w.V // 256)
+    ws0, ws1 = L.Workspace(), L.Workspace()
+    cE, cC = L.backward(E, C, y, lse, dl, EPS, IGN, workspace=ws0)                # Cauchy-Schwarz
+    s0 = L.read_status(ws0)
+    rE, rC = L.backward(E, C, y, lse, dl, EPS, IGN, workspace=ws1, row_max=rm)    # row maxima
+    s1 = L.read_status(ws1)
+    assert s0["status"] == 0 and s1["status"] == 0
+    assert s0["logit_tiles"] == -(-w.N // 128) * n_vt          # nothing provably flat
+    assert s1["logit_tiles"] == n_vt                             # only the peaky block is visited
+    assert s1["flat_units"] > 0
+    assert s0["live_tiles"] == s1["live_tiles"]                  # the same live units either way
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=EPS, tile=ELEM)
+    for gE, gC in ((cE, cC), (rE, rC)):
+        assert rel_fro(gE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
+        assert rel_fro(gC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
+
+
+def test_row_max_flag_without_fresh_maxima_visits_every_tile():
+    # CCE_BWD_ROW_MAX when cce_backward_prepare_rows has not stored maxima for
+    # this call (a fresh workspace, or maxima already used by a previous
+    # call): every block is treated as not flat -- the exact path, slower
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    from linear_cross_entropy_05_b200 import _native as N_
+    w = synth.GEMMA2_2B.with_sizes(N=500, V=6000, D=256)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    rm = torch.empty(w.N, device="cuda")
+    loss, lse = L.forward(E, C, y, IGN, row_max=rm)
+    dl = torch.from_numpy(synth.random_dloss(24, w.N)).cuda()
+    dE = torch.empty((w.N, w.D), device="cuda")
+    dC = torch.empty((w.V, w.D), device="cuda")
+    ws = L.Workspace()
+    buf = ws.get(L.cce_backward_workspace_size_ex(w.N, w.D, w.V, L.CCE_BWD_ROW_MAX))
+    buf.zero_()
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def run():
+        N_.cce_backward_ex(E.data_ptr(), C.data_ptr(), y.data_ptr(), lse.data_ptr(), dl.data_ptr(), w.N, w.D, w.V,
+                           IGN, EPS, L.CCE_BWD_ROW_MAX, dE.data_ptr(), dC.data_ptr(), buf.data_ptr(), buf.numel(),
+                           stream)
+        return L.read_status(ws)
+
+    n_tiles = -(-w.N // 128) * -(-w.V // 256)
+    assert run()["logit_tiles"] == n_tiles                       # never prepared
+    ref = (dE.clone(), dC.clone())
+    N_.cce_backward_prepare_rows(rm.data_ptr(), w.N, w.D, w.V, buf.data_ptr(), buf.numel(), stream)
+    st = run()
+    assert st["logit_tiles"] == 0 and st["flat_units"] > 0      # every block flat with the maxima
+    assert rel_fro(dE.cpu().numpy(), ref[0].cpu().numpy()) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(dC.cpu().numpy(), ref[1].cpu().numpy()) <= GRAD_REL_FILTER_OFF
+    assert run()["logit_tiles"] == n_tiles                       # maxima serve one call only

@@ -217,3 +217,21 @@ def test_forward_schedule_knobs_keep_the_result(sched):
     ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
     assert np.abs(loss - ol).max() <= LOSS_ABS
     assert np.abs(lse - olse).max() <= LOSS_ABS
+
+
+def test_forward_ex_writes_each_tokens_largest_logit():
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=700, V=9000 + 77, D=256)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    rm = torch.full((w.N,), float("nan"), device="cuda")
+    loss, lse = L.forward(E, C, y, IGN, row_max=rm)
+    z = oracle.logits(oracle.bf16_bits_to_f64(inp["E"]), oracle.bf16_bits_to_f64(inp["C"]))   # fp64 [N, V]
+    want = z.max(axis=1)
+    got = rm.cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()                            # ignored rows too
+    assert np.abs(got - want).max() <= 1e-4 * max(1.0, float(np.abs(want).max()))
+    # the same loss as the plain forward
+    loss0, lse0 = L.forward(E, C, y, IGN)
+    assert torch.equal(loss, loss0) and torch.equal(lse, lse0)
