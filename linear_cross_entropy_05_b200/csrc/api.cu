@@ -266,7 +266,7 @@ struct StripeLayout {
   int n_sb;              // super-blocks (launches)
   int Ns_pad, Vs;
   size_t off_ctr, ctr_bytes, off_G, G_bytes, bytes;
-  size_t n_doneA_v, n_doneA_ms, n_doneBC, n_doneC;
+  size_t n_doneA_v, n_doneA_ms, n_doneBC, n_doneC, n_nz;
 };
 
 StripeLayout plan_stripes(int64_t N, int64_t D, int64_t V, size_t base) {
@@ -289,7 +289,8 @@ StripeLayout plan_stripes(int64_t N, int64_t D, int64_t V, size_t base) {
   L.n_doneBC = (size_t)L.p.n_s;
   L.n_doneC = (size_t)L.p.n_m2 * L.p.n_dc;
   L.off_ctr = base;
-  L.ctr_bytes = align_up(8 + 4 * (L.n_doneA_v + L.n_doneA_ms + L.n_doneBC + L.n_doneC), 256);
+  L.n_nz = (size_t)L.p.n_s * L.p.n_m2 * L.p.vt_per_s;
+  L.ctr_bytes = align_up(8 + 4 * (L.n_doneA_v + L.n_doneA_ms + L.n_doneBC + L.n_doneC) + L.n_nz, 256);
   L.off_G = L.off_ctr + L.ctr_bytes;
   L.G_bytes = align_up((size_t)L.p.nbuf * L.Ns_pad * L.Vs * 2, 256);
   L.bytes = L.off_G + L.G_bytes;
@@ -584,6 +585,7 @@ cce_status_t backward_stripes(const void* E, const void* C, void* dE, void* dC, 
   sa.doneA_ms = sa.doneA_v + L.n_doneA_v;
   sa.doneBC = sa.doneA_ms + L.n_doneA_ms;
   sa.doneC = sa.doneBC + L.n_doneBC;
+  sa.nz = a.filter_eps > 0.f ? reinterpret_cast<unsigned char*>(sa.doneC + L.n_doneC) : nullptr;
   sa.ordered = ordered ? 1 : 0;
   sa.status = a.status;
   sa.wait_limit_ns = a.wait_limit_ns;

@@ -100,9 +100,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
   uint64_t* drain = tempty + 2;                   // leader: UMMA drain at exit
   uint64_t* task_full = drain + 1;                // each CTA [SP_RING]
   uint64_t* task_empty = task_full + SP_RING;     // leader [SP_RING]
-  // each CTA [SP_RING], 16-byte aligned (written with 16-byte stores)
+  // each CTA [SP_RING][2], 16-byte aligned (written with 16-byte stores):
+  // the task, then its 64-bit mask of live K blocks (B / C tasks)
   int4* task_slot = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(task_empty + SP_RING) + 15) & ~uintptr_t(15));
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(task_slot + SP_RING);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(task_slot + 2 * SP_RING);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -153,15 +154,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
   // Reads task k from this CTA's ring, then frees the slot on the leader
   // (one arrival per consumer).  With whole_warp, lane 0 waits and reads and
   // the warp follows its outcome, so the lanes never part ways on a wait.
-  auto take_task = [&](int k, StripeTaskDesc& t, bool whole_warp) -> bool {
+  auto take_task = [&](int k, StripeTaskDesc& t, unsigned long long& mask, bool whole_warp) -> bool {
     const int slot = k & (SP_RING - 1);
     int4 d = make_int4(TASK_END, 0, 0, 0);
+    unsigned mlo = 0u, mhi = 0u;
     int ok = 1;
     if (!whole_warp || lane == 0) {
       ok = mbar_wait_cluster(&task_full[slot], (uint32_t)(k / SP_RING) & 1u, wc) ? 1 : 0;
       if (ok) {
-        const volatile int* vs = reinterpret_cast<const volatile int*>(&task_slot[slot]);
+        const volatile int* vs = reinterpret_cast<const volatile int*>(&task_slot[2 * slot]);
         d = make_int4(vs[0], vs[1], vs[2], vs[3]);
+        mlo = (unsigned)vs[4];
+        mhi = (unsigned)vs[5];
         mbar_arrive_cluster(task_empty_leader0 + (uint32_t)(slot * 8));
       }
     }
@@ -171,9 +175,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
       d.y = __shfl_sync(0xffffffffu, d.y, 0);
       d.z = __shfl_sync(0xffffffffu, d.z, 0);
       d.w = __shfl_sync(0xffffffffu, d.w, 0);
+      mlo = __shfl_sync(0xffffffffu, mlo, 0);
+      mhi = __shfl_sync(0xffffffffu, mhi, 0);
     }
     t = StripeTaskDesc{d.x, d.y, d.z, d.w};
+    mask = ((unsigned long long)mhi << 32) | mlo;
     return ok != 0;
+  };
+  // K blocks (256 wide: a token block for B, a vocabulary tile for C) of a
+  // B or C task, and which of them hold a nonzero G tile.  Read after the
+  // task's inputs are complete; without the filter every block is live.
+  auto k_blocks = [&](const StripeTaskDesc& t) -> int {
+    return t.type == TASK_B ? a.Ns_pad / 256 : stripe_tiles(P, t.s);
+  };
+  auto live_mask = [&](const StripeTaskDesc& t) -> unsigned long long {
+    const int nb = k_blocks(t);
+    const unsigned long long all = nb >= 64 ? ~0ull : ((1ull << nb) - 1ull);
+    if (t.type == TASK_A || t.type == TASK_END || a.nz == nullptr) return all;
+    unsigned long long m = 0ull;
+    if (t.type == TASK_B) {
+      const unsigned char* f = a.nz + (size_t)t.s * P.n_m2 * P.vt_per_s + (t.a - t.s * P.vt_per_s);
+      for (int b = 0; b < nb; ++b)
+        if (__ldcg(f + (size_t)b * P.vt_per_s)) m |= 1ull << b;
+    } else {
+      const unsigned char* f = a.nz + ((size_t)t.s * P.n_m2 + t.a) * P.vt_per_s;
+      for (int b = 0; b < nb; ++b)
+        if (__ldcg(f + b)) m |= 1ull << b;
+    }
+    return m;
   };
   // Bounded wait taken by lane 0 for the whole warp (warp-uniform outcome).
   auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -227,6 +256,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
       };
       for (int k = 0;; ++k) {
         StripeTaskDesc t;
+        unsigned long long tmask = 0ull;
         if (leader) {
           const int slot = k & (SP_RING - 1);
           if (!mbar_wait(&task_empty[slot], ((uint32_t)(k / SP_RING) & 1u) ^ 1u, wc)) goto producer_done;
@@ -256,8 +286,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
             fence_proxy_async_global();  // the inputs were written by other CTAs' bulk stores
           }
           const int4 d = make_int4(t.type, t.s, t.a, t.b);
-          task_slot[slot] = d;
-          st_shared_cluster_v4(mapa_shared(smem_u32(&task_slot[slot]), 1), d);
+          tmask = live_mask(t);
+          const int4 dm = make_int4((int)(unsigned)tmask, (int)(unsigned)(tmask >> 32), 0, 0);
+          task_slot[2 * slot] = d;
+          task_slot[2 * slot + 1] = dm;
+          st_shared_cluster_v4(mapa_shared(smem_u32(&task_slot[2 * slot]), 1), d);
+          st_shared_cluster_v4(mapa_shared(smem_u32(&task_slot[2 * slot + 1]), 1), dm);
           mbar_arrive(&task_full[slot]);
           mbar_arrive_release_cluster(mapa_shared(smem_u32(&task_full[slot]), 1));
           if (t.type != TASK_END) drawn_next = atomicAdd(a.next, 1ull);
@@ -267,11 +301,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
             trace[k * 4 + 3] = (unsigned long long)t.type | ((now - t_dep0) << 8);
           }
         } else {
-          if (!take_task(k, t, false)) goto producer_done;
+          if (!take_task(k, t, tmask, false)) goto producer_done;
           fence_proxy_async_global();
         }
         if (t.type == TASK_END) break;
-        const int nk = k_steps(t);
+        // live K slices of the task, in order (A tasks: all of K = D)
+        const int nk = t.type == TASK_A ? k_steps(t) : 4 * __popcll(tmask);
         const int r = (int)rank;
         if (t.type == TASK_C && a.dE_prefetch && !a.withhold_loads) {
           // the dE rows this task's epilogue will add into: into L2 while it computes
@@ -287,8 +322,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
         const int nd = t.type == TASK_A ? 256 : chunk_width(a.D, t.b);
         const int half_boxes = nd / 128;                 // 2, or 1 for a 128-wide chunk
         const uint32_t cta_bytes = 16384u + (t.type == TASK_A ? 16384u : 8192u * (uint32_t)half_boxes);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (leader && kb == (nk > SP_STAGES ? nk - SP_STAGES : 0)) look_ahead();
+        unsigned long long rest = tmask;  // B / C: live K blocks not yet streamed
+        int blk = -1;
+        for (int j = 0; j < nk; ++j) {
+          if (leader && j == (nk > SP_STAGES ? nk - SP_STAGES : 0)) look_ahead();
+          if (t.type != TASK_A && (j & 3) == 0) {
+            blk = __ffsll((long long)rest) - 1;
+            rest &= rest - 1ull;
+          }
+          const int kb = t.type == TASK_A ? j : 4 * blk + (j & 3);
           if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
           uint8_t* X = stages + stage * SP_STAGE_BYTES;
           uint8_t* Y = X + 16384;
@@ -348,12 +390,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
       uint32_t acc_phase = 0;
       for (int k = 0;; ++k) {
         StripeTaskDesc t;
-        if (!take_task(k, t, false)) goto mma_done;
+        unsigned long long tmask;
+        if (!take_task(k, t, tmask, false)) goto mma_done;
         if (t.type == TASK_END) break;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, wc)) goto mma_done;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        const int nk = k_steps(t);
+        // the live K slices the producer streams, in the same order (a task
+        // with none leaves the accumulator untouched; its epilogue knows)
+        const int nk = t.type == TASK_A ? k_steps(t) : 4 * __popcll(tmask);
         const bool narrow = t.type != TASK_A && chunk_width(a.D, t.b) == 128;
         const uint32_t idesc_b = narrow ? IDESC_B128 : IDESC_B;
         const uint32_t idesc_c = narrow ? IDESC_C128 : IDESC_C;
@@ -413,13 +458,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
     const int r = (int)rank;
     int acc = 0;
     uint32_t acc_phase = 0;
-    unsigned long long n_tiles = 0, n_units = 0;
+    unsigned long long n_tiles = 0, n_units = 0, n_live = 0, n_inrange = 0;
     unsigned long long* trace = (a.trace && leader && warp == 2 && lane == 0)
                                     ? a.trace + (size_t)(blockIdx.x >> 1) * a.trace_cap * 4
                                     : nullptr;
     for (int k = 0;; ++k) {
       StripeTaskDesc t;
-      if (!take_task(k, t, true)) break;
+      unsigned long long tmask;
+      if (!take_task(k, t, tmask, true)) break;
       if (t.type == TASK_END) break;
       if (!warp_wait(&tfull[acc], acc_phase)) break;
       tc_fence_after();
@@ -445,12 +491,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
         const int sw = lane & 7;
         const int gcol = (t.b - t.s * P.vt_per_s) * BN + hsel * 128;
         const int grow = (t.s % P.nbuf) * a.Ns_pad + t.a * 256 + r * 128 + lg * 32;
+        unsigned live_units = 0;  // of this warp's four 32 x 32 units (filter on)
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           const int c = hsel * 4 + cc;  // 32-column chunk of the accumulator
           float x[32];
           tmem_ld32(tacc + (uint32_t)(c * 32), x);
           uint32_t pk[16];
+          bool kept = false;
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
             float g2[2];
@@ -461,11 +509,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
               float d = (col == ycol) ? p - 1.f : p;
               d = (valid && col < ncols) ? d : 0.f;
               // the entry filter (eps <= 0 keeps every entry)
-              d = fabsf(d) >= a.filter_eps ? d : 0.f;
-              g2[q] = dl * d;
+              const bool keep = fabsf(d) >= a.filter_eps && d != 0.f;
+              kept |= keep;
+              g2[q] = keep ? dl * d : 0.f;
             }
             pk[j >> 1] = pack_bf16x2(g2[0], g2[1]);
           }
+          live_units += __any_sync(0xffffffffu, kept) ? 1u : 0u;
           // staging box cc / 2 (64 columns), this lane's 128-byte row, 128B swizzle
           uint8_t* rowp = stg + (cc >> 1) * 4096 + lane * 128;
 #pragma unroll
@@ -485,6 +535,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
           tma_store_2d(&mp.gSt, stg, gcol, grow);
           tma_store_2d(&mp.gSt, stg + 4096, gcol + 64, grow);
           bulk_commit_group();
+          // this G tile holds a kept entry: B and C tasks must read it
+          if (a.nz && live_units)
+            a.nz[((size_t)t.s * P.n_m2 + t.a) * P.vt_per_s + (t.b - t.s * P.vt_per_s)] = 1;
+          n_live += live_units;
+          // in-range units of this warp: its 32-row group (if any row is a
+          // token of this launch's range) x its 32-column chunks inside V
+          if (a.tok0 + t.a * 256 + r * 128 + lg * 32 < a.N)
+            n_inrange += (unsigned long long)max(0, min(4, (ncols - hsel * 128 + 31) / 32));
           bulk_wait_group0();
           fence_proxy_async_global();
           red_release_gpu_add(a.doneA_v + t.b, 1u);
@@ -537,12 +595,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
           __syncwarp();
           if (!ok) break;
         }
+        // no live K block: the accumulator was not written; the tile is zero
+        // (stored as zeros by a dC task that writes, skipped by one that adds)
+        const bool empty_task = tmask == 0ull;
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           const int c = hsel * 4 + cc;
           if (c * 32 >= nd) break;  // a 128-wide chunk fills only the first half
+          if (empty_task && add) break;
           float v[32];
-          tmem_ld32(tacc + (uint32_t)(c * 32), v);
+          if (empty_task) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] = 0.f;
+          } else {
+            tmem_ld32(tacc + (uint32_t)(c * 32), v);
+          }
           const int x0 = t.b * 256 + c * 32;
           if (row0 < rows_lim && x0 < a.D) {
             // Two staging buffers in turn: the block staged here two pieces ago
@@ -583,7 +650,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
     if (lane == 0) bulk_wait_group0();
     if (lg == 0 && hsel == 0 && lane == 0) {
       atomicAdd(a.status + ST_TILES, n_tiles);
-      atomicAdd(a.status + ST_LIVE_TILES, n_units);
+      // without the filter every recomputed unit counts as live; with it, the
+      // units holding a kept entry are live and the others dead
+      if (!a.nz) atomicAdd(a.status + ST_LIVE_TILES, n_units);
+    }
+    if (a.nz && lane == 0) {
+      // (counted by every epilogue warp: in-range units of its rows and columns)
+      atomicAdd(a.status + ST_LIVE_TILES, n_live);
+      atomicAdd(a.status + ST_DEAD_TILES, n_inrange - n_live);
     }
   }
 

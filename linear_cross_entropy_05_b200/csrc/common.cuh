@@ -340,6 +340,10 @@ struct StripeArgs {
   unsigned long long wait_limit_ns;
   int withhold_loads;    // test hook: the TMA producers issue nothing
   float filter_eps;      // > 0: entries of G with |P - onehot| below it are zeroed
+  // filter on: [n_s][n_m2][vt_per_s] bytes, 1 where the 256 x 256 G tile of
+  // an A task holds a kept entry (zeroed per launch); B and C tasks skip the
+  // K blocks whose G tile is all zero
+  unsigned char* nz;
 };
 
 // Fixed-point exponent s: contributions are stored as round(x * 2^s) in int64.

@@ -155,6 +155,10 @@ def test_stripes_with_the_entry_filter(deterministic):
     assert st["logit_tiles"] == -(-w.N // 128) * -(-w.V // 256)      # every tile recomputed
     _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
     fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=(1, 1))
+    # every unit recomputed: live (some entry kept) or dead, as the oracle counts them
+    live = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, eps, (32, 32))
+    assert st["live_tiles"] + st["dead_tiles"] == live.size and st["pruned_tiles"] == 0
+    assert abs(st["live_tiles"] - int(live.sum())) <= max(2, live.size // 1000)
     assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
     # the default filtered path gives the same gradient up to the bf16
