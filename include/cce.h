@@ -196,17 +196,21 @@ typedef enum {
    * traffic than adding every logit tile's partial products, so the tensor
    * cores set the pace.  With filter_eps <= 0 this is the dense (exact)
    * backward, the same result as without the flag up to fp32 summation
-   * order.  With filter_eps > 0 the entries below the threshold are zeroed
-   * in G (the same entry filter) but no work is skipped: every tile is
-   * recomputed and both products are dense, so this beats the default
-   * filtered path (pre-pass, flat rows, per-tile contractions of live
-   * 32 x 32 units) only when a large share of the units is live (measured
-   * on a Gemma-2-2B-shaped head with peaky logits: 25 ms against 52-53 ms at
-   * 40-61 % live units, but 25 ms against 9.3 ms at 0.2 % and 0.1 ms when
-   * the blocks are flat); the status counters then report every unit as
-   * live.  With CCE_BWD_DETERMINISTIC the reduce-adds into each dE tile
+   * order.  With filter_eps > 0 the pre-pass runs first (flat blocks go to
+   * the flat-row kernel, as in the default path); the stripe kernel skips
+   * the recompute of 256-token blocks that are entirely flat, zeroes the
+   * entries below the threshold (and the flat blocks' rows) in G, and skips
+   * the all-zero G tiles in the dC and dE products.  This beats the default
+   * filtered path (per-tile contractions of live 32 x 32 units with fp32
+   * reduce-adds) when a large share of the units is live, and loses when
+   * the gradient is sparse (measured on a Gemma-2-2B-shaped head with peaky
+   * logits: 27 ms against 53 ms at 61 % live units; 11.5 ms against 9.7 ms
+   * when only the label entries are live; 2 ms against 0.01 ms when every
+   * block is flat, the cost of handing out the empty tasks).  With CCE_BWD_DETERMINISTIC the reduce-adds into each dE tile
    * happen in stripe order (and dC is written once per tile), so the fp32
-   * result is bitwise reproducible without the int64 accumulators; the flag
+   * result is bitwise reproducible without the int64 accumulators (with the
+   * filter on, every tile is then recomputed: flat blocks are not sent to
+   * the flat-row kernel, whose dC additions are unordered); the flag
    * is not available with CCE_BWD_BF16_GRADS (the workspace size query
    * returns 0).  Needs the workspace of cce_backward_workspace_size_ex with
    * this flag. */

@@ -557,7 +557,8 @@ namespace {
 // Dense backward through softmax-gradient stripes (bwd_stripe.cu): one
 // launch per token super-block; a: the common backward arguments.
 cce_status_t backward_stripes(const void* E, const void* C, void* dE, void* dC, const BwdPlan& bp, const BwdArgs& a,
-                              bool accumulate, bool ordered, int sms, char* ws, cudaStream_t stream) {
+                              bool accumulate, bool ordered, int sms, char* ws, cudaStream_t stream,
+                              const int* blk_flat = nullptr) {
   const StripeLayout& L = bp.stripes;
   void* G = ws + L.off_G;
   CUtensorMap maps[9];
@@ -586,6 +587,7 @@ cce_status_t backward_stripes(const void* E, const void* C, void* dE, void* dC, 
   sa.doneBC = sa.doneA_ms + L.n_doneA_ms;
   sa.doneC = sa.doneBC + L.n_doneBC;
   sa.nz = a.filter_eps > 0.f ? reinterpret_cast<unsigned char*>(sa.doneC + L.n_doneC) : nullptr;
+  sa.blk_flat = blk_flat;
   sa.ordered = ordered ? 1 : 0;
   sa.status = a.status;
   sa.wait_limit_ns = a.wait_limit_ns;
@@ -652,7 +654,8 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   const bool prepared = (flags & CCE_BWD_PREPARED) != 0;
   // the tokens' maximum logits from cce_backward_prepare_rows bound the
   // logits exactly; the filter then needs neither |E_i| nor max_v |C_v|
-  const bool row_max = (flags & CCE_BWD_ROW_MAX) != 0 && filter_on && !(flags & CCE_BWD_STRIPES);
+  const bool row_max = (flags & CCE_BWD_ROW_MAX) != 0 && filter_on;
+  const bool stripes = (flags & CCE_BWD_STRIPES) != 0 && !fixed;
   if ((prepared || row_max) && (filter_on || fixed)) {
     // keep header words HDR_CMAX (cce_backward_prepare) and HDR_ROWMAX
     // (cce_backward_prepare_rows); clear the rest
@@ -671,7 +674,6 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     // with the filter on only visited vocabulary tiles are cleared, after the pre-pass
     if (!filter_on && cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
   } else if (!accumulate) {
-    const bool stripes = (flags & CCE_BWD_STRIPES) != 0;
     if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
     // (the stripe path writes every entry of dC)
     if (!stripes && cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess)
@@ -709,11 +711,13 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.trace = g_bwd_trace.load();
   a.trace_cap = g_bwd_trace_cap.load();
 
-  // the stripe kernel applies the entry filter while it forms G and needs no
-  // pre-pass (it visits every tile)
-  if ((flags & CCE_BWD_STRIPES) && !fixed)
-    return backward_stripes(E, C, dE, dC, bp, a, accumulate, (flags & CCE_BWD_DETERMINISTIC) != 0, di.sms, ws,
-                            stream);
+  const bool ordered = (flags & CCE_BWD_DETERMINISTIC) != 0;
+  // the dense backward, and the stripe-ordered (bitwise reproducible) one
+  // with the filter: the stripe kernel alone, no pre-pass (the flat-row
+  // kernel's fp32 additions into shared dC rows would not be reproducible)
+  if (stripes && (!filter_on || ordered))
+    return backward_stripes(E, C, dE, dC, bp, a, accumulate, ordered, di.sms, ws, stream);
+  FlatArgs fa{};
   if (filter_on || fixed) {
     PrepArgs pp;
     pp.N = (int)N;
@@ -744,7 +748,6 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
       return CCE_ERR_CUDA;
     if (filter_on) {
       // the label entries of the flat blocks (their other entries are all below eps)
-      FlatArgs fa;
       fa.N = (int)N;
       fa.D = (int)D;
       fa.V = (int)V;
@@ -760,8 +763,16 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
       fa.accE = accE;
       fa.accC = accC;
       fa.status = status;
-      if (launch_flat_rows(E, C, y, lse, dloss, fa, stream) != cudaSuccess) return CCE_ERR_CUDA;
+      if (!stripes && launch_flat_rows(E, C, y, lse, dloss, fa, stream) != cudaSuccess) return CCE_ERR_CUDA;
     }
+  }
+  if (stripes) {
+    // the blocks that are not flat through the stripe kernel (which stores
+    // every dC tile), then the flat blocks' label entries added on top
+    const cce_status_t st = backward_stripes(E, C, dE, dC, bp, a, accumulate, ordered, di.sms, ws, stream,
+                                             reinterpret_cast<const int*>(ws + bp.off_flat));
+    if (st != CCE_OK) return st;
+    return launch_flat_rows(E, C, y, lse, dloss, fa, stream) == cudaSuccess ? CCE_OK : CCE_ERR_CUDA;
   }
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;

@@ -189,9 +189,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
     return t.type == TASK_B ? a.Ns_pad / 256 : stripe_tiles(P, t.s);
   };
   auto live_mask = [&](const StripeTaskDesc& t) -> unsigned long long {
+    if (t.type == TASK_A) {
+      // 1: recompute; 0: both 128-token blocks are flat (or past N), skip
+      if (a.blk_flat == nullptr) return 1ull;
+      const int row0 = a.tok0 + t.a * 256;
+      const bool f0 = __ldcg(a.blk_flat + row0 / BM) != 0;
+      const bool f1 = row0 + BM >= a.N || __ldcg(a.blk_flat + row0 / BM + 1) != 0;
+      return (f0 && f1) ? 0ull : 1ull;
+    }
     const int nb = k_blocks(t);
     const unsigned long long all = nb >= 64 ? ~0ull : ((1ull << nb) - 1ull);
-    if (t.type == TASK_A || t.type == TASK_END || a.nz == nullptr) return all;
+    if (t.type == TASK_END || a.nz == nullptr) return all;
     unsigned long long m = 0ull;
     if (t.type == TASK_B) {
       const unsigned char* f = a.nz + (size_t)t.s * P.n_m2 * P.vt_per_s + (t.a - t.s * P.vt_per_s);
@@ -306,7 +314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
         }
         if (t.type == TASK_END) break;
         // live K slices of the task, in order (A tasks: all of K = D)
-        const int nk = t.type == TASK_A ? k_steps(t) : 4 * __popcll(tmask);
+        const int nk = t.type == TASK_A ? (tmask ? k_steps(t) : 0) : 4 * __popcll(tmask);
         const int r = (int)rank;
         if (t.type == TASK_C && a.dE_prefetch && !a.withhold_loads) {
           // the dE rows this task's epilogue will add into: into L2 while it computes
@@ -398,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         // the live K slices the producer streams, in the same order (a task
         // with none leaves the accumulator untouched; its epilogue knows)
-        const int nk = t.type == TASK_A ? k_steps(t) : 4 * __popcll(tmask);
+        const int nk = t.type == TASK_A ? (tmask ? k_steps(t) : 0) : 4 * __popcll(tmask);
         const bool narrow = t.type != TASK_A && chunk_width(a.D, t.b) == 128;
         const uint32_t idesc_b = narrow ? IDESC_B128 : IDESC_B;
         const uint32_t idesc_c = narrow ? IDESC_C128 : IDESC_C;
@@ -471,10 +479,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
       tc_fence_after();
       if (trace && k < a.trace_cap) trace[k * 4 + 1] = global_timer_ns();
       const uint32_t tacc = tmem_base + lane_addr + (uint32_t)(acc * BN);
-      if (t.type == TASK_A) {
+      if (t.type == TASK_A && tmask == 0ull) {
+        // both token blocks flat: nothing was recomputed and nothing is stored
+        // (the G tile keeps its flag 0, so no B or C task reads it)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+          red_release_gpu_add(a.doneA_v + t.b, 1u);
+          red_release_gpu_add(a.doneA_ms + (size_t)t.s * P.n_m2 + t.a, 1u);
+        }
+        __syncwarp();
+      } else if (t.type == TASK_A) {
         // row = token; columns = this warp's 128 of the 256 vocabulary entries of tile t.b
         const int row = a.tok0 + t.a * 256 + r * 128 + lg * 32 + lane;
-        bool valid = row < a.N;
+        // a flat block's rows of G are zero: its label entries go to the flat-row kernel
+        const int blk_row0 = a.tok0 + t.a * 256 + r * 128;
+        const bool blk_is_flat = a.blk_flat != nullptr && blk_row0 < a.N && a.blk_flat[blk_row0 / BM] != 0;
+        bool valid = row < a.N && !blk_is_flat;
         long long yl = valid ? a.y[row] : a.ignore_index;
         if (yl == a.ignore_index) valid = false;
         if (a.shard_mode) {
@@ -541,7 +563,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
           n_live += live_units;
           // in-range units of this warp: its 32-row group (if any row is a
           // token of this launch's range) x its 32-column chunks inside V
-          if (a.tok0 + t.a * 256 + r * 128 + lg * 32 < a.N)
+          if (a.tok0 + t.a * 256 + r * 128 + lg * 32 < a.N && !blk_is_flat)
             n_inrange += (unsigned long long)max(0, min(4, (ncols - hsel * 128 + 31) / 32));
           bulk_wait_group0();
           fence_proxy_async_global();

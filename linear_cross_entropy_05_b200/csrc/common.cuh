@@ -344,6 +344,10 @@ struct StripeArgs {
   // an A task holds a kept entry (zeroed per launch); B and C tasks skip the
   // K blocks whose G tile is all zero
   unsigned char* nz;
+  // filter on: [ceil(N / 128)] from the pre-pass, nonzero for a flat 128-token
+  // block (its label entries go to the flat-row kernel; its rows of G are
+  // zero, and a recompute task whose two blocks are both flat is skipped)
+  const int* blk_flat;
 };
 
 // Fixed-point exponent s: contributions are stored as round(x * 2^s) in int64.

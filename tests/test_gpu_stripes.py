@@ -132,9 +132,12 @@ def test_stripe_task_order_keeps_the_bits(order):
 
 @pytest.mark.parametrize("deterministic", [False, True], ids=["atomic", "stripe-ordered"])
 def test_stripes_with_the_entry_filter(deterministic):
-    # CCE_BWD_STRIPES with filter_eps > 0: the entries below eps are zeroed
-    # in G and every tile is visited; the result is the element-filtered
-    # gradient, on a head whose scaled rows make some blocks non-flat
+    # CCE_BWD_STRIPES with filter_eps > 0: the pre-pass sends flat blocks to
+    # the flat-row kernel; the stripe kernel recomputes the 256-token blocks
+    # that hold a block that is not flat, zeroes the entries below eps (and
+    # the flat blocks' rows) in G, and skips the all-zero G tiles in the dC
+    # and dE products; the result is the element-filtered gradient, on a head
+    # whose scaled rows make blocks 1 and 2 (of six) non-flat
     import torch
     import linear_cross_entropy_05_b200 as L
     w = synth.GEMMA2_2B.with_sizes(N=700, V=3 * 4096 + 77, D=264)
@@ -152,12 +155,19 @@ def test_stripes_with_the_entry_filter(deterministic):
     dE, dC = L.backward(E, C, y, lse_t, dl, eps, IGN, workspace=ws, stripes=True, deterministic=deterministic)
     st = L.read_status(ws)
     assert st["status"] == 0 and st["flags"] == 0
-    assert st["logit_tiles"] == -(-w.N // 128) * -(-w.V // 256)      # every tile recomputed
+    n_vt = -(-w.V // 256)
+    if deterministic:
+        # stripe order alone, no flat-row path: every tile recomputed
+        assert st["logit_tiles"] == -(-w.N // 128) * n_vt and st["flat_units"] == 0
+    else:
+        assert st["logit_tiles"] == 4 * n_vt      # the two 256-token blocks holding blocks 1 and 2
+        assert st["flat_units"] > 0
     _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
     fE, fC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=(1, 1))
-    # every unit recomputed: live (some entry kept) or dead, as the oracle counts them
+    # live (some entry kept), dead (recomputed, none kept) and pruned (flat
+    # blocks' units without a label entry) add up to all units
     live = oracle.tile_live_map(inp["E"], inp["C"], inp["y"], olse, IGN, eps, (32, 32))
-    assert st["live_tiles"] + st["dead_tiles"] == live.size and st["pruned_tiles"] == 0
+    assert st["live_tiles"] + st["dead_tiles"] + st["pruned_tiles"] == live.size
     assert abs(st["live_tiles"] - int(live.sum())) <= max(2, live.size // 1000)
     assert rel_fro(dE.cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(dC.cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
@@ -170,3 +180,28 @@ def test_stripes_with_the_entry_filter(deterministic):
     if deterministic:
         dE2, dC2 = L.backward(E, C, y, lse_t, dl, eps, IGN, workspace=ws, stripes=True, deterministic=True)
         assert torch.equal(dE, dE2) and torch.equal(dC, dC2)
+
+
+def test_stripes_with_the_filter_on_a_flat_head_recompute_nothing():
+    # every block flat: the stripe kernel skips every recompute task and
+    # every dC / dE product; the gradient comes from the flat-row kernel
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=16384 + 300, V=12000, D=256)   # two token super-blocks
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    dloss = synth.random_dloss(25, w.N)
+    ws = L.Workspace()
+    dE, dC = L.backward(E, C, y, torch.from_numpy(lse).cuda(), torch.from_numpy(dloss).cuda(),
+                        synth.EPS_BF16_FILTER, IGN, workspace=ws, stripes=True)
+    st = L.read_status(ws)
+    assert st["status"] == 0 and st["flags"] == 0
+    assert st["logit_tiles"] == 0 and st["flat_units"] == st["live_tiles"] > 0
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    rows = np.concatenate([np.arange(0, 256), np.arange(w.N - 300, w.N)])
+    vrows = np.unique(np.concatenate([inp["y"][inp["y"] != IGN][:200], [0, w.V - 1]]))
+    fE, fC = oracle.backward_sampled(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, rows, vrows,
+                                     filter_eps=synth.EPS_BF16_FILTER, tile=(1, 1))
+    assert rel_fro(dE[torch.from_numpy(rows).cuda()].cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
+    assert rel_fro(dC[torch.from_numpy(vrows).cuda()].cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
