@@ -148,7 +148,8 @@ def test_backward_ex_workspace_and_flags(lib):
     assert cce_backward_workspace_size_ex(N, D, V, 8) == base   # prepared: no extra workspace
     # stripes: counters + three bf16 stripe buffers of 8192 tokens x 4096 columns
     n_vt, n_s, n_dc = -(-V // 256), -(-V // 4096), -(-D // 256)
-    ctr = up(8 + 4 * (n_vt + n_s * 32 + n_s + 32 * n_dc))
+    # task counters (u32) and one byte per G tile of every stripe (nonzero flags)
+    ctr = up(8 + 4 * (n_vt + n_s * 32 + n_s + 32 * n_dc) + n_s * 32 * 16)
     assert cce_backward_workspace_size_ex(N, D, V, 16) == base + ctr + up(3 * 8192 * 4096 * 2)
     # deterministic with stripes: fixed stripe order, no int64 accumulators
     assert cce_backward_workspace_size_ex(N, D, V, 17) == base + ctr + up(3 * 8192 * 4096 * 2)
