@@ -1018,8 +1018,10 @@ def run_suite(args):
         y = torch.from_numpy(inp["y"]).to(dev)
         dl = torch.from_numpy(synth.mean_dloss(inp["y"])).to(dev)
         wsf, wsb = L.Workspace(dev), L.Workspace(dev)
-        loss, lse = L.forward(E, C, y, IGN, workspace=wsf)
-        dE, dC = L.backward(E, C, y, lse, dl, w.filter_eps, IGN, workspace=wsb)
+        # the forward's row maxima feed the filter's pre-pass (as in the step)
+        rm = torch.empty(N, device=dev) if (w.filter_eps > 0 and not args.no_row_max) else None
+        loss, lse = L.forward(E, C, y, IGN, workspace=wsf, row_max=rm)
+        dE, dC = L.backward(E, C, y, lse, dl, w.filter_eps, IGN, workspace=wsb, row_max=rm)
         st = L.read_status(wsb)
         reps = 5
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
@@ -1027,9 +1029,9 @@ def run_suite(args):
         tf = tb = 0.0
         for _ in range(reps):
             ev[0].record()
-            L.forward(E, C, y, IGN, workspace=wsf, out=(loss, lse))
+            L.forward(E, C, y, IGN, workspace=wsf, out=(loss, lse), row_max=rm)
             ev[1].record()
-            L.backward(E, C, y, lse, dl, w.filter_eps, IGN, workspace=wsb, out=(dE, dC))
+            L.backward(E, C, y, lse, dl, w.filter_eps, IGN, workspace=wsb, out=(dE, dC), row_max=rm)
             ev[2].record()
             torch.cuda.synchronize()
             tf += ev[0].elapsed_time(ev[1]) / reps
