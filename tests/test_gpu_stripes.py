@@ -205,3 +205,31 @@ def test_stripes_with_the_filter_on_a_flat_head_recompute_nothing():
                                      filter_eps=synth.EPS_BF16_FILTER, tile=(1, 1))
     assert rel_fro(dE[torch.from_numpy(rows).cuda()].cpu().numpy(), fE) <= GRAD_REL_FILTER_OFF
     assert rel_fro(dC[torch.from_numpy(vrows).cuda()].cpu().numpy(), fC) <= GRAD_REL_FILTER_OFF
+
+
+def test_stripes_with_the_filter_accumulate():
+    # CCE_BWD_ACCUMULATE through the filtered stripe path: the stripes add
+    # their dC tiles (instead of storing them) and the flat-row kernel adds
+    # on top; the result is the prior contents plus this call's gradient
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=700, V=2 * 4096 + 77, D=264)
+    inp = synth.make_inputs(w)
+    E64 = oracle.bf16_bits_to_f64(inp["E"])
+    E64[128:256] *= 120.0                   # one block that is not flat
+    inp["E"] = synth.round_to_bf16_bits(E64.astype(np.float32))
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    lse_t = torch.from_numpy(lse).cuda()
+    dl = torch.from_numpy(synth.random_dloss(26, w.N)).cuda()
+    eps = synth.EPS_BF16_FILTER
+    gE, gC = L.backward(E, C, y, lse_t, dl, eps, IGN, workspace=L.Workspace(), stripes=True)
+    gen = torch.Generator().manual_seed(4)
+    pE = (torch.randn(gE.shape, generator=gen) * float(gE.abs().max())).cuda()
+    pC = (torch.randn(gC.shape, generator=gen) * float(gC.abs().max())).cuda()
+    aE, aC = pE.clone(), pC.clone()
+    ws = L.Workspace()
+    L.backward(E, C, y, lse_t, dl, eps, IGN, workspace=ws, out=(aE, aC), accumulate=True, stripes=True)
+    assert L.read_status(ws)["status"] == 0
+    assert rel_fro((aE - pE).cpu().numpy(), gE.cpu().numpy()) < 1e-5
+    assert rel_fro((aC - pC).cpu().numpy(), gC.cpu().numpy()) < 1e-5
