@@ -1,5 +1,6 @@
-// CCE backward with every gradient unit kept (filter off): the dense path,
-// through stripes of the softmax gradient.
+// CCE backward through stripes of the softmax gradient: the dense path
+// (filter off), and with the entry filter for heads whose softmax is not
+// flat (CCE_BWD_STRIPES with filter_eps > 0).
 //
 // Cut Cross-Entropy abstract, sentences 4 and 9: the logits are recomputed,
 // never stored; the backward forms G = dloss * (softmax - onehot) and
@@ -20,6 +21,14 @@
 // So the logits never exist in global memory: only nbuf stripes of G do,
 // O(N) bytes for a fixed stripe width (Vs = 4096: 24 KB per token with three
 // buffers), against N x V x 4 bytes of fp32 logits.
+//
+// With the filter on, entries below filter_eps are zeroed in G, and work is
+// skipped at two grains: an A task whose two 128-token blocks the pre-pass
+// proved flat is not recomputed (the flat-row kernel adds those blocks'
+// label entries afterwards; a flat half of a recomputed task gets zero rows),
+// and each A task flags its 256 x 256 G tile if it holds a kept entry, so a
+// B or C task streams only the K blocks (token blocks, resp. vocabulary
+// tiles) whose G tile is flagged; the mask travels with the task.
 //
 // One persistent kernel runs all three kinds on clusters of two CTAs.  Tasks
 // are drawn in a fixed global order from a counter by the leader CTA's
