@@ -165,8 +165,11 @@ typedef enum {
    * in which the tiles finish; a final pass converts to the output type.
    * Needs an extra (N + V) * D * 8 bytes of workspace. */
   CCE_BWD_DETERMINISTIC = 1,
-  /* dE and dC are written as bf16 (round to nearest even) instead of fp32;
-   * implies CCE_BWD_DETERMINISTIC (the accumulation is the same). */
+  /* dE and dC are written as bf16 (round to nearest even) instead of fp32.
+   * Without CCE_BWD_STRIPES it implies CCE_BWD_DETERMINISTIC (the same
+   * fixed-point accumulation, converted once); with CCE_BWD_STRIPES the
+   * sums go to fp32 scratch in the workspace ((N + V) * D * 4 bytes) and are
+   * rounded to bf16 once at the end. */
   CCE_BWD_BF16_GRADS = 2,
   /* Add this call's gradients to the contents of dE and dC instead of
    * overwriting them (no zeroing pass): gradient accumulation over
@@ -206,14 +209,15 @@ typedef enum {
    * the gradient is sparse (measured on a Gemma-2-2B-shaped head with peaky
    * logits: 27 ms against 53 ms at 61 % live units; 11.5 ms against 9.7 ms
    * when only the label entries are live; 2 ms against 0.01 ms when every
-   * block is flat, the cost of handing out the empty tasks).  With CCE_BWD_DETERMINISTIC the reduce-adds into each dE tile
-   * happen in stripe order (and dC is written once per tile), so the fp32
-   * result is bitwise reproducible without the int64 accumulators (with the
-   * filter on, every tile is then recomputed: flat blocks are not sent to
-   * the flat-row kernel, whose dC additions are unordered); the flag
-   * is not available with CCE_BWD_BF16_GRADS (the workspace size query
-   * returns 0).  Needs the workspace of cce_backward_workspace_size_ex with
-   * this flag. */
+   * block is flat, the cost of handing out the empty tasks).  With
+   * CCE_BWD_DETERMINISTIC the reduce-adds into each dE tile happen in
+   * stripe order (and dC is written once per tile), so the fp32 result is
+   * bitwise reproducible without the int64 accumulators (with the filter
+   * on, every tile is then recomputed: flat blocks are not sent to the
+   * flat-row kernel, whose dC additions are unordered).  With
+   * CCE_BWD_BF16_GRADS the sums go to fp32 scratch and are rounded to bf16
+   * once.  Needs the workspace of cce_backward_workspace_size_ex with this
+   * flag. */
   CCE_BWD_STRIPES = 16,
   /* With filter_eps > 0: cce_backward_prepare_rows has stored each token's
    * largest logit max_v E_i . C_v (from cce_forward_ex) in this workspace for

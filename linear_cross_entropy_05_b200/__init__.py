@@ -148,8 +148,8 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     (fixed-point accumulation, extra (N + V) * D * 8 bytes of workspace).
     accumulate=True adds them to the tensors given in `out` (required)
     instead of overwriting them.  prepared=True: backward_prepare already ran
-    on `workspace` for this C.  stripes (default: on when filter_eps <= 0
-    and not bf16_grads): the backward through softmax-gradient stripes
+    on `workspace` for this C.  stripes (default: on when filter_eps <= 0):
+    the backward through softmax-gradient stripes
     (CCE_BWD_STRIPES), which needs a larger workspace (about 24 KB per
     token, at most ~400 MB); with deterministic=True it sums in a fixed
     order instead of using the int64 fixed-point accumulators.  With
@@ -169,7 +169,7 @@ def backward(E, C, y, lse, dloss, filter_eps: float = 0.0, ignore_index: int = I
     flags = ((CCE_BWD_DETERMINISTIC if deterministic else 0) | (CCE_BWD_BF16_GRADS if bf16_grads else 0) |
              (CCE_BWD_ACCUMULATE if accumulate else 0) | (CCE_BWD_PREPARED if prepared else 0))
     if stripes is None:
-        stripes = filter_eps <= 0 and not bf16_grads
+        stripes = filter_eps <= 0
     if stripes:
         flags |= CCE_BWD_STRIPES
     use_rows = row_max is not None and filter_eps > 0 and not stripes

@@ -42,6 +42,7 @@ cudaError_t launch_clear_visited_rows(unsigned long long* acc, int V, int D, con
                                       const unsigned* hdr, int sms, cudaStream_t stream);
 cudaError_t launch_flat_rows(const void* E, const void* C, const int64_t* y, const float* lse, const float* dloss,
                              const FlatArgs& f, cudaStream_t stream);
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, size_t n, bool accumulate, int sms, cudaStream_t stream);
 }  // namespace cce
 
 using namespace cce;
@@ -310,6 +311,7 @@ constexpr unsigned kBwdFlagsAll = CCE_BWD_DETERMINISTIC | CCE_BWD_BF16_GRADS | C
 // CCE_BWD_STRIPES the deterministic mode is served by the stripe kernel's
 // fixed reduction order instead (filter off only, fp32 outputs).
 bool uses_fixed_point(unsigned flags) {
+  if (flags & CCE_BWD_STRIPES) return false;  // bf16 outputs: fp32 scratch, converted once
   if (flags & CCE_BWD_BF16_GRADS) return true;
   return (flags & CCE_BWD_DETERMINISTIC) && !(flags & CCE_BWD_STRIPES);
 }
@@ -330,8 +332,12 @@ bool plan_backward(int64_t N, int64_t D, int64_t V, BwdPlan* p, unsigned flags =
   p->off_rowmax = p->off_enorm + align_up((size_t)N * sizeof(float), 256);
   p->ws_bytes = p->off_rowmax + align_up((size_t)N * sizeof(float), 256);
   p->off_accE = p->off_accC = 0;
-  if ((flags & CCE_BWD_STRIPES) && (flags & CCE_BWD_BF16_GRADS)) return false;  // not combined
-  if (uses_fixed_point(flags)) {
+  if ((flags & CCE_BWD_STRIPES) && (flags & CCE_BWD_BF16_GRADS)) {
+    // the stripe path with bf16 outputs sums into fp32 dE / dC scratch
+    p->off_accE = p->ws_bytes;
+    p->off_accC = p->off_accE + align_up((size_t)N * D * 4, 256);
+    p->ws_bytes = p->off_accC + align_up((size_t)V * D * 4, 256);
+  } else if (uses_fixed_point(flags)) {
     p->off_accE = p->ws_bytes;
     p->off_accC = p->off_accE + align_up((size_t)N * D * 8, 256);
     p->ws_bytes = p->off_accC + align_up((size_t)V * D * 8, 256);
@@ -656,6 +662,12 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   // logits exactly; the filter then needs neither |E_i| nor max_v |C_v|
   const bool row_max = (flags & CCE_BWD_ROW_MAX) != 0 && filter_on;
   const bool stripes = (flags & CCE_BWD_STRIPES) != 0 && !fixed;
+  // bf16 outputs through the stripe path: every sum goes to fp32 scratch in
+  // the workspace (fresh each call), rounded to bf16 once at the end
+  const bool stripes_bf16 = stripes && bf16_out;
+  float* dE32 = stripes_bf16 ? reinterpret_cast<float*>(ws + bp.off_accE) : reinterpret_cast<float*>(dE);
+  float* dC32 = stripes_bf16 ? reinterpret_cast<float*>(ws + bp.off_accC) : reinterpret_cast<float*>(dC);
+  const bool acc32 = accumulate && !stripes_bf16;
   if ((prepared || row_max) && (filter_on || fixed)) {
     // keep header words HDR_CMAX (cce_backward_prepare) and HDR_ROWMAX
     // (cce_backward_prepare_rows); clear the rest
@@ -673,8 +685,8 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
     if (cudaMemsetAsync(accE, 0, (size_t)N * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
     // with the filter on only visited vocabulary tiles are cleared, after the pre-pass
     if (!filter_on && cudaMemsetAsync(accC, 0, (size_t)V * D * 8, stream) != cudaSuccess) return CCE_ERR_CUDA;
-  } else if (!accumulate) {
-    if (cudaMemsetAsync(dE, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
+  } else if (!acc32) {
+    if (cudaMemsetAsync(dE32, 0, (size_t)N * D * sizeof(float), stream) != cudaSuccess) return CCE_ERR_CUDA;
     // (the stripe path writes every entry of dC)
     if (!stripes && cudaMemsetAsync(dC, 0, (size_t)V * D * sizeof(float), stream) != cudaSuccess)
       return CCE_ERR_CUDA;
@@ -712,11 +724,21 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   a.trace_cap = g_bwd_trace_cap.load();
 
   const bool ordered = (flags & CCE_BWD_DETERMINISTIC) != 0;
+  // bf16 outputs of the stripe path: the fp32 scratch sums rounded once
+  auto finish_stripes = [&]() -> cce_status_t {
+    if (!stripes_bf16) return CCE_OK;
+    if (launch_f32_to_bf16(dE32, dE, (size_t)N * D, accumulate, di.sms, stream) != cudaSuccess ||
+        launch_f32_to_bf16(dC32, dC, (size_t)V * D, accumulate, di.sms, stream) != cudaSuccess)
+      return CCE_ERR_CUDA;
+    return CCE_OK;
+  };
   // the dense backward, and the stripe-ordered (bitwise reproducible) one
   // with the filter: the stripe kernel alone, no pre-pass (the flat-row
   // kernel's fp32 additions into shared dC rows would not be reproducible)
-  if (stripes && (!filter_on || ordered))
-    return backward_stripes(E, C, dE, dC, bp, a, accumulate, ordered, di.sms, ws, stream);
+  if (stripes && (!filter_on || ordered)) {
+    const cce_status_t st = backward_stripes(E, C, dE32, dC32, bp, a, acc32, ordered, di.sms, ws, stream);
+    return st != CCE_OK ? st : finish_stripes();
+  }
   FlatArgs fa{};
   if (filter_on || fixed) {
     PrepArgs pp;
@@ -755,11 +777,11 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
       fa.shard_mode = shard ? 1 : 0;
       fa.v_offset = v_offset;
       fa.filter_eps = filter_eps;
-      fa.accumulate = accumulate ? 1 : 0;
+      fa.accumulate = acc32 ? 1 : 0;
       fa.blk_flat = pp.blk_flat;
       fa.hdr = pp.hdr;
-      fa.dE = reinterpret_cast<float*>(dE);
-      fa.dC = reinterpret_cast<float*>(dC);
+      fa.dE = dE32;
+      fa.dC = dC32;
       fa.accE = accE;
       fa.accC = accC;
       fa.status = status;
@@ -769,10 +791,11 @@ cce_status_t backward_impl(const void* E, const void* C, const int64_t* y, const
   if (stripes) {
     // the blocks that are not flat through the stripe kernel (which stores
     // every dC tile), then the flat blocks' label entries added on top
-    const cce_status_t st = backward_stripes(E, C, dE, dC, bp, a, accumulate, ordered, di.sms, ws, stream,
+    const cce_status_t st = backward_stripes(E, C, dE32, dC32, bp, a, acc32, ordered, di.sms, ws, stream,
                                              reinterpret_cast<const int*>(ws + bp.off_flat));
     if (st != CCE_OK) return st;
-    return launch_flat_rows(E, C, y, lse, dloss, fa, stream) == cudaSuccess ? CCE_OK : CCE_ERR_CUDA;
+    if (launch_flat_rows(E, C, y, lse, dloss, fa, stream) != cudaSuccess) return CCE_ERR_CUDA;
+    return finish_stripes();
   }
   const int grid = filter_on ? di.sms : std::min(a.n_tiles, di.sms);
   if (record_event(1, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;

@@ -415,6 +415,30 @@ cudaError_t launch_fixed_to_out(const unsigned long long* acc, void* out, int ro
   return cudaGetLastError();
 }
 
+// bf16 gradient outputs of the stripe path: the fp32 sums, rounded once to
+// bf16 (with accumulate, added to what the output holds first).  n % 4 == 0.
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ src, uint2* dst, size_t n4,
+                                                          int accumulate) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 v = src[i];
+    if (accumulate) {
+      const uint2 o = dst[i];
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
+      const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
+      v = make_float4(v.x + a.x, v.y + a.y, v.z + b.x, v.w + b.y);
+    }
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+    dst[i] = make_uint2(*reinterpret_cast<const unsigned*>(&lo), *reinterpret_cast<const unsigned*>(&hi));
+  }
+}
+
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, size_t n, bool accumulate, int sms, cudaStream_t stream) {
+  f32_to_bf16_kernel<<<sms * 8, 256, 0, stream>>>(reinterpret_cast<const float4*>(src), reinterpret_cast<uint2*>(dst),
+                                                  n / 4, accumulate ? 1 : 0);
+  return cudaGetLastError();
+}
+
 // Norm pre-pass shared by the filter and the fixed-point scale: max_v |C_v|
 // (launch_cnorm; HDR_CMAX must start at zero), |E_i| per token and
 // max_i |E_i| (launch_enorm).

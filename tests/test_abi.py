@@ -153,7 +153,9 @@ def test_backward_ex_workspace_and_flags(lib):
     assert cce_backward_workspace_size_ex(N, D, V, 16) == base + ctr + up(3 * 8192 * 4096 * 2)
     # deterministic with stripes: fixed stripe order, no int64 accumulators
     assert cce_backward_workspace_size_ex(N, D, V, 17) == base + ctr + up(3 * 8192 * 4096 * 2)
-    assert cce_backward_workspace_size_ex(N, D, V, 18) == 0     # bf16 outputs and stripes do not combine
+    # bf16 outputs through stripes: fp32 dE / dC scratch, rounded once
+    assert cce_backward_workspace_size_ex(N, D, V, 18) == base + up(4 * N * D) + up(4 * V * D) + ctr + \
+        up(3 * 8192 * 4096 * 2)
     # token super-blocks of 16384 bound the stripe buffers whatever N
     big = cce_backward_workspace_size_ex(65536, 2048, 262144, 16) - cce_backward_workspace_size(65536, 2048, 262144)
     assert big < 3 * 16384 * 4096 * 2 + (1 << 20)

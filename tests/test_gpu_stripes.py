@@ -233,3 +233,43 @@ def test_stripes_with_the_filter_accumulate():
     assert L.read_status(ws)["status"] == 0
     assert rel_fro((aE - pE).cpu().numpy(), gE.cpu().numpy()) < 1e-5
     assert rel_fro((aC - pC).cpu().numpy(), gC.cpu().numpy()) < 1e-5
+
+
+@pytest.mark.parametrize("eps", [0.0, synth.EPS_BF16_FILTER], ids=["filter-off", "filter-on"])
+def test_stripes_with_bf16_outputs(eps):
+    # CCE_BWD_STRIPES | CCE_BWD_BF16_GRADS: fp32 scratch sums rounded once to
+    # bf16; with accumulate the old bf16 values are added before rounding
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=700, V=2 * 4096 + 77, D=264)
+    inp = synth.make_inputs(w)
+    E64 = oracle.bf16_bits_to_f64(inp["E"])
+    E64[128:256] *= 120.0                   # one block that is not flat
+    inp["E"] = synth.round_to_bf16_bits(E64.astype(np.float32))
+    E, C, y = to_dev(inp)
+    loss, lse, st = gpu_forward(E, C, y)
+    lse_t = torch.from_numpy(lse).cuda()
+    dloss = synth.random_dloss(27, w.N)
+    dl = torch.from_numpy(dloss).cuda()
+    ws = L.Workspace()
+    bE, bC = L.backward(E, C, y, lse_t, dl, eps, IGN, workspace=ws, stripes=True, bf16_grads=True)
+    assert bE.dtype == torch.bfloat16 and bC.dtype == torch.bfloat16
+    assert L.read_status(ws)["status"] == 0
+    fE, fC = L.backward(E, C, y, lse_t, dl, eps, IGN, workspace=L.Workspace(), stripes=True)   # fp32
+    # one rounding to bf16 of the same kind of sum: within a bf16 step
+    assert rel_fro(bE.float().cpu().numpy(), fE.cpu().numpy()) < 4e-3
+    assert rel_fro(bC.float().cpu().numpy(), fC.cpu().numpy()) < 4e-3
+    _, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    oE, oC = oracle.backward(inp["E"], inp["C"], inp["y"], olse, dloss, IGN, filter_eps=eps, tile=(1, 1))
+    assert rel_fro(bE.float().cpu().numpy(), oE) <= 1e-2
+    assert rel_fro(bC.float().cpu().numpy(), oC) <= 1e-2
+    # accumulation into existing bf16 gradients
+    gen = torch.Generator().manual_seed(5)
+    pE = (torch.randn(bE.shape, generator=gen) * float(bE.float().abs().max())).to(torch.bfloat16).cuda()
+    pC = (torch.randn(bC.shape, generator=gen) * float(bC.float().abs().max())).to(torch.bfloat16).cuda()
+    aE, aC = pE.clone(), pC.clone()
+    L.backward(E, C, y, lse_t, dl, eps, IGN, workspace=ws, out=(aE, aC), accumulate=True, stripes=True,
+               bf16_grads=True)
+    wE, wC = (pE.float() + fE).to(torch.bfloat16), (pC.float() + fC).to(torch.bfloat16)
+    assert rel_fro(aE.float().cpu().numpy(), wE.float().cpu().numpy()) < 4e-3
+    assert rel_fro(aC.float().cpu().numpy(), wC.float().cpu().numpy()) < 4e-3
