@@ -28,14 +28,18 @@
 // label entries afterwards; a flat half of a recomputed task gets zero rows),
 // and each A task flags its 256 x 256 G tile if it holds a kept entry, so a
 // B or C task streams only the K blocks (token blocks, resp. vocabulary
-// tiles) whose G tile is flagged; the mask travels with the task.
+// tiles) whose G tile is flagged; the mask travels with the task.  A task
+// left with nothing to do (an A task of two flat blocks, a dC task that adds
+// into dC with no flagged block, an unordered dE task with none) never
+// reaches the other roles: the producer retires it on the spot, raising its
+// completion counters by all of its arrivals.
 //
 // One persistent kernel runs all three kinds on clusters of two CTAs.  Tasks
 // are drawn in a fixed global order from a counter by the leader CTA's
 // producer thread, which also waits (bounded) until the task's inputs are
 // complete (counters in global memory, released by the epilogues that wrote
 // them), then hands the task to both CTAs through a small ring in shared
-// memory.  Roles per CTA (192 threads): warp 0 TMA producer, warp 1 UMMA
+// memory.  Roles per CTA (320 threads): warp 0 TMA producer, warp 1 UMMA
 // issuer (leader CTA only), warps 2-9 epilogue (two per TMEM lane group, one
 // per 128-column half).  Each CTA stages 32 KB of
 // operands per 64-wide K slice (5 stages) and double-buffers a 128 x 256 fp32
@@ -278,32 +282,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
           const int slot = k & (SP_RING - 1);
           if (!mbar_wait(&task_empty[slot], ((uint32_t)(k / SP_RING) & 1u) ^ 1u, wc)) goto producer_done;
           const uint64_t t_dep0 = trace ? global_timer_ns() : 0;
-          if (!next_known) look_ahead();
-          t = t_next;
-          next_known = false;
-          // wait until the task's inputs are complete (bounded)
-          if (t.type != TASK_END) {
-            if (dep_seen < dep_want) {
-              const uint64_t t0 = global_timer_ns();
-              bool ok = false;
-              while (true) {
-                __nanosleep(256);
-                if (ld_acquire_gpu(dep_ctr) >= dep_want) {
-                  ok = true;
-                  break;
+          // Draw until a task with work: a task with nothing to do (a
+          // recompute task of two flat blocks, a dC task that would add
+          // zeros, an unordered dE task with no live block) is retired here,
+          // its completion counters bumped for all its arrivals at once.
+          while (true) {
+            if (!next_known) look_ahead();
+            t = t_next;
+            next_known = false;
+            // wait until the task's inputs are complete (bounded)
+            if (t.type != TASK_END) {
+              if (dep_seen < dep_want) {
+                const uint64_t t0 = global_timer_ns();
+                bool ok = false;
+                while (true) {
+                  __nanosleep(256);
+                  if (ld_acquire_gpu(dep_ctr) >= dep_want) {
+                    ok = true;
+                    break;
+                  }
+                  if (*abort_flag) break;
+                  if (global_timer_ns() - t0 > a.wait_limit_ns) {
+                    *abort_flag = 1;
+                    break;
+                  }
                 }
-                if (*abort_flag) break;
-                if (global_timer_ns() - t0 > a.wait_limit_ns) {
-                  *abort_flag = 1;
-                  break;
-                }
+                if (!ok) goto producer_done;
               }
-              if (!ok) goto producer_done;
+              fence_proxy_async_global();  // the inputs were written by other CTAs' bulk stores
             }
-            fence_proxy_async_global();  // the inputs were written by other CTAs' bulk stores
+            tmask = live_mask(t);
+            const bool idle = tmask == 0ull && ((t.type == TASK_A) || (t.type == TASK_B && a.dC_add) ||
+                                                (t.type == TASK_C && !a.ordered));
+            if (!idle) break;
+            if (t.type == TASK_A) {
+              red_release_gpu_add(a.doneA_v + t.b, SP_DONE);
+              red_release_gpu_add(a.doneA_ms + (size_t)t.s * P.n_m2 + t.a, SP_DONE);
+            } else {
+              red_release_gpu_add(a.doneBC + t.s, SP_DONE);
+            }
+            drawn_next = atomicAdd(a.next, 1ull);
           }
           const int4 d = make_int4(t.type, t.s, t.a, t.b);
-          tmask = live_mask(t);
           const int4 dm = make_int4((int)(unsigned)tmask, (int)(unsigned)(tmask >> 32), 0, 0);
           task_slot[2 * slot] = d;
           task_slot[2 * slot + 1] = dm;
@@ -488,18 +508,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SP_THREADS, 1)
       tc_fence_after();
       if (trace && k < a.trace_cap) trace[k * 4 + 1] = global_timer_ns();
       const uint32_t tacc = tmem_base + lane_addr + (uint32_t)(acc * BN);
-      if (t.type == TASK_A && tmask == 0ull) {
-        // both token blocks flat: nothing was recomputed and nothing is stored
-        // (the G tile keeps its flag 0, so no B or C task reads it)
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-          red_release_gpu_add(a.doneA_v + t.b, 1u);
-          red_release_gpu_add(a.doneA_ms + (size_t)t.s * P.n_m2 + t.a, 1u);
-        }
-        __syncwarp();
-      } else if (t.type == TASK_A) {
+      if (t.type == TASK_A) {
+        // (an A task of two flat blocks never gets here: the producer retired
+        // it, and its G tile keeps flag 0, so no B or C task reads it)
         // row = token; columns = this warp's 128 of the 256 vocabulary entries of tile t.b
         const int row = a.tok0 + t.a * 256 + r * 128 + lg * 32 + lane;
         // a flat block's rows of G are zero: its label entries go to the flat-row kernel
