@@ -685,7 +685,8 @@ def run_gpu(args, w):
                            e_scale=args.e_scale,
                            backward_path=("stripes (CCE_BWD_STRIPES)" if args.bwd_stripes else
                                           "pre-pass, flat rows, tile kernel" if eps > 0 else "stripes"),
-                           forward_schedule=list(args.fwd_schedule) if args.fwd_schedule else None),
+                           forward_schedule=list(args.fwd_schedule) if args.fwd_schedule else None,
+                           forward_order=("round-robin" if args.fwd_order == 0 else "one queue per L2 half")),
             "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops (burst: the timed region is under a second)",
@@ -1096,6 +1097,8 @@ def main(argv=None):
                     help="forward schedule (A/B): vocabulary splits per token block and token blocks per raster "
                          "group (0 = chosen per shape), L2 hints of the pair kernel (bit 0: E evict_last, bit 1: C "
                          "evict_first), its operand stages (0 = default 7, or 6)")
+    ap.add_argument("--fwd-order", type=int, choices=[0, 1], default=None,
+                    help="unit order of the pair forward (A/B): 0 round-robin, 1 one queue per L2 half")
     ap.add_argument("--e-scale", type=float, default=None, metavar="F",
                     help="stress variant, not one of the workloads: E multiplied by F (a peaky softmax whose token "
                          "blocks are not flat)")
@@ -1117,7 +1120,8 @@ def main(argv=None):
                     help="per-workload table instead of the benchmark line (documentation)")
     args = ap.parse_args(argv)
     if args.impl == "cce" and (args.fwd_variant != "pair" or args.bwd_variant or args.prefetch or
-                               args.reduce_prefetch is not None or args.l2_hints or args.fwd_schedule):
+                               args.reduce_prefetch is not None or args.l2_hints or args.fwd_schedule or
+                               args.fwd_order is not None):
         import linear_cross_entropy_05_b200 as L
         L.cce_debug_set_forward_variant(1 if args.fwd_variant == "pair" else 0)
         L.cce_debug_set_backward_variant(args.bwd_variant)
@@ -1129,6 +1133,8 @@ def main(argv=None):
             L.cce_debug_set_l2_hints(True)
         if args.fwd_schedule:
             L.cce_debug_set_forward_schedule(*args.fwd_schedule)
+        if args.fwd_order is not None:
+            L.cce_debug_set_forward_order(args.fwd_order)
     if args.suite:
         return run_suite(args)
     if args.memory or args.trace:

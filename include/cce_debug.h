@@ -49,8 +49,9 @@ CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
  * n_split (0..256; 0 = chosen per shape: the fewest splits that minimise the
  * most-loaded worker's vocabulary tiles) is the number of vocabulary ranges
  * per token block, i.e. of (max, sum) partials per token; group_m (>= 0; 0 =
- * chosen per shape, ~48 MB of E rows) is the number of token blocks per
- * raster group; l2_hints (0..3, default 0; CTA-pair kernel only) gives the
+ * chosen per shape: ~48 MB of E rows in the round-robin order, ~24 MB per
+ * L2 half in the two-queue order) is the number of token blocks per raster
+ * group; l2_hints (0..3, default 0; CTA-pair kernel only) gives the
  * E slices the evict_last L2 policy (bit 0) and the C slices evict_first
  * (bit 1); stages (0 = the default 7, or 6 or 7; CTA-pair kernel only) is
  * the number of 32 KB operand stages per CTA (7 fill the 227 KB of shared
@@ -59,6 +60,38 @@ CCE_API cce_status_t cce_debug_set_prefetch(int fwd_slices, int bwd_slices);
  * changing it.  Process-wide.  Returns CCE_ERR_INVALID_ARG for other
  * values. */
 CCE_API cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hints, int stages);
+
+/* Unit order of the CTA-pair forward kernel, for A/B measurement.  0: the
+ * (token block, vocabulary split) units are dealt round-robin to the pairs.
+ * 1 (the default): two queues, one per L2 half of the GPU.  The L2 is split between the
+ * two dies, every line has a home half, and an SM reading a line homed in
+ * the other half keeps a copy in its own, so E (re-read for every vocabulary
+ * tile) fills both halves when every pair reads every token block.  Order 1
+ * gives each half its own token blocks (in proportion to its SMs; which SM
+ * is in which half is measured once per device and process by a small probe
+ * kernel, from the latency of atomics, which are served at a line's home),
+ * and the pairs draw units at run time from their half's queue, taking the
+ * other queue's units when theirs runs out or runs ahead.  Drawing units at
+ * run time also keeps the pairs that share C rows in step.  DRAM reads of
+ * one forward (ncu): 27.6 -> 8.1 GB on the Llama-3-8B-shaped head (16384 x
+ * 4096, V = 128256) and 141 -> 24 GB on the N = 65536 sweep, 8-12 % faster;
+ * no change on the Gemma-2-2B-shaped head (1.9 GB).  Each unit is computed
+ * the same way whoever computes it, so loss and lse are bitwise those of
+ * order 0; the split count may differ between the orders (the raster group
+ * enters its choice), so query cce_forward_workspace_size after changing
+ * the order.  Process-wide.  Returns CCE_ERR_INVALID_ARG for other
+ * values. */
+CCE_API cce_status_t cce_debug_set_forward_order(int order);
+
+/* The L2 half of each SM as the two-queue order's probe found it on the
+ * current device: half_of_sm[s] = 1 or 2 for SM id s (1: the half that is
+ * home to the probe's first line), 0 if not found (no forward in the
+ * two-queue order has run yet, or the SM's lines could not be told apart).
+ * Host memory, max_sms entries at most (SM ids 0..255 are kept).  Reads
+ * device memory synchronously: synchronize the stream of the forward first.
+ * Returns the number of entries written, or -1 (null pointer, max_sms <= 0,
+ * CUDA error). */
+CCE_API int cce_debug_l2_halves(int* half_of_sm, int max_sms);
 
 /* Tuning knobs of the dense stripe backward (CCE_BWD_STRIPES), for A/B
  * measurement: tokens_per_launch (a multiple of 256, at most 16384; 0 = the

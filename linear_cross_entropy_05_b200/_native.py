@@ -98,6 +98,10 @@ def load_library():
         lib.cce_debug_set_l2_hints.restype = ctypes.c_int
         lib.cce_debug_set_forward_schedule.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         lib.cce_debug_set_forward_schedule.restype = ctypes.c_int
+        lib.cce_debug_set_forward_order.argtypes = [ctypes.c_int]
+        lib.cce_debug_set_forward_order.restype = ctypes.c_int
+        lib.cce_debug_l2_halves.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+        lib.cce_debug_l2_halves.restype = ctypes.c_int
         lib.cce_debug_set_reduce_prefetch.argtypes = [ctypes.c_int]
         lib.cce_debug_set_reduce_prefetch.restype = ctypes.c_int
         lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 8 + [c_vp, c_i64]
@@ -337,3 +341,19 @@ def cce_debug_set_forward_schedule(n_split: int = 0, group_m: int = 0, l2_hints:
     operand stages per CTA (0 = default 7, or 6)."""
     _check(load_library().cce_debug_set_forward_schedule(int(n_split), int(group_m), int(l2_hints), int(stages)),
            "cce_debug_set_forward_schedule")
+
+
+def cce_debug_l2_halves(max_sms: int = 256) -> list:
+    """L2 half (1 or 2; 0 unknown) of SM ids 0 .. max_sms-1 on the current
+    device, as found by the two-queue forward's probe."""
+    buf = (ctypes.c_int * int(max_sms))()
+    n = load_library().cce_debug_l2_halves(buf, int(max_sms))
+    if n < 0:
+        raise RuntimeError("cce_debug_l2_halves failed")
+    return list(buf[:n])
+
+
+def cce_debug_set_forward_order(order: int) -> None:
+    """Unit order of the CTA-pair forward (A/B): 0 round-robin, 1 one queue
+    per L2 half of the GPU (same results bit for bit)."""
+    _check(load_library().cce_debug_set_forward_order(int(order)), "cce_debug_set_forward_order")

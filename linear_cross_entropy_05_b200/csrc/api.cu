@@ -21,6 +21,8 @@
 namespace cce {
 cudaError_t launch_fwd_lse(const CUtensorMap& tmE, const CUtensorMap& tmC, const FwdArgs& a, int grid,
                            cudaStream_t stream);
+cudaError_t launch_l2_half_probe(int sms, cudaStream_t stream);
+cudaError_t read_l2_halves(unsigned* out, int n);
 cudaError_t launch_fwd_lse_pair(const CUtensorMap& tmE, const CUtensorMap& tmCh, const FwdArgs& a, int grid,
                                 int stages, cudaStream_t stream);
 cudaError_t launch_fwd_finalize(const void* E, const void* C, const int64_t* y, const FinArgs& a, float* loss,
@@ -64,6 +66,9 @@ std::atomic<int> g_fwd_split{0};     // forward vocabulary splits per token bloc
 std::atomic<int> g_fwd_group_m{0};   // forward token blocks per raster group (0: chosen per shape)
 std::atomic<int> g_fwd_l2_hints{0};  // forward CTA-pair kernel: L2 eviction priorities (A/B)
 std::atomic<int> g_fwd_stages{PAIR_STAGES_MAX};  // forward CTA-pair kernel: operand stages per CTA
+std::atomic<int> g_fwd_order{1};     // forward CTA-pair kernel: 0 round-robin units, 1 one queue per L2 half
+constexpr int kMaxDevices = 64;
+std::atomic<bool> g_l2_probed[kMaxDevices];  // the L2-half probe was launched on this device
 std::atomic<int> g_bwd_pf{0};
 std::atomic<int> g_bwd_red_pf{0};  // L2 prefetch distance (K slices) of the backward's reduction targets
 std::atomic<int> g_bwd_l2_hints{0};  // L2 eviction priorities in the filtered backward (A/B)
@@ -235,8 +240,14 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
   const int workers = p->pair ? di.sms / 2 : di.sms;  // CTA pairs or CTAs
   p->n_mblk = (int)((N + rows - 1) / rows);
   p->n_vtile = (int)((V + BN - 1) / BN);
-  // keep at most ~48 MB of E rows in flight so they stay resident in the 126 MB L2
-  p->group_m = (int)std::max<int64_t>(1, std::min<int64_t>(p->n_mblk, (48ll << 20) / ((int64_t)rows * D * 2)));
+  // Token blocks per raster group.  Round-robin order: ~48 MB of E rows in
+  // flight.  Two-queue order (CTA pairs): ~24 MB per group of each L2 half;
+  // the halves' groups are in flight together, and every line read by the
+  // other half also has a copy in its home half, so each half holds about
+  // 1.5 x that of E next to the C tiles being streamed.
+  const bool two_queues = p->pair && g_fwd_order.load() == 1;
+  p->group_m = (int)std::max<int64_t>(
+      1, std::min<int64_t>(p->n_mblk, ((two_queues ? 24ll : 48ll) << 20) / ((int64_t)rows * D * 2)));
   if (g_fwd_group_m.load() > 0) p->group_m = std::min(p->n_mblk, g_fwd_group_m.load());
   p->n_split = g_fwd_split.load() > 0 ? std::min(p->n_vtile, g_fwd_split.load())
                                       : choose_splits(p->n_mblk, p->n_vtile, workers, p->group_m);
@@ -392,6 +403,17 @@ cce_status_t forward_impl(const void* E, const void* C, const int64_t* y, int64_
   a.withhold_loads = g_withhold_loads.load();
   a.pf = g_fwd_pf.load();
   a.l2_hints = g_fwd_l2_hints.load();
+  a.sched = p.pair ? g_fwd_order.load() : 0;
+  if (a.sched) {
+    // which L2 half each SM is in: found once per device and process (the
+    // first launch on a stream being captured goes into the graph, where it
+    // changes nothing when replayed); until it has run, pairs alternate
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CCE_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && !g_l2_probed[dev].exchange(true) &&
+        launch_l2_half_probe(device_info().sms, stream) != cudaSuccess)
+      return CCE_ERR_CUDA;
+  }
   if (record_event(0, 0, stream) != cudaSuccess) return CCE_ERR_CUDA;
   const cudaError_t le =
       p.pair ? launch_fwd_lse_pair(tmE, tmC, a, p.grid, g_fwd_stages.load(), stream)
@@ -470,6 +492,21 @@ cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hin
   g_fwd_group_m.store(group_m);
   g_fwd_l2_hints.store(l2_hints);
   g_fwd_stages.store(stages ? stages : PAIR_STAGES_MAX);
+  return CCE_OK;
+}
+
+int cce_debug_l2_halves(int* half_of_sm, int max_sms) {
+  if (!half_of_sm || max_sms <= 0) return -1;
+  const int n = std::min(max_sms, 256);
+  std::vector<unsigned> h((size_t)n, 0u);
+  if (read_l2_halves(h.data(), n) != cudaSuccess) return -1;
+  for (int i = 0; i < n; ++i) half_of_sm[i] = (int)h[(size_t)i];
+  return n;
+}
+
+cce_status_t cce_debug_set_forward_order(int order) {
+  if (order < 0 || order > 1) return CCE_ERR_INVALID_ARG;
+  g_fwd_order.store(order);
   return CCE_OK;
 }
 
@@ -935,6 +972,6 @@ const char* cce_status_string(cce_status_t s) {
   return "CCE_ERR_UNKNOWN";
 }
 
-int cce_version(void) { return 102; }
+int cce_version(void) { return 103; }
 
 }  // extern "C"

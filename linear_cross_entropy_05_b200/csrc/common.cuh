@@ -26,7 +26,8 @@ constexpr int G_BYTES = BM * BN * 2;        // bf16 softmax-gradient tile (4 swi
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
-// Status block at the head of every workspace (8 x u64, zeroed per call).
+// Status block at the head of every workspace (32 x u64, zeroed per call;
+// cce_read_status reads words 0-7).
 enum StatusWord : int {
   ST_FLAGS = 0,        // bit mask of StatusFlag
   ST_LIVE_TILES = 1,   // backward: 32x32 filter units whose contraction ran
@@ -35,6 +36,7 @@ enum StatusWord : int {
   ST_PRUNED = 4,       // backward: filter units proven negligible without recomputing them
   ST_NEXT_TILE = 5,    // backward: next work item to hand out (CTAs take tiles as they free up)
   ST_FLAT = 6,         // backward: live units of flat blocks, formed without recomputing a tile
+  ST_FWD_QUEUE = 8,    // forward, two-queue order: next unit of queue 0 (word 8) and queue 1 (word 9)
 };
 // Header words of the backward pre-pass (u32, after the status block).
 enum PrepHeader : int {
@@ -66,6 +68,12 @@ struct FwdArgs {
   int withhold_loads;          // test hook: the TMA producer issues nothing
   int pf;                      // L2 prefetch distance of the C stream in K slices (0: off)
   int l2_hints;                // CTA-pair kernel: bit 0 E slices evict_last, bit 1 C slices evict_first
+  // CTA-pair kernel, unit order.  0: units dealt round-robin to the pairs.
+  // 1: two queues, one per L2 half: the token blocks are split between the
+  // halves of the GPU (in proportion to their SMs), each pair draws units of
+  // its own half's blocks at run time, and takes the other queue's units when
+  // its own runs out or runs more than one vocabulary split ahead.
+  int sched;
 };
 
 struct FinArgs {

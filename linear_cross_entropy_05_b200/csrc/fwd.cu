@@ -16,6 +16,13 @@
 // fwd_lse_pair_kernel  the same on clusters of two CTAs (the default): one
 //                 256 x 256 logit tile per pair through tcgen05 cta_group::2,
 //                 each CTA loading 128 rows of E and 128 rows of C per slice.
+//                 Units are dealt round-robin, or (two-queue order) drawn at
+//                 run time from one queue per L2 half of the GPU, so that each
+//                 half keeps only its own token blocks' E rows in its L2.
+// l2_half_probe   tells the two L2 halves apart once per process: per SM,
+//                 the latency of atomics on eight lines 4 KB apart (an atomic
+//                 is served where its line is homed, ~2.5x faster in the SM's
+//                 own half).
 // fwd_finalize    one warp per token: merges the split partials into lse,
 //                 forms the correct-token logit E_i . C_{y_i} with coalesced
 //                 16-byte loads, and writes loss = lse - z_y (0 if ignored).
@@ -264,6 +271,72 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 
 // ----------------------------------------------------------------------------
+// L2 halves.  The L2 of this GPU is split between its two dies: every line has
+// a home half, and an SM that reads a line homed in the other half keeps a
+// copy in its own half.  Data that all SMs read (E, re-read for every
+// vocabulary tile) therefore fills both halves, and at N = 8192 on the 256K
+// vocabulary (37.7 MB of E) C is streamed from DRAM 1.7 times instead of once
+// (1.15 times at N = 2048).  The two-queue order gives each half its own token
+// blocks; this kernel finds which half each SM belongs to.
+//
+// An atomic is performed at the line's home, so its latency tells near from
+// far (about 260 against 690 SM cycles at 1.97 GHz).  Each block times short
+// chains of atomics (adding 0) on eight lines 4 KB apart, which the home hash
+// spreads over both halves; lines faster than the midpoint of its fastest and
+// slowest are near.  The SM's half is then "line 0 is near" (1) or not (2).
+// If no two lines differ by 1.5x the SM stays unknown (0).  The tables live
+// as long as the process; a table entry is written once (compare-and-swap),
+// so the kernel may run again (a replayed graph) without changing anything.
+// ----------------------------------------------------------------------------
+constexpr int kMaxSmid = 256;
+__device__ __align__(4096) unsigned long long g_l2_probe[8 * 512];  // 8 lines, 4 KB apart
+__device__ unsigned g_sm_half[kMaxSmid];                            // 0 unknown, 1 or 2
+__device__ unsigned g_half_sms[2];                                  // SMs found in half 1, half 2
+
+__device__ __forceinline__ unsigned sm_id() {
+  unsigned s;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(s));
+  return s;
+}
+
+__global__ void __launch_bounds__(32) l2_half_probe_kernel() {
+  if (threadIdx.x != 0) return;
+  const unsigned smid = sm_id();
+  if (smid >= (unsigned)kMaxSmid || *(volatile unsigned*)&g_sm_half[smid] != 0u) return;
+  long long lat[8];
+  unsigned long long v = 0ull;
+  for (int j = 0; j < 8; ++j) {
+    const int line = (blockIdx.x + j) & 7;  // blocks start on different lines
+    unsigned long long* p = g_l2_probe + line * 512;
+    const long long c0 = clock64();
+    for (int s = 0; s < 3; ++s) {
+      // each address depends on the previous result (v >> 63 is 0: the lines hold 0)
+      asm volatile("atom.global.add.u64 %0, [%1], 0;" : "=l"(v) : "l"(p + (v >> 63)) : "memory");
+    }
+    lat[line] = clock64() - c0 + (long long)(v >> 63);
+  }
+  long long mn = lat[0], mx = lat[0];
+  for (int j = 1; j < 8; ++j) {
+    mn = min(mn, lat[j]);
+    mx = max(mx, lat[j]);
+  }
+  if (2 * mx < 3 * mn) return;  // the lines could not be told apart
+  const unsigned half = 2 * lat[0] < mn + mx ? 1u : 2u;
+  if (atomicCAS(&g_sm_half[smid], 0u, half) == 0u) atomicAdd(&g_half_sms[half - 1], 1u);
+}
+
+cudaError_t launch_l2_half_probe(int sms, cudaStream_t stream) {
+  // four blocks per SM, so that every SM is all but certain to run one
+  l2_half_probe_kernel<<<4 * sms, 32, 0, stream>>>();
+  return cudaGetLastError();
+}
+
+// Copies the half of SMs 0 .. n-1 (0 unknown, 1, 2) to host memory.
+cudaError_t read_l2_halves(unsigned* out, int n) {
+  return cudaMemcpyFromSymbol(out, g_sm_half, (size_t)n * sizeof(unsigned));
+}
+
+// ----------------------------------------------------------------------------
 // CTA-pair variant: a cluster of two CTAs on two SMs computes 256 x 256 logit
 // tiles with tcgen05.mma.cta_group::2 (M = 256 split over the pair).  Each CTA
 // loads its own 128 token rows of E and 128 vocabulary rows of C per stage
@@ -288,8 +361,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tfull = bars + 2 * S;   // each CTA: accumulator ready
   uint64_t* tempty = tfull + 2;               // leader: both epilogues done with the accumulator
   uint64_t* drain = tempty + 2;               // leader: UMMA drain at exit
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* unit_full = drain + 1;            // each CTA [2]: two-queue order, a unit was published
+  uint64_t* unit_empty = unit_full + 2;       // leader [2]: every consumer has read the slot
+  int4* unit_slot = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(unit_empty + 2) + 15) & ~uintptr_t(15));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_slot + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  // readers of a published unit: the leader's MMA thread and 4 epilogue
+  // warps, the peer's producer and 4 epilogue warps
+  constexpr uint32_t UNIT_CONSUMERS = 10;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -306,6 +385,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 8);  // one arrival per epilogue warp of both CTAs
+      mbar_init(&unit_full[b], 1);
+      mbar_init(&unit_empty[b], UNIT_CONSUMERS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -326,6 +407,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const WaitCtl wc{abort_flag, a.wait_limit_ns};
   const int nkb = (a.D + BK - 1) / BK;
 
+  // Round-robin order: unit k of this pair is pair + k * n_pairs.  Two-queue
+  // order: the leader's producer draws each unit and publishes its (split,
+  // token block) to both CTAs through a two-slot ring; r < 0 ends the stream.
+  auto static_unit = [&](int k, int& r, int& m2) -> bool {
+    const int u = pair + k * n_pairs;
+    if (u >= a.n_units) return false;
+    unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m2);
+    return true;
+  };
+  const uint32_t unit_empty_leader = mapa_shared(smem_u32(&unit_empty[0]), 0);
+  // Reads published unit k (bounded wait) and frees the slot on the leader.
+  // With whole_warp, lane 0 waits and reads and the warp follows its outcome.
+  auto take_unit = [&](int k, int& r, int& m2, bool whole_warp) -> bool {
+    const int slot = k & 1;
+    int ok = 1, rr = -1, mm = -1;
+    if (!whole_warp || lane == 0) {
+      ok = mbar_wait_cluster(&unit_full[slot], (uint32_t)(k >> 1) & 1u, wc) ? 1 : 0;
+      if (ok) {
+        const volatile int* vs = reinterpret_cast<const volatile int*>(&unit_slot[slot]);
+        rr = vs[0];
+        mm = vs[1];
+        mbar_arrive_cluster(unit_empty_leader + (uint32_t)(slot * 8));
+      }
+    }
+    if (whole_warp) {
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      rr = __shfl_sync(0xffffffffu, rr, 0);
+      mm = __shfl_sync(0xffffffffu, mm, 0);
+    }
+    r = rr;
+    m2 = mm;
+    return ok != 0;
+  };
+
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs) ----------------
@@ -335,9 +450,83 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       // tile) kept, C (read by every token block in turn) evicted first
       const uint64_t pol_e = l2_policy_evict_last(), pol_c = l2_policy_evict_first();
       const bool hint_e = (a.l2_hints & 1) != 0, hint_c = (a.l2_hints & 2) != 0;
-      for (int u = a.withhold_loads ? a.n_units : pair; u < a.n_units; u += n_pairs) {
-        int r, m2;
-        unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m2);
+      // Two-queue order (leader): queue q holds the units of token blocks
+      // [m_lo[q], m_lo[q] + nq[q]), split-major in raster groups, and the
+      // token blocks are divided between the queues in proportion to the
+      // SMs of each L2 half.  The pair serves the queue of its own half.
+      int own = 0, nq[2] = {0, 0}, m_lo[2] = {0, 0}, gm_q[2] = {1, 1};
+      long long units_q[2] = {0, 0};
+      unsigned long long* qctr = a.status + ST_FWD_QUEUE;
+      if (a.sched && leader) {
+        const unsigned c1 = *(volatile unsigned*)&g_half_sms[0], c2 = *(volatile unsigned*)&g_half_sms[1];
+        int m_half = a.n_mblk / 2;
+        if (c1 != 0u && c2 != 0u)
+          m_half = (int)(((long long)a.n_mblk * c1 + (c1 + c2) / 2) / (c1 + c2));
+        m_half = max(0, min(a.n_mblk, m_half));
+        const unsigned smid = sm_id();
+        unsigned h = smid < (unsigned)kMaxSmid ? *(volatile unsigned*)&g_sm_half[smid] : 0u;
+        if (h == 0u) h = 1u + (unsigned)(pair & 1);  // half unknown: alternate
+        own = (int)h - 1;
+        nq[0] = m_half;
+        nq[1] = a.n_mblk - m_half;
+        m_lo[1] = m_half;
+        for (int q = 0; q < 2; ++q) {
+          units_q[q] = (long long)nq[q] * a.n_split;
+          // raster groups of at most group_m blocks, as even as possible
+          const int ng = max(1, (nq[q] + a.group_m - 1) / a.group_m);
+          gm_q[q] = max(1, (nq[q] + ng - 1) / ng);
+        }
+      }
+      // Next unit of the two-queue order.  The own queue first, unless it is
+      // more than one split ahead of the other (units are split-major inside
+      // a raster group, gm_q per split): then the other queue's, so both
+      // halves walk the vocabulary together and C rows are read by both while
+      // in L2.  When one queue is empty the other's units are taken.
+      auto draw = [&](int& r, int& m2) -> bool {
+        const int other = 1 - own;
+        int first = own;
+        if (units_q[own] > 0 && units_q[other] > 0) {
+          const long long io = (long long)*(volatile unsigned long long*)(qctr + own);
+          const long long ix = (long long)*(volatile unsigned long long*)(qctr + other);
+          if (ix < units_q[other] && io * gm_q[other] > (ix + gm_q[other]) * gm_q[own]) first = other;
+        }
+        for (int t = 0; t < 2; ++t) {
+          const int q = t == 0 ? first : 1 - first;
+          if (units_q[q] == 0) continue;
+          const unsigned long long i = atomicAdd(qctr + q, 1ull);
+          if (i < (unsigned long long)units_q[q]) {
+            int mloc;
+            unit_coords((int)i, nq[q], a.n_split, gm_q[q], r, mloc);
+            m2 = m_lo[q] + mloc;
+            return true;
+          }
+        }
+        return false;
+      };
+      // publishes unit k (r < 0: the end) to both CTAs
+      auto publish = [&](int k, int r, int m2) -> bool {
+        const int slot = k & 1;
+        if (!mbar_wait(&unit_empty[slot], ((uint32_t)(k >> 1) & 1u) ^ 1u, wc)) return false;
+        const int4 d = make_int4(r, m2, 0, 0);
+        unit_slot[slot] = d;
+        st_shared_cluster_v4(mapa_shared(smem_u32(&unit_slot[slot]), 1), d);
+        mbar_arrive(&unit_full[slot]);
+        mbar_arrive_release_cluster(mapa_shared(smem_u32(&unit_full[slot]), 1));
+        return true;
+      };
+      if (a.withhold_loads) goto producer_done;  // test hook: nothing is loaded or published
+      for (int k = 0;; ++k) {
+        int r = -1, m2 = -1;
+        if (!a.sched) {
+          if (!static_unit(k, r, m2)) break;
+        } else if (leader) {
+          if (!draw(r, m2)) r = m2 = -1;
+          if (!publish(k, r, m2)) goto producer_done;
+          if (r < 0) break;
+        } else {
+          if (!take_unit(k, r, m2, false)) goto producer_done;
+          if (r < 0) break;
+        }
         int v0, v1;
         split_range(r, a.n_vtile, a.n_split, v0, v1);
         for (int vt = v0; vt < v1; ++vt) {
@@ -390,9 +579,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int u = pair; u < a.n_units; u += n_pairs) {
+      for (int k = 0;; ++k) {
         int r, m2;
-        unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m2);
+        if (!a.sched) {
+          if (!static_unit(k, r, m2)) break;
+        } else {
+          if (!take_unit(k, r, m2, false)) goto mma_done;
+          if (r < 0) break;
+        }
         int v0, v1;
         split_range(r, a.n_vtile, a.n_split, v0, v1);
         for (int vt = v0; vt < v1; ++vt) {
@@ -438,9 +632,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = pair; u < a.n_units; u += n_pairs) {
+    for (int k = 0;; ++k) {
       int r, m2;
-      unit_coords(u, a.n_mblk, a.n_split, a.group_m, r, m2);
+      if (!a.sched) {
+        if (!static_unit(k, r, m2)) break;
+      } else {
+        if (!take_unit(k, r, m2, true)) break;
+        if (r < 0) break;
+      }
       int v0, v1;
       split_range(r, a.n_vtile, a.n_split, v0, v1);
       const int row = m2 * (2 * BM) + (int)rank * BM + row_in_blk;

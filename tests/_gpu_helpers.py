@@ -11,6 +11,7 @@ GRAD_REL_FILTER_OFF = 5e-3   # dE, dC relative Frobenius error, filter off
 GRAD_REL_FILTER_ON = 1e-2    # dE, dC relative Frobenius error, filter on (vs the exact gradient)
 
 DEFAULT_FWD_VARIANT = 1      # the library's default forward kernel: CTA pairs (tcgen05 cta_group::2)
+DEFAULT_FWD_ORDER = 1        # the pair kernel's default unit order (0 round-robin, 1 one queue per L2 half)
 
 
 def filter_on_bar(V):

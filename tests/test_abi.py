@@ -194,6 +194,16 @@ def test_shard_entry_points_validate_on_the_host(lib):
                               check=False) == 1
 
 
+def test_forward_order_knob_validates_on_the_host(lib):
+    import ctypes
+    assert lib.cce_debug_l2_halves(None, 4) == -1
+    assert lib.cce_debug_l2_halves((ctypes.c_int * 4)(), 0) == -1
+    assert lib.cce_debug_set_forward_order(-1) == 1
+    assert lib.cce_debug_set_forward_order(2) == 1
+    assert lib.cce_debug_set_forward_order(1) == 0
+    assert lib.cce_debug_set_forward_order(0) == 0
+
+
 def test_forward_schedule_knob_validates_on_the_host(lib):
     assert lib.cce_debug_set_forward_schedule(257, 0, 0, 0) == 1      # more than 256 splits
     assert lib.cce_debug_set_forward_schedule(0, -1, 0, 0) == 1

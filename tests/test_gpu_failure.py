@@ -12,7 +12,7 @@ import pytest
 import oracle
 from linear_cross_entropy_05_b200 import synth
 
-from _gpu_helpers import DEFAULT_FWD_VARIANT, IGN, LOSS_ABS, gpu_backward, gpu_forward, rel_fro, to_dev
+from _gpu_helpers import DEFAULT_FWD_ORDER, DEFAULT_FWD_VARIANT, IGN, LOSS_ABS, gpu_backward, gpu_forward, rel_fro, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -31,8 +31,12 @@ def test_withheld_loads_end_with_timeout_status_and_a_usable_context():
     L.cce_debug_set_wait_limit_ns(20_000_000)       # 20 ms per wait
     L.cce_debug_withhold_loads(True)
     try:
-        for variant in (0, 1):   # single-CTA and CTA-pair forward kernels
+        # single-CTA kernel; CTA-pair kernel with units dealt round-robin and
+        # drawn from the two queues (there the ring of published units is
+        # never fed either: every reader's wait gives up)
+        for variant, order in ((0, 0), (1, 0), (1, 1)):
             L.cce_debug_set_forward_variant(variant)
+            L.cce_debug_set_forward_order(order)
             ws = L.Workspace()
             l_t, s_t = L.forward(E, C, y, IGN, workspace=ws)
             st = L.read_status(ws)
@@ -40,6 +44,7 @@ def test_withheld_loads_end_with_timeout_status_and_a_usable_context():
             # partials were never written: the call's outputs are NaN, not stale values
             assert torch.isnan(l_t).all() and torch.isnan(s_t).all()
         L.cce_debug_set_forward_variant(DEFAULT_FWD_VARIANT)
+        L.cce_debug_set_forward_order(DEFAULT_FWD_ORDER)
         # filter off through the stripe kernel and through the fused kernel,
         # filter on (an eps far below every entry: no token block is flat, so
         # the tile kernel recomputes, and waits on, every tile)
@@ -50,6 +55,7 @@ def test_withheld_loads_end_with_timeout_status_and_a_usable_context():
             assert st["status"] == CCE_ERR_TIMEOUT and st["flags"] & 1
     finally:
         L.cce_debug_set_forward_variant(DEFAULT_FWD_VARIANT)
+        L.cce_debug_set_forward_order(DEFAULT_FWD_ORDER)
         L.cce_debug_withhold_loads(False)
         L.cce_debug_set_wait_limit_ns(1_000_000_000)
     torch.cuda.synchronize()

@@ -7,7 +7,7 @@ import pytest
 import oracle
 from linear_cross_entropy_05_b200 import synth
 
-from _gpu_helpers import DEFAULT_FWD_VARIANT, IGN, LOSS_ABS, MEAN_REL, gpu_forward, mean_of, to_dev
+from _gpu_helpers import DEFAULT_FWD_ORDER, DEFAULT_FWD_VARIANT, IGN, LOSS_ABS, MEAN_REL, gpu_forward, mean_of, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -217,6 +217,64 @@ def test_forward_schedule_knobs_keep_the_result(sched):
     ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
     assert np.abs(loss - ol).max() <= LOSS_ABS
     assert np.abs(lse - olse).max() <= LOSS_ABS
+
+
+@pytest.mark.parametrize("shape,sched", [
+    ((1300 + 77, 20000 + 77, 512), (37, 0, 0, 0)),  # ragged N and V, an odd number of 256-token blocks
+    ((200, 9000 + 5, 256), (5, 0, 0, 0)),           # one token block: one queue is empty
+    ((4096 + 100, 30000, 512), (64, 2, 0, 0)),      # raster groups inside each queue, many splits
+    ((2048 + 256, 5000, 128), (1, 0, 0, 0)),        # one split: a unit is a whole token block
+], ids=["ragged", "one-token-block", "groups-of-2-64-splits", "one-split"])
+def test_two_queue_order_gives_the_same_bits(shape, sched):
+    # the two-queue order changes which pair computes a unit and when, not
+    # how: every unit folds its vocabulary tiles in the same order, so with
+    # the same split count the loss, lse and row maxima are bit for bit those
+    # of the round-robin order
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    N, V, D = shape
+    w = synth.GEMMA2_2B.with_sizes(N=N, V=V, D=D)
+    inp = synth.make_inputs(w)
+    E, C, y = to_dev(inp)
+    out = {}
+    L.cce_debug_set_forward_schedule(*sched)
+    try:
+        for order in (0, 1, 1):   # the second order-1 call runs with the L2 halves known
+            L.cce_debug_set_forward_order(order)
+            rm = torch.full((N,), float("nan"), device="cuda")
+            loss, lse = L.forward(E, C, y, IGN, row_max=rm)
+            out.setdefault(order, []).append((loss, lse, rm))
+    finally:
+        L.cce_debug_set_forward_order(DEFAULT_FWD_ORDER)
+        L.cce_debug_set_forward_schedule(0, 0, 0, 0)
+    ref = out[0][0]
+    for got in out[1]:
+        for a, b in zip(ref, got):
+            assert torch.equal(a, b)
+    ol, olse = oracle.forward(inp["E"], inp["C"], inp["y"], IGN)
+    assert np.abs(ref[0].cpu().numpy() - ol).max() <= LOSS_ABS
+
+
+def test_l2_half_probe_finds_two_halves():
+    # the probe behind the two-queue order sorts the SMs by where atomics on
+    # its eight lines are fast; a B200's L2 is split between its two dies,
+    # so it must find two non-empty halves covering (nearly) every SM
+    import torch
+    import linear_cross_entropy_05_b200 as L
+    w = synth.GEMMA2_2B.with_sizes(N=600, V=5000, D=256)
+    E, C, y = to_dev(synth.make_inputs(w))
+    L.cce_debug_set_forward_order(1)
+    try:
+        L.forward(E, C, y, IGN)
+    finally:
+        L.cce_debug_set_forward_order(DEFAULT_FWD_ORDER)
+    torch.cuda.synchronize()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    halves = L.cce_debug_l2_halves(256)
+    assert set(halves) <= {0, 1, 2}
+    n1, n2 = halves.count(1), halves.count(2)
+    print(f"L2 halves: {n1} + {n2} of {sms} SMs")
+    assert n1 > 0 and n2 > 0 and n1 + n2 >= sms - 4
 
 
 def test_forward_ex_writes_each_tokens_largest_logit():
