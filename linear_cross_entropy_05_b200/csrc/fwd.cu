@@ -514,15 +514,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive_release_cluster(mapa_shared(smem_u32(&unit_full[slot]), 1));
         return true;
       };
+      // The leader draws one unit ahead: the next unit is drawn after the
+      // first load of the current one, while the stages are full, so the
+      // round trips of the draw never stall the operand stream at a unit
+      // boundary.
+      int next_r = -1, next_m2 = -1;
+      bool draw_pending = false;
       if (a.withhold_loads) goto producer_done;  // test hook: nothing is loaded or published
+      if (a.sched && leader && !draw(next_r, next_m2)) next_r = next_m2 = -1;
       for (int k = 0;; ++k) {
         int r = -1, m2 = -1;
         if (!a.sched) {
           if (!static_unit(k, r, m2)) break;
         } else if (leader) {
-          if (!draw(r, m2)) r = m2 = -1;
+          r = next_r;
+          m2 = next_m2;
           if (!publish(k, r, m2)) goto producer_done;
           if (r < 0) break;
+          draw_pending = true;
         } else {
           if (!take_unit(k, r, m2, false)) goto producer_done;
           if (r < 0) break;
@@ -545,6 +554,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             else
               tma_load_2d_pair(dB, &tmCh, &full[stage], kb * BK, yC);
             armed |= 1u << stage;
+            if (draw_pending) {
+              if (!draw(next_r, next_m2)) next_r = next_m2 = -1;
+              draw_pending = false;
+            }
             // L2 prefetch of this CTA's C rows a.pf slices ahead in the unit's
             // stream, by the pair on the first token block of the raster group
             // only (the other pairs on this split read the same rows)
@@ -558,6 +571,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               phase ^= 1u;
             }
           }
+        }
+        if (draw_pending) {  // a unit without loads (not reached: every split has a tile, D >= 8)
+          if (!draw(next_r, next_m2)) next_r = next_m2 = -1;
+          draw_pending = false;
         }
       }
     producer_done:
