@@ -278,12 +278,14 @@ def measured_peaks():
 
 
 def kernel_source_hash(which: str) -> str:
-    """Hash of the code of a kernel's sources, comments and blank lines
-    removed (a comment edit does not change the kernel the counters came from)."""
+    """Hash of the code of a kernel's sources and of the host code that plans
+    its launches (split counts, unit orders: they change the traffic too),
+    comments and blank lines removed (a comment edit does not change the
+    kernel the counters came from)."""
     import re
     base = os.path.join(ROOT, "linear_cross_entropy_05_b200", "csrc")
     h = hashlib.sha256()
-    for f in (f"{which}.cu", "common.cuh", "ptx.cuh"):
+    for f in (f"{which}.cu", "common.cuh", "ptx.cuh", "api.cu"):
         with open(os.path.join(base, f)) as fh:
             src = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
         for line in src.splitlines():

@@ -72,10 +72,11 @@ CCE_API cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, in
  * kernel, from the latency of atomics, which are served at a line's home),
  * and the pairs draw units at run time from their half's queue, taking the
  * other queue's units when theirs runs out or runs ahead.  Drawing units at
- * run time also keeps the pairs that share C rows in step.  DRAM reads of
- * one forward (ncu): 27.6 -> 8.1 GB on the Llama-3-8B-shaped head (16384 x
- * 4096, V = 128256) and 141 -> 24 GB on the N = 65536 sweep, 8-12 % faster;
- * no change on the Gemma-2-2B-shaped head (1.9 GB).  Each unit is computed
+ * run time also keeps the pairs that share C rows in step, and the units are
+ * short (at most ~8 vocabulary tiles).  DRAM reads of one forward (ncu):
+ * 1.9-2.9 -> 1.23 GB on the Gemma-2-2B-shaped head (C read once), 27.6 ->
+ * 6.0 GB on the Llama-3-8B-shaped head (16384 x 4096, V = 128256), 141 ->
+ * 7.6 GB on the N = 65536 sweep; the last two 10-14 % faster.  Each unit is computed
  * the same way whoever computes it, so loss and lse are bitwise those of
  * order 0; the split count may differ between the orders (the raster group
  * enters its choice), so query cce_forward_workspace_size after changing
