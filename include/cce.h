@@ -78,8 +78,10 @@ typedef struct {
 
 /* Workspace bytes needed by cce_forward for these sizes on the current device
  * (N * splits * 8 bytes of per-split (max, sum) pairs plus a 256-byte status
- * block, splits <= 64).  Returns 0 if the sizes are invalid or no device is
- * usable. */
+ * block; splits <= 128, or up to 256 when cce_debug_set_forward_schedule
+ * asks for them; 125 on a 256000-entry vocabulary).  Depends on the debug
+ * schedule knobs in force.  Returns 0 if the sizes are invalid or no device
+ * is usable. */
 CCE_API size_t cce_forward_workspace_size(int64_t N, int64_t D, int64_t V);
 
 /* Workspace bytes needed by cce_backward: the status block plus the
