@@ -94,6 +94,16 @@ CCE_API cce_status_t cce_debug_set_forward_order(int order);
  * CUDA error). */
 CCE_API int cce_debug_l2_halves(int* half_of_sm, int max_sms);
 
+/* The forward's launch plan for these sizes on a GPU with `sms` SMs, as
+ * cce_forward would choose it under the knobs in force (host arithmetic
+ * only: no device needed).  out[6] (host memory) receives: 1 if the
+ * CTA-pair kernel runs, the token blocks (of 256 rows for pairs, 128
+ * otherwise), the 256-wide vocabulary tiles, the vocabulary splits, the
+ * token blocks per raster group, and the grid in CTAs.  The workspace is
+ * 256 + N * splits * 8 bytes, rounded up to 256.  Returns 0, or -1 for
+ * invalid sizes, sms <= 0 or a null pointer. */
+CCE_API int cce_debug_forward_plan(int64_t N, int64_t D, int64_t V, int sms, int* out);
+
 /* Tuning knobs of the dense stripe backward (CCE_BWD_STRIPES), for A/B
  * measurement: tokens_per_launch (a multiple of 256, at most 16384; 0 = the
  * default 16384) bounds the tokens one launch takes (fewer tokens per launch

@@ -25,7 +25,7 @@ from . import _native
 from ._native import (CCE_BWD_ACCUMULATE, CCE_BWD_BF16_GRADS, CCE_BWD_DETERMINISTIC, CCE_BWD_PREPARED,
                       CCE_BWD_STRIPES, CCE_BWD_ROW_MAX, CCEError, cce_forward_ex, cce_backward_prepare_rows, cce_debug_stripe_schedule, cce_debug_set_reduce_prefetch,
                       cce_debug_set_stripe_params, cce_debug_set_l2_hints, cce_debug_set_forward_schedule,
-                      cce_debug_set_forward_order, cce_debug_l2_halves,
+                      cce_debug_set_forward_order, cce_debug_l2_halves, cce_debug_forward_plan,
                       cce_debug_set_stripe_order,
                       cce_backward, cce_backward_ex, cce_backward_prepare,
                       cce_backward_shard, cce_backward_workspace_size, cce_backward_workspace_size_ex,
@@ -41,7 +41,7 @@ __all__ = [
     "CCEError", "IGNORE_INDEX", "CCE_BWD_DETERMINISTIC", "CCE_BWD_BF16_GRADS", "CCE_BWD_ACCUMULATE",
     "CCE_BWD_PREPARED", "CCE_BWD_STRIPES", "cce_debug_stripe_schedule", "cce_debug_set_reduce_prefetch",
     "cce_debug_set_stripe_params", "cce_debug_set_l2_hints", "cce_debug_set_forward_schedule",
-    "cce_debug_set_forward_order", "cce_debug_l2_halves",
+    "cce_debug_set_forward_order", "cce_debug_l2_halves", "cce_debug_forward_plan",
     "cce_debug_set_stripe_order",
     "cce_backward_prepare",
     "backward_prepare", "cce_forward",

@@ -102,6 +102,9 @@ def load_library():
         lib.cce_debug_set_forward_order.restype = ctypes.c_int
         lib.cce_debug_l2_halves.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
         lib.cce_debug_l2_halves.restype = ctypes.c_int
+        lib.cce_debug_forward_plan.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                               ctypes.POINTER(ctypes.c_int)]
+        lib.cce_debug_forward_plan.restype = ctypes.c_int
         lib.cce_debug_set_reduce_prefetch.argtypes = [ctypes.c_int]
         lib.cce_debug_set_reduce_prefetch.restype = ctypes.c_int
         lib.cce_debug_stripe_schedule.argtypes = [ctypes.c_int] * 8 + [c_vp, c_i64]
@@ -341,6 +344,15 @@ def cce_debug_set_forward_schedule(n_split: int = 0, group_m: int = 0, l2_hints:
     operand stages per CTA (0 = default 7, or 6)."""
     _check(load_library().cce_debug_set_forward_schedule(int(n_split), int(group_m), int(l2_hints), int(stages)),
            "cce_debug_set_forward_schedule")
+
+
+def cce_debug_forward_plan(N: int, D: int, V: int, sms: int) -> dict:
+    """The forward's launch plan for these sizes on a GPU with `sms` SMs
+    (host arithmetic; no device needed)."""
+    out = (ctypes.c_int * 6)()
+    if load_library().cce_debug_forward_plan(int(N), int(D), int(V), int(sms), out) != 0:
+        raise ValueError("cce_debug_forward_plan: invalid sizes")
+    return dict(pair=bool(out[0]), n_mblk=out[1], n_vtile=out[2], n_split=out[3], group_m=out[4], grid=out[5])
 
 
 def cce_debug_l2_halves(max_sms: int = 256) -> list:

@@ -231,13 +231,12 @@ struct FwdPlan {
   size_t ws_bytes;
 };
 
-bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
-  if (!sizes_ok(N, D, V)) return false;
-  DeviceInfo di = device_info();
-  if (!di.ok || di.sms <= 0) return false;
-  p->pair = g_fwd_variant.load() == 1 && di.sms >= 2;
-  const int rows = p->pair ? 2 * BM : BM;           // token rows per work unit
-  const int workers = p->pair ? di.sms / 2 : di.sms;  // CTA pairs or CTAs
+// The forward's launch plan for a GPU with `sms` SMs (host arithmetic only).
+bool plan_forward_for(int64_t N, int64_t D, int64_t V, int sms, FwdPlan* p) {
+  if (!sizes_ok(N, D, V) || sms <= 0) return false;
+  p->pair = g_fwd_variant.load() == 1 && sms >= 2;
+  const int rows = p->pair ? 2 * BM : BM;       // token rows per work unit
+  const int workers = p->pair ? sms / 2 : sms;  // CTA pairs or CTAs
   p->n_mblk = (int)((N + rows - 1) / rows);
   p->n_vtile = (int)((V + BN - 1) / BN);
   // Token blocks per raster group.  Round-robin order: ~48 MB of E rows in
@@ -264,6 +263,13 @@ bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
   p->grid = (int)std::min<long long>(units, workers) * (p->pair ? 2 : 1);
   p->ws_bytes = STATUS_BYTES + align_up((size_t)p->n_split * (size_t)N * sizeof(float2), 256);
   return true;
+}
+
+bool plan_forward(int64_t N, int64_t D, int64_t V, FwdPlan* p) {
+  if (!sizes_ok(N, D, V)) return false;
+  const DeviceInfo di = device_info();
+  if (!di.ok || di.sms <= 0) return false;
+  return plan_forward_for(N, D, V, di.sms, p);
 }
 
 // Backward workspace: status | pre-pass header | dC row bits [ceil(V/32)] |
@@ -502,6 +508,19 @@ cce_status_t cce_debug_set_forward_schedule(int n_split, int group_m, int l2_hin
   g_fwd_l2_hints.store(l2_hints);
   g_fwd_stages.store(stages ? stages : PAIR_STAGES_MAX);
   return CCE_OK;
+}
+
+int cce_debug_forward_plan(int64_t N, int64_t D, int64_t V, int sms, int* out) {
+  if (!out) return -1;
+  FwdPlan p;
+  if (!plan_forward_for(N, D, V, sms, &p)) return -1;
+  out[0] = p.pair ? 1 : 0;
+  out[1] = p.n_mblk;
+  out[2] = p.n_vtile;
+  out[3] = p.n_split;
+  out[4] = p.group_m;
+  out[5] = p.grid;
+  return 0;
 }
 
 int cce_debug_l2_halves(int* half_of_sm, int max_sms) {
